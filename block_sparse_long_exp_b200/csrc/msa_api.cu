@@ -1,0 +1,286 @@
+// C ABI of libmsa (declared in include/msa.h): argument checks, workspace
+// layout, tensor-map creation and the launch sequence of each entry point.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "msa_internal.h"
+
+using namespace msa;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+bool shape_ok(const msa_shape_t* s) {
+  return s != nullptr && s->H > 0 && s->G > 0 && s->d > 0 && s->d_idx > 0 && s->B_k > 0 && s->k > 0;
+}
+
+msa_status_t check_shape(const msa_shape_t* s) {
+  if (!shape_ok(s)) return MSA_ERR_INVALID_ARG;
+  if (s->H % s->G != 0) return MSA_ERR_INVALID_ARG;
+  const int hg = s->H / s->G;
+  if (hg != 4 && hg != 8 && hg != 16) return MSA_ERR_UNSUPPORTED;
+  if (s->G != 1 && s->G != 2 && s->G != 4) return MSA_ERR_UNSUPPORTED;
+  if (s->d != 64 && s->d != 128) return MSA_ERR_UNSUPPORTED;
+  if (s->d_idx != 32 && s->d_idx != 64 && s->d_idx != 128) return MSA_ERR_UNSUPPORTED;
+  if (s->B_k != kBk) return MSA_ERR_UNSUPPORTED;
+  if (s->k < 1 || s->k > kMaxK) return MSA_ERR_UNSUPPORTED;
+  if (!(s->sm_scale > 0.f) || s->sm_scale != s->sm_scale) return MSA_ERR_INVALID_ARG;
+  return MSA_OK;
+}
+
+msa_status_t check_seqs(const msa_varlen_t* v) {
+  if (v == nullptr || v->cu_q == nullptr || v->cu_k == nullptr) return MSA_ERR_INVALID_ARG;
+  if (v->batch < 1 || v->total_q < 0 || v->total_k < 1 || v->max_q_len < 0 || v->max_k_len < 1)
+    return MSA_ERR_INVALID_ARG;
+  if (v->total_q > v->total_k || v->max_q_len > v->max_k_len) return MSA_ERR_INVALID_ARG;
+  if (v->total_k > (int64_t)INT32_MAX - 256 || v->total_q > (int64_t)INT32_MAX / kMaxK) return MSA_ERR_UNSUPPORTED;
+  return MSA_OK;
+}
+
+bool ws_ok(const void* ws, size_t have, size_t need) {
+  return ws != nullptr && (reinterpret_cast<uintptr_t>(ws) % kAlign) == 0 && have >= need;
+}
+
+int64_t total_blocks_bound(const msa_varlen_t* v) { return (v->total_k + kBk - 1) / kBk + v->batch; }
+
+// Slices of a sparse-attention workspace for chunks of `rows` query rows.
+struct AttnLayout {
+  size_t blk_off, counts, offsets, cursor, item_off, nitems, entries, items, part_acc, part_lse, total;
+  int64_t nlists, max_items;
+  int32_t qpi;
+};
+
+AttnLayout attn_layout(const msa_shape_t* s, const msa_varlen_t* v, int64_t rows) {
+  AttnLayout L{};
+  const int hg = s->H / s->G;
+  L.qpi = 8 * (128 / hg);                 // 8 tiles of 128 rows per work item
+  L.nlists = (int64_t)s->G * total_blocks_bound(v);
+  const int64_t nentries = rows * s->G * s->k;
+  L.max_items = L.nlists + (nentries + L.qpi - 1) / L.qpi + 1;
+  size_t off = kWsHeader;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, kAlign);
+    return o;
+  };
+  L.blk_off = take(sizeof(int32_t) * (v->batch + 1));
+  L.counts = take(sizeof(int32_t) * L.nlists);
+  L.offsets = take(sizeof(int32_t) * (L.nlists + 1));
+  L.cursor = take(sizeof(int32_t) * L.nlists);
+  L.item_off = take(sizeof(int32_t) * (L.nlists + 1));
+  L.nitems = take(sizeof(int32_t) * 2);
+  L.entries = take(sizeof(uint32_t) * nentries);
+  L.items = take(sizeof(Item) * L.max_items);
+  L.part_acc = take((size_t)nentries * hg * s->d * 2);
+  L.part_lse = take((size_t)nentries * hg * 4);
+  L.total = off;
+  return L;
+}
+
+int64_t chunk_rows(const msa_varlen_t* v, int64_t q_chunk) {
+  if (q_chunk <= 0 || q_chunk > v->total_q) return v->total_q;
+  return q_chunk;
+}
+
+msa_status_t attn_common(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q, const void* k,
+                         const void* v, const int32_t* sel, void* out, float* lse, int64_t q_chunk, void* ws,
+                         size_t ws_bytes, void* stream) {
+  msa_status_t st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  st = check_seqs(seqs);
+  if (st != MSA_OK) return st;
+  if (!q || !k || !v || !sel || !out) return MSA_ERR_INVALID_ARG;
+  if (seqs->total_q == 0) return MSA_OK;
+  const int64_t rows = chunk_rows(seqs, q_chunk);
+  const AttnLayout L = attn_layout(shape, seqs, rows);
+  if (!ws_ok(ws, ws_bytes, L.total)) return MSA_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  AttnArgs a{};
+  a.q = q; a.key = k; a.value = v; a.sel = sel; a.out = out; a.lse = lse;
+  a.cu_q = seqs->cu_q; a.cu_k = seqs->cu_k;
+  a.batch = seqs->batch; a.H = shape->H; a.G = shape->G; a.d = shape->d; a.k = shape->k;
+  a.sm_scale = shape->sm_scale;
+  a.total_q = seqs->total_q; a.total_k = seqs->total_k;
+  a.max_q_len = seqs->max_q_len; a.max_k_len = seqs->max_k_len;
+  a.err = reinterpret_cast<DevError*>(base);
+  a.blk_off = reinterpret_cast<int32_t*>(base + L.blk_off);
+  a.counts = reinterpret_cast<int32_t*>(base + L.counts);
+  a.offsets = reinterpret_cast<int32_t*>(base + L.offsets);
+  a.cursor = reinterpret_cast<int32_t*>(base + L.cursor);
+  a.item_off = reinterpret_cast<int32_t*>(base + L.item_off);
+  a.nitems = reinterpret_cast<int32_t*>(base + L.nitems);
+  a.entries = reinterpret_cast<uint32_t*>(base + L.entries);
+  a.items = reinterpret_cast<Item*>(base + L.items);
+  a.max_items = L.max_items;
+  a.nlists = L.nlists;
+  a.part_acc = base + L.part_acc;
+  a.part_lse = reinterpret_cast<float*>(base + L.part_lse);
+  a.queries_per_item = L.qpi;
+  for (int64_t t0 = 0; t0 < seqs->total_q; t0 += rows) {
+    a.t0 = t0;
+    a.t1 = t0 + rows < seqs->total_q ? t0 + rows : seqs->total_q;
+    if (launch_sparse_attn_pass(a, stream) != 0) return MSA_ERR_CUDA;
+  }
+  return MSA_OK;
+}
+
+}  // namespace
+
+namespace msa {
+
+int make_tmap_bf16(void* tmap_out, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                   const uint32_t* box, int swizzle_bytes) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (encode == nullptr) return (int)cudaErrorNotSupported;
+  cuuint64_t gdim[5];
+  cuuint64_t gstr[4];
+  cuuint32_t bdim[5], estr[5];
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bdim[i] = box[i];
+    estr[i] = 1;
+    if (i + 1 < rank) gstr[i] = strides_bytes[i];
+  }
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE;
+  const CUresult r = encode(reinterpret_cast<CUtensorMap*>(tmap_out), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                            (cuuint32_t)rank, const_cast<void*>(base), gdim, gstr, bdim, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : (int)cudaErrorInvalidValue;
+}
+
+}  // namespace msa
+
+extern "C" {
+
+const char* msa_version(void) { return "msa-b200 0.1 (sm_100a)"; }
+
+size_t msa_index_topk_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs) {
+  if (check_shape(shape) != MSA_OK || check_seqs(seqs) != MSA_OK) return 0;
+  size_t need = kWsHeader;
+  if (seqs->max_q_len <= 1)
+    need += align_up(decode_index_scratch_bytes(seqs->batch, seqs->total_k, shape->G, shape->k), kAlign);
+  return need;
+}
+
+msa_status_t msa_index_topk(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q_idx,
+                            const void* k_idx, int32_t* sel, void* ws, size_t ws_bytes, void* stream) {
+  msa_status_t st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  st = check_seqs(seqs);
+  if (st != MSA_OK) return st;
+  if (!q_idx || !k_idx || !sel) return MSA_ERR_INVALID_ARG;
+  const size_t need = msa_index_topk_workspace_size(shape, seqs);
+  if (!ws_ok(ws, ws_bytes, need)) return MSA_ERR_WORKSPACE;
+  if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  if (seqs->total_q == 0) return MSA_OK;
+  IndexTopkArgs a{};
+  a.q_idx = q_idx; a.k_idx = k_idx; a.sel = sel;
+  a.cu_q = seqs->cu_q; a.cu_k = seqs->cu_k;
+  a.batch = seqs->batch; a.G = shape->G; a.d_idx = shape->d_idx; a.k = shape->k;
+  a.total_q = seqs->total_q; a.total_k = seqs->total_k;
+  a.max_q_len = seqs->max_q_len; a.max_k_len = seqs->max_k_len;
+  a.err = static_cast<DevError*>(ws);
+  a.scratch = static_cast<uint8_t*>(ws) + kWsHeader;
+  a.scratch_bytes = ws_bytes - kWsHeader;
+  int rc;
+  if (seqs->max_q_len <= 1) {
+    rc = launch_index_topk_decode(a, stream);
+  } else {
+    if (seqs->batch > kMaxBatchTiles) return MSA_ERR_UNSUPPORTED;
+    rc = launch_index_topk_prefill(a, stream);
+  }
+  return rc == 0 ? MSA_OK : MSA_ERR_CUDA;
+}
+
+size_t msa_sparse_attn_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs, int64_t q_chunk) {
+  if (check_shape(shape) != MSA_OK || check_seqs(seqs) != MSA_OK) return 0;
+  return attn_layout(shape, seqs, chunk_rows(seqs, q_chunk)).total;
+}
+
+msa_status_t msa_sparse_attn_prefill(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q,
+                                     const void* k, const void* v, const int32_t* sel, void* out, float* lse,
+                                     int64_t q_chunk, void* ws, size_t ws_bytes, void* stream) {
+  return attn_common(shape, seqs, q, k, v, sel, out, lse, q_chunk, ws, ws_bytes, stream);
+}
+
+msa_status_t msa_sparse_attn_decode(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q,
+                                    const void* k_cache, const void* v_cache, const int32_t* sel, void* out,
+                                    float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (seqs != nullptr && seqs->max_q_len > 1) return MSA_ERR_INVALID_ARG;
+  return attn_common(shape, seqs, q, k_cache, v_cache, sel, out, lse, 0, ws, ws_bytes, stream);
+}
+
+msa_status_t msa_combine(const msa_shape_t* shape, int64_t T, const void* part_acc, const float* part_lse,
+                         const int32_t* sel, void* out, float* lse, void* stream) {
+  msa_status_t st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  if (T < 0 || !part_acc || !part_lse || !sel || !out) return MSA_ERR_INVALID_ARG;
+  if (T == 0) return MSA_OK;
+  return launch_combine(part_acc, part_lse, sel, out, lse, T, shape->H, shape->G, shape->d, shape->k, stream) == 0
+             ? MSA_OK
+             : MSA_ERR_CUDA;
+}
+
+size_t msa_dense_attn_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs) {
+  if (check_shape(shape) != MSA_OK || check_seqs(seqs) != MSA_OK) return 0;
+  return kWsHeader;
+}
+
+msa_status_t msa_dense_attn(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q, const void* k,
+                            const void* v, void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  msa_status_t st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  st = check_seqs(seqs);
+  if (st != MSA_OK) return st;
+  if (!q || !k || !v || !out) return MSA_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, kWsHeader)) return MSA_ERR_WORKSPACE;
+  if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  if (seqs->total_q == 0) return MSA_OK;
+  DenseArgs a{};
+  a.q = q; a.key = k; a.value = v; a.out = out; a.lse = lse;
+  a.cu_q = seqs->cu_q; a.cu_k = seqs->cu_k;
+  a.batch = seqs->batch; a.H = shape->H; a.G = shape->G; a.d = shape->d; a.sm_scale = shape->sm_scale;
+  a.total_q = seqs->total_q; a.total_k = seqs->total_k;
+  a.max_q_len = seqs->max_q_len; a.max_k_len = seqs->max_k_len;
+  a.err = static_cast<DevError*>(ws);
+  const int rc = launch_dense_attn(a, stream);
+  if (rc == (int)cudaErrorNotSupported) return MSA_ERR_UNSUPPORTED;
+  return rc == 0 ? MSA_OK : MSA_ERR_CUDA;
+}
+
+msa_status_t msa_get_device_error(void* ws, int32_t* code, int32_t* where, int32_t* info0, int32_t* info1,
+                                  void* stream) {
+  if (ws == nullptr || code == nullptr) return MSA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  DevError h{};
+  if (cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return MSA_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof(h), st) != cudaSuccess) return MSA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MSA_ERR_CUDA;
+  *code = h.code;
+  if (where) *where = h.where;
+  if (info0) *info0 = h.info0;
+  if (info1) *info1 = h.info1;
+  return MSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,421 @@
+// Index Branch, prefill shape: raw index scores on tcgen05, block max-pooling in
+// the TMEM epilogue, and a per-thread register top-(k-1) with the forced local
+// block (pnsm.cn explainer sec. 2 and sec. 7 "exp-free Top-k" / "per-thread
+// register top-k"; yifor-blog "設計核心" item 1; yhxrc.cn sec. 二 "block max
+// pooling").
+//
+// One persistent CTA per SM walks 128-query tiles (all G groups of a tile at
+// once, so each index-key block is loaded once for G MMAs).  Per key block j and
+// group g the tensor core computes S = Q_idx[128 x d_idx] * K_idx[j]^T into one of
+// four 128-column TMEM accumulators; an epilogue warpgroup reads its lane's 128
+// scores, takes the max (the block score) and offers (score, j) to the top list
+// of that (query, group).  Blocks arrive in ascending order, so a new block only
+// displaces a strictly lower score: ties stay with the lower block index.
+//
+// Warp roles (320 threads): warps 0-3 and 4-7 are two epilogue sets (set e
+// drains the accumulators of groups g with g % E == e), warp 8 issues TMA loads,
+// warp 9 owns TMEM and issues the MMAs.
+#include "msa_common.cuh"
+
+namespace msa {
+namespace {
+
+constexpr int kStages = 4;        // max index-key block stages in shared memory
+constexpr int kAcc = 4;           // 128-column TMEM accumulators (512 columns)
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kTile = 128;        // queries per tile = key-block size
+
+struct __align__(16) IndexCtl {
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kStages], k_empty[kStages];
+  uint64_t acc_full[kAcc], acc_empty[kAcc];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int32_t abort_flag;
+  int32_t ntiles;
+  int32_t pad;
+  int32_t tile_prefix[kMaxBatchTiles + 1];
+};
+
+struct TileInfo {
+  int q0;      // first query row of the tile
+  int rows;    // valid query rows (<= 128)
+  int pos0;    // absolute position of row 0 in its sequence
+  int n_kb;    // key blocks scanned: 0 .. n_kb-1 (lb of the last valid row)
+  int k0row;   // first key row of the sequence
+};
+
+__device__ __forceinline__ TileInfo tile_info(int tau, const IndexCtl* ctl, int batch, const int32_t* cu_q,
+                                              const int32_t* cu_k) {
+  int lo = 0, hi = batch;  // find b with prefix[b] <= tau < prefix[b+1]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (ctl->tile_prefix[mid] <= tau) lo = mid; else hi = mid;
+  }
+  const int b = lo;
+  const int i = tau - ctl->tile_prefix[b];
+  const int Tb = cu_q[b + 1] - cu_q[b];
+  const int Sb = cu_k[b + 1] - cu_k[b];
+  TileInfo t;
+  t.q0 = cu_q[b] + kTile * i;
+  t.rows = min(kTile, Tb - kTile * i);
+  t.pos0 = Sb - Tb + kTile * i;
+  t.n_kb = (t.pos0 + t.rows - 1) / kBk;
+  t.k0row = cu_k[b];
+  return t;
+}
+
+// Static snake schedule over tiles in longest-first order: iteration `it` of
+// CTA c takes slot it*grid + (it even ? c : grid-1-c); slot s is tile
+// ntiles-1-s (later tiles of a sequence scan more key blocks).
+__device__ __forceinline__ int snake_tile(int it, int ntiles) {
+  const int g = gridDim.x, c = blockIdx.x;
+  const int slot = it * g + ((it & 1) ? (g - 1 - c) : c);
+  return slot < ntiles ? (ntiles - 1 - slot) : -1;
+}
+
+template <int CAP>
+struct TopList {
+  float sc[CAP];
+  int ix[CAP];
+  int n;
+  float thr;  // score of the last entry when full
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int i = 0; i < CAP; ++i) { sc[i] = -INFINITY; ix[i] = 0x7fffffff; }
+    n = 0;
+    thr = -INFINITY;
+  }
+  // Candidates arrive with ascending j; a full list only takes a strictly
+  // higher score than its last entry.
+  __device__ __forceinline__ void offer(float s, int j, int cap) {
+    if (n >= cap && !(s > thr)) return;
+    bool gt[CAP];
+#pragma unroll
+    for (int i = 0; i < CAP; ++i) gt[i] = (i >= n) || (s > sc[i]);
+#pragma unroll
+    for (int i = CAP - 1; i >= 1; --i) {
+      if (i < cap) {
+        const float ns = gt[i - 1] ? sc[i - 1] : (gt[i] ? s : sc[i]);
+        const int ni = gt[i - 1] ? ix[i - 1] : (gt[i] ? j : ix[i]);
+        sc[i] = ns;
+        ix[i] = ni;
+      }
+    }
+    if (gt[0]) { sc[0] = s; ix[0] = j; }
+    n = min(n + 1, cap);
+    // the list is sorted descending, so its minimum is the last entry (a min
+    // reduction keeps the list in registers; a select on cap-1 would not)
+    float t = INFINITY;
+#pragma unroll
+    for (int i = 0; i < CAP; ++i) t = fminf(t, (i < cap) ? sc[i] : INFINITY);
+    thr = t;
+  }
+  // Write the selection ascending: the n chosen ids, then the local block,
+  // then -1 padding.
+  __device__ __forceinline__ void write(int32_t* dst, int k, int lb) const {
+#pragma unroll
+    for (int i = 0; i < CAP; ++i) {
+      if (i < n) {
+        int rank = 0;
+#pragma unroll
+        for (int j2 = 0; j2 < CAP; ++j2) rank += (j2 < n && ix[j2] < ix[i]) ? 1 : 0;
+        dst[rank] = ix[i];
+      }
+    }
+    dst[n] = lb;
+    for (int r = n + 1; r < k; ++r) dst[r] = -1;
+  }
+};
+
+__device__ __forceinline__ float max_of_16(const uint32_t (&r)[16]) {
+  const float a = fmax3(__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]));
+  const float b = fmax3(__uint_as_float(r[3]), __uint_as_float(r[4]), __uint_as_float(r[5]));
+  const float c = fmax3(__uint_as_float(r[6]), __uint_as_float(r[7]), __uint_as_float(r[8]));
+  const float d = fmax3(__uint_as_float(r[9]), __uint_as_float(r[10]), __uint_as_float(r[11]));
+  const float e = fmax3(__uint_as_float(r[12]), __uint_as_float(r[13]), __uint_as_float(r[14]));
+  return fmax3(fmax3(a, b, c), fmax3(d, e, __uint_as_float(r[15])), -INFINITY);
+}
+
+__device__ __forceinline__ float max_of_32(const uint32_t (&r)[32]) {
+  float m[11];
+#pragma unroll
+  for (int i = 0; i < 10; ++i)
+    m[i] = fmax3(__uint_as_float(r[3 * i]), __uint_as_float(r[3 * i + 1]), __uint_as_float(r[3 * i + 2]));
+  m[10] = fmaxf(__uint_as_float(r[30]), __uint_as_float(r[31]));
+  const float a = fmax3(m[0], m[1], m[2]);
+  const float b = fmax3(m[3], m[4], m[5]);
+  const float c = fmax3(m[6], m[7], m[8]);
+  return fmax3(fmax3(a, b, c), m[9], m[10]);
+}
+
+template <int KMAX, int G>
+__global__ void __launch_bounds__(kThreads, 1)
+index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                          int32_t* __restrict__ sel, const int32_t* __restrict__ cu_q,
+                          const int32_t* __restrict__ cu_k, int batch, int d_idx, int k, int nst,
+                          DevError* err) {
+  constexpr int CAP = KMAX - 1;
+  constexpr int E = G >= 2 ? 2 : 1;   // epilogue sets in use
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+
+  const int span = d_idx * 2 >= 128 ? 128 : d_idx * 2;   // bytes per swizzled row
+  const int span_el = span / 2;
+  const int nbox = (d_idx * 2) / span;                    // boxes per 128-row tile
+  const uint32_t tile_bytes = kTile * d_idx * 2;          // one [128 x d_idx] bf16 tile
+  uint8_t* q_s = smem;                                    // G tiles
+  uint8_t* k_s = smem + G * tile_bytes;                   // kStages tiles
+  IndexCtl* ctl = reinterpret_cast<IndexCtl*>(k_s + nst * tile_bytes);
+  volatile int32_t* abort_flag = &ctl->abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ctl->q_full, 1);
+    mbar_init(&ctl->q_empty, 1);
+    for (int s = 0; s < kStages; ++s) { mbar_init(&ctl->k_full[s], 1); mbar_init(&ctl->k_empty[s], 1); }
+    for (int a = 0; a < kAcc; ++a) { mbar_init(&ctl->acc_full[a], 1); mbar_init(&ctl->acc_empty[a], 4); }
+    mbar_init(&ctl->mma_done, 1);
+    ctl->abort_flag = 0;
+    // tiles per sequence (sequences with T_b > S_b are rejected and skipped)
+    int acc = 0;
+    for (int b = 0; b < batch; ++b) {
+      ctl->tile_prefix[b] = acc;
+      const int Tb = cu_q[b + 1] - cu_q[b];
+      const int Sb = cu_k[b + 1] - cu_k[b];
+      if (Tb < 0 || Tb > Sb) {
+        report_error(err, MSA_ERR_DEVICE_CHECK, kSiteIndexSeq, b, Tb);
+        continue;
+      }
+      acc += (Tb + kTile - 1) / kTile;
+    }
+    ctl->tile_prefix[batch] = acc;
+    ctl->ntiles = acc;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&ctl->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+  const int ntiles = ctl->ntiles;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      uint32_t kstep = 0, qiter = 0;
+      for (int it = 0;; ++it) {
+        const int tau = snake_tile(it, ntiles);
+        if (tau < 0 || *abort_flag) break;
+        const TileInfo ti = tile_info(tau, ctl, batch, cu_q, cu_k);
+        if (!mbar_wait(&ctl->q_empty, (qiter + 1) & 1)) {
+          report_error(err, MSA_ERR_TIMEOUT, kSiteIndexProducer, tau, -1);
+          *abort_flag = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&ctl->q_full, G * tile_bytes);
+        for (int g = 0; g < G; ++g)
+          for (int bx = 0; bx < nbox; ++bx)
+            tma_load_3d(q_s + g * tile_bytes + bx * kTile * span, &tm_q, &ctl->q_full, bx * span_el, g, ti.q0);
+        ++qiter;
+        for (int j = 0; j < ti.n_kb; ++j) {
+          const int st = kstep % nst;
+          if (!mbar_wait(&ctl->k_empty[st], ((kstep / nst) + 1) & 1)) {
+            report_error(err, MSA_ERR_TIMEOUT, kSiteIndexProducer, tau, j);
+            *abort_flag = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(&ctl->k_full[st], tile_bytes);
+          for (int bx = 0; bx < nbox; ++bx)
+            tma_load_2d(k_s + st * tile_bytes + bx * kTile * span, &tm_k, &ctl->k_full[st], bx * span_el,
+                        ti.k0row + kBk * j);
+          ++kstep;
+          if (*abort_flag) break;
+        }
+      }
+      // Drain: every load this thread issued has landed before the CTA exits.
+      if (qiter > 0) mbar_wait(&ctl->q_full, (qiter - 1) & 1);
+      for (int st = 0; st < nst; ++st) {
+        const uint32_t issued = kstep > (uint32_t)st ? (kstep - st + nst - 1) / nst : 0;
+        if (issued > 0) mbar_wait(&ctl->k_full[st], (issued - 1) & 1);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t mode = sw_mode_for(span);
+      const uint32_t sbo = 8 * span;
+      uint32_t kstep = 0, astep = 0, qiter = 0;
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        const int tau = snake_tile(it, ntiles);
+        if (tau < 0 || *abort_flag) break;
+        const TileInfo ti = tile_info(tau, ctl, batch, cu_q, cu_k);
+        if (!mbar_wait(&ctl->q_full, qiter & 1)) {
+          report_error(err, MSA_ERR_TIMEOUT, kSiteIndexMma, tau, -1);
+          ok = false;
+          break;
+        }
+        ++qiter;
+        tc_fence_after();
+        for (int j = 0; j < ti.n_kb && ok; ++j) {
+          const int st = kstep % nst;
+          if (!mbar_wait(&ctl->k_full[st], (kstep / nst) & 1)) {
+            report_error(err, MSA_ERR_TIMEOUT, kSiteIndexMma, tau, j);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t kaddr = smem_u32(k_s + st * tile_bytes);
+          for (int g = 0; g < G; ++g) {
+            const int a = astep % kAcc;
+            if (!mbar_wait(&ctl->acc_empty[a], ((astep / kAcc) + 1) & 1)) {
+              report_error(err, MSA_ERR_TIMEOUT, kSiteIndexMma, tau, 1000 + j);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t qaddr = smem_u32(q_s + g * tile_bytes);
+            for (int kk = 0; kk < d_idx / 16; ++kk) {
+              const uint32_t off = (32 * kk / span) * (kTile * span) + (32 * kk) % span;
+              umma_bf16_ss(tmem_base + a * 128, make_sdesc(qaddr + off, 16, sbo, mode),
+                           make_sdesc(kaddr + off, 16, sbo, mode), idesc, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&ctl->acc_full[a]);
+            ++astep;
+          }
+          umma_commit(&ctl->k_empty[st]);
+          ++kstep;
+          if (*abort_flag) ok = false;
+        }
+        umma_commit(&ctl->q_empty);
+      }
+      if (!ok) *abort_flag = 1;
+      // All issued MMAs complete before TMEM is released.
+      umma_commit(&ctl->mma_done);
+      mbar_wait(&ctl->mma_done, 0);
+    }
+  } else if (warp < 4 * E) {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp / 4;            // epilogue set
+    const int wq = warp % 4;           // TMEM lane quarter
+    const int row = 32 * wq + lane;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * wq) << 16);
+    TopList<CAP> list0, list1;
+    uint32_t astep = 0;
+    for (int it = 0;; ++it) {
+      const int tau = snake_tile(it, ntiles);
+      if (tau < 0 || *abort_flag) break;
+      const TileInfo ti = tile_info(tau, ctl, batch, cu_q, cu_k);
+      const bool valid = row < ti.rows;
+      const int lb = (ti.pos0 + row) / kBk;
+      list0.reset();
+      list1.reset();
+      bool ok = true;
+      for (int j = 0; j < ti.n_kb && ok; ++j, astep += G) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          if (g % E != e) continue;
+          const uint32_t as = astep + g;
+          const int a = as % kAcc;
+          if (!mbar_wait(&ctl->acc_full[a], (as / kAcc) & 1)) {
+            report_error(err, MSA_ERR_TIMEOUT, kSiteIndexEpilogue, tau, j);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t r0[16];
+          const uint32_t ta = lane_base + a * 128;
+          float m = -INFINITY;
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            tmem_ld16(ta + 16 * cc, r0);
+            tmem_ld_wait();
+            m = fmax3(m, max_of_16(r0), -INFINITY);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->acc_empty[a]);
+          if (m != m) m = -INFINITY;    // a block of NaN scores ranks as -inf
+          if (valid && j < lb) {
+            if (g / E == 0) list0.offer(m, j, k - 1); else list1.offer(m, j, k - 1);
+          }
+        }
+      }
+      if (!ok) break;
+      if (valid) {
+        int32_t* dst0 = sel + (static_cast<int64_t>(ti.q0 + row) * G + e) * k;
+        list0.write(dst0, k, lb);
+        if (G > 2) list1.write(dst0 + E * k, k, lb);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace
+
+int launch_index_topk_prefill(const IndexTopkArgs& a, void* stream) {
+  const int span = a.d_idx * 2 >= 128 ? 128 : a.d_idx * 2;
+  alignas(64) CUtensorMap tm_q, tm_k;
+  {
+    const uint64_t dims[3] = {(uint64_t)a.d_idx, (uint64_t)a.G, (uint64_t)a.total_q};
+    const uint64_t strides[2] = {(uint64_t)a.d_idx * 2, (uint64_t)a.G * a.d_idx * 2};
+    const uint32_t box[3] = {(uint32_t)(span / 2), 1u, (uint32_t)kTile};
+    int rc = make_tmap_bf16(&tm_q, a.q_idx, 3, dims, strides, box, span);
+    if (rc) return rc;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)a.d_idx, (uint64_t)a.total_k};
+    const uint64_t strides[1] = {(uint64_t)a.d_idx * 2};
+    const uint32_t box[2] = {(uint32_t)(span / 2), (uint32_t)kTile};
+    int rc = make_tmap_bf16(&tm_k, a.k_idx, 2, dims, strides, box, span);
+    if (rc) return rc;
+  }
+  const size_t tile_bytes = (size_t)kTile * a.d_idx * 2;
+  const int nst = a.d_idx >= 128 ? 2 : kStages;   // keep G + nst tiles within shared memory
+  size_t smem = 1024 + a.G * tile_bytes + nst * tile_bytes + sizeof(IndexCtl);
+  // at least 116 KB so that exactly one CTA (and one 512-column TMEM owner) sits on each SM
+  if (smem < 116 * 1024) smem = 116 * 1024;
+  int dev = 0, nsm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaErrorInvalidValue;
+#define MSA_IDX(KM, GG)                                                                                        \
+  if (a.k <= KM && a.G == GG) {                                                                                \
+    e = cudaFuncSetAttribute(index_topk_prefill_kernel<KM, GG>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                             (int)smem);                                                                       \
+    if (e != cudaSuccess) return (int)e;                                                                       \
+    index_topk_prefill_kernel<KM, GG><<<nsm, kThreads, smem, st>>>(tm_q, tm_k, a.sel, a.cu_q, a.cu_k, a.batch, \
+                                                                   a.d_idx, a.k, nst, a.err);                \
+    return (int)cudaGetLastError();                                                                            \
+  }
+  MSA_IDX(8, 1) MSA_IDX(8, 2) MSA_IDX(8, 4)
+  MSA_IDX(16, 1) MSA_IDX(16, 2) MSA_IDX(16, 4)
+  MSA_IDX(32, 1) MSA_IDX(32, 2) MSA_IDX(32, 4)
+#undef MSA_IDX
+  return (int)e;
+}
+
+}  // namespace msa

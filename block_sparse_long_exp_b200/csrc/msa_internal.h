@@ -1,0 +1,128 @@
+// Definitions shared by the host-side API and the kernels of libmsa.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/msa.h"
+
+namespace msa {
+
+constexpr int kBk = 128;          // block size the kernels are built for
+constexpr int kMaxK = 32;         // largest k
+constexpr int kMaxBatchTiles = 1024;  // sequences per prefill index launch
+
+// Device error word, at offset 0 of every workspace.
+struct DevError {
+  int32_t code;
+  int32_t where;
+  int32_t info0;
+  int32_t info1;
+};
+
+// Sites that can record an error (DevError::where).
+enum ErrorSite : int32_t {
+  kSiteIndexProducer = 101,
+  kSiteIndexMma = 102,
+  kSiteIndexEpilogue = 103,
+  kSiteIndexSeq = 104,
+  kSiteDecodeIndex = 111,
+  kSiteInvert = 121,
+  kSiteAttnLoad = 131,
+  kSiteAttnMma = 132,
+  kSiteAttnSoftmax = 133,
+  kSiteAttnItem = 134,
+  kSiteDense = 141,
+};
+
+// One KV-outer work item: up to `count` queries of the list of
+// (sequence seq, group g, block blk), entries [start, start + count) of the
+// packed query lists.
+struct Item {
+  int32_t seq;
+  int32_t blk;
+  int32_t g;
+  int32_t start;
+  int32_t count;
+  int32_t pad0, pad1, pad2;
+};
+
+constexpr size_t kWsHeader = 256;  // DevError + counters
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// -------------------------------------------------------- host launchers ---
+// Each returns the cudaError_t of its launch(es) (0 on success).
+
+struct IndexTopkArgs {
+  const void* q_idx;   // bf16 [T, G, d_idx]
+  const void* k_idx;   // bf16 [S, d_idx]
+  int32_t* sel;        // [T, G, k]
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int32_t batch, G, d_idx, k;
+  int64_t total_q, total_k;
+  int32_t max_q_len, max_k_len;
+  DevError* err;
+  void* scratch;       // decode path: block scores
+  size_t scratch_bytes;
+};
+int launch_index_topk_prefill(const IndexTopkArgs& a, void* stream);
+int launch_index_topk_decode(const IndexTopkArgs& a, void* stream);
+size_t decode_index_scratch_bytes(int32_t batch, int64_t total_k, int32_t G, int32_t k);
+
+struct AttnArgs {
+  const void* q;       // bf16 [T, H, d]
+  const void* key;     // bf16 [S, G, d]
+  const void* value;   // bf16 [S, G, d]
+  const int32_t* sel;  // [T, G, k]
+  void* out;           // bf16 [T, H, d]
+  float* lse;          // [T, H] or null
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int32_t batch, H, G, d, k;
+  float sm_scale;
+  int64_t total_q, total_k;
+  int32_t max_q_len, max_k_len;
+  int64_t t0, t1;      // query rows of this pass
+  DevError* err;
+  // workspace slices
+  int32_t* counts;     // [nlists]
+  int32_t* offsets;    // [nlists + 1]
+  int32_t* cursor;     // [nlists]
+  int32_t* item_off;   // [nlists + 1]
+  int32_t* nitems;     // [1]
+  uint32_t* entries;   // [(t1 - t0) * G * k]
+  Item* items;         // [max_items]
+  int64_t max_items;
+  int32_t* blk_off;    // [batch + 1] block offsets per sequence
+  int64_t nlists;      // G * total blocks
+  void* part_acc;      // f16 [(t1-t0), G, k, Hg, d]
+  float* part_lse;     // [(t1-t0), G, k, Hg]
+  int32_t queries_per_item;
+};
+int launch_sparse_attn_pass(const AttnArgs& a, void* stream);
+int launch_combine(const void* part_acc, const float* part_lse, const int32_t* sel, void* out,
+                   float* lse, int64_t T, int32_t H, int32_t G, int32_t d, int32_t k, void* stream);
+
+struct DenseArgs {
+  const void* q;
+  const void* key;
+  const void* value;
+  void* out;
+  float* lse;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int32_t batch, H, G, d;
+  float sm_scale;
+  int64_t total_q, total_k;
+  int32_t max_q_len, max_k_len;
+  DevError* err;
+};
+int launch_dense_attn(const DenseArgs& a, void* stream);
+
+// Tensor-map creation (driver entry point resolved at run time).
+int make_tmap_bf16(void* tmap_out, const void* base, int rank, const uint64_t* dims,
+                   const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes);
+
+}  // namespace msa

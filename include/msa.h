@@ -1,0 +1,193 @@
+/*
+ * msa.h — C ABI of the MiniMax Sparse Attention (MSA) forward hot path on
+ * NVIDIA B200 (sm_100a).  Library: libmsa.so.
+ *
+ * The operation (web pages on MSA, cited by title / address and section):
+ *   - pnsm.cn explainer "MiniMax Sparse Attention：一篇读懂百万上下文时代的稀疏注意力
+ *     工程化路线", sec. 2 (group-specific block selection on GQA, local block
+ *     always kept, B_k = 128, k = 16) and sec. 7 (exp-free Top-k, KV-outer
+ *     sparse attention, query gather, two-phase combine, load balancing);
+ *   - yifor-blog "MiniMax Sparse Attention (MSA): a Two-Branch Block-Sparse
+ *     Attention ...", section "設計核心" (Index Branch: block scores by
+ *     max-pooling, top-k; Main Branch: exact softmax on the chosen blocks);
+ *   - yhxrc.cn article, sec. 二 "MSA是怎么做的" (one index query head per group
+ *     and one shared index key head; current block mandatory; KV-outer).
+ *
+ * Conventions shared by every entry point
+ *   - All pointers named as device pointers must point to device memory of
+ *     the current CUDA device; the caller owns every buffer.  The library
+ *     allocates nothing: its scratch space is the caller's workspace `ws`
+ *     (size from the matching *_workspace_size query, 256-byte aligned).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t, 0 = legacy
+ *     default stream).  Calls that share a workspace must be ordered.
+ *   - Tensors are contiguous, row-major, bf16 unless stated:
+ *       q      [T, H, d]        query heads of every query token
+ *       k, v   [S, G, d]        keys / values (G = KV heads = GQA groups)
+ *       q_idx  [T, G, d_idx]    index query: one head per group
+ *       k_idx  [S, d_idx]       index key: one head shared by all groups
+ *       sel    [T, G, k] int32  selected block ids (local to the sequence),
+ *                               ascending, padded with -1
+ *       out    [T, H, d]        attention output
+ *       lse    [T, H] float     natural-log log-sum-exp of the scaled scores
+ *   - Sequences are packed: sequence b owns query rows cu_q[b]..cu_q[b+1]-1
+ *     and key rows cu_k[b]..cu_k[b+1]-1 (int32 device arrays of batch+1).
+ *     Its queries are its LAST T_b = cu_q[b+1]-cu_q[b] tokens: query i sits at
+ *     position S_b - T_b + i (prefill: T_b = S_b; decode: T_b = 1).
+ *     T_b <= S_b is required (checked on the device: MSA_ERR_DEVICE_CHECK).
+ *   - Query head h belongs to group g = h / (H / G).
+ *   - Block j of a sequence holds its tokens [j*B_k, (j+1)*B_k).  A query at
+ *     position p has local block lb = p / B_k and attends causally (keys <= p).
+ *   - Selection rule: the local block always; the other k-1 blocks are the
+ *     best of blocks 0..lb-1 by block score (max over the block's tokens of
+ *     <q_idx[t,g], k_idx[j]>), ties to the lower block index; NaN scores rank
+ *     as -inf; with lb+1 <= k all causal blocks are selected.
+ *
+ * Errors
+ *   - Arguments are checked on the host before any launch: MSA_ERR_INVALID_ARG
+ *     (null pointer, bad size), MSA_ERR_UNSUPPORTED (a size the kernels are not
+ *     built for), MSA_ERR_WORKSPACE (ws too small or misaligned).  Nothing is
+ *     launched when a check fails.
+ *   - A launch failure returns MSA_ERR_CUDA (cudaGetLastError after launch).
+ *   - Kernels record data-dependent failures (a bounded wait that ran out, a
+ *     block id out of range, T_b > S_b) in an error word at the start of `ws`.
+ *     Each call clears the word when it starts; read it with
+ *     msa_get_device_error after the call (it waits for the stream).
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = 1,
+  MSA_ERR_UNSUPPORTED = 2,
+  MSA_ERR_WORKSPACE = 3,
+  MSA_ERR_CUDA = 4,
+  MSA_ERR_TIMEOUT = 5,
+  MSA_ERR_DEVICE_CHECK = 6
+} msa_status_t;
+
+/* Layer shape.  Supported: H % G == 0 with H/G in {4, 8, 16}; G in {1, 2, 4};
+ * d in {64, 128}; d_idx in {32, 64, 128}; B_k == 128; 1 <= k <= 32. */
+typedef struct {
+  int32_t H;        /* query heads */
+  int32_t G;        /* KV heads = GQA groups = index query heads */
+  int32_t d;        /* head dim of q / k / v */
+  int32_t d_idx;    /* index head dim */
+  int32_t B_k;      /* block size in tokens */
+  int32_t k;        /* blocks selected per (query, group), local block included */
+  float sm_scale;   /* main-branch softmax scale (usually 1/sqrt(d)) */
+} msa_shape_t;
+
+/* Packed-sequence description.  cu_q / cu_k are DEVICE pointers; the other
+ * fields are host values that must agree with them: total_q = cu_q[batch],
+ * total_k = cu_k[batch], max_q_len / max_k_len the largest T_b / S_b. */
+typedef struct {
+  int32_t batch;
+  int32_t max_q_len;
+  int32_t max_k_len;
+  int32_t pad_;
+  int64_t total_q;
+  int64_t total_k;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+} msa_varlen_t;
+
+/* ---------------------------------------------------------------------- */
+/* Index Branch: block scoring + top-k with the forced local block.
+ * (pnsm.cn sec. 2 and sec. 7 "exp-free Top-k"; yifor-blog "設計核心" item 1;
+ *  yhxrc.cn sec. 二 "block max pooling".)
+ *
+ * Scores every causal, non-local block of every (query, group) with raw dot
+ * products (no exp), max-pools them per block and writes the selection
+ * sel[T, G, k].  Prefill-shaped calls (max_q_len > 1) run a tensor-core
+ * kernel over 128-query tiles; decode-shaped calls (max_q_len == 1) run a
+ * split scan of the index keys and a candidate merge.
+ * Selections are exact for inputs whose scores are exact in fp32 (for
+ * example integer-valued index q/k); otherwise they follow fp32 rounding. */
+size_t msa_index_topk_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs);
+
+msa_status_t msa_index_topk(const msa_shape_t* shape, const msa_varlen_t* seqs,
+                            const void* q_idx,  /* device bf16 [T, G, d_idx] */
+                            const void* k_idx,  /* device bf16 [S, d_idx] */
+                            int32_t* sel,       /* device int32 [T, G, k] (out) */
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Main Branch, prefill: exact causal softmax attention over the selected
+ * blocks (yifor-blog "設計核心" item 2; yololab.net "MSA的兩個主要步驟" step 2),
+ * computed KV-outer (pnsm.cn sec. 7; yhxrc.cn sec. 二; yololab.net "KV Outer
+ * Gather Q"): the selection is inverted into per-(sequence, group, block)
+ * query lists, each KV block is loaded once per work item and every query that
+ * chose it is gathered into tensor-core tiles; each (query, group, block)
+ * writes a softmax partial that a log-sum-exp combine merges (two-phase
+ * combine, no atomics on the output).
+ *
+ * `q_chunk` bounds how many query rows are processed per pass (0 = all); the
+ * workspace grows with it (about G*k*(H/G)*(2d+4) bytes per query row).  The
+ * call loops over chunks itself.  `lse` may be NULL. */
+size_t msa_sparse_attn_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs,
+                                      int64_t q_chunk);
+
+msa_status_t msa_sparse_attn_prefill(const msa_shape_t* shape, const msa_varlen_t* seqs,
+                                     const void* q,       /* device bf16 [T, H, d] */
+                                     const void* k,       /* device bf16 [S, G, d] */
+                                     const void* v,       /* device bf16 [S, G, d] */
+                                     const int32_t* sel,  /* device int32 [T, G, k] */
+                                     void* out,           /* device bf16 [T, H, d] (out) */
+                                     float* lse,          /* device f32 [T, H] (out) or NULL */
+                                     int64_t q_chunk,
+                                     void* ws, size_t ws_bytes, void* stream);
+
+/* Main Branch, decode: one query per sequence (T_b = 1, position S_b - 1,
+ * the cache already holding the new token).  Same contract as the prefill
+ * call; q_chunk is implied (all queries in one pass). */
+msa_status_t msa_sparse_attn_decode(const msa_shape_t* shape, const msa_varlen_t* seqs,
+                                    const void* q, const void* k_cache, const void* v_cache,
+                                    const int32_t* sel, void* out, float* lse,
+                                    void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Two-phase combine on its own (pnsm.cn sec. 7 "two-phase combine").
+ * Merges, for every query t and head h of group g, the partials of the slots
+ * s with sel[t, g, s] >= 0:
+ *   part_acc  device f16 [T, G, k, H/G, d]  softmax output over one block,
+ *                                           normalised by its own sum
+ *   part_lse  device f32 [T, G, k, H/G]     that block's log-sum-exp
+ * into out[t, h, :] = sum_s exp(lse_s - LSE) * acc_s with LSE = log sum_s
+ * exp(lse_s), and lse[t, h] = LSE (lse may be NULL). */
+msa_status_t msa_combine(const msa_shape_t* shape, int64_t T,
+                         const void* part_acc, const float* part_lse, const int32_t* sel,
+                         void* out, float* lse, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Dense causal GQA attention (every key <= the query position), the
+ * denominator of the pages' speedup comparison against GQA (pnsm.cn sec. 9).
+ * Same layouts as the sparse call; the workspace only holds the error word. */
+size_t msa_dense_attn_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs);
+
+msa_status_t msa_dense_attn(const msa_shape_t* shape, const msa_varlen_t* seqs,
+                            const void* q, const void* k, const void* v,
+                            void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Device error word of a workspace.  Waits for `stream`, copies the word to
+ * the host and clears it.  *code is an msa_status_t (MSA_OK if none);
+ * *where names the kernel site, *info0 / *info1 carry details. */
+msa_status_t msa_get_device_error(void* ws, int32_t* code, int32_t* where, int32_t* info0,
+                                  int32_t* info1, void* stream);
+
+/* Library version string. */
+const char* msa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H_ */

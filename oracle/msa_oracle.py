@@ -64,6 +64,8 @@ __all__ = [
     "block_max_pool",
     "select_blocks",
     "index_topk",
+    "index_topk_rows",
+    "attend",
     "selected_token_set",
     "main_branch",
     "msa_forward_rows",
@@ -137,6 +139,31 @@ def select_blocks(S, k: int) -> List[int]:
     return chosen + [lb]
 
 
+def index_topk_rows(q_idx_rows, k_idx_seq, positions: Sequence[int], k: int, B_k: int,
+                    row_chunk: int = 16) -> np.ndarray:
+    """Steps 1-3 for some queries of ONE sequence: sel[r, g, :] for the query at
+    absolute position positions[r] (ascending ids, -1 padded).
+
+    The token scores of a few rows at a time come from one matrix product
+    (k_idx[0..p_max] times their index queries); each row then keeps only its
+    causal keys j <= p, exactly as in ``index_scores``."""
+    q = _f64(q_idx_rows)
+    R, G, _ = q.shape
+    sel = np.full((R, G, k), -1, dtype=np.int32)
+    for r0 in range(0, R, row_chunk):
+        r1 = min(R, r0 + row_chunk)
+        pmax = int(max(positions[r0:r1]))
+        kk = _f64(k_idx_seq[: pmax + 1])
+        s_all = kk @ q[r0:r1].reshape((r1 - r0) * G, -1).T   # [pmax+1, rows*G]
+        for r in range(r0, r1):
+            p = int(positions[r])
+            for g in range(G):
+                s = s_all[: p + 1, (r - r0) * G + g]
+                blocks = select_blocks(block_max_pool(s, B_k), k)
+                sel[r, g, : len(blocks)] = blocks
+    return sel
+
+
 def index_topk(q_idx, k_idx, cu_q: Sequence[int], cu_k: Sequence[int], k: int,
                B_k: int) -> np.ndarray:
     """Index branch end to end: sel[t, g, :] = ascending selected block ids of
@@ -144,21 +171,16 @@ def index_topk(q_idx, k_idx, cu_q: Sequence[int], cu_k: Sequence[int], k: int,
 
     q_idx: [T, G, d_idx]; k_idx: [S, d_idx] (packed sequences, offsets cu_q and
     cu_k)."""
-    q_idx = _f64(q_idx)
-    k_idx = _f64(k_idx)
+    q_idx = np.asarray(q_idx)
     T, G, _ = q_idx.shape
     sel = np.full((T, G, k), -1, dtype=np.int32)
     for b in range(len(cu_q) - 1):
         q0, q1 = int(cu_q[b]), int(cu_q[b + 1])
         k0, k1 = int(cu_k[b]), int(cu_k[b + 1])
+        if q1 == q0:
+            continue
         pos = query_positions(q1 - q0, k1 - k0)
-        kseq = k_idx[k0:k1]
-        for i, p in enumerate(pos):
-            t = q0 + i
-            for g in range(G):
-                s = index_scores(q_idx[t, g], kseq, int(p))
-                blocks = select_blocks(block_max_pool(s, B_k), k)
-                sel[t, g, : len(blocks)] = blocks
+        sel[q0:q1] = index_topk_rows(q_idx[q0:q1], np.asarray(k_idx)[k0:k1], pos, k, B_k)
     return sel
 
 
@@ -178,18 +200,13 @@ def selected_token_set(blocks: Sequence[int], pos: int, B_k: int) -> np.ndarray:
     return np.concatenate(parts)
 
 
-def main_branch(q_tg, K_g, V_g, blocks: Sequence[int], pos: int, B_k: int,
-                sm_scale: float) -> Tuple[np.ndarray, np.ndarray]:
-    """Step 4.  Exact softmax attention of the query heads of one group over the
-    selected tokens ([yifor] "Main Branch"; [yololab] step 2 "精確注意力").
-
-    q_tg: [Hg, d] query heads of the group; K_g, V_g: [S_b, d] the group's keys
-    and values of this sequence.  Returns (o [Hg, d], lse [Hg]) in fp64, lse the
-    natural log-sum-exp of the scaled scores."""
+def attend(q_tg, K_J, V_J, sm_scale: float) -> Tuple[np.ndarray, np.ndarray]:
+    """Exact softmax attention of the query heads q_tg [Hg, d] over the token set
+    whose keys / values are K_J, V_J [|J|, d], in fp64.  Returns (o [Hg, d],
+    lse [Hg]), lse the natural log-sum-exp of the scaled scores."""
     q = _f64(q_tg)
-    J = selected_token_set(blocks, pos, B_k)
-    Kj = _f64(K_g)[J]
-    Vj = _f64(V_g)[J]
+    Kj = _f64(K_J)
+    Vj = _f64(V_J)
     s = sm_scale * (q @ Kj.T)                      # [Hg, |J|]
     m = s.max(axis=1, keepdims=True)
     e = np.exp(s - m)
@@ -197,6 +214,17 @@ def main_branch(q_tg, K_g, V_g, blocks: Sequence[int], pos: int, B_k: int,
     o = (e @ Vj) / l
     lse = (m + np.log(l))[:, 0]
     return o, lse
+
+
+def main_branch(q_tg, K_g, V_g, blocks: Sequence[int], pos: int, B_k: int,
+                sm_scale: float) -> Tuple[np.ndarray, np.ndarray]:
+    """Step 4.  Exact softmax attention of the query heads of one group over the
+    selected tokens ([yifor] "Main Branch"; [yololab] step 2 "精確注意力").
+
+    q_tg: [Hg, d] query heads of the group; K_g, V_g: [S_b, d] the group's keys
+    and values of this sequence.  Returns (o [Hg, d], lse [Hg])."""
+    J = selected_token_set(blocks, pos, B_k)
+    return attend(q_tg, np.asarray(K_g)[J], np.asarray(V_g)[J], sm_scale)
 
 
 def msa_forward_rows(q, k, v, sel, cu_q, cu_k, rows: Sequence[int], B_k: int,

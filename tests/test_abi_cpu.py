@@ -1,0 +1,73 @@
+"""The C-ABI library builds, loads and exports every symbol include/msa.h
+declares; host-side argument checks answer without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "msa.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(msa_[a-z_0-9]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_long_exp_b200 import build, msa
+    build.build()
+    return msa.load_library()
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for want in ("msa_index_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode", "msa_combine"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from block_sparse_long_exp_b200 import msa
+    names = _declared_functions()
+    assert sorted(set(msa.EXPORTED)) == names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_string(lib):
+    from block_sparse_long_exp_b200 import msa
+    assert "sm_100a" in msa.msa_version()
+
+
+def test_host_validation_without_gpu(lib):
+    from block_sparse_long_exp_b200 import msa
+    shape = msa.make_shape(64, 4, 128, 64, 16)
+    cu = (ctypes.c_int32 * 2)(0, 1024)
+    seqs = msa.Varlen(1, 1024, 1024, 0, 1024, 1024, ctypes.addressof(cu), ctypes.addressof(cu))
+    # supported shapes get a workspace size; unsupported ones get 0
+    assert lib.msa_index_topk_workspace_size(ctypes.byref(shape), ctypes.byref(seqs)) >= 256
+    assert lib.msa_sparse_attn_workspace_size(ctypes.byref(shape), ctypes.byref(seqs), 0) > 1024 * 4 * 16 * 16 * 128 * 2
+    bad = msa.make_shape(64, 4, 96, 64, 16)           # d = 96 is not built
+    assert lib.msa_index_topk_workspace_size(ctypes.byref(bad), ctypes.byref(seqs)) == 0
+    bad_bk = msa.make_shape(64, 4, 128, 64, 16, B_k=64)
+    assert lib.msa_sparse_attn_workspace_size(ctypes.byref(bad_bk), ctypes.byref(seqs), 0) == 0
+    # entry points reject invalid arguments before any launch
+    rc = lib.msa_index_topk(ctypes.byref(shape), ctypes.byref(seqs), None, None, None, None, 0, None)
+    assert rc == 1                                       # MSA_ERR_INVALID_ARG
+    rc = lib.msa_index_topk(ctypes.byref(bad), ctypes.byref(seqs), 1, 1, 1, 1, 1 << 20, None)
+    assert rc == 2                                       # MSA_ERR_UNSUPPORTED
+    rc = lib.msa_index_topk(None, ctypes.byref(seqs), 1, 1, 1, 1, 1 << 20, None)
+    assert rc == 1
+    rc = lib.msa_sparse_attn_prefill(ctypes.byref(shape), ctypes.byref(seqs), 256, 256, 256, 256, 256, None,
+                                     0, 256, 16, None)
+    assert rc == 3                                       # MSA_ERR_WORKSPACE (16 bytes is too small)
+    not_gqa = msa.make_shape(64, 3, 128, 64, 16)
+    rc = lib.msa_combine(ctypes.byref(not_gqa), 4, 1, 1, 1, 1, None, None)
+    assert rc == 1                                       # H % G != 0
+    more_q_than_k = msa.Varlen(1, 2048, 1024, 0, 2048, 1024, ctypes.addressof(cu), ctypes.addressof(cu))
+    rc = lib.msa_index_topk(ctypes.byref(shape), ctypes.byref(more_q_than_k), 1, 1, 1, 1, 1 << 20, None)
+    assert rc == 1
