@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark of the MSA forward hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole prefill hot path over one 128K-token layer:
+index branch (scores, block max-pool, top-k with the forced local block) and
+main branch (selection inversion, KV-outer sparse attention, combine).  The
+timed region holds K steps between a barrier and a device synchronize; the
+value is the whole-job throughput (query tokens/s, summed over ranks, each rank
+running its own independent layer: weak scaling, no data-path collective).
+
+Also reported on the same JSON line:
+  roofline     the dominant kernel's achieved TFLOP/s (or GB/s) against the
+               measured peak, from CUDA events the library records on its launch
+               stream around every launch during the timed region;
+  step_roofline  the whole step against max(FLOPs / tensor peak, bytes / HBM peak);
+  decode       decode step time (32 sequences, cache 128K..1M) and its HBM roofline;
+  e2e          the same prefill step through the public API with host (pinned)
+               buffers: host->device inputs and device->host output inside the
+               timed region;
+  cpu_baseline the fp64 oracle timed on this host's cores on a bounded sample;
+  clocks       nvidia-smi SM clocks and throttle reasons sampled while timing.
+
+--impl reference times the oracle alone (the reference arm of this comparison).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MSA prefill tokens/s @128K; decode µs/step; % of roofline on 1 B200"
+PREFILL = "prefill_n131072_hot2"
+DECODE = "decode_b32_l128k_1m_hot2"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks ---
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, pw, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+                pw.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        loaded = [s for s, m in zip(sm, mx) if s > 0.5 * m] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------- helpers ---
+
+def make_ctx(w, inp, torch, msa):
+    shape = msa.make_shape(w.H, w.G, w.d, w.d_idx, w.k)
+    seqs = msa.make_varlen(inp["cu_q"], inp["cu_k"], inp["cu_q_host"], inp["cu_k_host"])
+    T = inp["cu_q_host"][-1]
+    dev = inp["q"].device
+    ctx = dict(shape=shape, seqs=seqs, inp=inp, T=T)
+    ctx["sel"] = torch.empty((T, w.G, w.k), dtype=torch.int32, device=dev)
+    ctx["out"] = torch.empty((T, w.H, w.d), dtype=torch.bfloat16, device=dev)
+    lib = msa.load_library()
+    import ctypes
+    n_idx = lib.msa_index_topk_workspace_size(ctypes.byref(shape), ctypes.byref(seqs))
+    n_att = msa.msa_sparse_attn_workspace_size(shape, seqs, 0)
+    ctx["ws_idx"] = torch.empty(n_idx, dtype=torch.uint8, device=dev)
+    ctx["ws_att"] = torch.empty(n_att, dtype=torch.uint8, device=dev)
+    return ctx
+
+
+def step_prefill(ctx, msa, inp=None):
+    inp = inp or ctx["inp"]
+    msa.msa_index_topk(ctx["shape"], ctx["seqs"], inp["q_idx"], inp["k_idx"], sel=ctx["sel"], ws=ctx["ws_idx"],
+                       check=False)
+    msa.msa_sparse_attn_prefill(ctx["shape"], ctx["seqs"], inp["q"], inp["k"], inp["v"], ctx["sel"],
+                                out=ctx["out"], want_lse=False, ws=ctx["ws_att"], check=False)
+
+
+def step_decode(ctx, msa):
+    inp = ctx["inp"]
+    msa.msa_index_topk(ctx["shape"], ctx["seqs"], inp["q_idx"], inp["k_idx"], sel=ctx["sel"], ws=ctx["ws_idx"],
+                       check=False)
+    msa.msa_sparse_attn_decode(ctx["shape"], ctx["seqs"], inp["q"], inp["k"], inp["v"], ctx["sel"],
+                               out=ctx["out"], want_lse=False, ws=ctx["ws_att"], check=False)
+
+
+def device_errors(ctx, msa):
+    for key in ("ws_idx", "ws_att"):
+        code, where, i0, i1 = msa.msa_get_device_error(ctx[key])
+        if code != 0:
+            raise RuntimeError(f"device error {code} at site {where} ({i0}, {i1}) in {key}")
+
+
+def time_steps(fn, steps, torch, dist=None):
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    return s.elapsed_time(e)
+
+
+def max_over_ranks(x, torch, dist):
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, torch, dist):
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def traffic_for(kernel):
+    """DRAM bytes per full-size launch from a committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel)
+    if not d:
+        return None
+    src = os.path.join(ROOT, "block_sparse_long_exp_b200", "csrc", d.get("source", ""))
+    if not os.path.exists(src):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return d.get("dram_bytes_per_launch") if sha == d.get("source_sha") else None
+
+
+# ------------------------------------------------------------- CPU oracle ---
+
+def cpu_oracle_rate(w, inp, budget_s, torch, np, seed=0):
+    """Oracle throughput (query rows per second) on a seeded random sample of
+    rows, grown in batches until ~budget_s of CPU work."""
+    from oracle import msa_oracle as O
+    T = inp["cu_q_host"][-1]
+    g = torch.Generator().manual_seed(1234 + seed)
+    order = torch.randperm(T, generator=g).tolist()
+    full = {"q_idx": inp["q_idx"].float().cpu().numpy(), "k_idx": inp["k_idx"].float().cpu().numpy(),
+            "k": inp["k"].float().cpu().numpy(), "v": inp["v"].float().cpu().numpy()}
+    n_done, t_used, batch = 0, 0.0, 16
+    while t_used < budget_s and n_done < T:
+        rows = sorted(order[n_done:n_done + batch])
+        idx = torch.tensor(rows, dtype=torch.long, device=inp["q"].device)
+        host = dict(full, q=inp["q"].index_select(0, idx).float().cpu().numpy())
+        t0 = time.perf_counter()
+        _oracle_batch(w, host, rows, O, np)
+        t_used += time.perf_counter() - t0
+        n_done += len(rows)
+        batch = min(256, batch * 2)
+    return n_done / t_used, n_done, t_used
+
+
+def _oracle_batch(w, host, rows, O, np):
+    pos = np.asarray(rows)
+    sel = O.index_topk_rows(host["q_idx"][rows], host["k_idx"], pos, w.k, w.B_k)
+    Hg = w.H // w.G
+    for r, t in enumerate(rows):
+        for g in range(w.G):
+            J = O.selected_token_set([int(x) for x in sel[r, g]], int(t), w.B_k)
+            O.attend(host["q"][r, g * Hg:(g + 1) * Hg], host["k"][J, g], host["v"][J, g], w.sm_scale)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=1)
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------- arms ---
+
+def run_reference(args):
+    """The oracle as it stands, timed on this host's cores (rank 0 only)."""
+    import numpy as np
+    import torch
+    from block_sparse_long_exp_b200 import workloads as W
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = W.WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = W.make_inputs(w, dev)
+    T = inp["cu_q_host"][-1]
+    from oracle import msa_oracle as O
+    gen = torch.Generator().manual_seed(99)
+    order = torch.randperm(T, generator=gen).tolist()
+    per_step = args.ref_rows
+    host_full = {"q_idx": inp["q_idx"].float().cpu().numpy(), "k_idx": inp["k_idx"].float().cpu().numpy(),
+                 "k": inp["k"].float().cpu().numpy(), "v": inp["v"].float().cpu().numpy()}
+    times = []
+    for s in range(args.warmup + args.steps):
+        rows = sorted(order[(s * per_step) % T:(s * per_step) % T + per_step])
+        idx = torch.tensor(rows, dtype=torch.long, device=inp["q"].device)
+        host = dict(host_full, q=inp["q"].index_select(0, idx).float().cpu().numpy())
+        t0 = time.perf_counter()
+        _oracle_batch(w, host, rows, O, np)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+    sec = sum(times)
+    rate = per_step * len(times) / sec
+    cores = blas_threads() or len(os.sched_getaffinity(0))
+    sample = f"{per_step} random query rows of {args.workload} per step (of {T}); oracle selection + main branch"
+    line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * sec / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": args.workload, "T": T, "H": w.H, "G": w.G, "d": w.d,
+                                             "d_idx": w.d_idx, "B_k": w.B_k, "k": w.k},
+            "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    from block_sparse_long_exp_b200 import build as B
+    from block_sparse_long_exp_b200 import msa
+    from block_sparse_long_exp_b200 import roofline as R
+    from block_sparse_long_exp_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        dist = dist_mod
+    B.build()
+    msa.load_library()
+    peaks, peak_src = load_peaks()
+    w = W.WORKLOADS[args.workload]
+    # each rank runs an independent layer (its own seed): weak scaling
+    wr = W.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+    inp = W.make_inputs(wr, "cuda")
+    torch.cuda.synchronize()
+    ctx = make_ctx(wr, inp, torch, msa)
+    S_lens = [inp["cu_k_host"][i + 1] - inp["cu_k_host"][i] for i in range(len(inp["cu_k_host"]) - 1)]
+    T_lens = [inp["cu_q_host"][i + 1] - inp["cu_q_host"][i] for i in range(len(inp["cu_q_host"]) - 1)]
+    T = ctx["T"]
+    work = R.prefill_work(S_lens, T_lens, w.H, w.G, w.d, w.d_idx, w.B_k, w.k)
+
+    for _ in range(args.warmup):
+        step_prefill(ctx, msa)
+    torch.cuda.synchronize()
+    device_errors(ctx, msa)
+
+    gpu_uuid = str(torch.cuda.get_device_properties(local).uuid)
+    gpu_uuid = gpu_uuid if gpu_uuid.startswith("GPU-") else "GPU-" + gpu_uuid
+    clocks = ClockSampler(gpu_uuid)
+    clocks.start()
+    msa.msa_profile_reset()
+    msa.msa_profile_enable(True)
+    ms = time_steps(lambda: step_prefill(ctx, msa), args.steps, torch, dist)
+    msa.msa_profile_enable(False)
+    clk = clocks.stop()
+    device_errors(ctx, msa)
+    launches = msa.msa_profile_read(None)[1]
+    kernels = {}
+    for name in ("index_topk_prefill", "sparse_attn", "combine", "count", "scatter", "plan", "block_offsets"):
+        kms, n = msa.msa_profile_read(name)
+        if n:
+            kernels[name] = {"ms_per_launch": kms / n, "launches": n, "share": None}
+    tot = sum(v["ms_per_launch"] * v["launches"] for v in kernels.values()) or 1.0
+    for v in kernels.values():
+        v["share"] = v["ms_per_launch"] * v["launches"] / tot
+
+    ms_max = max_over_ranks(ms, torch, dist)
+    ms_step = ms_max / args.steps
+    tokens_all = sum_over_ranks(float(T * args.steps), torch, dist)
+    value = tokens_all / (ms_max / 1000.0)
+
+    # roofline of the dominant kernel (timed inside a long step: sustained peak)
+    per_kernel_work = {"sparse_attn": ("tensor", work["main_flops"]),
+                       "index_topk_prefill": ("tensor", work["index_flops"])}
+    dom = max(kernels, key=lambda n: kernels[n]["ms_per_launch"] * kernels[n]["launches"])
+    bound, units = per_kernel_work.get(dom, ("tensor", work["main_flops"]))
+    peak_t = peaks["bf16_tflops_sustained"]
+    launches_per_step = kernels[dom]["launches"] / args.steps
+    achieved = units / launches_per_step / (kernels[dom]["ms_per_launch"] / 1000.0) / 1e12
+    roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
+            "frac": achieved / peak_t, "traffic": traffic_for(dom),
+            "algorithmic_per_launch": units / launches_per_step,
+            "peak_source": f"bf16_tflops_sustained ({peak_src})"}
+    t_roof_ms = max(work["flops"] / (peaks["bf16_tflops"] * 1e12), work["bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    t_roof_sus = max(work["flops"] / (peak_t * 1e12), work["bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    step_roof = {"flops": work["flops"], "index_flops": work["index_flops"], "main_flops": work["main_flops"],
+                 "bytes": work["bytes"], "roofline_ms_burst": t_roof_ms, "roofline_ms_sustained": t_roof_sus,
+                 "frac_burst": t_roof_ms / ms_step, "frac_sustained": t_roof_sus / ms_step,
+                 "bound": "tensor" if work["flops"] / (peaks["bf16_tflops"] * 1e12) >
+                 work["bytes"] / (peaks["hbm_gbs"] * 1e9) else "hbm"}
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        keys = ("q", "k", "v", "q_idx", "k_idx")
+        host = {k_: inp[k_].cpu().pin_memory() for k_ in keys}
+        dev = {k_: torch.empty_like(inp[k_]) for k_ in keys}
+        host_out = torch.empty(ctx["out"].shape, dtype=ctx["out"].dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = host_out.numel() * host_out.element_size()
+
+        def e2e_step():
+            for k_ in keys:
+                dev[k_].copy_(host[k_], non_blocking=True)
+            step_prefill(ctx, msa, inp={**inp, **dev})
+            host_out.copy_(ctx["out"], non_blocking=True)
+
+        e2e_step()
+        e_steps = max(2, args.steps // 3)
+        ms_e = max_over_ranks(time_steps(e2e_step, e_steps, torch, dist), torch, dist)
+        e2e = {"value": sum_over_ranks(float(T * e_steps), torch, dist) / (ms_e / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e / e_steps}
+        del host, dev, host_out
+
+    # decode: 32 sequences with caches of 128K..1M tokens
+    decode = None
+    cpu = None
+    if rank == 0 and not args.no_decode:
+        del ctx
+        torch.cuda.empty_cache()
+        wd = W.WORKLOADS[DECODE]
+        dinp = W.make_inputs(wd, "cuda")
+        dctx = make_ctx(wd, dinp, torch, msa)
+        for _ in range(3):
+            step_decode(dctx, msa)
+        torch.cuda.synchronize()
+        device_errors(dctx, msa)
+        msa.msa_profile_reset()
+        msa.msa_profile_enable(True)
+        d_steps = max(5, args.steps)
+        d_ms = time_steps(lambda: step_decode(dctx, msa), d_steps, torch) / d_steps
+        msa.msa_profile_enable(False)
+        device_errors(dctx, msa)
+        L = [dinp["cu_k_host"][i + 1] - dinp["cu_k_host"][i] for i in range(wd.batch)]
+        dw = R.decode_work(L, wd.H, wd.G, wd.d, wd.d_idx, wd.B_k, wd.k)
+        dk = {}
+        for name in ("decode_scan", "decode_select", "sparse_attn", "combine", "count", "scatter", "plan"):
+            kms, n = msa.msa_profile_read(name)
+            if n:
+                dk[name] = {"ms_per_launch": kms / n, "launches": n}
+        scan_ms = dk.get("decode_scan", {}).get("ms_per_launch")
+        decode = {"workload": DECODE, "us_per_step": d_ms * 1000.0, "sum_L": sum(L),
+                  "algorithmic_bytes": dw["bytes"],
+                  "roofline_us": dw["bytes"] / (peaks["hbm_gbs"] * 1e9) * 1e6,
+                  "frac": dw["bytes"] / (peaks["hbm_gbs"] * 1e9) / (d_ms / 1000.0),
+                  "scan_kernel": None if scan_ms is None else {
+                      "bound": "hbm", "achieved": dw["index_bytes"] / (scan_ms / 1000.0) / 1e9,
+                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                      "frac": dw["index_bytes"] / (scan_ms / 1000.0) / 1e9 / peaks["hbm_gbs"]},
+                  "kernels": dk}
+        del dctx, dinp
+        torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, n_rows, secs = cpu_oracle_rate(w, inp, args.cpu_budget, torch, np)
+        cores = blas_threads() or len(os.sched_getaffinity(0))
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n_rows} random query rows of {args.workload} ({secs:.1f} s of fp64 oracle work: "
+                         f"selection + main branch per row)"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": args.workload, "T": T, "H": w.H, "G": w.G, "d": w.d, "d_idx": w.d_idx,
+                           "B_k": w.B_k, "k": w.k, "hot_block_frac": w.hot_frac,
+                           "l2": "inputs larger than L2 (q alone is %.1f GB)" % (inp["q"].numel() * 2 / 1e9),
+                           "parallelism": f"independent layer per GPU x{world}"},
+                "roofline": roof, "step_roofline": step_roof, "decode": decode, "e2e": e2e,
+                "cpu_baseline": cpu, "clocks": clk, "gpu_launches": launches, "kernels": kernels}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=PREFILL)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-rows", type=int, default=64)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        log("note: fewer than 3 warm-up steps")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -470,19 +470,31 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
   const int64_t nrows = a.t1 - a.t0;
   if (nrows <= 0) return 0;
   cudaError_t e;
-  block_offsets_kernel<<<1, 32, 0, st>>>(a.cu_k, a.batch, a.blk_off);
+  {
+    ProfScope p("block_offsets", stream);
+    block_offsets_kernel<<<1, 32, 0, st>>>(a.cu_k, a.batch, a.blk_off);
+  }
   e = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * a.nlists, st);
   if (e != cudaSuccess) return (int)e;
   e = cudaMemsetAsync(a.nitems, 0, sizeof(int32_t) * 2, st);   // nitems and the item ticket
   if (e != cudaSuccess) return (int)e;
   const int64_t nthreads = nrows * a.G;
   const int cs_blocks = (int)((nthreads + 255) / 256);
-  count_scatter_kernel<false><<<cs_blocks, 256, 0, st>>>(a.sel, a.t0, a.t1, a.G, a.k, a.batch, a.cu_q, a.cu_k,
-                                                         a.blk_off, a.counts, nullptr, a.err);
-  plan_kernel<<<1, 1024, 0, st>>>(a.counts, a.nlists, a.G, a.batch, a.blk_off, a.queries_per_item, a.offsets,
-                                  a.cursor, a.item_off, a.nitems, a.items, a.max_items, a.err);
-  count_scatter_kernel<true><<<cs_blocks, 256, 0, st>>>(a.sel, a.t0, a.t1, a.G, a.k, a.batch, a.cu_q, a.cu_k,
-                                                        a.blk_off, a.cursor, a.entries, a.err);
+  {
+    ProfScope p("count", stream);
+    count_scatter_kernel<false><<<cs_blocks, 256, 0, st>>>(a.sel, a.t0, a.t1, a.G, a.k, a.batch, a.cu_q, a.cu_k,
+                                                           a.blk_off, a.counts, nullptr, a.err);
+  }
+  {
+    ProfScope p("plan", stream);
+    plan_kernel<<<1, 1024, 0, st>>>(a.counts, a.nlists, a.G, a.batch, a.blk_off, a.queries_per_item, a.offsets,
+                                    a.cursor, a.item_off, a.nitems, a.items, a.max_items, a.err);
+  }
+  {
+    ProfScope p("scatter", stream);
+    count_scatter_kernel<true><<<cs_blocks, 256, 0, st>>>(a.sel, a.t0, a.t1, a.G, a.k, a.batch, a.cu_q, a.cu_k,
+                                                          a.blk_off, a.cursor, a.entries, a.err);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
 
@@ -501,13 +513,18 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   const float scale_log2 = a.sm_scale * 1.4426950408889634f;
-  sparse_attn_kernel<<<nsm, kAttnThreads, smem, st>>>(
-      tm_k, tm_v, reinterpret_cast<const __nv_bfloat16*>(a.q), a.items, a.nitems, a.nitems + 1, a.entries, a.cu_q,
-      a.cu_k, a.H, a.G, a.d, a.k, scale_log2, a.t0, reinterpret_cast<__half*>(a.part_acc), a.part_lse, a.err);
+  {
+    ProfScope p("sparse_attn", stream);
+    sparse_attn_kernel<<<nsm, kAttnThreads, smem, st>>>(
+        tm_k, tm_v, reinterpret_cast<const __nv_bfloat16*>(a.q), a.items, a.nitems, a.nitems + 1, a.entries,
+        a.cu_q, a.cu_k, a.H, a.G, a.d, a.k, scale_log2, a.t0, reinterpret_cast<__half*>(a.part_acc), a.part_lse,
+        a.err);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
   const int64_t rows = a.t1 - a.t0;
   const int64_t cthreads = rows * a.H * (a.d / 8);
+  ProfScope p("combine", stream);
   combine_kernel<<<(int)((cthreads + 255) / 256), 256, 0, st>>>(
       reinterpret_cast<const __half*>(a.part_acc), a.part_lse, a.sel + a.t0 * a.G * a.k,
       reinterpret_cast<__nv_bfloat16*>(a.out) + a.t0 * a.H * a.d, a.lse ? a.lse + a.t0 * a.H : nullptr, rows, a.H,
@@ -520,6 +537,7 @@ int launch_combine(const void* part_acc, const float* part_lse, const int32_t* s
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (T <= 0) return 0;
   const int64_t cthreads = T * H * (d / 8);
+  ProfScope p("combine", stream);
   combine_kernel<<<(int)((cthreads + 255) / 256), 256, 0, st>>>(
       reinterpret_cast<const __half*>(part_acc), part_lse, sel, reinterpret_cast<__nv_bfloat16*>(out), lse, T, H, G,
       d, k);

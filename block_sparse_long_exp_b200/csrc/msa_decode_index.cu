@@ -258,7 +258,10 @@ int launch_index_topk_decode(const IndexTopkArgs& a, void* stream) {
   float* bscore = reinterpret_cast<float*>(base + o_bs);
   int32_t* blk_off = reinterpret_cast<int32_t*>(base + o_bo);
   int32_t* chunk_off = reinterpret_cast<int32_t*>(base + o_co);
-  decode_prep_kernel<<<1, 32, 0, st>>>(a.cu_q, a.cu_k, a.batch, blk_off, chunk_off, a.err);
+  {
+    ProfScope p("decode_prep", stream);
+    decode_prep_kernel<<<1, 32, 0, st>>>(a.cu_q, a.cu_k, a.batch, blk_off, chunk_off, a.err);
+  }
 
   const int span = a.d_idx * 2 >= 128 ? 128 : a.d_idx * 2;
   alignas(64) CUtensorMap tm_k;
@@ -275,6 +278,7 @@ int launch_index_topk_decode(const IndexTopkArgs& a, void* stream) {
 #define MSA_SCAN(D)                                                                                          \
   e = cudaFuncSetAttribute(decode_scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);  \
   if (e != cudaSuccess) return (int)e;                                                                      \
+  ProfScope p("decode_scan", stream);                                                                       \
   decode_scan_kernel<D><<<(unsigned)max_chunks, kScanThreads, smem, st>>>(tm_k, qi, a.cu_q, a.cu_k, a.batch, \
                                                                         a.G, blk_off, chunk_off, bscore, a.err)
   if (a.d_idx == 32) { MSA_SCAN(32); }
@@ -282,6 +286,7 @@ int launch_index_topk_decode(const IndexTopkArgs& a, void* stream) {
   else { MSA_SCAN(128); }
 #undef MSA_SCAN
   const unsigned nsel = (unsigned)(a.batch * a.G);
+  ProfScope p("decode_select", stream);
   if (a.k <= 8) decode_select_kernel<7><<<nsel, kSelThreads, 0, st>>>(bscore, a.cu_q, a.cu_k, blk_off, a.G, a.k, a.sel);
   else if (a.k <= 16) decode_select_kernel<15><<<nsel, kSelThreads, 0, st>>>(bscore, a.cu_q, a.cu_k, blk_off, a.G, a.k, a.sel);
   else decode_select_kernel<31><<<nsel, kSelThreads, 0, st>>>(bscore, a.cu_q, a.cu_k, blk_off, a.G, a.k, a.sel);

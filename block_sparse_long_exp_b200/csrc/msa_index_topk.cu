@@ -407,6 +407,7 @@ int launch_index_topk_prefill(const IndexTopkArgs& a, void* stream) {
     e = cudaFuncSetAttribute(index_topk_prefill_kernel<KM, GG>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
                              (int)smem);                                                                       \
     if (e != cudaSuccess) return (int)e;                                                                       \
+    ProfScope p("index_topk_prefill", stream);                                                                 \
     index_topk_prefill_kernel<KM, GG><<<nsm, kThreads, smem, st>>>(tm_q, tm_k, a.sel, a.cu_q, a.cu_k, a.batch, \
                                                                    a.d_idx, a.k, nst, a.err);                \
     return (int)cudaGetLastError();                                                                            \

@@ -121,6 +121,24 @@ struct DenseArgs {
 };
 int launch_dense_attn(const DenseArgs& a, void* stream);
 
+// Launch accounting: a ProfScope wraps one kernel launch; it always counts the
+// launch and, while profiling is enabled (msa_profile_enable), records a CUDA
+// event pair around it on the launch stream.
+void prof_count_launch(int n);
+class ProfScope {
+ public:
+  ProfScope(const char* name, void* stream);
+  ~ProfScope();
+  ProfScope(const ProfScope&) = delete;
+  ProfScope& operator=(const ProfScope&) = delete;
+
+ private:
+  const char* name_;
+  void* stream_;
+  void* start_;
+  void* stop_;
+};
+
 // Tensor-map creation (driver entry point resolved at run time).
 int make_tmap_bf16(void* tmap_out, const void* base, int rank, const uint64_t* dims,
                    const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes);

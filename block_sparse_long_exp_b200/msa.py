@@ -25,6 +25,7 @@ EXPORTED = [
     "msa_index_topk_workspace_size", "msa_index_topk",
     "msa_sparse_attn_workspace_size", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
     "msa_combine", "msa_dense_attn_workspace_size", "msa_dense_attn",
+    "msa_profile_enable", "msa_profile_reset", "msa_profile_read",
     "msa_get_device_error", "msa_version",
 ]
 
@@ -78,6 +79,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_dense_attn.restype = i32
     lib.msa_get_device_error.argtypes = [vp, P(i32), P(i32), P(i32), P(i32), vp]
     lib.msa_get_device_error.restype = i32
+    lib.msa_profile_enable.argtypes = [ctypes.c_int]
+    lib.msa_profile_enable.restype = i32
+    lib.msa_profile_reset.argtypes = []
+    lib.msa_profile_reset.restype = i32
+    lib.msa_profile_read.argtypes = [ctypes.c_char_p, P(ctypes.c_double), P(i64)]
+    lib.msa_profile_read.restype = i32
     lib.msa_version.argtypes = []
     lib.msa_version.restype = ctypes.c_char_p
     _lib = lib
@@ -125,7 +132,7 @@ def _require_cuda(t: torch.Tensor):
 
 def msa_index_topk(shape: Shape, seqs: Varlen, q_idx: torch.Tensor, k_idx: torch.Tensor,
                    sel: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
-                   stream=None) -> torch.Tensor:
+                   stream=None, check: bool = True) -> torch.Tensor:
     lib = load_library()
     _require_cuda(q_idx)
     T = seqs.total_q
@@ -139,7 +146,8 @@ def msa_index_topk(shape: Shape, seqs: Varlen, q_idx: torch.Tensor, k_idx: torch
     rc = lib.msa_index_topk(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q_idx), _ptr(k_idx), _ptr(sel),
                             _ptr(ws), ws.numel(), _stream(stream))
     _check(rc, "msa_index_topk")
-    _device_check(ws, stream, "msa_index_topk")
+    if check:
+        _device_check(ws, stream, "msa_index_topk")
     return sel
 
 
@@ -244,6 +252,22 @@ def _device_check(ws: torch.Tensor, stream, what: str):
     code, where, i0, i1 = msa_get_device_error(ws, stream)
     if code != MSA_OK:
         raise MsaError(f"{what}: device reported {STATUS.get(code, code)} at site {where} ({i0}, {i1})")
+
+
+def msa_profile_enable(on: bool = True):
+    _check(load_library().msa_profile_enable(1 if on else 0), "msa_profile_enable")
+
+
+def msa_profile_reset():
+    _check(load_library().msa_profile_reset(), "msa_profile_reset")
+
+
+def msa_profile_read(kernel: Optional[str]) -> Tuple[float, int]:
+    """(total device ms, launches) of one kernel; kernel=None: (0, all launches)."""
+    ms, n = ctypes.c_double(), ctypes.c_int64()
+    rc = load_library().msa_profile_read(kernel.encode() if kernel else None, ctypes.byref(ms), ctypes.byref(n))
+    _check(rc, "msa_profile_read")
+    return ms.value, n.value
 
 
 def msa_version() -> str:

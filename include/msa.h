@@ -177,6 +177,19 @@ msa_status_t msa_dense_attn(const msa_shape_t* shape, const msa_varlen_t* seqs,
                             void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Measurement support (for benchmarks; no counterpart in the method).
+ * msa_profile_enable(1) makes every kernel launch of the library record a CUDA
+ * event pair on its launch stream; msa_profile_read(name, ...) waits for those
+ * events and returns the summed device time (ms) and launch count of the
+ * kernel `name` ("index_topk_prefill", "decode_scan", "decode_select",
+ * "sparse_attn", "combine", "count", "plan", "scatter", "dense_attn", ...).
+ * With name == NULL it returns the number of kernels launched since the last
+ * msa_profile_reset (launches are counted even while timing is disabled). */
+msa_status_t msa_profile_enable(int on);
+msa_status_t msa_profile_reset(void);
+msa_status_t msa_profile_read(const char* kernel, double* total_ms, int64_t* count);
+
+/* ---------------------------------------------------------------------- */
 /* Device error word of a workspace.  Waits for `stream`, copies the word to
  * the host and clears it.  *code is an msa_status_t (MSA_OK if none);
  * *where names the kernel site, *info0 / *info1 carry details. */
