@@ -25,6 +25,7 @@ EXPORTED = [
     "msa_index_topk_workspace_size", "msa_index_topk",
     "msa_sparse_attn_workspace_size", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
     "msa_combine", "msa_dense_attn_workspace_size", "msa_dense_attn",
+    "msa_index_topk_decode_noalloc_max_scratch", "msa_index_topk_decode_noalloc",
     "msa_profile_enable", "msa_profile_reset", "msa_profile_read",
     "msa_get_device_error", "msa_version",
 ]
@@ -79,6 +80,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_dense_attn.restype = i32
     lib.msa_get_device_error.argtypes = [vp, P(i32), P(i32), P(i32), P(i32), vp]
     lib.msa_get_device_error.restype = i32
+    lib.msa_index_topk_decode_noalloc_max_scratch.argtypes = []
+    lib.msa_index_topk_decode_noalloc_max_scratch.restype = sz
+    lib.msa_index_topk_decode_noalloc.argtypes = [P(Shape), P(Varlen), vp, vp, vp, vp, vp]
+    lib.msa_index_topk_decode_noalloc.restype = i32
     lib.msa_profile_enable.argtypes = [ctypes.c_int]
     lib.msa_profile_enable.restype = i32
     lib.msa_profile_reset.argtypes = []
@@ -149,6 +154,23 @@ def msa_index_topk(shape: Shape, seqs: Varlen, q_idx: torch.Tensor, k_idx: torch
     if check:
         _device_check(ws, stream, "msa_index_topk")
     return sel
+
+
+def msa_index_topk_decode_noalloc(shape: Shape, seqs: Varlen, q_idx: torch.Tensor, k_idx: torch.Tensor,
+                                  sel: torch.Tensor, device_error: Optional[torch.Tensor] = None,
+                                  stream=None) -> torch.Tensor:
+    """Decode-shaped index top-k on the library's fixed scratch array (no
+    workspace argument, no allocation inside the call).  `sel` must be given."""
+    lib = load_library()
+    _require_cuda(q_idx)
+    rc = lib.msa_index_topk_decode_noalloc(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q_idx), _ptr(k_idx),
+                                           _ptr(sel), _ptr(device_error), _stream(stream))
+    _check(rc, "msa_index_topk_decode_noalloc")
+    return sel
+
+
+def msa_index_topk_decode_noalloc_max_scratch() -> int:
+    return load_library().msa_index_topk_decode_noalloc_max_scratch()
 
 
 def msa_sparse_attn_workspace_size(shape: Shape, seqs: Varlen, q_chunk: int = 0) -> int:

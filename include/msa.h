@@ -177,6 +177,38 @@ msa_status_t msa_dense_attn(const msa_shape_t* shape, const msa_varlen_t* seqs,
                             void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Decode-shaped index top-k that allocates nothing (the pages have no
+ * counterpart: this is a deployment convenience).
+ *
+ * For callers that cannot allocate device memory when they call in, such as a
+ * serving loop whose framework reserves all device memory up front and hands
+ * out no scratch buffers, or a host that forbids cudaMalloc on the decode path
+ * because cudaMalloc synchronizes the device.  Same operation and layouts as
+ * msa_index_topk with max_q_len <= 1 (one query per sequence); the caller still
+ * passes the inputs and `sel`.
+ *
+ * Scratch: a fixed array inside the library, msa_index_topk_decode_noalloc_
+ * max_scratch() bytes (16 MiB) per GPU, held by every GPU that loads the
+ * library until the process exits.  A call whose scratch need
+ * (msa_index_topk_workspace_size) exceeds it returns MSA_ERR_WORKSPACE and
+ * launches nothing.  Calls and allocations: none (no cudaMalloc/cudaFree).
+ * The first call on a device looks the array's device address up (with that
+ * device current); make that first call before any stream capture.
+ * All calls share the one array, which keeps the last call's contents (each
+ * call clears the error word it needs zeroed): calls that overlap on the GPU
+ * (different streams or devices' contexts sharing it) race; order them.
+ * device_error (device int32, may be NULL) receives the call's device error
+ * code (an msa_status_t, MSA_OK if none), stream-ordered after the call. */
+size_t msa_index_topk_decode_noalloc_max_scratch(void);
+
+msa_status_t msa_index_topk_decode_noalloc(const msa_shape_t* shape, const msa_varlen_t* seqs,
+                                           const void* q_idx,   /* device bf16 [T, G, d_idx] */
+                                           const void* k_idx,   /* device bf16 [S, d_idx] */
+                                           int32_t* sel,        /* device int32 [T, G, k] (out) */
+                                           int32_t* device_error, /* device int32 [1] (out) or NULL */
+                                           void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* Measurement support (for benchmarks; no counterpart in the method).
  * msa_profile_enable(1) makes every kernel launch of the library record a CUDA
  * event pair on its launch stream; msa_profile_read(name, ...) waits for those
