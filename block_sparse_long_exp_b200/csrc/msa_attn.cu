@@ -165,24 +165,54 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
 }
 
 // ------------------------------------------------------------ attention ---
+//
+// Warp-specialised, persistent (one CTA per SM, 384 threads):
+//   warp 0      claims work items (atomic ticket), publishes them in a 4-deep
+//               ring and TMA-loads each item's K and V block into one of two
+//               shared-memory stages;
+//   warp 1      owns TMEM (512 columns = two slots of S/P + O) and issues the
+//               MMAs: S(t+1) = Q K^T is issued before O(t) = P V so the
+//               tensor core works while tile t's softmax runs;
+//   warps 2-3   gather the Q rows of each 128-row tile (cp.async, 16-byte
+//               chunks into the 128-byte-swizzled K-major layout), 3 slots;
+//   warps 4-7   softmax + epilogue of even tiles (TMEM slot 0),
+//   warps 8-11  the same for odd tiles (slot 1): S -> P (bf16, written back
+//               into the S columns, the A operand of the PV MMA), then O / l
+//               -> f16 partial and the log-sum-exp of each row.
 
-constexpr int kAttnThreads = 128;
+constexpr int kAttnThreads = 384;
+constexpr int kItemRing = 4;
+constexpr int kQSlots = 3;
+constexpr int kItemEmptyCount = 11;   // gather warps 2 + MMA 1 + softmax warps 8
 
-struct __align__(16) AttnCtl {
-  uint64_t kv_full, s_full, o_full, mma_done;
-  uint32_t tmem_base;
-  int32_t item;
-  int32_t abort_flag;
-  int32_t pad[3];
-  uint32_t entry[128];  // entries of the current 128-row tile (one per query)
+struct __align__(16) RingItem {
+  int32_t seq, blk, g, start, count, pad0, pad1, pad2;
 };
 
-// Layout of one K-major [128 rows x D] bf16 tile: D/64 column halves of
-// [128 rows x 128 bytes], 128-byte swizzle.
-__device__ __forceinline__ uint32_t kmajor_off(int row, int col_chunk /* 16-byte chunk along D */) {
-  const int half = col_chunk >> 3;
-  return half * (128 * 128) + swz_offset(row, col_chunk & 7, 128);
+struct __align__(16) AttnCtl {
+  uint64_t item_full[kItemRing], item_empty[kItemRing];
+  uint64_t kv_full[2], kv_empty[2];
+  uint64_t q_full[kQSlots], q_empty[kQSlots];
+  uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int32_t abort_flag;
+  int32_t pad[2];
+  RingItem ring[kItemRing];
+};
+
+// Byte offset of 16-byte chunk `col` (along the 2*D-byte row) of row `row` in a
+// K-major [128 x D] bf16 tile stored as D/64 column halves of [128 x 128 B]
+// with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t kmajor_off(int row, int col) {
+  return (col >> 3) * (128 * 128) + swz_offset(row, col & 7, 128);
 }
+
+struct TileRef {
+  int tau;        // tile counter of this CTA
+  int item_seq;   // item counter of this CTA
+  bool first, last;
+};
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -194,189 +224,280 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  const int tile_bytes = 128 * d * 2;       // one [128 x d] bf16 tile
-  uint8_t* k_s = smem;
-  uint8_t* v_s = k_s + tile_bytes;
-  uint8_t* q_s = v_s + tile_bytes;
-  uint8_t* p_s = q_s + tile_bytes;           // [128 x 128] bf16 = 32 KB
-  AttnCtl* ctl = reinterpret_cast<AttnCtl*>(p_s + 128 * 128 * 2);
+  const int tile_bytes = 128 * d * 2;         // one [128 x d] bf16 tile
+  uint8_t* kv_s = smem;                        // 2 stages x (K, V)
+  uint8_t* q_s = kv_s + 4 * tile_bytes;        // kQSlots tiles
+  AttnCtl* ctl = reinterpret_cast<AttnCtl*>(q_s + kQSlots * tile_bytes);
   volatile int32_t* abort_flag = &ctl->abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Hg = H / G;
-  const int qpt = 128 / Hg;                   // queries per 128-row tile
+  const int qpt = 128 / Hg;                    // queries per 128-row tile
   const int nhalf = d / 64;
+  const int nitems = *nitems_p;
 
   if (tid == 0) {
-    mbar_init(&ctl->kv_full, 1);
-    mbar_init(&ctl->s_full, 1);
-    mbar_init(&ctl->o_full, 1);
+    for (int i = 0; i < kItemRing; ++i) { mbar_init(&ctl->item_full[i], 1); mbar_init(&ctl->item_empty[i], kItemEmptyCount); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl->kv_full[i], 1); mbar_init(&ctl->kv_empty[i], 1);
+      mbar_init(&ctl->s_full[i], 1); mbar_init(&ctl->p_full[i], 4);
+      mbar_init(&ctl->o_full[i], 1); mbar_init(&ctl->o_free[i], 4);
+    }
+    for (int i = 0; i < kQSlots; ++i) { mbar_init(&ctl->q_full[i], 2); mbar_init(&ctl->q_empty[i], 1); }
     mbar_init(&ctl->mma_done, 1);
     ctl->abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
-  if (warp == 0) {
-    tmem_alloc(&ctl->tmem_base, 256);
+  if (warp == 1) {
+    tmem_alloc(&ctl->tmem_base, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_s = ctl->tmem_base;        // columns 0..127: S
-  const uint32_t tmem_o = ctl->tmem_base + 128;  // columns 128..128+d: O
-  const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
-  const int nitems = *nitems_p;
-  const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
-  const uint32_t idesc_o = idesc_bf16_f32(128, d, 0, 1);
-  uint32_t kv_phase = 0, s_phase = 0, o_phase = 0;
-  bool issued_kv = false;
+  const uint32_t tmem = ctl->tmem_base;
 
-  while (true) {
-    if (tid == 0) ctl->item = atomicAdd(ticket, 1);
-    __syncthreads();
-    const int it = ctl->item;
-    if (it >= nitems || *abort_flag) break;
-    const Item I = items[it];
-    const int Tb = cu_q[I.seq + 1] - cu_q[I.seq];
-    const int Sb = cu_k[I.seq + 1] - cu_k[I.seq];
-    const int64_t qrow0 = cu_q[I.seq];
-    const int blk_first_pos = I.blk * kBk;
-
-    if (tid == 0) {
-      mbar_arrive_expect_tx(&ctl->kv_full, 2 * tile_bytes);
-      const int krow = cu_k[I.seq] + I.blk * kBk;
-      for (int h = 0; h < nhalf; ++h) {
-        tma_load_3d(k_s + h * 128 * 128, &tm_k, &ctl->kv_full, 64 * h, I.g, krow);
-        tma_load_3d(v_s + h * 128 * 128, &tm_v, &ctl->kv_full, 64 * h, I.g, krow);
-      }
-      issued_kv = true;
+  // Reads the next ring item (every consumer warp calls this in the same order).
+  // whole_warp: all 32 lanes call it (else only lane 0 of the warp does).
+  auto take_item = [&](int n, RingItem& out, bool whole_warp) -> bool {
+    const int slot = n % kItemRing;
+    if (!mbar_wait(&ctl->item_full[slot], (n / kItemRing) & 1)) {
+      report_error(err, MSA_ERR_TIMEOUT, kSiteAttnItem, n, warp);
+      *abort_flag = 1;
+      return false;
     }
-    const int ntiles = (I.count + qpt - 1) / qpt;
-    bool ok = true;
-    for (int mt = 0; mt < ntiles && ok; ++mt) {
-      const int nq = min(qpt, I.count - mt * qpt);
-      if (tid < nq) ctl->entry[tid] = entries[I.start + mt * qpt + tid];
-      __syncthreads();
-      // ---- gather the Q rows of this tile: row r = ql * Hg + i
-      {
-        const int chunks_per_row = d / 8;               // 16-byte chunks
-        const int rows_per_pass = kAttnThreads / chunks_per_row;
-        const int c = tid % chunks_per_row;
-        for (int r = tid / chunks_per_row; r < nq * Hg; r += rows_per_pass) {
-          const int ql = r / Hg, i = r - ql * Hg;
-          const uint32_t e = ctl->entry[ql];
-          const int64_t t = t0 + e / k;
-          const __nv_bfloat16* src = q + ((t * H) + (int64_t)I.g * Hg + i) * d + c * 8;
-          cp_async_16(q_s + kmajor_off(r, c), src);
+    out = ctl->ring[slot];
+    if (whole_warp) __syncwarp();
+    if (lane == 0) mbar_arrive(&ctl->item_empty[slot]);
+    return out.count > 0;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------ scheduler + K/V loads
+    if (lane == 0) {
+      int n = 0;
+      while (true) {
+        const int slot = n % kItemRing;
+        if (!mbar_wait(&ctl->item_empty[slot], ((n / kItemRing) + 1) & 1)) {
+          report_error(err, MSA_ERR_TIMEOUT, kSiteAttnLoad, n, 0);
+          *abort_flag = 1;
+          break;
+        }
+        const int it = *abort_flag ? nitems : atomicAdd(ticket, 1);
+        RingItem r;
+        if (it >= nitems) {
+          r.count = 0;
+          ctl->ring[slot] = r;
+          mbar_arrive(&ctl->item_full[slot]);
+          break;
+        }
+        const Item I = items[it];
+        r.seq = I.seq; r.blk = I.blk; r.g = I.g; r.start = I.start; r.count = I.count;
+        ctl->ring[slot] = r;
+        mbar_arrive(&ctl->item_full[slot]);
+        const int st = n & 1;
+        if (!mbar_wait(&ctl->kv_empty[st], ((n >> 1) + 1) & 1)) {
+          report_error(err, MSA_ERR_TIMEOUT, kSiteAttnLoad, n, 1);
+          *abort_flag = 1;
+          break;
+        }
+        uint8_t* ks = kv_s + st * 2 * tile_bytes;
+        mbar_arrive_expect_tx(&ctl->kv_full[st], 2 * tile_bytes);
+        const int krow = cu_k[I.seq] + I.blk * kBk;
+        for (int h = 0; h < nhalf; ++h) {
+          tma_load_3d(ks + h * 128 * 128, &tm_k, &ctl->kv_full[st], 64 * h, I.g, krow);
+          tma_load_3d(ks + tile_bytes + h * 128 * 128, &tm_v, &ctl->kv_full[st], 64 * h, I.g, krow);
+        }
+        ++n;
+      }
+      // no K/V load may still be in flight when the CTA exits
+      for (int st = 0; st < 2; ++st) {
+        const int issued = n > st ? (n - st + 1) / 2 : 0;
+        if (issued > 0) mbar_wait(&ctl->kv_full[st], (issued - 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t idesc_o = idesc_bf16_f32(128, d, 0, 1);
+      int n = 0, tau = 0;
+      RingItem cur;
+      int cur_tiles = 0, mt = 0, cur_seq = -1;
+      bool have = false, ok = true;
+      // next tile in the stream (consumes items as needed)
+      auto next_tile = [&](TileRef& tr) -> bool {
+        if (!have || mt >= cur_tiles) {
+          if (!take_item(n, cur, false)) return false;
+          cur_seq = n++;
+          cur_tiles = (cur.count + qpt - 1) / qpt;
+          mt = 0;
+          have = true;
+        }
+        tr.tau = tau++;
+        tr.item_seq = cur_seq;
+        tr.first = (mt == 0);
+        tr.last = (mt == cur_tiles - 1);
+        ++mt;
+        return true;
+      };
+      auto issue_s = [&](const TileRef& tr) -> bool {
+        const int qs = tr.tau % kQSlots, s = tr.tau & 1, st = tr.item_seq & 1;
+        if (!mbar_wait(&ctl->q_full[qs], (tr.tau / kQSlots) & 1)) return false;
+        if (tr.first && !mbar_wait(&ctl->kv_full[st], (tr.item_seq >> 1) & 1)) return false;
+        tc_fence_after();
+        const uint32_t qa = smem_u32(q_s + qs * tile_bytes), ka = smem_u32(kv_s + st * 2 * tile_bytes);
+        for (int kk = 0; kk < d / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          umma_bf16_ss(tmem + s * 256, make_sdesc(qa + off, 16, 1024, kSw128), make_sdesc(ka + off, 16, 1024, kSw128),
+                       idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&ctl->s_full[s]);
+        umma_commit(&ctl->q_empty[qs]);
+        return true;
+      };
+      auto issue_pv = [&](const TileRef& tr) -> bool {
+        const int s = tr.tau & 1, st = tr.item_seq & 1;
+        if (!mbar_wait(&ctl->p_full[s], (tr.tau >> 1) & 1)) return false;
+        if (!mbar_wait(&ctl->o_free[s], ((tr.tau >> 1) + 1) & 1)) return false;
+        tc_fence_after();
+        const uint32_t va = smem_u32(kv_s + st * 2 * tile_bytes + tile_bytes);
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16_ts(tmem + s * 256 + 128, tmem + s * 256 + kk * 8,
+                       make_sdesc(va + kk * 2048, 128 * 128, 1024, kSw128), idesc_o, kk > 0 ? 1u : 0u);
+        umma_commit(&ctl->o_full[s]);
+        if (tr.last) umma_commit(&ctl->kv_empty[st]);
+        return true;
+      };
+      TileRef t0r, t1r;
+      if (next_tile(t0r)) {
+        ok = issue_s(t0r);
+        while (ok && !*abort_flag) {
+          const bool more = next_tile(t1r);
+          if (more && !(ok = issue_s(t1r))) break;
+          if (!(ok = issue_pv(t0r))) break;
+          if (!more) break;
+          t0r = t1r;
+        }
+      }
+      if (!ok) {
+        report_error(err, MSA_ERR_TIMEOUT, kSiteAttnMma, tau, n);
+        *abort_flag = 1;
+      }
+      umma_commit(&ctl->mma_done);
+      mbar_wait(&ctl->mma_done, 0);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ Q gather
+    const int gt = tid - 64;                   // 0..63
+    const int cpr = d / 8;                     // 16-byte chunks per row
+    int n = 0, tau = 0;
+    RingItem I;
+    while (!*abort_flag && take_item(n++, I, true)) {
+      const int ntiles = (I.count + qpt - 1) / qpt;
+      for (int mt = 0; mt < ntiles; ++mt, ++tau) {
+        const int qs = tau % kQSlots;
+        if (!mbar_wait(&ctl->q_empty[qs], ((tau / kQSlots) + 1) & 1)) {
+          report_error(err, MSA_ERR_TIMEOUT, kSiteAttnLoad, tau, 2);
+          *abort_flag = 1;
+          break;
+        }
+        const int nq = min(qpt, I.count - mt * qpt);
+        uint8_t* dst = q_s + qs * tile_bytes;
+        const uint32_t* ent = entries + I.start + mt * qpt;
+        for (int c = gt; c < nq * Hg * cpr; c += 64) {
+          const int row = c / cpr, col = c - row * cpr;
+          const int ql = row / Hg, i = row - ql * Hg;
+          const int64_t t = t0 + ent[ql] / k;
+          cp_async_16(dst + kmajor_off(row, col), q + ((t * H) + (int64_t)I.g * Hg + i) * d + col * 8);
         }
         cp_async_commit();
         cp_async_wait_all();
         fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->q_full[qs]);
       }
-      tc_fence_before();
-      __syncthreads();
-      // ---- S = Q K^T
-      if (tid == 0) {
-        if (mt == 0 && !mbar_wait(&ctl->kv_full, kv_phase)) {
-          report_error(err, MSA_ERR_TIMEOUT, kSiteAttnLoad, it, 0);
+    }
+  } else {
+    // ------------------------------------------------- softmax + epilogue
+    const int wg = (warp - 4) >> 2;           // slot handled by this warpgroup
+    const int wq = warp & 3;                  // TMEM lane quarter
+    const int r = 32 * wq + lane;             // tile row
+    const uint32_t lane_off = static_cast<uint32_t>(32 * wq) << 16;
+    const uint32_t s_col = tmem + wg * 256 + lane_off;      // S, then P (first 64 columns)
+    const uint32_t o_col = s_col + 128;                     // O
+    const int ql = r / Hg, hi = r - ql * Hg;
+    int n = 0, tau = 0;
+    RingItem I;
+    while (!*abort_flag && take_item(n++, I, true)) {
+      const int ntiles = (I.count + qpt - 1) / qpt;
+      const int Tb = cu_q[I.seq + 1] - cu_q[I.seq];
+      const int Sb = cu_k[I.seq + 1] - cu_k[I.seq];
+      const int64_t qrow0 = cu_q[I.seq];
+      const int64_t blk_first = (int64_t)I.blk * kBk;
+      for (int mt = 0; mt < ntiles; ++mt, ++tau) {
+        if ((tau & 1) != wg) continue;
+        const int nq = min(qpt, I.count - mt * qpt);
+        const bool valid = ql < nq;
+        uint32_t e = 0;
+        int limit = 127;
+        if (valid) {
+          e = entries[I.start + mt * qpt + ql];
+          const int64_t t = t0 + e / k;
+          const int64_t lim = (int64_t)Sb - Tb + (t - qrow0) - blk_first;
+          limit = lim >= 127 ? 127 : (int)lim;
+        }
+        if (!mbar_wait(&ctl->s_full[wg], (tau >> 1) & 1)) {
+          report_error(err, MSA_ERR_TIMEOUT, kSiteAttnSoftmax, tau, 0);
           *abort_flag = 1;
+          break;
         }
-        if (!*abort_flag) {
-          tc_fence_after();
-          const uint32_t qa = smem_u32(q_s), ka = smem_u32(k_s);
-          for (int kk = 0; kk < d / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-            umma_bf16_ss(tmem_s, make_sdesc(qa + off, 16, 1024, kSw128), make_sdesc(ka + off, 16, 1024, kSw128),
-                         idesc_s, kk > 0 ? 1u : 0u);
-          }
-        }
-        umma_commit(&ctl->s_full);
-      }
-      if (!mbar_wait(&ctl->s_full, s_phase)) {
-        report_error(err, MSA_ERR_TIMEOUT, kSiteAttnSoftmax, it, mt);
-        *abort_flag = 1;
-      }
-      s_phase ^= 1;
-      tc_fence_after();
-      // ---- softmax on this thread's row (lane of TMEM = row)
-      const int r = tid;
-      const int ql = r / Hg, hi = r - ql * Hg;
-      const bool valid = ql < nq;
-      int limit = 127;   // last visible key column of the block for this row
-      uint32_t e = 0;
-      if (valid) {
-        e = ctl->entry[ql];
-        const int64_t t = t0 + e / k;
-        const int64_t pos = (int64_t)Sb - Tb + (t - qrow0);
-        const int64_t lim = pos - blk_first_pos;
-        limit = lim >= 127 ? 127 : (int)lim;
-      }
-      float sv[128];
-      {
+        tc_fence_after();
         uint32_t rr[32];
-#pragma unroll
+        float m = -INFINITY;
+#pragma unroll 1
         for (int c4 = 0; c4 < 4; ++c4) {
-          tmem_ld32(tmem_s + lane_off + 32 * c4, rr);
+          tmem_ld32(s_col + 32 * c4, rr);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) sv[32 * c4 + j] = __uint_as_float(rr[j]);
+          for (int j = 0; j < 32; ++j)
+            if (32 * c4 + j <= limit) m = fmaxf(m, __uint_as_float(rr[j]));
         }
-      }
-      float m = -INFINITY;
+        const float ms = m * scale_log2;
+        float l = 0.f;
+#pragma unroll 1
+        for (int c4 = 0; c4 < 4; ++c4) {
+          tmem_ld32(s_col + 32 * c4, rr);
+          tmem_ld_wait();
+          uint32_t pk[16];
 #pragma unroll
-      for (int j = 0; j < 128; ++j) {
-        sv[j] = (j <= limit) ? sv[j] * scale_log2 : -INFINITY;
-        m = fmaxf(m, sv[j]);
-      }
-      float l = 0.f;
-#pragma unroll
-      for (int j = 0; j < 128; ++j) {
-        sv[j] = exp2f(sv[j] - m);
-        l += sv[j];
-      }
-      // P (unnormalised, bf16) -> shared memory, K-major over the 128 keys
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        uint4 w;
-        w.x = pack_bf16x2(sv[8 * c + 0], sv[8 * c + 1]);
-        w.y = pack_bf16x2(sv[8 * c + 2], sv[8 * c + 3]);
-        w.z = pack_bf16x2(sv[8 * c + 4], sv[8 * c + 5]);
-        w.w = pack_bf16x2(sv[8 * c + 6], sv[8 * c + 7]);
-        *reinterpret_cast<uint4*>(p_s + kmajor_off(r, c)) = w;
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      // ---- O = P V
-      if (tid == 0) {
-        tc_fence_after();
-        if (!*abort_flag) {
-          const uint32_t pa = smem_u32(p_s), va = smem_u32(v_s);
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t aoff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-            const uint32_t boff = kk * 16 * 128;   // 16 keys x 128-byte rows
-            umma_bf16_ss(tmem_o, make_sdesc(pa + aoff, 16, 1024, kSw128),
-                         make_sdesc(va + boff, 128 * 128, 1024, kSw128), idesc_o, kk > 0 ? 1u : 0u);
+          for (int j = 0; j < 16; ++j) {
+            const int c0 = 32 * c4 + 2 * j;
+            const float p0 = c0 <= limit ? exp2f(fmaf(__uint_as_float(rr[2 * j]), scale_log2, -ms)) : 0.f;
+            const float p1 = c0 + 1 <= limit ? exp2f(fmaf(__uint_as_float(rr[2 * j + 1]), scale_log2, -ms)) : 0.f;
+            l += p0 + p1;
+            pk[j] = pack_bf16x2(p0, p1);
           }
+          tmem_st16(s_col + 16 * c4, pk);
         }
-        umma_commit(&ctl->o_full);
-      }
-      if (!mbar_wait(&ctl->o_full, o_phase)) {
-        report_error(err, MSA_ERR_TIMEOUT, kSiteAttnSoftmax, it, 1000 + mt);
-        *abort_flag = 1;
-      }
-      o_phase ^= 1;
-      tc_fence_after();
-      // ---- epilogue: normalise, write the partial of (query, group, slot)
-      {
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->p_full[wg]);
+        // ---- epilogue: O / l -> f16 partial, lse
+        if (!mbar_wait(&ctl->o_full[wg], (tau >> 1) & 1)) {
+          report_error(err, MSA_ERR_TIMEOUT, kSiteAttnSoftmax, tau, 1);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
         const float inv_l = 1.f / l;
         const int64_t unit = valid ? ((int64_t)(e / k) * G + I.g) * k + (e % k) : 0;
         __half* dst = part_acc + (unit * Hg + hi) * d;
-        uint32_t rr[32];
         for (int c4 = 0; c4 < d / 32; ++c4) {
-          tmem_ld32(tmem_o + lane_off + 32 * c4, rr);
+          tmem_ld32(o_col + 32 * c4, rr);
           tmem_ld_wait();
           if (valid) {
 #pragma unroll
@@ -390,29 +511,20 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             }
           }
         }
-        if (valid) part_lse[unit * Hg + hi] = (m + __log2f(l)) * 0.69314718055994530942f;
+        if (valid) part_lse[unit * Hg + hi] = (ms + __log2f(l)) * 0.69314718055994530942f;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->o_free[wg]);
       }
-      tc_fence_before();
-      __syncthreads();
-      ok = !*abort_flag;
     }
-    if (ntiles == 0 && tid == 0) mbar_wait(&ctl->kv_full, kv_phase);  // never leave a load in flight
-    kv_phase ^= 1;
-    __syncthreads();
-    if (!ok) break;
   }
-  if (tid == 0) {
-    // nothing issued by this CTA may still be in flight when TMEM is released
-    umma_commit(&ctl->mma_done);
-    mbar_wait(&ctl->mma_done, 0);
-    if (*abort_flag && issued_kv) mbar_wait(&ctl->kv_full, kv_phase ^ 1);
-  }
+
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(ctl->tmem_base, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -506,7 +618,7 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
   if (rc) return rc;
   rc = make_tmap_bf16(&tm_v, a.value, 3, dims, strides, box, 128);
   if (rc) return rc;
-  const size_t smem = 1024 + 3 * (size_t)128 * a.d * 2 + 128 * 128 * 2 + sizeof(AttnCtl);
+  const size_t smem = 1024 + (4 + kQSlots) * (size_t)128 * a.d * 2 + sizeof(AttnCtl);
   e = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return (int)e;
   int dev = 0, nsm = 0;
