@@ -318,7 +318,7 @@ def run_ours(args):
     w = W.WORKLOADS[args.workload]
     # each rank runs an independent layer (its own seed): weak scaling
     wr = W.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
-    inp = W.make_inputs(wr, "cuda")
+    inp = W.make_inputs(wr, "cuda", T_override=args.T or None)
     torch.cuda.synchronize()
     ctx = make_ctx(wr, inp, torch, msa)
     S_lens = [inp["cu_k_host"][i + 1] - inp["cu_k_host"][i] for i in range(len(inp["cu_k_host"]) - 1)]
@@ -467,6 +467,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=PREFILL)
+    ap.add_argument("--T", type=int, default=0, help="shorter prefill (same heads/dims), for profiling")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
