@@ -49,7 +49,7 @@ int64_t total_blocks_bound(const msa_varlen_t* v) { return (v->total_k + kBk - 1
 
 // Slices of a sparse-attention workspace for chunks of `rows` query rows.
 struct AttnLayout {
-  size_t blk_off, counts, offsets, cursor, item_off, nitems, entries, items, part_acc, part_lse, total;
+  size_t blk_off, counts, cursor, tile_sums, nitems, entries, items, part_acc, part_lse, total;
   int64_t nlists, max_items;
   int32_t qpi;
 };
@@ -57,10 +57,12 @@ struct AttnLayout {
 AttnLayout attn_layout(const msa_shape_t* s, const msa_varlen_t* v, int64_t rows) {
   AttnLayout L{};
   const int hg = s->H / s->G;
-  L.qpi = 8 * (128 / hg);                 // 8 tiles of 128 rows per work item
+  const int qpt = 128 / (hg < 8 ? 8 : hg);            // queries per 128-row tile
+  L.qpi = 8 * qpt < kMaxItemQueries ? 8 * qpt : kMaxItemQueries;
   L.nlists = (int64_t)s->G * total_blocks_bound(v);
+  const int64_t nkeys = ((rows + kWindow - 1) / kWindow) * L.nlists;
   const int64_t nentries = rows * s->G * s->k;
-  L.max_items = L.nlists + (nentries + L.qpi - 1) / L.qpi + 1;
+  L.max_items = nentries / L.qpi + (nkeys < nentries ? nkeys : nentries) + 1;
   size_t off = kWsHeader;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -68,11 +70,10 @@ AttnLayout attn_layout(const msa_shape_t* s, const msa_varlen_t* v, int64_t rows
     return o;
   };
   L.blk_off = take(sizeof(int32_t) * (v->batch + 1));
-  L.counts = take(sizeof(int32_t) * L.nlists);
-  L.offsets = take(sizeof(int32_t) * (L.nlists + 1));
-  L.cursor = take(sizeof(int32_t) * L.nlists);
-  L.item_off = take(sizeof(int32_t) * (L.nlists + 1));
-  L.nitems = take(sizeof(int32_t) * 2);
+  L.counts = take(sizeof(int32_t) * nkeys);
+  L.cursor = take(sizeof(int32_t) * nkeys);
+  L.tile_sums = take(sizeof(int32_t) * 2 * ((nkeys + kScanTile - 1) / kScanTile + 1));
+  L.nitems = take(sizeof(int32_t) * 4);
   L.entries = take(sizeof(uint32_t) * nentries);
   L.items = take(sizeof(Item) * L.max_items);
   L.part_acc = take((size_t)nentries * hg * s->d * 2);
@@ -111,9 +112,8 @@ msa_status_t attn_common(const msa_shape_t* shape, const msa_varlen_t* seqs, con
   a.err = reinterpret_cast<DevError*>(base);
   a.blk_off = reinterpret_cast<int32_t*>(base + L.blk_off);
   a.counts = reinterpret_cast<int32_t*>(base + L.counts);
-  a.offsets = reinterpret_cast<int32_t*>(base + L.offsets);
   a.cursor = reinterpret_cast<int32_t*>(base + L.cursor);
-  a.item_off = reinterpret_cast<int32_t*>(base + L.item_off);
+  a.tile_sums = reinterpret_cast<int32_t*>(base + L.tile_sums);
   a.nitems = reinterpret_cast<int32_t*>(base + L.nitems);
   a.entries = reinterpret_cast<uint32_t*>(base + L.entries);
   a.items = reinterpret_cast<Item*>(base + L.items);

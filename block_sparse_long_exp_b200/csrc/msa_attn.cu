@@ -20,6 +20,7 @@
 namespace msa {
 namespace {
 
+
 // ------------------------------------------------------------- helpers ---
 
 __device__ __forceinline__ int find_seq(const int32_t* __restrict__ cu, int batch, int64_t row) {
@@ -44,7 +45,7 @@ __global__ void block_offsets_kernel(const int32_t* __restrict__ cu_k, int batch
 
 // Validates an entry and returns its list id, or -1 (slot empty or invalid).
 __device__ __forceinline__ int entry_list(int blk, int64_t t, int g, int G, int batch, const int32_t* cu_q,
-                                          const int32_t* cu_k, const int32_t* blk_off, DevError* err, int* seq_out) {
+                                          const int32_t* cu_k, const int32_t* blk_off, DevError* err) {
   if (blk < 0) return -1;
   const int b = find_seq(cu_q, batch, t);
   const int Tb = cu_q[b + 1] - cu_q[b];
@@ -54,139 +55,198 @@ __device__ __forceinline__ int entry_list(int blk, int64_t t, int g, int G, int 
     report_error(err, MSA_ERR_DEVICE_CHECK, kSiteInvert, (int)t, blk);
     return -1;
   }
-  *seq_out = b;
   return (blk_off[b] + blk) * G + g;
 }
 
-// Pass 1 and 3: one thread per (query, group).  scatter == false counts,
-// scatter == true claims positions from `cursor` and writes the entries.
+// Pass 1 and 3: one thread per (query, group).  Lists are keyed by
+// (window of kWindow query rows, sequence block, group) so that the work
+// items come out window-major (the queries of one window stay hot in L2).
+// kScatter == false counts, == true claims positions from `counter`
+// (the cursors) and writes the entries (t - t0) * k + slot.
 template <bool kScatter>
 __global__ void count_scatter_kernel(const int32_t* __restrict__ sel, int64_t t0, int64_t t1, int G, int k,
                                      int batch, const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_k,
-                                     const int32_t* __restrict__ blk_off, int32_t* __restrict__ counter,
-                                     uint32_t* __restrict__ entries, DevError* err) {
+                                     const int32_t* __restrict__ blk_off, int64_t nlists,
+                                     int32_t* __restrict__ counter, uint32_t* __restrict__ entries,
+                                     DevError* err) {
   const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t n = (t1 - t0) * G;
   const bool active = gid < n;
-  const int64_t t = t0 + (active ? gid / G : 0);
+  const int64_t tl = active ? gid / G : 0;
+  const int64_t t = t0 + tl;
   const int g = active ? (int)(gid % G) : 0;
+  const int64_t wbase = (tl / kWindow) * nlists;
   const int lane = threadIdx.x & 31;
   for (int s = 0; s < k; ++s) {
-    int L = -1, seq = 0;
-    if (active) L = entry_list(sel[(t * G + g) * k + s], t, g, G, batch, cu_q, cu_k, blk_off, err, &seq);
-    // warp-aggregated atomics: lanes with the same list share one atomic
-    const unsigned peers = __match_any_sync(0xffffffffu, L);
+    int64_t key = -1;
+    if (active) {
+      const int L = entry_list(sel[(t * G + g) * k + s], t, g, G, batch, cu_q, cu_k, blk_off, err);
+      if (L >= 0) key = wbase + L;
+    }
+    // warp-aggregated atomics: lanes with the same key share one atomic
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
     const int leader = __ffs(peers) - 1;
     const int rank = __popc(peers & ((1u << lane) - 1u));
     int base = 0;
-    if (L >= 0 && lane == leader) base = atomicAdd(&counter[L], __popc(peers));
+    if (key >= 0 && lane == leader) base = atomicAdd(&counter[key], __popc(peers));
     base = __shfl_sync(0xffffffffu, base, leader);
-    if (kScatter && L >= 0) entries[base + rank] = (uint32_t)((t - t0) * k + s);
+    if (kScatter && key >= 0) entries[base + rank] = (uint32_t)(tl * k + s);
   }
 }
 
-// Pass 2: one CTA.  offsets = exclusive scan of counts; items per list =
-// ceil(count / C); cursor = offsets (for the scatter); then the items.
-__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ counts, int64_t nlists, int G,
-                                                    int batch, const int32_t* __restrict__ blk_off, int C,
-                                                    int32_t* __restrict__ offsets, int32_t* __restrict__ cursor,
-                                                    int32_t* __restrict__ item_off, int32_t* __restrict__ nitems,
-                                                    Item* __restrict__ items, int64_t max_items, DevError* err) {
-  __shared__ int32_t warp_a[32], warp_b[32];
-  __shared__ int32_t carry_a, carry_b;
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  if (tid == 0) { carry_a = 0; carry_b = 0; }
+// Device-wide exclusive scan of the list counts (and of their item counts,
+// ceil(count / C)) in three passes over tiles of kScanTile keys.
+constexpr int kScanThreads = 512;
+constexpr int kScanPer = 8;
+static_assert(kScanTile == kScanThreads * kScanPer, "scan tile");
+
+__device__ __forceinline__ void block_scan2(int& a, int& b, int* sa, int* sb) {
+  // inclusive scan of (a, b) over the block; sa/sb: 32-int shared scratch
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int ya = __shfl_up_sync(0xffffffffu, a, o), yb = __shfl_up_sync(0xffffffffu, b, o);
+    if (lane >= o) { a += ya; b += yb; }
+  }
+  if (lane == 31) { sa[wid] = a; sb[wid] = b; }
   __syncthreads();
-  for (int64_t base = 0; base < nlists; base += 1024) {
-    const int64_t L = base + tid;
-    const int c = L < nlists ? counts[L] : 0;
-    const int ni = (c + C - 1) / C;
-    int a = c, b = ni;  // inclusive warp scans
+  if (wid == 0) {
+    int wa = lane < kScanThreads / 32 ? sa[lane] : 0, wb = lane < kScanThreads / 32 ? sb[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int ya = __shfl_up_sync(0xffffffffu, a, o), yb = __shfl_up_sync(0xffffffffu, b, o);
-      if (lane >= o) { a += ya; b += yb; }
+      const int ya = __shfl_up_sync(0xffffffffu, wa, o), yb = __shfl_up_sync(0xffffffffu, wb, o);
+      if (lane >= o) { wa += ya; wb += yb; }
     }
-    if (lane == 31) { warp_a[wid] = a; warp_b[wid] = b; }
-    __syncthreads();
-    if (wid == 0) {
-      int wa = warp_a[lane], wb = warp_b[lane];
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int ya = __shfl_up_sync(0xffffffffu, wa, o), yb = __shfl_up_sync(0xffffffffu, wb, o);
-        if (lane >= o) { wa += ya; wb += yb; }
-      }
-      warp_a[lane] = wa;
-      warp_b[lane] = wb;
-    }
-    __syncthreads();
-    const int pa = carry_a + (wid ? warp_a[wid - 1] : 0) + a - c;
-    const int pb = carry_b + (wid ? warp_b[wid - 1] : 0) + b - ni;
-    if (L < nlists) {
-      offsets[L] = pa;
-      cursor[L] = pa;
-      item_off[L] = pb;
-    }
-    __syncthreads();
-    if (tid == 1023) { carry_a = pa + c; carry_b = pb + ni; }
-    __syncthreads();
-  }
-  if (tid == 0) {
-    offsets[nlists] = carry_a;
-    item_off[nlists] = carry_b;
-    *nitems = carry_b <= max_items ? carry_b : 0;
-    if (carry_b > max_items) report_error(err, MSA_ERR_WORKSPACE, kSiteInvert, carry_b, (int)max_items);
+    if (lane < kScanThreads / 32) { sa[lane] = wa; sb[lane] = wb; }
   }
   __syncthreads();
-  if (item_off[nlists] > max_items) return;
-  // items
-  for (int64_t L = tid; L < nlists; L += 1024) {
-    const int c = counts[L];
-    if (c == 0) continue;
-    const int gb = (int)(L / G), g = (int)(L % G);
-    int lo = 0, hi = batch;
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (blk_off[mid] <= gb) lo = mid; else hi = mid;
+  if (wid > 0) { a += sa[wid - 1]; b += sb[wid - 1]; }
+}
+
+__global__ void __launch_bounds__(kScanThreads) scan_reduce_kernel(const int32_t* __restrict__ counts, int64_t nkeys,
+                                                                  int C, int32_t* __restrict__ tile_sums) {
+  __shared__ int sa[32], sb[32];
+  const int64_t base = (int64_t)blockIdx.x * kScanTile + (int64_t)threadIdx.x * kScanPer;
+  int a = 0, b = 0;
+#pragma unroll
+  for (int i = 0; i < kScanPer; ++i) {
+    const int c = base + i < nkeys ? counts[base + i] : 0;
+    a += c;
+    b += (c + C - 1) / C;
+  }
+  block_scan2(a, b, sa, sb);
+  if (threadIdx.x == kScanThreads - 1) {
+    tile_sums[2 * blockIdx.x] = a;
+    tile_sums[2 * blockIdx.x + 1] = b;
+  }
+}
+
+// One CTA: exclusive scan of the tile sums (in place); totals -> nitems.
+__global__ void __launch_bounds__(kScanThreads) scan_tiles_kernel(int32_t* __restrict__ tile_sums, int ntiles,
+                                                                 int32_t* __restrict__ totals, int64_t max_items,
+                                                                 DevError* err) {
+  __shared__ int sa[32], sb[32];
+  __shared__ int carry_a, carry_b;
+  if (threadIdx.x == 0) { carry_a = 0; carry_b = 0; }
+  __syncthreads();
+  for (int base = 0; base < ntiles; base += kScanThreads) {
+    const int i = base + threadIdx.x;
+    const int a0 = i < ntiles ? tile_sums[2 * i] : 0, b0 = i < ntiles ? tile_sums[2 * i + 1] : 0;
+    int a = a0, b = b0;
+    block_scan2(a, b, sa, sb);
+    const int ea = carry_a + a - a0, eb = carry_b + b - b0;
+    if (i < ntiles) { tile_sums[2 * i] = ea; tile_sums[2 * i + 1] = eb; }
+    __syncthreads();
+    if (threadIdx.x == kScanThreads - 1) { carry_a = ea + a0; carry_b = eb + b0; }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const bool fits = carry_b <= max_items;
+    totals[0] = fits ? carry_b : 0;      // items (the attention kernel's bound)
+    totals[1] = 0;                       // item ticket
+    totals[2] = carry_a;                 // entries
+    if (!fits) report_error(err, MSA_ERR_WORKSPACE, kSiteInvert, carry_b, (int)max_items);
+  }
+}
+
+// Final pass: list offsets and cursors, then the work items of each list
+// (chunks of at most C entries), in key order (window-major).
+__global__ void __launch_bounds__(kScanThreads) scan_items_kernel(const int32_t* __restrict__ counts, int64_t nkeys,
+                                                                 int64_t nlists, int G, int batch, int C,
+                                                                 const int32_t* __restrict__ tile_sums,
+                                                                 const int32_t* __restrict__ blk_off,
+                                                                 int32_t* __restrict__ cursor,
+                                                                 Item* __restrict__ items, int64_t max_items) {
+  __shared__ int sa[32], sb[32];
+  const int64_t base = (int64_t)blockIdx.x * kScanTile + (int64_t)threadIdx.x * kScanPer;
+  int cnt[kScanPer];
+  int a = 0, b = 0;
+#pragma unroll
+  for (int i = 0; i < kScanPer; ++i) {
+    cnt[i] = base + i < nkeys ? counts[base + i] : 0;
+    a += cnt[i];
+    b += (cnt[i] + C - 1) / C;
+  }
+  int ia = a, ib = b;
+  block_scan2(ia, ib, sa, sb);
+  int off = tile_sums[2 * blockIdx.x] + ia - a;
+  int io = tile_sums[2 * blockIdx.x + 1] + ib - b;
+#pragma unroll
+  for (int i = 0; i < kScanPer; ++i) {
+    const int64_t key = base + i;
+    if (key >= nkeys) break;
+    cursor[key] = off;
+    const int c = cnt[i];
+    if (c > 0) {
+      const int64_t L = key % nlists;
+      const int gb = (int)(L / G), g = (int)(L % G);
+      int lo = 0, hi = batch;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (blk_off[mid] <= gb) lo = mid; else hi = mid;
+      }
+      for (int s = 0; s < c; s += C, ++io) {
+        if (io >= max_items) break;
+        Item it;
+        it.seq = lo;
+        it.blk = gb - blk_off[lo];
+        it.g = g;
+        it.start = off + s;
+        it.count = min(C, c - s);
+        it.pad0 = it.pad1 = it.pad2 = 0;
+        items[io] = it;
+      }
     }
-    const int off = offsets[L];
-    int io = item_off[L];
-    for (int s = 0; s < c; s += C, ++io) {
-      Item it;
-      it.seq = lo;
-      it.blk = gb - blk_off[lo];
-      it.g = g;
-      it.start = off + s;
-      it.count = min(C, c - s);
-      it.pad0 = it.pad1 = it.pad2 = 0;
-      items[io] = it;
-    }
+    off += c;
   }
 }
 
 // ------------------------------------------------------------ attention ---
 //
 // Warp-specialised, persistent (one CTA per SM, 384 threads):
-//   warp 0      claims work items (atomic ticket), publishes them in a 4-deep
-//               ring and TMA-loads each item's K and V block into one of two
-//               shared-memory stages;
+//   warp 0      claims work items (atomic ticket) and publishes each one with
+//               its query entries in a 4-deep shared-memory ring; lane 0 then
+//               TMA-loads the item's K and V block into one of two stages and
+//               gathers each 128-row tile's query rows with one TMA box per
+//               (query, 64-column half) into one of three Q slots;
 //   warp 1      owns TMEM (512 columns = two slots of S/P + O) and issues the
 //               MMAs: S(t+1) = Q K^T is issued before O(t) = P V so the
 //               tensor core works while tile t's softmax runs;
-//   warps 2-3   gather the Q rows of each 128-row tile (cp.async, 16-byte
-//               chunks into the 128-byte-swizzled K-major layout), 3 slots;
 //   warps 4-7   softmax + epilogue of even tiles (TMEM slot 0),
 //   warps 8-11  the same for odd tiles (slot 1): S -> P (bf16, written back
 //               into the S columns, the A operand of the PV MMA), then O / l
 //               -> f16 partial and the log-sum-exp of each row.
+// A query occupies RQ = max(Hg, 8) tile rows (its Hg heads; with Hg = 4 the
+// box also brings 4 rows of the next heads, which are ignored).
 
 constexpr int kAttnThreads = 384;
 constexpr int kItemRing = 4;
 constexpr int kQSlots = 3;
-constexpr int kItemEmptyCount = 11;   // gather warps 2 + MMA 1 + softmax warps 8
+constexpr int kItemEmptyCount = 9;    // MMA 1 + softmax warps 8
 
 struct __align__(16) RingItem {
-  int32_t seq, blk, g, start, count, pad0, pad1, pad2;
+  int32_t seq, blk, g, start, count, Tb, Sb, qrow0;
+  uint32_t ent[kMaxItemQueries];
 };
 
 struct __align__(16) AttnCtl {
@@ -201,13 +261,6 @@ struct __align__(16) AttnCtl {
   RingItem ring[kItemRing];
 };
 
-// Byte offset of 16-byte chunk `col` (along the 2*D-byte row) of row `row` in a
-// K-major [128 x D] bf16 tile stored as D/64 column halves of [128 x 128 B]
-// with the 128-byte swizzle.
-__device__ __forceinline__ uint32_t kmajor_off(int row, int col) {
-  return (col >> 3) * (128 * 128) + swz_offset(row, col & 7, 128);
-}
-
 struct TileRef {
   int tau;        // tile counter of this CTA
   int item_seq;   // item counter of this CTA
@@ -216,7 +269,7 @@ struct TileRef {
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                   const __nv_bfloat16* __restrict__ q, const Item* __restrict__ items,
+                   const __grid_constant__ CUtensorMap tm_q, const Item* __restrict__ items,
                    const int32_t* __restrict__ nitems_p, int32_t* __restrict__ ticket,
                    const uint32_t* __restrict__ entries, const int32_t* __restrict__ cu_q,
                    const int32_t* __restrict__ cu_k, int H, int G, int d, int k, float scale_log2,
@@ -232,7 +285,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Hg = H / G;
-  const int qpt = 128 / Hg;                    // queries per 128-row tile
+  const int RQ = Hg < 8 ? 8 : Hg;              // tile rows per query
+  const int qpt = 128 / RQ;                    // queries per 128-row tile
   const int nhalf = d / 64;
   const int nitems = *nitems_p;
 
@@ -243,12 +297,13 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       mbar_init(&ctl->s_full[i], 1); mbar_init(&ctl->p_full[i], 4);
       mbar_init(&ctl->o_full[i], 1); mbar_init(&ctl->o_free[i], 4);
     }
-    for (int i = 0; i < kQSlots; ++i) { mbar_init(&ctl->q_full[i], 2); mbar_init(&ctl->q_empty[i], 1); }
+    for (int i = 0; i < kQSlots; ++i) { mbar_init(&ctl->q_full[i], 1); mbar_init(&ctl->q_empty[i], 1); }
     mbar_init(&ctl->mma_done, 1);
     ctl->abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_q);
   }
   if (warp == 1) {
     tmem_alloc(&ctl->tmem_base, 512);
@@ -259,63 +314,102 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
 
-  // Reads the next ring item (every consumer warp calls this in the same order).
+  // Waits for ring item n (consumers call this in the same order).
   // whole_warp: all 32 lanes call it (else only lane 0 of the warp does).
-  auto take_item = [&](int n, RingItem& out, bool whole_warp) -> bool {
+  auto wait_item = [&](int n) -> const RingItem* {
     const int slot = n % kItemRing;
     if (!mbar_wait(&ctl->item_full[slot], (n / kItemRing) & 1)) {
       report_error(err, MSA_ERR_TIMEOUT, kSiteAttnItem, n, warp);
       *abort_flag = 1;
-      return false;
+      return nullptr;
     }
-    out = ctl->ring[slot];
+    return &ctl->ring[slot];
+  };
+  auto release_item = [&](int n, bool whole_warp) {
     if (whole_warp) __syncwarp();
-    if (lane == 0) mbar_arrive(&ctl->item_empty[slot]);
-    return out.count > 0;
+    if (lane == 0) mbar_arrive(&ctl->item_empty[n % kItemRing]);
   };
 
   if (warp == 0) {
-    // ------------------------------------------------ scheduler + K/V loads
-    if (lane == 0) {
-      int n = 0;
-      while (true) {
-        const int slot = n % kItemRing;
-        if (!mbar_wait(&ctl->item_empty[slot], ((n / kItemRing) + 1) & 1)) {
-          report_error(err, MSA_ERR_TIMEOUT, kSiteAttnLoad, n, 0);
-          *abort_flag = 1;
-          break;
-        }
-        const int it = *abort_flag ? nitems : atomicAdd(ticket, 1);
-        RingItem r;
-        if (it >= nitems) {
-          r.count = 0;
-          ctl->ring[slot] = r;
+    // ---------------------------------------- scheduler, K/V and Q loads
+    int n = 0, tau = 0;
+    while (true) {
+      const int slot = n % kItemRing;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&ctl->item_empty[slot], ((n / kItemRing) + 1) & 1);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) {
+        if (lane == 0) report_error(err, MSA_ERR_TIMEOUT, kSiteAttnLoad, n, 0);
+        *abort_flag = 1;
+        break;
+      }
+      int it = 0;
+      if (lane == 0) it = *abort_flag ? nitems : atomicAdd(ticket, 1);
+      it = __shfl_sync(0xffffffffu, it, 0);
+      RingItem* R = &ctl->ring[slot];
+      if (it >= nitems) {
+        if (lane == 0) {
+          R->count = 0;
           mbar_arrive(&ctl->item_full[slot]);
-          break;
         }
-        const Item I = items[it];
-        r.seq = I.seq; r.blk = I.blk; r.g = I.g; r.start = I.start; r.count = I.count;
-        ctl->ring[slot] = r;
+        break;
+      }
+      const Item I = items[it];
+      for (int j = lane; j < I.count; j += 32) R->ent[j] = entries[I.start + j];
+      if (lane == 0) {
+        R->seq = I.seq; R->blk = I.blk; R->g = I.g; R->start = I.start; R->count = I.count;
+        R->Tb = cu_q[I.seq + 1] - cu_q[I.seq];
+        R->Sb = cu_k[I.seq + 1] - cu_k[I.seq];
+        R->qrow0 = cu_q[I.seq];
+      }
+      __syncwarp();
+      if (lane == 0) {
         mbar_arrive(&ctl->item_full[slot]);
+        // K / V block of this item
         const int st = n & 1;
-        if (!mbar_wait(&ctl->kv_empty[st], ((n >> 1) + 1) & 1)) {
+        ok = mbar_wait(&ctl->kv_empty[st], ((n >> 1) + 1) & 1);
+        if (ok) {
+          uint8_t* ks = kv_s + st * 2 * tile_bytes;
+          mbar_arrive_expect_tx(&ctl->kv_full[st], 2 * tile_bytes);
+          const int krow = cu_k[I.seq] + I.blk * kBk;
+          for (int h = 0; h < nhalf; ++h) {
+            tma_load_3d(ks + h * 128 * 128, &tm_k, &ctl->kv_full[st], 64 * h, I.g, krow);
+            tma_load_3d(ks + tile_bytes + h * 128 * 128, &tm_v, &ctl->kv_full[st], 64 * h, I.g, krow);
+          }
+        }
+        // Q rows of each tile
+        const int ntiles = (I.count + qpt - 1) / qpt;
+        for (int mt = 0; ok && mt < ntiles; ++mt, ++tau) {
+          const int qs = tau % kQSlots;
+          if (!(ok = mbar_wait(&ctl->q_empty[qs], ((tau / kQSlots) + 1) & 1))) break;
+          const int nq = min(qpt, I.count - mt * qpt);
+          uint8_t* dst = q_s + qs * tile_bytes;
+          mbar_arrive_expect_tx(&ctl->q_full[qs], nq * RQ * d * 2);
+          for (int ql = 0; ql < nq; ++ql) {
+            const int64_t t = t0 + R->ent[mt * qpt + ql] / k;
+            const int row = (int)(t * H + (int64_t)I.g * Hg);
+            for (int h = 0; h < nhalf; ++h)
+              tma_load_2d(dst + h * 128 * 128 + ql * RQ * 128, &tm_q, &ctl->q_full[qs], 64 * h, row);
+          }
+        }
+        if (!ok) {
           report_error(err, MSA_ERR_TIMEOUT, kSiteAttnLoad, n, 1);
           *abort_flag = 1;
-          break;
         }
-        uint8_t* ks = kv_s + st * 2 * tile_bytes;
-        mbar_arrive_expect_tx(&ctl->kv_full[st], 2 * tile_bytes);
-        const int krow = cu_k[I.seq] + I.blk * kBk;
-        for (int h = 0; h < nhalf; ++h) {
-          tma_load_3d(ks + h * 128 * 128, &tm_k, &ctl->kv_full[st], 64 * h, I.g, krow);
-          tma_load_3d(ks + tile_bytes + h * 128 * 128, &tm_v, &ctl->kv_full[st], 64 * h, I.g, krow);
-        }
-        ++n;
       }
-      // no K/V load may still be in flight when the CTA exits
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      ++n;
+    }
+    if (lane == 0) {
+      // no TMA load may still be in flight when the CTA exits
       for (int st = 0; st < 2; ++st) {
         const int issued = n > st ? (n - st + 1) / 2 : 0;
         if (issued > 0) mbar_wait(&ctl->kv_full[st], (issued - 1) & 1);
+      }
+      for (int qs = 0; qs < kQSlots; ++qs) {
+        const int issued = tau > qs ? (tau - qs + kQSlots - 1) / kQSlots : 0;
+        if (issued > 0) mbar_wait(&ctl->q_full[qs], (issued - 1) & 1);
       }
     }
   } else if (warp == 1) {
@@ -324,15 +418,19 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       const uint32_t idesc_o = idesc_bf16_f32(128, d, 0, 1);
       int n = 0, tau = 0;
-      RingItem cur;
       int cur_tiles = 0, mt = 0, cur_seq = -1;
-      bool have = false, ok = true;
-      // next tile in the stream (consumes items as needed)
+      bool have = false, ok = true, done = false;
+      // next tile in the stream (consumes ring items as needed)
       auto next_tile = [&](TileRef& tr) -> bool {
+        if (done) return false;
         if (!have || mt >= cur_tiles) {
-          if (!take_item(n, cur, false)) return false;
+          const RingItem* R = wait_item(n);
+          if (R == nullptr) { done = true; return false; }
+          const int cnt = R->count;
+          release_item(n, false);
+          if (cnt <= 0) { done = true; return false; }
           cur_seq = n++;
-          cur_tiles = (cur.count + qpt - 1) / qpt;
+          cur_tiles = (cnt + qpt - 1) / qpt;
           mt = 0;
           have = true;
         }
@@ -389,38 +487,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       umma_commit(&ctl->mma_done);
       mbar_wait(&ctl->mma_done, 0);
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ Q gather
-    const int gt = tid - 64;                   // 0..63
-    const int cpr = d / 8;                     // 16-byte chunks per row
-    int n = 0, tau = 0;
-    RingItem I;
-    while (!*abort_flag && take_item(n++, I, true)) {
-      const int ntiles = (I.count + qpt - 1) / qpt;
-      for (int mt = 0; mt < ntiles; ++mt, ++tau) {
-        const int qs = tau % kQSlots;
-        if (!mbar_wait(&ctl->q_empty[qs], ((tau / kQSlots) + 1) & 1)) {
-          report_error(err, MSA_ERR_TIMEOUT, kSiteAttnLoad, tau, 2);
-          *abort_flag = 1;
-          break;
-        }
-        const int nq = min(qpt, I.count - mt * qpt);
-        uint8_t* dst = q_s + qs * tile_bytes;
-        const uint32_t* ent = entries + I.start + mt * qpt;
-        for (int c = gt; c < nq * Hg * cpr; c += 64) {
-          const int row = c / cpr, col = c - row * cpr;
-          const int ql = row / Hg, i = row - ql * Hg;
-          const int64_t t = t0 + ent[ql] / k;
-          cp_async_16(dst + kmajor_off(row, col), q + ((t * H) + (int64_t)I.g * Hg + i) * d + col * 8);
-        }
-        cp_async_commit();
-        cp_async_wait_all();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->q_full[qs]);
-      }
-    }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------- softmax + epilogue
     const int wg = (warp - 4) >> 2;           // slot handled by this warpgroup
     const int wq = warp & 3;                  // TMEM lane quarter
@@ -428,23 +495,25 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const uint32_t lane_off = static_cast<uint32_t>(32 * wq) << 16;
     const uint32_t s_col = tmem + wg * 256 + lane_off;      // S, then P (first 64 columns)
     const uint32_t o_col = s_col + 128;                     // O
-    const int ql = r / Hg, hi = r - ql * Hg;
+    const int ql = r / RQ, hi = r - ql * RQ;
     int n = 0, tau = 0;
-    RingItem I;
-    while (!*abort_flag && take_item(n++, I, true)) {
-      const int ntiles = (I.count + qpt - 1) / qpt;
-      const int Tb = cu_q[I.seq + 1] - cu_q[I.seq];
-      const int Sb = cu_k[I.seq + 1] - cu_k[I.seq];
-      const int64_t qrow0 = cu_q[I.seq];
-      const int64_t blk_first = (int64_t)I.blk * kBk;
+    while (!*abort_flag) {
+      const RingItem* R = wait_item(n);
+      if (R == nullptr) break;
+      const int count = R->count;
+      if (count <= 0) { release_item(n, true); break; }
+      const int g = R->g, Tb = R->Tb, Sb = R->Sb;
+      const int64_t qrow0 = R->qrow0;
+      const int64_t blk_first = (int64_t)R->blk * kBk;
+      const int ntiles = (count + qpt - 1) / qpt;
+      // the item stays in the ring until this warpgroup's last tile of it
       for (int mt = 0; mt < ntiles; ++mt, ++tau) {
         if ((tau & 1) != wg) continue;
-        const int nq = min(qpt, I.count - mt * qpt);
-        const bool valid = ql < nq;
-        uint32_t e = 0;
+        const int idx = mt * qpt + ql;
+        const bool valid = ql < qpt && idx < count && hi < Hg;
+        const uint32_t e = valid ? R->ent[idx] : 0u;
         int limit = 127;
         if (valid) {
-          e = entries[I.start + mt * qpt + ql];
           const int64_t t = t0 + e / k;
           const int64_t lim = (int64_t)Sb - Tb + (t - qrow0) - blk_first;
           limit = lim >= 127 ? 127 : (int)lim;
@@ -494,8 +563,9 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         }
         tc_fence_after();
         const float inv_l = 1.f / l;
-        const int64_t unit = valid ? ((int64_t)(e / k) * G + I.g) * k + (e % k) : 0;
+        const int64_t unit = valid ? ((int64_t)(e / k) * G + g) * k + (e % k) : 0;
         __half* dst = part_acc + (unit * Hg + hi) * d;
+#pragma unroll 1
         for (int c4 = 0; c4 < d / 32; ++c4) {
           tmem_ld32(o_col + 32 * c4, rr);
           tmem_ld_wait();
@@ -516,6 +586,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->o_free[wg]);
       }
+      release_item(n, true);
+      ++n;
     }
   }
 
@@ -531,10 +603,14 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 // -------------------------------------------------------------- combine ---
 
 // One group of d/8 threads per (query, head); each thread owns 8 output
-// columns.  Slots with sel < 0 carry no partial.
-__global__ void combine_kernel(const __half* __restrict__ part_acc, const float* __restrict__ part_lse,
-                               const int32_t* __restrict__ sel, __nv_bfloat16* __restrict__ out,
-                               float* __restrict__ lse_out, int64_t T, int H, int G, int d, int k) {
+// columns.  Slots with sel < 0 carry no partial.  All partial loads of a
+// thread are issued before any is used (up to KMAX x 16 bytes in flight).
+template <int KMAX>
+__global__ void __launch_bounds__(256) combine_kernel(const __half* __restrict__ part_acc,
+                                                      const float* __restrict__ part_lse,
+                                                      const int32_t* __restrict__ sel, __nv_bfloat16* __restrict__ out,
+                                                      float* __restrict__ lse_out, int64_t T, int H, int G, int d,
+                                                      int k) {
   const int tpr = d / 8;                       // threads per (query, head)
   const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t pair = gid / tpr;
@@ -545,22 +621,33 @@ __global__ void combine_kernel(const __half* __restrict__ part_acc, const float*
   const int Hg = H / G, g = h / Hg, i = h % Hg;
   const int32_t* srow = sel + (t * G + g) * k;
   const int64_t ubase = (t * G + g) * k;
+  bool use[KMAX];
+  float ls[KMAX];
+  uint4 raw[KMAX];
   float m = -INFINITY;
-  for (int s = 0; s < k; ++s)
-    if (srow[s] >= 0) m = fmaxf(m, part_lse[(ubase + s) * Hg + i]);
+#pragma unroll
+  for (int s = 0; s < KMAX; ++s) {
+    use[s] = s < k && __ldg(srow + s) >= 0;
+    ls[s] = use[s] ? __ldg(part_lse + (ubase + s) * Hg + i) : -INFINITY;
+  }
+#pragma unroll
+  for (int s = 0; s < KMAX; ++s)
+    raw[s] = use[s] ? __ldg(reinterpret_cast<const uint4*>(part_acc + ((ubase + s) * Hg + i) * d + 8 * c))
+                    : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+  for (int s = 0; s < KMAX; ++s) m = fmaxf(m, ls[s]);
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   float wsum = 0.f;
-  for (int s = 0; s < k; ++s) {
-    if (srow[s] < 0) continue;
-    const float w = __expf(part_lse[(ubase + s) * Hg + i] - m);
+#pragma unroll
+  for (int s = 0; s < KMAX; ++s) {
+    const float w = use[s] ? __expf(ls[s] - m) : 0.f;
     wsum += w;
-    const uint4 raw = *reinterpret_cast<const uint4*>(part_acc + ((ubase + s) * Hg + i) * d + 8 * c);
-    const __half2* hp = reinterpret_cast<const __half2*>(&raw);
+    const __half2* hp = reinterpret_cast<const __half2*>(&raw[s]);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const float2 f = __half22float2(hp[j]);
-      acc[2 * j] += w * f.x;
-      acc[2 * j + 1] += w * f.y;
+      acc[2 * j] = fmaf(w, f.x, acc[2 * j]);
+      acc[2 * j + 1] = fmaf(w, f.y, acc[2 * j + 1]);
     }
   }
   const float inv = 1.f / wsum;
@@ -571,6 +658,16 @@ __global__ void combine_kernel(const __half* __restrict__ part_acc, const float*
   o.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
   *reinterpret_cast<uint4*>(out + (t * H + h) * d + 8 * c) = o;
   if (lse_out != nullptr && c == 0) lse_out[t * H + h] = m + __logf(wsum);
+}
+
+int launch_combine_kernel(const __half* part_acc, const float* part_lse, const int32_t* sel, __nv_bfloat16* out,
+                          float* lse, int64_t T, int H, int G, int d, int k, cudaStream_t st) {
+  const int64_t cthreads = T * H * (d / 8);
+  const unsigned blocks = (unsigned)((cthreads + 255) / 256);
+  if (k <= 8) combine_kernel<8><<<blocks, 256, 0, st>>>(part_acc, part_lse, sel, out, lse, T, H, G, d, k);
+  else if (k <= 16) combine_kernel<16><<<blocks, 256, 0, st>>>(part_acc, part_lse, sel, out, lse, T, H, G, d, k);
+  else combine_kernel<32><<<blocks, 256, 0, st>>>(part_acc, part_lse, sel, out, lse, T, H, G, d, k);
+  return (int)cudaGetLastError();
 }
 
 }  // namespace
@@ -586,38 +683,52 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
     ProfScope p("block_offsets", stream);
     block_offsets_kernel<<<1, 32, 0, st>>>(a.cu_k, a.batch, a.blk_off);
   }
-  e = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * a.nlists, st);
-  if (e != cudaSuccess) return (int)e;
-  e = cudaMemsetAsync(a.nitems, 0, sizeof(int32_t) * 2, st);   // nitems and the item ticket
+  const int64_t nwin = (nrows + kWindow - 1) / kWindow;
+  const int64_t nkeys = nwin * a.nlists;
+  e = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * nkeys, st);
   if (e != cudaSuccess) return (int)e;
   const int64_t nthreads = nrows * a.G;
   const int cs_blocks = (int)((nthreads + 255) / 256);
   {
     ProfScope p("count", stream);
     count_scatter_kernel<false><<<cs_blocks, 256, 0, st>>>(a.sel, a.t0, a.t1, a.G, a.k, a.batch, a.cu_q, a.cu_k,
-                                                           a.blk_off, a.counts, nullptr, a.err);
+                                                           a.blk_off, a.nlists, a.counts, nullptr, a.err);
   }
+  const int ntiles = (int)((nkeys + kScanTile - 1) / kScanTile);
   {
     ProfScope p("plan", stream);
-    plan_kernel<<<1, 1024, 0, st>>>(a.counts, a.nlists, a.G, a.batch, a.blk_off, a.queries_per_item, a.offsets,
-                                    a.cursor, a.item_off, a.nitems, a.items, a.max_items, a.err);
+    scan_reduce_kernel<<<ntiles, kScanThreads, 0, st>>>(a.counts, nkeys, a.queries_per_item, a.tile_sums);
+    scan_tiles_kernel<<<1, kScanThreads, 0, st>>>(a.tile_sums, ntiles, a.nitems, a.max_items, a.err);
+    scan_items_kernel<<<ntiles, kScanThreads, 0, st>>>(a.counts, nkeys, a.nlists, a.G, a.batch, a.queries_per_item,
+                                                       a.tile_sums, a.blk_off, a.cursor, a.items, a.max_items);
+    prof_count_launch(2);
   }
   {
     ProfScope p("scatter", stream);
     count_scatter_kernel<true><<<cs_blocks, 256, 0, st>>>(a.sel, a.t0, a.t1, a.G, a.k, a.batch, a.cu_q, a.cu_k,
-                                                          a.blk_off, a.cursor, a.entries, a.err);
+                                                          a.blk_off, a.nlists, a.cursor, a.entries, a.err);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
 
-  alignas(64) CUtensorMap tm_k, tm_v;
-  const uint64_t dims[3] = {(uint64_t)a.d, (uint64_t)a.G, (uint64_t)a.total_k};
-  const uint64_t strides[2] = {(uint64_t)a.d * 2, (uint64_t)a.G * a.d * 2};
-  const uint32_t box[3] = {64u, 1u, 128u};
-  int rc = make_tmap_bf16(&tm_k, a.key, 3, dims, strides, box, 128);
-  if (rc) return rc;
-  rc = make_tmap_bf16(&tm_v, a.value, 3, dims, strides, box, 128);
-  if (rc) return rc;
+  alignas(64) CUtensorMap tm_k, tm_v, tm_q;
+  {
+    const uint64_t dims[3] = {(uint64_t)a.d, (uint64_t)a.G, (uint64_t)a.total_k};
+    const uint64_t strides[2] = {(uint64_t)a.d * 2, (uint64_t)a.G * a.d * 2};
+    const uint32_t box[3] = {64u, 1u, 128u};
+    int rc = make_tmap_bf16(&tm_k, a.key, 3, dims, strides, box, 128);
+    if (rc) return rc;
+    rc = make_tmap_bf16(&tm_v, a.value, 3, dims, strides, box, 128);
+    if (rc) return rc;
+  }
+  {
+    const int hg = a.H / a.G;
+    const uint64_t dims[2] = {(uint64_t)a.d, (uint64_t)a.total_q * a.H};
+    const uint64_t strides[1] = {(uint64_t)a.d * 2};
+    const uint32_t box[2] = {64u, (uint32_t)(hg < 8 ? 8 : hg)};
+    int rc = make_tmap_bf16(&tm_q, a.q, 2, dims, strides, box, 128);
+    if (rc) return rc;
+  }
   const size_t smem = 1024 + (4 + kQSlots) * (size_t)128 * a.d * 2 + sizeof(AttnCtl);
   e = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return (int)e;
@@ -628,32 +739,25 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
   {
     ProfScope p("sparse_attn", stream);
     sparse_attn_kernel<<<nsm, kAttnThreads, smem, st>>>(
-        tm_k, tm_v, reinterpret_cast<const __nv_bfloat16*>(a.q), a.items, a.nitems, a.nitems + 1, a.entries,
-        a.cu_q, a.cu_k, a.H, a.G, a.d, a.k, scale_log2, a.t0, reinterpret_cast<__half*>(a.part_acc), a.part_lse,
-        a.err);
+        tm_k, tm_v, tm_q, a.items, a.nitems, a.nitems + 1, a.entries, a.cu_q, a.cu_k, a.H, a.G, a.d, a.k,
+        scale_log2, a.t0, reinterpret_cast<__half*>(a.part_acc), a.part_lse, a.err);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
   const int64_t rows = a.t1 - a.t0;
-  const int64_t cthreads = rows * a.H * (a.d / 8);
   ProfScope p("combine", stream);
-  combine_kernel<<<(int)((cthreads + 255) / 256), 256, 0, st>>>(
-      reinterpret_cast<const __half*>(a.part_acc), a.part_lse, a.sel + a.t0 * a.G * a.k,
-      reinterpret_cast<__nv_bfloat16*>(a.out) + a.t0 * a.H * a.d, a.lse ? a.lse + a.t0 * a.H : nullptr, rows, a.H,
-      a.G, a.d, a.k);
-  return (int)cudaGetLastError();
+  return launch_combine_kernel(reinterpret_cast<const __half*>(a.part_acc), a.part_lse, a.sel + a.t0 * a.G * a.k,
+                               reinterpret_cast<__nv_bfloat16*>(a.out) + a.t0 * a.H * a.d,
+                               a.lse ? a.lse + a.t0 * a.H : nullptr, rows, a.H, a.G, a.d, a.k, st);
 }
 
 int launch_combine(const void* part_acc, const float* part_lse, const int32_t* sel, void* out, float* lse,
                    int64_t T, int32_t H, int32_t G, int32_t d, int32_t k, void* stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (T <= 0) return 0;
-  const int64_t cthreads = T * H * (d / 8);
   ProfScope p("combine", stream);
-  combine_kernel<<<(int)((cthreads + 255) / 256), 256, 0, st>>>(
-      reinterpret_cast<const __half*>(part_acc), part_lse, sel, reinterpret_cast<__nv_bfloat16*>(out), lse, T, H, G,
-      d, k);
-  return (int)cudaGetLastError();
+  return launch_combine_kernel(reinterpret_cast<const __half*>(part_acc), part_lse, sel,
+                               reinterpret_cast<__nv_bfloat16*>(out), lse, T, H, G, d, k, st);
 }
 
 }  // namespace msa

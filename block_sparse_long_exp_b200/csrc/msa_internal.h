@@ -11,6 +11,9 @@ namespace msa {
 constexpr int kBk = 128;          // block size the kernels are built for
 constexpr int kMaxK = 32;         // largest k
 constexpr int kMaxBatchTiles = 1024;  // sequences per prefill index launch
+constexpr int kWindow = 1024;         // query rows per attention planning window
+constexpr int kScanTile = 4096;       // keys per CTA of the planning scan
+constexpr int kMaxItemQueries = 128;  // queries per attention work item (upper bound)
 
 // Device error word, at offset 0 of every workspace.
 struct DevError {
@@ -87,11 +90,10 @@ struct AttnArgs {
   int64_t t0, t1;      // query rows of this pass
   DevError* err;
   // workspace slices
-  int32_t* counts;     // [nlists]
-  int32_t* offsets;    // [nlists + 1]
-  int32_t* cursor;     // [nlists]
-  int32_t* item_off;   // [nlists + 1]
-  int32_t* nitems;     // [1]
+  int32_t* counts;     // [nwin * nlists]  entries per (window, list)
+  int32_t* cursor;     // [nwin * nlists]  list offsets, then scatter cursors
+  int32_t* tile_sums;  // [2 * ceil(nwin * nlists / kScanTile)]
+  int32_t* nitems;     // [4]: items, item ticket, entries
   uint32_t* entries;   // [(t1 - t0) * G * k]
   Item* items;         // [max_items]
   int64_t max_items;
