@@ -730,6 +730,7 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
     if (rc) return rc;
   }
   const size_t smem = 1024 + (4 + kQSlots) * (size_t)128 * a.d * 2 + sizeof(AttnCtl);
+  static_assert(1024 + 7 * 128 * 128 * 2 + sizeof(AttnCtl) <= 227 * 1024, "shared memory budget (d = 128)");
   e = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return (int)e;
   int dev = 0, nsm = 0;

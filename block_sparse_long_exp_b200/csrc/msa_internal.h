@@ -13,7 +13,7 @@ constexpr int kMaxK = 32;         // largest k
 constexpr int kMaxBatchTiles = 1024;  // sequences per prefill index launch
 constexpr int kWindow = 1024;         // query rows per attention planning window
 constexpr int kScanTile = 4096;       // keys per CTA of the planning scan
-constexpr int kMaxItemQueries = 128;  // queries per attention work item (upper bound)
+constexpr int kMaxItemQueries = 64;   // queries per attention work item (upper bound)
 
 // Device error word, at offset 0 of every workspace.
 struct DevError {
