@@ -525,31 +525,56 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         }
         tc_fence_after();
         uint32_t rr[32];
-        float m = -INFINITY;
+        float m = -INFINITY, l = 0.f, ms;
+        if (__all_sync(0xffffffffu, limit >= 127)) {
+          // no causal cut in this warp's rows (not the local block)
 #pragma unroll 1
-        for (int c4 = 0; c4 < 4; ++c4) {
-          tmem_ld32(s_col + 32 * c4, rr);
-          tmem_ld_wait();
+          for (int c4 = 0; c4 < 4; ++c4) {
+            tmem_ld32(s_col + 32 * c4, rr);
+            tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (32 * c4 + j <= limit) m = fmaxf(m, __uint_as_float(rr[j]));
-        }
-        const float ms = m * scale_log2;
-        float l = 0.f;
-#pragma unroll 1
-        for (int c4 = 0; c4 < 4; ++c4) {
-          tmem_ld32(s_col + 32 * c4, rr);
-          tmem_ld_wait();
-          uint32_t pk[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int c0 = 32 * c4 + 2 * j;
-            const float p0 = c0 <= limit ? exp2f(fmaf(__uint_as_float(rr[2 * j]), scale_log2, -ms)) : 0.f;
-            const float p1 = c0 + 1 <= limit ? exp2f(fmaf(__uint_as_float(rr[2 * j + 1]), scale_log2, -ms)) : 0.f;
-            l += p0 + p1;
-            pk[j] = pack_bf16x2(p0, p1);
+            for (int j = 0; j < 32; j += 2) m = fmax3(m, __uint_as_float(rr[j]), __uint_as_float(rr[j + 1]));
           }
-          tmem_st16(s_col + 16 * c4, pk);
+          ms = m * scale_log2;
+#pragma unroll 1
+          for (int c4 = 0; c4 < 4; ++c4) {
+            tmem_ld32(s_col + 32 * c4, rr);
+            tmem_ld_wait();
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float p0 = exp2f(fmaf(__uint_as_float(rr[2 * j]), scale_log2, -ms));
+              const float p1 = exp2f(fmaf(__uint_as_float(rr[2 * j + 1]), scale_log2, -ms));
+              l += p0 + p1;
+              pk[j] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(s_col + 16 * c4, pk);
+          }
+        } else {
+#pragma unroll 1
+          for (int c4 = 0; c4 < 4; ++c4) {
+            tmem_ld32(s_col + 32 * c4, rr);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (32 * c4 + j <= limit) m = fmaxf(m, __uint_as_float(rr[j]));
+          }
+          ms = m * scale_log2;
+#pragma unroll 1
+          for (int c4 = 0; c4 < 4; ++c4) {
+            tmem_ld32(s_col + 32 * c4, rr);
+            tmem_ld_wait();
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int c0 = 32 * c4 + 2 * j;
+              const float p0 = c0 <= limit ? exp2f(fmaf(__uint_as_float(rr[2 * j]), scale_log2, -ms)) : 0.f;
+              const float p1 = c0 + 1 <= limit ? exp2f(fmaf(__uint_as_float(rr[2 * j + 1]), scale_log2, -ms)) : 0.f;
+              l += p0 + p1;
+              pk[j] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(s_col + 16 * c4, pk);
+          }
         }
         tmem_st_wait();
         tc_fence_before();
@@ -564,7 +589,9 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         tc_fence_after();
         const float inv_l = 1.f / l;
         const int64_t unit = valid ? ((int64_t)(e / k) * G + g) * k + (e % k) : 0;
-        __half* dst = part_acc + (unit * Hg + hi) * d;
+        // partial layout per unit: [d/8 chunks][Hg heads][8 values], so the
+        // 16 heads of one query write 256 contiguous bytes per chunk
+        __half* dst = part_acc + unit * Hg * d + hi * 8;
 #pragma unroll 1
         for (int c4 = 0; c4 < d / 32; ++c4) {
           tmem_ld32(o_col + 32 * c4, rr);
@@ -577,7 +604,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
               w.y = pack_f16x2(__uint_as_float(rr[8 * j + 2]) * inv_l, __uint_as_float(rr[8 * j + 3]) * inv_l);
               w.z = pack_f16x2(__uint_as_float(rr[8 * j + 4]) * inv_l, __uint_as_float(rr[8 * j + 5]) * inv_l);
               w.w = pack_f16x2(__uint_as_float(rr[8 * j + 6]) * inv_l, __uint_as_float(rr[8 * j + 7]) * inv_l);
-              *reinterpret_cast<uint4*>(dst + 32 * c4 + 8 * j) = w;
+              *reinterpret_cast<uint4*>(dst + (4 * c4 + j) * Hg * 8) = w;
             }
           }
         }
@@ -602,45 +629,50 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 
 // -------------------------------------------------------------- combine ---
 
-// One group of d/8 threads per (query, head); each thread owns 8 output
-// columns.  Slots with sel < 0 carry no partial.  All partial loads of a
-// thread are issued before any is used (up to KMAX x 16 bytes in flight).
+// One thread per (query, group, 8-column chunk c, head i) with i fastest, so a
+// warp's loads of one partial are contiguous (layout per unit: [d/8][Hg][8]).
+// Every load of a thread (selection, log-sum-exps, partials) is issued before
+// any is used; empty slots (sel < 0) are masked afterwards.
 template <int KMAX>
 __global__ void __launch_bounds__(256) combine_kernel(const __half* __restrict__ part_acc,
                                                       const float* __restrict__ part_lse,
                                                       const int32_t* __restrict__ sel, __nv_bfloat16* __restrict__ out,
                                                       float* __restrict__ lse_out, int64_t T, int H, int G, int d,
                                                       int k) {
-  const int tpr = d / 8;                       // threads per (query, head)
+  const int Hg = H / G;
+  const int per = Hg * (d / 8);                // threads per (query, group)
   const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t pair = gid / tpr;
-  const int c = (int)(gid % tpr);
-  if (pair >= T * H) return;
-  const int64_t t = pair / H;
-  const int h = (int)(pair % H);
-  const int Hg = H / G, g = h / Hg, i = h % Hg;
-  const int32_t* srow = sel + (t * G + g) * k;
-  const int64_t ubase = (t * G + g) * k;
-  bool use[KMAX];
+  const int64_t tg = gid / per;
+  if (tg >= T * G) return;
+  const int rem = (int)(gid - tg * per);
+  const int c = rem / Hg, i = rem - c * Hg;
+  const int64_t t = tg / G;
+  const int g = (int)(tg - t * G);
+  const int32_t* srow = sel + tg * k;
+  const int64_t ubase = tg * k;
+  int sv[KMAX];
   float ls[KMAX];
   uint4 raw[KMAX];
-  float m = -INFINITY;
 #pragma unroll
   for (int s = 0; s < KMAX; ++s) {
-    use[s] = s < k && __ldg(srow + s) >= 0;
-    ls[s] = use[s] ? __ldg(part_lse + (ubase + s) * Hg + i) : -INFINITY;
+    if (s < k) {
+      sv[s] = __ldg(srow + s);
+      ls[s] = __ldg(part_lse + (ubase + s) * Hg + i);
+      raw[s] = __ldg(reinterpret_cast<const uint4*>(part_acc + ((ubase + s) * (d / 8) + c) * Hg * 8 + i * 8));
+    } else {
+      sv[s] = -1;
+    }
   }
+  float m = -INFINITY;
 #pragma unroll
   for (int s = 0; s < KMAX; ++s)
-    raw[s] = use[s] ? __ldg(reinterpret_cast<const uint4*>(part_acc + ((ubase + s) * Hg + i) * d + 8 * c))
-                    : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-  for (int s = 0; s < KMAX; ++s) m = fmaxf(m, ls[s]);
+    if (sv[s] >= 0) m = fmaxf(m, ls[s]);
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   float wsum = 0.f;
 #pragma unroll
   for (int s = 0; s < KMAX; ++s) {
-    const float w = use[s] ? __expf(ls[s] - m) : 0.f;
+    if (sv[s] < 0) continue;
+    const float w = __expf(ls[s] - m);
     wsum += w;
     const __half2* hp = reinterpret_cast<const __half2*>(&raw[s]);
 #pragma unroll
@@ -656,13 +688,14 @@ __global__ void __launch_bounds__(256) combine_kernel(const __half* __restrict__
   o.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
   o.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
   o.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+  const int h = g * Hg + i;
   *reinterpret_cast<uint4*>(out + (t * H + h) * d + 8 * c) = o;
   if (lse_out != nullptr && c == 0) lse_out[t * H + h] = m + __logf(wsum);
 }
 
 int launch_combine_kernel(const __half* part_acc, const float* part_lse, const int32_t* sel, __nv_bfloat16* out,
                           float* lse, int64_t T, int H, int G, int d, int k, cudaStream_t st) {
-  const int64_t cthreads = T * H * (d / 8);
+  const int64_t cthreads = T * H * (d / 8);   // = T * G * Hg * d/8
   const unsigned blocks = (unsigned)((cthreads + 255) / 256);
   if (k <= 8) combine_kernel<8><<<blocks, 256, 0, st>>>(part_acc, part_lse, sel, out, lse, T, H, G, d, k);
   else if (k <= 16) combine_kernel<16><<<blocks, 256, 0, st>>>(part_acc, part_lse, sel, out, lse, T, H, G, d, k);

@@ -12,19 +12,21 @@
 // of that (query, group).  Blocks arrive in ascending order, so a new block only
 // displaces a strictly lower score: ties stay with the lower block index.
 //
-// Warp roles (320 threads): warps 0-3 and 4-7 are two epilogue sets (set e
-// drains the accumulators of groups g with g % E == e), warp 8 issues TMA loads,
-// warp 9 owns TMEM and issues the MMAs.
+// Warp roles (576 threads): warps 4g .. 4g+3 form the epilogue set of group g
+// (G <= 4 sets; accumulator g belongs to group g), warp 16 issues TMA loads,
+// warp 17 owns TMEM and issues the MMAs.  While set g drains key block j, the
+// tensor core computes block j for the other groups, so each set has about G
+// MMA-times to read its 128 columns, pool them and update its lists.
 #include "msa_common.cuh"
 
 namespace msa {
 namespace {
 
 constexpr int kStages = 4;        // max index-key block stages in shared memory
-constexpr int kAcc = 4;           // 128-column TMEM accumulators (512 columns)
-constexpr int kThreads = 320;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kAcc = 4;           // 128-column TMEM accumulators (512 columns), one per group
+constexpr int kThreads = 576;
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
 constexpr int kTile = 128;        // queries per tile = key-block size
 
 struct __align__(16) IndexCtl {
@@ -159,7 +161,6 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                           const int32_t* __restrict__ cu_k, int batch, int d_idx, int k, int nst,
                           DevError* err) {
   constexpr int CAP = KMAX - 1;
-  constexpr int E = G >= 2 ? 2 : 1;   // epilogue sets in use
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -257,7 +258,7 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
       const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
       const uint32_t mode = sw_mode_for(span);
       const uint32_t sbo = 8 * span;
-      uint32_t kstep = 0, astep = 0, qiter = 0;
+      uint32_t kstep = 0, jstep = 0, qiter = 0;   // jstep: key blocks issued (all tiles)
       bool ok = true;
       for (int it = 0; ok; ++it) {
         const int tau = snake_tile(it, ntiles);
@@ -270,7 +271,7 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         }
         ++qiter;
         tc_fence_after();
-        for (int j = 0; j < ti.n_kb && ok; ++j) {
+        for (int j = 0; j < ti.n_kb && ok; ++j, ++jstep) {
           const int st = kstep % nst;
           if (!mbar_wait(&ctl->k_full[st], (kstep / nst) & 1)) {
             report_error(err, MSA_ERR_TIMEOUT, kSiteIndexMma, tau, j);
@@ -280,8 +281,7 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
           tc_fence_after();
           const uint32_t kaddr = smem_u32(k_s + st * tile_bytes);
           for (int g = 0; g < G; ++g) {
-            const int a = astep % kAcc;
-            if (!mbar_wait(&ctl->acc_empty[a], ((astep / kAcc) + 1) & 1)) {
+            if (!mbar_wait(&ctl->acc_empty[g], (jstep + 1) & 1)) {
               report_error(err, MSA_ERR_TIMEOUT, kSiteIndexMma, tau, 1000 + j);
               ok = false;
               break;
@@ -290,11 +290,10 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             const uint32_t qaddr = smem_u32(q_s + g * tile_bytes);
             for (int kk = 0; kk < d_idx / 16; ++kk) {
               const uint32_t off = (32 * kk / span) * (kTile * span) + (32 * kk) % span;
-              umma_bf16_ss(tmem_base + a * 128, make_sdesc(qaddr + off, 16, sbo, mode),
+              umma_bf16_ss(tmem_base + g * 128, make_sdesc(qaddr + off, 16, sbo, mode),
                            make_sdesc(kaddr + off, 16, sbo, mode), idesc, kk > 0 ? 1u : 0u);
             }
-            umma_commit(&ctl->acc_full[a]);
-            ++astep;
+            umma_commit(&ctl->acc_full[g]);
           }
           umma_commit(&ctl->k_empty[st]);
           ++kstep;
@@ -307,60 +306,46 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
       umma_commit(&ctl->mma_done);
       mbar_wait(&ctl->mma_done, 0);
     }
-  } else if (warp < 4 * E) {
+  } else if (warp < 4 * G) {
     // ------------------------------------------------------------ epilogue
-    const int e = warp / 4;            // epilogue set
+    const int g = warp / 4;            // group of this set = its accumulator
     const int wq = warp % 4;           // TMEM lane quarter
     const int row = 32 * wq + lane;
-    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * wq) << 16);
-    TopList<CAP> list0, list1;
-    uint32_t astep = 0;
+    const uint32_t ta = tmem_base + (static_cast<uint32_t>(32 * wq) << 16) + g * 128;
+    TopList<CAP> list;
+    uint32_t jstep = 0;
     for (int it = 0;; ++it) {
       const int tau = snake_tile(it, ntiles);
       if (tau < 0 || *abort_flag) break;
       const TileInfo ti = tile_info(tau, ctl, batch, cu_q, cu_k);
       const bool valid = row < ti.rows;
       const int lb = (ti.pos0 + row) / kBk;
-      list0.reset();
-      list1.reset();
+      list.reset();
       bool ok = true;
-      for (int j = 0; j < ti.n_kb && ok; ++j, astep += G) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          if (g % E != e) continue;
-          const uint32_t as = astep + g;
-          const int a = as % kAcc;
-          if (!mbar_wait(&ctl->acc_full[a], (as / kAcc) & 1)) {
-            report_error(err, MSA_ERR_TIMEOUT, kSiteIndexEpilogue, tau, j);
-            *abort_flag = 1;
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          uint32_t r0[16];
-          const uint32_t ta = lane_base + a * 128;
-          float m = -INFINITY;
-#pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            tmem_ld16(ta + 16 * cc, r0);
-            tmem_ld_wait();
-            m = fmax3(m, max_of_16(r0), -INFINITY);
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&ctl->acc_empty[a]);
-          if (m != m) m = -INFINITY;    // a block of NaN scores ranks as -inf
-          if (valid && j < lb) {
-            if (g / E == 0) list0.offer(m, j, k - 1); else list1.offer(m, j, k - 1);
-          }
+      for (int j = 0; j < ti.n_kb; ++j, ++jstep) {
+        if (!mbar_wait(&ctl->acc_full[g], jstep & 1)) {
+          report_error(err, MSA_ERR_TIMEOUT, kSiteIndexEpilogue, tau, j);
+          *abort_flag = 1;
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        uint32_t r0[32];
+        float m = -INFINITY;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          tmem_ld32(ta + 32 * cc, r0);
+          tmem_ld_wait();
+          m = fmaxf(m, max_of_32(r0));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->acc_empty[g]);
+        if (m != m) m = -INFINITY;    // a block of NaN scores ranks as -inf
+        if (valid && j < lb) list.offer(m, j, k - 1);
       }
       if (!ok) break;
-      if (valid) {
-        int32_t* dst0 = sel + (static_cast<int64_t>(ti.q0 + row) * G + e) * k;
-        list0.write(dst0, k, lb);
-        if (G > 2) list1.write(dst0 + E * k, k, lb);
-      }
+      if (valid) list.write(sel + (static_cast<int64_t>(ti.q0 + row) * G + g) * k, k, lb);
     }
   }
 

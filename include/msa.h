@@ -155,11 +155,12 @@ msa_status_t msa_sparse_attn_decode(const msa_shape_t* shape, const msa_varlen_t
 
 /* ---------------------------------------------------------------------- */
 /* Two-phase combine on its own (pnsm.cn sec. 7 "two-phase combine").
- * Merges, for every query t and head h of group g, the partials of the slots
- * s with sel[t, g, s] >= 0:
- *   part_acc  device f16 [T, G, k, H/G, d]  softmax output over one block,
- *                                           normalised by its own sum
- *   part_lse  device f32 [T, G, k, H/G]     that block's log-sum-exp
+ * Merges, for every query t and head h = g*(H/G) + i of group g, the partials
+ * of the slots s with sel[t, g, s] >= 0:
+ *   part_acc  device f16 [T, G, k, d/8, H/G, 8]  softmax output over one block,
+ *             normalised by its own sum: element (t, g, s, column 8c+e) of
+ *             head i is at [t][g][s][c][i][e]
+ *   part_lse  device f32 [T, G, k, H/G]          that block's log-sum-exp
  * into out[t, h, :] = sum_s exp(lse_s - LSE) * acc_s with LSE = log sum_s
  * exp(lse_s), and lse[t, h] = LSE (lse may be NULL). */
 msa_status_t msa_combine(const msa_shape_t* shape, int64_t T,

@@ -209,12 +209,14 @@ def test_combine_entry_point(M):
     Hg = H // G
     gen = torch.Generator().manual_seed(3)
     acc = torch.randn(T, G, k, Hg, d_, generator=gen).half()
+    # device layout: [T, G, k, d/8, Hg, 8]
+    acc_dev = acc.view(T, G, k, Hg, d_ // 8, 8).permute(0, 1, 2, 4, 3, 5).contiguous()
     plse = (torch.randn(T, G, k, Hg, generator=gen) * 3).float()
     sel = torch.randint(0, 50, (T, G, k), generator=gen, dtype=torch.int32)
     sel[::3, :, k - 1] = -1                      # some empty slots
     shape = M.make_shape(H, G, d_, 32, k)
     lse_out = torch.empty(T, H, device="cuda")
-    out, _ = M.msa_combine(shape, T, acc.cuda(), plse.cuda(), sel.cuda(), lse=lse_out)
+    out, _ = M.msa_combine(shape, T, acc_dev.cuda(), plse.cuda(), sel.cuda(), lse=lse_out)
     o = _f32(out)
     for t in range(T):
         for h in range(H):
