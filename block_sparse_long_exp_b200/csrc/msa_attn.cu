@@ -417,6 +417,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       const uint32_t idesc_o = idesc_bf16_f32(128, d, 0, 1);
+      // descriptors built once; per-slot / per-step byte offsets (>> 4) are added
+      const uint64_t qdesc0 = make_sdesc(smem_u32(q_s), 16, 1024, kSw128);
+      const uint64_t kvdesc0 = make_sdesc(smem_u32(kv_s), 16, 1024, kSw128);
+      const uint64_t vdesc0 = make_sdesc(smem_u32(kv_s + tile_bytes), 128 * 128, 1024, kSw128);
       int n = 0, tau = 0;
       int cur_tiles = 0, mt = 0, cur_seq = -1;
       bool have = false, ok = true, done = false;
@@ -446,11 +450,11 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         if (!mbar_wait(&ctl->q_full[qs], (tr.tau / kQSlots) & 1)) return false;
         if (tr.first && !mbar_wait(&ctl->kv_full[st], (tr.item_seq >> 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t qa = smem_u32(q_s + qs * tile_bytes), ka = smem_u32(kv_s + st * 2 * tile_bytes);
+        const uint64_t qd = qdesc0 + (uint64_t)((qs * tile_bytes) >> 4);
+        const uint64_t kd = kvdesc0 + (uint64_t)((st * 2 * tile_bytes) >> 4);
         for (int kk = 0; kk < d / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          umma_bf16_ss(tmem + s * 256, make_sdesc(qa + off, 16, 1024, kSw128), make_sdesc(ka + off, 16, 1024, kSw128),
-                       idesc_s, kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
+          umma_bf16_ss(tmem + s * 256, qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(&ctl->s_full[s]);
         umma_commit(&ctl->q_empty[qs]);
@@ -461,10 +465,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         if (!mbar_wait(&ctl->p_full[s], (tr.tau >> 1) & 1)) return false;
         if (!mbar_wait(&ctl->o_free[s], ((tr.tau >> 1) + 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t va = smem_u32(kv_s + st * 2 * tile_bytes + tile_bytes);
+        const uint64_t vd = vdesc0 + (uint64_t)((st * 2 * tile_bytes) >> 4);
+        const uint32_t pcol = tmem + s * 256, ocol = pcol + 128;
         for (int kk = 0; kk < 8; ++kk)
-          umma_bf16_ts(tmem + s * 256 + 128, tmem + s * 256 + kk * 8,
-                       make_sdesc(va + kk * 2048, 128 * 128, 1024, kSw128), idesc_o, kk > 0 ? 1u : 0u);
+          umma_bf16_ts(ocol, pcol + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : 0u);
         umma_commit(&ctl->o_full[s]);
         if (tr.last) umma_commit(&ctl->kv_empty[st]);
         return true;

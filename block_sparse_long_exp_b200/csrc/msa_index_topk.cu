@@ -258,6 +258,11 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
       const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
       const uint32_t mode = sw_mode_for(span);
       const uint32_t sbo = 8 * span;
+      // descriptors are built once; each K=16 step adds its byte offset (>> 4)
+      // to the start-address field
+      const int nk = d_idx / 16;
+      const int per_sh = span == 128 ? 2 : (span == 64 ? 1 : 0);   // log2(K steps per swizzled row)
+      const uint64_t qdesc0 = make_sdesc(smem_u32(q_s), 16, sbo, mode);
       uint32_t kstep = 0, jstep = 0, qiter = 0;   // jstep: key blocks issued (all tiles)
       bool ok = true;
       for (int it = 0; ok; ++it) {
@@ -279,7 +284,7 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
             break;
           }
           tc_fence_after();
-          const uint32_t kaddr = smem_u32(k_s + st * tile_bytes);
+          const uint64_t bdesc = make_sdesc(smem_u32(k_s + st * tile_bytes), 16, sbo, mode);
           for (int g = 0; g < G; ++g) {
             if (!mbar_wait(&ctl->acc_empty[g], (jstep + 1) & 1)) {
               report_error(err, MSA_ERR_TIMEOUT, kSiteIndexMma, tau, 1000 + j);
@@ -287,11 +292,11 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
               break;
             }
             tc_fence_after();
-            const uint32_t qaddr = smem_u32(q_s + g * tile_bytes);
-            for (int kk = 0; kk < d_idx / 16; ++kk) {
-              const uint32_t off = (32 * kk / span) * (kTile * span) + (32 * kk) % span;
-              umma_bf16_ss(tmem_base + g * 128, make_sdesc(qaddr + off, 16, sbo, mode),
-                           make_sdesc(kaddr + off, 16, sbo, mode), idesc, kk > 0 ? 1u : 0u);
+            const uint64_t adesc = qdesc0 + (uint64_t)((g * tile_bytes) >> 4);
+            for (int kk = 0; kk < nk; ++kk) {
+              const uint64_t off =
+                  (uint64_t)((((kk >> per_sh) * (kTile * span)) + ((kk & ((1 << per_sh) - 1)) * 32)) >> 4);
+              umma_bf16_ss(tmem_base + g * 128, adesc + off, bdesc + off, idesc, kk > 0 ? 1u : 0u);
             }
             umma_commit(&ctl->acc_full[g]);
           }
