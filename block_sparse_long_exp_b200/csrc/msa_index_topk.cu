@@ -4,35 +4,33 @@
 // register top-k"; yifor-blog "設計核心" item 1; yhxrc.cn sec. 二 "block max
 // pooling").
 //
-// One persistent CTA per SM walks 128-query tiles (all G groups of a tile at
-// once, so each index-key block is loaded once for G MMAs).  Per key block j and
-// group g the tensor core computes S = Q_idx[128 x d_idx] * K_idx[j]^T into one of
-// four 128-column TMEM accumulators; an epilogue warpgroup reads its lane's 128
-// scores, takes the max (the block score) and offers (score, j) to the top list
-// of that (query, group).  Blocks arrive in ascending order, so a new block only
+// One persistent CTA per SM walks work units = (128-query tile, pair of GQA
+// groups); the two groups of a unit share each index-key block load.  Per key
+// block j the tensor core computes S_g = Q_idx[g][128 x d_idx] * K_idx[j]^T for
+// both groups into one of two TMEM buffers (2 buffers x 2 groups x 128 columns),
+// so the epilogue drains block j while block j+1 is being computed.  An
+// epilogue warpgroup per group reads its lane's 128 scores, takes the max (the
+// block score) and offers (score, j) to the register top list of that
+// (query, group).  Blocks arrive in ascending order, so a new block only
 // displaces a strictly lower score: ties stay with the lower block index.
 //
-// Warp roles (576 threads): warps 4g .. 4g+3 form the epilogue set of group g
-// (G <= 4 sets; accumulator g belongs to group g), warp 16 issues TMA loads,
-// warp 17 owns TMEM and issues the MMAs.  While set g drains key block j, the
-// tensor core computes block j for the other groups, so each set has about G
-// MMA-times to read its 128 columns, pool them and update its lists.
+// Warp roles (320 threads): warps 4l .. 4l+3 are the epilogue of the unit's
+// l-th group, warp 8 issues TMA loads, warp 9 owns TMEM and issues the MMAs.
 #include "msa_common.cuh"
 
 namespace msa {
 namespace {
 
-constexpr int kStages = 4;        // max index-key block stages in shared memory
-constexpr int kAcc = 4;           // 128-column TMEM accumulators (512 columns), one per group
-constexpr int kThreads = 576;
-constexpr int kProducerWarp = 16;
-constexpr int kMmaWarp = 17;
+constexpr int kStages = 6;        // max index-key block stages in shared memory
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr int kTile = 128;        // queries per tile = key-block size
 
 struct __align__(16) IndexCtl {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t acc_full[kAcc], acc_empty[kAcc];
+  uint64_t acc_full[2], acc_empty[2];
   uint64_t mma_done;
   uint32_t tmem_base;
   int32_t abort_flag;
@@ -69,13 +67,13 @@ __device__ __forceinline__ TileInfo tile_info(int tau, const IndexCtl* ctl, int 
   return t;
 }
 
-// Static snake schedule over tiles in longest-first order: iteration `it` of
-// CTA c takes slot it*grid + (it even ? c : grid-1-c); slot s is tile
-// ntiles-1-s (later tiles of a sequence scan more key blocks).
-__device__ __forceinline__ int snake_tile(int it, int ntiles) {
+// Static snake schedule over work units in longest-first order: iteration
+// `it` of CTA c takes slot it*grid + (it even ? c : grid-1-c); slot s is unit
+// nunits-1-s (units of later tiles scan more key blocks).
+__device__ __forceinline__ int snake_unit(int it, int nunits) {
   const int g = gridDim.x, c = blockIdx.x;
   const int slot = it * g + ((it & 1) ? (g - 1 - c) : c);
-  return slot < ntiles ? (ntiles - 1 - slot) : -1;
+  return slot < nunits ? (nunits - 1 - slot) : -1;
 }
 
 template <int CAP>
@@ -161,6 +159,8 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
                           const int32_t* __restrict__ cu_k, int batch, int d_idx, int k, int nst,
                           DevError* err) {
   constexpr int CAP = KMAX - 1;
+  constexpr int GP = G < 2 ? G : 2;          // groups per work unit
+  constexpr int NPAIR = (G + GP - 1) / GP;   // units per tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -169,8 +169,8 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
   const int span_el = span / 2;
   const int nbox = (d_idx * 2) / span;                    // boxes per 128-row tile
   const uint32_t tile_bytes = kTile * d_idx * 2;          // one [128 x d_idx] bf16 tile
-  uint8_t* q_s = smem;                                    // G tiles
-  uint8_t* k_s = smem + G * tile_bytes;                   // kStages tiles
+  uint8_t* q_s = smem;                                    // GP tiles
+  uint8_t* k_s = smem + GP * tile_bytes;                  // nst tiles
   IndexCtl* ctl = reinterpret_cast<IndexCtl*>(k_s + nst * tile_bytes);
   volatile int32_t* abort_flag = &ctl->abort_flag;
 
@@ -181,7 +181,7 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
     mbar_init(&ctl->q_full, 1);
     mbar_init(&ctl->q_empty, 1);
     for (int s = 0; s < kStages; ++s) { mbar_init(&ctl->k_full[s], 1); mbar_init(&ctl->k_empty[s], 1); }
-    for (int a = 0; a < kAcc; ++a) { mbar_init(&ctl->acc_full[a], 1); mbar_init(&ctl->acc_empty[a], 4); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&ctl->acc_full[b], 1); mbar_init(&ctl->acc_empty[b], 4 * GP); }
     mbar_init(&ctl->mma_done, 1);
     ctl->abort_flag = 0;
     // tiles per sequence (sequences with T_b > S_b are rejected and skipped)
@@ -212,29 +212,31 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
-  const int ntiles = ctl->ntiles;
+  const int nunits = ctl->ntiles * NPAIR;
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
       uint32_t kstep = 0, qiter = 0;
       for (int it = 0;; ++it) {
-        const int tau = snake_tile(it, ntiles);
-        if (tau < 0 || *abort_flag) break;
-        const TileInfo ti = tile_info(tau, ctl, batch, cu_q, cu_k);
+        const int u = snake_unit(it, nunits);
+        if (u < 0 || *abort_flag) break;
+        const int pair = u % NPAIR;
+        const TileInfo ti = tile_info(u / NPAIR, ctl, batch, cu_q, cu_k);
         if (!mbar_wait(&ctl->q_empty, (qiter + 1) & 1)) {
-          report_error(err, MSA_ERR_TIMEOUT, kSiteIndexProducer, tau, -1);
+          report_error(err, MSA_ERR_TIMEOUT, kSiteIndexProducer, u, -1);
           *abort_flag = 1;
           break;
         }
-        mbar_arrive_expect_tx(&ctl->q_full, G * tile_bytes);
-        for (int g = 0; g < G; ++g)
+        mbar_arrive_expect_tx(&ctl->q_full, GP * tile_bytes);
+        for (int l = 0; l < GP; ++l)
           for (int bx = 0; bx < nbox; ++bx)
-            tma_load_3d(q_s + g * tile_bytes + bx * kTile * span, &tm_q, &ctl->q_full, bx * span_el, g, ti.q0);
+            tma_load_3d(q_s + l * tile_bytes + bx * kTile * span, &tm_q, &ctl->q_full, bx * span_el,
+                        pair * GP + l, ti.q0);
         ++qiter;
         for (int j = 0; j < ti.n_kb; ++j) {
           const int st = kstep % nst;
           if (!mbar_wait(&ctl->k_empty[st], ((kstep / nst) + 1) & 1)) {
-            report_error(err, MSA_ERR_TIMEOUT, kSiteIndexProducer, tau, j);
+            report_error(err, MSA_ERR_TIMEOUT, kSiteIndexProducer, u, j);
             *abort_flag = 1;
             break;
           }
@@ -263,14 +265,15 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
       const int nk = d_idx / 16;
       const int per_sh = span == 128 ? 2 : (span == 64 ? 1 : 0);   // log2(K steps per swizzled row)
       const uint64_t qdesc0 = make_sdesc(smem_u32(q_s), 16, sbo, mode);
-      uint32_t kstep = 0, jstep = 0, qiter = 0;   // jstep: key blocks issued (all tiles)
+      const uint64_t kdesc0 = make_sdesc(smem_u32(k_s), 16, sbo, mode);
+      uint32_t kstep = 0, jstep = 0, qiter = 0;   // jstep: key blocks issued (all units)
       bool ok = true;
       for (int it = 0; ok; ++it) {
-        const int tau = snake_tile(it, ntiles);
-        if (tau < 0 || *abort_flag) break;
-        const TileInfo ti = tile_info(tau, ctl, batch, cu_q, cu_k);
+        const int u = snake_unit(it, nunits);
+        if (u < 0 || *abort_flag) break;
+        const TileInfo ti = tile_info(u / NPAIR, ctl, batch, cu_q, cu_k);
         if (!mbar_wait(&ctl->q_full, qiter & 1)) {
-          report_error(err, MSA_ERR_TIMEOUT, kSiteIndexMma, tau, -1);
+          report_error(err, MSA_ERR_TIMEOUT, kSiteIndexMma, u, -1);
           ok = false;
           break;
         }
@@ -278,28 +281,26 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         tc_fence_after();
         for (int j = 0; j < ti.n_kb && ok; ++j, ++jstep) {
           const int st = kstep % nst;
-          if (!mbar_wait(&ctl->k_full[st], (kstep / nst) & 1)) {
-            report_error(err, MSA_ERR_TIMEOUT, kSiteIndexMma, tau, j);
+          const int buf = jstep & 1;
+          if (!mbar_wait(&ctl->k_full[st], (kstep / nst) & 1) ||
+              !mbar_wait(&ctl->acc_empty[buf], ((jstep >> 1) + 1) & 1)) {
+            report_error(err, MSA_ERR_TIMEOUT, kSiteIndexMma, u, j);
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t bdesc = make_sdesc(smem_u32(k_s + st * tile_bytes), 16, sbo, mode);
-          for (int g = 0; g < G; ++g) {
-            if (!mbar_wait(&ctl->acc_empty[g], (jstep + 1) & 1)) {
-              report_error(err, MSA_ERR_TIMEOUT, kSiteIndexMma, tau, 1000 + j);
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint64_t adesc = qdesc0 + (uint64_t)((g * tile_bytes) >> 4);
+          const uint64_t bdesc = kdesc0 + (uint64_t)((st * tile_bytes) >> 4);
+#pragma unroll
+          for (int l = 0; l < GP; ++l) {
+            const uint64_t adesc = qdesc0 + (uint64_t)((l * tile_bytes) >> 4);
+            const uint32_t acc = tmem_base + (buf * GP + l) * 128;
             for (int kk = 0; kk < nk; ++kk) {
               const uint64_t off =
                   (uint64_t)((((kk >> per_sh) * (kTile * span)) + ((kk & ((1 << per_sh) - 1)) * 32)) >> 4);
-              umma_bf16_ss(tmem_base + g * 128, adesc + off, bdesc + off, idesc, kk > 0 ? 1u : 0u);
+              umma_bf16_ss(acc, adesc + off, bdesc + off, idesc, kk > 0 ? 1u : 0u);
             }
-            umma_commit(&ctl->acc_full[g]);
           }
+          umma_commit(&ctl->acc_full[buf]);
           umma_commit(&ctl->k_empty[st]);
           ++kstep;
           if (*abort_flag) ok = false;
@@ -311,41 +312,45 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
       umma_commit(&ctl->mma_done);
       mbar_wait(&ctl->mma_done, 0);
     }
-  } else if (warp < 4 * G) {
+  } else if (warp < 4 * GP) {
     // ------------------------------------------------------------ epilogue
-    const int g = warp / 4;            // group of this set = its accumulator
+    const int l = warp / 4;            // group slot of this set within the unit
     const int wq = warp % 4;           // TMEM lane quarter
     const int row = 32 * wq + lane;
-    const uint32_t ta = tmem_base + (static_cast<uint32_t>(32 * wq) << 16) + g * 128;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * wq) << 16) + l * 128;
     TopList<CAP> list;
     uint32_t jstep = 0;
     for (int it = 0;; ++it) {
-      const int tau = snake_tile(it, ntiles);
-      if (tau < 0 || *abort_flag) break;
-      const TileInfo ti = tile_info(tau, ctl, batch, cu_q, cu_k);
+      const int u = snake_unit(it, nunits);
+      if (u < 0 || *abort_flag) break;
+      const int g = (u % NPAIR) * GP + l;
+      const TileInfo ti = tile_info(u / NPAIR, ctl, batch, cu_q, cu_k);
       const bool valid = row < ti.rows;
       const int lb = (ti.pos0 + row) / kBk;
       list.reset();
       bool ok = true;
       for (int j = 0; j < ti.n_kb; ++j, ++jstep) {
-        if (!mbar_wait(&ctl->acc_full[g], jstep & 1)) {
-          report_error(err, MSA_ERR_TIMEOUT, kSiteIndexEpilogue, tau, j);
+        const int buf = jstep & 1;
+        if (!mbar_wait(&ctl->acc_full[buf], (jstep >> 1) & 1)) {
+          report_error(err, MSA_ERR_TIMEOUT, kSiteIndexEpilogue, u, j);
           *abort_flag = 1;
           ok = false;
           break;
         }
         tc_fence_after();
-        uint32_t r0[32];
-        float m = -INFINITY;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          tmem_ld32(ta + 32 * cc, r0);
-          tmem_ld_wait();
-          m = fmaxf(m, max_of_32(r0));
-        }
+        const uint32_t ta = lane_base + buf * GP * 128;
+        uint32_t r0[32], r1[32];
+        tmem_ld32(ta, r0);
+        tmem_ld32(ta + 32, r1);
+        tmem_ld_wait();
+        float m = fmaxf(max_of_32(r0), max_of_32(r1));
+        tmem_ld32(ta + 64, r0);
+        tmem_ld32(ta + 96, r1);
+        tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->acc_empty[g]);
+        if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
+        m = fmax3(m, max_of_32(r0), max_of_32(r1));
         if (m != m) m = -INFINITY;    // a block of NaN scores ranks as -inf
         if (valid && j < lb) list.offer(m, j, k - 1);
       }
@@ -383,8 +388,9 @@ int launch_index_topk_prefill(const IndexTopkArgs& a, void* stream) {
     if (rc) return rc;
   }
   const size_t tile_bytes = (size_t)kTile * a.d_idx * 2;
-  const int nst = a.d_idx >= 128 ? 2 : kStages;   // keep G + nst tiles within shared memory
-  size_t smem = 1024 + a.G * tile_bytes + nst * tile_bytes + sizeof(IndexCtl);
+  const int gp = a.G < 2 ? a.G : 2;
+  const int nst = a.d_idx >= 128 ? 4 : kStages;   // keep gp + nst tiles within shared memory
+  size_t smem = 1024 + gp * tile_bytes + nst * tile_bytes + sizeof(IndexCtl);
   // at least 116 KB so that exactly one CTA (and one 512-column TMEM owner) sits on each SM
   if (smem < 116 * 1024) smem = 116 * 1024;
   int dev = 0, nsm = 0;
