@@ -129,16 +129,18 @@ def make_ctx(w, inp, torch, msa):
     lib = msa.load_library()
     import ctypes
     n_idx = lib.msa_index_topk_workspace_size(ctypes.byref(shape), ctypes.byref(seqs))
-    n_att = msa.msa_sparse_attn_workspace_size(shape, seqs, 0)
+    n_att = msa.msa_sparse_attn_workspace_size(shape, seqs, 0) if not getattr(make_ctx, "index_only", False) else 256
     ctx["ws_idx"] = torch.empty(n_idx, dtype=torch.uint8, device=dev)
     ctx["ws_att"] = torch.empty(n_att, dtype=torch.uint8, device=dev)
     return ctx
 
 
-def step_prefill(ctx, msa, inp=None):
+def step_prefill(ctx, msa, inp=None, index_only=False):
     inp = inp or ctx["inp"]
     msa.msa_index_topk(ctx["shape"], ctx["seqs"], inp["q_idx"], inp["k_idx"], sel=ctx["sel"], ws=ctx["ws_idx"],
                        check=False)
+    if index_only:
+        return
     msa.msa_sparse_attn_prefill(ctx["shape"], ctx["seqs"], inp["q"], inp["k"], inp["v"], ctx["sel"],
                                 out=ctx["out"], want_lse=False, ws=ctx["ws_att"], check=False)
 
@@ -320,14 +322,16 @@ def run_ours(args):
     wr = W.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
     inp = W.make_inputs(wr, "cuda", T_override=args.T or None)
     torch.cuda.synchronize()
+    make_ctx.index_only = args.index_only
     ctx = make_ctx(wr, inp, torch, msa)
+    make_ctx.index_only = False
     S_lens = [inp["cu_k_host"][i + 1] - inp["cu_k_host"][i] for i in range(len(inp["cu_k_host"]) - 1)]
     T_lens = [inp["cu_q_host"][i + 1] - inp["cu_q_host"][i] for i in range(len(inp["cu_q_host"]) - 1)]
     T = ctx["T"]
     work = R.prefill_work(S_lens, T_lens, w.H, w.G, w.d, w.d_idx, w.B_k, w.k)
 
     for _ in range(args.warmup):
-        step_prefill(ctx, msa)
+        step_prefill(ctx, msa, index_only=args.index_only)
     torch.cuda.synchronize()
     device_errors(ctx, msa)
 
@@ -337,7 +341,7 @@ def run_ours(args):
     clocks.start()
     msa.msa_profile_reset()
     msa.msa_profile_enable(True)
-    ms = time_steps(lambda: step_prefill(ctx, msa), args.steps, torch, dist)
+    ms = time_steps(lambda: step_prefill(ctx, msa, index_only=args.index_only), args.steps, torch, dist)
     msa.msa_profile_enable(False)
     clk = clocks.stop()
     device_errors(ctx, msa)
@@ -468,6 +472,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=PREFILL)
     ap.add_argument("--T", type=int, default=0, help="shorter prefill (same heads/dims), for profiling")
+    ap.add_argument("--index-only", action="store_true", help="time only the index branch (for profiling)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
