@@ -131,7 +131,8 @@ def make_ctx(w, inp, torch, msa):
     n_idx = lib.msa_index_topk_workspace_size(ctypes.byref(shape), ctypes.byref(seqs))
     n_att = msa.msa_sparse_attn_workspace_size(shape, seqs, 0) if not getattr(make_ctx, "index_only", False) else 256
     ctx["ws_idx"] = torch.empty(n_idx, dtype=torch.uint8, device=dev)
-    ctx["ws_att"] = torch.empty(n_att, dtype=torch.uint8, device=dev)
+    ctx["ws_att"] = torch.zeros(n_att, dtype=torch.uint8, device=dev) if n_att <= 256 else \
+        torch.empty(n_att, dtype=torch.uint8, device=dev)
     return ctx
 
 
