@@ -536,8 +536,14 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           for (int c4 = 0; c4 < 4; ++c4) {
             tmem_ld32(s_col + 32 * c4, rr);
             tmem_ld_wait();
+            float mm[16];
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) m = fmax3(m, __uint_as_float(rr[j]), __uint_as_float(rr[j + 1]));
+            for (int j = 0; j < 16; ++j) mm[j] = fmaxf(__uint_as_float(rr[2 * j]), __uint_as_float(rr[2 * j + 1]));
+#pragma unroll
+            for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+              for (int j = 0; j < w; ++j) mm[j] = fmaxf(mm[j], mm[j + w]);
+            m = fmaxf(m, mm[0]);
           }
           ms = m * scale_log2;
 #pragma unroll 1

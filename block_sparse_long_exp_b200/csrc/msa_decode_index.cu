@@ -144,8 +144,8 @@ decode_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16
           ldmatrix_x4(addr, a0, a1, a2, a3);
           mma_bf16_16816(c, a0, a1, a2, a3, bfrag[kk][0], bfrag[kk][1]);
         }
-        mx0 = fmax3(mx0, c[0], c[2]);
-        mx1 = fmax3(mx1, c[1], c[3]);
+        mx0 = fmaxf(mx0, fmaxf(c[0], c[2]));
+        mx1 = fmaxf(mx1, fmaxf(c[1], c[3]));
       }
 #pragma unroll
       for (int o = 4; o < 32; o <<= 1) {

@@ -131,25 +131,17 @@ struct TopList {
   }
 };
 
-__device__ __forceinline__ float max_of_16(const uint32_t (&r)[16]) {
-  const float a = fmax3(__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]));
-  const float b = fmax3(__uint_as_float(r[3]), __uint_as_float(r[4]), __uint_as_float(r[5]));
-  const float c = fmax3(__uint_as_float(r[6]), __uint_as_float(r[7]), __uint_as_float(r[8]));
-  const float d = fmax3(__uint_as_float(r[9]), __uint_as_float(r[10]), __uint_as_float(r[11]));
-  const float e = fmax3(__uint_as_float(r[12]), __uint_as_float(r[13]), __uint_as_float(r[14]));
-  return fmax3(fmax3(a, b, c), fmax3(d, e, __uint_as_float(r[15])), -INFINITY);
-}
-
+// Max of 32 scores as a tree of 2-input fmaxf (ALU pipe; the 3-input form
+// issues on the much narrower XU pipe).
 __device__ __forceinline__ float max_of_32(const uint32_t (&r)[32]) {
-  float m[11];
+  float m[16];
 #pragma unroll
-  for (int i = 0; i < 10; ++i)
-    m[i] = fmax3(__uint_as_float(r[3 * i]), __uint_as_float(r[3 * i + 1]), __uint_as_float(r[3 * i + 2]));
-  m[10] = fmaxf(__uint_as_float(r[30]), __uint_as_float(r[31]));
-  const float a = fmax3(m[0], m[1], m[2]);
-  const float b = fmax3(m[3], m[4], m[5]);
-  const float c = fmax3(m[6], m[7], m[8]);
-  return fmax3(fmax3(a, b, c), m[9], m[10]);
+  for (int i = 0; i < 16; ++i) m[i] = fmaxf(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
+  return m[0];
 }
 
 template <int KMAX, int G>
@@ -350,7 +342,7 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
-        m = fmax3(m, max_of_32(r0), max_of_32(r1));
+        m = fmaxf(m, fmaxf(max_of_32(r0), max_of_32(r1)));
         if (m != m) m = -INFINITY;    // a block of NaN scores ranks as -inf
         if (valid && j < lb) list.offer(m, j, k - 1);
       }
