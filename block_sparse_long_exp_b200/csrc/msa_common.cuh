@@ -70,14 +70,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// try_wait with a suspend-time hint: the thread may sleep (up to hint_ns) until
+// the phase completes instead of spinning.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 // Wait for the phase with the given parity to complete.  Returns false after
-// ~1 s; the caller then records MSA_ERR_TIMEOUT and unwinds.
+// ~1 s; the caller then records MSA_ERR_TIMEOUT and unwinds.  The wall clock
+// is read only every 64 failed tries (reading it each time floods the XU pipe
+// while many warps wait).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) return false;
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if ((n & 63u) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
   }
 }
 
