@@ -269,7 +269,8 @@ struct TileRef {
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                   const __grid_constant__ CUtensorMap tm_q, const Item* __restrict__ items,
+                   const __grid_constant__ CUtensorMap tm_q, const __nv_bfloat16* __restrict__ q_ptr,
+                   const Item* __restrict__ items,
                    const int32_t* __restrict__ nitems_p, int32_t* __restrict__ ticket,
                    const uint32_t* __restrict__ entries, const int32_t* __restrict__ cu_q,
                    const int32_t* __restrict__ cu_k, int H, int G, int d, int k, float scale_log2,
@@ -355,7 +356,13 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         break;
       }
       const Item I = items[it];
-      for (int j = lane; j < I.count; j += 32) R->ent[j] = entries[I.start + j];
+      for (int j = lane; j < I.count; j += 32) {
+        const uint32_t e = entries[I.start + j];
+        R->ent[j] = e;
+        // bring the query's Hg head rows into L2 ahead of the tile's TMA gather
+        const int64_t t = t0 + e / k;
+        prefetch_l2(q_ptr + ((t * H) + (int64_t)I.g * Hg) * d, (uint32_t)(Hg * d * 2));
+      }
       if (lane == 0) {
         R->seq = I.seq; R->blk = I.blk; R->g = I.g; R->start = I.start; R->count = I.count;
         R->Tb = cu_q[I.seq + 1] - cu_q[I.seq];
@@ -473,15 +480,48 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         if (tr.last) umma_commit(&ctl->kv_empty[st]);
         return true;
       };
-      TileRef t0r, t1r;
-      if (next_tile(t0r)) {
-        ok = issue_s(t0r);
-        while (ok && !*abort_flag) {
-          const bool more = next_tile(t1r);
-          if (more && !(ok = issue_s(t1r))) break;
-          if (!(ok = issue_pv(t0r))) break;
-          if (!more) break;
-          t0r = t1r;
+      // Event-driven issue: S(next) and PV(oldest pending) go out as soon as
+      // their inputs are ready, so a slow query gather never holds back the
+      // PV of an earlier tile.  At most two tiles are between S and PV (the two
+      // TMEM slots); S(t) may overwrite slot t%2 because PV(t-2) was issued first.
+      TileRef pend[2];
+      int npend = 0, head = 0;
+      TileRef nxt;
+      bool have_nxt = next_tile(nxt);
+      uint64_t t_idle = 0;
+      uint32_t spins = 0;
+      while (ok && (have_nxt || npend > 0)) {
+        bool progress = false;
+        if (have_nxt && npend < 2) {
+          const int qs = nxt.tau % kQSlots, st = nxt.item_seq & 1;
+          if (mbar_try_wait(&ctl->q_full[qs], (nxt.tau / kQSlots) & 1) &&
+              (!nxt.first || mbar_try_wait(&ctl->kv_full[st], (nxt.item_seq >> 1) & 1))) {
+            ok = issue_s(nxt);
+            pend[(head + npend) & 1] = nxt;
+            ++npend;
+            have_nxt = ok && next_tile(nxt);
+            progress = true;
+          }
+        }
+        if (ok && npend > 0) {
+          const TileRef& tp = pend[head];
+          const int s = tp.tau & 1;
+          if (mbar_try_wait(&ctl->p_full[s], (tp.tau >> 1) & 1) &&
+              mbar_try_wait(&ctl->o_free[s], ((tp.tau >> 1) + 1) & 1)) {
+            ok = issue_pv(tp);
+            head ^= 1;
+            --npend;
+            progress = true;
+          }
+        }
+        if (progress) {
+          spins = 0;
+          t_idle = 0;
+        } else if ((++spins & 255u) == 0) {
+          const uint64_t now = global_ns();
+          if (t_idle == 0) t_idle = now;
+          else if (now - t_idle > kWaitLimitNs) ok = false;
+          if (*abort_flag) break;
         }
       }
       if (!ok) {
@@ -783,7 +823,7 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
   {
     ProfScope p("sparse_attn", stream);
     sparse_attn_kernel<<<nsm, kAttnThreads, smem, st>>>(
-        tm_k, tm_v, tm_q, a.items, a.nitems, a.nitems + 1, a.entries, a.cu_q, a.cu_k, a.H, a.G, a.d, a.k,
+        tm_k, tm_v, tm_q, reinterpret_cast<const __nv_bfloat16*>(a.q), a.items, a.nitems, a.nitems + 1, a.entries, a.cu_q, a.cu_k, a.H, a.G, a.d, a.k,
         scale_log2, a.t0, reinterpret_cast<__half*>(a.part_acc), a.part_lse, a.err);
   }
   e = cudaGetLastError();

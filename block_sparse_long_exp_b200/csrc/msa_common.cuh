@@ -122,6 +122,11 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+// L2 prefetch of a contiguous global range (16-byte aligned, size % 16 == 0).
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ------------------------------------------------------ cp.async (gather) ---
 
 __device__ __forceinline__ void cp_async_16(void* dst, const void* src) {
