@@ -229,9 +229,10 @@ __global__ void __launch_bounds__(kScanThreads) scan_items_kernel(const int32_t*
 //               TMA-loads the item's K and V block into one of two stages and
 //               gathers each 128-row tile's query rows with one TMA box per
 //               (query, 64-column half) into one of three Q slots;
-//   warp 1      owns TMEM (512 columns = two slots of S/P + O) and issues the
-//               MMAs: S(t+1) = Q K^T is issued before O(t) = P V so the
-//               tensor core works while tile t's softmax runs;
+//   warp 1      owns TMEM (512 columns = two slots of S/P + O); its lane 0
+//               issues S = Q K^T, lane 0 of warp 2 issues O = P V (two
+//               issue/commit streams keep the tensor core fed while tile t's
+//               softmax runs);
 //   warps 4-7   softmax + epilogue of even tiles (TMEM slot 0),
 //   warps 8-11  the same for odd tiles (slot 1): S -> P (bf16, written back
 //               into the S columns, the A operand of the PV MMA), then O / l
@@ -242,7 +243,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_items_kernel(const int32_t*
 constexpr int kAttnThreads = 384;
 constexpr int kItemRing = 4;
 constexpr int kQSlots = 3;
-constexpr int kItemEmptyCount = 9;    // MMA 1 + softmax warps 8
+constexpr int kItemEmptyCount = 10;   // MMA issuers 2 + softmax warps 8
 
 struct __align__(16) RingItem {
   int32_t seq, blk, g, start, count, Tb, Sb, qrow0;
@@ -254,23 +255,16 @@ struct __align__(16) AttnCtl {
   uint64_t kv_full[2], kv_empty[2];
   uint64_t q_full[kQSlots], q_empty[kQSlots];
   uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
-  uint64_t mma_done;
+  uint64_t mma_done[2];
   uint32_t tmem_base;
   int32_t abort_flag;
   int32_t pad[2];
   RingItem ring[kItemRing];
 };
 
-struct TileRef {
-  int tau;        // tile counter of this CTA
-  int item_seq;   // item counter of this CTA
-  bool first, last;
-};
-
 __global__ void __launch_bounds__(kAttnThreads, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                   const __grid_constant__ CUtensorMap tm_q, const __nv_bfloat16* __restrict__ q_ptr,
-                   const Item* __restrict__ items,
+                   const __grid_constant__ CUtensorMap tm_q, const Item* __restrict__ items,
                    const int32_t* __restrict__ nitems_p, int32_t* __restrict__ ticket,
                    const uint32_t* __restrict__ entries, const int32_t* __restrict__ cu_q,
                    const int32_t* __restrict__ cu_k, int H, int G, int d, int k, float scale_log2,
@@ -299,7 +293,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       mbar_init(&ctl->o_full[i], 1); mbar_init(&ctl->o_free[i], 4);
     }
     for (int i = 0; i < kQSlots; ++i) { mbar_init(&ctl->q_full[i], 1); mbar_init(&ctl->q_empty[i], 1); }
-    mbar_init(&ctl->mma_done, 1);
+    mbar_init(&ctl->mma_done[0], 1);
+    mbar_init(&ctl->mma_done[1], 1);
     ctl->abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_k);
@@ -356,13 +351,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         break;
       }
       const Item I = items[it];
-      for (int j = lane; j < I.count; j += 32) {
-        const uint32_t e = entries[I.start + j];
-        R->ent[j] = e;
-        // bring the query's Hg head rows into L2 ahead of the tile's TMA gather
-        const int64_t t = t0 + e / k;
-        prefetch_l2(q_ptr + ((t * H) + (int64_t)I.g * Hg) * d, (uint32_t)(Hg * d * 2));
-      }
+      for (int j = lane; j < I.count; j += 32) R->ent[j] = entries[I.start + j];
       if (lane == 0) {
         R->seq = I.seq; R->blk = I.blk; R->g = I.g; R->start = I.start; R->count = I.count;
         R->Tb = cu_q[I.seq + 1] - cu_q[I.seq];
@@ -419,9 +408,15 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         if (issued > 0) mbar_wait(&ctl->q_full[qs], (issued - 1) & 1);
       }
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // -------------------------------------------------------- MMA issuers
+    // lane 0 of warp 1 issues every S = Q K^T, lane 0 of warp 2 every O = P V,
+    // each with its own commit stream (a thread that mixes commits into its
+    // MMAs issues at about half the MMA rate).  The two streams are not
+    // ordered against each other, so S(t) waits for PV(t-2) to complete
+    // before it overwrites slot t%2, whose first 64 columns hold P(t-2).
     if (lane == 0) {
+      const bool is_s = (warp == 1);
       const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       const uint32_t idesc_o = idesc_bf16_f32(128, d, 0, 1);
       // descriptors built once; per-slot / per-step byte offsets (>> 4) are added
@@ -429,107 +424,58 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       const uint64_t kvdesc0 = make_sdesc(smem_u32(kv_s), 16, 1024, kSw128);
       const uint64_t vdesc0 = make_sdesc(smem_u32(kv_s + tile_bytes), 128 * 128, 1024, kSw128);
       int n = 0, tau = 0;
-      int cur_tiles = 0, mt = 0, cur_seq = -1;
-      bool have = false, ok = true, done = false;
-      // next tile in the stream (consumes ring items as needed)
-      auto next_tile = [&](TileRef& tr) -> bool {
-        if (done) return false;
-        if (!have || mt >= cur_tiles) {
-          const RingItem* R = wait_item(n);
-          if (R == nullptr) { done = true; return false; }
-          const int cnt = R->count;
-          release_item(n, false);
-          if (cnt <= 0) { done = true; return false; }
-          cur_seq = n++;
-          cur_tiles = (cnt + qpt - 1) / qpt;
-          mt = 0;
-          have = true;
-        }
-        tr.tau = tau++;
-        tr.item_seq = cur_seq;
-        tr.first = (mt == 0);
-        tr.last = (mt == cur_tiles - 1);
-        ++mt;
-        return true;
-      };
-      auto issue_s = [&](const TileRef& tr) -> bool {
-        const int qs = tr.tau % kQSlots, s = tr.tau & 1, st = tr.item_seq & 1;
-        if (!mbar_wait(&ctl->q_full[qs], (tr.tau / kQSlots) & 1)) return false;
-        if (tr.first && !mbar_wait(&ctl->kv_full[st], (tr.item_seq >> 1) & 1)) return false;
-        tc_fence_after();
-        const uint64_t qd = qdesc0 + (uint64_t)((qs * tile_bytes) >> 4);
-        const uint64_t kd = kvdesc0 + (uint64_t)((st * 2 * tile_bytes) >> 4);
-        for (int kk = 0; kk < d / 16; ++kk) {
-          const uint64_t off = (uint64_t)(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
-          umma_bf16_ss(tmem + s * 256, qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&ctl->s_full[s]);
-        umma_commit(&ctl->q_empty[qs]);
-        return true;
-      };
-      auto issue_pv = [&](const TileRef& tr) -> bool {
-        const int s = tr.tau & 1, st = tr.item_seq & 1;
-        if (!mbar_wait(&ctl->p_full[s], (tr.tau >> 1) & 1)) return false;
-        if (!mbar_wait(&ctl->o_free[s], ((tr.tau >> 1) + 1) & 1)) return false;
-        tc_fence_after();
-        const uint64_t vd = vdesc0 + (uint64_t)((st * 2 * tile_bytes) >> 4);
-        const uint32_t pcol = tmem + s * 256, ocol = pcol + 128;
-        for (int kk = 0; kk < 8; ++kk)
-          umma_bf16_ts(ocol, pcol + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : 0u);
-        umma_commit(&ctl->o_full[s]);
-        if (tr.last) umma_commit(&ctl->kv_empty[st]);
-        return true;
-      };
-      // Event-driven issue: S(next) and PV(oldest pending) go out as soon as
-      // their inputs are ready, so a slow query gather never holds back the
-      // PV of an earlier tile.  At most two tiles are between S and PV (the two
-      // TMEM slots); S(t) may overwrite slot t%2 because PV(t-2) was issued first.
-      TileRef pend[2];
-      int npend = 0, head = 0;
-      TileRef nxt;
-      bool have_nxt = next_tile(nxt);
-      uint64_t t_idle = 0;
-      uint32_t spins = 0;
-      while (ok && (have_nxt || npend > 0)) {
-        bool progress = false;
-        if (have_nxt && npend < 2) {
-          const int qs = nxt.tau % kQSlots, st = nxt.item_seq & 1;
-          if (mbar_try_wait(&ctl->q_full[qs], (nxt.tau / kQSlots) & 1) &&
-              (!nxt.first || mbar_try_wait(&ctl->kv_full[st], (nxt.item_seq >> 1) & 1))) {
-            ok = issue_s(nxt);
-            pend[(head + npend) & 1] = nxt;
-            ++npend;
-            have_nxt = ok && next_tile(nxt);
-            progress = true;
+      bool ok = true;
+      while (ok && !*abort_flag) {
+        const RingItem* R = wait_item(n);
+        if (R == nullptr) { ok = false; break; }
+        const int cnt = R->count;
+        release_item(n, false);
+        if (cnt <= 0) break;
+        const int st = n & 1;
+        const int ntiles = (cnt + qpt - 1) / qpt;
+        for (int mt = 0; mt < ntiles && ok; ++mt, ++tau) {
+          const int s = tau & 1;
+          if (is_s) {
+            const int qs = tau % kQSlots;
+            if (!mbar_wait(&ctl->q_full[qs], (tau / kQSlots) & 1) ||
+                (mt == 0 && !mbar_wait(&ctl->kv_full[st], (n >> 1) & 1)) ||
+                !mbar_wait(&ctl->o_full[s], ((tau >> 1) + 1) & 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t qd = qdesc0 + (uint64_t)((qs * tile_bytes) >> 4);
+            const uint64_t kd = kvdesc0 + (uint64_t)((st * 2 * tile_bytes) >> 4);
+            for (int kk = 0; kk < d / 16; ++kk) {
+              const uint64_t off = (uint64_t)(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
+              umma_bf16_ss(tmem + s * 256, qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&ctl->s_full[s]);
+            umma_commit(&ctl->q_empty[qs]);
+          } else {
+            if (!mbar_wait(&ctl->p_full[s], (tau >> 1) & 1) ||
+                !mbar_wait(&ctl->o_free[s], ((tau >> 1) + 1) & 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t vd = vdesc0 + (uint64_t)((st * 2 * tile_bytes) >> 4);
+            const uint32_t pcol = tmem + s * 256, ocol = pcol + 128;
+            for (int kk = 0; kk < 8; ++kk)
+              umma_bf16_ts(ocol, pcol + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : 0u);
+            umma_commit(&ctl->o_full[s]);
+            // K was read by S MMAs that completed before P existed; V by these
+            if (mt == ntiles - 1) umma_commit(&ctl->kv_empty[st]);
           }
         }
-        if (ok && npend > 0) {
-          const TileRef& tp = pend[head];
-          const int s = tp.tau & 1;
-          if (mbar_try_wait(&ctl->p_full[s], (tp.tau >> 1) & 1) &&
-              mbar_try_wait(&ctl->o_free[s], ((tp.tau >> 1) + 1) & 1)) {
-            ok = issue_pv(tp);
-            head ^= 1;
-            --npend;
-            progress = true;
-          }
-        }
-        if (progress) {
-          spins = 0;
-          t_idle = 0;
-        } else if ((++spins & 255u) == 0) {
-          const uint64_t now = global_ns();
-          if (t_idle == 0) t_idle = now;
-          else if (now - t_idle > kWaitLimitNs) ok = false;
-          if (*abort_flag) break;
-        }
+        ++n;
       }
       if (!ok) {
-        report_error(err, MSA_ERR_TIMEOUT, kSiteAttnMma, tau, n);
+        report_error(err, MSA_ERR_TIMEOUT, kSiteAttnMma, tau, is_s ? 0 : 1);
         *abort_flag = 1;
       }
-      umma_commit(&ctl->mma_done);
-      mbar_wait(&ctl->mma_done, 0);
+      umma_commit(&ctl->mma_done[is_s ? 0 : 1]);
+      mbar_wait(&ctl->mma_done[is_s ? 0 : 1], 0);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------- softmax + epilogue
@@ -823,7 +769,7 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
   {
     ProfScope p("sparse_attn", stream);
     sparse_attn_kernel<<<nsm, kAttnThreads, smem, st>>>(
-        tm_k, tm_v, tm_q, reinterpret_cast<const __nv_bfloat16*>(a.q), a.items, a.nitems, a.nitems + 1, a.entries, a.cu_q, a.cu_k, a.H, a.G, a.d, a.k,
+        tm_k, tm_v, tm_q, a.items, a.nitems, a.nitems + 1, a.entries, a.cu_q, a.cu_k, a.H, a.G, a.d, a.k,
         scale_log2, a.t0, reinterpret_cast<__half*>(a.part_acc), a.part_lse, a.err);
   }
   e = cudaGetLastError();

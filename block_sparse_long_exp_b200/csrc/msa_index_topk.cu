@@ -14,24 +14,27 @@
 // (query, group).  Blocks arrive in ascending order, so a new block only
 // displaces a strictly lower score: ties stay with the lower block index.
 //
-// Warp roles (320 threads): warps 4l .. 4l+3 are the epilogue of the unit's
-// l-th group, warp 8 issues TMA loads, warp 9 owns TMEM and issues the MMAs.
+// Warp roles (352 threads): warps 4l .. 4l+3 are the epilogue of the unit's
+// l-th group, warp 8 issues TMA loads, warp 9 owns TMEM, and lane 0 of warp
+// 9 + l issues the MMAs of group l.  One issuing thread per group: a thread
+// that interleaves tcgen05.commit with its MMAs issues at about half the MMA
+// rate, so each group gets its own issue and commit stream.
 #include "msa_common.cuh"
 
 namespace msa {
 namespace {
 
 constexpr int kStages = 6;        // max index-key block stages in shared memory
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp = 9;     // and kMmaWarp + 1 for the second group of a pair
 constexpr int kTile = 128;        // queries per tile = key-block size
 
 struct __align__(16) IndexCtl {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t acc_full[2], acc_empty[2];
-  uint64_t mma_done;
+  uint64_t acc_full[2][2], acc_empty[2][2];   // [buffer][group slot]
+  uint64_t mma_done[2];
   uint32_t tmem_base;
   int32_t abort_flag;
   int32_t ntiles;
@@ -171,10 +174,12 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl->q_full, 1);
-    mbar_init(&ctl->q_empty, 1);
-    for (int s = 0; s < kStages; ++s) { mbar_init(&ctl->k_full[s], 1); mbar_init(&ctl->k_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&ctl->acc_full[b], 1); mbar_init(&ctl->acc_empty[b], 4 * GP); }
-    mbar_init(&ctl->mma_done, 1);
+    mbar_init(&ctl->q_empty, GP);
+    for (int s = 0; s < kStages; ++s) { mbar_init(&ctl->k_full[s], 1); mbar_init(&ctl->k_empty[s], GP); }
+    for (int b = 0; b < 2; ++b)
+      for (int l = 0; l < 2; ++l) { mbar_init(&ctl->acc_full[b][l], 1); mbar_init(&ctl->acc_empty[b][l], 4); }
+    mbar_init(&ctl->mma_done[0], 1);
+    mbar_init(&ctl->mma_done[1], 1);
     ctl->abort_flag = 0;
     // tiles per sequence (sequences with T_b > S_b are rejected and skipped)
     int acc = 0;
@@ -247,8 +252,9 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         if (issued > 0) mbar_wait(&ctl->k_full[st], (issued - 1) & 1);
       }
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp >= kMmaWarp && warp < kMmaWarp + GP) {
     if (lane == 0) {
+      const int l = warp - kMmaWarp;   // group slot issued by this thread
       const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
       const uint32_t mode = sw_mode_for(span);
       const uint32_t sbo = 8 * span;
@@ -256,7 +262,7 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
       // to the start-address field
       const int nk = d_idx / 16;
       const int per_sh = span == 128 ? 2 : (span == 64 ? 1 : 0);   // log2(K steps per swizzled row)
-      const uint64_t qdesc0 = make_sdesc(smem_u32(q_s), 16, sbo, mode);
+      const uint64_t adesc = make_sdesc(smem_u32(q_s + l * tile_bytes), 16, sbo, mode);
       const uint64_t kdesc0 = make_sdesc(smem_u32(k_s), 16, sbo, mode);
       uint32_t kstep = 0, jstep = 0, qiter = 0;   // jstep: key blocks issued (all units)
       bool ok = true;
@@ -275,41 +281,38 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
           const int st = kstep % nst;
           const int buf = jstep & 1;
           if (!mbar_wait(&ctl->k_full[st], (kstep / nst) & 1) ||
-              !mbar_wait(&ctl->acc_empty[buf], ((jstep >> 1) + 1) & 1)) {
+              !mbar_wait(&ctl->acc_empty[buf][l], ((jstep >> 1) + 1) & 1)) {
             report_error(err, MSA_ERR_TIMEOUT, kSiteIndexMma, u, j);
             ok = false;
             break;
           }
           tc_fence_after();
           const uint64_t bdesc = kdesc0 + (uint64_t)((st * tile_bytes) >> 4);
-#pragma unroll
-          for (int l = 0; l < GP; ++l) {
-            const uint64_t adesc = qdesc0 + (uint64_t)((l * tile_bytes) >> 4);
-            const uint32_t acc = tmem_base + (buf * GP + l) * 128;
-            for (int kk = 0; kk < nk; ++kk) {
-              const uint64_t off =
-                  (uint64_t)((((kk >> per_sh) * (kTile * span)) + ((kk & ((1 << per_sh) - 1)) * 32)) >> 4);
-              umma_bf16_ss(acc, adesc + off, bdesc + off, idesc, kk > 0 ? 1u : 0u);
-            }
+          const uint32_t acc = tmem_base + (buf * 2 + l) * 128;
+          for (int kk = 0; kk < nk; ++kk) {
+            const uint64_t off =
+                (uint64_t)((((kk >> per_sh) * (kTile * span)) + ((kk & ((1 << per_sh) - 1)) * 32)) >> 4);
+            umma_bf16_ss(acc, adesc + off, bdesc + off, idesc, kk > 0 ? 1u : 0u);
           }
-          umma_commit(&ctl->acc_full[buf]);
+          umma_commit(&ctl->acc_full[buf][l]);
           umma_commit(&ctl->k_empty[st]);
           ++kstep;
           if (*abort_flag) ok = false;
         }
+        // the Q tile is reused only after every group's MMAs are done
         umma_commit(&ctl->q_empty);
       }
       if (!ok) *abort_flag = 1;
       // All issued MMAs complete before TMEM is released.
-      umma_commit(&ctl->mma_done);
-      mbar_wait(&ctl->mma_done, 0);
+      umma_commit(&ctl->mma_done[l]);
+      mbar_wait(&ctl->mma_done[l], 0);
     }
   } else if (warp < 4 * GP) {
     // ------------------------------------------------------------ epilogue
     const int l = warp / 4;            // group slot of this set within the unit
     const int wq = warp % 4;           // TMEM lane quarter
     const int row = 32 * wq + lane;
-    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * wq) << 16) + l * 128;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * wq) << 16) + l * 128;   // + buf * 256
     TopList<CAP> list;
     uint32_t jstep = 0;
     for (int it = 0;; ++it) {
@@ -323,14 +326,14 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
       bool ok = true;
       for (int j = 0; j < ti.n_kb; ++j, ++jstep) {
         const int buf = jstep & 1;
-        if (!mbar_wait(&ctl->acc_full[buf], (jstep >> 1) & 1)) {
+        if (!mbar_wait(&ctl->acc_full[buf][l], (jstep >> 1) & 1)) {
           report_error(err, MSA_ERR_TIMEOUT, kSiteIndexEpilogue, u, j);
           *abort_flag = 1;
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t ta = lane_base + buf * GP * 128;
+        const uint32_t ta = lane_base + buf * 256;
         uint32_t r0[32], r1[32];
         tmem_ld32(ta, r0);
         tmem_ld32(ta + 32, r1);
@@ -341,7 +344,7 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->acc_empty[buf]);
+        if (lane == 0) mbar_arrive(&ctl->acc_empty[buf][l]);
         m = fmaxf(m, fmaxf(max_of_32(r0), max_of_32(r1)));
         if (m != m) m = -INFINITY;    // a block of NaN scores ranks as -inf
         if (valid && j < lb) list.offer(m, j, k - 1);
