@@ -233,21 +233,22 @@ __global__ void __launch_bounds__(kScanThreads) scan_items_kernel(const int32_t*
 //               issues S = Q K^T, lane 0 of warp 2 issues O = P V (two
 //               issue/commit streams keep the tensor core fed while tile t's
 //               softmax runs);
-//   warps 4-7   softmax + epilogue of even tiles (TMEM slot 0),
-//   warps 8-11  the same for odd tiles (slot 1): S -> P (bf16, written back
-//               into the S columns, the A operand of the PV MMA), then O / l
-//               -> f16 partial and the log-sum-exp of each row.
+//   warps 4-7   softmax of even tiles (TMEM slot 0), warps 8-11 of odd tiles
+//               (slot 1): S -> P (bf16, written back into the S columns, the A
+//               operand of the PV MMA); each row's max and sum go to shared
+//               memory (double-buffered per slot);
+//   warps 12-15 epilogue of every tile in order: O / l -> f16 partial and the
+//               log-sum-exp of each row.
 // A query occupies RQ = max(Hg, 8) tile rows (its Hg heads; with Hg = 4 the
 // box also brings 4 rows of the next heads, which are ignored).
 
-constexpr int kAttnThreads = 384;
+constexpr int kAttnThreads = 512;
 constexpr int kItemRing = 4;
 constexpr int kQSlots = 3;
-constexpr int kItemEmptyCount = 10;   // MMA issuers 2 + softmax warps 8
+constexpr int kItemEmptyCount = 14;   // MMA issuers 2 + softmax warps 8 + epilogue warps 4
 
 struct __align__(16) RingItem {
   int32_t seq, blk, g, start, count, Tb, Sb, qrow0;
-  uint32_t ent[kMaxItemQueries];
 };
 
 struct __align__(16) AttnCtl {
@@ -255,11 +256,13 @@ struct __align__(16) AttnCtl {
   uint64_t kv_full[2], kv_empty[2];
   uint64_t q_full[kQSlots], q_empty[kQSlots];
   uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
+  uint64_t stats_full[2];           // row sums of the slot's current tile are in row_sum
   uint64_t mma_done[2];
   uint32_t tmem_base;
   int32_t abort_flag;
   int32_t pad[2];
   RingItem ring[kItemRing];
+  float row_sum[2][128];            // row sums of the unnormalised probabilities, per slot
 };
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -291,6 +294,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       mbar_init(&ctl->kv_full[i], 1); mbar_init(&ctl->kv_empty[i], 1);
       mbar_init(&ctl->s_full[i], 1); mbar_init(&ctl->p_full[i], 4);
       mbar_init(&ctl->o_full[i], 1); mbar_init(&ctl->o_free[i], 4);
+      mbar_init(&ctl->stats_full[i], 4);
     }
     for (int i = 0; i < kQSlots; ++i) { mbar_init(&ctl->q_full[i], 1); mbar_init(&ctl->q_empty[i], 1); }
     mbar_init(&ctl->mma_done[0], 1);
@@ -351,15 +355,14 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         break;
       }
       const Item I = items[it];
-      for (int j = lane; j < I.count; j += 32) R->ent[j] = entries[I.start + j];
+      // this warp's lanes hold the item's entries (lane j: entries j, j + 32)
+      const uint32_t e0 = lane < I.count ? entries[I.start + lane] : 0u;
+      const uint32_t e1 = lane + 32 < I.count ? entries[I.start + lane + 32] : 0u;
       if (lane == 0) {
         R->seq = I.seq; R->blk = I.blk; R->g = I.g; R->start = I.start; R->count = I.count;
         R->Tb = cu_q[I.seq + 1] - cu_q[I.seq];
         R->Sb = cu_k[I.seq + 1] - cu_k[I.seq];
         R->qrow0 = cu_q[I.seq];
-      }
-      __syncwarp();
-      if (lane == 0) {
         mbar_arrive(&ctl->item_full[slot]);
         // K / V block of this item
         const int st = n & 1;
@@ -373,25 +376,32 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             tma_load_3d(ks + tile_bytes + h * 128 * 128, &tm_v, &ctl->kv_full[st], 64 * h, I.g, krow);
           }
         }
-        // Q rows of each tile
-        const int ntiles = (I.count + qpt - 1) / qpt;
-        for (int mt = 0; ok && mt < ntiles; ++mt, ++tau) {
-          const int qs = tau % kQSlots;
-          if (!(ok = mbar_wait(&ctl->q_empty[qs], ((tau / kQSlots) + 1) & 1))) break;
-          const int nq = min(qpt, I.count - mt * qpt);
-          uint8_t* dst = q_s + qs * tile_bytes;
-          mbar_arrive_expect_tx(&ctl->q_full[qs], nq * RQ * d * 2);
-          for (int ql = 0; ql < nq; ++ql) {
-            const int64_t t = t0 + R->ent[mt * qpt + ql] / k;
-            const int row = (int)(t * H + (int64_t)I.g * Hg);
-            for (int h = 0; h < nhalf; ++h)
-              tma_load_2d(dst + h * 128 * 128 + ql * RQ * 128, &tm_q, &ctl->q_full[qs], 64 * h, row);
-          }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      // Q rows of each tile: lane ql issues the boxes of query ql
+      const int ntiles = (I.count + qpt - 1) / qpt;
+      for (int mt = 0; ok && mt < ntiles; ++mt, ++tau) {
+        const int qs = tau % kQSlots;
+        if (lane == 0) ok = mbar_wait(&ctl->q_empty[qs], ((tau / kQSlots) + 1) & 1);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        const int nq = min(qpt, I.count - mt * qpt);
+        uint8_t* dst = q_s + qs * tile_bytes;
+        if (lane == 0) mbar_arrive_expect_tx(&ctl->q_full[qs], nq * RQ * d * 2);
+        __syncwarp();
+        const int j = mt * qpt + lane;          // entry index of this lane's query
+        const uint32_t ej = __shfl_sync(0xffffffffu, e0, j & 31);
+        const uint32_t ek = __shfl_sync(0xffffffffu, e1, j & 31);
+        if (lane < nq) {
+          const int64_t t = t0 + (j < 32 ? ej : ek) / k;
+          const int row = (int)(t * H + (int64_t)I.g * Hg);
+          for (int h = 0; h < nhalf; ++h)
+            tma_load_2d(dst + h * 128 * 128 + lane * RQ * 128, &tm_q, &ctl->q_full[qs], 64 * h, row);
         }
-        if (!ok) {
-          report_error(err, MSA_ERR_TIMEOUT, kSiteAttnLoad, n, 1);
-          *abort_flag = 1;
-        }
+      }
+      if (lane == 0 && !ok) {
+        report_error(err, MSA_ERR_TIMEOUT, kSiteAttnLoad, n, 1);
+        *abort_flag = 1;
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
@@ -477,14 +487,12 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       umma_commit(&ctl->mma_done[is_s ? 0 : 1]);
       mbar_wait(&ctl->mma_done[is_s ? 0 : 1], 0);
     }
-  } else if (warp >= 4) {
-    // ------------------------------------------------- softmax + epilogue
+  } else if (warp >= 4 && warp < 12) {
+    // ------------------------------------------------------------ softmax
     const int wg = (warp - 4) >> 2;           // slot handled by this warpgroup
     const int wq = warp & 3;                  // TMEM lane quarter
     const int r = 32 * wq + lane;             // tile row
-    const uint32_t lane_off = static_cast<uint32_t>(32 * wq) << 16;
-    const uint32_t s_col = tmem + wg * 256 + lane_off;      // S, then P (first 64 columns)
-    const uint32_t o_col = s_col + 128;                     // O
+    const uint32_t s_col = tmem + wg * 256 + (static_cast<uint32_t>(32 * wq) << 16);   // S, then P
     const int ql = r / RQ, hi = r - ql * RQ;
     int n = 0, tau = 0;
     while (!*abort_flag) {
@@ -492,7 +500,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       if (R == nullptr) break;
       const int count = R->count;
       if (count <= 0) { release_item(n, true); break; }
-      const int g = R->g, Tb = R->Tb, Sb = R->Sb;
+      const int Tb = R->Tb, Sb = R->Sb;
       const int64_t qrow0 = R->qrow0;
       const int64_t blk_first = (int64_t)R->blk * kBk;
       const int ntiles = (count + qpt - 1) / qpt;
@@ -501,7 +509,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         if ((tau & 1) != wg) continue;
         const int idx = mt * qpt + ql;
         const bool valid = ql < qpt && idx < count && hi < Hg;
-        const uint32_t e = valid ? R->ent[idx] : 0u;
+        const uint32_t e = valid ? entries[R->start + idx] : 0u;
         int limit = 127;
         if (valid) {
           const int64_t t = t0 + e / k;
@@ -576,18 +584,54 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->p_full[wg]);
-        // ---- epilogue: O / l -> f16 partial, lse
-        if (!mbar_wait(&ctl->o_full[wg], (tau >> 1) & 1)) {
+        if (valid) {
+          const int64_t unit = ((int64_t)(e / k) * G + R->g) * k + (e % k);
+          part_lse[unit * Hg + hi] = (ms + __log2f(l)) * 0.69314718055994530942f;
+        }
+        // the epilogue of tile tau-2 (same slot) has read row_sum[wg] once o_free fires
+        if (!mbar_wait(&ctl->o_free[wg], ((tau >> 1) + 1) & 1)) {
+          report_error(err, MSA_ERR_TIMEOUT, kSiteAttnSoftmax, tau, 2);
+          *abort_flag = 1;
+          break;
+        }
+        ctl->row_sum[wg][r] = l;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->stats_full[wg]);
+      }
+      release_item(n, true);
+      ++n;
+    }
+  } else if (warp >= 12) {
+    // ----------------------------------------------------------- epilogue
+    const int wq = warp & 3;                  // TMEM lane quarter
+    const int r = 32 * wq + lane;             // tile row
+    const uint32_t lane_off = static_cast<uint32_t>(32 * wq) << 16;
+    const int ql = r / RQ, hi = r - ql * RQ;
+    int n = 0, tau = 0;
+    while (!*abort_flag) {
+      const RingItem* R = wait_item(n);
+      if (R == nullptr) break;
+      const int count = R->count, g = R->g;
+      if (count <= 0) { release_item(n, true); break; }
+      const int ntiles = (count + qpt - 1) / qpt;
+      for (int mt = 0; mt < ntiles; ++mt, ++tau) {
+        const int s = tau & 1;
+        const int idx = mt * qpt + ql;
+        const bool valid = ql < qpt && idx < count && hi < Hg;
+        const uint32_t e = valid ? entries[R->start + idx] : 0u;
+        if (!mbar_wait(&ctl->stats_full[s], (tau >> 1) & 1) || !mbar_wait(&ctl->o_full[s], (tau >> 1) & 1)) {
           report_error(err, MSA_ERR_TIMEOUT, kSiteAttnSoftmax, tau, 1);
           *abort_flag = 1;
           break;
         }
         tc_fence_after();
-        const float inv_l = 1.f / l;
+        const float inv_l = 1.f / ctl->row_sum[s][r];
         const int64_t unit = valid ? ((int64_t)(e / k) * G + g) * k + (e % k) : 0;
         // partial layout per unit: [d/8 chunks][Hg heads][8 values], so the
         // 16 heads of one query write 256 contiguous bytes per chunk
         __half* dst = part_acc + unit * Hg * d + hi * 8;
+        const uint32_t o_col = tmem + s * 256 + 128 + lane_off;
+        uint32_t rr[32];
 #pragma unroll 1
         for (int c4 = 0; c4 < d / 32; ++c4) {
           tmem_ld32(o_col + 32 * c4, rr);
@@ -604,10 +648,9 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             }
           }
         }
-        if (valid) part_lse[unit * Hg + hi] = (ms + __log2f(l)) * 0.69314718055994530942f;
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->o_free[wg]);
+        if (lane == 0) mbar_arrive(&ctl->o_free[s]);
       }
       release_item(n, true);
       ++n;

@@ -127,6 +127,11 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// Non-bulk L2 prefetch of one line (does not go through the TMA engine).
+__device__ __forceinline__ void prefetch_line_l2(const void* p) {
+  asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p) : "memory");
+}
+
 // ------------------------------------------------------ cp.async (gather) ---
 
 __device__ __forceinline__ void cp_async_16(void* dst, const void* src) {
