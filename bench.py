@@ -317,7 +317,14 @@ def run_ours(args):
         dist = dist_mod
     B.build()
     msa.load_library()
+    msa.msa_set_tile_threshold(args.theta)
     peaks, peak_src = load_peaks()
+
+    def tile_theta(w_):
+        if args.theta >= 0:
+            return args.theta
+        uq = 2 * (128 // max(w_.H // w_.G, 8))
+        return (3 * uq + 7) // 8
     w = W.WORKLOADS[args.workload]
     # each rank runs an independent layer (its own seed): weak scaling
     wr = W.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
@@ -348,7 +355,8 @@ def run_ours(args):
     device_errors(ctx, msa)
     launches = msa.msa_profile_read(None)[1]
     kernels = {}
-    for name in ("index_topk_prefill", "sparse_attn", "combine", "count", "scatter", "plan", "block_offsets"):
+    for name in ("index_topk_prefill", "tile_plan", "tile_attn", "sparse_attn", "combine", "count", "scatter",
+                 "plan", "block_offsets"):
         kms, n = msa.msa_profile_read(name)
         if n:
             kernels[name] = {"ms_per_launch": kms / n, "launches": n, "share": None}
@@ -361,18 +369,33 @@ def run_ours(args):
     tokens_all = sum_over_ranks(float(T * args.steps), torch, dist)
     value = tokens_all / (ms_max / 1000.0)
 
-    # roofline of the dominant kernel (timed inside a long step: sustained peak)
-    per_kernel_work = {"sparse_attn": ("tensor", work["main_flops"]),
-                       "index_topk_prefill": ("tensor", work["index_flops"])}
-    dom = max(kernels, key=lambda n: kernels[n]["ms_per_launch"] * kernels[n]["launches"])
-    bound, units = per_kernel_work.get(dom, ("tensor", work["main_flops"]))
+    # algorithmic work of each kernel: the main branch split between the query
+    # tiles and the KV-outer lists as the library's planner splits it
+    split = None if args.index_only else R.tile_split(
+        ctx["sel"], inp["cu_q_host"], inp["cu_k_host"], w.H, w.G, w.d, w.B_k, tile_theta(w), 0)
+    per_kernel_work = {"index_topk_prefill": ("tensor", work["index_flops"])}
+    if split is not None:
+        per_kernel_work.update({"tile_attn": ("tensor", split["tile_flops"]),
+                                "sparse_attn": ("tensor", split["kv_flops"]),
+                                "combine": ("hbm", split["combine_bytes"])})
     peak_t = peaks["bf16_tflops_sustained"]
-    launches_per_step = kernels[dom]["launches"] / args.steps
-    achieved = units / launches_per_step / (kernels[dom]["ms_per_launch"] / 1000.0) / 1e12
-    roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
-            "frac": achieved / peak_t, "traffic": traffic_for(dom),
-            "algorithmic_per_launch": units / launches_per_step,
-            "peak_source": f"bf16_tflops_sustained ({peak_src})"}
+    for name, v in kernels.items():
+        if name in per_kernel_work:
+            bound, units = per_kernel_work[name]
+            per = units / (v["launches"] / args.steps)
+            v["algorithmic_per_launch"] = per
+            v["achieved"] = per / (v["ms_per_launch"] / 1000.0) / (1e12 if bound == "tensor" else 1e9)
+            v["frac"] = v["achieved"] / (peak_t if bound == "tensor" else peaks["hbm_gbs"])
+    # roofline of the dominant kernel (timed inside a long step: sustained peak)
+    dom = max((n for n in kernels if n in per_kernel_work),
+              key=lambda n: kernels[n]["ms_per_launch"] * kernels[n]["launches"])
+    bound = per_kernel_work[dom][0]
+    roof = {"kernel": dom, "bound": bound, "achieved": kernels[dom]["achieved"],
+            "peak": peak_t if bound == "tensor" else peaks["hbm_gbs"],
+            "unit": "TFLOP/s" if bound == "tensor" else "GB/s", "frac": kernels[dom]["frac"],
+            "traffic": traffic_for(dom), "algorithmic_per_launch": kernels[dom]["algorithmic_per_launch"],
+            "peak_source": (f"bf16_tflops_sustained ({peak_src})" if bound == "tensor"
+                            else f"hbm_gbs ({peak_src})")}
     t_roof_ms = max(work["flops"] / (peaks["bf16_tflops"] * 1e12), work["bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3
     t_roof_sus = max(work["flops"] / (peak_t * 1e12), work["bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3
     step_roof = {"flops": work["flops"], "index_flops": work["index_flops"], "main_flops": work["main_flops"],
@@ -403,6 +426,34 @@ def run_ours(args):
         e2e = {"value": sum_over_ranks(float(T * e_steps), torch, dist) / (ms_e / 1000.0), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e / e_steps}
         del host, dev, host_out
+
+    # dense causal GQA on the same q / k / v: the denominator of the speedup ratio
+    dense = None
+    if rank == 0 and not args.no_dense and not args.index_only:
+        dws = torch.empty(msa.load_library().msa_dense_attn_workspace_size(
+            __import__("ctypes").byref(ctx["shape"]), __import__("ctypes").byref(ctx["seqs"])),
+            dtype=torch.uint8, device=inp["q"].device)
+
+        def dense_step():
+            msa.msa_dense_attn(ctx["shape"], ctx["seqs"], inp["q"], inp["k"], inp["v"], out=ctx["out"], ws=dws,
+                               check=False)
+
+        dense_step()
+        torch.cuda.synchronize()
+        code = msa.msa_get_device_error(dws)[0]
+        if code != 0:
+            raise RuntimeError(f"dense attention device error {code}")
+        d_steps = 2
+        dms = time_steps(dense_step, d_steps, torch) / d_steps
+        dfl = R.dense_work(S_lens, T_lens, w.H, w.d)
+        main_ms = sum(kernels[n]["ms_per_launch"] * kernels[n]["launches"] for n in kernels
+                      if n != "index_topk_prefill") / args.steps
+        dense = {"workload": args.workload, "ms": dms, "flops": dfl,
+                 "achieved_tflops": dfl / (dms / 1000.0) / 1e12,
+                 "frac": dfl / (dms / 1000.0) / 1e12 / peak_t,
+                 "speedup_step": dms / ms_step, "speedup_main_branch": dms / main_ms,
+                 "flops_ratio": dfl / work["main_flops"]}
+        del dws
 
     # decode: 32 sequences with caches of 128K..1M tokens
     decode = None
@@ -457,7 +508,8 @@ def run_ours(args):
                            "B_k": w.B_k, "k": w.k, "hot_block_frac": w.hot_frac,
                            "l2": "inputs larger than L2 (q alone is %.1f GB)" % (inp["q"].numel() * 2 / 1e9),
                            "parallelism": f"independent layer per GPU x{world}"},
-                "roofline": roof, "step_roofline": step_roof, "decode": decode, "e2e": e2e,
+                "roofline": roof, "step_roofline": step_roof, "tile_split": split, "dense_gqa": dense,
+                "decode": decode, "e2e": e2e,
                 "cpu_baseline": cpu, "clocks": clk, "gpu_launches": launches, "kernels": kernels}
         print(json.dumps(line), flush=True)
     if dist is not None:
@@ -477,6 +529,9 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense causal GQA comparison")
+    ap.add_argument("--theta", type=int, default=-1,
+                    help="query-tile threshold of the prefill (-1 automatic, 0 off)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=64)
     args = ap.parse_args()

@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "msa_internal.h"
@@ -11,6 +12,9 @@
 using namespace msa;
 
 namespace {
+
+// Query-tile threshold (msa_set_tile_threshold): -1 automatic, 0 off.
+std::atomic<int> g_tile_theta{-1};
 
 constexpr size_t kAlign = 256;
 
@@ -49,7 +53,8 @@ int64_t total_blocks_bound(const msa_varlen_t* v) { return (v->total_k + kBk - 1
 
 // Slices of a sparse-attention workspace for chunks of `rows` query rows.
 struct AttnLayout {
-  size_t blk_off, counts, cursor, tile_sums, nitems, entries, items, part_acc, part_lse, total;
+  size_t blk_off, counts, cursor, tile_sums, nitems, entries, items, part_acc, part_lse;
+  size_t unit_blk, unit_nblk, unit_list, dmask, dstate, dmember, clist, tile_ctr, total;
   int64_t nlists, max_items;
   int32_t qpi;
 };
@@ -78,8 +83,25 @@ AttnLayout attn_layout(const msa_shape_t* s, const msa_varlen_t* v, int64_t rows
   L.items = take(sizeof(Item) * L.max_items);
   L.part_acc = take((size_t)nentries * hg * s->d * 2);
   L.part_lse = take((size_t)nentries * hg * 4);
+  const int UQ = tile_queries(s->H, s->G);
+  const int64_t nunits = ((rows + UQ - 1) / UQ) * s->G;
+  L.unit_blk = take(sizeof(int32_t) * nunits * kMaxDense);
+  L.unit_nblk = take(sizeof(int32_t) * nunits);
+  L.unit_list = take(sizeof(int32_t) * nunits);
+  L.dmask = take(sizeof(uint32_t) * rows * s->G);
+  L.dstate = take(sizeof(int32_t) * rows * s->G);
+  L.dmember = take(sizeof(uint64_t) * rows * s->G);
+  L.clist = take(sizeof(uint2) * rows * s->G);
+  L.tile_ctr = take(sizeof(int32_t) * 4);
   L.total = off;
   return L;
+}
+
+// Threshold for this call: the query tiles need several queries per sequence.
+int tile_theta(const msa_shape_t* s, const msa_varlen_t* v) {
+  const int set = g_tile_theta.load(std::memory_order_relaxed);
+  if (set == 0 || v->max_q_len <= 1) return 0;
+  return set < 0 ? tile_default_theta(tile_queries(s->H, s->G)) : set;
 }
 
 int64_t chunk_rows(const msa_varlen_t* v, int64_t q_chunk) {
@@ -122,6 +144,15 @@ msa_status_t attn_common(const msa_shape_t* shape, const msa_varlen_t* seqs, con
   a.part_acc = base + L.part_acc;
   a.part_lse = reinterpret_cast<float*>(base + L.part_lse);
   a.queries_per_item = L.qpi;
+  a.theta = tile_theta(shape, seqs);
+  a.unit_blk = reinterpret_cast<int32_t*>(base + L.unit_blk);
+  a.unit_nblk = reinterpret_cast<int32_t*>(base + L.unit_nblk);
+  a.unit_list = reinterpret_cast<int32_t*>(base + L.unit_list);
+  a.dmask = reinterpret_cast<uint32_t*>(base + L.dmask);
+  a.dstate = reinterpret_cast<int32_t*>(base + L.dstate);
+  a.dmember = reinterpret_cast<uint64_t*>(base + L.dmember);
+  a.clist = reinterpret_cast<uint2*>(base + L.clist);
+  a.tile_ctr = reinterpret_cast<int32_t*>(base + L.tile_ctr);
   for (int64_t t0 = 0; t0 < seqs->total_q; t0 += rows) {
     a.t0 = t0;
     a.t1 = t0 + rows < seqs->total_q ? t0 + rows : seqs->total_q;
@@ -234,6 +265,8 @@ msa_status_t msa_combine(const msa_shape_t* shape, int64_t T, const void* part_a
   msa_status_t st = check_shape(shape);
   if (st != MSA_OK) return st;
   if (T < 0 || !part_acc || !part_lse || !sel || !out) return MSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(part_acc) | reinterpret_cast<uintptr_t>(part_lse)) & 15u)
+    return MSA_ERR_INVALID_ARG;   // streamed with 16-byte bulk copies
   if (T == 0) return MSA_OK;
   return launch_combine(part_acc, part_lse, sel, out, lse, T, shape->H, shape->G, shape->d, shape->k, stream) == 0
              ? MSA_OK
@@ -242,7 +275,7 @@ msa_status_t msa_combine(const msa_shape_t* shape, int64_t T, const void* part_a
 
 size_t msa_dense_attn_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs) {
   if (check_shape(shape) != MSA_OK || check_seqs(seqs) != MSA_OK) return 0;
-  return kWsHeader;
+  return kWsHeader + dense_scratch_bytes(seqs->batch);
 }
 
 msa_status_t msa_dense_attn(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q, const void* k,
@@ -252,20 +285,25 @@ msa_status_t msa_dense_attn(const msa_shape_t* shape, const msa_varlen_t* seqs, 
   st = check_seqs(seqs);
   if (st != MSA_OK) return st;
   if (!q || !k || !v || !out) return MSA_ERR_INVALID_ARG;
-  if (!ws_ok(ws, ws_bytes, kWsHeader)) return MSA_ERR_WORKSPACE;
+  if (!ws_ok(ws, ws_bytes, msa_dense_attn_workspace_size(shape, seqs))) return MSA_ERR_WORKSPACE;
   if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MSA_ERR_CUDA;
   if (seqs->total_q == 0) return MSA_OK;
   DenseArgs a{};
+  a.scratch = static_cast<uint8_t*>(ws) + kWsHeader;
   a.q = q; a.key = k; a.value = v; a.out = out; a.lse = lse;
   a.cu_q = seqs->cu_q; a.cu_k = seqs->cu_k;
   a.batch = seqs->batch; a.H = shape->H; a.G = shape->G; a.d = shape->d; a.sm_scale = shape->sm_scale;
   a.total_q = seqs->total_q; a.total_k = seqs->total_k;
   a.max_q_len = seqs->max_q_len; a.max_k_len = seqs->max_k_len;
   a.err = static_cast<DevError*>(ws);
-  const int rc = launch_dense_attn(a, stream);
-  if (rc == (int)cudaErrorNotSupported) return MSA_ERR_UNSUPPORTED;
-  return rc == 0 ? MSA_OK : MSA_ERR_CUDA;
+  return launch_dense_attn(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
+}
+
+int32_t msa_set_tile_threshold(int32_t theta) {
+  const int32_t prev = g_tile_theta.load();
+  g_tile_theta.store(theta < 0 ? -1 : theta);
+  return prev;
 }
 
 msa_status_t msa_get_device_error(void* ws, int32_t* code, int32_t* where, int32_t* info0, int32_t* info1,

@@ -63,12 +63,15 @@ __device__ __forceinline__ int entry_list(int blk, int64_t t, int g, int G, int 
 // items come out window-major (the queries of one window stay hot in L2).
 // kScatter == false counts, == true claims positions from `counter`
 // (the cursors) and writes the entries (t - t0) * k + slot.
+// Slots whose bit is set in dmask (when given) were attended by a query tile
+// and get no list entry; they are still validated.  With clist (no query
+// tiles), the counting pass also writes every pair's combine-list entry.
 template <bool kScatter>
 __global__ void count_scatter_kernel(const int32_t* __restrict__ sel, int64_t t0, int64_t t1, int G, int k,
                                      int batch, const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_k,
                                      const int32_t* __restrict__ blk_off, int64_t nlists,
-                                     int32_t* __restrict__ counter, uint32_t* __restrict__ entries,
-                                     DevError* err) {
+                                     const uint32_t* __restrict__ dmask, int32_t* __restrict__ counter,
+                                     uint32_t* __restrict__ entries, uint2* __restrict__ clist, DevError* err) {
   const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t n = (t1 - t0) * G;
   const bool active = gid < n;
@@ -77,11 +80,15 @@ __global__ void count_scatter_kernel(const int32_t* __restrict__ sel, int64_t t0
   const int g = active ? (int)(gid % G) : 0;
   const int64_t wbase = (tl / kWindow) * nlists;
   const int lane = threadIdx.x & 31;
+  const uint32_t covered = (active && dmask != nullptr) ? dmask[gid] : 0u;
+  uint32_t live = 0;
   for (int s = 0; s < k; ++s) {
     int64_t key = -1;
     if (active) {
-      const int L = entry_list(sel[(t * G + g) * k + s], t, g, G, batch, cu_q, cu_k, blk_off, err);
-      if (L >= 0) key = wbase + L;
+      const int32_t blk = sel[(t * G + g) * k + s];
+      if (blk >= 0) live |= 1u << s;
+      const int L = entry_list(blk, t, g, G, batch, cu_q, cu_k, blk_off, err);
+      if (L >= 0 && !((covered >> s) & 1u)) key = wbase + L;
     }
     // warp-aggregated atomics: lanes with the same key share one atomic
     const unsigned peers = __match_any_sync(0xffffffffu, key);
@@ -92,6 +99,7 @@ __global__ void count_scatter_kernel(const int32_t* __restrict__ sel, int64_t t0
     base = __shfl_sync(0xffffffffu, base, leader);
     if (kScatter && key >= 0) entries[base + rank] = (uint32_t)(tl * k + s);
   }
+  if (!kScatter && clist != nullptr && active) clist[gid] = make_uint2((uint32_t)gid, live);
 }
 
 // Device-wide exclusive scan of the list counts (and of their item counts,
@@ -668,77 +676,180 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 
 // -------------------------------------------------------------- combine ---
 
-// One thread per (query, group, 8-column chunk c, head i) with i fastest, so a
-// warp's loads of one partial are contiguous (layout per unit: [d/8][Hg][8]).
-// Every load of a thread (selection, log-sum-exps, partials) is issued before
-// any is used; empty slots (sel < 0) are masked afterwards.
-template <int KMAX>
-__global__ void __launch_bounds__(256) combine_kernel(const __half* __restrict__ part_acc,
-                                                      const float* __restrict__ part_lse,
-                                                      const int32_t* __restrict__ sel, __nv_bfloat16* __restrict__ out,
-                                                      float* __restrict__ lse_out, int64_t T, int H, int G, int d,
-                                                      int k) {
+// Persistent combine: the partials of one (query, group) are one contiguous
+// run (k slots x [d/8][Hg][8] f16, 4 KB per slot at Hg = 16, d = 128), and
+// its k x Hg log-sum-exps another.  Thread 0 streams the slots to merge of P
+// (query, group) pairs into an nst-stage shared-memory ring with bulk async
+// copies; thread (pair, c, i) merges output columns 8c..8c+7 of head i from
+// shared memory (consecutive threads read consecutive 16-byte words: no bank
+// conflicts).  A pair spans Hg * d/8 threads, a multiple of 32.
+//   clist given: entry {pair, slot mask} per merged pair; only the slots in
+//                the mask are copied (the query tiles leave most slots empty);
+//   clist null : every pair, slots with sel >= 0 (each warp reads its pair's
+//                selection with one load per lane), whole runs copied.
+constexpr int kCombThreads = 256;
+constexpr int kCombMaxStages = 3;
+constexpr int kCombMaxPairs = 8;
+
+__global__ void __launch_bounds__(kCombThreads, 1)
+combine_kernel(const __half* __restrict__ part_acc, const float* __restrict__ part_lse,
+               const int32_t* __restrict__ sel, const uint2* __restrict__ clist,
+               const int32_t* __restrict__ npairs_dev, __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out,
+               int64_t T, int H, int G, int d, int k, int P, int nst, uint32_t acc_bytes, uint32_t lse_bytes,
+               uint32_t stage_bytes, DevError* err) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 127u) & ~127u) - raw);
+  __shared__ uint64_t full[kCombMaxStages];
   const int Hg = H / G;
-  const int per = Hg * (d / 8);                // threads per (query, group)
-  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t tg = gid / per;
-  if (tg >= T * G) return;
-  const int rem = (int)(gid - tg * per);
-  const int c = rem / Hg, i = rem - c * Hg;
-  const int64_t t = tg / G;
-  const int g = (int)(tg - t * G);
-  const int32_t* srow = sel + tg * k;
-  const int64_t ubase = tg * k;
-  int sv[KMAX];
-  float ls[KMAX];
-  uint4 raw[KMAX];
+  const int per = Hg * (d / 8);                 // threads per (query, group)
+  const uint32_t slot_bytes = acc_bytes / k;
+  const int64_t npairs = npairs_dev != nullptr ? (int64_t)*npairs_dev : T * G;
+  const int64_t nchunks = (npairs + P - 1) / P;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nst; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // the n-th chunk of this CTA is chunk blockIdx.x + n * gridDim.x
+  const int64_t my = blockIdx.x < nchunks ? (nchunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  // thread 0: list entries of a chunk (fetched one iteration before they are used)
+  uint2 ent[kCombMaxPairs];
+  auto fetch = [&](int64_t n) {
+    const int64_t p0 = (blockIdx.x + n * gridDim.x) * P;
 #pragma unroll
-  for (int s = 0; s < KMAX; ++s) {
-    if (s < k) {
-      sv[s] = __ldg(srow + s);
-      ls[s] = __ldg(part_lse + (ubase + s) * Hg + i);
-      raw[s] = __ldg(reinterpret_cast<const uint4*>(part_acc + ((ubase + s) * (d / 8) + c) * Hg * 8 + i * 8));
+    for (int i = 0; i < kCombMaxPairs; ++i)
+      if (i < P && p0 + i < npairs) ent[i] = clist != nullptr ? clist[p0 + i] : make_uint2((uint32_t)(p0 + i), ~0u);
+  };
+  auto issue = [&](int64_t n) {
+    const int stage = (int)(n % nst);
+    const int64_t p0 = (blockIdx.x + n * gridDim.x) * P;
+    const int64_t left = npairs - p0;
+    const int np = left < P ? (int)left : P;
+    uint8_t* dst = smem + stage * stage_bytes;
+    uint32_t bytes = 0;
+#pragma unroll
+    for (int i = 0; i < kCombMaxPairs; ++i)
+      if (i < np) bytes += (clist != nullptr ? __popc(ent[i].y) * slot_bytes : acc_bytes) + lse_bytes;
+    mbar_arrive_expect_tx(&full[stage], bytes);
+#pragma unroll
+    for (int i = 0; i < kCombMaxPairs; ++i) {
+      if (i >= np) continue;
+      const uint8_t* src = reinterpret_cast<const uint8_t*>(part_acc) + (int64_t)ent[i].x * acc_bytes;
+      if (clist != nullptr) {
+        for (uint32_t m = ent[i].y; m != 0u; m &= m - 1u) {
+          const int s2 = __ffs(m) - 1;
+          bulk_load(dst + i * acc_bytes + s2 * slot_bytes, src + s2 * slot_bytes, slot_bytes, &full[stage]);
+        }
+      } else {
+        bulk_load(dst + i * acc_bytes, src, acc_bytes, &full[stage]);
+      }
+      bulk_load(dst + P * acc_bytes + i * lse_bytes,
+                reinterpret_cast<const uint8_t*>(part_lse) + (int64_t)ent[i].x * lse_bytes, lse_bytes, &full[stage]);
+    }
+  };
+  if (threadIdx.x == 0)
+    for (int64_t n = 0; n < nst && n < my; ++n) {
+      fetch(n);
+      issue(n);
+    }
+  const int lane = threadIdx.x & 31;
+  const int pl = threadIdx.x / per;             // pair within the chunk (P * per == kCombThreads)
+  const int rem = threadIdx.x - pl * per;
+  const int cc = rem / Hg, i = rem - cc * Hg;
+  int64_t n = 0;
+  for (; n < my; ++n) {
+    const int stage = (int)(n % nst);
+    const int64_t idx = (blockIdx.x + n * gridDim.x) * P + pl;
+    const bool live = idx < npairs;
+    if (threadIdx.x == 0 && n + nst < my) fetch(n + nst);
+    int64_t pair = idx;
+    uint32_t valid;
+    if (clist != nullptr) {
+      const uint2 e = live ? clist[idx] : make_uint2(0u, 0u);
+      pair = e.x;
+      valid = e.y;
     } else {
-      sv[s] = -1;
+      const int32_t sv = (lane < k && live) ? __ldg(sel + pair * k + lane) : -1;
+      valid = __ballot_sync(0xffffffffu, sv >= 0);
     }
-  }
-  float m = -INFINITY;
-#pragma unroll
-  for (int s = 0; s < KMAX; ++s)
-    if (sv[s] >= 0) m = fmaxf(m, ls[s]);
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  float wsum = 0.f;
-#pragma unroll
-  for (int s = 0; s < KMAX; ++s) {
-    if (sv[s] < 0) continue;
-    const float w = __expf(ls[s] - m);
-    wsum += w;
-    const __half2* hp = reinterpret_cast<const __half2*>(&raw[s]);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = __half22float2(hp[j]);
-      acc[2 * j] = fmaf(w, f.x, acc[2 * j]);
-      acc[2 * j + 1] = fmaf(w, f.y, acc[2 * j + 1]);
+    const bool ok = mbar_wait(&full[stage], (uint32_t)((n / nst) & 1));
+    if (__syncthreads_or(!ok)) {
+      if (threadIdx.x == 0) report_error(err, MSA_ERR_TIMEOUT, kSiteAttnLoad, (int)n, -2);
+      break;
     }
+    if (live) {
+      const uint8_t* base = smem + stage * stage_bytes;
+      const __half* acc_s = reinterpret_cast<const __half*>(base + pl * acc_bytes);
+      const float* lse_s = reinterpret_cast<const float*>(base + P * acc_bytes + pl * lse_bytes);
+      float m = -INFINITY;
+      for (int s2 = 0; s2 < k; ++s2)
+        if ((valid >> s2) & 1u) m = fmaxf(m, lse_s[s2 * Hg + i]);
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float wsum = 0.f;
+      for (int s2 = 0; s2 < k; ++s2) {
+        if (!((valid >> s2) & 1u)) continue;
+        const float w = __expf(lse_s[s2 * Hg + i] - m);
+        wsum += w;
+        const uint4 rv = *reinterpret_cast<const uint4*>(acc_s + ((s2 * (d / 8) + cc) * Hg + i) * 8);
+        const __half2* hp = reinterpret_cast<const __half2*>(&rv);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __half22float2(hp[j]);
+          acc[2 * j] = fmaf(w, f.x, acc[2 * j]);
+          acc[2 * j + 1] = fmaf(w, f.y, acc[2 * j + 1]);
+        }
+      }
+      const float inv = 1.f / wsum;
+      uint4 o;
+      o.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+      o.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+      o.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+      o.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+      const int64_t t = pair / G;
+      const int h = (int)(pair - t * G) * Hg + i;
+      *reinterpret_cast<uint4*>(out + (t * H + h) * d + 8 * cc) = o;
+      if (lse_out != nullptr && cc == 0) lse_out[t * H + h] = m + __logf(wsum);
+    }
+    __syncthreads();                            // stage consumed by every thread
+    if (threadIdx.x == 0 && n + nst < my) issue(n + nst);
   }
-  const float inv = 1.f / wsum;
-  uint4 o;
-  o.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-  o.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-  o.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
-  o.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
-  const int h = g * Hg + i;
-  *reinterpret_cast<uint4*>(out + (t * H + h) * d + 8 * c) = o;
-  if (lse_out != nullptr && c == 0) lse_out[t * H + h] = m + __logf(wsum);
+  // after a timeout no bulk copy may still be writing when the CTA exits
+  if (threadIdx.x == 0 && n < my) {
+    const int64_t last = my < n + nst ? my : n + nst;
+    for (int64_t m2 = n; m2 < last; ++m2) mbar_wait(&full[m2 % nst], (uint32_t)((m2 / nst) & 1));
+  }
 }
 
-int launch_combine_kernel(const __half* part_acc, const float* part_lse, const int32_t* sel, __nv_bfloat16* out,
-                          float* lse, int64_t T, int H, int G, int d, int k, cudaStream_t st) {
-  const int64_t cthreads = T * H * (d / 8);   // = T * G * Hg * d/8
-  const unsigned blocks = (unsigned)((cthreads + 255) / 256);
-  if (k <= 8) combine_kernel<8><<<blocks, 256, 0, st>>>(part_acc, part_lse, sel, out, lse, T, H, G, d, k);
-  else if (k <= 16) combine_kernel<16><<<blocks, 256, 0, st>>>(part_acc, part_lse, sel, out, lse, T, H, G, d, k);
-  else combine_kernel<32><<<blocks, 256, 0, st>>>(part_acc, part_lse, sel, out, lse, T, H, G, d, k);
+int launch_combine_kernel(const __half* part_acc, const float* part_lse, const int32_t* sel, const uint2* clist,
+                          const int32_t* npairs_dev, __nv_bfloat16* out, float* lse, int64_t T, int H, int G, int d,
+                          int k, DevError* err, cudaStream_t st) {
+  if (T <= 0) return 0;
+  const int Hg = H / G;
+  const int per = Hg * (d / 8);
+  if (per % 32 != 0 || kCombThreads % per != 0 || k > 32) return (int)cudaErrorInvalidValue;
+  const int P = kCombThreads / per;
+  if (P > kCombMaxPairs) return (int)cudaErrorInvalidValue;
+  const uint32_t acc_bytes = (uint32_t)k * Hg * d * 2;
+  const uint32_t lse_bytes = (uint32_t)k * Hg * 4;
+  // bulk copies need 16-byte sizes and addresses
+  if (((acc_bytes | lse_bytes) & 15u) || ((reinterpret_cast<uintptr_t>(part_acc) |
+                                           reinterpret_cast<uintptr_t>(part_lse)) & 15u))
+    return (int)cudaErrorInvalidValue;
+  const uint32_t stage_bytes = (P * (acc_bytes + lse_bytes) + 127u) & ~127u;
+  const size_t avail = 227 * 1024 - 128 - 64;
+  const int nst = (int)(avail / stage_bytes < kCombMaxStages ? avail / stage_bytes : kCombMaxStages);
+  if (nst < 1) return (int)cudaErrorInvalidValue;
+  const size_t smem = 128 + (size_t)nst * stage_bytes;
+  cudaError_t e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return (int)e;
+  int dev = 0, nsm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t nchunks = (T * G + P - 1) / P;   // upper bound when a pair list is given
+  const int grid = (int)(nchunks < nsm ? nchunks : nsm);
+  combine_kernel<<<grid, kCombThreads, smem, st>>>(part_acc, part_lse, sel, clist, npairs_dev, out, lse, T, H, G, d,
+                                                  k, P, nst, acc_bytes, lse_bytes, stage_bytes, err);
   return (int)cudaGetLastError();
 }
 
@@ -759,12 +870,21 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
   const int64_t nkeys = nwin * a.nlists;
   e = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * nkeys, st);
   if (e != cudaSuccess) return (int)e;
+  const bool tiles = a.theta > 0;
+  if (tiles) {
+    e = cudaMemsetAsync(a.tile_ctr, 0, sizeof(int32_t) * 4, st);
+    if (e != cudaSuccess) return (int)e;
+    const int rc = launch_tile_plan(a, a.theta, stream);
+    if (rc) return rc;
+  }
+  const uint32_t* dmask = tiles ? a.dmask : nullptr;
   const int64_t nthreads = nrows * a.G;
   const int cs_blocks = (int)((nthreads + 255) / 256);
   {
     ProfScope p("count", stream);
     count_scatter_kernel<false><<<cs_blocks, 256, 0, st>>>(a.sel, a.t0, a.t1, a.G, a.k, a.batch, a.cu_q, a.cu_k,
-                                                           a.blk_off, a.nlists, a.counts, nullptr, a.err);
+                                                           a.blk_off, a.nlists, dmask, a.counts, nullptr,
+                                                           tiles ? nullptr : a.clist, a.err);
   }
   const int ntiles = (int)((nkeys + kScanTile - 1) / kScanTile);
   {
@@ -778,7 +898,8 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
   {
     ProfScope p("scatter", stream);
     count_scatter_kernel<true><<<cs_blocks, 256, 0, st>>>(a.sel, a.t0, a.t1, a.G, a.k, a.batch, a.cu_q, a.cu_k,
-                                                          a.blk_off, a.nlists, a.cursor, a.entries, a.err);
+                                                          a.blk_off, a.nlists, dmask, a.cursor, a.entries, nullptr,
+                                                          a.err);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
@@ -817,11 +938,16 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
+  if (tiles) {
+    const int rc = launch_tile_attn(a, stream);
+    if (rc) return rc;
+  }
   const int64_t rows = a.t1 - a.t0;
   ProfScope p("combine", stream);
   return launch_combine_kernel(reinterpret_cast<const __half*>(a.part_acc), a.part_lse, a.sel + a.t0 * a.G * a.k,
+                               a.clist, tiles ? a.tile_ctr : nullptr,
                                reinterpret_cast<__nv_bfloat16*>(a.out) + a.t0 * a.H * a.d,
-                               a.lse ? a.lse + a.t0 * a.H : nullptr, rows, a.H, a.G, a.d, a.k, st);
+                               a.lse ? a.lse + a.t0 * a.H : nullptr, rows, a.H, a.G, a.d, a.k, a.err, st);
 }
 
 int launch_combine(const void* part_acc, const float* part_lse, const int32_t* sel, void* out, float* lse,
@@ -829,8 +955,8 @@ int launch_combine(const void* part_acc, const float* part_lse, const int32_t* s
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (T <= 0) return 0;
   ProfScope p("combine", stream);
-  return launch_combine_kernel(reinterpret_cast<const __half*>(part_acc), part_lse, sel,
-                               reinterpret_cast<__nv_bfloat16*>(out), lse, T, H, G, d, k, st);
+  return launch_combine_kernel(reinterpret_cast<const __half*>(part_acc), part_lse, sel, nullptr, nullptr,
+                               reinterpret_cast<__nv_bfloat16*>(out), lse, T, H, G, d, k, nullptr, st);
 }
 
 }  // namespace msa

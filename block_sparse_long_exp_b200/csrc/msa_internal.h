@@ -3,6 +3,7 @@
 
 #include <stddef.h>
 #include <stdint.h>
+#include <vector_types.h>
 
 #include "../../include/msa.h"
 
@@ -14,6 +15,8 @@ constexpr int kMaxBatchTiles = 1024;  // sequences per prefill index launch
 constexpr int kWindow = 1024;         // query rows per attention planning window
 constexpr int kScanTile = 4096;       // keys per CTA of the planning scan
 constexpr int kMaxItemQueries = 64;   // queries per attention work item (upper bound)
+constexpr int kMaxDense = 64;         // dense blocks per query tile (Q-outer side)
+constexpr int32_t kDenseComplete = 0x100;   // dstate flag: the tile covers every selection of the query
 
 // Device error word, at offset 0 of every workspace.
 struct DevError {
@@ -36,6 +39,10 @@ enum ErrorSite : int32_t {
   kSiteAttnSoftmax = 133,
   kSiteAttnItem = 134,
   kSiteDense = 141,
+  kSiteTileUnit = 151,
+  kSiteTileLoad = 152,
+  kSiteTileMma = 153,
+  kSiteTileSoftmax = 154,
 };
 
 // One KV-outer work item: up to `count` queries of the list of
@@ -99,13 +106,27 @@ struct AttnArgs {
   int64_t max_items;
   int32_t* blk_off;    // [batch + 1] block offsets per sequence
   int64_t nlists;      // G * total blocks
-  void* part_acc;      // f16 [(t1-t0), G, k, Hg, d]
+  void* part_acc;      // f16 [(t1-t0), G, k, d/8, Hg, 8]
   float* part_lse;     // [(t1-t0), G, k, Hg]
   int32_t queries_per_item;
+  // query-tile (Q-outer) side; theta == 0 turns it off
+  int32_t theta;       // a block is a tile's dense block when >= theta of its queries chose it
+  int32_t* unit_blk;   // [units x G][kMaxDense]
+  int32_t* unit_nblk;  // [units x G]
+  int32_t* unit_list;  // [units x G] units with dense blocks
+  uint32_t* dmask;     // [(t1-t0) x G] slots covered by the tile
+  int32_t* dstate;     // [(t1-t0) x G] first covered slot | kDenseComplete, or -1
+  uint64_t* dmember;   // [(t1-t0) x G] positions of the covered blocks in the tile's list
+  uint2* clist;        // [(t1-t0) x G] combine list: {pair (t - t0) * G + g, slots to merge}
+  int32_t* tile_ctr;   // [4]: pairs, listed units, unit ticket
 };
 int launch_sparse_attn_pass(const AttnArgs& a, void* stream);
 int launch_combine(const void* part_acc, const float* part_lse, const int32_t* sel, void* out,
                    float* lse, int64_t T, int32_t H, int32_t G, int32_t d, int32_t k, void* stream);
+int tile_queries(int H, int G);        // query rows per tile unit
+int tile_default_theta(int UQ);
+int launch_tile_plan(const AttnArgs& a, int theta, void* stream);
+int launch_tile_attn(const AttnArgs& a, void* stream);
 
 struct DenseArgs {
   const void* q;
@@ -120,7 +141,9 @@ struct DenseArgs {
   int64_t total_q, total_k;
   int32_t max_q_len, max_k_len;
   DevError* err;
+  void* scratch;       // dense_scratch_bytes(batch)
 };
+size_t dense_scratch_bytes(int32_t batch);
 int launch_dense_attn(const DenseArgs& a, void* stream);
 
 // Launch accounting: a ProfScope wraps one kernel launch; it always counts the

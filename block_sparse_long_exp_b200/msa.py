@@ -27,7 +27,7 @@ EXPORTED = [
     "msa_combine", "msa_dense_attn_workspace_size", "msa_dense_attn",
     "msa_index_topk_decode_noalloc_max_scratch", "msa_index_topk_decode_noalloc",
     "msa_profile_enable", "msa_profile_reset", "msa_profile_read",
-    "msa_get_device_error", "msa_version",
+    "msa_get_device_error", "msa_version", "msa_set_tile_threshold",
 ]
 
 
@@ -92,6 +92,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_profile_read.restype = i32
     lib.msa_version.argtypes = []
     lib.msa_version.restype = ctypes.c_char_p
+    lib.msa_set_tile_threshold.argtypes = [i32]
+    lib.msa_set_tile_threshold.restype = i32
     _lib = lib
     return lib
 
@@ -243,7 +245,8 @@ def msa_combine(shape: Shape, T: int, part_acc: torch.Tensor, part_lse: torch.Te
 def msa_dense_attn(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                    out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                    want_lse: bool = False, ws: Optional[torch.Tensor] = None,
-                   stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+                   stream=None, check: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Dense causal GQA attention (every key at or before the query position)."""
     lib = load_library()
     _require_cuda(q)
     T = seqs.total_q
@@ -257,7 +260,8 @@ def msa_dense_attn(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.Tensor,
     rc = lib.msa_dense_attn(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
                             _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
     _check(rc, "msa_dense_attn")
-    _device_check(ws, stream, "msa_dense_attn")
+    if check:
+        _device_check(ws, stream, "msa_dense_attn")
     return out, lse
 
 
@@ -290,6 +294,12 @@ def msa_profile_read(kernel: Optional[str]) -> Tuple[float, int]:
     rc = load_library().msa_profile_read(kernel.encode() if kernel else None, ctypes.byref(ms), ctypes.byref(n))
     _check(rc, "msa_profile_read")
     return ms.value, n.value
+
+
+def msa_set_tile_threshold(theta: int) -> int:
+    """Query-tile threshold of the prefill main branch (-1 automatic, 0 off);
+    returns the previous value."""
+    return int(load_library().msa_set_tile_threshold(int(theta)))
 
 
 def msa_version() -> str:

@@ -91,3 +91,71 @@ def decode_work(L_lens: Sequence[int], H: int, G: int, d: int, d_idx: int, B_k: 
         min(L, (min(k, (L - 1) // B_k + 1) - 1) * B_k + ((L - 1) % B_k) + 1) for L in L_lens)
     return {"bytes": float(idx_bytes + kv_bytes + small), "index_bytes": float(idx_bytes),
             "kv_bytes": float(kv_bytes), "flops": float(flops)}
+
+
+def tile_split(sel, cu_q_host: Sequence[int], cu_k_host: Sequence[int], H: int, G: int, d: int, B_k: int,
+               theta: int, q_chunk: int = 0) -> Dict[str, float]:
+    """Algorithmic work of each main-branch kernel for one prefill call.
+
+    Re-derives, with torch ops on the selection `sel` [T, G, k] (device or
+    host), which selections the query tiles cover: a tile is UQ = 2 x 128 /
+    max(H/G, 8) consecutive rows of one pass that lie in one sequence, and a
+    block chosen by >= theta of its queries (for one group) is covered.
+    Returns the FLOPs of the covered selections (tile kernel) and of the rest
+    (KV-outer kernel), counted as 4 * d * (H/G) per attended (row, key), and
+    the bytes the combine must move: the merged slots' partials (f16) and
+    log-sum-exps read, and the merged outputs (bf16) and log-sum-exps written.
+    """
+    import torch
+
+    T, _, k = sel.shape
+    Hg = H // G
+    UQ = 2 * (128 // max(Hg, 8))
+    dev = sel.device
+    # query position and local block of every row
+    pos = torch.empty(T, dtype=torch.int64)
+    for b in range(len(cu_q_host) - 1):
+        Tb, Sb = cu_q_host[b + 1] - cu_q_host[b], cu_k_host[b + 1] - cu_k_host[b]
+        pos[cu_q_host[b]:cu_q_host[b + 1]] = torch.arange(Sb - Tb, Sb)
+    seq = torch.empty(T, dtype=torch.int64)
+    for b in range(len(cu_q_host) - 1):
+        seq[cu_q_host[b]:cu_q_host[b + 1]] = b
+    pos, seq = pos.to(dev), seq.to(dev)
+    s = sel.to(torch.int64)
+    valid = s >= 0
+    # attended keys per (row, group, slot): whole block, or up to the position in the local block
+    lb = (pos // B_k)[:, None, None]
+    att = torch.where(s < lb, torch.full_like(s, B_k), (pos % B_k + 1)[:, None, None].expand_as(s))
+    att = torch.where(valid, att, torch.zeros_like(att))
+    covered = torch.zeros_like(valid)
+    if theta > 0:
+        rows = T if q_chunk <= 0 else q_chunk
+        for t0 in range(0, T, rows):
+            t1 = min(T, t0 + rows)
+            n = t1 - t0
+            nu = (n + UQ - 1) // UQ
+            pad = nu * UQ - n
+            sp = torch.nn.functional.pad(s[t0:t1], (0, 0, 0, 0, 0, pad), value=-1)
+            sq = torch.nn.functional.pad(seq[t0:t1], (0, pad), value=-1)
+            one = sq.view(nu, UQ)
+            last = torch.tensor([min(UQ, n - u * UQ) - 1 for u in range(nu)], device=dev)
+            one_seq = one[:, 0] == one.gather(1, last[:, None])[:, 0]
+            u = sp.view(nu, UQ, G, k).permute(0, 2, 1, 3).reshape(nu * G, UQ * k)
+            big = torch.iinfo(torch.int64).max
+            v = torch.where(u >= 0, u, torch.full_like(u, big))
+            srt, _ = torch.sort(v, dim=1)
+            cnt = torch.searchsorted(srt, v, right=True) - torch.searchsorted(srt, v)
+            cov = (u >= 0) & (cnt >= theta) & one_seq.repeat_interleave(G)[:, None]
+            cov = cov.view(nu, G, UQ, k).permute(0, 2, 1, 3).reshape(nu * UQ, G, k)[:n]
+            covered[t0:t1] = cov
+    tile_att = (att * covered).sum().item()
+    kv_att = (att * (valid & ~covered)).sum().item()
+    ncov = covered.sum(-1)
+    complete = (ncov > 0) & (ncov == valid.sum(-1))
+    merged_slots = ((valid & ~covered).sum(-1) + (ncov > 0).to(torch.int64))[~complete]
+    npairs = int((~complete).sum().item())
+    comb_bytes = (merged_slots.sum().item() * Hg * d * 2 + npairs * (k * Hg * 4 + 8)
+                  + npairs * (Hg * d * 2 + Hg * 4))
+    return {"tile_flops": float(4 * d * Hg * tile_att), "kv_flops": float(4 * d * Hg * kv_att),
+            "combine_bytes": float(comb_bytes), "combine_pairs": npairs,
+            "complete_pairs": int(complete.sum().item()), "theta": theta, "tile_queries": UQ}

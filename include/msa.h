@@ -162,7 +162,10 @@ msa_status_t msa_sparse_attn_decode(const msa_shape_t* shape, const msa_varlen_t
  *             head i is at [t][g][s][c][i][e]
  *   part_lse  device f32 [T, G, k, H/G]          that block's log-sum-exp
  * into out[t, h, :] = sum_s exp(lse_s - LSE) * acc_s with LSE = log sum_s
- * exp(lse_s), and lse[t, h] = LSE (lse may be NULL). */
+ * exp(lse_s), and lse[t, h] = LSE (lse may be NULL).  part_acc and part_lse
+ * must start on 16-byte boundaries (MSA_ERR_INVALID_ARG otherwise); every
+ * query needs at least one slot with sel >= 0.  Slots with sel < 0 are never
+ * read. */
 msa_status_t msa_combine(const msa_shape_t* shape, int64_t T,
                          const void* part_acc, const float* part_lse, const int32_t* sel,
                          void* out, float* lse, void* stream);
@@ -170,12 +173,31 @@ msa_status_t msa_combine(const msa_shape_t* shape, int64_t T,
 /* ---------------------------------------------------------------------- */
 /* Dense causal GQA attention (every key <= the query position), the
  * denominator of the pages' speedup comparison against GQA (pnsm.cn sec. 9).
- * Same layouts as the sparse call; the workspace only holds the error word. */
+ * Same layouts and argument rules as msa_sparse_attn_prefill without `sel`
+ * (shape->k and shape->d_idx are ignored apart from the shape checks); the
+ * workspace (msa_dense_attn_workspace_size bytes, 256-byte aligned) holds the
+ * error word and the per-sequence tile counts.  A sequence with more queries
+ * than keys records MSA_ERR_DEVICE_CHECK in the error word and gets no output.
+ * Asynchronous on `stream`. */
 size_t msa_dense_attn_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs);
 
 msa_status_t msa_dense_attn(const msa_shape_t* shape, const msa_varlen_t* seqs,
                             const void* q, const void* k, const void* v,
                             void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Work split of the prefill main branch (process-wide; returns the previous
+ * value).  The prefill call groups query rows into tiles of 2 x 128/max(H/G, 8)
+ * consecutive queries of one sequence; a block chosen by at least `theta` of a
+ * tile's queries (for one group) is attended query-tile-major, merged with an
+ * online softmax into one result per query, instead of one KV-outer partial
+ * per (query, block).  The selected token sets and the exact softmax are the
+ * same either way; only the rounding order differs.
+ *   theta < 0   automatic: ceil(3/8 x tile queries) (the default)
+ *   theta == 0  off: every selection goes through the KV-outer lists
+ *   theta >= 1  that threshold (1: every selected block of a tile)
+ * Decode calls (one query per sequence) never use query tiles. */
+int32_t msa_set_tile_threshold(int32_t theta);
 
 /* ---------------------------------------------------------------------- */
 /* Decode-shaped index top-k that allocates nothing (the pages have no

@@ -227,6 +227,82 @@ def test_combine_entry_point(M):
             assert abs(lse_out[t, h].item() - rl) <= 1e-4
 
 
+# ------------------------------------------- query tiles and dense GQA ----
+
+def _prefill_with_threshold(M, theta, shape, seqs, d, sel, q_chunk=0):
+    prev = M.msa_set_tile_threshold(theta)
+    try:
+        return M.msa_sparse_attn_prefill(shape, seqs, d["q"], d["k"], d["v"], sel, q_chunk=q_chunk)
+    finally:
+        M.msa_set_tile_threshold(prev)
+
+
+@pytest.mark.parametrize("theta", [0, 1, 3, -1, 1000])
+def test_prefill_tile_threshold(M, theta):
+    """Every split of the selections between query tiles and KV-outer lists
+    gives the oracle's result: 0 (all KV-outer), 1 (every selected block of a
+    tile), 3, automatic, and a threshold no block reaches.  Hot blocks, ragged
+    tails, tiles that straddle a sequence boundary, queries that are the last
+    tokens of their sequence."""
+    w = _custom("tiles", 64, 4, 128, 64, 16, hot=0.05, seed=31)
+    inp = _inputs(w, lengths=[2600, 130, 1901], T_lens=[2600, 130, 1001])
+    shape, seqs, d = _to_dev(M, w, inp)
+    ref_sel = _oracle_sel(w, inp)
+    out, lse = _prefill_with_threshold(M, theta, shape, seqs, d, torch.from_numpy(ref_sel).cuda())
+    o_ref, lse_ref = _oracle_out(w, inp, ref_sel)
+    _check_out(out, lse, o_ref, lse_ref)
+
+
+@pytest.mark.parametrize("theta", [1, -1])
+def test_prefill_tiles_chunked_passes(M, theta):
+    """Passes of 700 rows: tiles restart at each pass start."""
+    w = _custom("tiles_q", 64, 4, 128, 64, 16, hot=0.05, seed=32)
+    inp = _inputs(w, lengths=[3001, 1500])
+    shape, seqs, d = _to_dev(M, w, inp)
+    ref_sel = _oracle_sel(w, inp)
+    out, lse = _prefill_with_threshold(M, theta, shape, seqs, d, torch.from_numpy(ref_sel).cuda(), q_chunk=700)
+    o_ref, lse_ref = _oracle_out(w, inp, ref_sel)
+    _check_out(out, lse, o_ref, lse_ref)
+
+
+@pytest.mark.parametrize("theta", [1, -1])
+def test_prefill_tiles_small_heads(M, theta):
+    """H/G = 16, 4 and 8 (tiles of 16, 32, 32 queries), d = 64 and 128."""
+    for (H, G, d_, k) in [(16, 1, 64, 4), (8, 2, 128, 6), (32, 4, 64, 8)]:
+        w = _custom("tiles_small", H, G, d_, 32, k, hot=0.05, seed=33)
+        inp = _inputs(w, lengths=[1500, 333])
+        shape, seqs, d = _to_dev(M, w, inp)
+        ref_sel = _oracle_sel(w, inp)
+        out, lse = _prefill_with_threshold(M, theta, shape, seqs, d, torch.from_numpy(ref_sel).cuda())
+        o_ref, lse_ref = _oracle_out(w, inp, ref_sel)
+        _check_out(out, lse, o_ref, lse_ref)
+
+
+def _all_blocks_sel(cu_q, cu_k, G, B_k=128):
+    """Selection of every causal block (k >= blocks): the oracle's dense case."""
+    T = cu_q[-1]
+    nbmax = max((cu_k[b + 1] - cu_k[b] + B_k - 1) // B_k for b in range(len(cu_q) - 1))
+    sel = np.full((T, G, nbmax), -1, dtype=np.int32)
+    for b in range(len(cu_q) - 1):
+        Tb, Sb = cu_q[b + 1] - cu_q[b], cu_k[b + 1] - cu_k[b]
+        for i in range(Tb):
+            nb = (Sb - Tb + i) // B_k + 1
+            sel[cu_q[b] + i, :, :nb] = np.arange(nb)
+    return sel
+
+
+@pytest.mark.parametrize("H,G,d_", [(64, 4, 128), (16, 2, 64), (8, 2, 128), (32, 4, 64)])
+def test_dense_causal_gqa(M, H, G, d_):
+    """msa_dense_attn against the oracle with every causal block selected."""
+    w = _custom("dense", H, G, d_, 32, 4, seed=41)
+    inp = _inputs(w, lengths=[1500, 129, 700], T_lens=[1500, 129, 301])
+    shape, seqs, d = _to_dev(M, w, inp)
+    out, lse = M.msa_dense_attn(shape, seqs, d["q"], d["k"], d["v"], want_lse=True)
+    sel = _all_blocks_sel(inp["cu_q_host"], inp["cu_k_host"], G)
+    o_ref, lse_ref = _oracle_out(w, inp, sel)
+    _check_out(out, lse, o_ref, lse_ref)
+
+
 # ------------------------------------------------------------ errors -------
 
 def test_out_of_range_selection_is_reported_not_faulted(M):
