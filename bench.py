@@ -177,10 +177,15 @@ def time_steps(fn, steps, torch, dist=None):
     return s.elapsed_time(e)
 
 
+def _reduce_device(dist):
+    """NCCL reduces device tensors; gloo (the CPU tests) host tensors."""
+    return "cuda" if dist.get_backend() == "nccl" else "cpu"
+
+
 def max_over_ranks(x, torch, dist):
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_reduce_device(dist))
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -188,9 +193,20 @@ def max_over_ranks(x, torch, dist):
 def sum_over_ranks(x, torch, dist):
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_reduce_device(dist))
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def job_rate(tokens_local, ms_local, torch, dist):
+    """Whole-job tokens/s: tokens of all ranks over the slowest rank's time."""
+    ms_max = max_over_ranks(ms_local, torch, dist)
+    return sum_over_ranks(float(tokens_local), torch, dist) / (ms_max / 1000.0), ms_max
+
+
+def rank_workload(w, rank, W):
+    """Each rank runs an independent layer of the same shape (its own seed)."""
+    return W.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
 
 
 def traffic_for(kernel):
@@ -327,7 +343,7 @@ def run_ours(args):
         return (3 * uq + 7) // 8
     w = W.WORKLOADS[args.workload]
     # each rank runs an independent layer (its own seed): weak scaling
-    wr = W.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+    wr = rank_workload(w, rank, W)
     inp = W.make_inputs(wr, "cuda", T_override=args.T or None)
     torch.cuda.synchronize()
     make_ctx.index_only = args.index_only
@@ -364,10 +380,8 @@ def run_ours(args):
     for v in kernels.values():
         v["share"] = v["ms_per_launch"] * v["launches"] / tot
 
-    ms_max = max_over_ranks(ms, torch, dist)
+    value, ms_max = job_rate(T * args.steps, ms, torch, dist)
     ms_step = ms_max / args.steps
-    tokens_all = sum_over_ranks(float(T * args.steps), torch, dist)
-    value = tokens_all / (ms_max / 1000.0)
 
     # algorithmic work of each kernel: the main branch split between the query
     # tiles and the KV-outer lists as the library's planner splits it
