@@ -64,8 +64,12 @@ __device__ __forceinline__ int entry_list(int blk, int64_t t, int g, int G, int 
 // kScatter == false counts, == true claims positions from `counter`
 // (the cursors) and writes the entries (t - t0) * k + slot.
 // Slots whose bit is set in dmask (when given) were attended by a query tile
-// and get no list entry; they are still validated.  With clist (no query
-// tiles), the counting pass also writes every pair's combine-list entry.
+// and get no list entry; they are still validated.  A pair's partials are
+// packed at the front of its k-slot run: the tile's merged partial (if any)
+// first, then its KV-outer slots in slot order, so that the combine reads one
+// contiguous run per pair; an entry (t - t0) * k + p names packed position p.
+// With clist (no query tiles), the counting pass also writes every pair's
+// combine-list entry {pair, number of packed partials}.
 template <bool kScatter>
 __global__ void count_scatter_kernel(const int32_t* __restrict__ sel, int64_t t0, int64_t t1, int G, int k,
                                      int batch, const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_k,
@@ -81,11 +85,14 @@ __global__ void count_scatter_kernel(const int32_t* __restrict__ sel, int64_t t0
   const int64_t wbase = (tl / kWindow) * nlists;
   const int lane = threadIdx.x & 31;
   const uint32_t covered = (active && dmask != nullptr) ? dmask[gid] : 0u;
-  uint32_t live = 0;
+  const int first = covered != 0u ? 1 : 0;   // packed position 0 holds the tile's merged partial
+  uint32_t live = 0;                          // live slots below s
   for (int s = 0; s < k; ++s) {
     int64_t key = -1;
+    int packed = 0;
     if (active) {
       const int32_t blk = sel[(t * G + g) * k + s];
+      packed = first + __popc(live & ~covered);
       if (blk >= 0) live |= 1u << s;
       const int L = entry_list(blk, t, g, G, batch, cu_q, cu_k, blk_off, err);
       if (L >= 0 && !((covered >> s) & 1u)) key = wbase + L;
@@ -97,9 +104,9 @@ __global__ void count_scatter_kernel(const int32_t* __restrict__ sel, int64_t t0
     int base = 0;
     if (key >= 0 && lane == leader) base = atomicAdd(&counter[key], __popc(peers));
     base = __shfl_sync(0xffffffffu, base, leader);
-    if (kScatter && key >= 0) entries[base + rank] = (uint32_t)(tl * k + s);
+    if (kScatter && key >= 0) entries[base + rank] = (uint32_t)(tl * k + packed);
   }
-  if (!kScatter && clist != nullptr && active) clist[gid] = make_uint2((uint32_t)gid, live);
+  if (!kScatter && clist != nullptr && active) clist[gid] = make_uint2((uint32_t)gid, (uint32_t)__popc(live));
 }
 
 // Device-wide exclusive scan of the list counts (and of their item counts,
@@ -676,120 +683,170 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 
 // -------------------------------------------------------------- combine ---
 
-// Persistent combine: the partials of one (query, group) are one contiguous
-// run (k slots x [d/8][Hg][8] f16, 4 KB per slot at Hg = 16, d = 128), and
-// its k x Hg log-sum-exps another.  Thread 0 streams the slots to merge of P
-// (query, group) pairs into an nst-stage shared-memory ring with bulk async
-// copies; thread (pair, c, i) merges output columns 8c..8c+7 of head i from
-// shared memory (consecutive threads read consecutive 16-byte words: no bank
-// conflicts).  A pair spans Hg * d/8 threads, a multiple of 32.
-//   clist given: entry {pair, slot mask} per merged pair; only the slots in
-//                the mask are copied (the query tiles leave most slots empty);
-//   clist null : every pair, slots with sel >= 0 (each warp reads its pair's
-//                selection with one load per lane), whole runs copied.
-constexpr int kCombThreads = 256;
-constexpr int kCombMaxStages = 3;
+// Persistent combine.  The partials of one (query, group) are one contiguous
+// run (k slots x [d/8][Hg][8] f16, 4 KB per slot at Hg = 16, d = 128), its
+// k x Hg log-sum-exps another.  A chunk is P (query, group) pairs, handled by
+// one consumer group of 256 threads: thread (pair, c, i) merges output columns
+// 8c..8c+7 of head i (a pair spans Hg * d/8 threads, a multiple of 32;
+// consecutive threads read consecutive 16-byte words of shared memory).
+//   clist given: entry {pair, n} per merged pair, partials packed in slots
+//                0..n-1: only those n slots are copied (the query tiles leave
+//                most slots empty);
+//   clist null : every pair, slots with sel >= 0, whole runs copied.
+// Warp 16 (lane 0) is the producer: it streams each chunk's runs with bulk
+// async copies into a byte-granular ring of shared memory (a chunk takes what
+// its runs need, so the bytes in flight follow the real sizes) and publishes
+// it in a queue of kCombQueue entries; consumer groups 0 and 1 take alternate
+// entries and release them through per-entry barriers, so the two groups and
+// the producer never wait for one another except on data.
+constexpr int kCombGroupThreads = 256;
+constexpr int kCombThreads = 2 * kCombGroupThreads + 32;
+constexpr int kCombQueue = 8;
 constexpr int kCombMaxPairs = 8;
+constexpr uint32_t kCombRing = 200 * 1024;
+
+struct CombEntry {
+  uint32_t off[kCombMaxPairs];   // ring offset of each pair's run (partials, then log-sum-exps)
+  uint32_t pair[kCombMaxPairs];
+  uint32_t n[kCombMaxPairs];     // slots copied
+};
+
+struct CombCtl {
+  uint64_t full[kCombQueue], consumed[kCombQueue];
+  uint64_t end_of[kCombQueue];   // producer: virtual ring offset after each entry
+  CombEntry e[kCombQueue];
+  int32_t abort_flag;
+};
 
 __global__ void __launch_bounds__(kCombThreads, 1)
 combine_kernel(const __half* __restrict__ part_acc, const float* __restrict__ part_lse,
                const int32_t* __restrict__ sel, const uint2* __restrict__ clist,
                const int32_t* __restrict__ npairs_dev, __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out,
-               int64_t T, int H, int G, int d, int k, int P, int nst, uint32_t acc_bytes, uint32_t lse_bytes,
-               uint32_t stage_bytes, DevError* err) {
+               int64_t T, int H, int G, int d, int k, int P, uint32_t acc_bytes, uint32_t lse_bytes,
+               DevError* err) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
-  uint8_t* smem = smem_raw + (((raw + 127u) & ~127u) - raw);
-  __shared__ uint64_t full[kCombMaxStages];
+  uint8_t* ring = smem_raw + (((raw + 127u) & ~127u) - raw);
+  __shared__ CombCtl ctl;
+  volatile int32_t* abort_flag = &ctl.abort_flag;
   const int Hg = H / G;
   const int per = Hg * (d / 8);                 // threads per (query, group)
-  const uint32_t slot_bytes = acc_bytes / k;
+  const uint32_t slot_bytes = acc_bytes / k;    // one slot's partial (multiple of 16)
+  const uint32_t slot_lse = lse_bytes / k;      // one slot's Hg log-sum-exps (multiple of 16)
   const int64_t npairs = npairs_dev != nullptr ? (int64_t)*npairs_dev : T * G;
   const int64_t nchunks = (npairs + P - 1) / P;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < nst; ++i) mbar_init(&full[i], 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int i = 0; i < kCombQueue; ++i) {
+      mbar_init(&ctl.full[i], 1);
+      mbar_init(&ctl.consumed[i], kCombGroupThreads / 32);
+    }
+    ctl.abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
-  // the n-th chunk of this CTA is chunk blockIdx.x + n * gridDim.x
+  // the m-th chunk of this CTA is chunk blockIdx.x + m * gridDim.x
   const int64_t my = blockIdx.x < nchunks ? (nchunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  // thread 0: list entries of a chunk (fetched one iteration before they are used)
-  uint2 ent[kCombMaxPairs];
-  auto fetch = [&](int64_t n) {
-    const int64_t p0 = (blockIdx.x + n * gridDim.x) * P;
+
+  if (warp == 2 * kCombGroupThreads / 32) {
+    // ------------------------------------------------------------ producer
+    if (lane != 0) return;
+    uint64_t alloc = 0, freed = 0;              // virtual ring offsets (physical = virtual % ring)
+    int64_t oldest = 0, m = 0;
+    bool ok = true;
+    for (; m < my && ok && !*abort_flag; ++m) {
+      const int q = (int)(m % kCombQueue);
+      const int64_t p0 = (blockIdx.x + m * gridDim.x) * P;
+      const int np = npairs - p0 < P ? (int)(npairs - p0) : P;
+      uint2 ent[kCombMaxPairs];
+      uint32_t bytes = 0;
 #pragma unroll
-    for (int i = 0; i < kCombMaxPairs; ++i)
-      if (i < P && p0 + i < npairs) ent[i] = clist != nullptr ? clist[p0 + i] : make_uint2((uint32_t)(p0 + i), ~0u);
-  };
-  auto issue = [&](int64_t n) {
-    const int stage = (int)(n % nst);
-    const int64_t p0 = (blockIdx.x + n * gridDim.x) * P;
-    const int64_t left = npairs - p0;
-    const int np = left < P ? (int)left : P;
-    uint8_t* dst = smem + stage * stage_bytes;
-    uint32_t bytes = 0;
-#pragma unroll
-    for (int i = 0; i < kCombMaxPairs; ++i)
-      if (i < np) bytes += (clist != nullptr ? __popc(ent[i].y) * slot_bytes : acc_bytes) + lse_bytes;
-    mbar_arrive_expect_tx(&full[stage], bytes);
-#pragma unroll
-    for (int i = 0; i < kCombMaxPairs; ++i) {
-      if (i >= np) continue;
-      const uint8_t* src = reinterpret_cast<const uint8_t*>(part_acc) + (int64_t)ent[i].x * acc_bytes;
-      if (clist != nullptr) {
-        for (uint32_t m = ent[i].y; m != 0u; m &= m - 1u) {
-          const int s2 = __ffs(m) - 1;
-          bulk_load(dst + i * acc_bytes + s2 * slot_bytes, src + s2 * slot_bytes, slot_bytes, &full[stage]);
+      for (int i = 0; i < kCombMaxPairs; ++i) {
+        ent[i] = make_uint2(0u, 0u);
+        if (i < np) {
+          ent[i] = clist != nullptr ? clist[p0 + i] : make_uint2((uint32_t)(p0 + i), (uint32_t)k);
+          bytes += ent[i].y * (slot_bytes + slot_lse);
         }
-      } else {
-        bulk_load(dst + i * acc_bytes, src, acc_bytes, &full[stage]);
       }
-      bulk_load(dst + P * acc_bytes + i * lse_bytes,
-                reinterpret_cast<const uint8_t*>(part_lse) + (int64_t)ent[i].x * lse_bytes, lse_bytes, &full[stage]);
+      // contiguous room in the ring (skip the ring's tail end when it is too short)
+      const uint64_t phys = alloc % kCombRing;
+      if (phys + bytes > kCombRing) alloc += kCombRing - phys;
+      // the queue entry and the bytes must both be free: retire the oldest entries in order
+      while (ok && (m - oldest >= kCombQueue || alloc + bytes - freed > kCombRing)) {
+        if (oldest == m) {                      // nothing in flight: the whole ring is free
+          freed = alloc;
+          continue;
+        }
+        const int qo = (int)(oldest % kCombQueue);
+        ok = mbar_wait(&ctl.consumed[qo], (uint32_t)((oldest / kCombQueue) & 1));
+        if (ok) { freed = ctl.end_of[qo]; ++oldest; }
+      }
+      if (!ok) break;
+      // entry q is free (its previous chunk was consumed): publish this chunk in it
+      CombEntry& E = ctl.e[q];
+      uint32_t off = (uint32_t)(alloc % kCombRing);
+      mbar_arrive_expect_tx(&ctl.full[q], bytes);
+#pragma unroll
+      for (int i = 0; i < kCombMaxPairs; ++i) {
+        if (i >= np) continue;
+        E.off[i] = off;
+        E.pair[i] = ent[i].x;
+        E.n[i] = ent[i].y;
+        const uint32_t na = ent[i].y * slot_bytes, nl = ent[i].y * slot_lse;
+        bulk_load(ring + off, reinterpret_cast<const uint8_t*>(part_acc) + (int64_t)ent[i].x * acc_bytes, na,
+                  &ctl.full[q]);
+        bulk_load(ring + off + na, reinterpret_cast<const uint8_t*>(part_lse) + (int64_t)ent[i].x * lse_bytes, nl,
+                  &ctl.full[q]);
+        off += na + nl;
+      }
+      alloc += bytes;
+      ctl.end_of[q] = alloc;
     }
-  };
-  if (threadIdx.x == 0)
-    for (int64_t n = 0; n < nst && n < my; ++n) {
-      fetch(n);
-      issue(n);
+    if (!ok) {
+      report_error(err, MSA_ERR_TIMEOUT, kSiteAttnLoad, (int)m, -2);
+      *abort_flag = 1;
     }
-  const int lane = threadIdx.x & 31;
-  const int pl = threadIdx.x / per;             // pair within the chunk (P * per == kCombThreads)
-  const int rem = threadIdx.x - pl * per;
+    // no bulk copy may still be writing when the CTA exits
+    for (int64_t j = oldest; j < m; ++j) mbar_wait(&ctl.full[j % kCombQueue], (uint32_t)((j / kCombQueue) & 1));
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int grp = warp / (kCombGroupThreads / 32);
+  const int gt = tid - grp * kCombGroupThreads;
+  const int pl = gt / per;                      // pair within the chunk (P * per == kCombGroupThreads)
+  const int rem = gt - pl * per;
   const int cc = rem / Hg, i = rem - cc * Hg;
-  int64_t n = 0;
-  for (; n < my; ++n) {
-    const int stage = (int)(n % nst);
-    const int64_t idx = (blockIdx.x + n * gridDim.x) * P + pl;
+  for (int64_t m = grp; m < my && !*abort_flag; m += 2) {
+    const int q = (int)(m % kCombQueue);
+    const int64_t idx = (blockIdx.x + m * gridDim.x) * P + pl;
     const bool live = idx < npairs;
-    if (threadIdx.x == 0 && n + nst < my) fetch(n + nst);
-    int64_t pair = idx;
-    uint32_t valid;
-    if (clist != nullptr) {
-      const uint2 e = live ? clist[idx] : make_uint2(0u, 0u);
-      pair = e.x;
-      valid = e.y;
-    } else {
-      const int32_t sv = (lane < k && live) ? __ldg(sel + pair * k + lane) : -1;
+    uint32_t valid = 0;
+    if (clist == nullptr) {
+      const int32_t sv = (lane < k && live) ? __ldg(sel + idx * k + lane) : -1;
       valid = __ballot_sync(0xffffffffu, sv >= 0);
     }
-    const bool ok = mbar_wait(&full[stage], (uint32_t)((n / nst) & 1));
-    if (__syncthreads_or(!ok)) {
-      if (threadIdx.x == 0) report_error(err, MSA_ERR_TIMEOUT, kSiteAttnLoad, (int)n, -2);
+    if (!mbar_wait(&ctl.full[q], (uint32_t)((m / kCombQueue) & 1))) {
+      report_error(err, MSA_ERR_TIMEOUT, kSiteAttnLoad, (int)m, -3);
+      *abort_flag = 1;
       break;
     }
     if (live) {
-      const uint8_t* base = smem + stage * stage_bytes;
-      const __half* acc_s = reinterpret_cast<const __half*>(base + pl * acc_bytes);
-      const float* lse_s = reinterpret_cast<const float*>(base + P * acc_bytes + pl * lse_bytes);
-      float m = -INFINITY;
-      for (int s2 = 0; s2 < k; ++s2)
-        if ((valid >> s2) & 1u) m = fmaxf(m, lse_s[s2 * Hg + i]);
+      const CombEntry& E = ctl.e[q];
+      const int n = (int)E.n[pl];
+      const int64_t pair = E.pair[pl];
+      if (clist != nullptr) valid = n >= 32 ? 0xffffffffu : (1u << n) - 1u;
+      const __half* acc_s = reinterpret_cast<const __half*>(ring + E.off[pl]);
+      const float* lse_s = reinterpret_cast<const float*>(ring + E.off[pl] + n * slot_bytes);
+      float m_ = -INFINITY;
+#pragma unroll 4
+      for (int s2 = 0; s2 < n; ++s2)
+        if ((valid >> s2) & 1u) m_ = fmaxf(m_, lse_s[s2 * Hg + i]);
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       float wsum = 0.f;
-      for (int s2 = 0; s2 < k; ++s2) {
-        if (!((valid >> s2) & 1u)) continue;
-        const float w = __expf(lse_s[s2 * Hg + i] - m);
+#pragma unroll 4
+      for (int s2 = 0; s2 < n; ++s2) {
+        const float w = ((valid >> s2) & 1u) ? __expf(lse_s[s2 * Hg + i] - m_) : 0.f;
         wsum += w;
         const uint4 rv = *reinterpret_cast<const uint4*>(acc_s + ((s2 * (d / 8) + cc) * Hg + i) * 8);
         const __half2* hp = reinterpret_cast<const __half2*>(&rv);
@@ -809,15 +866,10 @@ combine_kernel(const __half* __restrict__ part_acc, const float* __restrict__ pa
       const int64_t t = pair / G;
       const int h = (int)(pair - t * G) * Hg + i;
       *reinterpret_cast<uint4*>(out + (t * H + h) * d + 8 * cc) = o;
-      if (lse_out != nullptr && cc == 0) lse_out[t * H + h] = m + __logf(wsum);
+      if (lse_out != nullptr && cc == 0) lse_out[t * H + h] = m_ + __logf(wsum);
     }
-    __syncthreads();                            // stage consumed by every thread
-    if (threadIdx.x == 0 && n + nst < my) issue(n + nst);
-  }
-  // after a timeout no bulk copy may still be writing when the CTA exits
-  if (threadIdx.x == 0 && n < my) {
-    const int64_t last = my < n + nst ? my : n + nst;
-    for (int64_t m2 = n; m2 < last; ++m2) mbar_wait(&full[m2 % nst], (uint32_t)((m2 / nst) & 1));
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ctl.consumed[q]);
   }
 }
 
@@ -827,29 +879,26 @@ int launch_combine_kernel(const __half* part_acc, const float* part_lse, const i
   if (T <= 0) return 0;
   const int Hg = H / G;
   const int per = Hg * (d / 8);
-  if (per % 32 != 0 || kCombThreads % per != 0 || k > 32) return (int)cudaErrorInvalidValue;
-  const int P = kCombThreads / per;
+  if (per % 32 != 0 || kCombGroupThreads % per != 0 || k > 32) return (int)cudaErrorInvalidValue;
+  const int P = kCombGroupThreads / per;
   if (P > kCombMaxPairs) return (int)cudaErrorInvalidValue;
   const uint32_t acc_bytes = (uint32_t)k * Hg * d * 2;
   const uint32_t lse_bytes = (uint32_t)k * Hg * 4;
-  // bulk copies need 16-byte sizes and addresses
-  if (((acc_bytes | lse_bytes) & 15u) || ((reinterpret_cast<uintptr_t>(part_acc) |
-                                           reinterpret_cast<uintptr_t>(part_lse)) & 15u))
+  // bulk copies need 16-byte sizes and addresses; one chunk must fit the ring
+  if (((acc_bytes / k | lse_bytes / k) & 15u) || ((reinterpret_cast<uintptr_t>(part_acc) |
+                                                   reinterpret_cast<uintptr_t>(part_lse)) & 15u) ||
+      (uint64_t)P * (acc_bytes + lse_bytes) > kCombRing)
     return (int)cudaErrorInvalidValue;
-  const uint32_t stage_bytes = (P * (acc_bytes + lse_bytes) + 127u) & ~127u;
-  const size_t avail = 227 * 1024 - 128 - 64;
-  const int nst = (int)(avail / stage_bytes < kCombMaxStages ? avail / stage_bytes : kCombMaxStages);
-  if (nst < 1) return (int)cudaErrorInvalidValue;
-  const size_t smem = 128 + (size_t)nst * stage_bytes;
+  const size_t smem = 128 + kCombRing;
   cudaError_t e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return (int)e;
   int dev = 0, nsm = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t nchunks = (T * G + P - 1) / P;   // upper bound when a pair list is given
+  const int64_t nchunks = (T * G + P - 1) / P;   // upper bound when a list is given
   const int grid = (int)(nchunks < nsm ? nchunks : nsm);
   combine_kernel<<<grid, kCombThreads, smem, st>>>(part_acc, part_lse, sel, clist, npairs_dev, out, lse, T, H, G, d,
-                                                  k, P, nst, acc_bytes, lse_bytes, stage_bytes, err);
+                                                  k, P, acc_bytes, lse_bytes, err);
   return (int)cudaGetLastError();
 }
 

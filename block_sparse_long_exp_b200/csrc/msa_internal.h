@@ -106,7 +106,7 @@ struct AttnArgs {
   int64_t max_items;
   int32_t* blk_off;    // [batch + 1] block offsets per sequence
   int64_t nlists;      // G * total blocks
-  void* part_acc;      // f16 [(t1-t0), G, k, d/8, Hg, 8]
+  void* part_acc;      // f16 [(t1-t0), G, k, d/8, Hg, 8], each pair's partials packed at slots 0..n-1
   float* part_lse;     // [(t1-t0), G, k, Hg]
   int32_t queries_per_item;
   // query-tile (Q-outer) side; theta == 0 turns it off

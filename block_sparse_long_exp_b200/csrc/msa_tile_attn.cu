@@ -25,9 +25,9 @@
 //                    unit's dense blocks, ascending), and per query the slot
 //                    mask of those selections, their positions in the dense
 //                    list, whether they cover the query, and the combine
-//                    list: each query that still needs the combine with the
-//                    slots to merge (its KV-outer slots and the lowest covered
-//                    slot, which receives the tile's merged partial).
+//                    list: each query that still needs the combine with its
+//                    number of partials (packed at the front of its slot run:
+//                    the tile's merged partial first, then the KV-outer ones).
 // tile_attn_kernel   persistent, warp-specialised (one CTA per SM, 512 threads):
 //   warp 0      claims units (atomic ticket) and publishes them in a 2-deep
 //               shared-memory ring;
@@ -139,7 +139,7 @@ tile_plan_kernel(const int32_t* __restrict__ sel, int64_t t0, int64_t t1, int G,
   // lane q: masks of query q (UQ <= 32)
   const bool qv = lane < nq;
   bool need_combine = false;
-  uint32_t cmask = 0;
+  uint32_t cmask = 0;                          // number of packed partials to merge
   if (qv) {
     const int64_t t = r0 + lane;
     uint32_t dm = 0, vm = 0;
@@ -164,7 +164,7 @@ tile_plan_kernel(const int32_t* __restrict__ sel, int64_t t0, int64_t t1, int G,
     dmember[pr] = mem;
     dstate[pr] = dm == 0 ? -1 : ((__ffs(dm) - 1) | (complete ? kDenseComplete : 0));
     need_combine = !complete;
-    cmask = (vm & ~dm) | (dm & (0u - dm));   // KV-outer slots and the tile's merged partial
+    cmask = (uint32_t)__popc(vm & ~dm) + (dm != 0u ? 1u : 0u);   // packed: the tile's, then the KV-outer ones
   }
   const unsigned bal = __ballot_sync(0xffffffffu, need_combine);
   int base = 0;
@@ -221,7 +221,7 @@ struct TileParams {
   const int32_t* unit_blk;    // hybrid: [units x G][kMaxDense]
   const int32_t* unit_nblk;
   const uint64_t* dmember;    // hybrid: [rows x G] dense-list membership bits
-  const int32_t* dstate;      // hybrid: [rows x G] first dense slot | kDenseComplete, or -1
+  const int32_t* dstate;      // hybrid: [rows x G] kDenseComplete | first covered slot, or -1
   const int32_t* seq_units;   // dense: [batch + 1] prefix of units per sequence
   const int32_t* nunits;      // device count of units (hybrid: listed units; dense: all)
   int32_t* ticket;
@@ -704,7 +704,7 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         const int h = g * Hg + hi;
         const uint32_t o_col = tmem + x * 256 + 128 + lane_off;
         int64_t unit = 0;
-        if (has && !complete) unit = (((t - p.t0) * G + g) * p.k + (state & 0xff));
+        if (has && !complete) unit = ((t - p.t0) * G + g) * p.k;   // packed position 0
         uint32_t rr[32];
 #pragma unroll 1
         for (int c4 = 0; c4 < d / 32; ++c4) {

@@ -104,7 +104,9 @@ def tile_split(sel, cu_q_host: Sequence[int], cu_k_host: Sequence[int], H: int, 
     Returns the FLOPs of the covered selections (tile kernel) and of the rest
     (KV-outer kernel), counted as 4 * d * (H/G) per attended (row, key), and
     the bytes the combine must move: the merged slots' partials (f16) and
-    log-sum-exps read, and the merged outputs (bf16) and log-sum-exps written.
+    log-sum-exps read, and the merged outputs (bf16) and log-sum-exps written;
+    also the MMA work the tile kernel issues (whole 128-row tiles per dense
+    block, including the rows of queries that did not choose the block).
     """
     import torch
 
@@ -128,6 +130,9 @@ def tile_split(sel, cu_q_host: Sequence[int], cu_k_host: Sequence[int], H: int, 
     att = torch.where(s < lb, torch.full_like(s, B_k), (pos % B_k + 1)[:, None, None].expand_as(s))
     att = torch.where(valid, att, torch.zeros_like(att))
     covered = torch.zeros_like(valid)
+    tile_blocks = 0          # (unit, dense block, 128-row MMA tile) triples the tile kernel runs
+    RQ = max(Hg, 8)
+    qpt = 128 // RQ
     if theta > 0:
         rows = T if q_chunk <= 0 else q_chunk
         for t0 in range(0, T, rows):
@@ -145,7 +150,14 @@ def tile_split(sel, cu_q_host: Sequence[int], cu_k_host: Sequence[int], H: int, 
             v = torch.where(u >= 0, u, torch.full_like(u, big))
             srt, _ = torch.sort(v, dim=1)
             cnt = torch.searchsorted(srt, v, right=True) - torch.searchsorted(srt, v)
-            cov = (u >= 0) & (cnt >= theta) & one_seq.repeat_interleave(G)[:, None]
+            oneg = one_seq.repeat_interleave(G)
+            cov = (u >= 0) & (cnt >= theta) & oneg[:, None]
+            start = torch.ones_like(srt, dtype=torch.bool)
+            start[:, 1:] = srt[:, 1:] != srt[:, :-1]
+            runlen = torch.searchsorted(srt, srt, right=True) - torch.searchsorted(srt, srt)
+            nd = (start & (runlen >= theta) & (srt != big)).sum(1).clamp(max=64) * oneg
+            nq = torch.tensor([min(UQ, n - x * UQ) for x in range(nu)], device=dev).repeat_interleave(G)
+            tile_blocks += int((nd * torch.where(nq > qpt, 2, 1)).sum().item())
             cov = cov.view(nu, G, UQ, k).permute(0, 2, 1, 3).reshape(nu * UQ, G, k)[:n]
             covered[t0:t1] = cov
     tile_att = (att * covered).sum().item()
@@ -154,8 +166,9 @@ def tile_split(sel, cu_q_host: Sequence[int], cu_k_host: Sequence[int], H: int, 
     complete = (ncov > 0) & (ncov == valid.sum(-1))
     merged_slots = ((valid & ~covered).sum(-1) + (ncov > 0).to(torch.int64))[~complete]
     npairs = int((~complete).sum().item())
-    comb_bytes = (merged_slots.sum().item() * Hg * d * 2 + npairs * (k * Hg * 4 + 8)
+    comb_bytes = (merged_slots.sum().item() * Hg * (d * 2 + 4) + npairs * 8
                   + npairs * (Hg * d * 2 + Hg * 4))
     return {"tile_flops": float(4 * d * Hg * tile_att), "kv_flops": float(4 * d * Hg * kv_att),
+            "tile_mma_flops": float(tile_blocks * 4 * 128 * 128 * d),
             "combine_bytes": float(comb_bytes), "combine_pairs": npairs,
             "complete_pairs": int(complete.sum().item()), "theta": theta, "tile_queries": UQ}
