@@ -562,8 +562,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             uint32_t pk[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              const float p0 = exp2f(fmaf(__uint_as_float(rr[2 * j]), scale_log2, -ms));
-              const float p1 = exp2f(fmaf(__uint_as_float(rr[2 * j + 1]), scale_log2, -ms));
+              const float p0 = ex2_approx(fmaf(__uint_as_float(rr[2 * j]), scale_log2, -ms));
+              const float p1 = ex2_approx(fmaf(__uint_as_float(rr[2 * j + 1]), scale_log2, -ms));
               l += p0 + p1;
               pk[j] = pack_bf16x2(p0, p1);
             }
@@ -576,7 +576,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (32 * c4 + j <= limit) m = fmaxf(m, __uint_as_float(rr[j]));
+              m = fmaxf(m, 32 * c4 + j <= limit ? __uint_as_float(rr[j]) : -INFINITY);
           }
           ms = m * scale_log2;
 #pragma unroll 1
@@ -587,8 +587,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const int c0 = 32 * c4 + 2 * j;
-              const float p0 = c0 <= limit ? exp2f(fmaf(__uint_as_float(rr[2 * j]), scale_log2, -ms)) : 0.f;
-              const float p1 = c0 + 1 <= limit ? exp2f(fmaf(__uint_as_float(rr[2 * j + 1]), scale_log2, -ms)) : 0.f;
+              const float x0 = fmaf(__uint_as_float(rr[2 * j]), scale_log2, -ms);
+              const float x1 = fmaf(__uint_as_float(rr[2 * j + 1]), scale_log2, -ms);
+              const float p0 = ex2_approx(c0 <= limit ? x0 : -INFINITY);
+              const float p1 = ex2_approx(c0 + 1 <= limit ? x1 : -INFINITY);
               l += p0 + p1;
               pk[j] = pack_bf16x2(p0, p1);
             }

@@ -570,7 +570,7 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 32; ++q)
-              if (32 * c4 + q <= limit) mx = fmaxf(mx, __uint_as_float(rr[q]));
+              mx = fmaxf(mx, 32 * c4 + q <= limit ? __uint_as_float(rr[q]) : -INFINITY);
           }
         }
         const float mb = limit >= 0 ? mx * sl2 : -INFINITY;
@@ -598,8 +598,8 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             uint32_t pk[16];
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
-              const float p0 = exp2f(fmaf(__uint_as_float(rr[2 * q]), sl2, -m_new));
-              const float p1 = exp2f(fmaf(__uint_as_float(rr[2 * q + 1]), sl2, -m_new));
+              const float p0 = ex2_approx(fmaf(__uint_as_float(rr[2 * q]), sl2, -m_new));
+              const float p1 = ex2_approx(fmaf(__uint_as_float(rr[2 * q + 1]), sl2, -m_new));
               lsum += p0 + p1;
               pk[q] = pack_bf16x2(p0, p1);
             }
@@ -614,8 +614,10 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
               const int c0 = 32 * c4 + 2 * q;
-              const float p0 = c0 <= limit ? exp2f(fmaf(__uint_as_float(rr[2 * q]), sl2, -m_new)) : 0.f;
-              const float p1 = c0 + 1 <= limit ? exp2f(fmaf(__uint_as_float(rr[2 * q + 1]), sl2, -m_new)) : 0.f;
+              const float x0 = fmaf(__uint_as_float(rr[2 * q]), sl2, -m_new);
+              const float x1 = fmaf(__uint_as_float(rr[2 * q + 1]), sl2, -m_new);
+              const float p0 = ex2_approx(c0 <= limit ? x0 : -INFINITY);
+              const float p1 = ex2_approx(c0 + 1 <= limit ? x1 : -INFINITY);
               lsum += p0 + p1;
               pk[q] = pack_bf16x2(p0, p1);
             }
