@@ -340,7 +340,7 @@ def run_ours(args):
         if args.theta >= 0:
             return args.theta
         uq = 2 * (128 // max(w_.H // w_.G, 8))
-        return (3 * uq + 7) // 8
+        return (5 * uq + 7) // 8
     w = W.WORKLOADS[args.workload]
     # each rank runs an independent layer (its own seed): weak scaling
     wr = rank_workload(w, rank, W)

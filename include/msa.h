@@ -193,7 +193,7 @@ msa_status_t msa_dense_attn(const msa_shape_t* shape, const msa_varlen_t* seqs,
  * online softmax into one result per query, instead of one KV-outer partial
  * per (query, block).  The selected token sets and the exact softmax are the
  * same either way; only the rounding order differs.
- *   theta < 0   automatic: ceil(3/8 x tile queries) (the default)
+ *   theta < 0   automatic: ceil(5/8 x tile queries) (the default)
  *   theta == 0  off: every selection goes through the KV-outer lists
  *   theta >= 1  that threshold (1: every selected block of a tile)
  * Decode calls (one query per sequence) never use query tiles. */
