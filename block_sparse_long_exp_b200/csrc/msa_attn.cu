@@ -603,7 +603,9 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         if (lane == 0) mbar_arrive(&ctl->p_full[wg]);
         if (valid) {
           const int64_t unit = ((int64_t)(e / k) * G + R->g) * k + (e % k);
-          part_lse[unit * Hg + hi] = (ms + __log2f(l)) * 0.69314718055994530942f;
+          // write-once data: streaming stores (evict-first in L2), which keep the
+          // window's gathered Q rows resident
+          __stcs(part_lse + unit * Hg + hi, (ms + __log2f(l)) * 0.69314718055994530942f);
         }
         // the epilogue of tile tau-2 (same slot) has read row_sum[wg] once o_free fires
         if (!mbar_wait(&ctl->o_free[wg], ((tau >> 1) + 1) & 1)) {
@@ -661,7 +663,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
               w.y = pack_f16x2(__uint_as_float(rr[8 * j + 2]) * inv_l, __uint_as_float(rr[8 * j + 3]) * inv_l);
               w.z = pack_f16x2(__uint_as_float(rr[8 * j + 4]) * inv_l, __uint_as_float(rr[8 * j + 5]) * inv_l);
               w.w = pack_f16x2(__uint_as_float(rr[8 * j + 6]) * inv_l, __uint_as_float(rr[8 * j + 7]) * inv_l);
-              *reinterpret_cast<uint4*>(dst + (4 * c4 + j) * Hg * 8) = w;
+              __stcs(reinterpret_cast<uint4*>(dst + (4 * c4 + j) * Hg * 8), w);
             }
           }
         }
@@ -867,8 +869,8 @@ combine_kernel(const __half* __restrict__ part_acc, const float* __restrict__ pa
       o.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
       const int64_t t = pair / G;
       const int h = (int)(pair - t * G) * Hg + i;
-      *reinterpret_cast<uint4*>(out + (t * H + h) * d + 8 * cc) = o;
-      if (lse_out != nullptr && cc == 0) lse_out[t * H + h] = m_ + __logf(wsum);
+      __stcs(reinterpret_cast<uint4*>(out + (t * H + h) * d + 8 * cc), o);
+      if (lse_out != nullptr && cc == 0) __stcs(lse_out + t * H + h, m_ + __logf(wsum));
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&ctl.consumed[q]);

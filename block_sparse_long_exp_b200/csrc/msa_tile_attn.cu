@@ -722,7 +722,7 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 w.y = pack_bf16x2(__uint_as_float(rr[8 * q + 2]) * inv_l, __uint_as_float(rr[8 * q + 3]) * inv_l);
                 w.z = pack_bf16x2(__uint_as_float(rr[8 * q + 4]) * inv_l, __uint_as_float(rr[8 * q + 5]) * inv_l);
                 w.w = pack_bf16x2(__uint_as_float(rr[8 * q + 6]) * inv_l, __uint_as_float(rr[8 * q + 7]) * inv_l);
-                dst[q] = w;
+                __stcs(dst + q, w);            // write-once: evict-first in L2
               }
             } else {
               // partial layout per unit: [d/8 chunks][Hg heads][8 values]
@@ -734,16 +734,16 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 w.y = pack_f16x2(__uint_as_float(rr[8 * q + 2]) * inv_l, __uint_as_float(rr[8 * q + 3]) * inv_l);
                 w.z = pack_f16x2(__uint_as_float(rr[8 * q + 4]) * inv_l, __uint_as_float(rr[8 * q + 5]) * inv_l);
                 w.w = pack_f16x2(__uint_as_float(rr[8 * q + 6]) * inv_l, __uint_as_float(rr[8 * q + 7]) * inv_l);
-                *reinterpret_cast<uint4*>(dst + (4 * c4 + q) * Hg * 8) = w;
+                __stcs(reinterpret_cast<uint4*>(dst + (4 * c4 + q) * Hg * 8), w);
               }
             }
           }
         }
         if (has) {
           if (complete) {
-            if (p.lse != nullptr) p.lse[t * H + h] = lse_v;
+            if (p.lse != nullptr) __stcs(p.lse + t * H + h, lse_v);
           } else {
-            p.part_lse[unit * Hg + hi] = lse_v;
+            __stcs(p.part_lse + unit * Hg + hi, lse_v);
           }
         }
         tc_fence_before();

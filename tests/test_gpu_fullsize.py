@@ -83,7 +83,7 @@ def test_prefill_32k(M):
     w = W.WORKLOADS["prefill_n32768"]
     inp = W.make_inputs(w, "cuda")
     sel, out, lse = _run(M, w, inp)
-    rows = W.sample_rows([w.T], w.B_k, w.k, 1024, seed=101)
+    rows = W.sample_rows([w.T], w.B_k, w.k, 2048, seed=101)
     _check_rows(w, inp, sel, out, lse, rows)
     # every row's selection holds min(k, nb) ascending ids with the local block last
     s = sel.cpu().numpy()
@@ -102,7 +102,7 @@ def test_prefill_128k_hot(M):
     w = W.WORKLOADS["prefill_n131072_hot2"]
     inp = W.make_inputs(w, "cuda")
     sel, out, lse = _run(M, w, inp)
-    rows = W.sample_rows([w.T], w.B_k, w.k, 2048, seed=102, hot_blocks=inp["hot_blocks"])
+    rows = W.sample_rows([w.T], w.B_k, w.k, 4096, seed=102, hot_blocks=inp["hot_blocks"])
     _check_rows(w, inp, sel, out, lse, rows)
 
 
@@ -117,6 +117,6 @@ def test_prefill_1m_hot_chunked(M):
     w = W.WORKLOADS["prefill_n1048576_hot2"]
     inp = W.make_inputs(w, "cuda")
     sel, out, lse = _run(M, w, inp, q_chunk=131072)
-    rows = W.sample_rows([w.T], w.B_k, w.k, 1024, seed=104, hot_blocks=None)
+    rows = W.sample_rows([w.T], w.B_k, w.k, 4096, seed=104, hot_blocks=None)
     rows = sorted(set(rows) | {131071, 131072, 2 * 131072 + 5})   # rows at pass boundaries
     _check_rows(w, inp, sel, out, lse, rows)
