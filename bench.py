@@ -218,11 +218,21 @@ def traffic_for(kernel):
     d = json.load(open(p)).get(kernel)
     if not d:
         return None
-    src = os.path.join(ROOT, "block_sparse_long_exp_b200", "csrc", d.get("source", ""))
-    if not os.path.exists(src):
-        return None
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return d.get("dram_bytes_per_launch") if sha == d.get("source_sha") else None
+    sha = kernel_source_sha(d.get("source", ""))
+    return d.get("dram_bytes_per_launch") if sha is not None and sha == d.get("source_sha") else None
+
+
+def kernel_source_sha(source):
+    """Hash of a kernel's .cu file together with the headers every kernel
+    includes (a change to either makes recorded counters stale)."""
+    csrc = os.path.join(ROOT, "block_sparse_long_exp_b200", "csrc")
+    h = hashlib.sha256()
+    for f in (source, "msa_common.cuh", "msa_internal.h"):
+        p = os.path.join(csrc, f)
+        if not f or not os.path.exists(p):
+            return None
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
 
 
 # ------------------------------------------------------------- CPU oracle ---

@@ -12,7 +12,7 @@ namespace msa {
 constexpr int kBk = 128;          // block size the kernels are built for
 constexpr int kMaxK = 32;         // largest k
 constexpr int kMaxBatchTiles = 1024;  // sequences per prefill index launch
-constexpr int kWindow = 1024;         // query rows per attention planning window
+constexpr int kWindow = 4096;         // query rows per attention planning window (KV-outer lists)
 constexpr int kScanTile = 4096;       // keys per CTA of the planning scan
 constexpr int kMaxItemQueries = 64;   // queries per attention work item (upper bound)
 constexpr int kMaxDense = 64;         // dense blocks per query tile (Q-outer side)
