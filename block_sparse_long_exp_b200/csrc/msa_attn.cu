@@ -754,24 +754,47 @@ combine_kernel(const __half* __restrict__ part_acc, const float* __restrict__ pa
 
   if (warp == 2 * kCombGroupThreads / 32) {
     // ------------------------------------------------------------ producer
-    if (lane != 0) return;
+    // The whole warp loads the list entries of 32 chunks ahead (lane l: chunk
+    // m0 + l); lane 0 allocates ring space, waits and issues the copies.
+    auto load_batch = [&](int64_t m0, uint2 (&dst)[kCombMaxPairs]) {
+      const int64_t mm = m0 + lane;
+      const int64_t p0 = (blockIdx.x + mm * gridDim.x) * P;
+#pragma unroll
+      for (int i = 0; i < kCombMaxPairs; ++i) {
+        dst[i] = make_uint2(0u, 0u);
+        if (i < P && mm < my && p0 + i < npairs)
+          dst[i] = clist != nullptr ? clist[p0 + i] : make_uint2((uint32_t)(p0 + i), (uint32_t)k);
+      }
+    };
+    uint2 cur[kCombMaxPairs], nxt[kCombMaxPairs];
+    load_batch(0, cur);
+    load_batch(32, nxt);
     uint64_t alloc = 0, freed = 0;              // virtual ring offsets (physical = virtual % ring)
-    int64_t oldest = 0, m = 0;
+    int64_t oldest = 0, m = 0, issued = 0;      // issued: chunks whose copies were started (lane 0)
     bool ok = true;
-    for (; m < my && ok && !*abort_flag; ++m) {
+    for (; m < my; ++m) {
+      bool go = lane == 0 ? (ok && !*abort_flag) : true;
+      go = __shfl_sync(0xffffffffu, go ? 1 : 0, 0) != 0;
+      if (!go) break;
+      if (m > 0 && (m & 31) == 0) {
+#pragma unroll
+        for (int i = 0; i < kCombMaxPairs; ++i) cur[i] = nxt[i];
+        load_batch(m + 32, nxt);
+      }
+      uint2 ent[kCombMaxPairs];
+#pragma unroll
+      for (int i = 0; i < kCombMaxPairs; ++i) {
+        ent[i].x = __shfl_sync(0xffffffffu, cur[i].x, (int)(m & 31));
+        ent[i].y = __shfl_sync(0xffffffffu, cur[i].y, (int)(m & 31));
+      }
+      if (lane != 0) continue;
       const int q = (int)(m % kCombQueue);
       const int64_t p0 = (blockIdx.x + m * gridDim.x) * P;
       const int np = npairs - p0 < P ? (int)(npairs - p0) : P;
-      uint2 ent[kCombMaxPairs];
       uint32_t bytes = 0;
 #pragma unroll
-      for (int i = 0; i < kCombMaxPairs; ++i) {
-        ent[i] = make_uint2(0u, 0u);
-        if (i < np) {
-          ent[i] = clist != nullptr ? clist[p0 + i] : make_uint2((uint32_t)(p0 + i), (uint32_t)k);
-          bytes += ent[i].y * (slot_bytes + slot_lse);
-        }
-      }
+      for (int i = 0; i < kCombMaxPairs; ++i)
+        if (i < np) bytes += ent[i].y * (slot_bytes + slot_lse);
       // contiguous room in the ring (skip the ring's tail end when it is too short)
       const uint64_t phys = alloc % kCombRing;
       if (phys + bytes > kCombRing) alloc += kCombRing - phys;
@@ -785,7 +808,7 @@ combine_kernel(const __half* __restrict__ part_acc, const float* __restrict__ pa
         ok = mbar_wait(&ctl.consumed[qo], (uint32_t)((oldest / kCombQueue) & 1));
         if (ok) { freed = ctl.end_of[qo]; ++oldest; }
       }
-      if (!ok) break;
+      if (!ok) continue;                        // the next iteration's check ends the loop
       // entry q is free (its previous chunk was consumed): publish this chunk in it
       CombEntry& E = ctl.e[q];
       uint32_t off = (uint32_t)(alloc % kCombRing);
@@ -805,13 +828,16 @@ combine_kernel(const __half* __restrict__ part_acc, const float* __restrict__ pa
       }
       alloc += bytes;
       ctl.end_of[q] = alloc;
+      issued = m + 1;
     }
-    if (!ok) {
-      report_error(err, MSA_ERR_TIMEOUT, kSiteAttnLoad, (int)m, -2);
-      *abort_flag = 1;
+    if (lane == 0) {
+      if (!ok) {
+        report_error(err, MSA_ERR_TIMEOUT, kSiteAttnLoad, (int)m, -2);
+        *abort_flag = 1;
+      }
+      // no bulk copy may still be writing when the CTA exits
+      for (int64_t j = oldest; j < issued; ++j) mbar_wait(&ctl.full[j % kCombQueue], (uint32_t)((j / kCombQueue) & 1));
     }
-    // no bulk copy may still be writing when the CTA exits
-    for (int64_t j = oldest; j < m; ++j) mbar_wait(&ctl.full[j % kCombQueue], (uint32_t)((j / kCombQueue) & 1));
     return;
   }
 

@@ -32,8 +32,8 @@
 //   warp 0      claims units (atomic ticket) and publishes them in a 2-deep
 //               shared-memory ring;
 //   warp 1      owns TMEM (512 columns: per MMA tile 128 columns S/P + d columns
-//               O); its lane 0 issues S = Q K^T;
-//   warp 2      lane 0 issues O += P V;
+//               O); its lane 0 issues every MMA (S = Q K^T and O += P V of both
+//               tiles, interleaved; warp 2 is idle);
 //   warp 3      lane 0 TMA-loads the unit's Q tiles and every K / V block
 //               (two stages);
 //   warps 4-7   online softmax of MMA tile 0, warps 8-11 of MMA tile 1: S -> P
@@ -54,7 +54,7 @@ namespace {
 
 constexpr int kTileThreads = 512;
 constexpr int kUnitRing = 2;
-constexpr int kUnitEmptyCount = 15;      // S + PV issuers, loader, 8 softmax warps, 4 epilogue warps
+constexpr int kUnitEmptyCount = 14;      // MMA issuer, loader, 8 softmax warps, 4 epilogue warps
 constexpr float kRescaleLog2 = 8.f;      // rescale O only when the row max grows by more than 2^8
 constexpr int kPlanWarps = 4;
 constexpr int kPlanMaxEntries = 1024;    // UQ x k <= 32 x 32
@@ -430,10 +430,13 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       for (int x = 0; x < 2; ++x)
         if (uq[x] > 0) mbar_wait(&ctl->q_full[x], (uq[x] - 1) & 1);
     }
-  } else if (warp == 1 || warp == 2) {
-    // -------------------------------------------------------- MMA issuers
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    // One thread issues every MMA, interleaving the two tiles: S0(j), PV1(j-1),
+    // S1(j), PV0(j), S0(j+1), ...  tcgen05.mma operations of one thread run in
+    // issue order, so S(j+1) may overwrite the columns that PV(j) reads as P
+    // right after PV(j) is issued (no wait for its completion).
     if (lane == 0) {
-      const bool is_s = (warp == 1);
       const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       const uint32_t idesc_o = idesc_bf16_f32(128, d, 0, 1);
       const uint64_t qdesc0 = make_sdesc(smem_u32(q_s), 16, 1024, kSw128);
@@ -442,6 +445,30 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       int n = 0, ut[2] = {0, 0};
       int64_t kvc = 0, bt[2] = {0, 0};
       bool ok = true;
+      auto issue_s = [&](int x, int st) {
+        const uint64_t qd = qdesc0 + (uint64_t)((x * tile_bytes) >> 4);
+        const uint64_t kd = kdesc0 + (uint64_t)((st * 2 * tile_bytes) >> 4);
+        for (int kk = 0; kk < d / 16; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
+          umma_bf16_ss(tmem + x * 256, qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&ctl->s_full[x]);
+      };
+      // PV of tile x for its block j (stage st): waits for P (and, on a unit's
+      // first block, for the epilogue to have read O)
+      auto issue_pv = [&](int x, int j, int st) -> bool {
+        if (!mbar_wait(&ctl->p_full[x], (uint32_t)(bt[x] & 1)) ||
+            (j == 0 && !mbar_wait(&ctl->o_free[x], (ut[x] + 1) & 1)))
+          return false;
+        tc_fence_after();
+        const uint64_t vd = vdesc0 + (uint64_t)((st * 2 * tile_bytes) >> 4);
+        const uint32_t pcol = tmem + x * 256, ocol = pcol + 128;
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16_ts(ocol, pcol + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&ctl->pv_done[x]);
+        ++bt[x];
+        return true;
+      };
       while (ok && !*abort_flag) {
         const TileUnit* R = wait_unit(n);
         if (R == nullptr) { ok = false; break; }
@@ -450,50 +477,33 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         if (nblk < 0) break;
         for (int j = 0; j < nblk && ok; ++j, ++kvc) {
           const int st = (int)(kvc & 1);
-          if (is_s) {
-            if (!mbar_wait(&ctl->k_full[st], (uint32_t)((kvc >> 1) & 1))) { ok = false; break; }
-            const uint64_t kd = kdesc0 + (uint64_t)((st * 2 * tile_bytes) >> 4);
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-              if (x >= ntl || !ok) continue;
-              // S(x) overwrites the P(x) that the previous PV(x) read
-              if ((j == 0 && !mbar_wait(&ctl->q_full[x], ut[x] & 1)) ||
-                  !mbar_wait(&ctl->pv_done[x], (uint32_t)((bt[x] + 1) & 1))) {
-                ok = false;
-                continue;
-              }
-              tc_fence_after();
-              const uint64_t qd = qdesc0 + (uint64_t)((x * tile_bytes) >> 4);
-              for (int kk = 0; kk < d / 16; ++kk) {
-                const uint64_t off = (uint64_t)(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
-                umma_bf16_ss(tmem + x * 256, qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
-              }
-              umma_commit(&ctl->s_full[x]);
-              if (j == nblk - 1) umma_commit(&ctl->q_empty[x]);
-              ++bt[x];
-            }
-          } else {
-            if (!mbar_wait(&ctl->v_full[st], (uint32_t)((kvc >> 1) & 1))) { ok = false; break; }
-            const uint64_t vd = vdesc0 + (uint64_t)((st * 2 * tile_bytes) >> 4);
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-              if (x >= ntl || !ok) continue;
-              if (!mbar_wait(&ctl->p_full[x], (uint32_t)(bt[x] & 1)) ||
-                  (j == 0 && !mbar_wait(&ctl->o_free[x], (ut[x] + 1) & 1))) {
-                ok = false;
-                continue;
-              }
-              tc_fence_after();
-              const uint32_t pcol = tmem + x * 256, ocol = pcol + 128;
-              for (int kk = 0; kk < 8; ++kk)
-                umma_bf16_ts(ocol, pcol + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_o,
-                             (j > 0 || kk > 0) ? 1u : 0u);
-              umma_commit(&ctl->pv_done[x]);
-              ++bt[x];
-            }
-            // K was read by S MMAs that completed before P existed; V by these
-            if (ok) umma_commit(&ctl->kv_empty[st]);
+          if (!mbar_wait(&ctl->k_full[st], (uint32_t)((kvc >> 1) & 1)) ||
+              !mbar_wait(&ctl->v_full[st], (uint32_t)((kvc >> 1) & 1)) ||
+              (j == 0 && !mbar_wait(&ctl->q_full[0], ut[0] & 1))) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          issue_s(0, st);
+          if (j == nblk - 1) umma_commit(&ctl->q_empty[0]);
+          if (ntl == 2) {
+            if (j > 0) {
+              // tile 1's PV of the previous block; then both tiles are done with it
+              if (!issue_pv(1, j - 1, st ^ 1)) { ok = false; break; }
+              umma_commit(&ctl->kv_empty[st ^ 1]);
+            }
+            if (j == 0 && !mbar_wait(&ctl->q_full[1], ut[1] & 1)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(1, st);
+            if (j == nblk - 1) umma_commit(&ctl->q_empty[1]);
+          }
+          if (!issue_pv(0, j, st)) { ok = false; break; }
+          if (ntl == 1) umma_commit(&ctl->kv_empty[st]);
+        }
+        if (ok && ntl == 2 && nblk > 0) {
+          const int st = (int)((kvc - 1) & 1);
+          if (!issue_pv(1, nblk - 1, st)) ok = false;
+          else umma_commit(&ctl->kv_empty[st]);
         }
 #pragma unroll
         for (int x = 0; x < 2; ++x)
@@ -501,11 +511,11 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         ++n;
       }
       if (!ok) {
-        report_error(p.err, MSA_ERR_TIMEOUT, kSiteTileMma, n, is_s ? 0 : 1);
+        report_error(p.err, MSA_ERR_TIMEOUT, kSiteTileMma, n, 0);
         *abort_flag = 1;
       }
-      umma_commit(&ctl->mma_done[is_s ? 0 : 1]);
-      mbar_wait(&ctl->mma_done[is_s ? 0 : 1], 0);
+      umma_commit(&ctl->mma_done[0]);
+      mbar_wait(&ctl->mma_done[0], 0);
     }
   } else if (warp >= 4 && warp < 12) {
     // ----------------------------------------------------- online softmax
