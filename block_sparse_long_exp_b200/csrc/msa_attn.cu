@@ -245,9 +245,9 @@ __global__ void __launch_bounds__(kScanThreads) scan_items_kernel(const int32_t*
 //               gathers each 128-row tile's query rows with one TMA box per
 //               (query, 64-column half) into one of three Q slots;
 //   warp 1      owns TMEM (512 columns = two slots of S/P + O); its lane 0
-//               issues S = Q K^T, lane 0 of warp 2 issues O = P V (two
-//               issue/commit streams keep the tensor core fed while tile t's
-//               softmax runs);
+//               issues every MMA, PV one tile behind S (S(t), PV(t-1), ...),
+//               so the tensor core works on the next tile while tile t's
+//               softmax runs (warps 2 and 3 are idle);
 //   warps 4-7   softmax of even tiles (TMEM slot 0), warps 8-11 of odd tiles
 //               (slot 1): S -> P (bf16, written back into the S columns, the A
 //               operand of the PV MMA); each row's max and sum go to shared
@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_items_kernel(const int32_t*
 constexpr int kAttnThreads = 512;
 constexpr int kItemRing = 4;
 constexpr int kQSlots = 3;
-constexpr int kItemEmptyCount = 14;   // MMA issuers 2 + softmax warps 8 + epilogue warps 4
+constexpr int kItemEmptyCount = 13;   // MMA issuer 1 + softmax warps 8 + epilogue warps 4
 
 struct __align__(16) RingItem {
   int32_t seq, blk, g, start, count, Tb, Sb, qrow0;
@@ -433,15 +433,13 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         if (issued > 0) mbar_wait(&ctl->q_full[qs], (issued - 1) & 1);
       }
     }
-  } else if (warp == 1 || warp == 2) {
-    // -------------------------------------------------------- MMA issuers
-    // lane 0 of warp 1 issues every S = Q K^T, lane 0 of warp 2 every O = P V,
-    // each with its own commit stream (a thread that mixes commits into its
-    // MMAs issues at about half the MMA rate).  The two streams are not
-    // ordered against each other, so S(t) waits for PV(t-2) to complete
-    // before it overwrites slot t%2, whose first 64 columns hold P(t-2).
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    // One thread issues every MMA, one tile behind for PV: S(t), PV(t-1),
+    // S(t+1), PV(t), ...  tcgen05.mma operations of one thread run in issue
+    // order, so S(t) may overwrite slot t%2, whose first 64 columns hold the
+    // P(t-2) that PV(t-2) read, as soon as PV(t-2) has been issued.
     if (lane == 0) {
-      const bool is_s = (warp == 1);
       const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       const uint32_t idesc_o = idesc_bf16_f32(128, d, 0, 1);
       // descriptors built once; per-slot / per-step byte offsets (>> 4) are added
@@ -450,6 +448,22 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       const uint64_t vdesc0 = make_sdesc(smem_u32(kv_s + tile_bytes), 128 * 128, 1024, kSw128);
       int n = 0, tau = 0;
       bool ok = true;
+      bool pend = false, pend_last = false;     // PV of tile tau-1 not yet issued
+      int pend_st = 0;
+      // PV of tile t (K/V stage st); the item's last tile releases the stage
+      auto issue_pv = [&](int t, int st, bool last) -> bool {
+        const int s = t & 1;
+        if (!mbar_wait(&ctl->p_full[s], (t >> 1) & 1) || !mbar_wait(&ctl->o_free[s], ((t >> 1) + 1) & 1))
+          return false;
+        tc_fence_after();
+        const uint64_t vd = vdesc0 + (uint64_t)((st * 2 * tile_bytes) >> 4);
+        const uint32_t pcol = tmem + s * 256, ocol = pcol + 128;
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16_ts(ocol, pcol + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : 0u);
+        umma_commit(&ctl->o_full[s]);
+        if (last) umma_commit(&ctl->kv_empty[st]);
+        return true;
+      };
       while (ok && !*abort_flag) {
         const RingItem* R = wait_item(n);
         if (R == nullptr) { ok = false; break; }
@@ -460,47 +474,38 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         const int ntiles = (cnt + qpt - 1) / qpt;
         for (int mt = 0; mt < ntiles && ok; ++mt, ++tau) {
           const int s = tau & 1;
-          if (is_s) {
-            const int qs = tau % kQSlots;
-            if (!mbar_wait(&ctl->q_full[qs], (tau / kQSlots) & 1) ||
-                (mt == 0 && !mbar_wait(&ctl->kv_full[st], (n >> 1) & 1)) ||
-                !mbar_wait(&ctl->o_full[s], ((tau >> 1) + 1) & 1)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint64_t qd = qdesc0 + (uint64_t)((qs * tile_bytes) >> 4);
-            const uint64_t kd = kvdesc0 + (uint64_t)((st * 2 * tile_bytes) >> 4);
-            for (int kk = 0; kk < d / 16; ++kk) {
-              const uint64_t off = (uint64_t)(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
-              umma_bf16_ss(tmem + s * 256, qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
-            }
-            umma_commit(&ctl->s_full[s]);
-            umma_commit(&ctl->q_empty[qs]);
-          } else {
-            if (!mbar_wait(&ctl->p_full[s], (tau >> 1) & 1) ||
-                !mbar_wait(&ctl->o_free[s], ((tau >> 1) + 1) & 1)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint64_t vd = vdesc0 + (uint64_t)((st * 2 * tile_bytes) >> 4);
-            const uint32_t pcol = tmem + s * 256, ocol = pcol + 128;
-            for (int kk = 0; kk < 8; ++kk)
-              umma_bf16_ts(ocol, pcol + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : 0u);
-            umma_commit(&ctl->o_full[s]);
-            // K was read by S MMAs that completed before P existed; V by these
-            if (mt == ntiles - 1) umma_commit(&ctl->kv_empty[st]);
+          const int qs = tau % kQSlots;
+          if (!mbar_wait(&ctl->q_full[qs], (tau / kQSlots) & 1) ||
+              (mt == 0 && !mbar_wait(&ctl->kv_full[st], (n >> 1) & 1))) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          const uint64_t qd = qdesc0 + (uint64_t)((qs * tile_bytes) >> 4);
+          const uint64_t kd = kvdesc0 + (uint64_t)((st * 2 * tile_bytes) >> 4);
+          for (int kk = 0; kk < d / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
+            umma_bf16_ss(tmem + s * 256, qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&ctl->s_full[s]);
+          umma_commit(&ctl->q_empty[qs]);
+          if (pend && !issue_pv(tau - 1, pend_st, pend_last)) {
+            ok = false;
+            break;
+          }
+          pend = true;
+          pend_st = st;
+          pend_last = (mt == ntiles - 1);
         }
         ++n;
       }
+      if (ok && pend && !issue_pv(tau - 1, pend_st, pend_last)) ok = false;
       if (!ok) {
-        report_error(err, MSA_ERR_TIMEOUT, kSiteAttnMma, tau, is_s ? 0 : 1);
+        report_error(err, MSA_ERR_TIMEOUT, kSiteAttnMma, tau, 0);
         *abort_flag = 1;
       }
-      umma_commit(&ctl->mma_done[is_s ? 0 : 1]);
-      mbar_wait(&ctl->mma_done[is_s ? 0 : 1], 0);
+      umma_commit(&ctl->mma_done[0]);
+      mbar_wait(&ctl->mma_done[0], 0);
     }
   } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ softmax
