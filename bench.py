@@ -501,7 +501,7 @@ def run_ours(args):
         L = [dinp["cu_k_host"][i + 1] - dinp["cu_k_host"][i] for i in range(wd.batch)]
         dw = R.decode_work(L, wd.H, wd.G, wd.d, wd.d_idx, wd.B_k, wd.k)
         dk = {}
-        for name in ("decode_scan", "decode_select", "sparse_attn", "combine", "count", "scatter", "plan"):
+        for name in ("decode_scan", "decode_select", "rows_attn", "sparse_attn", "combine", "count", "scatter", "plan"):
             kms, n = msa.msa_profile_read(name)
             if n:
                 dk[name] = {"ms_per_launch": kms / n, "launches": n}

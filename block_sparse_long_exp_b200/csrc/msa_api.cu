@@ -156,7 +156,10 @@ msa_status_t attn_common(const msa_shape_t* shape, const msa_varlen_t* seqs, con
   for (int64_t t0 = 0; t0 < seqs->total_q; t0 += rows) {
     a.t0 = t0;
     a.t1 = t0 + rows < seqs->total_q ? t0 + rows : seqs->total_q;
-    if (launch_sparse_attn_pass(a, stream) != 0) return MSA_ERR_CUDA;
+    // one query per sequence: each (query, group) attends its selected blocks
+    // query-major (no lists, partials or combine)
+    const int rc = seqs->max_q_len <= 1 ? launch_rows_attn(a, stream) : launch_sparse_attn_pass(a, stream);
+    if (rc != 0) return MSA_ERR_CUDA;
   }
   return MSA_OK;
 }

@@ -127,6 +127,7 @@ int tile_queries(int H, int G);        // query rows per tile unit
 int tile_default_theta(int UQ);
 int launch_tile_plan(const AttnArgs& a, int theta, void* stream);
 int launch_tile_attn(const AttnArgs& a, void* stream);
+int launch_rows_attn(const AttnArgs& a, void* stream);   // one query per unit (decode)
 
 struct DenseArgs {
   const void* q;

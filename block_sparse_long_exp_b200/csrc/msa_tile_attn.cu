@@ -42,9 +42,11 @@
 //               (only then);
 //   warps 12-15 epilogue: O / l -> bf16 output (or an f16 partial) and the
 //               log-sum-exp.
-// In dense mode (kDense) a unit's blocks are 0 .. the last query's block and a
-// row attends every key at or before its position: dense causal GQA, the
-// baseline of the pages' speedup comparison (pnsm.cn sec. 9).
+// In dense mode a unit's blocks are 0 .. the last query's block and a row
+// attends every key at or before its position: dense causal GQA, the baseline
+// of the pages' speedup comparison (pnsm.cn sec. 9).  In rows mode a unit is
+// one query and its selection row (decode: one query per sequence), written
+// straight to the output.
 #include <climits>
 
 #include "msa_common.cuh"
@@ -57,6 +59,14 @@ constexpr int kUnitRing = 2;
 constexpr int kUnitEmptyCount = 14;      // MMA issuer, loader, 8 softmax warps, 4 epilogue warps
 constexpr float kRescaleLog2 = 8.f;      // rescale O only when the row max grows by more than 2^8
 constexpr int kPlanWarps = 4;
+
+// What a unit is (template argument of tile_attn_kernel):
+//   kModeTiles  a tile of UQ queries and its dense blocks (tile_plan_kernel);
+//   kModeDense  a tile of UQ queries and every block up to its last query
+//               (dense causal GQA);
+//   kModeRows   one query and the blocks of its selection row (decode: the
+//               Q-outer form of a single query, no partials).
+constexpr int kModeTiles = 0, kModeDense = 1, kModeRows = 2;
 constexpr int kPlanMaxEntries = 1024;    // UQ x k <= 32 x 32
 
 __device__ __forceinline__ int find_seq_t(const int32_t* __restrict__ cu, int batch, int64_t row) {
@@ -223,7 +233,9 @@ struct TileParams {
   const uint64_t* dmember;    // hybrid: [rows x G] dense-list membership bits
   const int32_t* dstate;      // hybrid: [rows x G] kDenseComplete | first covered slot, or -1
   const int32_t* seq_units;   // dense: [batch + 1] prefix of units per sequence
-  const int32_t* nunits;      // device count of units (hybrid: listed units; dense: all)
+  const int32_t* nunits;      // device count of units (tiles: listed units; dense: all); null: nunits_host
+  int64_t nunits_host;        // rows mode: rows x G
+  const int32_t* sel;         // rows mode: [T, G, k]
   int32_t* ticket;
   const int32_t* cu_q;
   const int32_t* cu_k;
@@ -237,7 +249,7 @@ struct TileParams {
   DevError* err;
 };
 
-template <bool kDense>
+template <int kMode>
 __global__ void __launch_bounds__(kTileThreads, 1)
 tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ TileParams p) {
@@ -301,7 +313,7 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 
   if (warp == 0) {
     // ------------------------------------------------------------ scheduler
-    const int64_t nun = *p.nunits;
+    const int64_t nun = p.nunits != nullptr ? (int64_t)*p.nunits : p.nunits_host;
     int n = 0;
     while (true) {
       const int slot = n % kUnitRing;
@@ -326,7 +338,14 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       }
       int32_t uid, g, nq, nblk, seq;
       int64_t r0;
-      if (kDense) {
+      if (kMode == kModeRows) {
+        const int64_t t = p.t0 + it / G;
+        g = (int)(it - (t - p.t0) * G);
+        r0 = t;
+        nq = 1;
+        seq = find_seq_t(p.cu_q, p.batch, r0);
+        uid = (int32_t)it;
+      } else if (kMode == kModeDense) {
         // longest units first: reverse order (the last tiles of a sequence see the most blocks)
         const int64_t v = nun - 1 - it;
         const int64_t tg = v / G;
@@ -351,7 +370,22 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       }
       const int Tb = p.cu_q[seq + 1] - p.cu_q[seq];
       const int Sb = p.cu_k[seq + 1] - p.cu_k[seq];
-      if (kDense) {
+      if (kMode == kModeRows) {
+        // the selection row: valid ids first, then -1 padding
+        const int32_t b = lane < p.k ? p.sel[(r0 * G + g) * p.k + lane] : -1;
+        const unsigned v = __ballot_sync(0xffffffffu, b >= 0);
+        nblk = __popc(v);
+        const int64_t pos = (int64_t)Sb - Tb + (r0 - p.cu_q[seq]);
+        if (b >= 0) {
+          U->blk[lane] = b;
+          if (Tb > Sb || b > pos / kBk) report_error(p.err, MSA_ERR_DEVICE_CHECK, kSiteInvert, (int)r0, b);
+        }
+        if (v != (nblk >= 32 ? 0xffffffffu : (1u << nblk) - 1u)) {
+          // ids must come first: anything else is not a selection row
+          if (lane == 0) report_error(p.err, MSA_ERR_DEVICE_CHECK, kSiteInvert, (int)r0, -1);
+          nblk = 0;
+        }
+      } else if (kMode == kModeDense) {
         const int64_t pos_last = (int64_t)Sb - Tb + (r0 + nq - 1 - p.cu_q[seq]);
         nblk = (int)(pos_last / kBk) + 1;
         if (Tb > Sb) {
@@ -401,7 +435,7 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
           const int st = (int)(kvc & 1);
           ok = mbar_wait(&ctl->kv_empty[st], ((kvc >> 1) + 1) & 1);
           if (!ok) break;
-          const int blk = kDense ? j : R->blk[j];
+          const int blk = kMode == kModeDense ? j : R->blk[j];
           const int krow = kbase + blk * kBk;
           uint8_t* ks = kv_s + st * 2 * tile_bytes;
           mbar_arrive_expect_tx(&ctl->k_full[st], tile_bytes);
@@ -541,12 +575,12 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       const int64_t pos = valid ? (int64_t)R->Sb - R->Tb + (t - R->qrow0) : -1;
       const int lb = valid ? (int)(pos / kBk) : -1;
       uint64_t mem = 0;
-      if (!kDense && valid) mem = p.dmember[(t - p.t0) * G + R->g];
+      if (kMode == kModeTiles && valid) mem = p.dmember[(t - p.t0) * G + R->g];
       float m_run = -INFINITY, l_run = 0.f;
       bool failed = false;
       for (int j = 0; j < nblk; ++j, ++bt) {
-        const int blk = kDense ? j : R->blk[j];
-        const bool member = valid && (kDense || ((mem >> j) & 1ull)) && blk <= lb;
+        const int blk = kMode == kModeDense ? j : R->blk[j];
+        const bool member = valid && (kMode != kModeTiles || ((mem >> j) & 1ull)) && blk <= lb;
         int limit = -1;                          // last attended key of the block, -1: none
         if (member) limit = blk < lb ? kBk - 1 : (int)(pos - (int64_t)blk * kBk);
         if (!mbar_wait(&ctl->s_full[x], (uint32_t)(bt & 1))) {
@@ -708,7 +742,7 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         tc_fence_after();
         const float l = ctl->row_l[x][r], m = ctl->row_m[x][r];
         int32_t state = kDenseComplete;
-        if (!kDense && valid) state = p.dstate[(t - p.t0) * G + g];
+        if (kMode == kModeTiles && valid) state = p.dstate[(t - p.t0) * G + g];
         const bool has = valid && l > 0.f && state >= 0;
         const bool complete = (state & kDenseComplete) != 0;
         const float inv_l = has ? 1.f / l : 0.f;
@@ -796,18 +830,18 @@ int make_tile_maps(CUtensorMap* tm_k, CUtensorMap* tm_v, CUtensorMap* tm_q, cons
   return make_tmap_bf16(tm_q, q, 3, dims, strides, box, 128);
 }
 
-template <bool kDense>
+template <int kMode>
 int launch_tile_attn_kernel(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_q,
                             const TileParams& prm, cudaStream_t st) {
   const size_t smem = 1024 + 6 * (size_t)128 * prm.d * 2 + sizeof(TileCtl);
   static_assert(1024 + 6 * 128 * 128 * 2 + sizeof(TileCtl) <= 227 * 1024, "shared memory budget (d = 128)");
   cudaError_t e =
-      cudaFuncSetAttribute(tile_attn_kernel<kDense>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cudaFuncSetAttribute(tile_attn_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return (int)e;
   int dev = 0, nsm = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  tile_attn_kernel<kDense><<<nsm, kTileThreads, smem, st>>>(tm_k, tm_v, tm_q, prm);
+  tile_attn_kernel<kMode><<<nsm, kTileThreads, smem, st>>>(tm_k, tm_v, tm_q, prm);
   return (int)cudaGetLastError();
 }
 
@@ -852,7 +886,30 @@ int launch_tile_attn(const AttnArgs& a, void* stream) {
   prm.part_lse = a.part_lse;
   prm.err = a.err;
   ProfScope ps("tile_attn", stream);
-  return launch_tile_attn_kernel<false>(tm_k, tm_v, tm_q, prm, st);
+  return launch_tile_attn_kernel<kModeTiles>(tm_k, tm_v, tm_q, prm, st);
+}
+
+int launch_rows_attn(const AttnArgs& a, void* stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t rows = a.t1 - a.t0;
+  if (rows <= 0) return 0;
+  cudaError_t e = cudaMemsetAsync(a.tile_ctr, 0, sizeof(int32_t) * 4, st);
+  if (e != cudaSuccess) return (int)e;
+  alignas(64) CUtensorMap tm_k, tm_v, tm_q;
+  int rc = make_tile_maps(&tm_k, &tm_v, &tm_q, a.q, a.key, a.value, a.total_q, a.total_k, a.H, a.G, a.d);
+  if (rc) return rc;
+  TileParams prm{};
+  prm.nunits = nullptr; prm.nunits_host = rows * a.G; prm.ticket = a.tile_ctr + 2;
+  prm.sel = a.sel;
+  prm.cu_q = a.cu_q; prm.cu_k = a.cu_k;
+  prm.batch = a.batch; prm.H = a.H; prm.G = a.G; prm.d = a.d; prm.k = a.k; prm.UQ = 1;
+  prm.scale_log2 = a.sm_scale * 1.4426950408889634f;
+  prm.t0 = a.t0; prm.t1 = a.t1;
+  prm.out = reinterpret_cast<__nv_bfloat16*>(a.out);
+  prm.lse = a.lse;
+  prm.err = a.err;
+  ProfScope ps("rows_attn", stream);
+  return launch_tile_attn_kernel<kModeRows>(tm_k, tm_v, tm_q, prm, st);
 }
 
 size_t dense_scratch_bytes(int32_t batch) { return align_up(sizeof(int32_t) * (batch + 1), 256) + 256; }
@@ -883,7 +940,7 @@ int launch_dense_attn(const DenseArgs& a, void* stream) {
   prm.lse = a.lse;
   prm.err = a.err;
   ProfScope ps("dense_attn", stream);
-  return launch_tile_attn_kernel<true>(tm_k, tm_v, tm_q, prm, st);
+  return launch_tile_attn_kernel<kModeDense>(tm_k, tm_v, tm_q, prm, st);
 }
 
 }  // namespace msa
