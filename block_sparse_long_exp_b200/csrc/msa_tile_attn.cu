@@ -216,7 +216,7 @@ struct __align__(16) TileCtl {
   uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[2], v_full[2], kv_empty[2];
-  uint64_t s_full[2], p_full[2], pv_done[2], o_free[2], stats_full[2];
+  uint64_t s_full[2], p_half[2], p_full[2], pv_done[2], o_free[2], stats_full[2];
   uint64_t mma_done[2];
   uint32_t tmem_base;
   int32_t abort_flag;
@@ -277,7 +277,7 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl->q_full[i], 1); mbar_init(&ctl->q_empty[i], 1);
       mbar_init(&ctl->k_full[i], 1); mbar_init(&ctl->v_full[i], 1); mbar_init(&ctl->kv_empty[i], 1);
-      mbar_init(&ctl->s_full[i], 1); mbar_init(&ctl->p_full[i], 4);
+      mbar_init(&ctl->s_full[i], 1); mbar_init(&ctl->p_half[i], 4); mbar_init(&ctl->p_full[i], 4);
       mbar_init(&ctl->pv_done[i], 1); mbar_init(&ctl->o_free[i], 4);
       mbar_init(&ctl->stats_full[i], 4);
       mbar_init(&ctl->mma_done[i], 1);
@@ -491,14 +491,19 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       // PV of tile x for its block j (stage st): waits for P (and, on a unit's
       // first block, for the epilogue to have read O)
       auto issue_pv = [&](int x, int j, int st) -> bool {
-        if (!mbar_wait(&ctl->p_full[x], (uint32_t)(bt[x] & 1)) ||
+        // keys 0-63 as soon as their P is published, keys 64-127 after the rest
+        if (!mbar_wait(&ctl->p_half[x], (uint32_t)(bt[x] & 1)) ||
             (j == 0 && !mbar_wait(&ctl->o_free[x], (ut[x] + 1) & 1)))
           return false;
         tc_fence_after();
         const uint64_t vd = vdesc0 + (uint64_t)((st * 2 * tile_bytes) >> 4);
         const uint32_t pcol = tmem + x * 256, ocol = pcol + 128;
-        for (int kk = 0; kk < 8; ++kk)
+        for (int kk = 0; kk < 4; ++kk)
           umma_bf16_ts(ocol, pcol + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+        if (!mbar_wait(&ctl->p_full[x], (uint32_t)(bt[x] & 1))) return false;
+        tc_fence_after();
+        for (int kk = 4; kk < 8; ++kk)
+          umma_bf16_ts(ocol, pcol + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_o, 1u);
         umma_commit(&ctl->pv_done[x]);
         ++bt[x];
         return true;
@@ -627,51 +632,9 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             alpha = exp2f(m_run - mb);
           }
         }
-        float lsum = 0.f;
-        if (!any_row) {
-          uint32_t z[16];
-#pragma unroll
-          for (int q = 0; q < 16; ++q) z[q] = 0u;
-#pragma unroll 1
-          for (int c4 = 0; c4 < 4; ++c4) tmem_st16(s_col + 16 * c4, z);
-        } else if (all_full) {
-#pragma unroll 1
-          for (int c4 = 0; c4 < 4; ++c4) {
-            tmem_ld32(s_col + 32 * c4, rr);
-            tmem_ld_wait();
-            uint32_t pk[16];
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-              const float p0 = ex2_approx(fmaf(__uint_as_float(rr[2 * q]), sl2, -m_new));
-              const float p1 = ex2_approx(fmaf(__uint_as_float(rr[2 * q + 1]), sl2, -m_new));
-              lsum += p0 + p1;
-              pk[q] = pack_bf16x2(p0, p1);
-            }
-            tmem_st16(s_col + 16 * c4, pk);
-          }
-        } else {
-#pragma unroll 1
-          for (int c4 = 0; c4 < 4; ++c4) {
-            tmem_ld32(s_col + 32 * c4, rr);
-            tmem_ld_wait();
-            uint32_t pk[16];
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-              const int c0 = 32 * c4 + 2 * q;
-              const float x0 = fmaf(__uint_as_float(rr[2 * q]), sl2, -m_new);
-              const float x1 = fmaf(__uint_as_float(rr[2 * q + 1]), sl2, -m_new);
-              const float p0 = ex2_approx(c0 <= limit ? x0 : -INFINITY);
-              const float p1 = ex2_approx(c0 + 1 <= limit ? x1 : -INFINITY);
-              lsum += p0 + p1;
-              pk[q] = pack_bf16x2(p0, p1);
-            }
-            tmem_st16(s_col + 16 * c4, pk);
-          }
-        }
-        l_run = l_run * alpha + lsum;
-        m_run = m_new;
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
           // rescale this warp's O rows once the previous PV of this tile has landed
+          // (before any of this block's P is published: PV(j) accumulates into O)
           if (!mbar_wait(&ctl->pv_done[x], (uint32_t)((bt + 1) & 1))) {
             report_error(p.err, MSA_ERR_TIMEOUT, kSiteTileSoftmax, (int)bt, 1);
             failed = true;
@@ -692,6 +655,61 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             tmem_st16(o_col + 32 * c + 16, up);
           }
         }
+        // P of keys 0-63 is published first, so that the PV MMA can start on it
+        auto publish_half = [&]() {
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->p_half[x]);
+        };
+        float lsum = 0.f;
+        if (!any_row) {
+          uint32_t z[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) z[q] = 0u;
+#pragma unroll 1
+          for (int c4 = 0; c4 < 4; ++c4) {
+            tmem_st16(s_col + 16 * c4, z);
+            if (c4 == 1) publish_half();
+          }
+        } else if (all_full) {
+#pragma unroll 1
+          for (int c4 = 0; c4 < 4; ++c4) {
+            tmem_ld32(s_col + 32 * c4, rr);
+            tmem_ld_wait();
+            uint32_t pk[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const float p0 = ex2_approx(fmaf(__uint_as_float(rr[2 * q]), sl2, -m_new));
+              const float p1 = ex2_approx(fmaf(__uint_as_float(rr[2 * q + 1]), sl2, -m_new));
+              lsum += p0 + p1;
+              pk[q] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(s_col + 16 * c4, pk);
+            if (c4 == 1) publish_half();
+          }
+        } else {
+#pragma unroll 1
+          for (int c4 = 0; c4 < 4; ++c4) {
+            tmem_ld32(s_col + 32 * c4, rr);
+            tmem_ld_wait();
+            uint32_t pk[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const int c0 = 32 * c4 + 2 * q;
+              const float x0 = fmaf(__uint_as_float(rr[2 * q]), sl2, -m_new);
+              const float x1 = fmaf(__uint_as_float(rr[2 * q + 1]), sl2, -m_new);
+              const float p0 = ex2_approx(c0 <= limit ? x0 : -INFINITY);
+              const float p1 = ex2_approx(c0 + 1 <= limit ? x1 : -INFINITY);
+              lsum += p0 + p1;
+              pk[q] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(s_col + 16 * c4, pk);
+            if (c4 == 1) publish_half();
+          }
+        }
+        l_run = l_run * alpha + lsum;
+        m_run = m_new;
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
