@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <climits>
 #include <mutex>
 
 #include "msa_internal.h"
@@ -164,6 +165,41 @@ msa_status_t attn_common(const msa_shape_t* shape, const msa_varlen_t* seqs, con
   return MSA_OK;
 }
 
+// Paged decode: workspace slices and argument checks.
+struct PagedLayout {
+  size_t cu_q, cu_k, tile_ctr, idx_scratch, total;
+  int64_t total_k;   // upper bound of the cached tokens
+};
+
+msa_status_t check_paged(const msa_shape_t* s, const msa_paged_t* pg) {
+  msa_status_t st = check_shape(s);
+  if (st != MSA_OK) return st;
+  if (pg == nullptr || pg->seqlens == nullptr || pg->block_table == nullptr) return MSA_ERR_INVALID_ARG;
+  if (pg->batch < 1 || pg->max_blocks < 1 || pg->num_pages < 1 || pg->max_seqlen < 1) return MSA_ERR_INVALID_ARG;
+  if (pg->max_seqlen > (int64_t)pg->max_blocks * kBk) return MSA_ERR_INVALID_ARG;
+  // key rows are int32 coordinates; cached tokens are summed in int32
+  if (pg->num_pages > (INT32_MAX - kBk) / kBk) return MSA_ERR_UNSUPPORTED;
+  if ((int64_t)pg->batch * pg->max_blocks * kBk > (int64_t)INT32_MAX - 256) return MSA_ERR_UNSUPPORTED;
+  return MSA_OK;
+}
+
+PagedLayout paged_layout(const msa_shape_t* s, const msa_paged_t* pg) {
+  PagedLayout L{};
+  L.total_k = (int64_t)pg->batch * pg->max_blocks * kBk;
+  size_t off = kWsHeader;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, kAlign);
+    return o;
+  };
+  L.cu_q = take(sizeof(int32_t) * (pg->batch + 1));
+  L.cu_k = take(sizeof(int32_t) * (pg->batch + 1));
+  L.tile_ctr = take(sizeof(int32_t) * 4);
+  L.idx_scratch = take(decode_index_scratch_bytes(pg->batch, L.total_k, s->G, s->k));
+  L.total = off;
+  return L;
+}
+
 }  // namespace
 
 namespace msa {
@@ -301,6 +337,70 @@ msa_status_t msa_dense_attn(const msa_shape_t* shape, const msa_varlen_t* seqs, 
   a.max_q_len = seqs->max_q_len; a.max_k_len = seqs->max_k_len;
   a.err = static_cast<DevError*>(ws);
   return launch_dense_attn(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
+}
+
+size_t msa_decode_paged_workspace_size(const msa_shape_t* shape, const msa_paged_t* pages) {
+  if (check_paged(shape, pages) != MSA_OK) return 0;
+  return paged_layout(shape, pages).total;
+}
+
+msa_status_t msa_index_topk_decode_paged(const msa_shape_t* shape, const msa_paged_t* pages, const void* q_idx,
+                                         const void* k_idx_pages, int32_t* sel, void* ws, size_t ws_bytes,
+                                         void* stream) {
+  msa_status_t st = check_paged(shape, pages);
+  if (st != MSA_OK) return st;
+  if (!q_idx || !k_idx_pages || !sel) return MSA_ERR_INVALID_ARG;
+  const PagedLayout L = paged_layout(shape, pages);
+  if (!ws_ok(ws, ws_bytes, L.total)) return MSA_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  int32_t* cu_q = reinterpret_cast<int32_t*>(base + L.cu_q);
+  int32_t* cu_k = reinterpret_cast<int32_t*>(base + L.cu_k);
+  if (launch_paged_prep(pages->seqlens, pages->batch, pages->max_blocks, cu_q, cu_k, reinterpret_cast<DevError*>(ws),
+                        stream) != 0)
+    return MSA_ERR_CUDA;
+  IndexTopkArgs a{};
+  a.q_idx = q_idx; a.k_idx = k_idx_pages; a.sel = sel;
+  a.cu_q = cu_q; a.cu_k = cu_k;
+  a.batch = pages->batch; a.G = shape->G; a.d_idx = shape->d_idx; a.k = shape->k;
+  a.total_q = pages->batch; a.total_k = L.total_k;
+  a.max_q_len = 1; a.max_k_len = pages->max_seqlen;
+  a.err = reinterpret_cast<DevError*>(ws);
+  a.scratch = base + L.idx_scratch;
+  a.scratch_bytes = L.total - L.idx_scratch;
+  a.block_table = pages->block_table; a.max_blocks = pages->max_blocks; a.num_pages = pages->num_pages;
+  return launch_index_topk_decode(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
+}
+
+msa_status_t msa_sparse_attn_decode_paged(const msa_shape_t* shape, const msa_paged_t* pages, const void* q,
+                                          const void* k_pages, const void* v_pages, const int32_t* sel, void* out,
+                                          float* lse, void* ws, size_t ws_bytes, void* stream) {
+  msa_status_t st = check_paged(shape, pages);
+  if (st != MSA_OK) return st;
+  if (!q || !k_pages || !v_pages || !sel || !out) return MSA_ERR_INVALID_ARG;
+  const PagedLayout L = paged_layout(shape, pages);
+  if (!ws_ok(ws, ws_bytes, L.total)) return MSA_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  int32_t* cu_q = reinterpret_cast<int32_t*>(base + L.cu_q);
+  int32_t* cu_k = reinterpret_cast<int32_t*>(base + L.cu_k);
+  if (launch_paged_prep(pages->seqlens, pages->batch, pages->max_blocks, cu_q, cu_k, reinterpret_cast<DevError*>(ws),
+                        stream) != 0)
+    return MSA_ERR_CUDA;
+  AttnArgs a{};
+  a.q = q; a.key = k_pages; a.value = v_pages; a.sel = sel; a.out = out; a.lse = lse;
+  a.cu_q = cu_q; a.cu_k = cu_k;
+  a.batch = pages->batch; a.H = shape->H; a.G = shape->G; a.d = shape->d; a.k = shape->k;
+  a.sm_scale = shape->sm_scale;
+  a.total_q = pages->batch; a.total_k = L.total_k;
+  a.max_q_len = 1; a.max_k_len = pages->max_seqlen;
+  a.t0 = 0; a.t1 = pages->batch;
+  a.err = reinterpret_cast<DevError*>(ws);
+  a.tile_ctr = reinterpret_cast<int32_t*>(base + L.tile_ctr);
+  a.block_table = pages->block_table; a.max_blocks = pages->max_blocks; a.num_pages = pages->num_pages;
+  return launch_rows_attn(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
 }
 
 int32_t msa_set_tile_threshold(int32_t theta) {

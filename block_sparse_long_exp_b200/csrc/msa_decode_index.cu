@@ -11,6 +11,8 @@
 //   select : one CTA per (sequence, group): per-thread top-(k-1) over a strided
 //            slice of the block scores, then k-1 rounds of block-wide argmax on
 //            64-bit keys (score, then lower block index).
+#include <climits>
+
 #include "msa_common.cuh"
 
 namespace msa {
@@ -74,7 +76,8 @@ __global__ void __launch_bounds__(kScanThreads)
 decode_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restrict__ q_idx,
                    const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_k, int batch, int G,
                    const int32_t* __restrict__ blk_off, const int32_t* __restrict__ chunk_off,
-                   float* __restrict__ bscore, DevError* err) {
+                   float* __restrict__ bscore, const int32_t* __restrict__ block_table, int max_blocks,
+                   int64_t num_pages, DevError* err) {
   constexpr int SPAN = DIDX * 2 >= 128 ? 128 : DIDX * 2;
   constexpr int NBOX = DIDX * 2 / SPAN;
   constexpr int BLOCK_BYTES = kBk * DIDX * 2;
@@ -99,14 +102,25 @@ decode_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16
   const int nblk = min(kCB, lb - j0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  // first key row of block j0 + i (packed: after the sequence's start; paged:
+  // its page); -1: an invalid page, whose block is not read
+  auto block_row = [&](int i) -> int64_t {
+    if (block_table == nullptr) return (int64_t)cu_k[b] + (int64_t)kBk * (j0 + i);
+    const int32_t pg = block_table[(int64_t)b * max_blocks + j0 + i];
+    return (pg >= 0 && pg < num_pages) ? (int64_t)pg * kBk : -1;
+  };
   if (threadIdx.x == 0) {
     for (int i = 0; i < kCB; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
     for (int i = 0; i < nblk; ++i) {
+      const int64_t row = block_row(i);
+      if (row < 0) {
+        report_error(err, MSA_ERR_DEVICE_CHECK, kSitePaged, b, j0 + i);
+        continue;
+      }
       mbar_arrive_expect_tx(&bars[i], BLOCK_BYTES);
       for (int bx = 0; bx < NBOX; ++bx)
-        tma_load_2d(smem + i * BLOCK_BYTES + bx * kBk * SPAN, &tm_k, &bars[i], bx * (SPAN / 2),
-                    cu_k[b] + kBk * (j0 + i));
+        tma_load_2d(smem + i * BLOCK_BYTES + bx * kBk * SPAN, &tm_k, &bars[i], bx * (SPAN / 2), (int)row);
     }
   }
   // B operand: q_idx of this sequence's query, n = group (zero for n >= G).
@@ -124,7 +138,10 @@ decode_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16
     }
   }
   __syncthreads();
-  if (warp < nblk) {
+  if (warp < nblk && block_row(warp) < 0) {
+    // an invalid page: the block was not read and ranks last
+    if (lane < G) bscore[(int64_t)(blk_off[b] + j0 + warp) * G + lane] = -INFINITY;
+  } else if (warp < nblk) {
     if (!mbar_wait(&bars[warp], 0)) {
       report_error(err, MSA_ERR_TIMEOUT, kSiteDecodeIndex, chunk, warp);
     } else {
@@ -162,7 +179,27 @@ decode_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16
   }
   // no load may remain in flight when the CTA exits
   if (threadIdx.x == 0)
-    for (int i = 0; i < nblk; ++i) mbar_wait(&bars[i], 0);
+    for (int i = 0; i < nblk; ++i)
+      if (block_row(i) >= 0) mbar_wait(&bars[i], 0);
+}
+
+// Paged decode: logical offsets of one query per sequence and its cache.
+__global__ void paged_prep_kernel(const int32_t* __restrict__ seqlens, int batch, int max_blocks,
+                                  int32_t* __restrict__ cu_q, int32_t* __restrict__ cu_k, DevError* err) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int64_t acc = 0;
+  for (int b = 0; b < batch; ++b) {
+    cu_q[b] = b;
+    cu_k[b] = (int32_t)acc;
+    int32_t L = seqlens[b];
+    if (L < 1 || (int64_t)L > (int64_t)max_blocks * kBk || acc + L > INT32_MAX) {
+      report_error(err, MSA_ERR_DEVICE_CHECK, kSitePaged, b, L);
+      L = 0;                                   // the sequence then takes no part
+    }
+    acc += L;
+  }
+  cu_q[batch] = batch;
+  cu_k[batch] = (int32_t)acc;
 }
 
 // 64-bit ranking key: order-preserving score bits, then the complement of the
@@ -181,7 +218,12 @@ decode_select_kernel(const float* __restrict__ bscore, const int32_t* __restrict
   const int b = blockIdx.x / G, g = blockIdx.x % G;
   const int Tb = cu_q[b + 1] - cu_q[b];
   const int Sb = cu_k[b + 1] - cu_k[b];
-  if (Tb != 1 || Sb < 1) return;
+  if (Tb == 1 && Sb < 1) {
+    // a query without keys (an error the prep recorded): an empty selection
+    if (threadIdx.x < k) sel[((int64_t)cu_q[b] * G + g) * k + threadIdx.x] = -1;
+    return;
+  }
+  if (Tb != 1) return;
   const int lb = (Sb - 1) / kBk;
   const int cap = k - 1;
   const float* sc = bscore + (int64_t)blk_off[b] * G + g;
@@ -265,7 +307,8 @@ int launch_index_topk_decode(const IndexTopkArgs& a, void* stream) {
 
   const int span = a.d_idx * 2 >= 128 ? 128 : a.d_idx * 2;
   alignas(64) CUtensorMap tm_k;
-  const uint64_t dims[2] = {(uint64_t)a.d_idx, (uint64_t)a.total_k};
+  const uint64_t rows = a.block_table != nullptr ? (uint64_t)a.num_pages * kBk : (uint64_t)a.total_k;
+  const uint64_t dims[2] = {(uint64_t)a.d_idx, rows};
   const uint64_t strides[1] = {(uint64_t)a.d_idx * 2};
   const uint32_t box[2] = {(uint32_t)(span / 2), (uint32_t)kBk};
   int rc = make_tmap_bf16(&tm_k, a.k_idx, 2, dims, strides, box, span);
@@ -279,8 +322,9 @@ int launch_index_topk_decode(const IndexTopkArgs& a, void* stream) {
   e = cudaFuncSetAttribute(decode_scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);  \
   if (e != cudaSuccess) return (int)e;                                                                      \
   ProfScope p("decode_scan", stream);                                                                       \
-  decode_scan_kernel<D><<<(unsigned)max_chunks, kScanThreads, smem, st>>>(tm_k, qi, a.cu_q, a.cu_k, a.batch, \
-                                                                        a.G, blk_off, chunk_off, bscore, a.err)
+  decode_scan_kernel<D><<<(unsigned)max_chunks, kScanThreads, smem, st>>>(                                  \
+      tm_k, qi, a.cu_q, a.cu_k, a.batch, a.G, blk_off, chunk_off, bscore, a.block_table, a.max_blocks,       \
+      a.num_pages, a.err)
   if (a.d_idx == 32) { MSA_SCAN(32); }
   else if (a.d_idx == 64) { MSA_SCAN(64); }
   else { MSA_SCAN(128); }
@@ -290,6 +334,14 @@ int launch_index_topk_decode(const IndexTopkArgs& a, void* stream) {
   if (a.k <= 8) decode_select_kernel<7><<<nsel, kSelThreads, 0, st>>>(bscore, a.cu_q, a.cu_k, blk_off, a.G, a.k, a.sel);
   else if (a.k <= 16) decode_select_kernel<15><<<nsel, kSelThreads, 0, st>>>(bscore, a.cu_q, a.cu_k, blk_off, a.G, a.k, a.sel);
   else decode_select_kernel<31><<<nsel, kSelThreads, 0, st>>>(bscore, a.cu_q, a.cu_k, blk_off, a.G, a.k, a.sel);
+  return (int)cudaGetLastError();
+}
+
+int launch_paged_prep(const int32_t* seqlens, int32_t batch, int32_t max_blocks, int32_t* cu_q, int32_t* cu_k,
+                      DevError* err, void* stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  ProfScope p("paged_prep", stream);
+  paged_prep_kernel<<<1, 32, 0, st>>>(seqlens, batch, max_blocks, cu_q, cu_k, err);
   return (int)cudaGetLastError();
 }
 

@@ -43,6 +43,7 @@ enum ErrorSite : int32_t {
   kSiteTileLoad = 152,
   kSiteTileMma = 153,
   kSiteTileSoftmax = 154,
+  kSitePaged = 161,
 };
 
 // One KV-outer work item: up to `count` queries of the list of
@@ -76,6 +77,10 @@ struct IndexTopkArgs {
   DevError* err;
   void* scratch;       // decode path: block scores
   size_t scratch_bytes;
+  // paged caches (decode): block j of sequence b is page block_table[b * max_blocks + j]
+  const int32_t* block_table;   // null: packed rows cu_k[b] + j * B_k
+  int32_t max_blocks;
+  int64_t num_pages;
 };
 int launch_index_topk_prefill(const IndexTopkArgs& a, void* stream);
 int launch_index_topk_decode(const IndexTopkArgs& a, void* stream);
@@ -119,6 +124,10 @@ struct AttnArgs {
   uint64_t* dmember;   // [(t1-t0) x G] positions of the covered blocks in the tile's list
   uint2* clist;        // [(t1-t0) x G] combine list: {pair (t - t0) * G + g, slots to merge}
   int32_t* tile_ctr;   // [4]: pairs, listed units, unit ticket
+  // paged caches (decode, rows mode): see IndexTopkArgs
+  const int32_t* block_table;
+  int32_t max_blocks;
+  int64_t num_pages;
 };
 int launch_sparse_attn_pass(const AttnArgs& a, void* stream);
 int launch_combine(const void* part_acc, const float* part_lse, const int32_t* sel, void* out,
@@ -128,6 +137,10 @@ int tile_default_theta(int UQ);
 int launch_tile_plan(const AttnArgs& a, int theta, void* stream);
 int launch_tile_attn(const AttnArgs& a, void* stream);
 int launch_rows_attn(const AttnArgs& a, void* stream);   // one query per unit (decode)
+// Paged decode: cu_q[b] = b and cu_k = prefix of seqlens (a length outside
+// [1, max_blocks * B_k] counts as 0 and records MSA_ERR_DEVICE_CHECK).
+int launch_paged_prep(const int32_t* seqlens, int32_t batch, int32_t max_blocks, int32_t* cu_q, int32_t* cu_k,
+                      DevError* err, void* stream);
 
 struct DenseArgs {
   const void* q;

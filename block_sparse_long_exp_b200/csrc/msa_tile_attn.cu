@@ -209,7 +209,8 @@ struct __align__(16) TileUnit {
   int32_t uid, g, nq, nblk;   // nblk < 0: no more work
   int32_t ntl, Tb, Sb, qrow0;
   int32_t kbase, pad0, pad1, pad2;
-  int32_t blk[kMaxDense];     // hybrid mode: the unit's blocks, ascending
+  int32_t blk[kMaxDense];     // tiles / rows mode: the unit's blocks, ascending
+  int32_t page[kMaxDense];    // rows mode with a page table: each block's page
 };
 
 struct __align__(16) TileCtl {
@@ -236,6 +237,9 @@ struct TileParams {
   const int32_t* nunits;      // device count of units (tiles: listed units; dense: all); null: nunits_host
   int64_t nunits_host;        // rows mode: rows x G
   const int32_t* sel;         // rows mode: [T, G, k]
+  const int32_t* block_table; // rows mode, paged caches: [batch, max_blocks] page per block (else null)
+  int32_t max_blocks;
+  int64_t num_pages;
   int32_t* ticket;
   const int32_t* cu_q;
   const int32_t* cu_k;
@@ -371,18 +375,32 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       const int Tb = p.cu_q[seq + 1] - p.cu_q[seq];
       const int Sb = p.cu_k[seq + 1] - p.cu_k[seq];
       if (kMode == kModeRows) {
-        // the selection row: valid ids first, then -1 padding
+        // the selection row: valid ids first, then -1 padding; a row with an
+        // id past the query's block (or a page outside the cache) is reported
+        // and skipped before anything is read
         const int32_t b = lane < p.k ? p.sel[(r0 * G + g) * p.k + lane] : -1;
         const unsigned v = __ballot_sync(0xffffffffu, b >= 0);
         nblk = __popc(v);
         const int64_t pos = (int64_t)Sb - Tb + (r0 - p.cu_q[seq]);
+        bool bad = b >= 0 && (Tb > Sb || pos < 0 || b > pos / kBk);
+        int32_t pg = -1;
+        if (b >= 0 && !bad && p.block_table != nullptr) {
+          bad = b >= p.max_blocks;
+          if (!bad) {
+            pg = p.block_table[(int64_t)seq * p.max_blocks + b];
+            bad = pg < 0 || pg >= p.num_pages;
+          }
+        }
+        if (bad) report_error(p.err, MSA_ERR_DEVICE_CHECK, p.block_table != nullptr ? kSitePaged : kSiteInvert,
+                              (int)r0, b);
         if (b >= 0) {
           U->blk[lane] = b;
-          if (Tb > Sb || b > pos / kBk) report_error(p.err, MSA_ERR_DEVICE_CHECK, kSiteInvert, (int)r0, b);
+          U->page[lane] = pg;
         }
-        if (v != (nblk >= 32 ? 0xffffffffu : (1u << nblk) - 1u)) {
+        const bool any_bad = __any_sync(0xffffffffu, bad);
+        if (any_bad || v != (nblk >= 32 ? 0xffffffffu : (1u << nblk) - 1u)) {
           // ids must come first: anything else is not a selection row
-          if (lane == 0) report_error(p.err, MSA_ERR_DEVICE_CHECK, kSiteInvert, (int)r0, -1);
+          if (lane == 0 && !any_bad) report_error(p.err, MSA_ERR_DEVICE_CHECK, kSiteInvert, (int)r0, -1);
           nblk = 0;
         }
       } else if (kMode == kModeDense) {
@@ -436,7 +454,7 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
           ok = mbar_wait(&ctl->kv_empty[st], ((kvc >> 1) + 1) & 1);
           if (!ok) break;
           const int blk = kMode == kModeDense ? j : R->blk[j];
-          const int krow = kbase + blk * kBk;
+          const int krow = (kMode == kModeRows && p.block_table != nullptr) ? R->page[j] * kBk : kbase + blk * kBk;
           uint8_t* ks = kv_s + st * 2 * tile_bytes;
           mbar_arrive_expect_tx(&ctl->k_full[st], tile_bytes);
           for (int h = 0; h < nhalf; ++h) tma_load_3d(ks + h * 128 * 128, &tm_k, &ctl->k_full[st], 64 * h, g, krow);
@@ -914,11 +932,13 @@ int launch_rows_attn(const AttnArgs& a, void* stream) {
   cudaError_t e = cudaMemsetAsync(a.tile_ctr, 0, sizeof(int32_t) * 4, st);
   if (e != cudaSuccess) return (int)e;
   alignas(64) CUtensorMap tm_k, tm_v, tm_q;
-  int rc = make_tile_maps(&tm_k, &tm_v, &tm_q, a.q, a.key, a.value, a.total_q, a.total_k, a.H, a.G, a.d);
+  const int64_t krows = a.block_table != nullptr ? a.num_pages * kBk : a.total_k;
+  int rc = make_tile_maps(&tm_k, &tm_v, &tm_q, a.q, a.key, a.value, a.total_q, krows, a.H, a.G, a.d);
   if (rc) return rc;
   TileParams prm{};
   prm.nunits = nullptr; prm.nunits_host = rows * a.G; prm.ticket = a.tile_ctr + 2;
   prm.sel = a.sel;
+  prm.block_table = a.block_table; prm.max_blocks = a.max_blocks; prm.num_pages = a.num_pages;
   prm.cu_q = a.cu_q; prm.cu_k = a.cu_k;
   prm.batch = a.batch; prm.H = a.H; prm.G = a.G; prm.d = a.d; prm.k = a.k; prm.UQ = 1;
   prm.scale_log2 = a.sm_scale * 1.4426950408889634f;

@@ -28,6 +28,7 @@ EXPORTED = [
     "msa_index_topk_decode_noalloc_max_scratch", "msa_index_topk_decode_noalloc",
     "msa_profile_enable", "msa_profile_reset", "msa_profile_read",
     "msa_get_device_error", "msa_version", "msa_set_tile_threshold",
+    "msa_decode_paged_workspace_size", "msa_index_topk_decode_paged", "msa_sparse_attn_decode_paged",
 ]
 
 
@@ -46,6 +47,12 @@ class Varlen(ctypes.Structure):
                 ("max_k_len", ctypes.c_int32), ("pad_", ctypes.c_int32),
                 ("total_q", ctypes.c_int64), ("total_k", ctypes.c_int64),
                 ("cu_q", ctypes.c_void_p), ("cu_k", ctypes.c_void_p)]
+
+
+class Paged(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("max_blocks", ctypes.c_int32), ("max_seqlen", ctypes.c_int32),
+                ("pad_", ctypes.c_int32), ("num_pages", ctypes.c_int64),
+                ("seqlens", ctypes.c_void_p), ("block_table", ctypes.c_void_p)]
 
 
 _lib = None
@@ -94,6 +101,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_version.restype = ctypes.c_char_p
     lib.msa_set_tile_threshold.argtypes = [i32]
     lib.msa_set_tile_threshold.restype = i32
+    lib.msa_decode_paged_workspace_size.argtypes = [P(Shape), P(Paged)]
+    lib.msa_decode_paged_workspace_size.restype = sz
+    lib.msa_index_topk_decode_paged.argtypes = [P(Shape), P(Paged), vp, vp, vp, vp, sz, vp]
+    lib.msa_index_topk_decode_paged.restype = i32
+    lib.msa_sparse_attn_decode_paged.argtypes = [P(Shape), P(Paged), vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.msa_sparse_attn_decode_paged.restype = i32
     _lib = lib
     return lib
 
@@ -294,6 +307,63 @@ def msa_profile_read(kernel: Optional[str]) -> Tuple[float, int]:
     rc = load_library().msa_profile_read(kernel.encode() if kernel else None, ctypes.byref(ms), ctypes.byref(n))
     _check(rc, "msa_profile_read")
     return ms.value, n.value
+
+
+def make_paged(seqlens: torch.Tensor, block_table: torch.Tensor, max_seqlen: int, num_pages: int) -> Paged:
+    """Paged-cache description: seqlens int32 [batch] and block_table int32
+    [batch, max_blocks] on the device; max_seqlen >= every seqlens[b]."""
+    assert seqlens.dtype == torch.int32 and block_table.dtype == torch.int32 and block_table.dim() == 2
+    assert seqlens.is_cuda and block_table.is_cuda and block_table.is_contiguous()
+    p = Paged()
+    p.batch, p.max_blocks = block_table.shape[0], block_table.shape[1]
+    p.max_seqlen, p.num_pages = int(max_seqlen), int(num_pages)
+    p.seqlens, p.block_table = seqlens.data_ptr(), block_table.data_ptr()
+    p._keep = (seqlens, block_table)
+    return p
+
+
+def _paged_ws(shape: Shape, pages: Paged, ws, device):
+    need = load_library().msa_decode_paged_workspace_size(ctypes.byref(shape), ctypes.byref(pages))
+    if need == 0:
+        raise MsaError("msa_decode_paged_workspace_size: shape or paged description rejected")
+    return _workspace(need, device) if ws is None else ws
+
+
+def msa_index_topk_decode_paged(shape: Shape, pages: Paged, q_idx: torch.Tensor, k_idx_pages: torch.Tensor,
+                                sel: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                                stream=None, check: bool = True) -> torch.Tensor:
+    lib = load_library()
+    _require_cuda(q_idx)
+    if sel is None:
+        sel = torch.empty((pages.batch, shape.G, shape.k), dtype=torch.int32, device=q_idx.device)
+    ws = _paged_ws(shape, pages, ws, q_idx.device)
+    rc = lib.msa_index_topk_decode_paged(ctypes.byref(shape), ctypes.byref(pages), _ptr(q_idx), _ptr(k_idx_pages),
+                                         _ptr(sel), _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "msa_index_topk_decode_paged")
+    if check:
+        _device_check(ws, stream, "msa_index_topk_decode_paged")
+    return sel
+
+
+def msa_sparse_attn_decode_paged(shape: Shape, pages: Paged, q: torch.Tensor, k_pages: torch.Tensor,
+                                 v_pages: torch.Tensor, sel: torch.Tensor, out: Optional[torch.Tensor] = None,
+                                 lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+                                 ws: Optional[torch.Tensor] = None, stream=None,
+                                 check: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    lib = load_library()
+    _require_cuda(q)
+    if out is None:
+        out = torch.empty((pages.batch, shape.H, shape.d), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((pages.batch, shape.H), dtype=torch.float32, device=q.device)
+    ws = _paged_ws(shape, pages, ws, q.device)
+    rc = lib.msa_sparse_attn_decode_paged(ctypes.byref(shape), ctypes.byref(pages), _ptr(q), _ptr(k_pages),
+                                          _ptr(v_pages), _ptr(sel), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                          _stream(stream))
+    _check(rc, "msa_sparse_attn_decode_paged")
+    if check:
+        _device_check(ws, stream, "msa_sparse_attn_decode_paged")
+    return out, lse
 
 
 def msa_set_tile_threshold(theta: int) -> int:

@@ -154,6 +154,48 @@ msa_status_t msa_sparse_attn_decode(const msa_shape_t* shape, const msa_varlen_t
                                     void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Decode over a paged KV cache (a serving layout; the pages describe the
+ * method, not a cache format, and this is the plainest paged form of their
+ * decode step: pnsm.cn sec. 9, yhxrc.cn sec. 二).  A page holds one B_k-token
+ * block: page p is rows [p*B_k, (p+1)*B_k) of
+ *   k_idx_pages  device bf16 [num_pages*B_k, d_idx]
+ *   k_pages      device bf16 [num_pages*B_k, G, d]
+ *   v_pages      device bf16 [num_pages*B_k, G, d]
+ * Sequence b holds seqlens[b] tokens (the new token included, so its one
+ * query sits at position seqlens[b]-1); its block j lives in page
+ * block_table[b*max_blocks + j] for j < ceil(seqlens[b]/B_k).  Token rows
+ * past seqlens[b] in the last page are never attended.  q / q_idx / sel /
+ * out / lse have one row per sequence ([batch, ...], as in the packed decode
+ * call).  Results equal those of the packed calls on the same tokens. */
+typedef struct {
+  int32_t batch;
+  int32_t max_blocks;        /* columns of block_table */
+  int32_t max_seqlen;        /* host upper bound of seqlens[b] */
+  int32_t pad_;
+  int64_t num_pages;
+  const int32_t* seqlens;    /* device [batch] */
+  const int32_t* block_table;/* device [batch, max_blocks] */
+} msa_paged_t;
+
+/* Workspace of either paged call (the same size serves both). */
+size_t msa_decode_paged_workspace_size(const msa_shape_t* shape, const msa_paged_t* pages);
+
+/* Index branch over the paged index keys: sel [batch, G, k] as
+ * msa_index_topk.  A page id outside [0, num_pages) or seqlens[b] outside
+ * [1, max_blocks*B_k] records MSA_ERR_DEVICE_CHECK in the error word (the
+ * sequence is skipped; nothing is read out of range). */
+msa_status_t msa_index_topk_decode_paged(const msa_shape_t* shape, const msa_paged_t* pages,
+                                         const void* q_idx, const void* k_idx_pages, int32_t* sel,
+                                         void* ws, size_t ws_bytes, void* stream);
+
+/* Main branch over the paged K / V: out [batch, H, d] (and lse [batch, H] or
+ * NULL) from the selection sel [batch, G, k].  Same device checks. */
+msa_status_t msa_sparse_attn_decode_paged(const msa_shape_t* shape, const msa_paged_t* pages,
+                                          const void* q, const void* k_pages, const void* v_pages,
+                                          const int32_t* sel, void* out, float* lse,
+                                          void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* Two-phase combine on its own (pnsm.cn sec. 7 "two-phase combine").
  * Merges, for every query t and head h = g*(H/G) + i of group g, the partials
  * of the slots s with sel[t, g, s] >= 0:
