@@ -129,7 +129,12 @@ def make_ctx(w, inp, torch, msa):
     lib = msa.load_library()
     import ctypes
     n_idx = lib.msa_index_topk_workspace_size(ctypes.byref(shape), ctypes.byref(seqs))
-    n_att = msa.msa_sparse_attn_workspace_size(shape, seqs, 0) if not getattr(make_ctx, "index_only", False) else 256
+    # passes of at most q_chunk query rows (the partials of a pass must fit the device)
+    ctx["q_chunk"] = getattr(make_ctx, "q_chunk", 0)
+    if ctx["q_chunk"] < 0:
+        ctx["q_chunk"] = 131072 if T > 131072 else 0
+    n_att = (msa.msa_sparse_attn_workspace_size(shape, seqs, ctx["q_chunk"])
+             if not getattr(make_ctx, "index_only", False) else 256)
     ctx["ws_idx"] = torch.empty(n_idx, dtype=torch.uint8, device=dev)
     ctx["ws_att"] = torch.zeros(n_att, dtype=torch.uint8, device=dev) if n_att <= 256 else \
         torch.empty(n_att, dtype=torch.uint8, device=dev)
@@ -143,6 +148,7 @@ def step_prefill(ctx, msa, inp=None, index_only=False):
     if index_only:
         return
     msa.msa_sparse_attn_prefill(ctx["shape"], ctx["seqs"], inp["q"], inp["k"], inp["v"], ctx["sel"],
+                                q_chunk=ctx.get("q_chunk", 0),
                                 out=ctx["out"], want_lse=False, ws=ctx["ws_att"], check=False)
 
 
@@ -357,8 +363,10 @@ def run_ours(args):
     inp = W.make_inputs(wr, "cuda", T_override=args.T or None)
     torch.cuda.synchronize()
     make_ctx.index_only = args.index_only
+    make_ctx.q_chunk = args.q_chunk
     ctx = make_ctx(wr, inp, torch, msa)
     make_ctx.index_only = False
+    make_ctx.q_chunk = -1
     S_lens = [inp["cu_k_host"][i + 1] - inp["cu_k_host"][i] for i in range(len(inp["cu_k_host"]) - 1)]
     T_lens = [inp["cu_q_host"][i + 1] - inp["cu_q_host"][i] for i in range(len(inp["cu_q_host"]) - 1)]
     T = ctx["T"]
@@ -392,6 +400,7 @@ def run_ours(args):
 
     value, ms_max = job_rate(T * args.steps, ms, torch, dist)
     ms_step = ms_max / args.steps
+    ctx_q_chunk = ctx["q_chunk"]
 
     # algorithmic work of each kernel: the main branch split between the query
     # tiles and the KV-outer lists as the library's planner splits it
@@ -531,7 +540,8 @@ def run_ours(args):
                 "config": {"workload": args.workload, "T": T, "H": w.H, "G": w.G, "d": w.d, "d_idx": w.d_idx,
                            "B_k": w.B_k, "k": w.k, "hot_block_frac": w.hot_frac,
                            "l2": "inputs larger than L2 (q alone is %.1f GB)" % (inp["q"].numel() * 2 / 1e9),
-                           "parallelism": f"independent layer per GPU x{world}"},
+                           "parallelism": f"independent layer per GPU x{world}",
+                           "attention_pass_rows": ctx_q_chunk or T},
                 "roofline": roof, "step_roofline": step_roof, "tile_split": split, "dense_gqa": dense,
                 "decode": decode, "e2e": e2e,
                 "cpu_baseline": cpu, "clocks": clk, "gpu_launches": launches, "kernels": kernels}
@@ -554,6 +564,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense causal GQA comparison")
+    ap.add_argument("--q-chunk", type=int, default=-1,
+                    help="query rows per attention pass (-1: 131072 above 128K tokens, else one pass)")
     ap.add_argument("--theta", type=int, default=-1,
                     help="query-tile threshold of the prefill (-1 automatic, 0 off)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
