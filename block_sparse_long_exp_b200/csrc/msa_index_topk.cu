@@ -95,6 +95,10 @@ struct TopList {
   // Candidates arrive with ascending j; a full list only takes a strictly
   // higher score than its last entry.
   __device__ __forceinline__ void offer(float s, int j, int cap) {
+    if (cap == CAP && n == CAP) {
+      offer_full(s, j);
+      return;
+    }
     if (n >= cap && !(s > thr)) return;
     bool gt[CAP];
 #pragma unroll
@@ -116,6 +120,23 @@ struct TopList {
 #pragma unroll
     for (int i = 0; i < CAP; ++i) t = fminf(t, (i < cap) ? sc[i] : INFINITY);
     thr = t;
+  }
+  // The common case: all CAP entries in use (cap == CAP).  Sorted descending,
+  // so the threshold is the last entry; no capacity checks, no min pass.
+  __device__ __forceinline__ void offer_full(float s, int j) {
+    if (!(s > sc[CAP - 1])) return;
+    bool gt[CAP];
+#pragma unroll
+    for (int i = 0; i < CAP; ++i) gt[i] = s > sc[i];
+#pragma unroll
+    for (int i = CAP - 1; i >= 1; --i) {
+      const float ns = gt[i - 1] ? sc[i - 1] : (gt[i] ? s : sc[i]);
+      const int ni = gt[i - 1] ? ix[i - 1] : (gt[i] ? j : ix[i]);
+      sc[i] = ns;
+      ix[i] = ni;
+    }
+    if (gt[0]) { sc[0] = s; ix[0] = j; }
+    thr = sc[CAP - 1];
   }
   // Write the selection ascending: the n chosen ids, then the local block,
   // then -1 padding.
