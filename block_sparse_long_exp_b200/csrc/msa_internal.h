@@ -16,7 +16,7 @@ constexpr int kWindow = 4096;         // query rows per attention planning windo
 constexpr int kScanTile = 4096;       // keys per CTA of the planning scan
 constexpr int kMaxItemQueries = 64;   // queries per attention work item (upper bound)
 constexpr int kMaxDense = 64;         // dense blocks per query tile (Q-outer side)
-constexpr int32_t kDenseComplete = 0x100;   // dstate flag: the tile covers every selection of the query
+constexpr int32_t kDenseComplete = 1;   // dstate: the tile covers every selection of the query
 
 // Device error word, at offset 0 of every workspace.
 struct DevError {
@@ -120,7 +120,7 @@ struct AttnArgs {
   int32_t* unit_nblk;  // [units x G]
   int32_t* unit_list;  // [units x G] units with dense blocks
   uint32_t* dmask;     // [(t1-t0) x G] slots covered by the tile
-  int32_t* dstate;     // [(t1-t0) x G] first covered slot | kDenseComplete, or -1
+  int32_t* dstate;     // [(t1-t0) x G] -1: no slot covered; 0: some; kDenseComplete: all
   uint64_t* dmember;   // [(t1-t0) x G] positions of the covered blocks in the tile's list
   uint2* clist;        // [(t1-t0) x G] combine list: {pair (t - t0) * G + g, slots to merge}
   int32_t* tile_ctr;   // [4]: pairs, listed units, unit ticket

@@ -172,7 +172,7 @@ tile_plan_kernel(const int32_t* __restrict__ sel, int64_t t0, int64_t t1, int G,
     const bool complete = dm != 0 && dm == vm;
     dmask[pr] = dm;
     dmember[pr] = mem;
-    dstate[pr] = dm == 0 ? -1 : ((__ffs(dm) - 1) | (complete ? kDenseComplete : 0));
+    dstate[pr] = dm == 0 ? -1 : (complete ? kDenseComplete : 0);
     need_combine = !complete;
     cmask = (uint32_t)__popc(vm & ~dm) + (dm != 0u ? 1u : 0u);   // packed: the tile's, then the KV-outer ones
   }
@@ -232,7 +232,7 @@ struct TileParams {
   const int32_t* unit_blk;    // hybrid: [units x G][kMaxDense]
   const int32_t* unit_nblk;
   const uint64_t* dmember;    // hybrid: [rows x G] dense-list membership bits
-  const int32_t* dstate;      // hybrid: [rows x G] kDenseComplete | first covered slot, or -1
+  const int32_t* dstate;      // tiles mode: [rows x G] -1 none covered, 0 some, kDenseComplete all
   const int32_t* seq_units;   // dense: [batch + 1] prefix of units per sequence
   const int32_t* nunits;      // device count of units (tiles: listed units; dense: all); null: nunits_host
   int64_t nunits_host;        // rows mode: rows x G

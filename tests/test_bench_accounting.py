@@ -1,0 +1,90 @@
+"""The bench's per-kernel work split (roofline.tile_split, vectorised with torch
+sorting) against the planner's rule written out with plain loops: tiles of
+UQ consecutive rows of a pass that lie in one sequence; a block chosen by at
+least theta of a tile's queries (one group) is covered; a query whose every
+selection is covered needs no combine."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import msa_oracle as O
+from block_sparse_long_exp_b200 import roofline as R
+
+
+def _selection(lengths, G, k, seed):
+    rng = np.random.default_rng(seed)
+    S = sum(lengths)
+    d_idx = 8
+    q_idx = rng.integers(-2, 3, size=(S, G, d_idx)).astype(np.float64)
+    k_idx = rng.integers(-2, 3, size=(S, d_idx)).astype(np.float64)
+    cu = [0]
+    for L in lengths:
+        cu.append(cu[-1] + L)
+    return O.index_topk(q_idx, k_idx, cu, cu, k, 128), cu
+
+
+def _brute(sel, cu, H, G, d, theta, q_chunk):
+    T, _, k = sel.shape
+    Hg = H // G
+    UQ = 2 * (128 // max(Hg, 8))
+    qpt = UQ // 2
+    seq_of = np.searchsorted(np.array(cu), np.arange(T), side="right") - 1
+    pos = np.array([t - cu[seq_of[t]] for t in range(T)])     # prefill: S_b == T_b
+    covered = np.zeros(sel.shape, dtype=bool)
+    mma_tiles = 0
+    rows = T if q_chunk <= 0 else q_chunk
+    for t0 in range(0, T, rows):
+        t1 = min(T, t0 + rows)
+        for r0 in range(t0, t1, UQ):
+            r1 = min(t1, r0 + UQ)
+            if seq_of[r0] != seq_of[r1 - 1] or theta <= 0:
+                continue
+            for g in range(G):
+                count = {}
+                for t in range(r0, r1):
+                    for b in sel[t, g]:
+                        if b >= 0:
+                            count[int(b)] = count.get(int(b), 0) + 1
+                dense = {b for b, c in count.items() if c >= theta}
+                mma_tiles += len(dense) * (2 if r1 - r0 > qpt else 1)
+                for t in range(r0, r1):
+                    for s in range(k):
+                        covered[t, g, s] = sel[t, g, s] >= 0 and int(sel[t, g, s]) in dense
+    tile = kv = 0
+    merged = npairs = complete = 0
+    for t in range(T):
+        lb = pos[t] // 128
+        for g in range(G):
+            valid = sel[t, g] >= 0
+            for s in range(k):
+                if not valid[s]:
+                    continue
+                att = 128 if sel[t, g, s] < lb else pos[t] % 128 + 1
+                if covered[t, g, s]:
+                    tile += att
+                else:
+                    kv += att
+            ncov = covered[t, g].sum()
+            if ncov > 0 and ncov == valid.sum():
+                complete += 1
+            else:
+                npairs += 1
+                merged += (valid & ~covered[t, g]).sum() + (1 if ncov > 0 else 0)
+    comb = merged * Hg * (d * 2 + 4) + npairs * 8 + npairs * (Hg * d * 2 + Hg * 4)
+    return {"tile_flops": 4.0 * d * Hg * tile, "kv_flops": 4.0 * d * Hg * kv, "combine_bytes": float(comb),
+            "combine_pairs": npairs, "complete_pairs": complete,
+            "tile_mma_flops": float(mma_tiles * 4 * 128 * 128 * d)}
+
+
+@pytest.mark.parametrize("H,G", [(64, 4), (8, 2)])
+@pytest.mark.parametrize("theta,q_chunk", [(0, 0), (1, 0), (3, 0), (5, 0), (3, 300)])
+def test_tile_split_matches_the_rule(H, G, theta, q_chunk):
+    lengths = [1500, 130, 917]                    # up to 12 blocks, k = 4: real top-k choices
+    sel, cu = _selection(lengths, G, k=4, seed=5)
+    got = R.tile_split(torch.from_numpy(sel), cu, cu, H, G, 64, 128, theta, q_chunk)
+    ref = _brute(sel, cu, H, G, 64, theta, q_chunk)
+    for key, v in ref.items():
+        assert got[key] == pytest.approx(v), key
+    # the split never loses work: it always adds up to the method's main-branch FLOPs
+    work = R.prefill_work(lengths, lengths, H, G, 64, 8, 128, 4)
+    assert got["tile_flops"] + got["kv_flops"] == pytest.approx(work["main_flops"])
