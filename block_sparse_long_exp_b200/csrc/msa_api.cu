@@ -117,7 +117,8 @@ msa_status_t attn_common(const msa_shape_t* shape, const msa_varlen_t* seqs, con
   if (st != MSA_OK) return st;
   st = check_seqs(seqs);
   if (st != MSA_OK) return st;
-  if (!q || !k || !v || !sel || !out) return MSA_ERR_INVALID_ARG;
+  // no queries: nothing is read or written (empty tensors may have no storage)
+  if (seqs->total_q > 0 && (!q || !k || !v || !sel || !out)) return MSA_ERR_INVALID_ARG;
   if (seqs->total_q == 0) return MSA_OK;
   const int64_t rows = chunk_rows(seqs, q_chunk);
   const AttnLayout L = attn_layout(shape, seqs, rows);
@@ -256,7 +257,7 @@ msa_status_t msa_index_topk(const msa_shape_t* shape, const msa_varlen_t* seqs, 
   if (st != MSA_OK) return st;
   st = check_seqs(seqs);
   if (st != MSA_OK) return st;
-  if (!q_idx || !k_idx || !sel) return MSA_ERR_INVALID_ARG;
+  if (seqs->total_q > 0 && (!q_idx || !k_idx || !sel)) return MSA_ERR_INVALID_ARG;
   const size_t need = msa_index_topk_workspace_size(shape, seqs);
   if (!ws_ok(ws, ws_bytes, need)) return MSA_ERR_WORKSPACE;
   if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
@@ -303,10 +304,11 @@ msa_status_t msa_combine(const msa_shape_t* shape, int64_t T, const void* part_a
                          const int32_t* sel, void* out, float* lse, void* stream) {
   msa_status_t st = check_shape(shape);
   if (st != MSA_OK) return st;
-  if (T < 0 || !part_acc || !part_lse || !sel || !out) return MSA_ERR_INVALID_ARG;
+  if (T < 0) return MSA_ERR_INVALID_ARG;
+  if (T == 0) return MSA_OK;                 // nothing to merge (pointers may be NULL)
+  if (!part_acc || !part_lse || !sel || !out) return MSA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(part_acc) | reinterpret_cast<uintptr_t>(part_lse)) & 15u)
     return MSA_ERR_INVALID_ARG;   // streamed with 16-byte bulk copies
-  if (T == 0) return MSA_OK;
   return launch_combine(part_acc, part_lse, sel, out, lse, T, shape->H, shape->G, shape->d, shape->k, stream) == 0
              ? MSA_OK
              : MSA_ERR_CUDA;
@@ -323,7 +325,7 @@ msa_status_t msa_dense_attn(const msa_shape_t* shape, const msa_varlen_t* seqs, 
   if (st != MSA_OK) return st;
   st = check_seqs(seqs);
   if (st != MSA_OK) return st;
-  if (!q || !k || !v || !out) return MSA_ERR_INVALID_ARG;
+  if (seqs->total_q > 0 && (!q || !k || !v || !out)) return MSA_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, msa_dense_attn_workspace_size(shape, seqs))) return MSA_ERR_WORKSPACE;
   if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MSA_ERR_CUDA;

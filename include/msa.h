@@ -63,6 +63,10 @@
 extern "C" {
 #endif
 
+/* A call with no queries (total_q == 0; T == 0 for msa_combine) launches
+ * nothing and returns MSA_OK after the argument checks; its data pointers may
+ * then be NULL (empty tensors need no storage).  The workspace rules still
+ * apply and its error word is cleared. */
 typedef enum {
   MSA_OK = 0,
   MSA_ERR_INVALID_ARG = 1,
