@@ -1,5 +1,5 @@
 """The bench's N > 1 path on CPU: two gloo ranks (127.0.0.1) run the same
-reductions the NCCL ranks run on the GPU machine -- the slowest rank's time, the
+reductions the NCCL ranks run on GPUs -- the slowest rank's time, the
 sum of all ranks' tokens -- and draw their independent layers (weak scaling:
 same shapes, different seeds)."""
 import importlib.util
