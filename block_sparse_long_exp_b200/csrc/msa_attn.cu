@@ -4,17 +4,23 @@
 // yololab.net "KV Outer Gather Q").
 //
 // A pass over query rows [t0, t1):
-//   1. count    : per (sequence, group, block) list, how many (query, slot)
-//                 entries chose it (warp-aggregated atomics);
+//   0. tiles    : (msa_tile_attn.cu) the blocks that many queries of a small
+//                 query tile share are marked for the query-tile kernel;
+//   1. count    : per (window, sequence, group, block) list, how many of the
+//                 remaining (query, slot) entries chose it (warp-aggregated
+//                 atomics);
 //   2. plan     : exclusive scans -> list offsets, work items of at most
 //                 `queries_per_item` queries per list;
-//   3. scatter  : list entries (t - t0) * k + slot;
+//   3. scatter  : list entries (t - t0) * k + packed slot;
 //   4. attend   : one work item = one KV block (TMA, loaded once) and up to
 //                 queries_per_item gathered queries; per 128-row tile
 //                 (128 / Hg queries x Hg heads) S = Q K^T and O = P V run on
 //                 tcgen05 with fp32 accumulators in TMEM; each (query, group,
 //                 block) writes its normalised output (f16) and log-sum-exp;
-//   5. combine  : per (query, head) log-sum-exp merge of its partials.
+//      (the query-tile kernel then writes the shared blocks' results: final
+//      outputs, or one merged partial per query)
+//   5. combine  : per (query, head) log-sum-exp merge of the packed partials
+//                 of every query on the combine list.
 #include "msa_common.cuh"
 
 namespace msa {
@@ -238,7 +244,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_items_kernel(const int32_t*
 
 // ------------------------------------------------------------ attention ---
 //
-// Warp-specialised, persistent (one CTA per SM, 384 threads):
+// Warp-specialised, persistent (one CTA per SM, 512 threads):
 //   warp 0      claims work items (atomic ticket) and publishes each one with
 //               its query entries in a 4-deep shared-memory ring; lane 0 then
 //               TMA-loads the item's K and V block into one of two stages and
@@ -249,9 +255,9 @@ __global__ void __launch_bounds__(kScanThreads) scan_items_kernel(const int32_t*
 //               so the tensor core works on the next tile while tile t's
 //               softmax runs (warps 2 and 3 are idle);
 //   warps 4-7   softmax of even tiles (TMEM slot 0), warps 8-11 of odd tiles
-//               (slot 1): S -> P (bf16, written back into the S columns, the A
-//               operand of the PV MMA); each row's max and sum go to shared
-//               memory (double-buffered per slot);
+//               (slot 1): S -> P (bf16, written back into the first 64 S
+//               columns, the A operand of the PV MMA); each row's sum goes to
+//               shared memory for the epilogue, its log-sum-exp to the partials;
 //   warps 12-15 epilogue of every tile in order: O / l -> f16 partial and the
 //               log-sum-exp of each row.
 // A query occupies RQ = max(Hg, 8) tile rows (its Hg heads; with Hg = 4 the
