@@ -71,3 +71,35 @@ def test_host_validation_without_gpu(lib):
     more_q_than_k = msa.Varlen(1, 2048, 1024, 0, 2048, 1024, ctypes.addressof(cu), ctypes.addressof(cu))
     rc = lib.msa_index_topk(ctypes.byref(shape), ctypes.byref(more_q_than_k), 1, 1, 1, 1, 1 << 20, None)
     assert rc == 1
+
+
+def test_paged_decode_host_validation_without_gpu(lib):
+    from block_sparse_long_exp_b200 import msa
+    shape = msa.make_shape(64, 4, 128, 64, 16)
+    lens = (ctypes.c_int32 * 2)(1000, 300)
+    table = (ctypes.c_int32 * 16)(*range(16))
+    ok = msa.Paged(2, 8, 1000, 0, 64, ctypes.addressof(lens), ctypes.addressof(table))
+    assert lib.msa_decode_paged_workspace_size(ctypes.byref(shape), ctypes.byref(ok)) >= 256
+    # lengths beyond the table, missing pointers, too many pages: rejected before any launch
+    too_long = msa.Paged(2, 8, 8 * 128 + 1, 0, 64, ctypes.addressof(lens), ctypes.addressof(table))
+    assert lib.msa_decode_paged_workspace_size(ctypes.byref(shape), ctypes.byref(too_long)) == 0
+    no_table = msa.Paged(2, 8, 1000, 0, 64, ctypes.addressof(lens), None)
+    rc = lib.msa_index_topk_decode_paged(ctypes.byref(shape), ctypes.byref(no_table), 1, 1, 1, 1, 1 << 20, None)
+    assert rc == 1                                       # MSA_ERR_INVALID_ARG
+    huge = msa.Paged(2, 8, 1000, 0, 1 << 26, ctypes.addressof(lens), ctypes.addressof(table))
+    rc = lib.msa_sparse_attn_decode_paged(ctypes.byref(shape), ctypes.byref(huge), 1, 1, 1, 1, 1, None, 1, 1 << 20,
+                                          None)
+    assert rc == 2                                       # MSA_ERR_UNSUPPORTED (rows past int32)
+    rc = lib.msa_sparse_attn_decode_paged(ctypes.byref(shape), ctypes.byref(ok), 1, 1, 1, 1, 1, None, 256, 16, None)
+    assert rc == 3                                       # MSA_ERR_WORKSPACE
+
+
+def test_tile_threshold_setting_round_trips(lib):
+    from block_sparse_long_exp_b200 import msa
+    prev = msa.msa_set_tile_threshold(0)
+    try:
+        assert msa.msa_set_tile_threshold(7) == 0
+        assert msa.msa_set_tile_threshold(-5) == 7        # any negative value means automatic
+        assert msa.msa_set_tile_threshold(-1) == -1
+    finally:
+        msa.msa_set_tile_threshold(prev)
