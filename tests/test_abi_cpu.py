@@ -103,3 +103,21 @@ def test_tile_threshold_setting_round_trips(lib):
         assert msa.msa_set_tile_threshold(-1) == -1
     finally:
         msa.msa_set_tile_threshold(prev)
+
+
+def test_plain_c_program_uses_the_boundary(lib, tmp_path):
+    """A C program that includes only include/msa.h and links libmsa.so."""
+    import shutil
+    import subprocess
+    from block_sparse_long_exp_b200 import msa
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(msa.LIB_PATH)
+    exe = tmp_path / "abi_host"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c", "abi_host.c"), "-L", libdir, "-lmsa",
+                    "-Wl,-rpath," + libdir, "-o", str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    assert "abi_host ok" in r.stdout
