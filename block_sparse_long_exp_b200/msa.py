@@ -4,6 +4,22 @@ Argument marshalling only: every step of the MSA forward runs in the CUDA
 kernels of libmsa.so.  PyTorch provides device memory and streams.  The
 functions carry the C entry points' names.  There is no fallback: if the
 library is missing or no CUDA device is present, every call raises.
+
+One layer's forward (packed sequences; queries are the last T_b tokens of
+each sequence, all tensors bf16 on the GPU except the int32 offsets):
+
+    shape = make_shape(H=64, G=4, d=128, d_idx=64, k=16)        # B_k = 128
+    seqs = make_varlen(cu_q, cu_k, cu_q_host, cu_k_host)
+    sel = msa_index_topk(shape, seqs, q_idx, k_idx)              # [T, G, k] int32
+    out, lse = msa_sparse_attn_prefill(shape, seqs, q, k, v, sel) # [T, H, d], [T, H]
+
+with q [T, H, d], k / v [S, G, d], q_idx [T, G, d_idx], k_idx [S, d_idx].
+Decode (one query per sequence) is msa_index_topk + msa_sparse_attn_decode,
+or the *_decode_paged pair over a paged cache (make_paged).  Each call
+allocates its workspace unless `ws` is given, and by default reads the
+device error word afterwards (a synchronisation); pass check=False inside
+timed or captured regions and call msa_get_device_error on the workspace
+later.
 """
 from __future__ import annotations
 
@@ -153,6 +169,9 @@ def _require_cuda(t: torch.Tensor):
 def msa_index_topk(shape: Shape, seqs: Varlen, q_idx: torch.Tensor, k_idx: torch.Tensor,
                    sel: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
                    stream=None, check: bool = True) -> torch.Tensor:
+    """Index branch: scores, block max-pool and top-k with the forced local
+    block.  Returns sel [T, G, k] int32: the selected block ids of each
+    (query, group), ascending, padded with -1."""
     lib = load_library()
     _require_cuda(q_idx)
     T = seqs.total_q
@@ -197,6 +216,10 @@ def msa_sparse_attn_prefill(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torc
                             lse: Optional[torch.Tensor] = None, want_lse: bool = True, q_chunk: int = 0,
                             ws: Optional[torch.Tensor] = None, stream=None,
                             check: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Main branch: exact causal softmax attention of every query over the
+    tokens of its selected blocks.  Returns out [T, H, d] bf16 and lse [T, H]
+    (natural log; None with want_lse=False).  q_chunk > 0 runs the attention
+    in passes of that many query rows (bounded workspace)."""
     lib = load_library()
     _require_cuda(q)
     T = seqs.total_q
@@ -223,6 +246,8 @@ def msa_sparse_attn_decode(shape: Shape, seqs: Varlen, q: torch.Tensor, k_cache:
                            lse: Optional[torch.Tensor] = None, want_lse: bool = True,
                            ws: Optional[torch.Tensor] = None, stream=None,
                            check: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Main branch for one query per sequence (its position is the cache's
+    last token).  Same outputs as msa_sparse_attn_prefill."""
     lib = load_library()
     _require_cuda(q)
     T = seqs.total_q
