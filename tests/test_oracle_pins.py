@@ -298,3 +298,62 @@ def test_invert_selection_round_trip():
         for g in range(G):
             want = [int(x) for x in sel[t, g] if x >= 0]
             assert sorted(rebuilt[(t, g)]) == want
+
+
+# -------------------------------------------------- randomised properties ----
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@st.composite
+def _tiny_layer(draw):
+    G = draw(st.sampled_from([1, 2]))
+    Hg = draw(st.sampled_from([1, 2]))
+    B_k = draw(st.sampled_from([3, 4]))
+    k = draw(st.integers(1, 5))
+    nseq = draw(st.integers(1, 3))
+    S_lens = [draw(st.integers(1, 24)) for _ in range(nseq)]
+    T_lens = [draw(st.integers(0, S)) for S in S_lens]
+    seed = draw(st.integers(0, 2 ** 31 - 1))
+    return G, Hg, B_k, k, S_lens, T_lens, seed
+
+
+@settings(max_examples=60, deadline=None)
+@given(_tiny_layer())
+def test_random_layers_match_brute_force_and_masked_sdpa(layer):
+    """Random varlen layers (queries are the last T_b tokens): the selection
+    equals subset enumeration, the output equals fp64 SDPA with a token mask
+    built by loops, sequence by sequence."""
+    G, Hg, B_k, k, S_lens, T_lens, seed = layer
+    rng = np.random.default_rng(seed)
+    H, d, d_idx = G * Hg, 4, 3
+    S, T = sum(S_lens), sum(T_lens)
+    cu_k = np.concatenate([[0], np.cumsum(S_lens)]).tolist()
+    cu_q = np.concatenate([[0], np.cumsum(T_lens)]).tolist()
+    q = rng.standard_normal((T, H, d))
+    kk = rng.standard_normal((S, G, d))
+    v = rng.standard_normal((S, G, d))
+    q_idx = rng.integers(-2, 3, size=(T, G, d_idx)).astype(np.float64)
+    k_idx = rng.integers(-2, 3, size=(S, d_idx)).astype(np.float64)
+    sel = O.index_topk(q_idx, k_idx, cu_q, cu_k, k, B_k)
+    scale = 1 / math.sqrt(d)
+    o, _ = O.msa_forward_rows(q, kk, v, sel, cu_q, cu_k, list(range(T)), B_k, scale)
+    for b in range(len(S_lens)):
+        Tb, Sb = T_lens[b], S_lens[b]
+        if Tb == 0:
+            continue
+        ks = k_idx[cu_k[b]:cu_k[b + 1]]
+        mask = np.zeros((H, Tb, Sb), dtype=bool)
+        for i in range(Tb):
+            t, pos = cu_q[b] + i, Sb - Tb + i
+            for g in range(G):
+                want = _brute_select(q_idx[t, g], ks, pos, B_k, k)
+                got = [int(x) for x in sel[t, g] if x >= 0]
+                assert got == want, (b, i, g)
+                for h in range(g * Hg, (g + 1) * Hg):
+                    for j in range(pos + 1):
+                        mask[h, i, j] = (j // B_k) in want
+        # SDPA over this sequence's queries and keys
+        qb = q[cu_q[b]:cu_q[b + 1]]
+        ref = _sdpa(qb, kk[cu_k[b]:cu_k[b + 1]], v[cu_k[b]:cu_k[b + 1]], mask, scale)
+        np.testing.assert_allclose(o[cu_q[b]:cu_q[b + 1]], ref, rtol=0, atol=1e-12)
