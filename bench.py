@@ -229,16 +229,45 @@ def traffic_for(kernel):
     return d.get("dram_bytes_per_launch") if sha is not None and sha == d.get("source_sha") else None
 
 
+def code_tokens(text):
+    """C/C++/CUDA source with its comments removed (string and character
+    literals kept as they are), whitespace runs collapsed and blank lines
+    dropped: two sources with equal results differ only in comments or layout."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":                                   # literal: copy through its closing quote
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (" ".join(line.split()) for line in "".join(out).split("\n"))
+    return "\n".join(line for line in lines if line)
+
+
 def kernel_source_sha(source):
-    """Hash of a kernel's .cu file together with the headers every kernel
-    includes (a change to either makes recorded counters stale)."""
+    """Hash of the code (comments and layout ignored) of a kernel's .cu file
+    together with the headers every kernel includes: a change to the code of
+    either makes recorded counters stale."""
     csrc = os.path.join(ROOT, "block_sparse_long_exp_b200", "csrc")
     h = hashlib.sha256()
     for f in (source, "msa_common.cuh", "msa_internal.h"):
         p = os.path.join(csrc, f)
         if not f or not os.path.exists(p):
             return None
-        h.update(open(p, "rb").read())
+        h.update(code_tokens(open(p, encoding="utf-8").read()).encode())
+        h.update(b"\0")
     return h.hexdigest()[:16]
 
 

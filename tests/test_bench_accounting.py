@@ -88,3 +88,30 @@ def test_tile_split_matches_the_rule(H, G, theta, q_chunk):
     # the split never loses work: it always adds up to the method's main-branch FLOPs
     work = R.prefill_work(lengths, lengths, H, G, 64, 8, 128, 4)
     assert got["tile_flops"] + got["kv_flops"] == pytest.approx(work["main_flops"])
+
+
+def test_code_hash_ignores_comments_and_layout_only():
+    """roofline.traffic stays valid across comment edits, not across code edits."""
+    import bench
+    a = 'int x = 1; // note\n/* a\n block */ float y;\nconst char* s = "// kept";\nchar c = \'"\';\n'
+    b = 'int x = 1;\n\n   float   y;   // other note\nconst char* s = "// kept";\nchar c = \'"\';\n'
+    c = 'int x = 2; // note\n float y;\nconst char* s = "// kept";\nchar c = \'"\';\n'
+    d = 'int x = 1;\n float y;\nconst char* s = "// kept!";\nchar c = \'"\';\n'
+    T = bench.code_tokens
+    assert T(a) == T(b)
+    assert T(a) != T(c) and T(a) != T(d)          # code and string literals count
+    assert "// kept" in T(a)
+
+
+def test_recorded_traffic_matches_current_code():
+    """Every entry of profiles/traffic.json names a kernel file that exists, and the
+    bench reads its figure back exactly when the code hash matches."""
+    import json
+    import os
+    import bench
+    d = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    for name, e in d.items():
+        sha = bench.kernel_source_sha(e["source"])
+        assert sha is not None, name
+        want = e["dram_bytes_per_launch"] if sha == e["source_sha"] else None
+        assert bench.traffic_for(name) == want
