@@ -20,6 +20,12 @@ allocates its workspace unless `ws` is given, and by default reads the
 device error word afterwards (a synchronisation); pass check=False inside
 timed or captured regions and call msa_get_device_error on the workspace
 later.
+
+Every call checks its tensors on the host first (dtype, exact shape of the
+layout above, row-major contiguity, one CUDA device) and make_varlen checks
+the offsets (start at 0, never decrease, T_b <= S_b); a failed check raises
+MsaError before anything reaches the GPU, since the C entry points receive
+bare pointers and cannot see a buffer's size.
 """
 from __future__ import annotations
 
@@ -149,11 +155,35 @@ def make_shape(H: int, G: int, d: int, d_idx: int, k: int, B_k: int = 128,
 
 def make_varlen(cu_q: torch.Tensor, cu_k: torch.Tensor, cu_q_host: Sequence[int],
                 cu_k_host: Sequence[int]) -> Varlen:
-    """cu_q / cu_k: int32 device tensors [B+1]; the host copies give the sizes."""
+    """cu_q / cu_k: int32 device tensors [B+1]; the host copies give the sizes
+    and must hold the same values (they are not read back from the device).
+    Checks on the host: both start at 0 and never decrease, T_b <= S_b for
+    every sequence, totals fit int32."""
+    cu_q_host = [int(x) for x in cu_q_host]
+    cu_k_host = [int(x) for x in cu_k_host]
+    if len(cu_q_host) < 1 or len(cu_q_host) != len(cu_k_host):
+        raise MsaError(f"make_varlen: cu_q_host has {len(cu_q_host)} entries, cu_k_host {len(cu_k_host)} "
+                       "(both need batch + 1)")
+    if cu_q_host[0] != 0 or cu_k_host[0] != 0:
+        raise MsaError("make_varlen: cu_q_host and cu_k_host must start at 0")
     T_lens = [cu_q_host[i + 1] - cu_q_host[i] for i in range(len(cu_q_host) - 1)]
     S_lens = [cu_k_host[i + 1] - cu_k_host[i] for i in range(len(cu_k_host) - 1)]
-    return Varlen(len(T_lens), max(T_lens) if T_lens else 0, max(S_lens) if S_lens else 0, 0,
-                  int(cu_q_host[-1]), int(cu_k_host[-1]), cu_q.data_ptr(), cu_k.data_ptr())
+    for b, (Tb, Sb) in enumerate(zip(T_lens, S_lens)):
+        if Tb < 0 or Sb < 0:
+            raise MsaError(f"make_varlen: offsets decrease at sequence {b}")
+        if Tb > Sb:
+            raise MsaError(f"make_varlen: sequence {b} has {Tb} queries but {Sb} keys "
+                           "(queries are the last T_b of its tokens)")
+    if cu_k_host[-1] >= 2 ** 31 or cu_q_host[-1] >= 2 ** 31:
+        raise MsaError("make_varlen: totals beyond int32 offsets")
+    B = len(T_lens)
+    _arg("cu_q", cu_q, torch.int32, shape=(B + 1,))
+    _arg("cu_k", cu_k, torch.int32, shape=(B + 1,))
+    _require_cuda(cu_q, cu_k)
+    v = Varlen(B, max(T_lens) if T_lens else 0, max(S_lens) if S_lens else 0, 0,
+               cu_q_host[-1], cu_k_host[-1], cu_q.data_ptr(), cu_k.data_ptr())
+    v._keep = (cu_q, cu_k)
+    return v
 
 
 def _workspace(nbytes: int, device) -> torch.Tensor:
@@ -161,9 +191,56 @@ def _workspace(nbytes: int, device) -> torch.Tensor:
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
-def _require_cuda(t: torch.Tensor):
-    if not t.is_cuda:
-        raise MsaError("the MSA kernels need CUDA tensors (no CPU path exists)")
+def _require_cuda(*ts: Optional[torch.Tensor]):
+    """Every given tensor lives on one CUDA device (the kernels read them
+    through plain device pointers)."""
+    dev = None
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise MsaError("the MSA kernels need CUDA tensors (no CPU path exists)")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise MsaError(f"tensors on different devices ({dev} and {t.device})")
+
+
+def _arg(name: str, t, dtype: torch.dtype, shape: Optional[Sequence[int]] = None,
+         numel: Optional[int] = None, optional: bool = False):
+    """Host check of one tensor argument against the layout the C entry point
+    reads: dtype, exact shape (or element count for blocked layouts) and
+    row-major contiguity.  Raises MsaError before anything reaches the device."""
+    if t is None:
+        if optional:
+            return
+        raise MsaError(f"{name}: a tensor is required")
+    if not isinstance(t, torch.Tensor):
+        raise MsaError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise MsaError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(int(x) for x in shape):
+        raise MsaError(f"{name}: shape {tuple(t.shape)}, expected {tuple(int(x) for x in shape)}")
+    if numel is not None and t.numel() != int(numel):
+        raise MsaError(f"{name}: {t.numel()} elements, expected {int(numel)}")
+    if not t.is_contiguous():
+        raise MsaError(f"{name}: must be contiguous (row-major)")
+
+
+def _ws_arg(ws: Optional[torch.Tensor]):
+    if ws is not None and not (isinstance(ws, torch.Tensor) and ws.is_contiguous()):
+        raise MsaError("ws: expected a contiguous tensor")
+
+
+def _nbytes(t: torch.Tensor) -> int:
+    return t.numel() * t.element_size()
+
+
+def _groups(shape: Shape) -> int:
+    """Heads per group; the C entry points reject the shape if H % G != 0."""
+    if shape.G <= 0 or shape.H % shape.G != 0:
+        raise MsaError(f"shape: H = {shape.H} is not a multiple of G = {shape.G}")
+    return shape.H // shape.G
 
 
 def msa_index_topk(shape: Shape, seqs: Varlen, q_idx: torch.Tensor, k_idx: torch.Tensor,
@@ -173,8 +250,12 @@ def msa_index_topk(shape: Shape, seqs: Varlen, q_idx: torch.Tensor, k_idx: torch
     block.  Returns sel [T, G, k] int32: the selected block ids of each
     (query, group), ascending, padded with -1."""
     lib = load_library()
-    _require_cuda(q_idx)
-    T = seqs.total_q
+    T, S = seqs.total_q, seqs.total_k
+    _arg("q_idx", q_idx, torch.bfloat16, (T, shape.G, shape.d_idx))
+    _arg("k_idx", k_idx, torch.bfloat16, (S, shape.d_idx))
+    _arg("sel", sel, torch.int32, (T, shape.G, shape.k), optional=True)
+    _ws_arg(ws)
+    _require_cuda(q_idx, k_idx, sel, ws)
     if sel is None:
         sel = torch.empty((T, shape.G, shape.k), dtype=torch.int32, device=q_idx.device)
     need = lib.msa_index_topk_workspace_size(ctypes.byref(shape), ctypes.byref(seqs))
@@ -183,7 +264,7 @@ def msa_index_topk(shape: Shape, seqs: Varlen, q_idx: torch.Tensor, k_idx: torch
     if ws is None:
         ws = _workspace(need, q_idx.device)
     rc = lib.msa_index_topk(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q_idx), _ptr(k_idx), _ptr(sel),
-                            _ptr(ws), ws.numel(), _stream(stream))
+                            _ptr(ws), _nbytes(ws), _stream(stream))
     _check(rc, "msa_index_topk")
     if check:
         _device_check(ws, stream, "msa_index_topk")
@@ -196,7 +277,15 @@ def msa_index_topk_decode_noalloc(shape: Shape, seqs: Varlen, q_idx: torch.Tenso
     """Decode-shaped index top-k on the library's fixed scratch array (no
     workspace argument, no allocation inside the call).  `sel` must be given."""
     lib = load_library()
-    _require_cuda(q_idx)
+    T, S = seqs.total_q, seqs.total_k
+    _arg("q_idx", q_idx, torch.bfloat16, (T, shape.G, shape.d_idx))
+    _arg("k_idx", k_idx, torch.bfloat16, (S, shape.d_idx))
+    _arg("sel", sel, torch.int32, (T, shape.G, shape.k))
+    if device_error is not None:
+        _arg("device_error", device_error, torch.int32)
+        if device_error.numel() < 1:
+            raise MsaError("device_error: needs one int32 element")
+    _require_cuda(q_idx, k_idx, sel, device_error)
     rc = lib.msa_index_topk_decode_noalloc(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q_idx), _ptr(k_idx),
                                            _ptr(sel), _ptr(device_error), _stream(stream))
     _check(rc, "msa_index_topk_decode_noalloc")
@@ -221,8 +310,15 @@ def msa_sparse_attn_prefill(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torc
     (natural log; None with want_lse=False).  q_chunk > 0 runs the attention
     in passes of that many query rows (bounded workspace)."""
     lib = load_library()
-    _require_cuda(q)
-    T = seqs.total_q
+    T, S = seqs.total_q, seqs.total_k
+    _arg("q", q, torch.bfloat16, (T, shape.H, shape.d))
+    _arg("k", k, torch.bfloat16, (S, shape.G, shape.d))
+    _arg("v", v, torch.bfloat16, (S, shape.G, shape.d))
+    _arg("sel", sel, torch.int32, (T, shape.G, shape.k))
+    _arg("out", out, torch.bfloat16, (T, shape.H, shape.d), optional=True)
+    _arg("lse", lse, torch.float32, (T, shape.H), optional=True)
+    _ws_arg(ws)
+    _require_cuda(q, k, v, sel, out, lse, ws)
     if out is None:
         out = torch.empty((T, shape.H, shape.d), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
@@ -233,7 +329,7 @@ def msa_sparse_attn_prefill(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torc
     if ws is None:
         ws = _workspace(need, q.device)
     rc = lib.msa_sparse_attn_prefill(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q), _ptr(k), _ptr(v),
-                                     _ptr(sel), _ptr(out), _ptr(lse), q_chunk, _ptr(ws), ws.numel(),
+                                     _ptr(sel), _ptr(out), _ptr(lse), q_chunk, _ptr(ws), _nbytes(ws),
                                      _stream(stream))
     _check(rc, "msa_sparse_attn_prefill")
     if check:
@@ -249,8 +345,15 @@ def msa_sparse_attn_decode(shape: Shape, seqs: Varlen, q: torch.Tensor, k_cache:
     """Main branch for one query per sequence (its position is the cache's
     last token).  Same outputs as msa_sparse_attn_prefill."""
     lib = load_library()
-    _require_cuda(q)
-    T = seqs.total_q
+    T, S = seqs.total_q, seqs.total_k
+    _arg("q", q, torch.bfloat16, (T, shape.H, shape.d))
+    _arg("k_cache", k_cache, torch.bfloat16, (S, shape.G, shape.d))
+    _arg("v_cache", v_cache, torch.bfloat16, (S, shape.G, shape.d))
+    _arg("sel", sel, torch.int32, (T, shape.G, shape.k))
+    _arg("out", out, torch.bfloat16, (T, shape.H, shape.d), optional=True)
+    _arg("lse", lse, torch.float32, (T, shape.H), optional=True)
+    _ws_arg(ws)
+    _require_cuda(q, k_cache, v_cache, sel, out, lse, ws)
     if out is None:
         out = torch.empty((T, shape.H, shape.d), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
@@ -259,7 +362,7 @@ def msa_sparse_attn_decode(shape: Shape, seqs: Varlen, q: torch.Tensor, k_cache:
     if ws is None:
         ws = _workspace(need, q.device)
     rc = lib.msa_sparse_attn_decode(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q), _ptr(k_cache),
-                                    _ptr(v_cache), _ptr(sel), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                    _ptr(v_cache), _ptr(sel), _ptr(out), _ptr(lse), _ptr(ws), _nbytes(ws),
                                     _stream(stream))
     _check(rc, "msa_sparse_attn_decode")
     if check:
@@ -270,8 +373,16 @@ def msa_sparse_attn_decode(shape: Shape, seqs: Varlen, q: torch.Tensor, k_cache:
 def msa_combine(shape: Shape, T: int, part_acc: torch.Tensor, part_lse: torch.Tensor, sel: torch.Tensor,
                 out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                 stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Log-sum-exp merge of per-block partials: part_acc f16 [T, G, k, d/8, H/G, 8],
+    part_lse f32 [T, G, k, H/G], sel int32 [T, G, k] (slots with sel < 0 unused)."""
     lib = load_library()
-    _require_cuda(part_acc)
+    Hg = _groups(shape)
+    _arg("part_acc", part_acc, torch.float16, numel=T * shape.G * shape.k * Hg * shape.d)
+    _arg("part_lse", part_lse, torch.float32, numel=T * shape.G * shape.k * Hg)
+    _arg("sel", sel, torch.int32, (T, shape.G, shape.k))
+    _arg("out", out, torch.bfloat16, (T, shape.H, shape.d), optional=True)
+    _arg("lse", lse, torch.float32, (T, shape.H), optional=True)
+    _require_cuda(part_acc, part_lse, sel, out, lse)
     if out is None:
         out = torch.empty((T, shape.H, shape.d), dtype=torch.bfloat16, device=part_acc.device)
     rc = lib.msa_combine(ctypes.byref(shape), T, _ptr(part_acc), _ptr(part_lse), _ptr(sel), _ptr(out),
@@ -286,8 +397,14 @@ def msa_dense_attn(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.Tensor,
                    stream=None, check: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Dense causal GQA attention (every key at or before the query position)."""
     lib = load_library()
-    _require_cuda(q)
-    T = seqs.total_q
+    T, S = seqs.total_q, seqs.total_k
+    _arg("q", q, torch.bfloat16, (T, shape.H, shape.d))
+    _arg("k", k, torch.bfloat16, (S, shape.G, shape.d))
+    _arg("v", v, torch.bfloat16, (S, shape.G, shape.d))
+    _arg("out", out, torch.bfloat16, (T, shape.H, shape.d), optional=True)
+    _arg("lse", lse, torch.float32, (T, shape.H), optional=True)
+    _ws_arg(ws)
+    _require_cuda(q, k, v, out, lse, ws)
     if out is None:
         out = torch.empty((T, shape.H, shape.d), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
@@ -296,7 +413,7 @@ def msa_dense_attn(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.Tensor,
     if ws is None:
         ws = _workspace(need, q.device)
     rc = lib.msa_dense_attn(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
-                            _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
+                            _ptr(lse), _ptr(ws), _nbytes(ws), _stream(stream))
     _check(rc, "msa_dense_attn")
     if check:
         _device_check(ws, stream, "msa_dense_attn")
@@ -337,8 +454,13 @@ def msa_profile_read(kernel: Optional[str]) -> Tuple[float, int]:
 def make_paged(seqlens: torch.Tensor, block_table: torch.Tensor, max_seqlen: int, num_pages: int) -> Paged:
     """Paged-cache description: seqlens int32 [batch] and block_table int32
     [batch, max_blocks] on the device; max_seqlen >= every seqlens[b]."""
-    assert seqlens.dtype == torch.int32 and block_table.dtype == torch.int32 and block_table.dim() == 2
-    assert seqlens.is_cuda and block_table.is_cuda and block_table.is_contiguous()
+    if not isinstance(block_table, torch.Tensor) or block_table.dim() != 2:
+        raise MsaError("block_table: expected a 2-D int32 tensor [batch, max_blocks]")
+    _arg("block_table", block_table, torch.int32)
+    _arg("seqlens", seqlens, torch.int32, (block_table.shape[0],))
+    if int(num_pages) < 0 or int(max_seqlen) < 0:
+        raise MsaError("make_paged: num_pages and max_seqlen must be >= 0")
+    _require_cuda(seqlens, block_table)
     p = Paged()
     p.batch, p.max_blocks = block_table.shape[0], block_table.shape[1]
     p.max_seqlen, p.num_pages = int(max_seqlen), int(num_pages)
@@ -357,13 +479,21 @@ def _paged_ws(shape: Shape, pages: Paged, ws, device):
 def msa_index_topk_decode_paged(shape: Shape, pages: Paged, q_idx: torch.Tensor, k_idx_pages: torch.Tensor,
                                 sel: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
                                 stream=None, check: bool = True) -> torch.Tensor:
+    """Index branch of one query per sequence over a paged cache: q_idx bf16
+    [batch, G, d_idx], k_idx_pages bf16 [num_pages * B_k, d_idx]; returns sel
+    int32 [batch, G, k]."""
     lib = load_library()
-    _require_cuda(q_idx)
+    B, rows = pages.batch, pages.num_pages * shape.B_k
+    _arg("q_idx", q_idx, torch.bfloat16, (B, shape.G, shape.d_idx))
+    _arg("k_idx_pages", k_idx_pages, torch.bfloat16, (rows, shape.d_idx))
+    _arg("sel", sel, torch.int32, (B, shape.G, shape.k), optional=True)
+    _ws_arg(ws)
+    _require_cuda(q_idx, k_idx_pages, sel, ws)
     if sel is None:
         sel = torch.empty((pages.batch, shape.G, shape.k), dtype=torch.int32, device=q_idx.device)
     ws = _paged_ws(shape, pages, ws, q_idx.device)
     rc = lib.msa_index_topk_decode_paged(ctypes.byref(shape), ctypes.byref(pages), _ptr(q_idx), _ptr(k_idx_pages),
-                                         _ptr(sel), _ptr(ws), ws.numel(), _stream(stream))
+                                         _ptr(sel), _ptr(ws), _nbytes(ws), _stream(stream))
     _check(rc, "msa_index_topk_decode_paged")
     if check:
         _device_check(ws, stream, "msa_index_topk_decode_paged")
@@ -375,15 +505,26 @@ def msa_sparse_attn_decode_paged(shape: Shape, pages: Paged, q: torch.Tensor, k_
                                  lse: Optional[torch.Tensor] = None, want_lse: bool = True,
                                  ws: Optional[torch.Tensor] = None, stream=None,
                                  check: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Main branch of one query per sequence over paged K / V: q bf16 [batch, H, d],
+    k_pages / v_pages bf16 [num_pages * B_k, G, d], sel int32 [batch, G, k];
+    returns out bf16 [batch, H, d] and lse f32 [batch, H]."""
     lib = load_library()
-    _require_cuda(q)
+    B, rows = pages.batch, pages.num_pages * shape.B_k
+    _arg("q", q, torch.bfloat16, (B, shape.H, shape.d))
+    _arg("k_pages", k_pages, torch.bfloat16, (rows, shape.G, shape.d))
+    _arg("v_pages", v_pages, torch.bfloat16, (rows, shape.G, shape.d))
+    _arg("sel", sel, torch.int32, (B, shape.G, shape.k))
+    _arg("out", out, torch.bfloat16, (B, shape.H, shape.d), optional=True)
+    _arg("lse", lse, torch.float32, (B, shape.H), optional=True)
+    _ws_arg(ws)
+    _require_cuda(q, k_pages, v_pages, sel, out, lse, ws)
     if out is None:
         out = torch.empty((pages.batch, shape.H, shape.d), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((pages.batch, shape.H), dtype=torch.float32, device=q.device)
     ws = _paged_ws(shape, pages, ws, q.device)
     rc = lib.msa_sparse_attn_decode_paged(ctypes.byref(shape), ctypes.byref(pages), _ptr(q), _ptr(k_pages),
-                                          _ptr(v_pages), _ptr(sel), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                          _ptr(v_pages), _ptr(sel), _ptr(out), _ptr(lse), _ptr(ws), _nbytes(ws),
                                           _stream(stream))
     _check(rc, "msa_sparse_attn_decode_paged")
     if check:
