@@ -91,7 +91,13 @@ typedef struct {
 
 /* Packed-sequence description.  cu_q / cu_k are DEVICE pointers; the other
  * fields are host values that must agree with them: total_q = cu_q[batch],
- * total_k = cu_k[batch], max_q_len / max_k_len the largest T_b / S_b. */
+ * total_k = cu_k[batch], max_q_len / max_k_len the largest T_b / S_b, and
+ * cu_q[0] = cu_k[0] = 0 with both non-decreasing.  The library sizes its
+ * launches and buffers from the host values and does not read the device
+ * arrays back (that would synchronise the stream), so this agreement is the
+ * caller's to keep: offsets beyond total_q / total_k make kernels read and
+ * write outside the caller's buffers.  T_b > S_b is checked on the device
+ * (MSA_ERR_DEVICE_CHECK).  The Python binding checks the host copies. */
 typedef struct {
   int32_t batch;
   int32_t max_q_len;
