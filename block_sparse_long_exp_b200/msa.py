@@ -296,8 +296,24 @@ def msa_index_topk_decode_noalloc_max_scratch() -> int:
     return load_library().msa_index_topk_decode_noalloc_max_scratch()
 
 
+def msa_index_topk_workspace_size(shape: Shape, seqs: Varlen) -> int:
+    """Workspace bytes msa_index_topk needs (0: shape or sizes unsupported)."""
+    return load_library().msa_index_topk_workspace_size(ctypes.byref(shape), ctypes.byref(seqs))
+
+
 def msa_sparse_attn_workspace_size(shape: Shape, seqs: Varlen, q_chunk: int = 0) -> int:
+    """Workspace bytes of the main-branch calls (0: unsupported)."""
     return load_library().msa_sparse_attn_workspace_size(ctypes.byref(shape), ctypes.byref(seqs), q_chunk)
+
+
+def msa_dense_attn_workspace_size(shape: Shape, seqs: Varlen) -> int:
+    """Workspace bytes msa_dense_attn needs (0: unsupported)."""
+    return load_library().msa_dense_attn_workspace_size(ctypes.byref(shape), ctypes.byref(seqs))
+
+
+def msa_decode_paged_workspace_size(shape: Shape, pages: Paged) -> int:
+    """Workspace bytes of either paged decode call (0: rejected)."""
+    return load_library().msa_decode_paged_workspace_size(ctypes.byref(shape), ctypes.byref(pages))
 
 
 def msa_sparse_attn_prefill(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
