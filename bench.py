@@ -119,6 +119,23 @@ class ClockSampler:
 
 # --------------------------------------------------------------- helpers ---
 
+def pass_rows(q_chunk, T):
+    """Query rows per attention pass: q_chunk < 0 picks passes of 131072 rows
+    above 128K tokens (the partials of a pass must fit the device), 0 = one pass."""
+    if q_chunk < 0:
+        return 131072 if T > 131072 else 0
+    return q_chunk
+
+
+def run_config(args, w, T, world):
+    """The workload description, printed the same by both arms."""
+    return {"workload": args.workload, "T": T, "H": w.H, "G": w.G, "d": w.d, "d_idx": w.d_idx,
+            "B_k": w.B_k, "k": w.k, "hot_block_frac": w.hot_frac,
+            "l2": "inputs larger than L2 (q alone is %.1f GB)" % (T * w.H * w.d * 2 / 1e9),
+            "parallelism": f"independent layer per GPU x{world}",
+            "attention_pass_rows": pass_rows(args.q_chunk, T) or T}
+
+
 def make_ctx(w, inp, torch, msa):
     shape = msa.make_shape(w.H, w.G, w.d, w.d_idx, w.k)
     seqs = msa.make_varlen(inp["cu_q"], inp["cu_k"], inp["cu_q_host"], inp["cu_k_host"])
@@ -131,9 +148,7 @@ def make_ctx(w, inp, torch, msa):
     import ctypes
     n_idx = lib.msa_index_topk_workspace_size(ctypes.byref(shape), ctypes.byref(seqs))
     # passes of at most q_chunk query rows (the partials of a pass must fit the device)
-    ctx["q_chunk"] = getattr(make_ctx, "q_chunk", 0)
-    if ctx["q_chunk"] < 0:
-        ctx["q_chunk"] = 131072 if T > 131072 else 0
+    ctx["q_chunk"] = pass_rows(getattr(make_ctx, "q_chunk", 0), T)
     n_att = (msa.msa_sparse_attn_workspace_size(shape, seqs, ctx["q_chunk"])
              if not getattr(make_ctx, "index_only", False) else 256)
     ctx["ws_idx"] = torch.empty(n_idx, dtype=torch.uint8, device=dev)
@@ -326,7 +341,7 @@ def run_reference(args):
         return
     w = W.WORKLOADS[args.workload]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    inp = W.make_inputs(w, dev)
+    inp = W.make_inputs(w, dev, T_override=args.T or None)
     T = inp["cu_q_host"][-1]
     from oracle import msa_oracle as O
     gen = torch.Generator().manual_seed(99)
@@ -351,8 +366,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * sec / len(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": args.workload, "T": T, "H": w.H, "G": w.G, "d": w.d,
-                                             "d_idx": w.d_idx, "B_k": w.B_k, "k": w.k},
+            "data": "synthetic", "config": run_config(args, w, T, args.gpus),
             "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -430,7 +444,6 @@ def run_ours(args):
 
     value, ms_max = job_rate(T * args.steps, ms, torch, dist)
     ms_step = ms_max / args.steps
-    ctx_q_chunk = ctx["q_chunk"]
 
     # algorithmic work of each kernel: the main branch split between the query
     # tiles and the KV-outer lists as the library's planner splits it
@@ -567,11 +580,7 @@ def run_ours(args):
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": args.workload, "T": T, "H": w.H, "G": w.G, "d": w.d, "d_idx": w.d_idx,
-                           "B_k": w.B_k, "k": w.k, "hot_block_frac": w.hot_frac,
-                           "l2": "inputs larger than L2 (q alone is %.1f GB)" % (inp["q"].numel() * 2 / 1e9),
-                           "parallelism": f"independent layer per GPU x{world}",
-                           "attention_pass_rows": ctx_q_chunk or T},
+                "config": run_config(args, w, T, world),
                 "roofline": roof, "step_roofline": step_roof, "tile_split": split, "dense_gqa": dense,
                 "decode": decode, "e2e": e2e,
                 "cpu_baseline": cpu, "clocks": clk, "gpu_launches": launches, "kernels": kernels}
@@ -581,7 +590,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def main():
+def build_parser():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
@@ -600,7 +609,11 @@ def main():
                     help="query-tile threshold of the prefill (-1 automatic, 0 off)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=64)
-    args = ap.parse_args()
+    return ap
+
+
+def main():
+    args = build_parser().parse_args()
     if args.warmup < 3:
         log("note: fewer than 3 warm-up steps")
     if args.impl == "reference":

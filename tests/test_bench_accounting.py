@@ -115,3 +115,31 @@ def test_recorded_traffic_matches_current_code():
         assert sha is not None, name
         want = e["dram_bytes_per_launch"] if sha == e["source_sha"] else None
         assert bench.traffic_for(name) == want
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` (the oracle on the host cores) prints one JSON
+    line with the contract's keys and the same config our arm prints."""
+    import json
+    import os
+    import subprocess
+    import sys
+    import bench
+    from block_sparse_long_exp_b200 import workloads as W
+    root = bench.ROOT
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload",
+                        "tiny_n4096", "--steps", "2", "--warmup", "1"], capture_output=True, text=True,
+                       timeout=600, cwd=root, env={**os.environ, "CUDA_VISIBLE_DEVICES": ""})
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["steps"] == 2
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+    w = W.WORKLOADS["tiny_n4096"]
+    args = bench.build_parser().parse_args(["--workload", "tiny_n4096"])
+    assert line["config"] == bench.run_config(args, w, line["config"]["T"], 1)
+    assert bench.pass_rows(-1, 131072) == 0 and bench.pass_rows(-1, 131073) == 131072
+    assert bench.pass_rows(700, 5000) == 700
