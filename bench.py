@@ -119,6 +119,9 @@ class ClockSampler:
 
 # --------------------------------------------------------------- helpers ---
 
+L2_BYTES = 126 * 1024 * 1024     # B200 L2
+
+
 def pass_rows(q_chunk, T):
     """Query rows per attention pass: q_chunk < 0 picks passes of 131072 rows
     above 128K tokens (the partials of a pass must fit the device), 0 = one pass."""
@@ -131,7 +134,10 @@ def run_config(args, w, T, world):
     """The workload description, printed the same by both arms."""
     return {"workload": args.workload, "T": T, "H": w.H, "G": w.G, "d": w.d, "d_idx": w.d_idx,
             "B_k": w.B_k, "k": w.k, "hot_block_frac": w.hot_frac,
-            "l2": "inputs larger than L2 (q alone is %.1f GB)" % (T * w.H * w.d * 2 / 1e9),
+            "l2": ("inputs larger than L2 (q alone is %.1f GB)" % (T * w.H * w.d * 2 / 1e9)
+                   if T * w.H * w.d * 2 > L2_BYTES else
+                   "inputs fit in L2 (q is %.0f MB, L2 not flushed): a profiling size, not a timing one"
+                   % (T * w.H * w.d * 2 / 1e6)),
             "parallelism": f"independent layer per GPU x{world}",
             "attention_pass_rows": pass_rows(args.q_chunk, T) or T}
 
