@@ -119,13 +119,13 @@ msa_status_t attn_common(const msa_shape_t* shape, const msa_varlen_t* seqs, con
   if (st != MSA_OK) return st;
   // no queries: nothing is read or written (empty tensors may have no storage)
   if (seqs->total_q > 0 && (!q || !k || !v || !sel || !out)) return MSA_ERR_INVALID_ARG;
-  if (seqs->total_q == 0) return MSA_OK;
   const int64_t rows = chunk_rows(seqs, q_chunk);
   const AttnLayout L = attn_layout(shape, seqs, rows);
   if (!ws_ok(ws, ws_bytes, L.total)) return MSA_ERR_WORKSPACE;
   uint8_t* base = static_cast<uint8_t*>(ws);
   if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MSA_ERR_CUDA;
+  if (seqs->total_q == 0) return MSA_OK;
   AttnArgs a{};
   a.q = q; a.key = k; a.value = v; a.sel = sel; a.out = out; a.lse = lse;
   a.cu_q = seqs->cu_q; a.cu_k = seqs->cu_k;
@@ -245,6 +245,7 @@ const char* msa_version(void) { return "msa-b200 0.1 (sm_100a)"; }
 
 size_t msa_index_topk_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs) {
   if (check_shape(shape) != MSA_OK || check_seqs(seqs) != MSA_OK) return 0;
+  if (seqs->max_q_len > 1 && seqs->batch > kMaxBatchTiles) return 0;
   size_t need = kWsHeader;
   if (seqs->max_q_len <= 1)
     need += align_up(decode_index_scratch_bytes(seqs->batch, seqs->total_k, shape->G, shape->k), kAlign);
@@ -257,6 +258,8 @@ msa_status_t msa_index_topk(const msa_shape_t* shape, const msa_varlen_t* seqs, 
   if (st != MSA_OK) return st;
   st = check_seqs(seqs);
   if (st != MSA_OK) return st;
+  // prefill-shaped calls keep a per-sequence tile prefix in shared memory
+  if (seqs->max_q_len > 1 && seqs->batch > kMaxBatchTiles) return MSA_ERR_UNSUPPORTED;
   if (seqs->total_q > 0 && (!q_idx || !k_idx || !sel)) return MSA_ERR_INVALID_ARG;
   const size_t need = msa_index_topk_workspace_size(shape, seqs);
   if (!ws_ok(ws, ws_bytes, need)) return MSA_ERR_WORKSPACE;
@@ -276,7 +279,6 @@ msa_status_t msa_index_topk(const msa_shape_t* shape, const msa_varlen_t* seqs, 
   if (seqs->max_q_len <= 1) {
     rc = launch_index_topk_decode(a, stream);
   } else {
-    if (seqs->batch > kMaxBatchTiles) return MSA_ERR_UNSUPPORTED;
     rc = launch_index_topk_prefill(a, stream);
   }
   return rc == 0 ? MSA_OK : MSA_ERR_CUDA;

@@ -120,7 +120,10 @@ typedef struct {
  * kernel over 128-query tiles; decode-shaped calls (max_q_len == 1) run a
  * split scan of the index keys and a candidate merge.
  * Selections are exact for inputs whose scores are exact in fp32 (for
- * example integer-valued index q/k); otherwise they follow fp32 rounding. */
+ * example integer-valued index q/k); otherwise they follow fp32 rounding.
+ * Prefill-shaped calls take at most 1024 sequences (MSA_ERR_UNSUPPORTED
+ * beyond, and the workspace query returns 0); decode-shaped calls have no
+ * such limit. */
 size_t msa_index_topk_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs);
 
 msa_status_t msa_index_topk(const msa_shape_t* shape, const msa_varlen_t* seqs,

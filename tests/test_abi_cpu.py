@@ -121,3 +121,26 @@ def test_plain_c_program_uses_the_boundary(lib, tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stderr
     assert "abi_host ok" in r.stdout
+
+
+def test_limits_and_empty_calls_answer_before_any_launch(lib):
+    """Prefill-shaped index calls take at most 1024 sequences: the workspace query
+    returns 0 and the call MSA_ERR_UNSUPPORTED before anything is launched.
+    A call with no queries still obeys the workspace rule."""
+    from block_sparse_long_exp_b200 import msa
+    shape = msa.make_shape(64, 4, 128, 64, 16)
+    cu = (ctypes.c_int32 * 2)(0, 0)
+    many = msa.Varlen(1025, 2, 2, 0, 2050, 2050, ctypes.addressof(cu), ctypes.addressof(cu))
+    assert lib.msa_index_topk_workspace_size(ctypes.byref(shape), ctypes.byref(many)) == 0
+    rc = lib.msa_index_topk(ctypes.byref(shape), ctypes.byref(many), 256, 256, 256, 256, 1 << 20, None)
+    assert rc == 2                                       # MSA_ERR_UNSUPPORTED
+    decode_shaped = msa.Varlen(1025, 1, 2, 0, 1025, 2050, ctypes.addressof(cu), ctypes.addressof(cu))
+    assert lib.msa_index_topk_workspace_size(ctypes.byref(shape), ctypes.byref(decode_shaped)) > 0
+    empty = msa.Varlen(1, 0, 10, 0, 0, 10, ctypes.addressof(cu), ctypes.addressof(cu))
+    for fn in (lib.msa_sparse_attn_prefill,):
+        rc = fn(ctypes.byref(shape), ctypes.byref(empty), None, None, None, None, None, None, 0, None, 0, None)
+        assert rc == 3                                   # MSA_ERR_WORKSPACE: no workspace given
+    rc = lib.msa_dense_attn(ctypes.byref(shape), ctypes.byref(empty), None, None, None, None, None, None, 0, None)
+    assert rc == 3
+    rc = lib.msa_index_topk(ctypes.byref(shape), ctypes.byref(empty), None, None, None, None, 0, None)
+    assert rc == 3
