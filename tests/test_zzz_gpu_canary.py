@@ -3,8 +3,7 @@ buffer the library is given sits between two 8 KB guard bands filled with a
 known byte, and after each call the bands must be intact, the inputs
 unchanged, and the results bit-identical to the same call on plain buffers.
 Ragged lengths put the edges of every buffer next to a partial block.  (Runs
-after the tests that have passed on a GPU: a failure here must not hide
-them.)"""
+after the parity files.)"""
 import numpy as np
 import pytest
 import torch

@@ -3,7 +3,7 @@ sequences (the prefill index kernel's limit) of 1-600 tokens each, so that
 128-query tiles end at a sequence boundary almost everywhere, and a decode
 of 2048 sequences (decode-shaped calls have no batch limit).  The prefill is
 compared on sampled rows (each sequence's last row among them), the decode
-on every row.  (Runs after the tests that have passed on a GPU.)"""
+on every row.  (Runs after the parity files.)"""
 import numpy as np
 import pytest
 import torch
