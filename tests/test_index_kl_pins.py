@@ -198,3 +198,36 @@ def test_selected_mass_is_the_lse_ratio():
     # queries whose causal blocks all fit in k hold all of the weight
     pos_small = [t for t in rows if t < 3 * L["B_k"]]
     np.testing.assert_allclose(mass[pos_small], 1.0, rtol=0, atol=1e-12)
+
+
+def test_block_split_reproduces_the_kl():
+    """KL = sum P log P - sum P z + log sum exp z over the support, each sum taken
+    block by block (two plain sums and one (max, sum) pair per block) and merged:
+    the split a kernel uses, checked against the oracle on every row."""
+    L = _layer(21, S_lens=[33, 18], T_lens=[33, 7], G=2, Hg=3, k=3, B_k=4)
+    sm, tau = 0.55, 0.8
+    T = L["cu_q"][-1]
+    want = K.index_kl_rows(L["q"], L["k"], L["q_idx"], L["k_idx"], L["sel"], L["cu_q"], L["cu_k"], list(range(T)),
+                           L["B_k"], sm, tau)
+    H, G = L["q"].shape[1], L["k"].shape[1]
+    Hg = H // G
+    for t in range(T):
+        b = int(np.searchsorted(L["cu_q"], t, side="right") - 1)
+        T_b, S_b = L["cu_q"][b + 1] - L["cu_q"][b], L["cu_k"][b + 1] - L["cu_k"][b]
+        pos, k0 = S_b - T_b + (t - L["cu_q"][b]), L["cu_k"][b]
+        for g in range(G):
+            J = O.selected_token_set([int(x) for x in L["sel"][t, g]], pos, L["B_k"]) + k0
+            s = sm * L["q"][t, g * Hg:(g + 1) * Hg] @ L["k"][J, g].T          # [Hg, |J|]
+            lse_h = np.log(np.exp(s).sum(axis=1))                            # the forward's lse over J
+            A = Bsum = 0.0
+            m_z, l_z = -np.inf, 0.0
+            for blk in sorted({int(j - k0) // L["B_k"] for j in J}):
+                cols = [i for i, j in enumerate(J) if (j - k0) // L["B_k"] == blk]
+                Pbar = np.exp(s[:, cols] - lse_h[:, None]).mean(axis=0)
+                z = tau * L["k_idx"][J[cols]] @ L["q_idx"][t, g]
+                A += float(np.sum(Pbar * np.log(Pbar)))
+                Bsum += float(np.sum(Pbar * z))
+                m_new = max(m_z, float(z.max()))
+                l_z = l_z * math.exp(m_z - m_new) + float(np.exp(z - m_new).sum())
+                m_z = m_new
+            assert A - Bsum + (m_z + math.log(l_z)) == pytest.approx(want[t, g], rel=1e-10, abs=1e-12)
