@@ -14,7 +14,9 @@ than itself (CPU only):
   selected;
 * the selected share of the dense attention weight equals
   exp(lse over the selected tokens - lse over all causal tokens), both from the
-  main-branch oracle.
+  main-branch oracle;
+* the block-by-block split of the KL (two plain sums and an online
+  log-sum-exp, the form a kernel computes) reproduces it on every row.
 """
 import math
 
