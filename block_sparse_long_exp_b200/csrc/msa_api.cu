@@ -408,9 +408,7 @@ msa_status_t msa_sparse_attn_decode_paged(const msa_shape_t* shape, const msa_pa
 }
 
 int32_t msa_set_tile_threshold(int32_t theta) {
-  const int32_t prev = g_tile_theta.load();
-  g_tile_theta.store(theta < 0 ? -1 : theta);
-  return prev;
+  return g_tile_theta.exchange(theta < 0 ? -1 : theta);
 }
 
 msa_status_t msa_get_device_error(void* ws, int32_t* code, int32_t* where, int32_t* info0, int32_t* info1,

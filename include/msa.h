@@ -251,7 +251,9 @@ msa_status_t msa_dense_attn(const msa_shape_t* shape, const msa_varlen_t* seqs,
  *   theta < 0   automatic: ceil(5/8 x tile queries) (the default)
  *   theta == 0  off: every selection goes through the KV-outer lists
  *   theta >= 1  that threshold (1: every selected block of a tile)
- * Decode calls (one query per sequence) never use query tiles. */
+ * Decode calls (one query per sequence) never use query tiles.  The value is
+ * one atomic word: safe to set from any thread; a call reads it once, when
+ * it starts, and uses that value throughout. */
 int32_t msa_set_tile_threshold(int32_t theta);
 
 /* ---------------------------------------------------------------------- */
