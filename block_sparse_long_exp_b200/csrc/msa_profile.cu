@@ -77,17 +77,21 @@ msa_status_t msa_profile_reset(void) {
 msa_status_t msa_profile_read(const char* kernel, double* total_ms, int64_t* count) {
   if (total_ms == nullptr || count == nullptr) return MSA_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lk(msa::g_mu);
-  for (auto& p : msa::g_pending) {
+  auto& pend = msa::g_pending;
+  for (size_t i = 0; i < pend.size(); ++i) {
     float ms = 0.f;
-    if (cudaEventSynchronize(p.stop) != cudaSuccess || cudaEventElapsedTime(&ms, p.start, p.stop) != cudaSuccess)
+    if (cudaEventSynchronize(pend[i].stop) != cudaSuccess ||
+        cudaEventElapsedTime(&ms, pend[i].start, pend[i].stop) != cudaSuccess) {
+      pend.erase(pend.begin(), pend.begin() + i);   // keep only the pairs not yet folded in and destroyed
       return MSA_ERR_CUDA;
-    auto& slot = msa::g_done[p.name];
+    }
+    auto& slot = msa::g_done[pend[i].name];
     slot.first += ms;
     slot.second += 1;
-    cudaEventDestroy(p.start);
-    cudaEventDestroy(p.stop);
+    cudaEventDestroy(pend[i].start);
+    cudaEventDestroy(pend[i].stop);
   }
-  msa::g_pending.clear();
+  pend.clear();
   if (kernel == nullptr) {
     *total_ms = 0.0;
     *count = msa::g_launches.load();
