@@ -42,6 +42,7 @@ msa_status_t check_seqs(const msa_varlen_t* v) {
   if (v->batch < 1 || v->total_q < 0 || v->total_k < 1 || v->max_q_len < 0 || v->max_k_len < 1)
     return MSA_ERR_INVALID_ARG;
   if (v->total_q > v->total_k || v->max_q_len > v->max_k_len) return MSA_ERR_INVALID_ARG;
+  if (v->max_q_len > v->total_q || v->max_k_len > v->total_k) return MSA_ERR_INVALID_ARG;  // a length beyond its total
   if (v->total_k > (int64_t)INT32_MAX - 256 || v->total_q > (int64_t)INT32_MAX / kMaxK) return MSA_ERR_UNSUPPORTED;
   return MSA_OK;
 }

@@ -144,3 +144,14 @@ def test_limits_and_empty_calls_answer_before_any_launch(lib):
     assert rc == 3
     rc = lib.msa_index_topk(ctypes.byref(shape), ctypes.byref(empty), None, None, None, None, 0, None)
     assert rc == 3
+
+
+def test_lengths_beyond_their_totals_are_rejected(lib):
+    from block_sparse_long_exp_b200 import msa
+    shape = msa.make_shape(64, 4, 128, 64, 16)
+    cu = (ctypes.c_int32 * 2)(0, 0)
+    for bad in (msa.Varlen(1, 300, 400, 0, 200, 400, ctypes.addressof(cu), ctypes.addressof(cu)),    # max_q > total_q
+                msa.Varlen(1, 100, 500, 0, 100, 400, ctypes.addressof(cu), ctypes.addressof(cu))):   # max_k > total_k
+        assert lib.msa_index_topk_workspace_size(ctypes.byref(shape), ctypes.byref(bad)) == 0
+        rc = lib.msa_index_topk(ctypes.byref(shape), ctypes.byref(bad), 256, 256, 256, 256, 1 << 20, None)
+        assert rc == 1                                   # MSA_ERR_INVALID_ARG
