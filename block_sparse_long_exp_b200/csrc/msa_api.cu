@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "msa_internal.h"
+#include "msa_kl.h"
 
 using namespace msa;
 
@@ -406,6 +407,31 @@ msa_status_t msa_sparse_attn_decode_paged(const msa_shape_t* shape, const msa_pa
   a.tile_ctr = reinterpret_cast<int32_t*>(base + L.tile_ctr);
   a.block_table = pages->block_table; a.max_blocks = pages->max_blocks; a.num_pages = pages->num_pages;
   return launch_rows_attn(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
+}
+
+msa_status_t msa_index_kl(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q, const void* k,
+                          const void* q_idx, const void* k_idx, const int32_t* sel, const float* lse, float tau,
+                          int32_t dense, float* kl, void* ws, size_t ws_bytes, void* stream) {
+  msa_status_t st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  st = check_seqs(seqs);
+  if (st != MSA_OK) return st;
+  if (!(tau == tau) || tau > 3.0e38f || tau < -3.0e38f) return MSA_ERR_INVALID_ARG;   // NaN or infinite
+  if (seqs->total_q > 0 && (!q || !k || !q_idx || !k_idx || !lse || !kl || (!dense && !sel)))
+    return MSA_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, kWsHeader)) return MSA_ERR_WORKSPACE;
+  if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  if (seqs->total_q == 0) return MSA_OK;
+  IndexKlArgs a{};
+  a.q = q; a.key = k; a.q_idx = q_idx; a.k_idx = k_idx; a.sel = sel; a.lse = lse;
+  a.cu_q = seqs->cu_q; a.cu_k = seqs->cu_k;
+  a.batch = seqs->batch; a.H = shape->H; a.G = shape->G; a.d = shape->d; a.d_idx = shape->d_idx; a.k = shape->k;
+  a.total_q = seqs->total_q;
+  a.sm_scale = shape->sm_scale; a.tau = tau; a.dense = dense != 0;
+  a.kl = kl;
+  a.err = static_cast<DevError*>(ws);
+  return launch_index_kl(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
 }
 
 int32_t msa_set_tile_threshold(int32_t theta) {

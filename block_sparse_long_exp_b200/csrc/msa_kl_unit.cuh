@@ -1,0 +1,153 @@
+// msa_kl_unit.cuh — the index-alignment target of one (query, group), split
+// over threads: the per-thread partial sums and their merge.
+//
+// The Index Branch is trained by a KL divergence that pulls its distribution
+// towards the Main Branch's attention on the selected support, with the
+// gradient kept away from the backbone (pnsm.cn "MiniMax Sparse Attention：
+// 一篇读懂百万上下文时代的稀疏注意力工程化路线", sec. 4 and sec. 5; yhxrc.cn
+// sec. 二).  Over the support J of query t and group g:
+//   teacher  P_j = mean over the group's heads h of exp(sm_scale q_h.k_j - lse_h)
+//            (lse_h: the main branch's log-sum-exp over J, so each head's
+//            distribution sums to 1 and so does their mean),
+//   student  Q_j = softmax_J(z), z_j = tau q_idx.k_idx_j,
+//   KL(P || Q) = sum_j P_j log P_j - sum_j P_j z_j + log sum_j exp(z_j).
+// The three sums split over any partition of J: each thread keeps A = sum
+// P log P, B = sum P z and a (max, sum) pair for the log-sum-exp; the merge
+// adds A and B and combines the pairs.  J is the selected blocks' tokens cut
+// at the query (sparse form) or every token 0..pos (the dense form used while
+// the index branch warms up on full attention).
+//
+// Plain fp32 arithmetic on bf16 bit patterns; compiled for the device by the
+// kernel and for the host by a test, which checks it against an fp64 oracle.
+#pragma once
+
+#include <stdint.h>
+
+#include <cmath>
+#include <cstring>
+#ifndef __CUDACC__
+#define MSA_KL_HD inline
+#else
+#define MSA_KL_HD __host__ __device__ __forceinline__
+#endif
+
+namespace msa {
+
+struct KlPartial {
+  float A;   // sum of P log P
+  float B;   // sum of P z
+  float m;   // running max of z
+  float l;   // sum of exp(z - m)
+};
+
+MSA_KL_HD float kl_bf16(uint16_t bits) {
+  const uint32_t u = static_cast<uint32_t>(bits) << 16;
+  float x;
+#ifdef __CUDA_ARCH__
+  x = __uint_as_float(u);
+#else
+  std::memcpy(&x, &u, 4);
+#endif
+  return x;
+}
+
+MSA_KL_HD float kl_exp(float x) {
+#ifdef __CUDA_ARCH__
+  return __expf(x);
+#else
+  return std::exp(x);
+#endif
+}
+
+MSA_KL_HD float kl_log(float x) {
+#ifdef __CUDA_ARCH__
+  return __logf(x);
+#else
+  return std::log(x);
+#endif
+}
+
+// Everything one (query, group) needs.  qf: the group's Hg query heads as
+// float [Hg * d]; qif: its index query as float [d_idx]; lse: the heads'
+// log-sum-exps over J [Hg]; krow / kirow: the sequence's keys (bf16 bits,
+// key row j of group g at krow + (j * G + g) * d) and index keys (kirow +
+// j * d_idx); blocks: the selected block ids (ascending, -1 padding).
+struct KlUnit {
+  const float* qf;
+  const float* qif;
+  const float* lse;
+  const uint16_t* krow;
+  const uint16_t* kirow;
+  const int32_t* blocks;
+  int nsel, Hg, d, d_idx, G, g, B_k;
+  int64_t pos;
+  float sm_scale, tau;
+  bool dense;
+};
+
+// Partial sums over the support tokens n = tid, tid + nthreads, ... (tokens
+// numbered in ascending order).  A block id outside 0..pos / B_k sets *bad and
+// is skipped, so no read leaves the sequence.
+MSA_KL_HD KlPartial kl_thread(const KlUnit& u, int tid, int nthreads, int* bad) {
+  KlPartial r{0.f, 0.f, -INFINITY, 0.f};
+  const int64_t lb = u.pos / u.B_k;
+  const int nblk = u.dense ? static_cast<int>(lb) + 1 : u.nsel;
+  int64_t base = 0;   // support tokens before this block
+  for (int i = 0; i < nblk; ++i) {
+    const int64_t b = u.dense ? i : u.blocks[i];
+    if (b < 0) continue;
+    if (b > lb) {
+      *bad = 1;
+      continue;
+    }
+    const int64_t j0 = b * u.B_k;
+    const int64_t j1 = (b + 1) * u.B_k < u.pos + 1 ? (b + 1) * u.B_k : u.pos + 1;
+    const int64_t n0 = base;
+    base += j1 - j0;
+    // first token of this block that belongs to thread tid
+    int64_t first = (tid - n0) % nthreads;
+    if (first < 0) first += nthreads;
+    for (int64_t j = j0 + first; j < j1; j += nthreads) {
+      const uint16_t* kj = u.krow + (j * u.G + u.g) * u.d;
+      float pbar = 0.f;
+      for (int h = 0; h < u.Hg; ++h) {
+        const float* qh = u.qf + h * u.d;
+        float s = 0.f;
+        for (int c = 0; c < u.d; ++c) s += qh[c] * kl_bf16(kj[c]);
+        pbar += kl_exp(u.sm_scale * s - u.lse[h]);
+      }
+      pbar *= 1.f / u.Hg;
+      const uint16_t* kij = u.kirow + j * u.d_idx;
+      float zs = 0.f;
+      for (int c = 0; c < u.d_idx; ++c) zs += u.qif[c] * kl_bf16(kij[c]);
+      const float z = u.tau * zs;
+      if (pbar > 0.f) r.A += pbar * kl_log(pbar);
+      r.B += pbar * z;
+      if (z > r.m) {
+        r.l = r.l * kl_exp(r.m - z) + 1.f;
+        r.m = z;
+      } else {
+        r.l += kl_exp(z - r.m);
+      }
+    }
+  }
+  return r;
+}
+
+// KL = sum A - sum B + log-sum-exp merged over the partials.
+MSA_KL_HD float kl_merge(const KlPartial* p, int n) {
+  float A = 0.f, B = 0.f, m = -INFINITY;
+  for (int i = 0; i < n; ++i) {
+    A += p[i].A;
+    B += p[i].B;
+    if (p[i].l > 0.f && p[i].m > m) m = p[i].m;
+  }
+  float l = 0.f;
+  for (int i = 0; i < n; ++i)
+    if (p[i].l > 0.f) l += p[i].l * kl_exp(p[i].m - m);
+  return l > 0.f ? A - B + m + kl_log(l) : 0.f;
+}
+
+}  // namespace msa
+
+#undef MSA_KL_HD

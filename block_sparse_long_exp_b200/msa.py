@@ -51,6 +51,7 @@ EXPORTED = [
     "msa_profile_enable", "msa_profile_reset", "msa_profile_read",
     "msa_get_device_error", "msa_version", "msa_set_tile_threshold",
     "msa_decode_paged_workspace_size", "msa_index_topk_decode_paged", "msa_sparse_attn_decode_paged",
+    "msa_index_kl",
 ]
 
 
@@ -129,6 +130,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_index_topk_decode_paged.restype = i32
     lib.msa_sparse_attn_decode_paged.argtypes = [P(Shape), P(Paged), vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.msa_sparse_attn_decode_paged.restype = i32
+    lib.msa_index_kl.argtypes = [P(Shape), P(Varlen), vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp, vp, sz, vp]
+    lib.msa_index_kl.restype = i32
     _lib = lib
     return lib
 
@@ -546,6 +549,40 @@ def msa_sparse_attn_decode_paged(shape: Shape, pages: Paged, q: torch.Tensor, k_
     if check:
         _device_check(ws, stream, "msa_sparse_attn_decode_paged")
     return out, lse
+
+
+def msa_index_kl(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.Tensor, q_idx: torch.Tensor,
+                 k_idx: torch.Tensor, sel: Optional[torch.Tensor], lse: torch.Tensor, tau: float,
+                 dense: bool = False, kl: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                 stream=None, check: bool = True) -> torch.Tensor:
+    """Index-alignment target: KL(P || Q) per (query, group) over the support
+    (the selected tokens, or with dense=True every token up to the query).
+    P: the main branch's attention on the support, averaged over the group's
+    heads (lse [T, H] float: its log-sum-exp over that support, as the prefill
+    or dense call returns it); Q: softmax of tau * index score.  Returns kl
+    float [T, G]."""
+    lib = load_library()
+    T, S = seqs.total_q, seqs.total_k
+    _arg("q", q, torch.bfloat16, (T, shape.H, shape.d))
+    _arg("k", k, torch.bfloat16, (S, shape.G, shape.d))
+    _arg("q_idx", q_idx, torch.bfloat16, (T, shape.G, shape.d_idx))
+    _arg("k_idx", k_idx, torch.bfloat16, (S, shape.d_idx))
+    _arg("sel", sel, torch.int32, (T, shape.G, shape.k), optional=dense)
+    _arg("lse", lse, torch.float32, (T, shape.H))
+    _arg("kl", kl, torch.float32, (T, shape.G), optional=True)
+    _ws_arg(ws)
+    _require_cuda(q, k, q_idx, k_idx, sel, lse, kl, ws)
+    if kl is None:
+        kl = torch.empty((T, shape.G), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = _workspace(256, q.device)
+    rc = lib.msa_index_kl(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q), _ptr(k), _ptr(q_idx), _ptr(k_idx),
+                          _ptr(sel), _ptr(lse), float(tau), 1 if dense else 0, _ptr(kl), _ptr(ws), _nbytes(ws),
+                          _stream(stream))
+    _check(rc, "msa_index_kl")
+    if check:
+        _device_check(ws, stream, "msa_index_kl")
+    return kl
 
 
 def msa_set_tile_threshold(theta: int) -> int:

@@ -209,6 +209,31 @@ msa_status_t msa_sparse_attn_decode_paged(const msa_shape_t* shape, const msa_pa
                                           void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Index-alignment target (pnsm.cn sec. 4 "KL alignment", sec. 5 "Indexer
+ * warmup"; yhxrc.cn sec. 二): for every query t and group g, the KL divergence
+ * KL(P || Q) over the support J (the tokens of the selected blocks sel[t, g]
+ * cut at the query, or with dense != 0 every token up to the query), where
+ *   P_j = mean over the group's heads h of exp(sm_scale q_h.k_j - lse[t, h])
+ *         (the Main Branch's attention on J: lse must be the log-sum-exp over
+ *         the same J, as msa_sparse_attn_prefill returns it for the sparse
+ *         support and msa_dense_attn for the dense one),
+ *   Q_j = softmax over J of tau * <q_idx[t, g], k_idx[j]>  (the Index Branch).
+ *   kl   device float [T, G] (out)
+ * The teacher P is a constant of this value (its gradient is not the index
+ * branch's to follow).  ws: at least 256 bytes, 256-byte aligned (the error
+ * word).  A selected block id past the query's block is recorded as
+ * MSA_ERR_DEVICE_CHECK and skipped.  A first, CUDA-core form (one CTA per
+ * (query, group)). */
+msa_status_t msa_index_kl(const msa_shape_t* shape, const msa_varlen_t* seqs,
+                          const void* q,      /* device bf16 [T, H, d] */
+                          const void* k,      /* device bf16 [S, G, d] */
+                          const void* q_idx,  /* device bf16 [T, G, d_idx] */
+                          const void* k_idx,  /* device bf16 [S, d_idx] */
+                          const int32_t* sel, /* device int32 [T, G, k]; NULL allowed when dense */
+                          const float* lse,   /* device float [T, H] */
+                          float tau, int32_t dense, float* kl, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* Two-phase combine on its own (pnsm.cn sec. 7 "two-phase combine").
  * Merges, for every query t and head h = g*(H/G) + i of group g, the partials
  * of the slots s with sel[t, g, s] >= 0:

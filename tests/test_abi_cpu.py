@@ -155,3 +155,21 @@ def test_lengths_beyond_their_totals_are_rejected(lib):
         assert lib.msa_index_topk_workspace_size(ctypes.byref(shape), ctypes.byref(bad)) == 0
         rc = lib.msa_index_topk(ctypes.byref(shape), ctypes.byref(bad), 256, 256, 256, 256, 1 << 20, None)
         assert rc == 1                                   # MSA_ERR_INVALID_ARG
+
+
+def test_index_kl_host_validation_without_gpu(lib):
+    from block_sparse_long_exp_b200 import msa
+    shape = msa.make_shape(64, 4, 128, 64, 16)
+    cu = (ctypes.c_int32 * 2)(0, 0)
+    seqs = msa.Varlen(1, 300, 300, 0, 300, 300, ctypes.addressof(cu), ctypes.addressof(cu))
+    args = (256, 256, 256, 256)
+    rc = lib.msa_index_kl(ctypes.byref(shape), ctypes.byref(seqs), *args, None, 256, 0.5, 0, 256, 256, 1 << 20, None)
+    assert rc == 1                                       # sparse support without a selection
+    rc = lib.msa_index_kl(ctypes.byref(shape), ctypes.byref(seqs), *args, 256, 256, float("nan"), 0, 256, 256,
+                          1 << 20, None)
+    assert rc == 1                                       # tau must be finite
+    rc = lib.msa_index_kl(ctypes.byref(shape), ctypes.byref(seqs), *args, None, 256, 0.5, 1, 256, 256, 16, None)
+    assert rc == 3                                       # dense: no selection needed, but the workspace is
+    bad = msa.make_shape(64, 4, 96, 64, 16)
+    rc = lib.msa_index_kl(ctypes.byref(bad), ctypes.byref(seqs), *args, 256, 256, 0.5, 0, 256, 256, 1 << 20, None)
+    assert rc == 2                                       # d = 96 is not built

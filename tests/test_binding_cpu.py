@@ -129,3 +129,20 @@ def test_paged_calls_check_their_tensors(M):
     with pytest.raises(M.MsaError, match="CUDA"):
         M.msa_sparse_attn_decode_paged(shape, pages, _bf(3, H, d), _bf(rows, G, d), _bf(rows, G, d),
                                        torch.zeros(3, G, k, dtype=torch.int32))
+
+
+def test_index_kl_checks_its_tensors(M):
+    shape = M.make_shape(H, G, d, d_idx, k)
+    s = _seqs(M, 10, 30)
+    q, kv = _bf(10, H, d), _bf(30, G, d)
+    qi, ki = _bf(10, G, d_idx), _bf(30, d_idx)
+    sel = torch.zeros(10, G, k, dtype=torch.int32)
+    lse = torch.zeros(10, H)
+    with pytest.raises(M.MsaError, match="sel: a tensor is required"):
+        M.msa_index_kl(shape, s, q, kv, qi, ki, None, lse, 0.5)
+    with pytest.raises(M.MsaError, match="lse: shape"):
+        M.msa_index_kl(shape, s, q, kv, qi, ki, sel, torch.zeros(10, G), 0.5)
+    with pytest.raises(M.MsaError, match="kl: dtype"):
+        M.msa_index_kl(shape, s, q, kv, qi, ki, sel, lse, 0.5, kl=torch.zeros(10, G, dtype=torch.float64))
+    with pytest.raises(M.MsaError, match="CUDA"):
+        M.msa_index_kl(shape, s, q, kv, qi, ki, None, lse, 0.5, dense=True)
