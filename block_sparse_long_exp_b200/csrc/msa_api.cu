@@ -409,29 +409,60 @@ msa_status_t msa_sparse_attn_decode_paged(const msa_shape_t* shape, const msa_pa
   return launch_rows_attn(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
 }
 
-msa_status_t msa_index_kl(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q, const void* k,
-                          const void* q_idx, const void* k_idx, const int32_t* sel, const float* lse, float tau,
-                          int32_t dense, float* kl, void* ws, size_t ws_bytes, void* stream) {
+static msa_status_t index_kl_common(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q, const void* k,
+                                   const void* q_idx, const void* k_idx, const int32_t* sel, const float* lse,
+                                   float tau, int32_t dense, void* ws, size_t ws_bytes, void* stream,
+                                   IndexKlArgs* a) {
   msa_status_t st = check_shape(shape);
   if (st != MSA_OK) return st;
   st = check_seqs(seqs);
   if (st != MSA_OK) return st;
   if (!(tau == tau) || tau > 3.0e38f || tau < -3.0e38f) return MSA_ERR_INVALID_ARG;   // NaN or infinite
-  if (seqs->total_q > 0 && (!q || !k || !q_idx || !k_idx || !lse || !kl || (!dense && !sel)))
-    return MSA_ERR_INVALID_ARG;
+  if (seqs->total_q > 0 && (!q || !k || !q_idx || !k_idx || !lse || (!dense && !sel))) return MSA_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, kWsHeader)) return MSA_ERR_WORKSPACE;
   if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MSA_ERR_CUDA;
-  if (seqs->total_q == 0) return MSA_OK;
+  a->q = q; a->key = k; a->q_idx = q_idx; a->k_idx = k_idx; a->sel = sel; a->lse = lse;
+  a->cu_q = seqs->cu_q; a->cu_k = seqs->cu_k;
+  a->batch = seqs->batch; a->H = shape->H; a->G = shape->G; a->d = shape->d; a->d_idx = shape->d_idx;
+  a->k = shape->k;
+  a->total_q = seqs->total_q;
+  a->sm_scale = shape->sm_scale; a->tau = tau; a->dense = dense != 0;
+  a->err = static_cast<DevError*>(ws);
+  return MSA_OK;
+}
+
+msa_status_t msa_index_kl(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q, const void* k,
+                          const void* q_idx, const void* k_idx, const int32_t* sel, const float* lse, float tau,
+                          int32_t dense, float* kl, float* lse_z, void* ws, size_t ws_bytes, void* stream) {
+  if (seqs != nullptr && seqs->total_q > 0 && kl == nullptr) return MSA_ERR_INVALID_ARG;
   IndexKlArgs a{};
-  a.q = q; a.key = k; a.q_idx = q_idx; a.k_idx = k_idx; a.sel = sel; a.lse = lse;
-  a.cu_q = seqs->cu_q; a.cu_k = seqs->cu_k;
-  a.batch = seqs->batch; a.H = shape->H; a.G = shape->G; a.d = shape->d; a.d_idx = shape->d_idx; a.k = shape->k;
-  a.total_q = seqs->total_q;
-  a.sm_scale = shape->sm_scale; a.tau = tau; a.dense = dense != 0;
+  const msa_status_t st = index_kl_common(shape, seqs, q, k, q_idx, k_idx, sel, lse, tau, dense, ws, ws_bytes,
+                                          stream, &a);
+  if (st != MSA_OK || seqs->total_q == 0) return st;
   a.kl = kl;
-  a.err = static_cast<DevError*>(ws);
+  a.lse_z = lse_z;
   return launch_index_kl(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
+}
+
+msa_status_t msa_index_kl_backward(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q,
+                                   const void* k, const void* q_idx, const void* k_idx, const int32_t* sel,
+                                   const float* lse, const float* lse_z, float tau, int32_t dense, float* dq_idx,
+                                   float* dk_idx, void* ws, size_t ws_bytes, void* stream) {
+  if (seqs != nullptr && seqs->total_q > 0 && (lse_z == nullptr || dq_idx == nullptr || dk_idx == nullptr))
+    return MSA_ERR_INVALID_ARG;
+  IndexKlArgs a{};
+  const msa_status_t st = index_kl_common(shape, seqs, q, k, q_idx, k_idx, sel, lse, tau, dense, ws, ws_bytes,
+                                          stream, &a);
+  if (st != MSA_OK || seqs->total_q == 0) return st;
+  // the key gradient is accumulated over every query that reaches a key row
+  if (cudaMemsetAsync(dk_idx, 0, sizeof(float) * (size_t)seqs->total_k * shape->d_idx,
+                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  a.lse_z = const_cast<float*>(lse_z);
+  a.dq_idx = dq_idx;
+  a.dk_idx = dk_idx;
+  return launch_index_kl_backward(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
 }
 
 int32_t msa_set_tile_threshold(int32_t theta) {

@@ -22,10 +22,14 @@ struct IndexKlArgs {
   int64_t total_q;
   float sm_scale, tau;
   int32_t dense;       // 1: the support is every causal token
-  float* kl;           // out [T, G]
+  float* kl;           // forward out [T, G]
+  float* lse_z;        // forward out [T, G] (or null): the student's log-sum-exp; backward in
+  float* dq_idx;       // backward out [T, G, d_idx]
+  float* dk_idx;       // backward out [S, d_idx] (accumulated: zero it first)
   DevError* err;
 };
 
 int launch_index_kl(const IndexKlArgs& a, void* stream);
+int launch_index_kl_backward(const IndexKlArgs& a, void* stream);
 
 }  // namespace msa

@@ -85,11 +85,12 @@ struct KlUnit {
   bool dense;
 };
 
-// Partial sums over the support tokens n = tid, tid + nthreads, ... (tokens
-// numbered in ascending order).  A block id outside 0..pos / B_k sets *bad and
-// is skipped, so no read leaves the sequence.
-MSA_KL_HD KlPartial kl_thread(const KlUnit& u, int tid, int nthreads, int* bad) {
-  KlPartial r{0.f, 0.f, -INFINITY, 0.f};
+// Visits this thread's support tokens n = tid, tid + nthreads, ... (tokens
+// numbered in ascending order) with f(j, P_j, raw index score, index-key
+// row).  A block id outside 0..pos / B_k sets *bad and is skipped, so no read
+// leaves the sequence.
+template <class F>
+MSA_KL_HD void kl_for_tokens(const KlUnit& u, int tid, int nthreads, int* bad, F&& f) {
   const int64_t lb = u.pos / u.B_k;
   const int nblk = u.dense ? static_cast<int>(lb) + 1 : u.nsel;
   int64_t base = 0;   // support tokens before this block
@@ -120,22 +121,31 @@ MSA_KL_HD KlPartial kl_thread(const KlUnit& u, int tid, int nthreads, int* bad) 
       const uint16_t* kij = u.kirow + j * u.d_idx;
       float zs = 0.f;
       for (int c = 0; c < u.d_idx; ++c) zs += u.qif[c] * kl_bf16(kij[c]);
-      const float z = u.tau * zs;
-      if (pbar > 0.f) r.A += pbar * kl_log(pbar);
-      r.B += pbar * z;
-      if (z > r.m) {
-        r.l = r.l * kl_exp(r.m - z) + 1.f;
-        r.m = z;
-      } else {
-        r.l += kl_exp(z - r.m);
-      }
+      f(j, pbar, zs, kij);
     }
   }
+}
+
+// This thread's partial sums of the KL.
+MSA_KL_HD KlPartial kl_thread(const KlUnit& u, int tid, int nthreads, int* bad) {
+  KlPartial r{0.f, 0.f, -INFINITY, 0.f};
+  kl_for_tokens(u, tid, nthreads, bad, [&](int64_t, float pbar, float zs, const uint16_t*) {
+    const float z = u.tau * zs;
+    if (pbar > 0.f) r.A += pbar * kl_log(pbar);
+    r.B += pbar * z;
+    if (z > r.m) {
+      r.l = r.l * kl_exp(r.m - z) + 1.f;
+      r.m = z;
+    } else {
+      r.l += kl_exp(z - r.m);
+    }
+  });
   return r;
 }
 
-// KL = sum A - sum B + log-sum-exp merged over the partials.
-MSA_KL_HD float kl_merge(const KlPartial* p, int n) {
+// KL = sum A - sum B + log-sum-exp merged over the partials; *lse_z (if
+// given) receives the student's log-sum-exp log sum_j exp(z_j).
+MSA_KL_HD float kl_merge(const KlPartial* p, int n, float* lse_z = nullptr) {
   float A = 0.f, B = 0.f, m = -INFINITY;
   for (int i = 0; i < n; ++i) {
     A += p[i].A;
@@ -145,7 +155,33 @@ MSA_KL_HD float kl_merge(const KlPartial* p, int n) {
   float l = 0.f;
   for (int i = 0; i < n; ++i)
     if (p[i].l > 0.f) l += p[i].l * kl_exp(p[i].m - m);
+  if (lse_z != nullptr) *lse_z = l > 0.f ? m + kl_log(l) : -INFINITY;
   return l > 0.f ? A - B + m + kl_log(l) : 0.f;
+}
+
+MSA_KL_HD void kl_add(float* dst, float v) {
+#ifdef __CUDA_ARCH__
+  atomicAdd(dst, v);
+#else
+  *dst += v;
+#endif
+}
+
+// Gradient of KL(P || Q) with the teacher P held constant, over this thread's
+// support tokens: with w_j = tau (Q_j - P_j), Q_j = exp(z_j - lse_z),
+//   dq[c]              += w_j k_idx[j][c]   (the index query's gradient)
+//   dk[j * d_idx + c]  += w_j q_idx[c]      (the index keys' gradient)
+// Both are added atomically on the device (dq: the CTA's threads share one
+// accumulator; dk: other queries add to the same key rows).
+// dk points at the sequence's first key row of the fp32 [S, d_idx] gradient.
+MSA_KL_HD void kl_grad_thread(const KlUnit& u, float lse_z, int tid, int nthreads, float* dq, float* dk, int* bad) {
+  kl_for_tokens(u, tid, nthreads, bad, [&](int64_t j, float pbar, float zs, const uint16_t* kij) {
+    const float w = u.tau * (kl_exp(u.tau * zs - lse_z) - pbar);
+    for (int c = 0; c < u.d_idx; ++c) {
+      kl_add(dq + c, w * kl_bf16(kij[c]));
+      kl_add(dk + j * u.d_idx + c, w * u.qif[c]);
+    }
+  });
 }
 
 }  // namespace msa

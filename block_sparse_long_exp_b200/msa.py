@@ -51,7 +51,7 @@ EXPORTED = [
     "msa_profile_enable", "msa_profile_reset", "msa_profile_read",
     "msa_get_device_error", "msa_version", "msa_set_tile_threshold",
     "msa_decode_paged_workspace_size", "msa_index_topk_decode_paged", "msa_sparse_attn_decode_paged",
-    "msa_index_kl",
+    "msa_index_kl", "msa_index_kl_backward",
 ]
 
 
@@ -130,8 +130,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_index_topk_decode_paged.restype = i32
     lib.msa_sparse_attn_decode_paged.argtypes = [P(Shape), P(Paged), vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.msa_sparse_attn_decode_paged.restype = i32
-    lib.msa_index_kl.argtypes = [P(Shape), P(Varlen), vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp, vp, sz, vp]
+    lib.msa_index_kl.argtypes = [P(Shape), P(Varlen), vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp, vp, vp, sz,
+                                 vp]
     lib.msa_index_kl.restype = i32
+    lib.msa_index_kl_backward.argtypes = [P(Shape), P(Varlen), vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp,
+                                          vp, vp, sz, vp]
+    lib.msa_index_kl_backward.restype = i32
     _lib = lib
     return lib
 
@@ -551,17 +555,7 @@ def msa_sparse_attn_decode_paged(shape: Shape, pages: Paged, q: torch.Tensor, k_
     return out, lse
 
 
-def msa_index_kl(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.Tensor, q_idx: torch.Tensor,
-                 k_idx: torch.Tensor, sel: Optional[torch.Tensor], lse: torch.Tensor, tau: float,
-                 dense: bool = False, kl: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
-                 stream=None, check: bool = True) -> torch.Tensor:
-    """Index-alignment target: KL(P || Q) per (query, group) over the support
-    (the selected tokens, or with dense=True every token up to the query).
-    P: the main branch's attention on the support, averaged over the group's
-    heads (lse [T, H] float: its log-sum-exp over that support, as the prefill
-    or dense call returns it); Q: softmax of tau * index score.  Returns kl
-    float [T, G]."""
-    lib = load_library()
+def _index_kl_args(shape, seqs, q, k, q_idx, k_idx, sel, lse, dense):
     T, S = seqs.total_q, seqs.total_k
     _arg("q", q, torch.bfloat16, (T, shape.H, shape.d))
     _arg("k", k, torch.bfloat16, (S, shape.G, shape.d))
@@ -569,20 +563,63 @@ def msa_index_kl(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.Tensor, q
     _arg("k_idx", k_idx, torch.bfloat16, (S, shape.d_idx))
     _arg("sel", sel, torch.int32, (T, shape.G, shape.k), optional=dense)
     _arg("lse", lse, torch.float32, (T, shape.H))
+
+
+def msa_index_kl(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.Tensor, q_idx: torch.Tensor,
+                 k_idx: torch.Tensor, sel: Optional[torch.Tensor], lse: torch.Tensor, tau: float,
+                 dense: bool = False, kl: Optional[torch.Tensor] = None, want_lse_z: bool = False,
+                 ws: Optional[torch.Tensor] = None, stream=None, check: bool = True):
+    """Index-alignment target: KL(P || Q) per (query, group) over the support
+    (the selected tokens, or with dense=True every token up to the query).
+    P: the main branch's attention on the support, averaged over the group's
+    heads (lse [T, H] float: its log-sum-exp over that support, as the prefill
+    or dense call returns it); Q: softmax of tau * index score.  Returns kl
+    float [T, G], or (kl, lse_z) with want_lse_z (the student's log-sum-exp,
+    which msa_index_kl_backward takes)."""
+    lib = load_library()
+    T = seqs.total_q
+    _index_kl_args(shape, seqs, q, k, q_idx, k_idx, sel, lse, dense)
     _arg("kl", kl, torch.float32, (T, shape.G), optional=True)
     _ws_arg(ws)
     _require_cuda(q, k, q_idx, k_idx, sel, lse, kl, ws)
     if kl is None:
         kl = torch.empty((T, shape.G), dtype=torch.float32, device=q.device)
+    lse_z = torch.empty((T, shape.G), dtype=torch.float32, device=q.device) if want_lse_z else None
     if ws is None:
         ws = _workspace(256, q.device)
     rc = lib.msa_index_kl(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q), _ptr(k), _ptr(q_idx), _ptr(k_idx),
-                          _ptr(sel), _ptr(lse), float(tau), 1 if dense else 0, _ptr(kl), _ptr(ws), _nbytes(ws),
-                          _stream(stream))
+                          _ptr(sel), _ptr(lse), float(tau), 1 if dense else 0, _ptr(kl), _ptr(lse_z), _ptr(ws),
+                          _nbytes(ws), _stream(stream))
     _check(rc, "msa_index_kl")
     if check:
         _device_check(ws, stream, "msa_index_kl")
-    return kl
+    return (kl, lse_z) if want_lse_z else kl
+
+
+def msa_index_kl_backward(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.Tensor, q_idx: torch.Tensor,
+                          k_idx: torch.Tensor, sel: Optional[torch.Tensor], lse: torch.Tensor, lse_z: torch.Tensor,
+                          tau: float, dense: bool = False, ws: Optional[torch.Tensor] = None, stream=None,
+                          check: bool = True) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Gradient of the summed KL with respect to the index query and keys, the
+    teacher held constant: returns dq_idx float [T, G, d_idx] and dk_idx float
+    [S, d_idx].  lse_z: from msa_index_kl(..., want_lse_z=True)."""
+    lib = load_library()
+    T, S = seqs.total_q, seqs.total_k
+    _index_kl_args(shape, seqs, q, k, q_idx, k_idx, sel, lse, dense)
+    _arg("lse_z", lse_z, torch.float32, (T, shape.G))
+    _ws_arg(ws)
+    _require_cuda(q, k, q_idx, k_idx, sel, lse, lse_z, ws)
+    dq = torch.empty((T, shape.G, shape.d_idx), dtype=torch.float32, device=q.device)
+    dk = torch.empty((S, shape.d_idx), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = _workspace(256, q.device)
+    rc = lib.msa_index_kl_backward(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q), _ptr(k), _ptr(q_idx),
+                                   _ptr(k_idx), _ptr(sel), _ptr(lse), _ptr(lse_z), float(tau), 1 if dense else 0,
+                                   _ptr(dq), _ptr(dk), _ptr(ws), _nbytes(ws), _stream(stream))
+    _check(rc, "msa_index_kl_backward")
+    if check:
+        _device_check(ws, stream, "msa_index_kl_backward")
+    return dq, dk
 
 
 def msa_set_tile_threshold(theta: int) -> int:

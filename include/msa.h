@@ -218,7 +218,9 @@ msa_status_t msa_sparse_attn_decode_paged(const msa_shape_t* shape, const msa_pa
  *         the same J, as msa_sparse_attn_prefill returns it for the sparse
  *         support and msa_dense_attn for the dense one),
  *   Q_j = softmax over J of tau * <q_idx[t, g], k_idx[j]>  (the Index Branch).
- *   kl   device float [T, G] (out)
+ *   kl     device float [T, G] (out)
+ *   lse_z  device float [T, G] (out, or NULL): the student's log-sum-exp
+ *          log sum_j exp(z_j), which the backward call takes
  * The teacher P is a constant of this value (its gradient is not the index
  * branch's to follow).  ws: at least 256 bytes, 256-byte aligned (the error
  * word).  A selected block id past the query's block is recorded as
@@ -231,7 +233,21 @@ msa_status_t msa_index_kl(const msa_shape_t* shape, const msa_varlen_t* seqs,
                           const void* k_idx,  /* device bf16 [S, d_idx] */
                           const int32_t* sel, /* device int32 [T, G, k]; NULL allowed when dense */
                           const float* lse,   /* device float [T, H] */
-                          float tau, int32_t dense, float* kl, void* ws, size_t ws_bytes, void* stream);
+                          float tau, int32_t dense, float* kl, float* lse_z, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* Gradient of sum_{t,g} KL(P || Q) with respect to the index query and the
+ * index keys, the teacher held constant (pnsm.cn sec. 4 "gradient detach"):
+ * with w_j = tau (Q_j - P_j) over the support of (t, g),
+ *   dq_idx[t, g, :] = sum_j w_j k_idx[j, :]             (out, float [T, G, d_idx])
+ *   dk_idx[j, :]    = sum over (t, g) of w_j q_idx[t, g, :]  (out, float [S, d_idx];
+ *                     zeroed by the call, then accumulated atomically, so
+ *                     its rounding order varies from run to run)
+ * Arguments as msa_index_kl, plus lse_z from it. */
+msa_status_t msa_index_kl_backward(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q,
+                                   const void* k, const void* q_idx, const void* k_idx, const int32_t* sel,
+                                   const float* lse, const float* lse_z, float tau, int32_t dense, float* dq_idx,
+                                   float* dk_idx, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------- */
 /* Two-phase combine on its own (pnsm.cn sec. 7 "two-phase combine").

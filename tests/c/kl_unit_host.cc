@@ -3,8 +3,10 @@
 // heads, index query and log-sum-exps are staged as float, every thread of a
 // CTA computes its partial sums, and the partials are merged.  Threads are run
 // one after another, for a CTA of 128 threads and of 7 (another partition of
-// the same support).  Reads a case written by tests/test_kl_unit_cpu.py and
-// writes kl[T, G] for both CTA sizes.
+// the same support); then the gradient pass the same way, with the student's
+// log-sum-exp from the forward.  Reads a case written by
+// tests/test_kl_unit_cpu.py and writes, for both CTA sizes, kl[T, G], then
+// dq_idx[T, G, d_idx], then dk_idx[S, d_idx].
 #include <cstdint>
 #include <cstdio>
 #include <vector>
@@ -36,6 +38,7 @@ int main(int argc, char** argv) {
   fclose(f);
   const int Hg = H / G;
   std::vector<float> out((size_t)2 * T * G);
+  std::vector<float> dq((size_t)2 * T * G * d_idx, 0.f), dk((size_t)2 * S * d_idx, 0.f);
   int bad_total = 0;
   for (int b = 0; b < batch; ++b) {
     const int Tb = cu_q[b + 1] - cu_q[b], Sb = cu_k[b + 1] - cu_k[b];
@@ -60,7 +63,12 @@ int main(int argc, char** argv) {
           int bad = 0;
           for (int tid = 0; tid < sizes[s]; ++tid) parts[tid] = msa::kl_thread(u, tid, sizes[s], &bad);
           bad_total += bad;
-          out[(size_t)s * T * G + t * G + g] = msa::kl_merge(parts.data(), sizes[s]);
+          float lse_z = 0.f;
+          out[(size_t)s * T * G + t * G + g] = msa::kl_merge(parts.data(), sizes[s], &lse_z);
+          float* dqu = dq.data() + ((size_t)s * T * G + t * G + g) * d_idx;
+          float* dku = dk.data() + ((size_t)s * S + cu_k[b]) * d_idx;
+          for (int tid = 0; tid < sizes[s]; ++tid) msa::kl_grad_thread(u, lse_z, tid, sizes[s], dqu, dku, &bad);
+          bad_total += bad;
         }
       }
     }
@@ -68,6 +76,8 @@ int main(int argc, char** argv) {
   FILE* o = fopen(argv[2], "wb");
   if (!o) return 2;
   fwrite(out.data(), 4, out.size(), o);
+  fwrite(dq.data(), 4, dq.size(), o);
+  fwrite(dk.data(), 4, dk.size(), o);
   fclose(o);
   printf("bad %d\n", bad_total);
   return 0;

@@ -163,13 +163,18 @@ def test_index_kl_host_validation_without_gpu(lib):
     cu = (ctypes.c_int32 * 2)(0, 0)
     seqs = msa.Varlen(1, 300, 300, 0, 300, 300, ctypes.addressof(cu), ctypes.addressof(cu))
     args = (256, 256, 256, 256)
-    rc = lib.msa_index_kl(ctypes.byref(shape), ctypes.byref(seqs), *args, None, 256, 0.5, 0, 256, 256, 1 << 20, None)
+    rc = lib.msa_index_kl(ctypes.byref(shape), ctypes.byref(seqs), *args, None, 256, 0.5, 0, 256, None, 256, 1 << 20,
+                          None)
     assert rc == 1                                       # sparse support without a selection
-    rc = lib.msa_index_kl(ctypes.byref(shape), ctypes.byref(seqs), *args, 256, 256, float("nan"), 0, 256, 256,
+    rc = lib.msa_index_kl(ctypes.byref(shape), ctypes.byref(seqs), *args, 256, 256, float("nan"), 0, 256, None, 256,
                           1 << 20, None)
     assert rc == 1                                       # tau must be finite
-    rc = lib.msa_index_kl(ctypes.byref(shape), ctypes.byref(seqs), *args, None, 256, 0.5, 1, 256, 256, 16, None)
+    rc = lib.msa_index_kl(ctypes.byref(shape), ctypes.byref(seqs), *args, None, 256, 0.5, 1, 256, None, 256, 16, None)
     assert rc == 3                                       # dense: no selection needed, but the workspace is
     bad = msa.make_shape(64, 4, 96, 64, 16)
-    rc = lib.msa_index_kl(ctypes.byref(bad), ctypes.byref(seqs), *args, 256, 256, 0.5, 0, 256, 256, 1 << 20, None)
+    rc = lib.msa_index_kl(ctypes.byref(bad), ctypes.byref(seqs), *args, 256, 256, 0.5, 0, 256, None, 256, 1 << 20,
+                          None)
     assert rc == 2                                       # d = 96 is not built
+    rc = lib.msa_index_kl_backward(ctypes.byref(shape), ctypes.byref(seqs), *args, 256, 256, None, 0.5, 0, 256, 256,
+                                   256, 1 << 20, None)
+    assert rc == 1                                       # the backward needs the student's log-sum-exp

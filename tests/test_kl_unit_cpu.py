@@ -1,8 +1,10 @@
-"""The index-alignment kernel's arithmetic (msa_kl_unit.cuh: per-thread
-partial sums over a CTA's share of the support, then their merge), built for
+"""The index-alignment kernels' arithmetic (msa_kl_unit.cuh: per-thread
+partial sums over a CTA's share of the support, then their merge; the
+gradient pass with the teacher held constant), built for
 the host with g++ and run on a ragged varlen case for CTAs of 128 and of 7
 threads, against the fp64 oracle of the same target (oracle/index_kl.py), for
-the sparse support and the dense (warmup) one.  Inputs are bf16 values and the
+the sparse support and the dense (warmup) one: the KL and its gradient with
+respect to the index query and keys.  Inputs are bf16 values and the
 log-sum-exps are the oracle's over the same support, so what differs is fp32
 accumulation only."""
 import os
@@ -73,8 +75,17 @@ def test_kl_unit_matches_the_oracle(exe, tmp_path, dense):
     r = subprocess.run([exe, str(case), str(res)], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "bad 0" in r.stdout
-    got = np.fromfile(res, dtype=np.float32).reshape(2, T, G)
+    flat = np.fromfile(res, dtype=np.float32)
+    n_kl, n_dq = 2 * T * G, 2 * T * G * d_idx
+    got = flat[:n_kl].reshape(2, T, G)
+    got_dq = flat[n_kl:n_kl + n_dq].reshape(2, T, G, d_idx)
+    got_dk = flat[n_kl + n_dq:].reshape(2, S, d_idx)
     want = K.index_kl_rows(q, kk, q_idx, k_idx, sel, cu_q, cu_k, rows, B_k, sm, tau, dense=dense)
     assert np.all(want > -1e-9)
+    _, want_dq, want_dk = K.index_kl_loss_and_grad(q, kk, q_idx, k_idx, sel, cu_q, cu_k, B_k, sm, tau, dense=dense)
     for cta in range(2):
         np.testing.assert_allclose(got[cta], want, rtol=2e-4, atol=2e-4)
+        # gradients: fp32 sums of up to 2048 terms of magnitude ~tau * 4
+        scale = np.abs(want_dq).max()
+        np.testing.assert_allclose(got_dq[cta], want_dq, rtol=0, atol=2e-4 * scale)
+        np.testing.assert_allclose(got_dk[cta], want_dk, rtol=0, atol=2e-4 * np.abs(want_dk).max())

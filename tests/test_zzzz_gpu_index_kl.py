@@ -1,5 +1,6 @@
-"""The index-alignment target on the GPU (msa_index_kl) against the fp64
-oracle (oracle/index_kl.py) on every row of a ragged varlen layer whose
+"""The index-alignment target on the GPU (msa_index_kl and its gradient,
+msa_index_kl_backward) against the fp64 oracle (oracle/index_kl.py) on every
+row of a ragged varlen layer whose
 queries are the last T_b tokens: the sparse support with the selection the
 library computed, and the dense (warmup) support.  The log-sum-exps come from
 the oracle (the kernel alone is compared) and then from the library's own
@@ -53,12 +54,20 @@ def test_index_kl_matches_the_oracle(M, dense):
     want = K.index_kl_rows(h["q"], h["k"], h["q_idx"], h["k_idx"], sel_np, cu_q, cu_k, rows, w.B_k, w.sm_scale,
                            TAU, dense=dense)
     lse_dev = torch.from_numpy(lse_ref.astype(np.float32)).cuda()
-    kl = M.msa_index_kl(shape, seqs, d["q"], d["k"], d["q_idx"], d["k_idx"], None if dense else sel, lse_dev, TAU,
-                        dense=dense)
+    s_arg = None if dense else sel
+    kl, lse_z = M.msa_index_kl(shape, seqs, d["q"], d["k"], d["q_idx"], d["k_idx"], s_arg, lse_dev, TAU,
+                               dense=dense, want_lse_z=True)
+    dq, dk = M.msa_index_kl_backward(shape, seqs, d["q"], d["k"], d["q_idx"], d["k_idx"], s_arg, lse_dev, lse_z,
+                                     TAU, dense=dense)
     torch.cuda.synchronize()
     got = kl.cpu().numpy()
     assert np.all(np.isfinite(got)) and np.all(want > -1e-9)
     np.testing.assert_allclose(got, want, rtol=1e-3, atol=1e-3)
+    # gradient with respect to the index query and keys, the teacher held constant
+    _, want_dq, want_dk = K.index_kl_loss_and_grad(h["q"], h["k"], h["q_idx"], h["k_idx"], sel_np, cu_q, cu_k,
+                                                   w.B_k, w.sm_scale, TAU, dense=dense)
+    np.testing.assert_allclose(dq.cpu().numpy(), want_dq, rtol=0, atol=2e-3 * np.abs(want_dq).max())
+    np.testing.assert_allclose(dk.cpu().numpy(), want_dk, rtol=0, atol=2e-3 * np.abs(want_dk).max())
     # the same with the library's own log-sum-exps
     if dense:
         _, lse_lib = M.msa_dense_attn(shape, seqs, d["q"], d["k"], d["v"], want_lse=True)
