@@ -10,6 +10,7 @@
 
 #include "msa_internal.h"
 #include "msa_kl.h"
+#include "msa_window.h"
 
 using namespace msa;
 
@@ -463,6 +464,24 @@ msa_status_t msa_index_kl_backward(const msa_shape_t* shape, const msa_varlen_t*
   a.dq_idx = dq_idx;
   a.dk_idx = dk_idx;
   return launch_index_kl_backward(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
+}
+
+msa_status_t msa_select_window(const msa_shape_t* shape, const msa_varlen_t* seqs, int32_t n_sink, int32_t* sel,
+                               void* ws, size_t ws_bytes, void* stream) {
+  msa_status_t st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  st = check_seqs(seqs);
+  if (st != MSA_OK) return st;
+  if (n_sink < 0 || n_sink >= shape->k) return MSA_ERR_INVALID_ARG;
+  if (seqs->total_q > 0 && sel == nullptr) return MSA_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, kWsHeader)) return MSA_ERR_WORKSPACE;
+  if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  if (seqs->total_q == 0) return MSA_OK;
+  return launch_window_select(seqs->cu_q, seqs->cu_k, seqs->batch, shape->G, shape->k, n_sink, seqs->total_q, sel,
+                              static_cast<DevError*>(ws), stream) == 0
+             ? MSA_OK
+             : MSA_ERR_CUDA;
 }
 
 int32_t msa_set_tile_threshold(int32_t theta) {

@@ -51,7 +51,7 @@ EXPORTED = [
     "msa_profile_enable", "msa_profile_reset", "msa_profile_read",
     "msa_get_device_error", "msa_version", "msa_set_tile_threshold",
     "msa_decode_paged_workspace_size", "msa_index_topk_decode_paged", "msa_sparse_attn_decode_paged",
-    "msa_index_kl", "msa_index_kl_backward",
+    "msa_index_kl", "msa_index_kl_backward", "msa_select_window",
 ]
 
 
@@ -136,6 +136,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_index_kl_backward.argtypes = [P(Shape), P(Varlen), vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp,
                                           vp, vp, sz, vp]
     lib.msa_index_kl_backward.restype = i32
+    lib.msa_select_window.argtypes = [P(Shape), P(Varlen), i32, vp, vp, sz, vp]
+    lib.msa_select_window.restype = i32
     _lib = lib
     return lib
 
@@ -620,6 +622,29 @@ def msa_index_kl_backward(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.
     if check:
         _device_check(ws, stream, "msa_index_kl_backward")
     return dq, dk
+
+
+def msa_select_window(shape: Shape, seqs: Varlen, n_sink: int = 1, sel: Optional[torch.Tensor] = None,
+                      ws: Optional[torch.Tensor] = None, device=None, stream=None, check: bool = True) -> torch.Tensor:
+    """The FLOP-matched sliding-window baseline's selection: the first n_sink
+    blocks and the k - n_sink most recent ones per (query, group), in
+    msa_index_topk's layout (sel int32 [T, G, k]), for the main-branch calls."""
+    lib = load_library()
+    T = seqs.total_q
+    _arg("sel", sel, torch.int32, (T, shape.G, shape.k), optional=True)
+    _ws_arg(ws)
+    dev = sel.device if sel is not None else (device or torch.device("cuda"))
+    if sel is None:
+        sel = torch.empty((T, shape.G, shape.k), dtype=torch.int32, device=dev)
+    _require_cuda(sel, ws)
+    if ws is None:
+        ws = _workspace(256, sel.device)
+    rc = lib.msa_select_window(ctypes.byref(shape), ctypes.byref(seqs), int(n_sink), _ptr(sel), _ptr(ws),
+                               _nbytes(ws), _stream(stream))
+    _check(rc, "msa_select_window")
+    if check:
+        _device_check(ws, stream, "msa_select_window")
+    return sel
 
 
 def msa_set_tile_threshold(theta: int) -> int:

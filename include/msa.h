@@ -209,6 +209,18 @@ msa_status_t msa_sparse_attn_decode_paged(const msa_shape_t* shape, const msa_pa
                                           void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* The FLOP-matched sliding-window baseline's selection (pnsm.cn sec. 6
+ * "Learnable sink 和滑动窗口消融"; yhxrc.cn sec. 三): for every (query, group)
+ * the first n_sink blocks and the k - n_sink most recent ones (the query's own
+ * block last), ascending, -1 padded; every causal block when there are at most
+ * k.  No index scores: sel has msa_index_topk's layout, so the main-branch
+ * calls run the baseline unchanged.  0 <= n_sink < k.  ws: at least 256
+ * bytes, 256-byte aligned (the error word). */
+msa_status_t msa_select_window(const msa_shape_t* shape, const msa_varlen_t* seqs, int32_t n_sink,
+                               int32_t* sel, /* device int32 [T, G, k] (out) */
+                               void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* Index-alignment target (pnsm.cn sec. 4 "KL alignment", sec. 5 "Indexer
  * warmup"; yhxrc.cn sec. 二): for every query t and group g, the KL divergence
  * KL(P || Q) over the support J (the tokens of the selected blocks sel[t, g]
