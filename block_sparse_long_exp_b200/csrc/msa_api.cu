@@ -11,6 +11,7 @@
 #include "msa_internal.h"
 #include "msa_kl.h"
 #include "msa_window.h"
+#include "msa_bwd.h"
 
 using namespace msa;
 
@@ -482,6 +483,36 @@ msa_status_t msa_select_window(const msa_shape_t* shape, const msa_varlen_t* seq
                               static_cast<DevError*>(ws), stream) == 0
              ? MSA_OK
              : MSA_ERR_CUDA;
+}
+
+msa_status_t msa_sparse_attn_backward(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q,
+                                      const void* k, const void* v, const int32_t* sel, const void* out,
+                                      const float* lse, const void* dout, int32_t dense, float* dq, float* dk,
+                                      float* dv, void* ws, size_t ws_bytes, void* stream) {
+  msa_status_t st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  st = check_seqs(seqs);
+  if (st != MSA_OK) return st;
+  if (seqs->total_q > 0 &&
+      (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || (!dense && !sel)))
+    return MSA_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, kWsHeader)) return MSA_ERR_WORKSPACE;
+  cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(DevError), st_) != cudaSuccess) return MSA_ERR_CUDA;
+  if (seqs->total_q == 0) return MSA_OK;
+  // dk and dv are accumulated over every query that reaches a key row
+  const size_t kv_bytes = sizeof(float) * (size_t)seqs->total_k * shape->G * shape->d;
+  if (cudaMemsetAsync(dk, 0, kv_bytes, st_) != cudaSuccess || cudaMemsetAsync(dv, 0, kv_bytes, st_) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  AttnBwdArgs a{};
+  a.q = q; a.key = k; a.value = v; a.sel = sel; a.out = out; a.lse = lse; a.dout = dout;
+  a.cu_q = seqs->cu_q; a.cu_k = seqs->cu_k;
+  a.batch = seqs->batch; a.H = shape->H; a.G = shape->G; a.d = shape->d; a.k = shape->k;
+  a.total_q = seqs->total_q;
+  a.sm_scale = shape->sm_scale; a.dense = dense != 0;
+  a.dq = dq; a.dk = dk; a.dv = dv;
+  a.err = static_cast<DevError*>(ws);
+  return launch_sparse_attn_backward(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
 }
 
 int32_t msa_set_tile_threshold(int32_t theta) {

@@ -51,7 +51,7 @@ EXPORTED = [
     "msa_profile_enable", "msa_profile_reset", "msa_profile_read",
     "msa_get_device_error", "msa_version", "msa_set_tile_threshold",
     "msa_decode_paged_workspace_size", "msa_index_topk_decode_paged", "msa_sparse_attn_decode_paged",
-    "msa_index_kl", "msa_index_kl_backward", "msa_select_window",
+    "msa_index_kl", "msa_index_kl_backward", "msa_select_window", "msa_sparse_attn_backward",
 ]
 
 
@@ -138,6 +138,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_index_kl_backward.restype = i32
     lib.msa_select_window.argtypes = [P(Shape), P(Varlen), i32, vp, vp, sz, vp]
     lib.msa_select_window.restype = i32
+    lib.msa_sparse_attn_backward.argtypes = [P(Shape), P(Varlen), vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, sz,
+                                             vp]
+    lib.msa_sparse_attn_backward.restype = i32
     _lib = lib
     return lib
 
@@ -645,6 +648,39 @@ def msa_select_window(shape: Shape, seqs: Varlen, n_sink: int = 1, sel: Optional
     if check:
         _device_check(ws, stream, "msa_select_window")
     return sel
+
+
+def msa_sparse_attn_backward(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                             sel: Optional[torch.Tensor], out: torch.Tensor, lse: torch.Tensor, dout: torch.Tensor,
+                             dense: bool = False, ws: Optional[torch.Tensor] = None, stream=None,
+                             check: bool = True) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Main Branch backward over the support (the selected tokens, or with
+    dense=True every token up to the query): returns dq float [T, H, d] and
+    dk, dv float [S, G, d].  out / lse: the forward's outputs for the same
+    support; dout: bf16 [T, H, d]."""
+    lib = load_library()
+    T, S = seqs.total_q, seqs.total_k
+    _arg("q", q, torch.bfloat16, (T, shape.H, shape.d))
+    _arg("k", k, torch.bfloat16, (S, shape.G, shape.d))
+    _arg("v", v, torch.bfloat16, (S, shape.G, shape.d))
+    _arg("sel", sel, torch.int32, (T, shape.G, shape.k), optional=dense)
+    _arg("out", out, torch.bfloat16, (T, shape.H, shape.d))
+    _arg("lse", lse, torch.float32, (T, shape.H))
+    _arg("dout", dout, torch.bfloat16, (T, shape.H, shape.d))
+    _ws_arg(ws)
+    _require_cuda(q, k, v, sel, out, lse, dout, ws)
+    dq = torch.empty((T, shape.H, shape.d), dtype=torch.float32, device=q.device)
+    dk = torch.empty((S, shape.G, shape.d), dtype=torch.float32, device=q.device)
+    dv = torch.empty((S, shape.G, shape.d), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = _workspace(256, q.device)
+    rc = lib.msa_sparse_attn_backward(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q), _ptr(k), _ptr(v), _ptr(sel),
+                                      _ptr(out), _ptr(lse), _ptr(dout), 1 if dense else 0, _ptr(dq), _ptr(dk),
+                                      _ptr(dv), _ptr(ws), _nbytes(ws), _stream(stream))
+    _check(rc, "msa_sparse_attn_backward")
+    if check:
+        _device_check(ws, stream, "msa_sparse_attn_backward")
+    return dq, dk, dv
 
 
 def msa_set_tile_threshold(theta: int) -> int:

@@ -209,6 +209,33 @@ msa_status_t msa_sparse_attn_decode_paged(const msa_shape_t* shape, const msa_pa
                                           void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Main Branch backward: the gradients of the attention over the support J
+ * (the selected blocks' tokens cut at the query, or with dense != 0 every
+ * token up to it) for an upstream gradient dout.  With P_j = exp(sm_scale
+ * q_h.k_j - lse[t, h]), dP_j = dout_h.v_j, D = dout_h.out_h, dS_j = P_j (dP_j
+ * - D):
+ *   dq[t, h]  = sm_scale sum_j dS_j k_j                 (out, float [T, H, d])
+ *   dk[j, g] += sm_scale dS_j q[t, h],  dv[j, g] += P_j dout[t, h]
+ *                                                      (out, float [S, G, d];
+ *               zeroed by the call, then accumulated atomically, so their
+ *               rounding order varies from run to run)
+ * out and lse are the forward's outputs for the same support (prefill or
+ * dense call).  The selection is not differentiated.  ws: at least 256
+ * bytes, 256-byte aligned.  A selected block id past the query's block is
+ * recorded as MSA_ERR_DEVICE_CHECK and left out.  A first, CUDA-core form
+ * (one CTA per (query, group)). */
+msa_status_t msa_sparse_attn_backward(const msa_shape_t* shape, const msa_varlen_t* seqs,
+                                      const void* q,      /* device bf16 [T, H, d] */
+                                      const void* k,      /* device bf16 [S, G, d] */
+                                      const void* v,      /* device bf16 [S, G, d] */
+                                      const int32_t* sel, /* device int32 [T, G, k]; NULL allowed when dense */
+                                      const void* out,    /* device bf16 [T, H, d] */
+                                      const float* lse,   /* device float [T, H] */
+                                      const void* dout,   /* device bf16 [T, H, d] */
+                                      int32_t dense, float* dq, float* dk, float* dv, void* ws, size_t ws_bytes,
+                                      void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* The FLOP-matched sliding-window baseline's selection (pnsm.cn sec. 6
  * "Learnable sink 和滑动窗口消融"; yhxrc.cn sec. 三): for every (query, group)
  * the first n_sink blocks and the k - n_sink most recent ones (the query's own

@@ -63,6 +63,7 @@ def main_branch_backward(q, k, v, sel, dout, cu_q, cu_k, B_k: int, sm_scale: flo
                     dP = Vj @ dout[t, h]
                     dS = P * (dP - dout[t, h] @ o)
                     dq[t, h] = sm_scale * (dS @ Kj)
-                    np.add.at(dk[:, g], k0 + J, sm_scale * np.outer(dS, q[t, h]))
-                    np.add.at(dv[:, g], k0 + J, np.outer(P, dout[t, h]))
+                    # J holds each token once, so indexed += adds every row exactly once
+                    dk[k0 + J, g] += sm_scale * np.outer(dS, q[t, h])
+                    dv[k0 + J, g] += np.outer(P, dout[t, h])
     return dq, dk, dv

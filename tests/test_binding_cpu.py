@@ -146,3 +146,18 @@ def test_index_kl_checks_its_tensors(M):
         M.msa_index_kl(shape, s, q, kv, qi, ki, sel, lse, 0.5, kl=torch.zeros(10, G, dtype=torch.float64))
     with pytest.raises(M.MsaError, match="CUDA"):
         M.msa_index_kl(shape, s, q, kv, qi, ki, None, lse, 0.5, dense=True)
+
+
+def test_backward_checks_its_tensors(M):
+    shape = M.make_shape(H, G, d, d_idx, k)
+    s = _seqs(M, 10, 30)
+    q, kv, sel = _bf(10, H, d), _bf(30, G, d), torch.zeros(10, G, k, dtype=torch.int32)
+    lse = torch.zeros(10, H)
+    with pytest.raises(M.MsaError, match="dout: shape"):
+        M.msa_sparse_attn_backward(shape, s, q, kv, kv, sel, q, lse, _bf(10, H, d + 1))
+    with pytest.raises(M.MsaError, match="out: dtype"):
+        M.msa_sparse_attn_backward(shape, s, q, kv, kv, sel, q.float(), lse, q)
+    with pytest.raises(M.MsaError, match="sel: a tensor is required"):
+        M.msa_sparse_attn_backward(shape, s, q, kv, kv, None, q, lse, q)
+    with pytest.raises(M.MsaError, match="CUDA"):
+        M.msa_sparse_attn_backward(shape, s, q, kv, kv, None, q, lse, q, dense=True)
