@@ -515,6 +515,12 @@ msa_status_t msa_sparse_attn_backward(const msa_shape_t* shape, const msa_varlen
   return launch_sparse_attn_backward(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
 }
 
+msa_status_t msa_selected_share(const float* lse_sel, const float* lse_all, int64_t n, float* share, void* stream) {
+  if (n < 0) return MSA_ERR_INVALID_ARG;
+  if (n > 0 && (!lse_sel || !lse_all || !share)) return MSA_ERR_INVALID_ARG;
+  return launch_selected_share(lse_sel, lse_all, n, share, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
+}
+
 int32_t msa_set_tile_threshold(int32_t theta) {
   return g_tile_theta.exchange(theta < 0 ? -1 : theta);
 }

@@ -32,6 +32,8 @@ MSA_WIN_HD void window_blocks(int64_t lb, int k, int n_sink, int32_t* out) {
 
 int launch_window_select(const int32_t* cu_q, const int32_t* cu_k, int32_t batch, int32_t G, int32_t k,
                          int32_t n_sink, int64_t total_q, int32_t* sel, DevError* err, void* stream);
+// share[i] = exp(lse_sel[i] - lse_all[i]) for i < n (msa_window_select.cu).
+int launch_selected_share(const float* lse_sel, const float* lse_all, int64_t n, float* share, void* stream);
 
 }  // namespace msa
 

@@ -54,3 +54,33 @@ int launch_window_select(const int32_t* cu_q, const int32_t* cu_k, int32_t batch
 }
 
 }  // namespace msa
+
+// ---------------------------------------------------------------------------
+// The share of each head's dense causal attention weight that the selected
+// tokens hold (the pages report the selection covering most of the Main
+// Branch's attention weight; yhxrc.cn sec. 二): with lse_sel the log-sum-exp
+// over the selected tokens and lse_all the one over every causal token,
+// share = sum_{j in J} softmax_all(s)_j = exp(lse_sel - lse_all).
+namespace msa {
+namespace {
+
+__global__ void __launch_bounds__(256)
+selected_share_kernel(const float* __restrict__ lse_sel, const float* __restrict__ lse_all, int64_t n,
+                      float* __restrict__ share) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) share[i] = __expf(lse_sel[i] - lse_all[i]);
+}
+
+}  // namespace
+
+int launch_selected_share(const float* lse_sel, const float* lse_all, int64_t n, float* share, void* stream) {
+  if (n <= 0) return 0;
+  const int64_t blocks = (n + 255) / 256;
+  if (blocks > 0x7fffffffLL) return (int)cudaErrorInvalidValue;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  ProfScope p("selected_share", stream);
+  selected_share_kernel<<<(unsigned)blocks, 256, 0, st>>>(lse_sel, lse_all, n, share);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace msa

@@ -52,6 +52,7 @@ EXPORTED = [
     "msa_get_device_error", "msa_version", "msa_set_tile_threshold",
     "msa_decode_paged_workspace_size", "msa_index_topk_decode_paged", "msa_sparse_attn_decode_paged",
     "msa_index_kl", "msa_index_kl_backward", "msa_select_window", "msa_sparse_attn_backward",
+    "msa_selected_share",
 ]
 
 
@@ -141,6 +142,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_sparse_attn_backward.argtypes = [P(Shape), P(Varlen), vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, sz,
                                              vp]
     lib.msa_sparse_attn_backward.restype = i32
+    lib.msa_selected_share.argtypes = [vp, vp, i64, vp, vp]
+    lib.msa_selected_share.restype = i32
     _lib = lib
     return lib
 
@@ -681,6 +684,20 @@ def msa_sparse_attn_backward(shape: Shape, seqs: Varlen, q: torch.Tensor, k: tor
     if check:
         _device_check(ws, stream, "msa_sparse_attn_backward")
     return dq, dk, dv
+
+
+def msa_selected_share(lse_sel: torch.Tensor, lse_all: torch.Tensor, stream=None) -> torch.Tensor:
+    """Share of each head's dense causal attention weight on the selected
+    tokens: exp(lse_sel - lse_all), lse_sel from msa_sparse_attn_prefill and
+    lse_all from msa_dense_attn (float [T, H] each)."""
+    lib = load_library()
+    _arg("lse_sel", lse_sel, torch.float32)
+    _arg("lse_all", lse_all, torch.float32, tuple(lse_sel.shape))
+    _require_cuda(lse_sel, lse_all)
+    share = torch.empty_like(lse_sel)
+    rc = lib.msa_selected_share(_ptr(lse_sel), _ptr(lse_all), lse_sel.numel(), _ptr(share), _stream(stream))
+    _check(rc, "msa_selected_share")
+    return share
 
 
 def msa_set_tile_threshold(theta: int) -> int:

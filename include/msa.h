@@ -247,6 +247,14 @@ msa_status_t msa_select_window(const msa_shape_t* shape, const msa_varlen_t* seq
                                int32_t* sel, /* device int32 [T, G, k] (out) */
                                void* ws, size_t ws_bytes, void* stream);
 
+/* The share of each head's dense causal attention weight that the selected
+ * tokens hold, the monitor the pages report for the selection (yhxrc.cn sec.
+ * 二): share[i] = exp(lse_sel[i] - lse_all[i]), with lse_sel from
+ * msa_sparse_attn_prefill and lse_all from msa_dense_attn on the same layer
+ * (both device float [T, H]; n = T * H). */
+msa_status_t msa_selected_share(const float* lse_sel, const float* lse_all, int64_t n, float* share,
+                                void* stream);
+
 /* ---------------------------------------------------------------------- */
 /* Index-alignment target (pnsm.cn sec. 4 "KL alignment", sec. 5 "Indexer
  * warmup"; yhxrc.cn sec. 二): for every query t and group g, the KL divergence

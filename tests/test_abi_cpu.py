@@ -178,3 +178,9 @@ def test_index_kl_host_validation_without_gpu(lib):
     rc = lib.msa_index_kl_backward(ctypes.byref(shape), ctypes.byref(seqs), *args, 256, 256, None, 0.5, 0, 256, 256,
                                    256, 1 << 20, None)
     assert rc == 1                                       # the backward needs the student's log-sum-exp
+
+
+def test_selected_share_host_checks(lib):
+    assert lib.msa_selected_share(None, None, 0, None, None) == 0       # nothing to do
+    assert lib.msa_selected_share(None, 256, 5, 256, None) == 1
+    assert lib.msa_selected_share(256, 256, -1, 256, None) == 1
