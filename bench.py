@@ -131,14 +131,17 @@ def pass_rows(q_chunk, T):
 
 
 def run_config(args, w, T, world):
-    """The workload description, printed the same by both arms."""
+    """The workload description, printed the same by both arms (T: the
+    layer's query tokens)."""
+    par = (f"query ranges of one layer x{world}" if getattr(args, "shard", "none") == "queries"
+           else f"independent layer per GPU x{world}")
     return {"workload": args.workload, "T": T, "H": w.H, "G": w.G, "d": w.d, "d_idx": w.d_idx,
             "B_k": w.B_k, "k": w.k, "hot_block_frac": w.hot_frac,
             "l2": ("inputs larger than L2 (q alone is %.1f GB)" % (T * w.H * w.d * 2 / 1e9)
                    if T * w.H * w.d * 2 > L2_BYTES else
                    "inputs fit in L2 (q is %.0f MB, L2 not flushed): a profiling size, not a timing one"
                    % (T * w.H * w.d * 2 / 1e6)),
-            "parallelism": f"independent layer per GPU x{world}",
+            "parallelism": par,
             "attention_pass_rows": pass_rows(args.q_chunk, T) or T}
 
 
@@ -408,9 +411,20 @@ def run_ours(args):
         uq = 2 * (128 // max(w_.H // w_.G, 8))
         return (5 * uq + 7) // 8
     w = W.WORKLOADS[args.workload]
-    # each rank runs an independent layer (its own seed): weak scaling
-    wr = rank_workload(w, rank, W)
+    shard_q = args.shard == "queries"
+    # weak scaling: each rank runs an independent layer (its own seed); with
+    # --shard queries every rank holds the same layer and computes one range
+    # of its queries as a chunked prefill (strong scaling, no collective)
+    wr = w if shard_q else rank_workload(w, rank, W)
     inp = W.make_inputs(wr, "cuda", T_override=args.T or None)
+    T_layer = inp["cu_q_host"][-1]
+    if shard_q:
+        from block_sparse_long_exp_b200 import shard as SH
+        if len(inp["cu_q_host"]) != 2 or w.kind != "prefill":
+            raise SystemExit("--shard queries takes a single-sequence prefill workload")
+        work_q = SH.query_work(T_layer, w.H, w.G, w.d, w.d_idx, w.B_k, w.k)
+        a_, b_ = SH.split_query_ranges(work_q, world, align=w.B_k)[rank]
+        inp = SH.chunk_of(inp, a_, b_)
     torch.cuda.synchronize()
     make_ctx.index_only = args.index_only
     make_ctx.q_chunk = args.q_chunk
@@ -584,9 +598,10 @@ def run_ours(args):
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+                "scaling": "strong" if shard_q else "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": run_config(args, w, T, world),
+                "config": run_config(args, w, T_layer, world),
                 "roofline": roof, "step_roofline": step_roof, "tile_split": split, "dense_gqa": dense,
                 "decode": decode, "e2e": e2e,
                 "cpu_baseline": cpu, "clocks": clk, "gpu_launches": launches, "kernels": kernels}
@@ -615,6 +630,9 @@ def build_parser():
                     help="query-tile threshold of the prefill (-1 automatic, 0 off)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--shard", choices=["none", "queries"], default="none",
+                    help="N > 1: independent layers per rank (none, weak scaling) or the query ranges of one "
+                         "layer split across ranks (queries, strong scaling)")
     return ap
 
 

@@ -1,0 +1,66 @@
+"""Splitting one long sequence's prefill across ranks by query ranges.
+
+A query's result depends only on its own position and the keys before it, so
+rank r can compute the queries [a_r, b_r) of a sequence by itself as a chunked
+prefill: queries [a_r, b_r) over keys [0, b_r) (the calls take the queries of
+a sequence as its last T_b tokens).  No collective is needed while the output
+stays sharded; the keys [0, b_r) must be present on rank r.
+
+The work per query grows with its position (the index branch scores every
+earlier block), so equal row counts would leave the last rank the most work:
+the ranges are cut at equal shares of the algorithmic work instead.
+"""
+from __future__ import annotations
+
+from typing import Dict, List, Tuple
+
+import numpy as np
+
+
+def query_work(S: int, H: int, G: int, d: int, d_idx: int, B_k: int, k: int) -> np.ndarray:
+    """Algorithmic FLOPs of each query position 0 .. S-1 of a prefill (index
+    branch: 2 G d_idx B_k (nb - 1) when nb > k; main branch: 4 H d att)."""
+    p = np.arange(S, dtype=np.int64)
+    nb = p // B_k + 1
+    idx = np.where(nb > k, 2 * G * d_idx * B_k * (nb - 1), 0)
+    att = np.where(nb > k, (k - 1) * B_k + p % B_k + 1, p + 1)
+    return (idx + 4 * H * d * att).astype(np.float64)
+
+
+def split_query_ranges(work: np.ndarray, world: int, align: int = 1) -> List[Tuple[int, int]]:
+    """Contiguous ranges [a, b) covering 0 .. len(work) whose work sums are as
+    equal as cuts at multiples of `align` allow (a rank may get an empty range
+    only when there are fewer aligned rows than ranks)."""
+    n = len(work)
+    if world < 1:
+        raise ValueError("world must be >= 1")
+    csum = np.concatenate([[0.0], np.cumsum(work)])
+    cuts = [0]
+    for r in range(1, world):
+        target = csum[-1] * r / world
+        c = int(np.searchsorted(csum, target))
+        c = min(n, max(cuts[-1], int(round(c / align)) * align))
+        cuts.append(c)
+    cuts.append(n)
+    return [(cuts[r], cuts[r + 1]) for r in range(world)]
+
+
+def chunk_of(inp: Dict[str, object], a: int, b: int) -> Dict[str, object]:
+    """The inputs of one sequence's prefill (q/q_idx [S, ...], k/v/k_idx
+    [S, ...], torch tensors) cut to the chunked call of queries [a, b): queries
+    rows a .. b-1, keys rows 0 .. b-1, offsets [0, b-a] and [0, b]."""
+    import torch
+    dev = inp["q"].device
+    return {
+        "q": inp["q"][a:b], "q_idx": inp["q_idx"][a:b],
+        "k": inp["k"][:b], "v": inp["v"][:b], "k_idx": inp["k_idx"][:b],
+        "cu_q": torch.tensor([0, b - a], dtype=torch.int32, device=dev),
+        "cu_k": torch.tensor([0, b], dtype=torch.int32, device=dev),
+        "cu_q_host": [0, b - a], "cu_k_host": [0, b],
+    }
+
+
+def imbalance(work: np.ndarray, ranges: List[Tuple[int, int]]) -> float:
+    """Largest rank's work over the mean (1.0 = perfect balance)."""
+    per = [float(work[a:b].sum()) for a, b in ranges]
+    return max(per) / (sum(per) / len(per))

@@ -1,0 +1,86 @@
+"""Query-range sharding of one sequence's prefill (block_sparse_long_exp_b200/
+shard.py): the planner's ranges cover every query once and balance the
+algorithmic work; and on two gloo ranks, each rank's chunked-prefill oracle
+result (queries [a, b) over keys [0, b)) gathered on rank 0 equals the
+unsharded oracle result row for row."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from block_sparse_long_exp_b200 import roofline as R
+from block_sparse_long_exp_b200 import shard as SH
+
+
+def test_ranges_cover_and_balance():
+    H, G, d, d_idx, B_k, k = 64, 4, 128, 64, 128, 16
+    S = 131072
+    work = SH.query_work(S, H, G, d, d_idx, B_k, k)
+    # the per-query work sums to the layer's algorithmic FLOPs
+    w = R.prefill_work([S], [S], H, G, d, d_idx, B_k, k)
+    assert work.sum() == pytest.approx(w["flops"], rel=1e-12)
+    for world in (1, 2, 3, 8):
+        ranges = SH.split_query_ranges(work, world, align=128)
+        assert ranges[0][0] == 0 and ranges[-1][1] == S
+        assert all(a <= b for a, b in ranges) and all(ranges[i][1] == ranges[i + 1][0] for i in range(world - 1))
+        assert all(a % 128 == 0 for a, _ in ranges)
+        assert SH.imbalance(work, ranges) < 1.01
+        if world > 1:   # equal row counts would be far worse: the index work grows with position
+            even = [(r * S // world, (r + 1) * S // world) for r in range(world)]
+            assert SH.imbalance(work, even) > SH.imbalance(work, ranges) + 0.1
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, result):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from block_sparse_long_exp_b200 import workloads as W
+        from oracle import msa_oracle as O
+        w = W.Workload("shard", "prefill", H=8, G=2, d=16, d_idx=8, B_k=4, k=3, seed=5, hot_frac=0.1)
+        inp = W.make_inputs(w, "cpu", lengths=[61])
+        work = SH.query_work(61, w.H, w.G, w.d, w.d_idx, w.B_k, w.k)
+        a, b = SH.split_query_ranges(work, world)[rank]
+        c = SH.chunk_of(inp, a, b)
+        f = lambda t: t.float().numpy().astype(np.float64)  # noqa: E731
+        sel = O.index_topk(f(c["q_idx"]), f(c["k_idx"]), c["cu_q_host"], c["cu_k_host"], w.k, w.B_k)
+        o, lse = O.msa_forward_rows(f(c["q"]), f(c["k"]), f(c["v"]), sel, c["cu_q_host"], c["cu_k_host"],
+                                    list(range(b - a)), w.B_k, w.sm_scale)
+        parts = [None] * world
+        dist.all_gather_object(parts, (a, b, sel, o, lse))
+        if rank == 0:
+            full_sel = O.index_topk(f(inp["q_idx"]), f(inp["k_idx"]), [0, 61], [0, 61], w.k, w.B_k)
+            full_o, full_l = O.msa_forward_rows(f(inp["q"]), f(inp["k"]), f(inp["v"]), full_sel, [0, 61], [0, 61],
+                                                list(range(61)), w.B_k, w.sm_scale)
+            ok = sorted(p[:2] for p in parts) == sorted(SH.split_query_ranges(work, world))
+            for a_, b_, s_, o_, l_ in parts:
+                ok = ok and np.array_equal(s_, full_sel[a_:b_])
+                ok = ok and np.allclose(o_, full_o[a_:b_], rtol=0, atol=1e-12)
+                ok = ok and np.allclose(l_, full_l[a_:b_], rtol=0, atol=1e-12)
+            result.put(bool(ok))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_oracle_equals_unsharded_on_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    result = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, result)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+    assert all(p.exitcode == 0 for p in procs)
+    assert result.get(timeout=10) is True
