@@ -64,3 +64,19 @@ def imbalance(work: np.ndarray, ranges: List[Tuple[int, int]]) -> float:
     """Largest rank's work over the mean (1.0 = perfect balance)."""
     per = [float(work[a:b].sum()) for a, b in ranges]
     return max(per) / (sum(per) / len(per))
+
+
+def decode_shards(lengths, world: int) -> List[List[int]]:
+    """Decode sequences split across ranks: longest first, each to the rank
+    with the least cached tokens so far (the decode step streams every cached
+    index key, so its time follows the cached length).  Returns each rank's
+    sequence ids, ascending."""
+    if world < 1:
+        raise ValueError("world must be >= 1")
+    load = [0] * world
+    out: List[List[int]] = [[] for _ in range(world)]
+    for i in sorted(range(len(lengths)), key=lambda i: (-int(lengths[i]), i)):
+        r = min(range(world), key=lambda r: (load[r], r))
+        out[r].append(i)
+        load[r] += int(lengths[i])
+    return [sorted(o) for o in out]

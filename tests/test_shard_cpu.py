@@ -84,3 +84,16 @@ def test_sharded_oracle_equals_unsharded_on_two_gloo_ranks():
         p.join(timeout=300)
     assert all(p.exitcode == 0 for p in procs)
     assert result.get(timeout=10) is True
+
+
+def test_decode_shards_cover_and_balance():
+    from block_sparse_long_exp_b200 import workloads as W
+    w = W.WORKLOADS["decode_b32_l128k_1m_hot2"]
+    L = W.seq_lengths(w, torch.Generator().manual_seed(w.seed))
+    for world in (1, 2, 4, 8):
+        parts = SH.decode_shards(L, world)
+        assert sorted(i for p in parts for i in p) == list(range(len(L)))
+        loads = [sum(L[i] for i in p) for p in parts]
+        # longest-first greedy: no rank exceeds the mean by more than the longest cache
+        assert max(loads) <= sum(loads) / world + max(L)
+        assert max(loads) / (sum(loads) / world) < 1.2
