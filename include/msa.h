@@ -392,7 +392,21 @@ msa_status_t msa_profile_read(const char* kernel, double* total_ms, int64_t* cou
 /* ---------------------------------------------------------------------- */
 /* Device error word of a workspace.  Waits for `stream`, copies the word to
  * the host and clears it.  *code is an msa_status_t (MSA_OK if none);
- * *where names the kernel site, *info0 / *info1 carry details. */
+ * *where names the kernel site, *info0 / *info1 carry details.  The first
+ * failure of a call is kept.  Sites (where):
+ *   101-104  prefill index top-k (loads, MMA, epilogue, a sequence with T_b > S_b;
+ *            info0 = sequence, info1 = T_b for 104)
+ *   111      decode index scan / selection (info0 = sequence)
+ *   121      a selection row with an id past the query's block, or not ids-first
+ *            (info0 = query row, info1 = block id)
+ *   131-134  KV-outer attention (loads, MMA, softmax, work items)
+ *   141      dense attention (info0 = sequence with T_b > S_b)
+ *   151-154  query-tile attention (scheduler, loads, MMA, softmax)
+ *   161      paged decode: a page outside the cache or a bad length
+ *   171      index-alignment target / its gradient   181  window selection
+ *   191      main-branch backward
+ * MSA_ERR_TIMEOUT codes come from a bounded wait that ran out (about a
+ * second); the call's results are then not valid, the context still is. */
 msa_status_t msa_get_device_error(void* ws, int32_t* code, int32_t* where, int32_t* info0,
                                   int32_t* info1, void* stream);
 
