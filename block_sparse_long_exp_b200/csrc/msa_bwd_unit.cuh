@@ -27,13 +27,16 @@
 #include <cstring>
 #ifndef __CUDACC__
 #define MSA_BWD_HD inline
+#define MSA_BWD_HD_UNROLL
 #else
 #define MSA_BWD_HD __host__ __device__ __forceinline__
+#define MSA_BWD_HD_UNROLL _Pragma("unroll")
 #endif
 
 namespace msa {
 
 constexpr int kBwdChunk = 64;     // support tokens per chunk
+constexpr int kBwdMaxHeads = 16;  // query heads per group (H / G) the unit code supports
 constexpr int kBwdMaxBlocks = 64; // selected blocks (k <= 32) or dense blocks per pass of the block list
 
 MSA_BWD_HD float bwd_bf16(uint16_t bits) {
@@ -124,24 +127,40 @@ MSA_BWD_HD int64_t bwd_token(const int64_t* first, const int64_t* base, int n, i
 MSA_BWD_HD void bwd_phase1(const BwdUnit& u, int64_t j, int slot, float* dS, uint16_t* kstage, float* dk, float* dv) {
   const uint16_t* kj = u.krow + (j * u.G + u.g) * u.d;
   const uint16_t* vj = u.vrow + (j * u.G + u.g) * u.d;
-  for (int c = 0; c < u.d; ++c) kstage[c] = kj[c];
   float* dkj = dk + (j * u.G + u.g) * u.d;
   float* dvj = dv + (j * u.G + u.g) * u.d;
-  for (int h = 0; h < u.Hg; ++h) {
-    const float* qh = u.qf + h * u.d;
-    const float* doh = u.dof + h * u.d;
-    float s = 0.f, dp = 0.f;
-    for (int c = 0; c < u.d; ++c) {
-      s += qh[c] * bwd_bf16(kj[c]);
-      dp += doh[c] * bwd_bf16(vj[c]);
+  // every head's score and dP, reading the key and value rows once
+  float s[kBwdMaxHeads], dp[kBwdMaxHeads], p[kBwdMaxHeads], ds[kBwdMaxHeads];
+MSA_BWD_HD_UNROLL
+  for (int h = 0; h < kBwdMaxHeads; ++h) s[h] = dp[h] = p[h] = ds[h] = 0.f;
+  for (int c = 0; c < u.d; ++c) {
+    kstage[c] = kj[c];
+    const float kc = bwd_bf16(kj[c]), vc = bwd_bf16(vj[c]);
+MSA_BWD_HD_UNROLL
+    for (int h = 0; h < kBwdMaxHeads; ++h)
+      if (h < u.Hg) {
+        s[h] += u.qf[h * u.d + c] * kc;
+        dp[h] += u.dof[h * u.d + c] * vc;
+      }
+  }
+MSA_BWD_HD_UNROLL
+  for (int h = 0; h < kBwdMaxHeads; ++h)
+    if (h < u.Hg) {
+      p[h] = bwd_exp(u.sm_scale * s[h] - u.lse[h]);
+      ds[h] = p[h] * (dp[h] - u.D[h]);
+      dS[h * kBwdChunk + slot] = ds[h];
     }
-    const float p = bwd_exp(u.sm_scale * s - u.lse[h]);
-    const float ds = p * (dp - u.D[h]);
-    dS[h * kBwdChunk + slot] = ds;
-    for (int c = 0; c < u.d; ++c) {
-      bwd_add(dkj + c, u.sm_scale * ds * qh[c]);
-      bwd_add(dvj + c, p * doh[c]);
-    }
+  // the token's dk / dv rows: one atomic add per element, summed over the heads first
+  for (int c = 0; c < u.d; ++c) {
+    float gk = 0.f, gv = 0.f;
+MSA_BWD_HD_UNROLL
+    for (int h = 0; h < kBwdMaxHeads; ++h)
+      if (h < u.Hg) {
+        gk += ds[h] * u.qf[h * u.d + c];
+        gv += p[h] * u.dof[h * u.d + c];
+      }
+    bwd_add(dkj + c, u.sm_scale * gk);
+    bwd_add(dvj + c, gv);
   }
 }
 
@@ -157,3 +176,4 @@ MSA_BWD_HD float bwd_phase2(const BwdUnit& u, const float* dS, const uint16_t* k
 }  // namespace msa
 
 #undef MSA_BWD_HD
+#undef MSA_BWD_HD_UNROLL

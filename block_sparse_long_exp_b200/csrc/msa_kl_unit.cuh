@@ -27,11 +27,15 @@
 #include <cstring>
 #ifndef __CUDACC__
 #define MSA_KL_HD inline
+#define MSA_KL_HD_UNROLL
 #else
 #define MSA_KL_HD __host__ __device__ __forceinline__
+#define MSA_KL_HD_UNROLL _Pragma("unroll")
 #endif
 
 namespace msa {
+
+constexpr int kKlMaxHeads = 16;   // query heads per group (H / G) the unit code supports
 
 struct KlPartial {
   float A;   // sum of P log P
@@ -110,13 +114,20 @@ MSA_KL_HD void kl_for_tokens(const KlUnit& u, int tid, int nthreads, int* bad, F
     if (first < 0) first += nthreads;
     for (int64_t j = j0 + first; j < j1; j += nthreads) {
       const uint16_t* kj = u.krow + (j * u.G + u.g) * u.d;
-      float pbar = 0.f;
-      for (int h = 0; h < u.Hg; ++h) {
-        const float* qh = u.qf + h * u.d;
-        float s = 0.f;
-        for (int c = 0; c < u.d; ++c) s += qh[c] * kl_bf16(kj[c]);
-        pbar += kl_exp(u.sm_scale * s - u.lse[h]);
+      // every head's score, reading the key row once (kKlMaxHeads sums in registers)
+      float s[kKlMaxHeads];
+MSA_KL_HD_UNROLL
+      for (int h = 0; h < kKlMaxHeads; ++h) s[h] = 0.f;
+      for (int c = 0; c < u.d; ++c) {
+        const float kc = kl_bf16(kj[c]);
+MSA_KL_HD_UNROLL
+        for (int h = 0; h < kKlMaxHeads; ++h)
+          if (h < u.Hg) s[h] += u.qf[h * u.d + c] * kc;
       }
+      float pbar = 0.f;
+MSA_KL_HD_UNROLL
+      for (int h = 0; h < kKlMaxHeads; ++h)
+        if (h < u.Hg) pbar += kl_exp(u.sm_scale * s[h] - u.lse[h]);
       pbar *= 1.f / u.Hg;
       const uint16_t* kij = u.kirow + j * u.d_idx;
       float zs = 0.f;
@@ -187,3 +198,4 @@ MSA_KL_HD void kl_grad_thread(const KlUnit& u, float lse_z, int tid, int nthread
 }  // namespace msa
 
 #undef MSA_KL_HD
+#undef MSA_KL_HD_UNROLL
