@@ -12,6 +12,7 @@
 #include "msa_kl.h"
 #include "msa_window.h"
 #include "msa_bwd.h"
+#include "msa_policy.h"
 
 using namespace msa;
 
@@ -519,6 +520,26 @@ msa_status_t msa_selected_share(const float* lse_sel, const float* lse_all, int6
   if (n < 0) return MSA_ERR_INVALID_ARG;
   if (n > 0 && (!lse_sel || !lse_all || !share)) return MSA_ERR_INVALID_ARG;
   return launch_selected_share(lse_sel, lse_all, n, share, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
+}
+
+msa_status_t msa_index_topk_policy(const msa_shape_t* shape, const msa_varlen_t* seqs, int32_t n_sink,
+                                   int32_t n_local, const void* q_idx, const void* k_idx, int32_t* sel, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  msa_status_t st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  st = check_seqs(seqs);
+  if (st != MSA_OK) return st;
+  if (n_sink < 0 || n_local < 1 || n_sink + n_local > shape->k) return MSA_ERR_INVALID_ARG;
+  if ((int64_t)seqs->max_k_len > (int64_t)8192 * kBk) return MSA_ERR_UNSUPPORTED;   // block scores in shared memory
+  if (seqs->total_q > 0 && (!q_idx || !k_idx || !sel)) return MSA_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, kWsHeader)) return MSA_ERR_WORKSPACE;
+  if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  if (seqs->total_q == 0) return MSA_OK;
+  return launch_policy_select(q_idx, k_idx, seqs->cu_q, seqs->cu_k, seqs->batch, shape->G, shape->d_idx, shape->k,
+                              n_sink, n_local, seqs->total_q, sel, static_cast<DevError*>(ws), stream) == 0
+             ? MSA_OK
+             : MSA_ERR_CUDA;
 }
 
 int32_t msa_set_tile_threshold(int32_t theta) {

@@ -52,7 +52,7 @@ EXPORTED = [
     "msa_get_device_error", "msa_version", "msa_set_tile_threshold",
     "msa_decode_paged_workspace_size", "msa_index_topk_decode_paged", "msa_sparse_attn_decode_paged",
     "msa_index_kl", "msa_index_kl_backward", "msa_select_window", "msa_sparse_attn_backward",
-    "msa_selected_share",
+    "msa_selected_share", "msa_index_topk_policy",
 ]
 
 
@@ -144,6 +144,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_sparse_attn_backward.restype = i32
     lib.msa_selected_share.argtypes = [vp, vp, i64, vp, vp]
     lib.msa_selected_share.restype = i32
+    lib.msa_index_topk_policy.argtypes = [P(Shape), P(Varlen), i32, i32, vp, vp, vp, vp, sz, vp]
+    lib.msa_index_topk_policy.restype = i32
     _lib = lib
     return lib
 
@@ -684,6 +686,31 @@ def msa_sparse_attn_backward(shape: Shape, seqs: Varlen, q: torch.Tensor, k: tor
     if check:
         _device_check(ws, stream, "msa_sparse_attn_backward")
     return dq, dk, dv
+
+
+def msa_index_topk_policy(shape: Shape, seqs: Varlen, q_idx: torch.Tensor, k_idx: torch.Tensor, n_sink: int = 1,
+                          n_local: int = 1, sel: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                          stream=None, check: bool = True) -> torch.Tensor:
+    """Index Branch with n_sink forced first blocks and an n_local-block forced
+    local window, the rest of the k blocks by score; sel int32 [T, G, k] as
+    msa_index_topk (n_sink=0, n_local=1 is its rule)."""
+    lib = load_library()
+    T, S = seqs.total_q, seqs.total_k
+    _arg("q_idx", q_idx, torch.bfloat16, (T, shape.G, shape.d_idx))
+    _arg("k_idx", k_idx, torch.bfloat16, (S, shape.d_idx))
+    _arg("sel", sel, torch.int32, (T, shape.G, shape.k), optional=True)
+    _ws_arg(ws)
+    _require_cuda(q_idx, k_idx, sel, ws)
+    if sel is None:
+        sel = torch.empty((T, shape.G, shape.k), dtype=torch.int32, device=q_idx.device)
+    if ws is None:
+        ws = _workspace(256, q_idx.device)
+    rc = lib.msa_index_topk_policy(ctypes.byref(shape), ctypes.byref(seqs), int(n_sink), int(n_local), _ptr(q_idx),
+                                   _ptr(k_idx), _ptr(sel), _ptr(ws), _nbytes(ws), _stream(stream))
+    _check(rc, "msa_index_topk_policy")
+    if check:
+        _device_check(ws, stream, "msa_index_topk_policy")
+    return sel
 
 
 def msa_selected_share(lse_sel: torch.Tensor, lse_all: torch.Tensor, stream=None) -> torch.Tensor:

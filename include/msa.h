@@ -247,6 +247,19 @@ msa_status_t msa_select_window(const msa_shape_t* shape, const msa_varlen_t* seq
                                int32_t* sel, /* device int32 [T, G, k] (out) */
                                void* ws, size_t ws_bytes, void* stream);
 
+/* The Index Branch under the scored selection policies the pages compare the
+ * final rule with (pnsm.cn sec. 3 and its forced sink / local ablation;
+ * yhxrc.cn sec. 二): blocks 0 .. n_sink-1 and the n_local most recent ones
+ * (the query's own included) are forced, the rest of the k by block score
+ * (score desc, id asc; NaN as -inf); every causal block when there are at
+ * most k.  n_sink = 0, n_local = 1 is msa_index_topk's rule.  Requires
+ * n_sink >= 0, n_local >= 1, n_sink + n_local <= k, max_k_len <= 1M tokens.
+ * sel as msa_index_topk; ws: at least 256 bytes, 256-byte aligned.  A first,
+ * CUDA-core form (one CTA per (query, group)). */
+msa_status_t msa_index_topk_policy(const msa_shape_t* shape, const msa_varlen_t* seqs, int32_t n_sink,
+                                   int32_t n_local, const void* q_idx, const void* k_idx, int32_t* sel, void* ws,
+                                   size_t ws_bytes, void* stream);
+
 /* The share of each head's dense causal attention weight that the selected
  * tokens hold, the monitor the pages report for the selection (yhxrc.cn sec.
  * 二): share[i] = exp(lse_sel[i] - lse_all[i]), with lse_sel from
@@ -404,7 +417,7 @@ msa_status_t msa_profile_read(const char* kernel, double* total_ms, int64_t* cou
  *   151-154  query-tile attention (scheduler, loads, MMA, softmax)
  *   161      paged decode: a page outside the cache or a bad length
  *   171      index-alignment target / its gradient   181  window selection
- *   191      main-branch backward
+ *   191      main-branch backward                      201  policy selection
  * MSA_ERR_TIMEOUT codes come from a bounded wait that ran out (about a
  * second); the call's results are then not valid, the context still is. */
 msa_status_t msa_get_device_error(void* ws, int32_t* code, int32_t* where, int32_t* info0,
