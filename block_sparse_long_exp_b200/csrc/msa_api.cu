@@ -13,6 +13,7 @@
 #include "msa_window.h"
 #include "msa_bwd.h"
 #include "msa_policy.h"
+#include "msa_gather.h"
 
 using namespace msa;
 
@@ -538,6 +539,27 @@ msa_status_t msa_index_topk_policy(const msa_shape_t* shape, const msa_varlen_t*
   if (seqs->total_q == 0) return MSA_OK;
   return launch_policy_select(q_idx, k_idx, seqs->cu_q, seqs->cu_k, seqs->batch, shape->G, shape->d_idx, shape->k,
                               n_sink, n_local, seqs->total_q, sel, static_cast<DevError*>(ws), stream) == 0
+             ? MSA_OK
+             : MSA_ERR_CUDA;
+}
+
+msa_status_t msa_gather_pages(const msa_varlen_t* seqs, const int32_t* block_table, int32_t max_blocks,
+                              int64_t num_pages, int64_t row_bytes, const void* pages, void* packed, void* ws,
+                              size_t ws_bytes, void* stream) {
+  if (seqs == nullptr || seqs->cu_k == nullptr || seqs->batch < 1 || seqs->max_k_len < 0 || seqs->total_k < 0)
+    return MSA_ERR_INVALID_ARG;
+  if (block_table == nullptr || max_blocks < 1 || num_pages < 1) return MSA_ERR_INVALID_ARG;
+  if ((int64_t)seqs->max_k_len > (int64_t)max_blocks * kBk) return MSA_ERR_INVALID_ARG;
+  if (row_bytes <= 0 || row_bytes % 16 != 0) return MSA_ERR_INVALID_ARG;
+  if (seqs->total_k > 0 &&
+      (!pages || !packed || ((reinterpret_cast<uintptr_t>(pages) | reinterpret_cast<uintptr_t>(packed)) & 15u)))
+    return MSA_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, kWsHeader)) return MSA_ERR_WORKSPACE;
+  if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  if (seqs->total_k == 0) return MSA_OK;
+  return launch_gather_pages(seqs->cu_k, seqs->batch, seqs->max_k_len, block_table, max_blocks, num_pages, row_bytes,
+                             pages, packed, static_cast<DevError*>(ws), stream) == 0
              ? MSA_OK
              : MSA_ERR_CUDA;
 }

@@ -52,7 +52,7 @@ EXPORTED = [
     "msa_get_device_error", "msa_version", "msa_set_tile_threshold",
     "msa_decode_paged_workspace_size", "msa_index_topk_decode_paged", "msa_sparse_attn_decode_paged",
     "msa_index_kl", "msa_index_kl_backward", "msa_select_window", "msa_sparse_attn_backward",
-    "msa_selected_share", "msa_index_topk_policy",
+    "msa_selected_share", "msa_index_topk_policy", "msa_gather_pages",
 ]
 
 
@@ -146,6 +146,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_selected_share.restype = i32
     lib.msa_index_topk_policy.argtypes = [P(Shape), P(Varlen), i32, i32, vp, vp, vp, vp, sz, vp]
     lib.msa_index_topk_policy.restype = i32
+    lib.msa_gather_pages.argtypes = [P(Varlen), vp, i32, i64, i64, vp, vp, vp, sz, vp]
+    lib.msa_gather_pages.restype = i32
     _lib = lib
     return lib
 
@@ -711,6 +713,53 @@ def msa_index_topk_policy(shape: Shape, seqs: Varlen, q_idx: torch.Tensor, k_idx
     if check:
         _device_check(ws, stream, "msa_index_topk_policy")
     return sel
+
+
+def _table_arg(seqs: Varlen, block_table: torch.Tensor) -> int:
+    """Checks a block table [batch, max_blocks] int32; returns max_blocks."""
+    if not isinstance(block_table, torch.Tensor) or block_table.dim() != 2:
+        raise MsaError("block_table: expected a 2-D int32 tensor [batch, max_blocks]")
+    _arg("block_table", block_table, torch.int32)
+    if block_table.shape[0] != seqs.batch:
+        raise MsaError(f"block_table: {block_table.shape[0]} rows for {seqs.batch} sequences")
+    return int(block_table.shape[1])
+
+
+def msa_gather_pages(seqs: Varlen, block_table: torch.Tensor, num_pages: int, pages: torch.Tensor,
+                     ws: Optional[torch.Tensor] = None, stream=None, check: bool = True) -> torch.Tensor:
+    """Rows of a paged cache (pages [num_pages * B_k, ...]) gathered into packed
+    rows [total_k, ...] of the sequences seqs describes (cu_k: lengths)."""
+    lib = load_library()
+    max_blocks = _table_arg(seqs, block_table)
+    if not isinstance(pages, torch.Tensor) or pages.dim() < 1 or pages.shape[0] != int(num_pages) * 128:
+        raise MsaError("pages: expected a tensor of num_pages * 128 rows")
+    _arg("pages", pages, pages.dtype)
+    row_bytes = pages[0].numel() * pages.element_size() if pages.shape[0] else 0
+    packed = torch.empty((seqs.total_k,) + tuple(pages.shape[1:]), dtype=pages.dtype, device=pages.device)
+    _ws_arg(ws)
+    _require_cuda(block_table, pages, ws)
+    if ws is None:
+        ws = _workspace(256, pages.device)
+    rc = lib.msa_gather_pages(ctypes.byref(seqs), _ptr(block_table), max_blocks, int(num_pages), int(row_bytes),
+                              _ptr(pages), _ptr(packed), _ptr(ws), _nbytes(ws), _stream(stream))
+    _check(rc, "msa_gather_pages")
+    if check:
+        _device_check(ws, stream, "msa_gather_pages")
+    return packed
+
+
+def msa_prefill_paged(shape: Shape, seqs: Varlen, block_table: torch.Tensor, num_pages: int, q: torch.Tensor,
+                      q_idx: torch.Tensor, k_idx_pages: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                      q_chunk: int = 0, stream=None):
+    """A prefill (or a chunk of one) over a paged cache: the pages gathered into
+    packed rows, then msa_index_topk and msa_sparse_attn_prefill.  Returns
+    (sel, out, lse)."""
+    k_idx = msa_gather_pages(seqs, block_table, num_pages, k_idx_pages, stream=stream)
+    k = msa_gather_pages(seqs, block_table, num_pages, k_pages, stream=stream)
+    v = msa_gather_pages(seqs, block_table, num_pages, v_pages, stream=stream)
+    sel = msa_index_topk(shape, seqs, q_idx, k_idx, stream=stream)
+    out, lse = msa_sparse_attn_prefill(shape, seqs, q, k, v, sel, q_chunk=q_chunk, stream=stream)
+    return sel, out, lse
 
 
 def msa_selected_share(lse_sel: torch.Tensor, lse_all: torch.Tensor, stream=None) -> torch.Tensor:

@@ -209,6 +209,22 @@ msa_status_t msa_sparse_attn_decode_paged(const msa_shape_t* shape, const msa_pa
                                           void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Prefill (or a chunk of one) over a paged KV cache: gather the pages into
+ * packed rows, then run the packed calls.  Packed row cu_k[b] + j of sequence
+ * b is row (p * B_k + j mod B_k) of `pages`, p = block_table[b * max_blocks +
+ * j / B_k]; rows are row_bytes each (a multiple of 16; index keys: d_idx * 2,
+ * keys or values: G * d * 2).  seqs gives the lengths (cu_k, max_k_len <=
+ * max_blocks * B_k); pages holds num_pages * B_k rows and packed total_k rows,
+ * both 16-byte aligned.  A page outside [0, num_pages) is recorded as
+ * MSA_ERR_DEVICE_CHECK and its rows are written as zeros.  ws: at least 256
+ * bytes, 256-byte aligned.  The gather is one extra pass over the rows (HBM
+ * bound); the results of the packed calls on its output are those of the
+ * same calls on the same tokens stored packed. */
+msa_status_t msa_gather_pages(const msa_varlen_t* seqs, const int32_t* block_table, int32_t max_blocks,
+                              int64_t num_pages, int64_t row_bytes, const void* pages, void* packed, void* ws,
+                              size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* Main Branch backward: the gradients of the attention over the support J
  * (the selected blocks' tokens cut at the query, or with dense != 0 every
  * token up to it) for an upstream gradient dout.  With P_j = exp(sm_scale
@@ -418,6 +434,7 @@ msa_status_t msa_profile_read(const char* kernel, double* total_ms, int64_t* cou
  *   161      paged decode: a page outside the cache or a bad length
  *   171      index-alignment target / its gradient   181  window selection
  *   191      main-branch backward                      201  policy selection
+ *   211      page gather (info0 = sequence, info1 = block)
  * MSA_ERR_TIMEOUT codes come from a bounded wait that ran out (about a
  * second); the call's results are then not valid, the context still is. */
 msa_status_t msa_get_device_error(void* ws, int32_t* code, int32_t* where, int32_t* info0,

@@ -184,3 +184,16 @@ def test_selected_share_host_checks(lib):
     assert lib.msa_selected_share(None, None, 0, None, None) == 0       # nothing to do
     assert lib.msa_selected_share(None, 256, 5, 256, None) == 1
     assert lib.msa_selected_share(256, 256, -1, 256, None) == 1
+
+
+def test_gather_pages_host_checks(lib):
+    from block_sparse_long_exp_b200 import msa
+    cu = (ctypes.c_int32 * 2)(0, 0)
+    table = (ctypes.c_int32 * 8)(*range(8))
+    seqs = msa.Varlen(1, 900, 900, 0, 900, 900, ctypes.addressof(cu), ctypes.addressof(cu))
+    T = ctypes.addressof(table)
+    assert lib.msa_gather_pages(ctypes.byref(seqs), None, 8, 8, 128, 256, 256, 256, 1 << 20, None) == 1  # no table
+    assert lib.msa_gather_pages(ctypes.byref(seqs), T, 7, 8, 128, 256, 256, 256, 1 << 20, None) == 1     # 900 > 7 * 128
+    assert lib.msa_gather_pages(ctypes.byref(seqs), T, 8, 8, 100, 256, 256, 256, 1 << 20, None) == 1     # row bytes
+    assert lib.msa_gather_pages(ctypes.byref(seqs), T, 8, 8, 128, 258, 256, 256, 1 << 20, None) == 1     # alignment
+    assert lib.msa_gather_pages(ctypes.byref(seqs), T, 8, 8, 128, 256, 256, 256, 16, None) == 3          # workspace

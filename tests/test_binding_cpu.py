@@ -161,3 +161,17 @@ def test_backward_checks_its_tensors(M):
         M.msa_sparse_attn_backward(shape, s, q, kv, kv, None, q, lse, q)
     with pytest.raises(M.MsaError, match="CUDA"):
         M.msa_sparse_attn_backward(shape, s, q, kv, kv, None, q, lse, q, dense=True)
+
+
+def test_gather_pages_checks_its_tensors(M):
+    s = _seqs(M, 10, 300)
+    table = torch.zeros(1, 3, dtype=torch.int32)
+    pages = torch.zeros(4 * 128, G, d, dtype=torch.bfloat16)
+    with pytest.raises(M.MsaError, match="block_table"):
+        M.msa_gather_pages(s, table[0], 4, pages)
+    with pytest.raises(M.MsaError, match="2 rows for 1"):
+        M.msa_gather_pages(s, torch.zeros(2, 3, dtype=torch.int32), 4, pages)
+    with pytest.raises(M.MsaError, match="num_pages"):
+        M.msa_gather_pages(s, table, 5, pages)
+    with pytest.raises(M.MsaError, match="CUDA"):
+        M.msa_gather_pages(s, table, 4, pages)
