@@ -41,11 +41,9 @@ def exe(tmp_path_factory):
     return out
 
 
-@pytest.mark.parametrize("dense", [False, True])
-def test_kl_unit_matches_the_oracle(exe, tmp_path, dense):
-    rng = np.random.default_rng(31)
-    H, G, d, d_idx, k, B_k = 8, 2, 64, 32, 4, 128
-    S_lens, T_lens = [700, 129, 1000], [700, 5, 300]
+def _replay(exe, tmp_path, dense, seed, H, G, d, d_idx, k, S_lens, T_lens):
+    B_k = 128
+    rng = np.random.default_rng(seed)
     cu_k = np.concatenate([[0], np.cumsum(S_lens)]).astype(np.int32)
     cu_q = np.concatenate([[0], np.cumsum(T_lens)]).astype(np.int32)
     T, S = int(cu_q[-1]), int(cu_k[-1])
@@ -57,7 +55,8 @@ def test_kl_unit_matches_the_oracle(exe, tmp_path, dense):
     sm, tau = d ** -0.5, 0.125
     rows = list(range(T))
     if dense:
-        every = np.tile(np.arange(16, dtype=np.int32)[None, None, :], (T, G, 1))
+        n_blk = (max(S_lens) + B_k - 1) // B_k
+        every = np.tile(np.arange(n_blk, dtype=np.int32)[None, None, :], (T, G, 1))
         _, lse = O.msa_forward_rows(q, kk, np.zeros_like(kk), every, cu_q, cu_k, rows, B_k, sm)
     else:
         _, lse = O.msa_forward_rows(q, kk, np.zeros_like(kk), sel, cu_q, cu_k, rows, B_k, sm)
@@ -89,3 +88,18 @@ def test_kl_unit_matches_the_oracle(exe, tmp_path, dense):
         scale = np.abs(want_dq).max()
         np.testing.assert_allclose(got_dq[cta], want_dq, rtol=0, atol=2e-4 * scale)
         np.testing.assert_allclose(got_dk[cta], want_dk, rtol=0, atol=2e-4 * np.abs(want_dk).max())
+
+
+@pytest.mark.parametrize("dense", [False, True])
+def test_kl_unit_matches_the_oracle(exe, tmp_path, dense):
+    _replay(exe, tmp_path, dense, 31, 8, 2, 64, 32, 4, [700, 129, 1000], [700, 5, 300])
+
+
+# The largest group the kernels take (16 heads) with d = d_idx = 128, and a
+# group of 4 heads whose support is the query's own block alone (k = 1).
+@pytest.mark.parametrize("H,G,d,d_idx,k,S_lens,T_lens", [
+    (32, 2, 128, 128, 8, [1100, 70], [180, 70]),
+    (4, 1, 64, 64, 1, [334, 500], [166, 257]),
+])
+def test_kl_unit_other_shapes(exe, tmp_path, H, G, d, d_idx, k, S_lens, T_lens):
+    _replay(exe, tmp_path, False, 33, H, G, d, d_idx, k, S_lens, T_lens)

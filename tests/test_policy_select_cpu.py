@@ -32,11 +32,9 @@ def exe(tmp_path_factory):
     return out
 
 
-@pytest.mark.parametrize("n_sink,n_local", [(0, 1), (1, 1), (2, 3), (1, 7), (0, 4)])
-def test_policy_matches_the_oracle(exe, tmp_path, n_sink, n_local):
-    rng = np.random.default_rng(17)
-    G, d_idx, k, B_k = 2, 32, 8, 128
-    S_lens, T_lens = [2500, 129, 1400], [700, 129, 300]
+def _replay(exe, tmp_path, seed, G, d_idx, k, S_lens, T_lens, n_sink, n_local):
+    B_k = 128
+    rng = np.random.default_rng(seed)
     cu_k = np.concatenate([[0], np.cumsum(S_lens)]).astype(np.int32)
     cu_q = np.concatenate([[0], np.cumsum(T_lens)]).astype(np.int32)
     T, S = int(cu_q[-1]), int(cu_k[-1])
@@ -58,6 +56,19 @@ def test_policy_matches_the_oracle(exe, tmp_path, n_sink, n_local):
     np.testing.assert_array_equal(got, want)
     if (n_sink, n_local) == (0, 1):
         np.testing.assert_array_equal(got, O.index_topk(q_idx, k_idx, cu_q.tolist(), cu_k.tolist(), k, B_k))
+
+
+@pytest.mark.parametrize("n_sink,n_local", [(0, 1), (1, 1), (2, 3), (1, 7), (0, 4)])
+def test_policy_matches_the_oracle(exe, tmp_path, n_sink, n_local):
+    _replay(exe, tmp_path, 17, 2, 32, 8, [2500, 129, 1400], [700, 129, 300], n_sink, n_local)
+
+
+# d_idx = 128 (the widest index row the kernel takes) with k = 1, where only the
+# forced block can be chosen, and k = 32 (the largest k it takes) over a
+# sequence of 47 blocks, so that scores still decide.
+@pytest.mark.parametrize("G,d_idx,k,n_sink,n_local", [(1, 128, 1, 0, 1), (2, 128, 32, 0, 1), (2, 64, 32, 4, 8)])
+def test_policy_other_shapes(exe, tmp_path, G, d_idx, k, n_sink, n_local):
+    _replay(exe, tmp_path, 19, G, d_idx, k, [6000, 300], [200, 300], n_sink, n_local)
 
 
 def test_policy_entry_point_host_checks():
