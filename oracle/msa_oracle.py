@@ -53,7 +53,6 @@ routine); see ``tests/test_oracle_pins.py``.
 """
 from __future__ import annotations
 
-import math
 from typing import Dict, List, Sequence, Tuple
 
 import numpy as np

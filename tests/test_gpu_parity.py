@@ -2,7 +2,6 @@
 sizes the oracle finishes in seconds: every row compared, several 128-query
 tiles and ragged tails.  Selections must match exactly; outputs within
 max-abs 2e-2 and mean-relative 5e-3 of fp64."""
-import math
 
 import numpy as np
 import pytest
