@@ -9,10 +9,16 @@ stays sharded; the keys [0, b_r) must be present on rank r.
 The work per query grows with its position (the index branch scores every
 earlier block), so equal row counts would leave the last rank the most work:
 the ranges are cut at equal shares of the algorithmic work instead.
+
+The backward of such a split has one exchange step.  Rank r's chunk reaches
+the keys [0, b_r), so its dk, dv (and the index-alignment target's dk_idx)
+hold only its own queries' contributions to those rows.  The layer's key-side
+gradients are the sum of these over the ranks (sum_key_grads).  dq and dq_idx
+stay sharded with the queries, as the output does.
 """
 from __future__ import annotations
 
-from typing import Dict, List, Tuple
+from typing import Dict, List, Sequence, Tuple
 
 import numpy as np
 
@@ -58,6 +64,37 @@ def chunk_of(inp: Dict[str, object], a: int, b: int) -> Dict[str, object]:
         "cu_k": torch.tensor([0, b], dtype=torch.int32, device=dev),
         "cu_q_host": [0, b - a], "cu_k_host": [0, b],
     }
+
+
+def sum_key_grads(grads: Sequence[object], S: int, group=None) -> List[object]:
+    """Key-side gradients of a query-range split summed over the ranks.
+
+    grads: this rank's tensors [b_r, ...] (dk, dv, dk_idx: rows 0 .. b_r-1 of
+    the sequence's keys, the rows its chunk reaches).  Each is placed in a zero
+    tensor [S, ...]; all of them are summed across the process group by one
+    all-reduce over a flat buffer (NCCL on the GPUs, gloo on the host); without
+    an initialised group the padded tensors are returned as they are.  Returns
+    the [S, ...] sums, equal on every rank."""
+    import torch
+    import torch.distributed as dist
+    full = []
+    for g in grads:
+        if g.dim() < 1 or g.shape[0] > S:
+            raise ValueError(f"a key-side gradient has {g.shape[0] if g.dim() else 0} rows, more than S = {S}")
+        t = torch.zeros((S,) + tuple(g.shape[1:]), dtype=g.dtype, device=g.device)
+        t[:g.shape[0]] = g
+        full.append(t)
+    if not (dist.is_available() and dist.is_initialized()) or not full:
+        return full
+    if len({(t.dtype, t.device) for t in full}) != 1:
+        raise ValueError("the key-side gradients must share one dtype and device")
+    flat = torch.cat([t.reshape(-1) for t in full])
+    dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+    out, at = [], 0
+    for t in full:
+        out.append(flat[at:at + t.numel()].view(t.shape))
+        at += t.numel()
+    return out
 
 
 def imbalance(work: np.ndarray, ranges: List[Tuple[int, int]]) -> float:

@@ -2,7 +2,10 @@
 shard.py): the planner's ranges cover every query once and balance the
 algorithmic work; and on two gloo ranks, each rank's chunked-prefill oracle
 result (queries [a, b) over keys [0, b)) gathered on rank 0 equals the
-unsharded oracle result row for row."""
+unsharded oracle result row for row; and the backward of the split: each
+rank's key-side gradients (dk, dv, the KL target's dk_idx) summed over the
+ranks by sum_key_grads, with the query-side ones (dq, dq_idx) gathered, equal
+the unsharded backward oracles."""
 import os
 import socket
 
@@ -84,6 +87,74 @@ def test_sharded_oracle_equals_unsharded_on_two_gloo_ranks():
         p.join(timeout=300)
     assert all(p.exitcode == 0 for p in procs)
     assert result.get(timeout=10) is True
+
+
+def _rank_bwd(rank, world, port, result):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from block_sparse_long_exp_b200 import workloads as W
+        from oracle import index_kl as K
+        from oracle import main_backward as B
+        from oracle import msa_oracle as O
+        w = W.Workload("shard_bwd", "prefill", H=8, G=2, d=16, d_idx=8, B_k=4, k=3, seed=7, hot_frac=0.1)
+        S, tau = 61, 0.5
+        inp = W.make_inputs(w, "cpu", lengths=[S])
+        dout = torch.randn(inp["q"].shape, generator=torch.Generator().manual_seed(8), dtype=torch.float64)
+        work = SH.query_work(S, w.H, w.G, w.d, w.d_idx, w.B_k, w.k)
+        a, b = SH.split_query_ranges(work, world)[rank]
+        c = SH.chunk_of(inp, a, b)
+        f = lambda t: t.double().numpy()  # noqa: E731
+        cq, ck = c["cu_q_host"], c["cu_k_host"]
+        sel = O.index_topk(f(c["q_idx"]), f(c["k_idx"]), cq, ck, w.k, w.B_k)
+        dq, dk, dv = B.main_branch_backward(f(c["q"]), f(c["k"]), f(c["v"]), sel, dout[a:b].numpy(), cq, ck,
+                                            w.B_k, w.sm_scale)
+        loss, dqi, dki = K.index_kl_loss_and_grad(f(c["q"]), f(c["k"]), f(c["q_idx"]), f(c["k_idx"]), sel, cq, ck,
+                                                  w.B_k, w.sm_scale, tau)
+        assert dk.shape[0] == b and dki.shape[0] == b
+        loss_t = torch.tensor([loss], dtype=torch.float64)
+        dist.all_reduce(loss_t)
+        sk, sv, ski = SH.sum_key_grads([torch.from_numpy(dk), torch.from_numpy(dv), torch.from_numpy(dki)], S)
+        parts = [None] * world
+        dist.all_gather_object(parts, (a, b, dq, dqi))
+        if rank == 0:
+            fi = {k_: f(inp[k_]) for k_ in ("q", "k", "v", "q_idx", "k_idx")}
+            full_sel = O.index_topk(fi["q_idx"], fi["k_idx"], [0, S], [0, S], w.k, w.B_k)
+            w_dq, w_dk, w_dv = B.main_branch_backward(fi["q"], fi["k"], fi["v"], full_sel, dout.numpy(), [0, S],
+                                                      [0, S], w.B_k, w.sm_scale)
+            w_loss, w_dqi, w_dki = K.index_kl_loss_and_grad(fi["q"], fi["k"], fi["q_idx"], fi["k_idx"], full_sel,
+                                                            [0, S], [0, S], w.B_k, w.sm_scale, tau)
+            close = lambda x, y: np.allclose(x, y, rtol=0, atol=1e-12 * max(1.0, np.abs(y).max()))  # noqa: E731
+            ok = all(close(x.numpy(), y) for x, y in ((sk, w_dk), (sv, w_dv), (ski, w_dki)))
+            ok = ok and abs(float(loss_t[0]) - w_loss) <= 1e-12 * max(1.0, abs(w_loss))
+            for a_, b_, dq_, dqi_ in parts:
+                ok = ok and close(dq_, w_dq[a_:b_]) and close(dqi_, w_dqi[a_:b_])
+            # the exchange is needed: the later rank's queries reach rank 0's key rows too
+            ok = ok and not np.allclose(dk, w_dk[:b]) and not np.allclose(dki, w_dki[:b])
+            result.put(bool(ok))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_backward_sums_key_grads_on_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    result = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_bwd, args=(r, 2, port, result)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+    assert all(p.exitcode == 0 for p in procs)
+    assert result.get(timeout=10) is True
+
+
+def test_sum_key_grads_without_a_group_pads():
+    g = torch.arange(6, dtype=torch.float32).reshape(3, 2)
+    (out,) = SH.sum_key_grads([g], 5)
+    assert out.shape == (5, 2) and torch.equal(out[:3], g) and not out[3:].any()
+    with pytest.raises(ValueError):
+        SH.sum_key_grads([torch.zeros(6, 2)], 5)
 
 
 def test_decode_shards_cover_and_balance():
