@@ -185,6 +185,58 @@ def step_decode(ctx, msa):
                                out=ctx["out"], want_lse=False, ws=ctx["ws_att"], check=False)
 
 
+def training_leg(args, w, W, R, msa, torch, device="cuda"):
+    """The training-side kernels on one prefill layer of args.training_T tokens
+    with the workload's heads and dimensions: the Main Branch backward for a
+    seeded upstream gradient, then the KL target (tau = 0.125) and its
+    gradient, fed by the forward's selection and log-sum-exps.  Each kernel is
+    timed by the library's CUDA events on its launching stream over args.steps
+    passes after args.warmup (inputs larger than L2).  They run on the CUDA
+    cores, so the roofline is the fp32 FMA rate."""
+    tinp = W.make_inputs(w, device, T_override=args.training_T)
+    shape = msa.make_shape(w.H, w.G, w.d, w.d_idx, w.k)
+    seqs = msa.make_varlen(tinp["cu_q"], tinp["cu_k"], tinp["cu_q_host"], tinp["cu_k_host"])
+    q, k, v, q_idx, k_idx = (tinp[n] for n in ("q", "k", "v", "q_idx", "k_idx"))
+    sel = msa.msa_index_topk(shape, seqs, q_idx, k_idx)
+    out, lse = msa.msa_sparse_attn_prefill(shape, seqs, q, k, v, sel)
+    gen = torch.Generator(device=q.device).manual_seed(w.seed + 1000)
+    dout = torch.randn(tuple(q.shape), generator=gen, device=q.device).to(torch.bfloat16)
+    tau = 0.125
+
+    def one(check):
+        msa.msa_sparse_attn_backward(shape, seqs, q, k, v, sel, out, lse, dout, check=check)
+        _, lse_z = msa.msa_index_kl(shape, seqs, q, k, q_idx, k_idx, sel, lse, tau, want_lse_z=True, check=check)
+        msa.msa_index_kl_backward(shape, seqs, q, k, q_idx, k_idx, sel, lse, lse_z, tau, check=check)
+
+    one(True)
+    for _ in range(args.warmup):
+        one(False)
+    torch.cuda.synchronize()
+    msa.msa_profile_reset()
+    msa.msa_profile_enable(True)
+    for _ in range(args.steps):
+        one(False)
+    torch.cuda.synchronize()
+    msa.msa_profile_enable(False)
+    one(True)                                 # device checks after the timed passes
+    S_lens = [tinp["cu_k_host"][i + 1] - tinp["cu_k_host"][i] for i in range(len(tinp["cu_k_host"]) - 1)]
+    T_lens = [tinp["cu_q_host"][i + 1] - tinp["cu_q_host"][i] for i in range(len(tinp["cu_q_host"]) - 1)]
+    tw = R.training_work(S_lens, T_lens, w.H, w.G, w.d, w.d_idx, w.B_k, w.k)
+    peak = R.alu_fp32_tflops()
+    res = {"workload": f"{args.workload} at T = {sum(T_lens)}", "T": sum(T_lens), "tau": tau,
+           "steps": args.steps, "warmup": args.warmup, "peak": peak, "unit": "TFLOP/s",
+           "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOPs x 1965 MHz (CUDA cores, nominal)",
+           "kernels": {}}
+    for name, key in (("attn_bwd", "backward_flops"), ("index_kl", "kl_flops"), ("index_kl_grad", "kl_grad_flops")):
+        kms, n = msa.msa_profile_read(name)
+        if n:
+            per = kms / n
+            ach = tw[key] / (per / 1000.0) / 1e12
+            res["kernels"][name] = {"ms_per_launch": per, "launches": n, "flops_per_launch": tw[key],
+                                    "bound": "alu", "achieved": ach, "frac": ach / peak}
+    return res
+
+
 def device_errors(ctx, msa):
     for key in ("ws_idx", "ws_att"):
         code, where, i0, i1 = msa.msa_get_device_error(ctx[key])
@@ -589,6 +641,10 @@ def run_ours(args):
                   "kernels": dk}
         del dctx, dinp
         torch.cuda.empty_cache()
+    training = None
+    if rank == 0 and args.training:
+        training = training_leg(args, w, W, R, msa, torch)
+        torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, n_rows, secs = cpu_oracle_rate(w, inp, args.cpu_budget, torch, np)
         cores = blas_threads() or len(os.sched_getaffinity(0))
@@ -605,6 +661,8 @@ def run_ours(args):
                 "roofline": roof, "step_roofline": step_roof, "tile_split": split, "dense_gqa": dense,
                 "decode": decode, "e2e": e2e,
                 "cpu_baseline": cpu, "clocks": clk, "gpu_launches": launches, "kernels": kernels}
+        if training is not None:
+            line["training"] = training
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
@@ -630,6 +688,9 @@ def build_parser():
                     help="query-tile threshold of the prefill (-1 automatic, 0 off)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--training", action="store_true",
+                    help="also time the backward and KL kernels (CUDA cores) on a --training-T layer")
+    ap.add_argument("--training-T", type=int, default=32768)
     ap.add_argument("--shard", choices=["none", "queries"], default="none",
                     help="N > 1: independent layers per rank (none, weak scaling) or the query ranges of one "
                          "layer split across ranks (queries, strong scaling)")

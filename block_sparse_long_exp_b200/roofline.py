@@ -11,6 +11,12 @@ lists, block scores) are excluded.
 * prefill bytes: q, k, v, q_idx, k_idx read once and the output written once.
 * decode bytes: the whole index-key cache once, plus the K and V rows of the
   selected blocks, plus q / q_idx / out.
+* training kernels, over the same supports (att(t) keys per query and head):
+  backward 10 * d per (query, head, key) (S = q.k, dP = dO.v, dq += dS k,
+  dk += dS q, dv += P dO: 2.5x the main FLOPs); the KL target 2 * d per head
+  score plus 2 * d_idx for the index score per (query, group, key); its
+  gradient that plus 4 * d_idx (dq_idx and dk_idx).  Exponentials and
+  logarithms are not counted.
 """
 from __future__ import annotations
 
@@ -67,6 +73,23 @@ def prefill_work(S_lens: Sequence[int], T_lens: Sequence[int], H: int, G: int, d
     nbytes = 2 * (T_tot * H * d + 2 * S_tot * G * d + T_tot * G * d_idx + S_tot * d_idx + T_tot * H * d)
     return {"index_flops": float(idx), "main_flops": float(main), "flops": float(idx + main),
             "bytes": float(nbytes)}
+
+
+def training_work(S_lens: Sequence[int], T_lens: Sequence[int], H: int, G: int, d: int, d_idx: int,
+                  B_k: int, k: int) -> Dict[str, float]:
+    """FLOPs of the Main Branch backward and of the KL target and its gradient
+    over the selected supports of a prefill layer."""
+    main = prefill_work(S_lens, T_lens, H, G, d, d_idx, B_k, k)["main_flops"]
+    pairs = main / (4 * H * d)            # attended (query, key) pairs of one head
+    return {"pairs": pairs, "backward_flops": 10.0 * H * d * pairs,
+            "kl_flops": pairs * (2.0 * H * d + 2.0 * G * d_idx),
+            "kl_grad_flops": pairs * (2.0 * H * d + 6.0 * G * d_idx)}
+
+
+def alu_fp32_tflops(sms: int = 148, lanes: int = 128, mhz: float = 1965.0) -> float:
+    """Peak fp32 FMA rate of the CUDA cores (two FLOPs per lane per clock):
+    B200 has 148 SMs of 128 fp32 lanes, clocks.max.sm 1965 MHz: 74.4 TFLOP/s."""
+    return sms * lanes * 2.0 * mhz * 1e6 / 1e12
 
 
 def dense_work(S_lens: Sequence[int], T_lens: Sequence[int], H: int, d: int) -> float:

@@ -91,3 +91,35 @@ def test_pages_compute_ratio_at_1m():
     assert dense / (w128["index_flops"] + w128["main_flops"]) == pytest.approx(28.4, rel=1e-2)
     w64 = R.prefill_work([N], [N], 64, 4, 128, 64, 128, 16)
     assert dense / (w64["index_flops"] + w64["main_flops"]) == pytest.approx(51.5, rel=1e-2)
+
+
+def test_training_flops_follow_the_oracle_selection():
+    # per attended (query, head, key): 10 d for the backward; per (query, group,
+    # key): 2 d per head of the group and 2 d_idx for the KL, 4 d_idx more for
+    # its gradient; the key sets are the oracle's selected token sets
+    rng = np.random.default_rng(6)
+    H, G, d, d_idx, B_k, k = 6, 2, 8, 5, 4, 2
+    S_lens, T_lens = [30, 7, 19], [30, 7, 4]
+    cu_k = np.concatenate([[0], np.cumsum(S_lens)]).tolist()
+    cu_q = np.concatenate([[0], np.cumsum(T_lens)]).tolist()
+    q_idx = rng.integers(-2, 3, size=(cu_q[-1], G, d_idx)).astype(np.float64)
+    k_idx = rng.integers(-2, 3, size=(cu_k[-1], d_idx)).astype(np.float64)
+    sel = O.index_topk(q_idx, k_idx, cu_q, cu_k, k, B_k)
+    bwd = kl = klg = 0
+    for b in range(len(S_lens)):
+        for i, pos in enumerate(O.query_positions(T_lens[b], S_lens[b])):
+            t = cu_q[b] + i
+            for g in range(G):
+                n = len(O.selected_token_set([int(x) for x in sel[t, g]], int(pos), B_k))
+                bwd += 10 * d * (H // G) * n
+                kl += n * (2 * d * (H // G) + 2 * d_idx)
+                klg += n * (2 * d * (H // G) + 6 * d_idx)
+    tw = R.training_work(S_lens, T_lens, H, G, d, d_idx, B_k, k)
+    assert tw["backward_flops"] == bwd
+    assert tw["kl_flops"] == kl and tw["kl_grad_flops"] == klg
+    assert tw["backward_flops"] == 2.5 * R.prefill_work(S_lens, T_lens, H, G, d, d_idx, B_k, k)["main_flops"]
+
+
+def test_cuda_core_peak():
+    # 148 SMs x 128 fp32 lanes x 2 FLOPs (one FMA) x 1965 MHz
+    assert R.alu_fp32_tflops() == pytest.approx(74.44992, rel=1e-9)
