@@ -70,18 +70,11 @@ __all__ = [
     "msa_forward_rows",
     "lse_combine",
     "invert_selection",
-    "group_of_head",
 ]
 
 
 def _f64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
-
-
-def group_of_head(h: int, H: int, G: int) -> int:
-    """GQA map: group g serves heads [g*H/G, (g+1)*H/G) ([pnsm] sec. 2: 64 query
-    heads share 4 KV heads, one KV head per group)."""
-    return h // (H // G)
 
 
 def query_positions(T_b: int, S_b: int) -> np.ndarray:
