@@ -143,3 +143,55 @@ def test_reference_arm_prints_the_contract_line():
     assert line["config"] == bench.run_config(args, w, line["config"]["T"], 1)
     assert bench.pass_rows(-1, 131072) == 0 and bench.pass_rows(-1, 131073) == 131072
     assert bench.pass_rows(700, 5000) == 700
+
+
+def test_training_leg_reports_each_kernel_against_the_alu_peak():
+    # the leg's plumbing, with stand-ins for the library calls that accept
+    # exactly the arguments the real binding functions take
+    import inspect
+    import types
+
+    import bench
+    from block_sparse_long_exp_b200 import msa as M
+    from block_sparse_long_exp_b200 import workloads as W
+
+    w = W.WORKLOADS[bench.PREFILL]
+    T = 300
+    calls = []
+
+    def stand_in(name, ret):
+        sig = inspect.signature(getattr(M, name))
+
+        def f(*a, **kw):
+            sig.bind(*a, **kw)
+            calls.append(name)
+            return ret(*a, **kw)
+        return f
+    lib = types.SimpleNamespace(
+        make_shape=M.make_shape,
+        make_varlen=stand_in("make_varlen", lambda *a: None),
+        msa_index_topk=stand_in("msa_index_topk", lambda *a, **kw: torch.zeros(T, w.G, w.k, dtype=torch.int32)),
+        msa_sparse_attn_prefill=stand_in("msa_sparse_attn_prefill",
+                                         lambda sh, sq, q, *a, **kw: (torch.zeros_like(q), torch.zeros(T, w.H))),
+        msa_sparse_attn_backward=stand_in("msa_sparse_attn_backward", lambda *a, **kw: (None, None, None)),
+        msa_index_kl=stand_in("msa_index_kl", lambda *a, **kw: (torch.zeros(T, w.G), torch.zeros(T, w.G))),
+        msa_index_kl_backward=stand_in("msa_index_kl_backward", lambda *a, **kw: (None, None)),
+        msa_profile_reset=stand_in("msa_profile_reset", lambda: None),
+        msa_profile_enable=stand_in("msa_profile_enable", lambda on: None),
+        msa_profile_read=stand_in("msa_profile_read", lambda name=None: (8.0, 4)))
+    args = bench.build_parser().parse_args(["--training", "--training-T", str(T), "--steps", "4", "--warmup", "3"])
+    sync = torch.cuda.synchronize
+    torch.cuda.synchronize = lambda *a: None
+    try:
+        res = bench.training_leg(args, w, W, R, lib, torch, device="cpu")
+    finally:
+        torch.cuda.synchronize = sync
+    # one checked pass, the warm-up, the timed passes, one checked pass
+    assert calls.count("msa_sparse_attn_backward") == 1 + 3 + 4 + 1
+    tw = R.training_work([T], [T], w.H, w.G, w.d, w.d_idx, w.B_k, w.k)
+    assert res["T"] == T and res["peak"] == R.alu_fp32_tflops()
+    for name, key in (("attn_bwd", "backward_flops"), ("index_kl", "kl_flops"), ("index_kl_grad", "kl_grad_flops")):
+        kr = res["kernels"][name]
+        assert kr["bound"] == "alu" and kr["ms_per_launch"] == 2.0 and kr["flops_per_launch"] == tw[key]
+        assert kr["achieved"] == pytest.approx(tw[key] / 2e-3 / 1e12)
+        assert kr["frac"] == pytest.approx(kr["achieved"] / R.alu_fp32_tflops())
