@@ -210,7 +210,10 @@ msa_status_t msa_sparse_attn_decode_paged(const msa_shape_t* shape, const msa_pa
 
 /* ---------------------------------------------------------------------- */
 /* Prefill (or a chunk of one) over a paged KV cache: gather the pages into
- * packed rows, then run the packed calls.  Packed row cu_k[b] + j of sequence
+ * packed rows, then run the packed calls.  The pages give no cache format.
+ * lumevalley.com says MSA on GQA keeps a serving stack's existing KV-cache
+ * management and replaces only the attention kernel; this is the plainest
+ * way to take such a cache into the prefill.  Packed row cu_k[b] + j of sequence
  * b is row (p * B_k + j mod B_k) of `pages`, p = block_table[b * max_blocks +
  * j / B_k]; rows are row_bytes each (a multiple of 16; index keys: d_idx * 2,
  * keys or values: G * d * 2).  seqs gives the lengths (cu_k, max_k_len <=
@@ -227,7 +230,9 @@ msa_status_t msa_gather_pages(const msa_varlen_t* seqs, const int32_t* block_tab
 /* ---------------------------------------------------------------------- */
 /* Main Branch backward: the gradients of the attention over the support J
  * (the selected blocks' tokens cut at the query, or with dense != 0 every
- * token up to it) for an upstream gradient dout.  With P_j = exp(sm_scale
+ * token up to it) for an upstream gradient dout.  MSA is trained end to end,
+ * so the forward that yifor-blog "設計核心" item 2 and pnsm.cn sec. 2 define
+ * is differentiated like any softmax attention.  With P_j = exp(sm_scale
  * q_h.k_j - lse[t, h]), dP_j = dout_h.v_j, D = dout_h.out_h, dS_j = P_j (dP_j
  * - D):
  *   dq[t, h]  = sm_scale sum_j dS_j k_j                 (out, float [T, H, d])
