@@ -159,8 +159,9 @@ msa_status_t msa_sparse_attn_prefill(const msa_shape_t* shape, const msa_varlen_
                                      void* ws, size_t ws_bytes, void* stream);
 
 /* Main Branch, decode: one query per sequence (T_b = 1, position S_b - 1,
- * the cache already holding the new token).  Same contract as the prefill
- * call; q_chunk is implied (all queries in one pass). */
+ * the cache already holding the new token), the decode step of pnsm.cn
+ * sec. 9 and yhxrc.cn sec. 二.  Same contract as the prefill call; q_chunk
+ * is implied (all queries in one pass). */
 msa_status_t msa_sparse_attn_decode(const msa_shape_t* shape, const msa_varlen_t* seqs,
                                     const void* q, const void* k_cache, const void* v_cache,
                                     const int32_t* sel, void* out, float* lse,
@@ -364,7 +365,9 @@ msa_status_t msa_dense_attn(const msa_shape_t* shape, const msa_varlen_t* seqs,
 
 /* ---------------------------------------------------------------------- */
 /* Work split of the prefill main branch (process-wide; returns the previous
- * value).  The prefill call groups query rows into tiles of 2 x 128/max(H/G, 8)
+ * value).  This library's own scheduling choice: the pages' kernel runs
+ * KV-outer throughout (pnsm.cn sec. 7; yololab.net "KV Outer Gather Q").
+ * The prefill call groups query rows into tiles of 2 x 128/max(H/G, 8)
  * consecutive queries of one sequence; a block chosen by at least `theta` of a
  * tile's queries (for one group) is attended query-tile-major, merged with an
  * online softmax into one result per query, instead of one KV-outer partial
