@@ -18,6 +18,29 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
 
 
+# GPU test files in run order.  Files with parity evidence on a B200 come
+# first.  The newer ones follow, from the simplest kernel to the one that chains
+# the others.  Under -x a failure in a newer file then never hides the older
+# evidence.  A GPU file missing from the list runs last.
+GPU_FILE_ORDER = (
+    "test_gpu_edges.py", "test_gpu_fullsize.py", "test_gpu_paged.py", "test_gpu_parity.py",
+    "test_gpu_no_alloc.py", "test_gpu_canary.py", "test_gpu_max_batch.py", "test_gpu_share.py",
+    "test_gpu_window.py",
+    "test_gpu_paged_prefill.py", "test_gpu_policy.py", "test_gpu_backward.py", "test_gpu_index_kl.py",
+    "test_gpu_autograd.py",
+)
+
+
+def pytest_collection_modifyitems(session, config, items):
+    rank = {name: i for i, name in enumerate(GPU_FILE_ORDER)}
+
+    def key(item):
+        if item.get_closest_marker("gpu") is None:
+            return -1                                   # CPU tests keep their place, first
+        return rank.get(os.path.basename(str(item.fspath)), len(GPU_FILE_ORDER))
+    items.sort(key=key)                                 # stable: order within a file is kept
+
+
 def max_abs(o, r):
     return float(np.max(np.abs(np.asarray(o, np.float64) - np.asarray(r, np.float64))))
 
