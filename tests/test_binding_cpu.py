@@ -175,3 +175,15 @@ def test_gather_pages_checks_its_tensors(M):
         M.msa_gather_pages(s, table, 5, pages)
     with pytest.raises(M.MsaError, match="CUDA"):
         M.msa_gather_pages(s, table, 4, pages)
+
+
+def test_a_missing_library_fails_loudly(tmp_path):
+    # no fallback: without the built library every call stops with an error
+    from block_sparse_long_exp_b200 import msa as M
+    saved = M._lib
+    M._lib = None
+    try:
+        with pytest.raises(M.MsaError, match="no CPU fallback"):
+            M.load_library(str(tmp_path / "libmsa.so"))
+    finally:
+        M._lib = saved
