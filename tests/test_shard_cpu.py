@@ -2,7 +2,7 @@
 shard.py): the planner's ranges cover every query once and balance the
 algorithmic work; and on two gloo ranks, each rank's chunked-prefill oracle
 result (queries [a, b) over keys [0, b)) gathered on rank 0 equals the
-unsharded oracle result row for row; and the backward of the split: each
+unsharded oracle result row for row; and the backward of the split on two and three ranks: each
 rank's key-side gradients (dk, dv, the KL target's dk_idx) summed over the
 ranks by sum_key_grads, with the query-side ones (dq, dq_idx) gathered, equal
 the unsharded backward oracles."""
@@ -136,11 +136,12 @@ def _rank_bwd(rank, world, port, result):
         dist.destroy_process_group()
 
 
-def test_sharded_backward_sums_key_grads_on_two_gloo_ranks():
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_backward_sums_key_grads_on_gloo_ranks(world):
     ctx = mp.get_context("spawn")
     result = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_bwd, args=(r, 2, port, result)) for r in range(2)]
+    procs = [ctx.Process(target=_rank_bwd, args=(r, world, port, result)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
