@@ -1,10 +1,10 @@
 """Query-range sharding of one sequence's prefill (block_sparse_long_exp_b200/
-shard.py): the planner's ranges cover every query once and balance the
-algorithmic work; and on two gloo ranks, each rank's chunked-prefill oracle
-result (queries [a, b) over keys [0, b)) gathered on rank 0 equals the
-unsharded oracle result row for row; and the backward of the split on two and three ranks: each
-rank's key-side gradients (dk, dv, the KL target's dk_idx) summed over the
-ranks by sum_key_grads, with the query-side ones (dq, dq_idx) gathered, equal
+shard.py).  The planner's ranges cover every query once and balance the
+algorithmic work.  On two gloo ranks, each rank's chunked-prefill oracle result
+(queries [a, b) over keys [0, b)), gathered on rank 0, equals the unsharded
+oracle result row for row.  For the backward of the split, on two and on three
+ranks, sum_key_grads sums each rank's key-side gradients (dk, dv, the KL
+target's dk_idx); with the query-side ones (dq, dq_idx) gathered, they equal
 the unsharded backward oracles."""
 import os
 import socket
