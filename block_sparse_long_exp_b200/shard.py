@@ -15,6 +15,11 @@ the keys [0, b_r), so its dk, dv (and the index-alignment target's dk_idx)
 hold only its own queries' contributions to those rows.  The layer's key-side
 gradients are the sum of these over the ranks (sum_key_grads).  dq and dq_idx
 stay sharded with the queries, as the output does.
+
+A layer can also be split by GQA group (split_groups, group_slice): each rank
+runs the whole path on its G / world groups and their query heads, with the
+index keys replicated, and no collective unless the output is wanted whole
+(gather_heads: one all-gather over the heads).
 """
 from __future__ import annotations
 
@@ -95,6 +100,44 @@ def sum_key_grads(grads: Sequence[object], S: int, group=None) -> List[object]:
         out.append(flat[at:at + t.numel()].view(t.shape))
         at += t.numel()
     return out
+
+
+def split_groups(G: int, world: int) -> List[Tuple[int, int]]:
+    """GQA groups [g0, g1) of each rank for a group-sharded prefill: G / world
+    consecutive groups each (world must divide G).  Every group's index
+    branch and main branch are independent of the others'; only the index
+    keys are shared, so they are replicated."""
+    if world < 1 or G % world:
+        raise ValueError(f"{world} ranks cannot share {G} groups evenly")
+    n = G // world
+    return [(r * n, (r + 1) * n) for r in range(world)]
+
+
+def group_slice(inp: Dict[str, object], H: int, G: int, g0: int, g1: int) -> Dict[str, object]:
+    """The inputs of groups [g0, g1) of a layer, as a layer of g1 - g0 groups:
+    their query heads [g0 H/G, g1 H/G) of q, their rows of k, v and q_idx,
+    and every index key.  The library's calls take it with the shape
+    (H (g1 - g0) / G heads, g1 - g0 groups); the offsets are unchanged."""
+    Hg = H // G
+    out = dict(inp)
+    out["q"] = inp["q"][:, g0 * Hg:g1 * Hg].contiguous()
+    out["k"] = inp["k"][:, g0:g1].contiguous()
+    out["v"] = inp["v"][:, g0:g1].contiguous()
+    out["q_idx"] = inp["q_idx"][:, g0:g1].contiguous()
+    return out
+
+
+def gather_heads(out_part, group=None):
+    """The full output [T, H, d] from every rank's heads [T, H / world, d] of
+    a group-sharded prefill (one all-gather; ranks hold consecutive groups in
+    rank order).  Without an initialised group the part is returned."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return out_part
+    parts = [torch.empty_like(out_part) for _ in range(dist.get_world_size(group))]
+    dist.all_gather(parts, out_part.contiguous(), group=group)
+    return torch.cat(parts, dim=1)
 
 
 def imbalance(work: np.ndarray, ranges: List[Tuple[int, int]]) -> float:

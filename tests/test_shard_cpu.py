@@ -5,7 +5,9 @@ algorithmic work.  On two gloo ranks, each rank's chunked-prefill oracle result
 oracle result row for row.  For the backward of the split, on two and on three
 ranks, sum_key_grads sums each rank's key-side gradients (dk, dv, the KL
 target's dk_idx); with the query-side ones (dq, dq_idx) gathered, they equal
-the unsharded backward oracles."""
+the unsharded backward oracles.  Split by GQA group on two and four ranks,
+every rank's selection equals its groups' columns of the unsharded one, and
+the outputs gathered over the heads equal the unsharded output."""
 import os
 import socket
 
@@ -148,6 +150,61 @@ def test_sharded_backward_sums_key_grads_on_gloo_ranks(world):
         p.join(timeout=300)
     assert all(p.exitcode == 0 for p in procs)
     assert result.get(timeout=10) is True
+
+
+def _rank_groups(rank, world, port, result):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from block_sparse_long_exp_b200 import workloads as W
+        from oracle import msa_oracle as O
+        w = W.Workload("shard_groups", "prefill", H=8, G=4, d=16, d_idx=8, B_k=4, k=3, seed=9, hot_frac=0.1)
+        inp = W.make_inputs(w, "cpu", lengths=[45, 30])
+        cq, ck = inp["cu_q_host"], inp["cu_k_host"]
+        f = lambda t: t.double().numpy()  # noqa: E731
+        g0, g1 = SH.split_groups(w.G, world)[rank]
+        part = SH.group_slice(inp, w.H, w.G, g0, g1)
+        assert part["q"].shape[1] == w.H * (g1 - g0) // w.G and part["k_idx"] is inp["k_idx"]
+        sel = O.index_topk(f(part["q_idx"]), f(part["k_idx"]), cq, ck, w.k, w.B_k)
+        o, lse = O.msa_forward_rows(f(part["q"]), f(part["k"]), f(part["v"]), sel, cq, ck, list(range(cq[-1])),
+                                    w.B_k, w.sm_scale)
+        full_o = SH.gather_heads(torch.from_numpy(o))
+        full_l = SH.gather_heads(torch.from_numpy(lse)[:, :, None])[:, :, 0]
+        sels = [None] * world
+        dist.all_gather_object(sels, (g0, g1, sel))
+        if rank == 0:
+            want_sel = O.index_topk(f(inp["q_idx"]), f(inp["k_idx"]), cq, ck, w.k, w.B_k)
+            want_o, want_l = O.msa_forward_rows(f(inp["q"]), f(inp["k"]), f(inp["v"]), want_sel, cq, ck,
+                                                list(range(cq[-1])), w.B_k, w.sm_scale)
+            ok = all(np.array_equal(s_, want_sel[:, a_:b_]) for a_, b_, s_ in sels)
+            ok = ok and np.allclose(full_o.numpy(), want_o, rtol=0, atol=1e-12)
+            ok = ok and np.allclose(full_l.numpy(), want_l, rtol=0, atol=1e-12)
+            result.put(bool(ok))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_group_sharded_oracle_equals_unsharded_on_gloo_ranks(world):
+    ctx = mp.get_context("spawn")
+    result = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_groups, args=(r, world, port, result)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+    assert all(p.exitcode == 0 for p in procs)
+    assert result.get(timeout=10) is True
+
+
+def test_split_groups():
+    assert SH.split_groups(4, 1) == [(0, 4)]
+    assert SH.split_groups(4, 2) == [(0, 2), (2, 4)]
+    assert SH.split_groups(4, 4) == [(0, 1), (1, 2), (2, 3), (3, 4)]
+    for bad in (3, 8, 0):
+        with pytest.raises(ValueError):
+            SH.split_groups(4, bad)
 
 
 def test_sum_key_grads_without_a_group_pads():
