@@ -27,7 +27,7 @@ GPU_FILE_ORDER = (
     "test_gpu_no_alloc.py", "test_gpu_canary.py", "test_gpu_max_batch.py", "test_gpu_share.py",
     "test_gpu_window.py",
     "test_gpu_paged_prefill.py", "test_gpu_policy.py", "test_gpu_backward.py", "test_gpu_index_kl.py",
-    "test_gpu_autograd.py",
+    "test_gpu_autograd.py", "test_gpu_group_shard.py",
 )
 
 
