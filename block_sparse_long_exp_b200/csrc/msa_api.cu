@@ -17,14 +17,9 @@
 
 using namespace msa;
 
-namespace {
+namespace msa {
 
-// Query-tile threshold (msa_set_tile_threshold): -1 automatic, 0 off.
-std::atomic<int> g_tile_theta{-1};
-
-constexpr size_t kAlign = 256;
-
-bool shape_ok(const msa_shape_t* s) {
+static bool shape_ok(const msa_shape_t* s) {
   return s != nullptr && s->H > 0 && s->G > 0 && s->d > 0 && s->d_idx > 0 && s->B_k > 0 && s->k > 0;
 }
 
@@ -52,6 +47,17 @@ msa_status_t check_seqs(const msa_varlen_t* v) {
   return MSA_OK;
 }
 
+}  // namespace msa
+
+namespace {
+
+// Query-tile threshold (msa_set_tile_threshold): -1 automatic, 0 off.
+std::atomic<int> g_tile_theta{-1};
+// Query rows per planning window of the KV-outer lists (msa_set_attn_window).
+std::atomic<int> g_attn_window{kDefaultWindow};
+
+constexpr size_t kAlign = 256;
+
 bool ws_ok(const void* ws, size_t have, size_t need) {
   return ws != nullptr && (reinterpret_cast<uintptr_t>(ws) % kAlign) == 0 && have >= need;
 }
@@ -63,7 +69,7 @@ struct AttnLayout {
   size_t blk_off, counts, cursor, tile_sums, nitems, entries, items, part_acc, part_lse;
   size_t unit_blk, unit_nblk, unit_list, dmask, dstate, dmember, clist, tile_ctr, total;
   int64_t nlists, max_items;
-  int32_t qpi;
+  int32_t qpi, win;
 };
 
 AttnLayout attn_layout(const msa_shape_t* s, const msa_varlen_t* v, int64_t rows) {
@@ -72,7 +78,8 @@ AttnLayout attn_layout(const msa_shape_t* s, const msa_varlen_t* v, int64_t rows
   const int qpt = 128 / (hg < 8 ? 8 : hg);            // queries per 128-row tile
   L.qpi = 8 * qpt < kMaxItemQueries ? 8 * qpt : kMaxItemQueries;
   L.nlists = (int64_t)s->G * total_blocks_bound(v);
-  const int64_t nkeys = ((rows + kWindow - 1) / kWindow) * L.nlists;
+  L.win = attn_window_rows();
+  const int64_t nkeys = ((rows + L.win - 1) / L.win) * L.nlists;
   const int64_t nentries = rows * s->G * s->k;
   L.max_items = nentries / L.qpi + (nkeys < nentries ? nkeys : nentries) + 1;
   size_t off = kWsHeader;
@@ -149,6 +156,7 @@ msa_status_t attn_common(const msa_shape_t* shape, const msa_varlen_t* seqs, con
   a.items = reinterpret_cast<Item*>(base + L.items);
   a.max_items = L.max_items;
   a.nlists = L.nlists;
+  a.win_rows = L.win;
   a.part_acc = base + L.part_acc;
   a.part_lse = reinterpret_cast<float*>(base + L.part_lse);
   a.queries_per_item = L.qpi;
@@ -210,6 +218,8 @@ PagedLayout paged_layout(const msa_shape_t* s, const msa_paged_t* pg) {
 }  // namespace
 
 namespace msa {
+
+int attn_window_rows() { return g_attn_window.load(std::memory_order_relaxed); }
 
 int make_tmap_bf16(void* tmap_out, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
                    const uint32_t* box, int swizzle_bytes) {
@@ -566,6 +576,13 @@ msa_status_t msa_gather_pages(const msa_varlen_t* seqs, const int32_t* block_tab
 
 int32_t msa_set_tile_threshold(int32_t theta) {
   return g_tile_theta.exchange(theta < 0 ? -1 : theta);
+}
+
+int32_t msa_set_attn_window(int32_t rows) {
+  if (rows <= 0) rows = kDefaultWindow;
+  if (rows < kMinWindow) rows = kMinWindow;
+  if (rows > kMaxWindow) rows = kMaxWindow;
+  return g_attn_window.exchange(rows);
 }
 
 msa_status_t msa_get_device_error(void* ws, int32_t* code, int32_t* where, int32_t* info0, int32_t* info1,

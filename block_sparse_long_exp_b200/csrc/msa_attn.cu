@@ -6,7 +6,7 @@
 // A pass over query rows [t0, t1):
 //   0. tiles    : (msa_tile_attn.cu) the blocks that many queries of a small
 //                 query tile share are marked for the query-tile kernel;
-//   1. count    : per (window, sequence, group, block) list, how many of the
+//   1. count    : per (group, window, sequence block) list, how many of the
 //                 remaining (query, slot) entries chose it (warp-aggregated
 //                 atomics);
 //   2. plan     : exclusive scans -> list offsets, work items of at most
@@ -49,9 +49,10 @@ __global__ void block_offsets_kernel(const int32_t* __restrict__ cu_k, int batch
   }
 }
 
-// Validates an entry and returns its list id, or -1 (slot empty or invalid).
-__device__ __forceinline__ int entry_list(int blk, int64_t t, int g, int G, int batch, const int32_t* cu_q,
-                                          const int32_t* cu_k, const int32_t* blk_off, DevError* err) {
+// Validates an entry and returns its block's index over the whole batch
+// (blk_off[b] + blk), or -1 (slot empty or invalid).
+__device__ __forceinline__ int entry_block(int blk, int64_t t, int batch, const int32_t* cu_q, const int32_t* cu_k,
+                                           const int32_t* blk_off, DevError* err) {
   if (blk < 0) return -1;
   const int b = find_seq(cu_q, batch, t);
   const int Tb = cu_q[b + 1] - cu_q[b];
@@ -61,12 +62,14 @@ __device__ __forceinline__ int entry_list(int blk, int64_t t, int g, int G, int 
     report_error(err, MSA_ERR_DEVICE_CHECK, kSiteInvert, (int)t, blk);
     return -1;
   }
-  return (blk_off[b] + blk) * G + g;
+  return blk_off[b] + blk;
 }
 
 // Pass 1 and 3: one thread per (query, group).  Lists are keyed by
-// (window of kWindow query rows, sequence block, group) so that the work
-// items come out window-major (the queries of one window stay hot in L2).
+// (group, window of win_rows query rows, block): the work items come out
+// group-major and, within a group, window by window, so the gathered rows of
+// one group and window (win_rows x Hg x d x 2 bytes) stay hot in L2 while its
+// items run, and consecutive windows of a group reuse that group's K/V blocks.
 // kScatter == false counts, == true claims positions from `counter`
 // (the cursors) and writes the entries (t - t0) * k + slot.
 // Slots whose bit is set in dmask (when given) were attended by a query tile
@@ -79,8 +82,8 @@ __device__ __forceinline__ int entry_list(int blk, int64_t t, int g, int G, int 
 template <bool kScatter>
 __global__ void count_scatter_kernel(const int32_t* __restrict__ sel, int64_t t0, int64_t t1, int G, int k,
                                      int batch, const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_k,
-                                     const int32_t* __restrict__ blk_off, int64_t nlists,
-                                     const uint32_t* __restrict__ dmask, int32_t* __restrict__ counter,
+                                     const int32_t* __restrict__ blk_off, int64_t nblocks, int64_t nwin,
+                                     int win_rows, const uint32_t* __restrict__ dmask, int32_t* __restrict__ counter,
                                      uint32_t* __restrict__ entries, uint2* __restrict__ clist, DevError* err) {
   const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t n = (t1 - t0) * G;
@@ -88,7 +91,7 @@ __global__ void count_scatter_kernel(const int32_t* __restrict__ sel, int64_t t0
   const int64_t tl = active ? gid / G : 0;
   const int64_t t = t0 + tl;
   const int g = active ? (int)(gid % G) : 0;
-  const int64_t wbase = (tl / kWindow) * nlists;
+  const int64_t wbase = ((int64_t)g * nwin + tl / win_rows) * nblocks;
   const int lane = threadIdx.x & 31;
   const uint32_t covered = (active && dmask != nullptr) ? dmask[gid] : 0u;
   const int first = covered != 0u ? 1 : 0;   // packed position 0 holds the tile's merged partial
@@ -100,8 +103,8 @@ __global__ void count_scatter_kernel(const int32_t* __restrict__ sel, int64_t t0
       const int32_t blk = sel[(t * G + g) * k + s];
       packed = first + __popc(live & ~covered);
       if (blk >= 0) live |= 1u << s;
-      const int L = entry_list(blk, t, g, G, batch, cu_q, cu_k, blk_off, err);
-      if (L >= 0 && !((covered >> s) & 1u)) key = wbase + L;
+      const int gb = entry_block(blk, t, batch, cu_q, cu_k, blk_off, err);
+      if (gb >= 0 && !((covered >> s) & 1u)) key = wbase + gb;
     }
     // warp-aggregated atomics: lanes with the same key share one atomic
     const unsigned peers = __match_any_sync(0xffffffffu, key);
@@ -191,9 +194,9 @@ __global__ void __launch_bounds__(kScanThreads) scan_tiles_kernel(int32_t* __res
 }
 
 // Final pass: list offsets and cursors, then the work items of each list
-// (chunks of at most C entries), in key order (window-major).
+// (chunks of at most C entries), in key order (group-major, then window by window).
 __global__ void __launch_bounds__(kScanThreads) scan_items_kernel(const int32_t* __restrict__ counts, int64_t nkeys,
-                                                                 int64_t nlists, int G, int batch, int C,
+                                                                 int64_t nblocks, int64_t nwin, int batch, int C,
                                                                  const int32_t* __restrict__ tile_sums,
                                                                  const int32_t* __restrict__ blk_off,
                                                                  int32_t* __restrict__ cursor,
@@ -219,8 +222,9 @@ __global__ void __launch_bounds__(kScanThreads) scan_items_kernel(const int32_t*
     cursor[key] = off;
     const int c = cnt[i];
     if (c > 0) {
-      const int64_t L = key % nlists;
-      const int gb = (int)(L / G), g = (int)(L % G);
+      // key = (g * nwin + window) * nblocks + block of the batch
+      const int gb = (int)(key % nblocks);
+      const int g = (int)(key / (nblocks * nwin));
       int lo = 0, hi = batch;
       while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
@@ -956,8 +960,10 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
     ProfScope p("block_offsets", stream);
     block_offsets_kernel<<<1, 32, 0, st>>>(a.cu_k, a.batch, a.blk_off);
   }
-  const int64_t nwin = (nrows + kWindow - 1) / kWindow;
+  const int win = a.win_rows;
+  const int64_t nwin = (nrows + win - 1) / win;
   const int64_t nkeys = nwin * a.nlists;
+  const int64_t nblocks = a.nlists / a.G;
   e = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * nkeys, st);
   if (e != cudaSuccess) return (int)e;
   const bool tiles = a.theta > 0;
@@ -973,7 +979,7 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
   {
     ProfScope p("count", stream);
     count_scatter_kernel<false><<<cs_blocks, 256, 0, st>>>(a.sel, a.t0, a.t1, a.G, a.k, a.batch, a.cu_q, a.cu_k,
-                                                           a.blk_off, a.nlists, dmask, a.counts, nullptr,
+                                                           a.blk_off, nblocks, nwin, win, dmask, a.counts, nullptr,
                                                            tiles ? nullptr : a.clist, a.err);
   }
   const int ntiles = (int)((nkeys + kScanTile - 1) / kScanTile);
@@ -981,14 +987,15 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
     ProfScope p("plan", stream);
     scan_reduce_kernel<<<ntiles, kScanThreads, 0, st>>>(a.counts, nkeys, a.queries_per_item, a.tile_sums);
     scan_tiles_kernel<<<1, kScanThreads, 0, st>>>(a.tile_sums, ntiles, a.nitems, a.max_items, a.err);
-    scan_items_kernel<<<ntiles, kScanThreads, 0, st>>>(a.counts, nkeys, a.nlists, a.G, a.batch, a.queries_per_item,
+    scan_items_kernel<<<ntiles, kScanThreads, 0, st>>>(a.counts, nkeys, nblocks, nwin, a.batch, a.queries_per_item,
                                                        a.tile_sums, a.blk_off, a.cursor, a.items, a.max_items);
     prof_count_launch(2);
   }
   {
     ProfScope p("scatter", stream);
     count_scatter_kernel<true><<<cs_blocks, 256, 0, st>>>(a.sel, a.t0, a.t1, a.G, a.k, a.batch, a.cu_q, a.cu_k,
-                                                          a.blk_off, a.nlists, dmask, a.cursor, a.entries, nullptr,
+                                                          a.blk_off, nblocks, nwin, win, dmask, a.cursor, a.entries,
+                                                          nullptr,
                                                           a.err);
   }
   e = cudaGetLastError();

@@ -82,15 +82,41 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 // Wait for the phase with the given parity to complete.  Returns false after
-// ~1 s; the caller then records MSA_ERR_TIMEOUT and unwinds.  The wall clock
-// is read only every 64 failed tries (reading it each time floods the XU pipe
-// while many warps wait).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// limit_ns (~1 s by default); the caller then records MSA_ERR_TIMEOUT and
+// unwinds.  The wall clock is read only every 64 failed tries (reading it each
+// time floods the XU pipe while many warps wait).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
-    if ((n & 63u) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
+    if ((n & 63u) == 0 && global_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// Acquire load of a 32-bit word in global memory (gpu scope): pairs with a
+// release (red.release.gpu) of another CTA, so that what that CTA wrote
+// before its release is visible after this load sees the released value.
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_add_release_gpu(int32_t* p, int32_t v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Wait until a counter in global memory that other CTAs of the same launch
+// advance reaches `target`.  Returns false after limit_ns (~1 s by default);
+// the caller then records MSA_ERR_TIMEOUT and unwinds.
+__device__ __forceinline__ bool flag_wait_geq(const int32_t* flag, int32_t target,
+                                              uint64_t limit_ns = kWaitLimitNs) {
+  if (ld_acquire_gpu(flag) >= target) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t n = 1;; ++n) {
+    __nanosleep(200);
+    if (ld_acquire_gpu(flag) >= target) return true;
+    if ((n & 15u) == 0 && global_ns() - t0 > limit_ns) return false;
   }
 }
 

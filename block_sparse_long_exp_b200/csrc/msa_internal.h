@@ -12,7 +12,9 @@ namespace msa {
 constexpr int kBk = 128;          // block size the kernels are built for
 constexpr int kMaxK = 32;         // largest k
 constexpr int kMaxBatchTiles = 1024;  // sequences per prefill index launch
-constexpr int kWindow = 4096;         // query rows per attention planning window (KV-outer lists)
+constexpr int kDefaultWindow = 8192;  // query rows per attention planning window (KV-outer lists)
+constexpr int kMinWindow = 128;
+constexpr int kMaxWindow = 1 << 20;
 constexpr int kScanTile = 4096;       // keys per CTA of the planning scan
 constexpr int kMaxItemQueries = 64;   // queries per attention work item (upper bound)
 constexpr int kMaxDense = 64;         // dense blocks per query tile (Q-outer side)
@@ -44,6 +46,7 @@ enum ErrorSite : int32_t {
   kSiteTileMma = 153,
   kSiteTileSoftmax = 154,
   kSitePaged = 161,
+  kSiteSelfTest = 171,
 };
 
 // One KV-outer work item: up to `count` queries of the list of
@@ -61,6 +64,10 @@ struct Item {
 constexpr size_t kWsHeader = 256;  // DevError + counters
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Host-side argument checks shared by the entry points (msa_api.cu).
+msa_status_t check_shape(const msa_shape_t* s);
+msa_status_t check_seqs(const msa_varlen_t* v);
 
 // -------------------------------------------------------- host launchers ---
 // Each returns the cudaError_t of its launch(es) (0 on success).
@@ -111,6 +118,7 @@ struct AttnArgs {
   int64_t max_items;
   int32_t* blk_off;    // [batch + 1] block offsets per sequence
   int64_t nlists;      // G * total blocks
+  int32_t win_rows;    // query rows per planning window (lists are keyed by (group, window, block))
   void* part_acc;      // f16 [(t1-t0), G, k, d/8, Hg, 8], each pair's partials packed at slots 0..n-1
   float* part_lse;     // [(t1-t0), G, k, Hg]
   int32_t queries_per_item;
@@ -130,6 +138,7 @@ struct AttnArgs {
   int64_t num_pages;
 };
 int launch_sparse_attn_pass(const AttnArgs& a, void* stream);
+int attn_window_rows();                // planning window of the prefill calls (msa_set_attn_window)
 int launch_combine(const void* part_acc, const float* part_lse, const int32_t* sel, void* out,
                    float* lse, int64_t T, int32_t H, int32_t G, int32_t d, int32_t k, void* stream);
 int tile_queries(int H, int G);        // query rows per tile unit

@@ -49,7 +49,8 @@ EXPORTED = [
     "msa_combine", "msa_dense_attn_workspace_size", "msa_dense_attn",
     "msa_index_topk_decode_noalloc_max_scratch", "msa_index_topk_decode_noalloc",
     "msa_profile_enable", "msa_profile_reset", "msa_profile_read",
-    "msa_get_device_error", "msa_version", "msa_set_tile_threshold",
+    "msa_get_device_error", "msa_version", "msa_set_tile_threshold", "msa_set_attn_window",
+    "msa_selftest_wait_timeout_workspace_size", "msa_selftest_wait_timeout",
     "msa_decode_paged_workspace_size", "msa_index_topk_decode_paged", "msa_sparse_attn_decode_paged",
     "msa_index_kl", "msa_index_kl_backward", "msa_select_window", "msa_sparse_attn_backward",
     "msa_selected_share", "msa_index_topk_policy", "msa_gather_pages",
@@ -125,6 +126,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_version.restype = ctypes.c_char_p
     lib.msa_set_tile_threshold.argtypes = [i32]
     lib.msa_set_tile_threshold.restype = i32
+    lib.msa_set_attn_window.argtypes = [i32]
+    lib.msa_set_attn_window.restype = i32
+    lib.msa_selftest_wait_timeout_workspace_size.argtypes = []
+    lib.msa_selftest_wait_timeout_workspace_size.restype = sz
+    lib.msa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp, sz, vp]
+    lib.msa_selftest_wait_timeout.restype = i32
     lib.msa_decode_paged_workspace_size.argtypes = [P(Shape), P(Paged)]
     lib.msa_decode_paged_workspace_size.restype = sz
     lib.msa_index_topk_decode_paged.argtypes = [P(Shape), P(Paged), vp, vp, vp, vp, sz, vp]
@@ -780,6 +787,26 @@ def msa_set_tile_threshold(theta: int) -> int:
     """Query-tile threshold of the prefill main branch (-1 automatic, 0 off);
     returns the previous value."""
     return int(load_library().msa_set_tile_threshold(int(theta)))
+
+
+def msa_selftest_wait_timeout(limit_us: int = 2000, stream=None) -> Tuple[int, int, int, int]:
+    """Run the bounded-wait self-test (two waits that nothing ever ends, each
+    with a `limit_us` limit) and return (error code, site, waits that ran out,
+    0) once the stream has drained."""
+    lib = load_library()
+    n = int(lib.msa_selftest_wait_timeout_workspace_size())
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    _check(lib.msa_selftest_wait_timeout(int(limit_us), _ptr(ws), n, _stream(stream)), "msa_selftest_wait_timeout")
+    code, where, _, _ = msa_get_device_error(ws, stream)
+    timed_out = int(ws[260:264].view(torch.int32).item())
+    return code, where, timed_out, 0
+
+
+def msa_set_attn_window(rows: int) -> int:
+    """Query rows per planning window of the prefill's KV-outer lists (<= 0:
+    the default); returns the previous value.  Query workspace sizes after
+    setting it."""
+    return int(load_library().msa_set_attn_window(int(rows)))
 
 
 def msa_version() -> str:

@@ -381,6 +381,37 @@ msa_status_t msa_dense_attn(const msa_shape_t* shape, const msa_varlen_t* seqs,
  * it starts, and uses that value throughout. */
 int32_t msa_set_tile_threshold(int32_t theta);
 
+/* Planning window of the prefill main branch's KV-outer lists (process-wide;
+ * returns the previous value).  Also this library's scheduling choice: the
+ * pages invert the selection into one query list per selected KV block
+ * (pnsm.cn sec. 9 "reverse index"); here the lists are cut into windows of
+ * `rows` consecutive query rows of a pass and keyed (group, window, block), so
+ * the work items run group by group and, within a group, window by window:
+ * the gathered query rows of the current window stay in L2, at the price of
+ * loading a block once per window that selects it.  Results do not depend on
+ * the value (each selection is attended exactly once either way).
+ *   rows <= 0   the default (8192)
+ *   otherwise   clamped to [128, 2^20]
+ * The workspace size of msa_sparse_attn_prefill depends on it: query the size
+ * after setting it.  One atomic word, read once per call. */
+int32_t msa_set_attn_window(int32_t rows);
+
+/* ---------------------------------------------------------------------- */
+/* Self-test of the bounded waits (no counterpart on the pages: a failure-
+ * detection check of this library).  Every spin-wait in the kernels gives up
+ * after about a second and records MSA_ERR_TIMEOUT in the call's error word
+ * instead of hanging the GPU.  This call launches one small kernel whose two
+ * waits can never end (an mbarrier nobody arrives on, a workspace counter
+ * nobody advances), each with the library's own wait given `limit_us`
+ * microseconds (1 ... 1,000,000); both give up, the kernel returns, and
+ * msa_get_device_error(ws) then reads MSA_ERR_TIMEOUT (site 171).  The word
+ * at ws + 256 + 4 (int32) counts the waits that ran out (2).
+ * ws: device, 256-byte aligned, msa_selftest_wait_timeout_workspace_size()
+ * bytes; cleared by the call.  Returns MSA_ERR_INVALID_ARG for a limit out of
+ * range, MSA_ERR_WORKSPACE for a missing or short workspace, before any launch. */
+size_t msa_selftest_wait_timeout_workspace_size(void);
+msa_status_t msa_selftest_wait_timeout(uint32_t limit_us, void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------------- */
 /* Decode-shaped index top-k that allocates nothing (the pages have no
  * counterpart: this is a deployment convenience).
@@ -390,18 +421,25 @@ int32_t msa_set_tile_threshold(int32_t theta);
  * out no scratch buffers, or a host that forbids cudaMalloc on the decode path
  * because cudaMalloc synchronizes the device.  Same operation and layouts as
  * msa_index_topk with max_q_len <= 1 (one query per sequence); the caller still
- * passes the inputs and `sel`.
+ * passes the inputs and `sel`.  Arguments are checked as msa_index_topk checks
+ * them, in the same order; with no queries the data pointers may be NULL.
  *
  * Scratch: a fixed array inside the library, msa_index_topk_decode_noalloc_
  * max_scratch() bytes (16 MiB) per GPU, held by every GPU that loads the
- * library until the process exits.  A call whose scratch need
- * (msa_index_topk_workspace_size) exceeds it returns MSA_ERR_WORKSPACE and
- * launches nothing.  Calls and allocations: none (no cudaMalloc/cudaFree).
+ * library until the process exits.  The need is 4*G bytes per cached block
+ * plus small offsets, so the array holds about 1.05 million blocks: about
+ * 134 million cached tokens (sum of the cache lengths) at G = 4 and B_k = 128.
+ * A call whose scratch need (msa_index_topk_workspace_size) exceeds it returns
+ * MSA_ERR_WORKSPACE and launches nothing.  Calls and allocations: none (no
+ * cudaMalloc/cudaFree).
  * The first call on a device looks the array's device address up (with that
- * device current); make that first call before any stream capture.
- * All calls share the one array, which keeps the last call's contents (each
- * call clears the error word it needs zeroed): calls that overlap on the GPU
- * (different streams or devices' contexts sharing it) race; order them.
+ * device current) and keeps it; make that first call before any stream capture.
+ * A cudaDeviceReset of that device ends the use of this entry point on it for
+ * the rest of the process (the kept address would be stale).
+ * All calls on one device share its array, which keeps the last call's
+ * contents (each call clears the error word it needs zeroed): calls that
+ * overlap on the same device (different streams) race, so order them; calls
+ * on different devices use separate copies.
  * device_error (device int32, may be NULL) receives the call's device error
  * code (an msa_status_t, MSA_OK if none), stream-ordered after the call. */
 size_t msa_index_topk_decode_noalloc_max_scratch(void);

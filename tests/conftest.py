@@ -21,13 +21,15 @@ def pytest_configure(config):
 # GPU test files in run order.  Files with parity evidence on a B200 come
 # first.  The newer ones follow, from the simplest kernel to the one that chains
 # the others.  Under -x a failure in a newer file then never hides the older
-# evidence.  A GPU file missing from the list runs last.
+# evidence.  A GPU file missing from the list runs after the listed ones but
+# before test_zz_no_alloc.py, which stays the very last.
 GPU_FILE_ORDER = (
     "test_gpu_edges.py", "test_gpu_fullsize.py", "test_gpu_paged.py", "test_gpu_parity.py",
-    "test_gpu_no_alloc.py", "test_gpu_canary.py", "test_gpu_max_batch.py", "test_gpu_share.py",
+    "test_gpu_canary.py", "test_gpu_max_batch.py", "test_gpu_share.py",
     "test_gpu_window.py",
     "test_gpu_paged_prefill.py", "test_gpu_policy.py", "test_gpu_backward.py", "test_gpu_index_kl.py",
-    "test_gpu_autograd.py", "test_gpu_group_shard.py",
+    "test_gpu_autograd.py", "test_gpu_group_shard.py", "test_gpu_timeout.py",
+    "test_zz_no_alloc.py",          # the allocation-free entry point: always the last file
 )
 
 
@@ -37,7 +39,10 @@ def pytest_collection_modifyitems(session, config, items):
     def key(item):
         if item.get_closest_marker("gpu") is None:
             return -1                                   # CPU tests keep their place, first
-        return rank.get(os.path.basename(str(item.fspath)), len(GPU_FILE_ORDER))
+        name = os.path.basename(str(item.fspath))
+        if name == GPU_FILE_ORDER[-1]:
+            return len(GPU_FILE_ORDER) + 1
+        return rank.get(name, len(GPU_FILE_ORDER))
     items.sort(key=key)                                 # stable: order within a file is kept
 
 

@@ -197,3 +197,49 @@ def test_gather_pages_host_checks(lib):
     assert lib.msa_gather_pages(ctypes.byref(seqs), T, 8, 8, 100, 256, 256, 256, 1 << 20, None) == 1     # row bytes
     assert lib.msa_gather_pages(ctypes.byref(seqs), T, 8, 8, 128, 258, 256, 256, 1 << 20, None) == 1     # alignment
     assert lib.msa_gather_pages(ctypes.byref(seqs), T, 8, 8, 128, 256, 256, 256, 16, None) == 3          # workspace
+
+
+def test_noalloc_host_checks_match_msa_index_topk(lib):
+    """The allocation-free decode index call checks its arguments as
+    msa_index_topk does, in the same order, before it looks anything up on a
+    device: a bad shape or sequence description gives the same status, and the
+    data pointers are only required when there are queries."""
+    from block_sparse_long_exp_b200 import msa
+    shape = msa.make_shape(64, 4, 128, 64, 16)
+    bad_bk = msa.make_shape(64, 4, 128, 64, 16, B_k=64)
+    cu = (ctypes.c_int32 * 3)(0, 1, 2)
+    cuk = (ctypes.c_int32 * 3)(0, 500, 900)
+    seqs = msa.Varlen(2, 1, 500, 0, 2, 900, ctypes.addressof(cu), ctypes.addressof(cuk))
+    no_cu = msa.Varlen(2, 1, 500, 0, 2, 900, None, ctypes.addressof(cuk))
+
+    def both(sh, sq, ptr):
+        a = lib.msa_index_topk(sh, sq, ptr, ptr, ptr, None, 0, None)
+        b = lib.msa_index_topk_decode_noalloc(sh, sq, ptr, ptr, ptr, None, None)
+        return a, b
+
+    a, b = both(ctypes.byref(shape), ctypes.byref(no_cu), 256)
+    assert a == b == 1                                   # MSA_ERR_INVALID_ARG: null cu_q
+    a, b = both(ctypes.byref(bad_bk), ctypes.byref(seqs), 256)
+    assert a == b == 2                                   # MSA_ERR_UNSUPPORTED: B_k = 64
+    a, b = both(None, ctypes.byref(seqs), 256)
+    assert a == b == 1
+    # queries present: null data pointers are rejected
+    assert lib.msa_index_topk_decode_noalloc(ctypes.byref(shape), ctypes.byref(seqs), None, None, None, None,
+                                             None) == 1
+    # no queries: null data pointers are allowed (without a GPU the call then
+    # stops at the device lookup, never at the argument check)
+    none_q = msa.Varlen(2, 0, 500, 0, 0, 900, ctypes.addressof(cu), ctypes.addressof(cuk))
+    rc = lib.msa_index_topk_decode_noalloc(ctypes.byref(shape), ctypes.byref(none_q), None, None, None, None, None)
+    assert rc != 1
+
+
+def test_selftest_wait_host_checks(lib):
+    """The bounded-wait self-test rejects a limit outside 1 us ... 1 s and a
+    missing or short workspace before it launches anything."""
+    n = lib.msa_selftest_wait_timeout_workspace_size()
+    assert n >= 264
+    assert lib.msa_selftest_wait_timeout(0, 256, n, None) == 1            # MSA_ERR_INVALID_ARG
+    assert lib.msa_selftest_wait_timeout(1000001, 256, n, None) == 1
+    assert lib.msa_selftest_wait_timeout(1000, None, n, None) == 3        # MSA_ERR_WORKSPACE
+    assert lib.msa_selftest_wait_timeout(1000, 256, n - 1, None) == 3
+    assert lib.msa_selftest_wait_timeout(1000, 272, n, None) == 3         # not 256-byte aligned

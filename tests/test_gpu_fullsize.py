@@ -117,6 +117,6 @@ def test_prefill_1m_hot_chunked(M):
     w = W.WORKLOADS["prefill_n1048576_hot2"]
     inp = W.make_inputs(w, "cuda")
     sel, out, lse = _run(M, w, inp, q_chunk=131072)
-    rows = W.sample_rows([w.T], w.B_k, w.k, 4096, seed=104, hot_blocks=None)
+    rows = W.sample_rows([w.T], w.B_k, w.k, 4096, seed=104, hot_blocks=inp["hot_blocks"])
     rows = sorted(set(rows) | {131071, 131072, 2 * 131072 + 5})   # rows at pass boundaries
     _check_rows(w, inp, sel, out, lse, rows)
