@@ -58,6 +58,23 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+HBM_SPEC_GBS = 7700.0            # B200 HBM3e, nominal (HGX figure)
+
+
+def tensor_peak(peaks, src, clk):
+    """The bf16 tensor peak the sampled clocks support: the burst figure
+    (measured at the maximum SM clock) when the median SM clock under load was
+    within 5% of the maximum, else the sustained one (measured under the power
+    cap).  Returns (peak, source text)."""
+    med, mx = (clk or {}).get("sm_mhz"), (clk or {}).get("sm_max_mhz")
+    at_max = bool(med and mx and med >= 0.95 * mx)
+    if at_max:
+        return peaks["bf16_tflops"], (f"bf16_tflops, burst ({src}): median SM clock {med:.0f} of {mx:.0f} MHz "
+                                      f"under load")
+    how = f"median SM clock {med:.0f} of {mx:.0f} MHz" if med and mx else "clocks not sampled"
+    return peaks["bf16_tflops_sustained"], f"bf16_tflops_sustained ({src}): {how}"
+
+
 # ------------------------------------------------------------------ clocks ---
 
 class ClockSampler:
@@ -234,6 +251,94 @@ def training_leg(args, w, W, R, msa, torch, device="cuda"):
             ach = tw[key] / (per / 1000.0) / 1e12
             res["kernels"][name] = {"ms_per_launch": per, "launches": n, "flops_per_launch": tw[key],
                                     "bound": "alu", "achieved": ach, "frac": ach / peak}
+    return res
+
+
+def decode_result(name, d_ms, L, dw, dk, scan_ms, peaks, peak_src):
+    """Decode step against its HBM roofline.  Two denominators, each labelled:
+    the measured copy bandwidth (hbm_gbs: a read + write stream) and the
+    nominal HBM3e bandwidth.  A read-only stream (the index-key scan) can run
+    above the copy figure, which pays for read-write turnarounds; part of the
+    index keys can also stay in L2 between timed steps."""
+    achieved_scan = None if scan_ms is None else dw["index_bytes"] / (scan_ms / 1000.0) / 1e9
+    return {"workload": name, "us_per_step": d_ms * 1000.0, "sum_L": sum(L),
+            "algorithmic_bytes": dw["bytes"],
+            "roofline_us": dw["bytes"] / (peaks["hbm_gbs"] * 1e9) * 1e6,
+            "frac": dw["bytes"] / (peaks["hbm_gbs"] * 1e9) / (d_ms / 1000.0),
+            "frac_of_spec_hbm": dw["bytes"] / (HBM_SPEC_GBS * 1e9) / (d_ms / 1000.0),
+            "peak_source": f"hbm_gbs {peaks['hbm_gbs']:.0f} GB/s ({peak_src} copy); spec {HBM_SPEC_GBS:.0f} GB/s",
+            "scan_kernel": None if scan_ms is None else {
+                "bound": "hbm", "achieved": achieved_scan, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved_scan / peaks["hbm_gbs"], "frac_of_spec_hbm": achieved_scan / HBM_SPEC_GBS},
+            "kernels": dk}
+
+
+def decode_leg(args, W, R, msa, torch, peaks, peak_src):
+    """Decode step of args.decode_workload (one query per sequence against its
+    cache), timed by CUDA events over max(5, steps) steps after 3 warm-up ones,
+    with the library's per-kernel events."""
+    wd = W.WORKLOADS[args.decode_workload]
+    dinp = W.make_inputs(wd, "cuda")
+    dctx = make_ctx(wd, dinp, torch, msa)
+    for _ in range(3):
+        step_decode(dctx, msa)
+    torch.cuda.synchronize()
+    device_errors(dctx, msa)
+    msa.msa_profile_reset()
+    msa.msa_profile_enable(True)
+    d_steps = max(5, args.steps)
+    d_ms = time_steps(lambda: step_decode(dctx, msa), d_steps, torch) / d_steps
+    msa.msa_profile_enable(False)
+    device_errors(dctx, msa)
+    L = [dinp["cu_k_host"][i + 1] - dinp["cu_k_host"][i] for i in range(wd.batch)]
+    dw = R.decode_work(L, wd.H, wd.G, wd.d, wd.d_idx, wd.B_k, wd.k)
+    dk = {}
+    for name in ("decode_scan", "decode_select", "rows_attn", "sparse_attn", "combine", "count", "scatter", "plan"):
+        kms, n = msa.msa_profile_read(name)
+        if n:
+            dk[name] = {"ms_per_launch": kms / n, "launches": n}
+    scan_ms = dk.get("decode_scan", {}).get("ms_per_launch")
+    res = decode_result(args.decode_workload, d_ms, L, dw, dk, scan_ms, peaks, peak_src)
+    del dctx, dinp
+    torch.cuda.empty_cache()
+    return res
+
+
+def config_leg(args, name, W, R, msa, torch, peaks, peak_t, peak_t_src):
+    """One more prefill configuration (the 32K layer, the 1M layer in passes of
+    131072 query rows): ms per step, query tokens/s and the step against its
+    roofline, timed by CUDA events after 3 warm-up steps (inputs larger than
+    L2).  Not the headline line."""
+    w = W.WORKLOADS[name]
+    inp = W.make_inputs(w, "cuda")
+    make_ctx.q_chunk = -1
+    ctx = make_ctx(w, inp, torch, msa)
+    for _ in range(3):
+        step_prefill(ctx, msa)
+    torch.cuda.synchronize()
+    device_errors(ctx, msa)
+    steps = 3 if ctx["T"] > 131072 else max(5, args.steps)
+    msa.msa_profile_reset()
+    msa.msa_profile_enable(True)
+    ms = time_steps(lambda: step_prefill(ctx, msa), steps, torch) / steps
+    msa.msa_profile_enable(False)
+    device_errors(ctx, msa)
+    S_lens = [inp["cu_k_host"][i + 1] - inp["cu_k_host"][i] for i in range(len(inp["cu_k_host"]) - 1)]
+    T_lens = [inp["cu_q_host"][i + 1] - inp["cu_q_host"][i] for i in range(len(inp["cu_q_host"]) - 1)]
+    work = R.prefill_work(S_lens, T_lens, w.H, w.G, w.d, w.d_idx, w.B_k, w.k)
+    t_b = max(work["flops"] / (peaks["bf16_tflops"] * 1e12), work["bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    t_s = max(work["flops"] / (peaks["bf16_tflops_sustained"] * 1e12), work["bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    ks = {}
+    for kn in ("index_topk_prefill", "tile_plan", "tile_attn", "sparse_attn", "combine"):
+        kms, n = msa.msa_profile_read(kn)
+        if n:
+            ks[kn] = {"ms_per_step": kms / steps, "launches_per_step": n / steps}
+    res = {"workload": name, "T": ctx["T"], "steps": steps, "warmup": 3, "ms_per_step": ms,
+           "value": ctx["T"] / (ms / 1000.0), "unit": "tokens/s",
+           "attention_pass_rows": ctx["q_chunk"] or ctx["T"],
+           "roofline_ms_burst": t_b, "roofline_ms_sustained": t_s,
+           "frac_burst": t_b / ms, "frac_sustained": t_s / ms, "kernels": ks}
+    del ctx, inp
     return res
 
 
@@ -422,14 +527,14 @@ def run_reference(args):
             times.append(dt)
     sec = sum(times)
     rate = per_step * len(times) / sec
-    cores = blas_threads() or len(os.sched_getaffinity(0))
+    cores = len(os.sched_getaffinity(0))
     sample = f"{per_step} random query rows of {args.workload} per step (of {T}); oracle selection + main branch"
     line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * sec / len(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": run_config(args, w, T, args.gpus),
-            "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "blas_threads": blas_threads(),
+                             "kind": "oracle", "sample": sample},
             "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -455,7 +560,16 @@ def run_ours(args):
     B.build()
     msa.load_library()
     msa.msa_set_tile_threshold(args.theta)
+    if args.window:
+        msa.msa_set_attn_window(args.window)
     peaks, peak_src = load_peaks()
+    if args.decode_only:
+        if rank == 0:
+            print(json.dumps({"metric": "decode µs/step (decode leg alone: a profiling run, not the headline)",
+                              "decode": decode_leg(args, W, R, msa, torch, peaks, peak_src)}), flush=True)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
 
     def tile_theta(w_):
         if args.theta >= 0:
@@ -526,15 +640,20 @@ def run_ours(args):
         per_kernel_work.update({"tile_attn": ("tensor", split["tile_flops"]),
                                 "sparse_attn": ("tensor", split["kv_flops"]),
                                 "combine": ("hbm", split["combine_bytes"])})
-    peak_t = peaks["bf16_tflops_sustained"]
+    peak_t, peak_t_src = tensor_peak(peaks, peak_src, clk)
     for name, v in kernels.items():
         if name in per_kernel_work:
             bound, units = per_kernel_work[name]
             per = units / (v["launches"] / args.steps)
             v["algorithmic_per_launch"] = per
             v["achieved"] = per / (v["ms_per_launch"] / 1000.0) / (1e12 if bound == "tensor" else 1e9)
-            v["frac"] = v["achieved"] / (peak_t if bound == "tensor" else peaks["hbm_gbs"])
-    # roofline of the dominant kernel (timed inside a long step: sustained peak)
+            if bound == "tensor":
+                v["frac"] = v["achieved"] / peak_t
+                v["frac_burst"] = v["achieved"] / peaks["bf16_tflops"]
+                v["frac_sustained"] = v["achieved"] / peaks["bf16_tflops_sustained"]
+            else:
+                v["frac"] = v["achieved"] / peaks["hbm_gbs"]
+    # roofline of the dominant kernel, against the peak the sampled clocks support
     dom = max((n for n in kernels if n in per_kernel_work),
               key=lambda n: kernels[n]["ms_per_launch"] * kernels[n]["launches"])
     bound = per_kernel_work[dom][0]
@@ -542,10 +661,13 @@ def run_ours(args):
             "peak": peak_t if bound == "tensor" else peaks["hbm_gbs"],
             "unit": "TFLOP/s" if bound == "tensor" else "GB/s", "frac": kernels[dom]["frac"],
             "traffic": traffic_for(dom), "algorithmic_per_launch": kernels[dom]["algorithmic_per_launch"],
-            "peak_source": (f"bf16_tflops_sustained ({peak_src})" if bound == "tensor"
-                            else f"hbm_gbs ({peak_src})")}
+            "peak_source": peak_t_src if bound == "tensor" else f"hbm_gbs ({peak_src})"}
+    if bound == "tensor":
+        roof["frac_burst"] = kernels[dom]["frac_burst"]
+        roof["frac_sustained"] = kernels[dom]["frac_sustained"]
     t_roof_ms = max(work["flops"] / (peaks["bf16_tflops"] * 1e12), work["bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3
-    t_roof_sus = max(work["flops"] / (peak_t * 1e12), work["bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    t_roof_sus = max(work["flops"] / (peaks["bf16_tflops_sustained"] * 1e12),
+                     work["bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3
     step_roof = {"flops": work["flops"], "index_flops": work["index_flops"], "main_flops": work["main_flops"],
                  "bytes": work["bytes"], "roofline_ms_burst": t_roof_ms, "roofline_ms_sustained": t_roof_sus,
                  "frac_burst": t_roof_ms / ms_step, "frac_sustained": t_roof_sus / ms_step,
@@ -599,56 +721,35 @@ def run_ours(args):
         dense = {"workload": args.workload, "ms": dms, "flops": dfl,
                  "achieved_tflops": dfl / (dms / 1000.0) / 1e12,
                  "frac": dfl / (dms / 1000.0) / 1e12 / peak_t,
+                 "frac_burst": dfl / (dms / 1000.0) / 1e12 / peaks["bf16_tflops"],
+                 "frac_sustained": dfl / (dms / 1000.0) / 1e12 / peaks["bf16_tflops_sustained"],
                  "speedup_step": dms / ms_step, "speedup_main_branch": dms / main_ms,
                  "flops_ratio": dfl / work["main_flops"]}
         del dws
 
+    # dense GQA done: the prefill context's workspace is no longer needed
+    ctx = None
+    torch.cuda.empty_cache()
     # decode: 32 sequences with caches of 128K..1M tokens
     decode = None
     cpu = None
     if rank == 0 and not args.no_decode:
-        del ctx
-        torch.cuda.empty_cache()
-        wd = W.WORKLOADS[DECODE]
-        dinp = W.make_inputs(wd, "cuda")
-        dctx = make_ctx(wd, dinp, torch, msa)
-        for _ in range(3):
-            step_decode(dctx, msa)
-        torch.cuda.synchronize()
-        device_errors(dctx, msa)
-        msa.msa_profile_reset()
-        msa.msa_profile_enable(True)
-        d_steps = max(5, args.steps)
-        d_ms = time_steps(lambda: step_decode(dctx, msa), d_steps, torch) / d_steps
-        msa.msa_profile_enable(False)
-        device_errors(dctx, msa)
-        L = [dinp["cu_k_host"][i + 1] - dinp["cu_k_host"][i] for i in range(wd.batch)]
-        dw = R.decode_work(L, wd.H, wd.G, wd.d, wd.d_idx, wd.B_k, wd.k)
-        dk = {}
-        for name in ("decode_scan", "decode_select", "rows_attn", "sparse_attn", "combine", "count", "scatter", "plan"):
-            kms, n = msa.msa_profile_read(name)
-            if n:
-                dk[name] = {"ms_per_launch": kms / n, "launches": n}
-        scan_ms = dk.get("decode_scan", {}).get("ms_per_launch")
-        decode = {"workload": DECODE, "us_per_step": d_ms * 1000.0, "sum_L": sum(L),
-                  "algorithmic_bytes": dw["bytes"],
-                  "roofline_us": dw["bytes"] / (peaks["hbm_gbs"] * 1e9) * 1e6,
-                  "frac": dw["bytes"] / (peaks["hbm_gbs"] * 1e9) / (d_ms / 1000.0),
-                  "scan_kernel": None if scan_ms is None else {
-                      "bound": "hbm", "achieved": dw["index_bytes"] / (scan_ms / 1000.0) / 1e9,
-                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                      "frac": dw["index_bytes"] / (scan_ms / 1000.0) / 1e9 / peaks["hbm_gbs"]},
-                  "kernels": dk}
-        del dctx, dinp
-        torch.cuda.empty_cache()
+        decode = decode_leg(args, W, R, msa, torch, peaks, peak_src)
+    # the other prefill configurations, one line each (not the headline)
+    configs = None
+    if rank == 0 and world == 1 and args.configs:
+        configs = {}
+        for name in [c for c in args.configs.split(",") if c]:
+            configs[name] = config_leg(args, name, W, R, msa, torch, peaks, peak_t, peak_t_src)
+            torch.cuda.empty_cache()
     training = None
     if rank == 0 and args.training:
         training = training_leg(args, w, W, R, msa, torch)
         torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, n_rows, secs = cpu_oracle_rate(w, inp, args.cpu_budget, torch, np)
-        cores = blas_threads() or len(os.sched_getaffinity(0))
-        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+        cores = len(os.sched_getaffinity(0))
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "blas_threads": blas_threads(), "kind": "oracle",
                "sample": f"{n_rows} random query rows of {args.workload} ({secs:.1f} s of fp64 oracle work: "
                          f"selection + main branch per row)"}
 
@@ -659,7 +760,7 @@ def run_ours(args):
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": run_config(args, w, T_layer, world),
                 "roofline": roof, "step_roofline": step_roof, "tile_split": split, "dense_gqa": dense,
-                "decode": decode, "e2e": e2e,
+                "decode": decode, "configs": configs, "e2e": e2e,
                 "cpu_baseline": cpu, "clocks": clk, "gpu_launches": launches, "kernels": kernels}
         if training is not None:
             line["training"] = training
@@ -679,6 +780,11 @@ def build_parser():
     ap.add_argument("--T", type=int, default=0, help="shorter prefill (same heads/dims), for profiling")
     ap.add_argument("--index-only", action="store_true", help="time only the index branch (for profiling)")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-workload", default=DECODE, help="decode workload of the decode leg")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the decode leg and print its line (for profiler captures)")
+    ap.add_argument("--configs", default="prefill_n32768,prefill_n1048576_hot2",
+                    help="other prefill workloads timed after the headline (comma list; empty: none)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense causal GQA comparison")
@@ -686,6 +792,8 @@ def build_parser():
                     help="query rows per attention pass (-1: 131072 above 128K tokens, else one pass)")
     ap.add_argument("--theta", type=int, default=-1,
                     help="query-tile threshold of the prefill (-1 automatic, 0 off)")
+    ap.add_argument("--window", type=int, default=0,
+                    help="query rows per planning window of the KV-outer lists (0: the library's default)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--training", action="store_true",

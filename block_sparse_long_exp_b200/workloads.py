@@ -63,6 +63,11 @@ WORKLOADS: Dict[str, Workload] = {
                  hot_frac=0.02),
         Workload("prefill_n1048576_hot2", "prefill", H=64, G=4, d=128, d_idx=64,
                  B_k=128, k=16, seed=4, T=1048576, hot_frac=0.02),
+        # a smaller decode batch of the same shape for profiler captures: its
+        # index keys (~0.4 GB) still exceed L2, its K/V caches are ~6 GB
+        Workload("decode_b4_l512k_1m_hot2", "decode", H=64, G=4, d=128, d_idx=64,
+                 B_k=128, k=16, seed=5, batch=4, L_min=524288, L_max=1048576,
+                 hot_frac=0.02),
     ]
 }
 
