@@ -31,7 +31,7 @@ msa_status_t check_shape(const msa_shape_t* s) {
   if (s->G != 1 && s->G != 2 && s->G != 4) return MSA_ERR_UNSUPPORTED;
   if (s->d != 64 && s->d != 128) return MSA_ERR_UNSUPPORTED;
   if (s->d_idx != 32 && s->d_idx != 64 && s->d_idx != 128) return MSA_ERR_UNSUPPORTED;
-  if (s->B_k != kBk) return MSA_ERR_UNSUPPORTED;
+  if (s->B_k != 32 && s->B_k != 64 && s->B_k != kBk) return MSA_ERR_UNSUPPORTED;
   if (s->k < 1 || s->k > kMaxK) return MSA_ERR_UNSUPPORTED;
   if (!(s->sm_scale > 0.f) || s->sm_scale != s->sm_scale) return MSA_ERR_INVALID_ARG;
   return MSA_OK;
@@ -45,6 +45,14 @@ msa_status_t check_seqs(const msa_varlen_t* v) {
   if (v->max_q_len > v->total_q || v->max_k_len > v->total_k) return MSA_ERR_INVALID_ARG;  // a length beyond its total
   if (v->total_k > (int64_t)INT32_MAX - 256 || v->total_q > (int64_t)INT32_MAX / kMaxK) return MSA_ERR_UNSUPPORTED;
   return MSA_OK;
+}
+
+// Entry points built for 128-token blocks only (the training-side kernels,
+// the selection variants and paged caches, whose pages are 128-row blocks).
+msa_status_t check_shape_bk128(const msa_shape_t* s) {
+  const msa_status_t st = check_shape(s);
+  if (st != MSA_OK) return st;
+  return s->B_k == kBk ? MSA_OK : MSA_ERR_UNSUPPORTED;
 }
 
 }  // namespace msa
@@ -62,7 +70,7 @@ bool ws_ok(const void* ws, size_t have, size_t need) {
   return ws != nullptr && (reinterpret_cast<uintptr_t>(ws) % kAlign) == 0 && have >= need;
 }
 
-int64_t total_blocks_bound(const msa_varlen_t* v) { return (v->total_k + kBk - 1) / kBk + v->batch; }
+int64_t total_blocks_bound(const msa_varlen_t* v, int B_k) { return (v->total_k + B_k - 1) / B_k + v->batch; }
 
 // Slices of a sparse-attention workspace for chunks of `rows` query rows.
 struct AttnLayout {
@@ -77,7 +85,7 @@ AttnLayout attn_layout(const msa_shape_t* s, const msa_varlen_t* v, int64_t rows
   const int hg = s->H / s->G;
   const int qpt = 128 / (hg < 8 ? 8 : hg);            // queries per 128-row tile
   L.qpi = 8 * qpt < kMaxItemQueries ? 8 * qpt : kMaxItemQueries;
-  L.nlists = (int64_t)s->G * total_blocks_bound(v);
+  L.nlists = (int64_t)s->G * total_blocks_bound(v, s->B_k);
   L.win = attn_window_rows();
   const int64_t nkeys = ((rows + L.win - 1) / L.win) * L.nlists;
   const int64_t nentries = rows * s->G * s->k;
@@ -143,6 +151,7 @@ msa_status_t attn_common(const msa_shape_t* shape, const msa_varlen_t* seqs, con
   a.q = q; a.key = k; a.value = v; a.sel = sel; a.out = out; a.lse = lse;
   a.cu_q = seqs->cu_q; a.cu_k = seqs->cu_k;
   a.batch = seqs->batch; a.H = shape->H; a.G = shape->G; a.d = shape->d; a.k = shape->k;
+  a.B_k = shape->B_k;
   a.sm_scale = shape->sm_scale;
   a.total_q = seqs->total_q; a.total_k = seqs->total_k;
   a.max_q_len = seqs->max_q_len; a.max_k_len = seqs->max_k_len;
@@ -187,7 +196,7 @@ struct PagedLayout {
 };
 
 msa_status_t check_paged(const msa_shape_t* s, const msa_paged_t* pg) {
-  msa_status_t st = check_shape(s);
+  msa_status_t st = check_shape_bk128(s);
   if (st != MSA_OK) return st;
   if (pg == nullptr || pg->seqlens == nullptr || pg->block_table == nullptr) return MSA_ERR_INVALID_ARG;
   if (pg->batch < 1 || pg->max_blocks < 1 || pg->num_pages < 1 || pg->max_seqlen < 1) return MSA_ERR_INVALID_ARG;
@@ -210,7 +219,7 @@ PagedLayout paged_layout(const msa_shape_t* s, const msa_paged_t* pg) {
   L.cu_q = take(sizeof(int32_t) * (pg->batch + 1));
   L.cu_k = take(sizeof(int32_t) * (pg->batch + 1));
   L.tile_ctr = take(sizeof(int32_t) * 4);
-  L.idx_scratch = take(decode_index_scratch_bytes(pg->batch, L.total_k, s->G, s->k));
+  L.idx_scratch = take(decode_index_scratch_bytes(pg->batch, L.total_k, s->G, kBk));
   L.total = off;
   return L;
 }
@@ -264,7 +273,7 @@ size_t msa_index_topk_workspace_size(const msa_shape_t* shape, const msa_varlen_
   if (seqs->max_q_len > 1 && seqs->batch > kMaxBatchTiles) return 0;
   size_t need = kWsHeader;
   if (seqs->max_q_len <= 1)
-    need += align_up(decode_index_scratch_bytes(seqs->batch, seqs->total_k, shape->G, shape->k), kAlign);
+    need += align_up(decode_index_scratch_bytes(seqs->batch, seqs->total_k, shape->G, shape->B_k), kAlign);
   return need;
 }
 
@@ -285,7 +294,7 @@ msa_status_t msa_index_topk(const msa_shape_t* shape, const msa_varlen_t* seqs, 
   IndexTopkArgs a{};
   a.q_idx = q_idx; a.k_idx = k_idx; a.sel = sel;
   a.cu_q = seqs->cu_q; a.cu_k = seqs->cu_k;
-  a.batch = seqs->batch; a.G = shape->G; a.d_idx = shape->d_idx; a.k = shape->k;
+  a.batch = seqs->batch; a.G = shape->G; a.d_idx = shape->d_idx; a.k = shape->k; a.B_k = shape->B_k;
   a.total_q = seqs->total_q; a.total_k = seqs->total_k;
   a.max_q_len = seqs->max_q_len; a.max_k_len = seqs->max_k_len;
   a.err = static_cast<DevError*>(ws);
@@ -298,6 +307,36 @@ msa_status_t msa_index_topk(const msa_shape_t* shape, const msa_varlen_t* seqs, 
     rc = launch_index_topk_prefill(a, stream);
   }
   return rc == 0 ? MSA_OK : MSA_ERR_CUDA;
+}
+
+msa_status_t msa_index_topk_decode_candidates(const msa_shape_t* shape, const msa_varlen_t* seqs,
+                                              const void* q_idx, const void* k_idx, int32_t all_blocks,
+                                              int32_t* cand_ids, float* cand_scores, void* ws, size_t ws_bytes,
+                                              void* stream) {
+  msa_status_t st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  st = check_seqs(seqs);
+  if (st != MSA_OK) return st;
+  if (seqs->max_q_len > 1) return MSA_ERR_INVALID_ARG;          // one query per sequence
+  if (all_blocks != 0 && all_blocks != 1) return MSA_ERR_INVALID_ARG;
+  const bool any = seqs->total_q > 0 && shape->k > 1;          // k = 1: no candidates, only the local block
+  if (any && (!q_idx || !k_idx || !cand_ids || !cand_scores)) return MSA_ERR_INVALID_ARG;
+  const size_t need = msa_index_topk_workspace_size(shape, seqs);
+  if (!ws_ok(ws, ws_bytes, need)) return MSA_ERR_WORKSPACE;
+  if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  if (!any) return MSA_OK;
+  IndexTopkArgs a{};
+  a.q_idx = q_idx; a.k_idx = k_idx; a.sel = cand_ids; a.cand_score = cand_scores;
+  a.all_blocks = all_blocks;
+  a.cu_q = seqs->cu_q; a.cu_k = seqs->cu_k;
+  a.batch = seqs->batch; a.G = shape->G; a.d_idx = shape->d_idx; a.k = shape->k; a.B_k = shape->B_k;
+  a.total_q = seqs->total_q; a.total_k = seqs->total_k;
+  a.max_q_len = seqs->max_q_len; a.max_k_len = seqs->max_k_len;
+  a.err = static_cast<DevError*>(ws);
+  a.scratch = static_cast<uint8_t*>(ws) + kWsHeader;
+  a.scratch_bytes = ws_bytes - kWsHeader;
+  return launch_index_topk_decode(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
 }
 
 size_t msa_sparse_attn_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs, int64_t q_chunk) {
@@ -383,7 +422,7 @@ msa_status_t msa_index_topk_decode_paged(const msa_shape_t* shape, const msa_pag
   IndexTopkArgs a{};
   a.q_idx = q_idx; a.k_idx = k_idx_pages; a.sel = sel;
   a.cu_q = cu_q; a.cu_k = cu_k;
-  a.batch = pages->batch; a.G = shape->G; a.d_idx = shape->d_idx; a.k = shape->k;
+  a.batch = pages->batch; a.G = shape->G; a.d_idx = shape->d_idx; a.k = shape->k; a.B_k = kBk;
   a.total_q = pages->batch; a.total_k = L.total_k;
   a.max_q_len = 1; a.max_k_len = pages->max_seqlen;
   a.err = reinterpret_cast<DevError*>(ws);
@@ -412,7 +451,7 @@ msa_status_t msa_sparse_attn_decode_paged(const msa_shape_t* shape, const msa_pa
   AttnArgs a{};
   a.q = q; a.key = k_pages; a.value = v_pages; a.sel = sel; a.out = out; a.lse = lse;
   a.cu_q = cu_q; a.cu_k = cu_k;
-  a.batch = pages->batch; a.H = shape->H; a.G = shape->G; a.d = shape->d; a.k = shape->k;
+  a.batch = pages->batch; a.H = shape->H; a.G = shape->G; a.d = shape->d; a.k = shape->k; a.B_k = kBk;
   a.sm_scale = shape->sm_scale;
   a.total_q = pages->batch; a.total_k = L.total_k;
   a.max_q_len = 1; a.max_k_len = pages->max_seqlen;
@@ -427,7 +466,7 @@ static msa_status_t index_kl_common(const msa_shape_t* shape, const msa_varlen_t
                                    const void* q_idx, const void* k_idx, const int32_t* sel, const float* lse,
                                    float tau, int32_t dense, void* ws, size_t ws_bytes, void* stream,
                                    IndexKlArgs* a) {
-  msa_status_t st = check_shape(shape);
+  msa_status_t st = check_shape_bk128(shape);
   if (st != MSA_OK) return st;
   st = check_seqs(seqs);
   if (st != MSA_OK) return st;
@@ -481,7 +520,7 @@ msa_status_t msa_index_kl_backward(const msa_shape_t* shape, const msa_varlen_t*
 
 msa_status_t msa_select_window(const msa_shape_t* shape, const msa_varlen_t* seqs, int32_t n_sink, int32_t* sel,
                                void* ws, size_t ws_bytes, void* stream) {
-  msa_status_t st = check_shape(shape);
+  msa_status_t st = check_shape_bk128(shape);
   if (st != MSA_OK) return st;
   st = check_seqs(seqs);
   if (st != MSA_OK) return st;
@@ -501,7 +540,7 @@ msa_status_t msa_sparse_attn_backward(const msa_shape_t* shape, const msa_varlen
                                       const void* k, const void* v, const int32_t* sel, const void* out,
                                       const float* lse, const void* dout, int32_t dense, float* dq, float* dk,
                                       float* dv, void* ws, size_t ws_bytes, void* stream) {
-  msa_status_t st = check_shape(shape);
+  msa_status_t st = check_shape_bk128(shape);
   if (st != MSA_OK) return st;
   st = check_seqs(seqs);
   if (st != MSA_OK) return st;
@@ -536,7 +575,7 @@ msa_status_t msa_selected_share(const float* lse_sel, const float* lse_all, int6
 msa_status_t msa_index_topk_policy(const msa_shape_t* shape, const msa_varlen_t* seqs, int32_t n_sink,
                                    int32_t n_local, const void* q_idx, const void* k_idx, int32_t* sel, void* ws,
                                    size_t ws_bytes, void* stream) {
-  msa_status_t st = check_shape(shape);
+  msa_status_t st = check_shape_bk128(shape);
   if (st != MSA_OK) return st;
   st = check_seqs(seqs);
   if (st != MSA_OK) return st;

@@ -38,12 +38,13 @@ __device__ __forceinline__ int find_seq(const int32_t* __restrict__ cu, int batc
   return lo;
 }
 
-__global__ void block_offsets_kernel(const int32_t* __restrict__ cu_k, int batch, int32_t* __restrict__ blk_off) {
+__global__ void block_offsets_kernel(const int32_t* __restrict__ cu_k, int batch, int B_k,
+                                     int32_t* __restrict__ blk_off) {
   if (threadIdx.x == 0 && blockIdx.x == 0) {
     int acc = 0;
     for (int b = 0; b < batch; ++b) {
       blk_off[b] = acc;
-      acc += (cu_k[b + 1] - cu_k[b] + kBk - 1) / kBk;
+      acc += (cu_k[b + 1] - cu_k[b] + B_k - 1) / B_k;
     }
     blk_off[batch] = acc;
   }
@@ -51,14 +52,14 @@ __global__ void block_offsets_kernel(const int32_t* __restrict__ cu_k, int batch
 
 // Validates an entry and returns its block's index over the whole batch
 // (blk_off[b] + blk), or -1 (slot empty or invalid).
-__device__ __forceinline__ int entry_block(int blk, int64_t t, int batch, const int32_t* cu_q, const int32_t* cu_k,
-                                           const int32_t* blk_off, DevError* err) {
+__device__ __forceinline__ int entry_block(int blk, int64_t t, int batch, int B_k, const int32_t* cu_q,
+                                           const int32_t* cu_k, const int32_t* blk_off, DevError* err) {
   if (blk < 0) return -1;
   const int b = find_seq(cu_q, batch, t);
   const int Tb = cu_q[b + 1] - cu_q[b];
   const int Sb = cu_k[b + 1] - cu_k[b];
   const int64_t pos = (int64_t)Sb - Tb + (t - cu_q[b]);
-  if (Tb > Sb || blk > pos / kBk) {
+  if (Tb > Sb || blk > pos / B_k) {
     report_error(err, MSA_ERR_DEVICE_CHECK, kSiteInvert, (int)t, blk);
     return -1;
   }
@@ -81,7 +82,8 @@ __device__ __forceinline__ int entry_block(int blk, int64_t t, int batch, const 
 // combine-list entry {pair, number of packed partials}.
 template <bool kScatter>
 __global__ void count_scatter_kernel(const int32_t* __restrict__ sel, int64_t t0, int64_t t1, int G, int k,
-                                     int batch, const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_k,
+                                     int batch, int B_k, const int32_t* __restrict__ cu_q,
+                                     const int32_t* __restrict__ cu_k,
                                      const int32_t* __restrict__ blk_off, int64_t nblocks, int64_t nwin,
                                      int win_rows, const uint32_t* __restrict__ dmask, int32_t* __restrict__ counter,
                                      uint32_t* __restrict__ entries, uint2* __restrict__ clist, DevError* err) {
@@ -103,7 +105,7 @@ __global__ void count_scatter_kernel(const int32_t* __restrict__ sel, int64_t t0
       const int32_t blk = sel[(t * G + g) * k + s];
       packed = first + __popc(live & ~covered);
       if (blk >= 0) live |= 1u << s;
-      const int gb = entry_block(blk, t, batch, cu_q, cu_k, blk_off, err);
+      const int gb = entry_block(blk, t, batch, B_k, cu_q, cu_k, blk_off, err);
       if (gb >= 0 && !((covered >> s) & 1u)) key = wbase + gb;
     }
     // warp-aggregated atomics: lanes with the same key share one atomic
@@ -295,7 +297,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                    const __grid_constant__ CUtensorMap tm_q, const Item* __restrict__ items,
                    const int32_t* __restrict__ nitems_p, int32_t* __restrict__ ticket,
                    const uint32_t* __restrict__ entries, const int32_t* __restrict__ cu_q,
-                   const int32_t* __restrict__ cu_k, int H, int G, int d, int k, float scale_log2,
+                   const int32_t* __restrict__ cu_k, int H, int G, int d, int k, int B_k, float scale_log2,
                    int64_t t0, __half* __restrict__ part_acc, float* __restrict__ part_lse, DevError* err) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -395,7 +397,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         if (ok) {
           uint8_t* ks = kv_s + st * 2 * tile_bytes;
           mbar_arrive_expect_tx(&ctl->kv_full[st], 2 * tile_bytes);
-          const int krow = cu_k[I.seq] + I.blk * kBk;
+          // the 128-row K/V tile starting at the block: B_k rows of it are the block
+          const int krow = cu_k[I.seq] + I.blk * B_k;
           for (int h = 0; h < nhalf; ++h) {
             tma_load_3d(ks + h * 128 * 128, &tm_k, &ctl->kv_full[st], 64 * h, I.g, krow);
             tma_load_3d(ks + tile_bytes + h * 128 * 128, &tm_v, &ctl->kv_full[st], 64 * h, I.g, krow);
@@ -532,7 +535,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       if (count <= 0) { release_item(n, true); break; }
       const int Tb = R->Tb, Sb = R->Sb;
       const int64_t qrow0 = R->qrow0;
-      const int64_t blk_first = (int64_t)R->blk * kBk;
+      const int64_t blk_first = (int64_t)R->blk * B_k;
       const int ntiles = (count + qpt - 1) / qpt;
       // the item stays in the ring until this warpgroup's last tile of it
       for (int mt = 0; mt < ntiles; ++mt, ++tau) {
@@ -540,11 +543,12 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         const int idx = mt * qpt + ql;
         const bool valid = ql < qpt && idx < count && hi < Hg;
         const uint32_t e = valid ? entries[R->start + idx] : 0u;
-        int limit = 127;
+        // last attended key of the tile: the block's last (B_k - 1), or the causal cut
+        int limit = B_k - 1;
         if (valid) {
           const int64_t t = t0 + e / k;
           const int64_t lim = (int64_t)Sb - Tb + (t - qrow0) - blk_first;
-          limit = lim >= 127 ? 127 : (int)lim;
+          limit = lim >= B_k - 1 ? B_k - 1 : (int)lim;
         }
         if (!mbar_wait(&ctl->s_full[wg], (tau >> 1) & 1)) {
           report_error(err, MSA_ERR_TIMEOUT, kSiteAttnSoftmax, tau, 0);
@@ -891,7 +895,9 @@ combine_kernel(const __half* __restrict__ part_acc, const float* __restrict__ pa
       float wsum = 0.f;
 #pragma unroll 4
       for (int s2 = 0; s2 < n; ++s2) {
-        const float w = ((valid >> s2) & 1u) ? __expf(lse_s[s2 * Hg + i] - m_) : 0.f;
+        // an unused slot is skipped, not weighted by 0: its buffer may hold anything (NaN included)
+        if (!((valid >> s2) & 1u)) continue;
+        const float w = __expf(lse_s[s2 * Hg + i] - m_);
         wsum += w;
         const uint4 rv = *reinterpret_cast<const uint4*>(acc_s + ((s2 * (d / 8) + cc) * Hg + i) * 8);
         const __half2* hp = reinterpret_cast<const __half2*>(&rv);
@@ -958,7 +964,7 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
   cudaError_t e;
   {
     ProfScope p("block_offsets", stream);
-    block_offsets_kernel<<<1, 32, 0, st>>>(a.cu_k, a.batch, a.blk_off);
+    block_offsets_kernel<<<1, 32, 0, st>>>(a.cu_k, a.batch, a.B_k, a.blk_off);
   }
   const int win = a.win_rows;
   const int64_t nwin = (nrows + win - 1) / win;
@@ -978,7 +984,7 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
   const int cs_blocks = (int)((nthreads + 255) / 256);
   {
     ProfScope p("count", stream);
-    count_scatter_kernel<false><<<cs_blocks, 256, 0, st>>>(a.sel, a.t0, a.t1, a.G, a.k, a.batch, a.cu_q, a.cu_k,
+    count_scatter_kernel<false><<<cs_blocks, 256, 0, st>>>(a.sel, a.t0, a.t1, a.G, a.k, a.batch, a.B_k, a.cu_q, a.cu_k,
                                                            a.blk_off, nblocks, nwin, win, dmask, a.counts, nullptr,
                                                            tiles ? nullptr : a.clist, a.err);
   }
@@ -993,7 +999,7 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
   }
   {
     ProfScope p("scatter", stream);
-    count_scatter_kernel<true><<<cs_blocks, 256, 0, st>>>(a.sel, a.t0, a.t1, a.G, a.k, a.batch, a.cu_q, a.cu_k,
+    count_scatter_kernel<true><<<cs_blocks, 256, 0, st>>>(a.sel, a.t0, a.t1, a.G, a.k, a.batch, a.B_k, a.cu_q, a.cu_k,
                                                           a.blk_off, nblocks, nwin, win, dmask, a.cursor, a.entries,
                                                           nullptr,
                                                           a.err);
@@ -1030,7 +1036,7 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
   {
     ProfScope p("sparse_attn", stream);
     sparse_attn_kernel<<<nsm, kAttnThreads, smem, st>>>(
-        tm_k, tm_v, tm_q, a.items, a.nitems, a.nitems + 1, a.entries, a.cu_q, a.cu_k, a.H, a.G, a.d, a.k,
+        tm_k, tm_v, tm_q, a.items, a.nitems, a.nitems + 1, a.entries, a.cu_q, a.cu_k, a.H, a.G, a.d, a.k, a.B_k,
         scale_log2, a.t0, reinterpret_cast<__half*>(a.part_acc), a.part_lse, a.err);
   }
   e = cudaGetLastError();

@@ -4,10 +4,11 @@
 // sec. 二).
 //
 // The step is bound by HBM: every cached index key (d_idx bf16) is read once.
-//   scan   : a CTA takes CB consecutive blocks of one sequence; TMA brings each
-//            [128 x d_idx] block into swizzled shared memory; one warp per block
-//            computes the 128 x G scores with mma.sync (bf16 in, fp32 out;
-//            the G index-query heads padded to n = 8) and max-pools them.
+//   scan   : a CTA takes CB consecutive 128-key tiles of one sequence; TMA
+//            brings each [128 x d_idx] tile into swizzled shared memory; one
+//            warp per tile computes the 128 x G scores with mma.sync (bf16 in,
+//            fp32 out; the G index-query heads padded to n = 8) and max-pools
+//            them per block of B_k keys (128 / B_k blocks per tile).
 //   select : one CTA per (sequence, group): per-thread top-(k-1) over a strided
 //            slice of the block scores, then k-1 rounds of block-wide argmax on
 //            64-bit keys (score, then lower block index).
@@ -22,9 +23,9 @@ constexpr int kCB = 4;            // blocks per scan CTA (one warp each)
 constexpr int kScanThreads = 32 * kCB;
 constexpr int kSelThreads = 256;
 
-size_t scratch_layout(int32_t batch, int64_t total_k, int32_t G, size_t* bscore_off, size_t* blk_off_off,
-                      size_t* chunk_off_off) {
-  const int64_t nblocks = (total_k + kBk - 1) / kBk + batch;
+size_t scratch_layout(int32_t batch, int64_t total_k, int32_t G, int32_t B_k, size_t* bscore_off,
+                      size_t* blk_off_off, size_t* chunk_off_off) {
+  const int64_t nblocks = (total_k + B_k - 1) / B_k + batch;
   size_t off = 0;
   *bscore_off = off;
   off = align_up(off + sizeof(float) * nblocks * G, 256);
@@ -37,7 +38,8 @@ size_t scratch_layout(int32_t batch, int64_t total_k, int32_t G, size_t* bscore_
 
 // blk_off[b]: first block id of sequence b; chunk_off[b]: first scan chunk.
 __global__ void decode_prep_kernel(const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_k, int batch,
-                                   int32_t* __restrict__ blk_off, int32_t* __restrict__ chunk_off, DevError* err) {
+                                   int B_k, int all_blocks, int32_t* __restrict__ blk_off,
+                                   int32_t* __restrict__ chunk_off, DevError* err) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   int bo = 0, co = 0;
   for (int b = 0; b < batch; ++b) {
@@ -48,10 +50,13 @@ __global__ void decode_prep_kernel(const int32_t* __restrict__ cu_q, const int32
     if (Tb < 0 || Tb > 1 || Tb > Sb) {
       report_error(err, MSA_ERR_DEVICE_CHECK, kSiteDecodeIndex, b, Tb);
     } else if (Tb == 1) {
-      const int lb = (Sb - 1) / kBk;          // blocks before the local one
-      co += (lb + kCB - 1) / kCB;
+      // blocks scored: those before the query's local block, or (all_blocks)
+      // every complete block of the keys when the query lies after them
+      const int lb = all_blocks ? Sb / B_k : (Sb - 1) / B_k;
+      const int ntile = (lb * B_k + kBk - 1) / kBk;   // 128-key tiles holding them
+      co += (ntile + kCB - 1) / kCB;
     }
-    bo += (Sb + kBk - 1) / kBk;
+    bo += (Sb + B_k - 1) / B_k;
   }
   blk_off[batch] = bo;
   chunk_off[batch] = co;
@@ -74,7 +79,8 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
 template <int DIDX>
 __global__ void __launch_bounds__(kScanThreads)
 decode_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restrict__ q_idx,
-                   const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_k, int batch, int G,
+                   const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_k, int batch, int G, int B_k,
+                   int all_blocks,
                    const int32_t* __restrict__ blk_off, const int32_t* __restrict__ chunk_off,
                    float* __restrict__ bscore, const int32_t* __restrict__ block_table, int max_blocks,
                    int64_t num_pages, DevError* err) {
@@ -97,9 +103,11 @@ decode_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16
   }
   const int b = lo;
   const int Sb = cu_k[b + 1] - cu_k[b];
-  const int lb = (Sb - 1) / kBk;
-  const int j0 = (chunk - chunk_off[b]) * kCB;
-  const int nblk = min(kCB, lb - j0);
+  const int lb = all_blocks ? Sb / B_k : (Sb - 1) / B_k;   // blocks scored: 0 .. lb - 1
+  const int ntile = (lb * B_k + kBk - 1) / kBk;     // 128-key tiles holding them
+  const int bpt = kBk / B_k;                        // blocks per tile
+  const int j0 = (chunk - chunk_off[b]) * kCB;      // first tile of this chunk
+  const int nblk = min(kCB, ntile - j0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // first key row of block j0 + i (packed: after the sequence's start; paged:
@@ -146,6 +154,7 @@ decode_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16
       report_error(err, MSA_ERR_TIMEOUT, kSiteDecodeIndex, chunk, warp);
     } else {
       const uint32_t base = smem_u32(smem + warp * BLOCK_BYTES);
+      const int mt_per_blk = B_k / 16;                 // 16-row MMA tiles per block
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll 2
       for (int mt = 0; mt < kBk / 16; ++mt) {
@@ -163,17 +172,23 @@ decode_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16
         }
         mx0 = fmaxf(mx0, fmaxf(c[0], c[2]));
         mx1 = fmaxf(mx1, fmaxf(c[1], c[3]));
-      }
+        if ((mt + 1) % mt_per_blk == 0) {
+          // the last rows of block (tile j0 + warp) * bpt + mt / mt_per_blk
 #pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-      }
-      if (lane < 4) {
-        const int64_t gb = (int64_t)(blk_off[b] + j0 + warp) * G;
-        const int g0 = 2 * lane, g1 = 2 * lane + 1;
-        if (g0 < G) bscore[gb + g0] = (mx0 != mx0) ? -INFINITY : mx0;
-        if (g1 < G) bscore[gb + g1] = (mx1 != mx1) ? -INFINITY : mx1;
+          for (int o = 4; o < 32; o <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+          }
+          const int blk = (j0 + warp) * bpt + mt / mt_per_blk;
+          if (lane < 4 && blk < lb) {
+            const int64_t gb = (int64_t)(blk_off[b] + blk) * G;
+            const int g0 = 2 * lane, g1 = 2 * lane + 1;
+            if (g0 < G) bscore[gb + g0] = (mx0 != mx0) ? -INFINITY : mx0;
+            if (g1 < G) bscore[gb + g1] = (mx1 != mx1) ? -INFINITY : mx1;
+          }
+          mx0 = -INFINITY;
+          mx1 = -INFINITY;
+        }
       }
     }
   }
@@ -210,21 +225,29 @@ __device__ __forceinline__ uint64_t rank_key(float s, int j) {
   return (static_cast<uint64_t>(u) << 32) | static_cast<uint32_t>(~j);
 }
 
-template <int CAP>
+// kCand == false: the selection (best k-1 earlier blocks, then the forced
+// local block; ascending ids, -1 padding).  kCand == true: the candidates of a
+// key range (the best k-1 of the scored blocks in rank order, with their
+// scores; -1 / -inf padding), for a selection merged over several ranges.
+template <int CAP, bool kCand>
 __global__ void __launch_bounds__(kSelThreads)
 decode_select_kernel(const float* __restrict__ bscore, const int32_t* __restrict__ cu_q,
-                     const int32_t* __restrict__ cu_k, const int32_t* __restrict__ blk_off, int G, int k,
-                     int32_t* __restrict__ sel) {
+                     const int32_t* __restrict__ cu_k, const int32_t* __restrict__ blk_off, int G, int k, int B_k,
+                     int all_blocks, int32_t* __restrict__ sel, float* __restrict__ cand_score) {
   const int b = blockIdx.x / G, g = blockIdx.x % G;
   const int Tb = cu_q[b + 1] - cu_q[b];
   const int Sb = cu_k[b + 1] - cu_k[b];
+  const int width = kCand ? k - 1 : k;   // output entries per (query, group)
   if (Tb == 1 && Sb < 1) {
     // a query without keys (an error the prep recorded): an empty selection
-    if (threadIdx.x < k) sel[((int64_t)cu_q[b] * G + g) * k + threadIdx.x] = -1;
+    if (threadIdx.x < width) {
+      sel[((int64_t)cu_q[b] * G + g) * width + threadIdx.x] = -1;
+      if (kCand) cand_score[((int64_t)cu_q[b] * G + g) * width + threadIdx.x] = -INFINITY;
+    }
     return;
   }
   if (Tb != 1) return;
-  const int lb = (Sb - 1) / kBk;
+  const int lb = all_blocks ? Sb / B_k : (Sb - 1) / B_k;
   const int cap = k - 1;
   const float* sc = bscore + (int64_t)blk_off[b] * G + g;
   // per-thread sorted (descending) list of the best keys of its slice
@@ -247,6 +270,7 @@ decode_select_kernel(const float* __restrict__ bscore, const int32_t* __restrict
   // k-1 rounds of block-wide argmax over the list heads
   __shared__ uint64_t warp_best[kSelThreads / 32];
   __shared__ int32_t chosen[kMaxK];
+  __shared__ float chosen_score[kMaxK];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int nsel = min(cap, lb);
   for (int r = 0; r < nsel; ++r) {
@@ -266,8 +290,23 @@ decode_select_kernel(const float* __restrict__ bscore, const int32_t* __restrict
       for (int i = 0; i < CAP - 1; ++i) list[i] = list[i + 1];
       list[CAP - 1] = 0;
     }
-    if (threadIdx.x == 0) chosen[r] = (int)~static_cast<uint32_t>(top & 0xffffffffu);
+    if (threadIdx.x == 0) {
+      chosen[r] = (int)~static_cast<uint32_t>(top & 0xffffffffu);
+      // the key's upper half holds the order-preserving score bits
+      uint32_t u = static_cast<uint32_t>(top >> 32);
+      u = (u & 0x80000000u) ? (u & 0x7fffffffu) : ~u;
+      chosen_score[r] = __uint_as_float(u);
+    }
     __syncthreads();
+  }
+  if (kCand) {
+    // candidates in the order chosen (score descending, lower id first)
+    if (threadIdx.x < width) {
+      const int64_t o = ((int64_t)cu_q[b] * G + g) * width + threadIdx.x;
+      sel[o] = threadIdx.x < nsel ? chosen[threadIdx.x] : -1;
+      cand_score[o] = threadIdx.x < nsel ? chosen_score[threadIdx.x] : -INFINITY;
+    }
+    return;
   }
   if (threadIdx.x == 0) {
     // ascending ids, then the local block, then -1
@@ -286,15 +325,15 @@ decode_select_kernel(const float* __restrict__ bscore, const int32_t* __restrict
 
 }  // namespace
 
-size_t decode_index_scratch_bytes(int32_t batch, int64_t total_k, int32_t G, int32_t /*k*/) {
+size_t decode_index_scratch_bytes(int32_t batch, int64_t total_k, int32_t G, int32_t B_k) {
   size_t a, b, c;
-  return scratch_layout(batch, total_k, G, &a, &b, &c);
+  return scratch_layout(batch, total_k, G, B_k, &a, &b, &c);
 }
 
 int launch_index_topk_decode(const IndexTopkArgs& a, void* stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   size_t o_bs, o_bo, o_co;
-  const size_t need = scratch_layout(a.batch, a.total_k, a.G, &o_bs, &o_bo, &o_co);
+  const size_t need = scratch_layout(a.batch, a.total_k, a.G, a.B_k, &o_bs, &o_bo, &o_co);
   if (a.scratch_bytes < need) return (int)cudaErrorInvalidValue;
   uint8_t* base = static_cast<uint8_t*>(a.scratch);
   float* bscore = reinterpret_cast<float*>(base + o_bs);
@@ -302,7 +341,7 @@ int launch_index_topk_decode(const IndexTopkArgs& a, void* stream) {
   int32_t* chunk_off = reinterpret_cast<int32_t*>(base + o_co);
   {
     ProfScope p("decode_prep", stream);
-    decode_prep_kernel<<<1, 32, 0, st>>>(a.cu_q, a.cu_k, a.batch, blk_off, chunk_off, a.err);
+    decode_prep_kernel<<<1, 32, 0, st>>>(a.cu_q, a.cu_k, a.batch, a.B_k, a.all_blocks, blk_off, chunk_off, a.err);
   }
 
   const int span = a.d_idx * 2 >= 128 ? 128 : a.d_idx * 2;
@@ -323,7 +362,8 @@ int launch_index_topk_decode(const IndexTopkArgs& a, void* stream) {
   if (e != cudaSuccess) return (int)e;                                                                      \
   ProfScope p("decode_scan", stream);                                                                       \
   decode_scan_kernel<D><<<(unsigned)max_chunks, kScanThreads, smem, st>>>(                                  \
-      tm_k, qi, a.cu_q, a.cu_k, a.batch, a.G, blk_off, chunk_off, bscore, a.block_table, a.max_blocks,       \
+      tm_k, qi, a.cu_q, a.cu_k, a.batch, a.G, a.B_k, a.all_blocks, blk_off, chunk_off, bscore, a.block_table,  \
+      a.max_blocks,                                                                                          \
       a.num_pages, a.err)
   if (a.d_idx == 32) { MSA_SCAN(32); }
   else if (a.d_idx == 64) { MSA_SCAN(64); }
@@ -331,9 +371,17 @@ int launch_index_topk_decode(const IndexTopkArgs& a, void* stream) {
 #undef MSA_SCAN
   const unsigned nsel = (unsigned)(a.batch * a.G);
   ProfScope p("decode_select", stream);
-  if (a.k <= 8) decode_select_kernel<7><<<nsel, kSelThreads, 0, st>>>(bscore, a.cu_q, a.cu_k, blk_off, a.G, a.k, a.sel);
-  else if (a.k <= 16) decode_select_kernel<15><<<nsel, kSelThreads, 0, st>>>(bscore, a.cu_q, a.cu_k, blk_off, a.G, a.k, a.sel);
-  else decode_select_kernel<31><<<nsel, kSelThreads, 0, st>>>(bscore, a.cu_q, a.cu_k, blk_off, a.G, a.k, a.sel);
+#define MSA_SEL(CAP)                                                                                         \
+  if (a.cand_score != nullptr)                                                                               \
+    decode_select_kernel<CAP, true><<<nsel, kSelThreads, 0, st>>>(bscore, a.cu_q, a.cu_k, blk_off, a.G, a.k,  \
+                                                                 a.B_k, a.all_blocks, a.sel, a.cand_score);  \
+  else                                                                                                       \
+    decode_select_kernel<CAP, false><<<nsel, kSelThreads, 0, st>>>(bscore, a.cu_q, a.cu_k, blk_off, a.G, a.k, \
+                                                                  a.B_k, a.all_blocks, a.sel, nullptr);
+  if (a.k <= 8) { MSA_SEL(7) }
+  else if (a.k <= 16) { MSA_SEL(15) }
+  else { MSA_SEL(31) }
+#undef MSA_SEL
   return (int)cudaGetLastError();
 }
 

@@ -46,12 +46,12 @@ struct TileInfo {
   int q0;      // first query row of the tile
   int rows;    // valid query rows (<= 128)
   int pos0;    // absolute position of row 0 in its sequence
-  int n_kb;    // key blocks scanned: 0 .. n_kb-1 (lb of the last valid row)
+  int n_kb;    // 128-key tiles scanned: 0 .. n_kb-1 (they hold the blocks before the last row's local block)
   int k0row;   // first key row of the sequence
 };
 
 __device__ __forceinline__ TileInfo tile_info(int tau, const IndexCtl* ctl, int batch, const int32_t* cu_q,
-                                              const int32_t* cu_k) {
+                                              const int32_t* cu_k, int B_k) {
   int lo = 0, hi = batch;  // find b with prefix[b] <= tau < prefix[b+1]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -65,7 +65,7 @@ __device__ __forceinline__ TileInfo tile_info(int tau, const IndexCtl* ctl, int 
   t.q0 = cu_q[b] + kTile * i;
   t.rows = min(kTile, Tb - kTile * i);
   t.pos0 = Sb - Tb + kTile * i;
-  t.n_kb = (t.pos0 + t.rows - 1) / kBk;
+  t.n_kb = ((t.pos0 + t.rows - 1) / B_k * B_k + kBk - 1) / kBk;
   t.k0row = cu_k[b];
   return t;
 }
@@ -172,7 +172,7 @@ template <int KMAX, int G>
 __global__ void __launch_bounds__(kThreads, 1)
 index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           int32_t* __restrict__ sel, const int32_t* __restrict__ cu_q,
-                          const int32_t* __restrict__ cu_k, int batch, int d_idx, int k, int nst,
+                          const int32_t* __restrict__ cu_k, int batch, int d_idx, int k, int B_k, int nst,
                           DevError* err) {
   constexpr int CAP = KMAX - 1;
   constexpr int GP = G < 2 ? G : 2;          // groups per work unit
@@ -239,7 +239,7 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         const int u = snake_unit(it, nunits);
         if (u < 0 || *abort_flag) break;
         const int pair = u % NPAIR;
-        const TileInfo ti = tile_info(u / NPAIR, ctl, batch, cu_q, cu_k);
+        const TileInfo ti = tile_info(u / NPAIR, ctl, batch, cu_q, cu_k, B_k);
         if (!mbar_wait(&ctl->q_empty, (qiter + 1) & 1)) {
           report_error(err, MSA_ERR_TIMEOUT, kSiteIndexProducer, u, -1);
           *abort_flag = 1;
@@ -290,7 +290,7 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
       for (int it = 0; ok; ++it) {
         const int u = snake_unit(it, nunits);
         if (u < 0 || *abort_flag) break;
-        const TileInfo ti = tile_info(u / NPAIR, ctl, batch, cu_q, cu_k);
+        const TileInfo ti = tile_info(u / NPAIR, ctl, batch, cu_q, cu_k, B_k);
         if (!mbar_wait(&ctl->q_full, qiter & 1)) {
           report_error(err, MSA_ERR_TIMEOUT, kSiteIndexMma, u, -1);
           ok = false;
@@ -340,9 +340,9 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
       const int u = snake_unit(it, nunits);
       if (u < 0 || *abort_flag) break;
       const int g = (u % NPAIR) * GP + l;
-      const TileInfo ti = tile_info(u / NPAIR, ctl, batch, cu_q, cu_k);
+      const TileInfo ti = tile_info(u / NPAIR, ctl, batch, cu_q, cu_k, B_k);
       const bool valid = row < ti.rows;
-      const int lb = (ti.pos0 + row) / kBk;
+      const int lb = (ti.pos0 + row) / B_k;
       list.reset();
       bool ok = true;
       for (int j = 0; j < ti.n_kb; ++j, ++jstep) {
@@ -359,16 +359,31 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         tmem_ld32(ta, r0);
         tmem_ld32(ta + 32, r1);
         tmem_ld_wait();
-        float m = fmaxf(max_of_32(r0), max_of_32(r1));
+        const float m0 = max_of_32(r0), m1 = max_of_32(r1);
         tmem_ld32(ta + 64, r0);
         tmem_ld32(ta + 96, r1);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->acc_empty[buf][l]);
-        m = fmaxf(m, fmaxf(max_of_32(r0), max_of_32(r1)));
-        if (m != m) m = -INFINITY;    // a block of NaN scores ranks as -inf
-        if (valid && j < lb) list.offer(m, j, k - 1);
+        const float m2 = max_of_32(r0), m3 = max_of_32(r1);
+        // the tile's 128 keys hold 128 / B_k blocks; offered in ascending order
+        // (a block of NaN scores ranks as -inf)
+        auto offer = [&](float m, int b) {
+          if (m != m) m = -INFINITY;
+          if (valid && b < lb) list.offer(m, b, k - 1);
+        };
+        if (B_k == kBk) {
+          offer(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)), j);
+        } else if (B_k == 64) {
+          offer(fmaxf(m0, m1), 2 * j);
+          offer(fmaxf(m2, m3), 2 * j + 1);
+        } else {
+          offer(m0, 4 * j);
+          offer(m1, 4 * j + 1);
+          offer(m2, 4 * j + 2);
+          offer(m3, 4 * j + 3);
+        }
       }
       if (!ok) break;
       if (valid) list.write(sel + (static_cast<int64_t>(ti.q0 + row) * G + g) * k, k, lb);
@@ -421,7 +436,7 @@ int launch_index_topk_prefill(const IndexTopkArgs& a, void* stream) {
     if (e != cudaSuccess) return (int)e;                                                                       \
     ProfScope p("index_topk_prefill", stream);                                                                 \
     index_topk_prefill_kernel<KM, GG><<<nsm, kThreads, smem, st>>>(tm_q, tm_k, a.sel, a.cu_q, a.cu_k, a.batch, \
-                                                                   a.d_idx, a.k, nst, a.err);                \
+                                                                   a.d_idx, a.k, a.B_k, nst, a.err);         \
     return (int)cudaGetLastError();                                                                            \
   }
   MSA_IDX(8, 1) MSA_IDX(8, 2) MSA_IDX(8, 4)

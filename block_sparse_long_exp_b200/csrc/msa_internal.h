@@ -9,7 +9,7 @@
 
 namespace msa {
 
-constexpr int kBk = 128;          // block size the kernels are built for
+constexpr int kBk = 128;          // key tile of the kernels (the largest block size B_k; 32 and 64 divide it)
 constexpr int kMaxK = 32;         // largest k
 constexpr int kMaxBatchTiles = 1024;  // sequences per prefill index launch
 constexpr int kDefaultWindow = 8192;  // query rows per attention planning window (KV-outer lists)
@@ -47,6 +47,7 @@ enum ErrorSite : int32_t {
   kSiteTileSoftmax = 154,
   kSitePaged = 161,
   kSiteSelfTest = 171,
+  kSiteKeySplit = 181,
 };
 
 // One KV-outer work item: up to `count` queries of the list of
@@ -67,6 +68,7 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Host-side argument checks shared by the entry points (msa_api.cu).
 msa_status_t check_shape(const msa_shape_t* s);
+msa_status_t check_shape_bk128(const msa_shape_t* s);
 msa_status_t check_seqs(const msa_varlen_t* v);
 
 // -------------------------------------------------------- host launchers ---
@@ -79,6 +81,9 @@ struct IndexTopkArgs {
   const int32_t* cu_q;
   const int32_t* cu_k;
   int32_t batch, G, d_idx, k;
+  int32_t B_k;         // block size: 32, 64 or 128 (a divisor of the 128-key tile)
+  int32_t all_blocks;  // decode: the query lies after the keys (every complete block is scored)
+  float* cand_score;   // decode: non-null -> write the k-1 candidates (ids in sel [T, G, k-1]) and their scores
   int64_t total_q, total_k;
   int32_t max_q_len, max_k_len;
   DevError* err;
@@ -91,7 +96,7 @@ struct IndexTopkArgs {
 };
 int launch_index_topk_prefill(const IndexTopkArgs& a, void* stream);
 int launch_index_topk_decode(const IndexTopkArgs& a, void* stream);
-size_t decode_index_scratch_bytes(int32_t batch, int64_t total_k, int32_t G, int32_t k);
+size_t decode_index_scratch_bytes(int32_t batch, int64_t total_k, int32_t G, int32_t B_k);
 
 struct AttnArgs {
   const void* q;       // bf16 [T, H, d]
@@ -103,6 +108,7 @@ struct AttnArgs {
   const int32_t* cu_q;
   const int32_t* cu_k;
   int32_t batch, H, G, d, k;
+  int32_t B_k;         // block size: 32, 64 or 128
   float sm_scale;
   int64_t total_q, total_k;
   int32_t max_q_len, max_k_len;

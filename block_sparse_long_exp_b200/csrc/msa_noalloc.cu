@@ -72,7 +72,7 @@ extern "C" msa_status_t msa_index_topk_decode_noalloc(const msa_shape_t* shape, 
     IndexTopkArgs a{};
     a.q_idx = q_idx; a.k_idx = k_idx; a.sel = sel;
     a.cu_q = seqs->cu_q; a.cu_k = seqs->cu_k;
-    a.batch = seqs->batch; a.G = shape->G; a.d_idx = shape->d_idx; a.k = shape->k;
+    a.batch = seqs->batch; a.G = shape->G; a.d_idx = shape->d_idx; a.k = shape->k; a.B_k = shape->B_k;
     a.total_q = seqs->total_q; a.total_k = seqs->total_k;
     a.max_q_len = seqs->max_q_len; a.max_k_len = seqs->max_k_len;
     a.err = static_cast<DevError*>(scratch);

@@ -244,6 +244,7 @@ struct TileParams {
   const int32_t* cu_q;
   const int32_t* cu_k;
   int32_t batch, H, G, d, k, UQ;
+  int32_t bk;                 // block size B_k (tiles and rows modes; dense mode works in 128-key tiles)
   float scale_log2;
   int64_t t0, t1;
   __nv_bfloat16* out;         // [T, H, d] (absolute rows)
@@ -382,7 +383,7 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         const unsigned v = __ballot_sync(0xffffffffu, b >= 0);
         nblk = __popc(v);
         const int64_t pos = (int64_t)Sb - Tb + (r0 - p.cu_q[seq]);
-        bool bad = b >= 0 && (Tb > Sb || pos < 0 || b > pos / kBk);
+        bool bad = b >= 0 && (Tb > Sb || pos < 0 || b > pos / p.bk);
         int32_t pg = -1;
         if (b >= 0 && !bad && p.block_table != nullptr) {
           bad = b >= p.max_blocks;
@@ -454,7 +455,9 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
           ok = mbar_wait(&ctl->kv_empty[st], ((kvc >> 1) + 1) & 1);
           if (!ok) break;
           const int blk = kMode == kModeDense ? j : R->blk[j];
-          const int krow = (kMode == kModeRows && p.block_table != nullptr) ? R->page[j] * kBk : kbase + blk * kBk;
+          // a block's 128-row K/V tile: B_k rows of it are the block (paged caches: B_k = 128)
+          const int krow = (kMode == kModeRows && p.block_table != nullptr) ? R->page[j] * kBk
+                         : kbase + blk * (kMode == kModeDense ? kBk : p.bk);
           uint8_t* ks = kv_s + st * 2 * tile_bytes;
           mbar_arrive_expect_tx(&ctl->k_full[st], tile_bytes);
           for (int h = 0; h < nhalf; ++h) tma_load_3d(ks + h * 128 * 128, &tm_k, &ctl->k_full[st], 64 * h, g, krow);
@@ -596,7 +599,8 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       const bool valid = ql < qpt && qi < R->nq && hi < Hg;
       const int64_t t = R->r0 + qi;
       const int64_t pos = valid ? (int64_t)R->Sb - R->Tb + (t - R->qrow0) : -1;
-      const int lb = valid ? (int)(pos / kBk) : -1;
+      const int bk = kMode == kModeDense ? kBk : p.bk;
+      const int lb = valid ? (int)(pos / bk) : -1;
       uint64_t mem = 0;
       if (kMode == kModeTiles && valid) mem = p.dmember[(t - p.t0) * G + R->g];
       float m_run = -INFINITY, l_run = 0.f;
@@ -605,7 +609,7 @@ tile_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         const int blk = kMode == kModeDense ? j : R->blk[j];
         const bool member = valid && (kMode != kModeTiles || ((mem >> j) & 1ull)) && blk <= lb;
         int limit = -1;                          // last attended key of the block, -1: none
-        if (member) limit = blk < lb ? kBk - 1 : (int)(pos - (int64_t)blk * kBk);
+        if (member) limit = blk < lb ? bk - 1 : (int)(pos - (int64_t)blk * bk);
         if (!mbar_wait(&ctl->s_full[x], (uint32_t)(bt & 1))) {
           report_error(p.err, MSA_ERR_TIMEOUT, kSiteTileSoftmax, (int)bt, 0);
           failed = true;
@@ -914,6 +918,7 @@ int launch_tile_attn(const AttnArgs& a, void* stream) {
   prm.nunits = a.tile_ctr + 1; prm.ticket = a.tile_ctr + 2;
   prm.cu_q = a.cu_q; prm.cu_k = a.cu_k;
   prm.batch = a.batch; prm.H = a.H; prm.G = a.G; prm.d = a.d; prm.k = a.k; prm.UQ = tile_queries(a.H, a.G);
+  prm.bk = a.B_k;
   prm.scale_log2 = a.sm_scale * 1.4426950408889634f;
   prm.t0 = a.t0; prm.t1 = a.t1;
   prm.out = reinterpret_cast<__nv_bfloat16*>(a.out);
@@ -941,6 +946,7 @@ int launch_rows_attn(const AttnArgs& a, void* stream) {
   prm.block_table = a.block_table; prm.max_blocks = a.max_blocks; prm.num_pages = a.num_pages;
   prm.cu_q = a.cu_q; prm.cu_k = a.cu_k;
   prm.batch = a.batch; prm.H = a.H; prm.G = a.G; prm.d = a.d; prm.k = a.k; prm.UQ = 1;
+  prm.bk = a.B_k;
   prm.scale_log2 = a.sm_scale * 1.4426950408889634f;
   prm.t0 = a.t0; prm.t1 = a.t1;
   prm.out = reinterpret_cast<__nv_bfloat16*>(a.out);
@@ -972,6 +978,7 @@ int launch_dense_attn(const DenseArgs& a, void* stream) {
   prm.nunits = ctr + 1; prm.ticket = ctr + 2;
   prm.cu_q = a.cu_q; prm.cu_k = a.cu_k;
   prm.batch = a.batch; prm.H = a.H; prm.G = a.G; prm.d = a.d; prm.k = 1; prm.UQ = UQ;
+  prm.bk = kBk;
   prm.scale_log2 = a.sm_scale * 1.4426950408889634f;
   prm.t0 = 0; prm.t1 = a.total_q;
   prm.out = reinterpret_cast<__nv_bfloat16*>(a.out);

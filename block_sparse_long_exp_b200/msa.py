@@ -51,6 +51,7 @@ EXPORTED = [
     "msa_profile_enable", "msa_profile_reset", "msa_profile_read",
     "msa_get_device_error", "msa_version", "msa_set_tile_threshold", "msa_set_attn_window",
     "msa_selftest_wait_timeout_workspace_size", "msa_selftest_wait_timeout",
+    "msa_index_topk_decode_candidates", "msa_merge_candidates", "msa_select_block_range",
     "msa_decode_paged_workspace_size", "msa_index_topk_decode_paged", "msa_sparse_attn_decode_paged",
     "msa_index_kl", "msa_index_kl_backward", "msa_select_window", "msa_sparse_attn_backward",
     "msa_selected_share", "msa_index_topk_policy", "msa_gather_pages",
@@ -128,6 +129,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_set_tile_threshold.restype = i32
     lib.msa_set_attn_window.argtypes = [i32]
     lib.msa_set_attn_window.restype = i32
+    lib.msa_index_topk_decode_candidates.argtypes = [P(Shape), P(Varlen), vp, vp, i32, vp, vp, vp, sz, vp]
+    lib.msa_index_topk_decode_candidates.restype = i32
+    lib.msa_merge_candidates.argtypes = [P(Shape), i32, i32, vp, vp, vp, vp, vp, sz, vp]
+    lib.msa_merge_candidates.restype = i32
+    lib.msa_select_block_range.argtypes = [P(Shape), i32, vp, vp, vp, vp, vp]
+    lib.msa_select_block_range.restype = i32
     lib.msa_selftest_wait_timeout_workspace_size.argtypes = []
     lib.msa_selftest_wait_timeout_workspace_size.restype = sz
     lib.msa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp, sz, vp]
@@ -787,6 +794,76 @@ def msa_set_tile_threshold(theta: int) -> int:
     """Query-tile threshold of the prefill main branch (-1 automatic, 0 off);
     returns the previous value."""
     return int(load_library().msa_set_tile_threshold(int(theta)))
+
+
+def msa_index_topk_decode_candidates(shape: Shape, seqs: Varlen, q_idx: torch.Tensor, k_idx: torch.Tensor,
+                                     all_blocks: bool, ws: Optional[torch.Tensor] = None, stream=None,
+                                     check: bool = True) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per (query, group) the k-1 best blocks of a key slice and their scores
+    (decode shape; ids local to the slice, -1 / -inf padding): the candidates
+    of one rank of a key-range split (see msa_merge_candidates)."""
+    lib = load_library()
+    G, kc = shape.G, max(shape.k - 1, 0)
+    T = int(seqs.total_q)
+    _arg("q_idx", q_idx, torch.bfloat16, (T, G, shape.d_idx))
+    _arg("k_idx", k_idx, torch.bfloat16, (int(seqs.total_k), shape.d_idx))
+    _require_cuda(q_idx, k_idx)
+    ids = torch.full((T, G, kc), -1, dtype=torch.int32, device=q_idx.device)
+    scores = torch.full((T, G, kc), float("-inf"), dtype=torch.float32, device=q_idx.device)
+    if ws is None:
+        ws = _workspace(lib.msa_index_topk_workspace_size(ctypes.byref(shape), ctypes.byref(seqs)), q_idx.device)
+    _ws_arg(ws)
+    rc = lib.msa_index_topk_decode_candidates(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q_idx), _ptr(k_idx),
+                                              int(bool(all_blocks)), _ptr(ids), _ptr(scores), _ptr(ws), _nbytes(ws),
+                                              _stream(stream))
+    _check(rc, "msa_index_topk_decode_candidates")
+    if check:
+        _device_check(ws, stream, "msa_index_topk_decode_candidates")
+    return ids, scores
+
+
+def msa_merge_candidates(shape: Shape, cand_ids: torch.Tensor, cand_scores: torch.Tensor,
+                         local_block: torch.Tensor, stream=None, check: bool = True) -> torch.Tensor:
+    """The selection of a key-range split: the top k-1 of the candidates
+    [batch, G, n_cand] (global block ids) in the selection order, with the
+    local block [batch] forced; sel [batch, G, k] as msa_index_topk writes it."""
+    lib = load_library()
+    G = shape.G
+    _arg("cand_ids", cand_ids, torch.int32)
+    if cand_ids.dim() != 3 or cand_ids.shape[1] != G:
+        raise MsaError(f"cand_ids: expected [batch, {G}, n_cand], got {tuple(cand_ids.shape)}")
+    B, _, n = cand_ids.shape
+    _arg("cand_scores", cand_scores, torch.float32, (B, G, n))
+    _arg("local_block", local_block, torch.int32, (B,))
+    _require_cuda(cand_ids, cand_scores, local_block)
+    sel = torch.empty((B, G, shape.k), dtype=torch.int32, device=cand_ids.device)
+    ws = _workspace(256, cand_ids.device)
+    rc = lib.msa_merge_candidates(ctypes.byref(shape), B, n, _ptr(cand_ids), _ptr(cand_scores), _ptr(local_block),
+                                  _ptr(sel), _ptr(ws), _nbytes(ws), _stream(stream))
+    _check(rc, "msa_merge_candidates")
+    if check:
+        _device_check(ws, stream, "msa_merge_candidates")
+    return sel
+
+
+def msa_select_block_range(shape: Shape, sel: torch.Tensor, blk_lo: torch.Tensor, blk_hi: torch.Tensor,
+                           stream=None) -> torch.Tensor:
+    """The blocks of a selection [batch, G, k] inside [blk_lo[b], blk_hi[b]),
+    re-based to the range, ascending, -1 padded."""
+    lib = load_library()
+    G = shape.G
+    _arg("sel", sel, torch.int32)
+    if sel.dim() != 3 or sel.shape[1:] != (G, shape.k):
+        raise MsaError(f"sel: expected [batch, {G}, {shape.k}], got {tuple(sel.shape)}")
+    B = sel.shape[0]
+    _arg("blk_lo", blk_lo, torch.int32, (B,))
+    _arg("blk_hi", blk_hi, torch.int32, (B,))
+    _require_cuda(sel, blk_lo, blk_hi)
+    out = torch.empty_like(sel)
+    rc = lib.msa_select_block_range(ctypes.byref(shape), B, _ptr(sel), _ptr(blk_lo), _ptr(blk_hi), _ptr(out),
+                                    _stream(stream))
+    _check(rc, "msa_select_block_range")
+    return out
 
 
 def msa_selftest_wait_timeout(limit_us: int = 2000, stream=None) -> Tuple[int, int, int, int]:

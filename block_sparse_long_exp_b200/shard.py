@@ -160,3 +160,111 @@ def decode_shards(lengths, world: int) -> List[List[int]]:
         out[r].append(i)
         load[r] += int(lengths[i])
     return [sorted(o) for o in out]
+
+
+# ---------------------------------------------- decode split by key range ---
+#
+# One very long decode sequence can be cut by key range: rank r holds the
+# keys of a consecutive run of blocks of every sequence (the last rank holds
+# the block of the query), the query itself is on every rank.  The selection
+# needs the top k-1 blocks of the whole cache; it is within the union of each
+# range's own top k-1 (msa_index_topk_decode_candidates), exchanged with one
+# small all-gather and merged by the library (msa_merge_candidates).  Each
+# rank then attends its own selected blocks (msa_select_block_range +
+# msa_sparse_attn_decode) and the per-rank outputs are merged by log-sum-exp
+# (msa_combine, one slot per rank) after one more all-gather.
+
+
+def split_key_blocks(L: int, world: int, B_k: int) -> List[Tuple[int, int]]:
+    """Block ranges [lo, hi) of each rank for a cache of L tokens (blocks of
+    B_k, the query at position L-1): the ceil(L / B_k) blocks cut into world
+    consecutive runs as equal as possible; the last run holds the query's
+    block.  Every rank needs at least one block."""
+    nb = -(-int(L) // B_k)
+    if world < 1 or nb < world:
+        raise ValueError(f"{nb} blocks cannot be split over {world} ranks")
+    cuts = [r * nb // world for r in range(world + 1)]
+    return [(cuts[r], cuts[r + 1]) for r in range(world)]
+
+
+def key_slice(inp: Dict[str, object], lengths: Sequence[int], rank: int, world: int, B_k: int) -> Dict[str, object]:
+    """Rank `rank`'s part of a decode batch (one query per sequence; k, v,
+    k_idx packed over the sequences with offsets cu_k): every query and its
+    q_idx, the keys of the rank's block range of each sequence, packed, and
+    per sequence the range's first / last-plus-one block (blk_lo, blk_hi,
+    global ids) and the query's local block.  all_blocks is True unless the
+    rank holds the queries' blocks (the last rank): its keys then all lie
+    before the query."""
+    import torch
+    dev = inp["q"].device
+    cu = inp["cu_k_host"]
+    rows, cu_k, lo, hi, local = [], [0], [], [], []
+    for b, L in enumerate(lengths):
+        a, z = split_key_blocks(L, world, B_k)[rank]
+        k0, k1 = cu[b] + a * B_k, cu[b] + min(z * B_k, L)
+        rows.append(torch.arange(k0, k1, device=dev))
+        cu_k.append(cu_k[-1] + (k1 - k0))
+        lo.append(a)
+        hi.append(z)
+        local.append((L - 1) // B_k)
+    idx = torch.cat(rows)
+    out = dict(inp)
+    for name in ("k", "v", "k_idx"):
+        out[name] = inp[name].index_select(0, idx).contiguous()
+    i32 = lambda v: torch.tensor(v, dtype=torch.int32, device=dev)  # noqa: E731
+    out.update(cu_k=i32(cu_k), cu_k_host=cu_k, blk_lo=i32(lo), blk_hi=i32(hi), local_block=i32(local),
+               all_blocks=rank < world - 1)
+    return out
+
+
+def gather_candidates(ids, scores, blk_lo, group=None):
+    """Every rank's candidates [B, G, c] (ids local to its range, -1 = none)
+    made global (+ blk_lo[b]) and joined over the ranks along the last axis
+    (one all-gather of ids and scores; without an initialised group the
+    rank's own, made global)."""
+    import torch
+    import torch.distributed as dist
+    glob = torch.where(ids >= 0, ids + blk_lo.view(-1, 1, 1).to(ids.dtype), ids)
+    if not (dist.is_available() and dist.is_initialized()):
+        return glob, scores
+    n = dist.get_world_size(group)
+    gi = [torch.empty_like(glob) for _ in range(n)]
+    gs = [torch.empty_like(scores) for _ in range(n)]
+    dist.all_gather(gi, glob.contiguous(), group=group)
+    dist.all_gather(gs, scores.contiguous(), group=group)
+    return torch.cat(gi, dim=2), torch.cat(gs, dim=2)
+
+
+def rank_partials(outs, lses, sels, H: int, G: int):
+    """The per-rank decode outputs laid out for msa_combine with one slot per
+    rank: part_acc f16 [B, G, R, d/8, H/G, 8], part_lse f32 [B, G, R, H/G],
+    slot sel int32 [B, G, R] (the rank's index where its range view of the
+    selection, sels[r] [B, G, k], holds a block, else -1).  outs[r] bf16
+    [B, H, d] and lses[r] f32 [B, H] are rank r's normalised output and
+    log-sum-exp over its own selected tokens."""
+    import torch
+    R = len(outs)
+    B, _, d = outs[0].shape
+    Hg = H // G
+    acc = torch.stack(outs).view(R, B, G, Hg, d // 8, 8).permute(1, 2, 0, 4, 3, 5).contiguous().half()
+    lse = torch.stack(lses).view(R, B, G, Hg).permute(1, 2, 0, 3).contiguous()
+    has = torch.stack([(s >= 0).any(dim=2) for s in sels])            # [R, B, G]
+    rank_id = torch.arange(R, dtype=torch.int32, device=has.device).view(R, 1, 1).expand_as(has)
+    slot = torch.where(has, rank_id, torch.full_like(rank_id, -1)).permute(1, 2, 0).contiguous()
+    return acc, lse, slot
+
+
+def gather_rank_outputs(out, lse, sel_local, group=None):
+    """All ranks' outputs, log-sum-exps and range views (lists in rank order;
+    one all-gather each; without an initialised group the rank's own)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return [out], [lse], [sel_local]
+    n = dist.get_world_size(group)
+    res = []
+    for t in (out, lse, sel_local):
+        parts = [torch.empty_like(t) for _ in range(n)]
+        dist.all_gather(parts, t.contiguous(), group=group)
+        res.append(parts)
+    return res[0], res[1], res[2]

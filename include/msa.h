@@ -397,6 +397,47 @@ int32_t msa_set_tile_threshold(int32_t theta);
 int32_t msa_set_attn_window(int32_t rows);
 
 /* ---------------------------------------------------------------------- */
+/* Decode of one long sequence split across ranks by key range (this
+ * library's multi-GPU form of the pages' decode step, pnsm.cn sec. 9; the
+ * pages select per query the top-k blocks of the whole cache with the local
+ * block forced, sec. 2).  Rank r holds the keys [a_r, b_r) of each sequence
+ * (block aligned, the last rank holding the query's local block); the query
+ * is on every rank.  The global top-(k-1) is within the union of each range's
+ * own top-(k-1), so:
+ *   1. msa_index_topk_decode_candidates on each rank's key slice: per (query,
+ *      group) the k-1 best blocks of the slice and their raw scores, in the
+ *      selection order (score descending, lower id first), ids local to the
+ *      slice; -1 / -inf padding.  all_blocks = 1 when the query lies after
+ *      the slice's keys (every complete block is a candidate), 0 for the
+ *      slice that ends with the query (its last block is the local block and
+ *      is not scored, as in msa_index_topk).  Same workspace and checks as
+ *      msa_index_topk's decode shape; k = 1 writes nothing.
+ *      cand_ids int32 [T, G, k-1] and cand_scores f32 [T, G, k-1] (device).
+ *   2. the callers exchange the candidates (ids made global by adding each
+ *      slice's first block) and msa_merge_candidates merges n_cand of them
+ *      per (query, group) under the same order, with local_block[b] (global
+ *      id, device int32 [batch]) forced: sel int32 [batch, G, k] as
+ *      msa_index_topk writes it.  A candidate id >= the local block is
+ *      recorded as MSA_ERR_DEVICE_CHECK (site 181) and skipped; n_cand <= 256.
+ *      ws: at least 256 bytes (the error word).
+ *   3. msa_select_block_range cuts one rank's part out of a selection: ids in
+ *      [blk_lo[b], blk_hi[b]) minus blk_lo[b], ascending, -1 padded (device
+ *      int32 [batch] bounds; sel and sel_out [batch, G, k]); the rank then
+ *      runs msa_sparse_attn_decode on its slice with it.
+ *   4. the per-rank outputs are merged with msa_combine (one slot per rank).
+ * All device buffers belong to the caller; errors before any launch as for
+ * the other calls. */
+msa_status_t msa_index_topk_decode_candidates(const msa_shape_t* shape, const msa_varlen_t* seqs,
+                                              const void* q_idx, const void* k_idx, int32_t all_blocks,
+                                              int32_t* cand_ids, float* cand_scores, void* ws, size_t ws_bytes,
+                                              void* stream);
+msa_status_t msa_merge_candidates(const msa_shape_t* shape, int32_t batch, int32_t n_cand,
+                                  const int32_t* cand_ids, const float* cand_scores, const int32_t* local_block,
+                                  int32_t* sel, void* ws, size_t ws_bytes, void* stream);
+msa_status_t msa_select_block_range(const msa_shape_t* shape, int32_t batch, const int32_t* sel,
+                                    const int32_t* blk_lo, const int32_t* blk_hi, int32_t* sel_out, void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* Self-test of the bounded waits (no counterpart on the pages: a failure-
  * detection check of this library).  Every spin-wait in the kernels gives up
  * after about a second and records MSA_ERR_TIMEOUT in the call's error word

@@ -70,6 +70,8 @@ __all__ = [
     "msa_forward_rows",
     "lse_combine",
     "invert_selection",
+    "block_candidates",
+    "merge_block_candidates",
 ]
 
 
@@ -279,3 +281,34 @@ def invert_selection(sel, cu_q, cu_k, B_k: int) -> Dict[Tuple[int, int, int], Li
                         continue
                     lists.setdefault((b, g, int(blk)), []).append(t)
     return lists
+
+
+# --------------------------------------------- key-range split of a decode ---
+#
+# Step 3 over a cache cut into key ranges: the k-1 blocks a query chooses by
+# score are the first k-1 of all its non-local blocks under the order (score
+# descending, index ascending), so they are also the first k-1 of the union of
+# every range's own first k-1.  These two functions restate step 3 in that
+# form; with the whole cache as one range they reduce to ``select_blocks``.
+
+
+def block_candidates(S, k: int) -> Tuple[List[int], List[float]]:
+    """The first k-1 blocks of one key range under the order of step 3 (score
+    descending, index ascending; NaN as -inf), with their scores.  S holds the
+    scores of the range's competing blocks (none of them the query's local
+    block), indexed from 0."""
+    S = _f64(S)
+    keys = np.where(np.isnan(S), -np.inf, S)
+    order = np.lexsort((np.arange(keys.shape[0]), -keys))[: max(k - 1, 0)]
+    return [int(b) for b in order], [float(keys[b]) for b in order]
+
+
+def merge_block_candidates(ids: Sequence[int], scores: Sequence[float], lb: int, k: int) -> List[int]:
+    """Step 3 from the candidates of several ranges (global block ids, all
+    below the local block lb): the first k-1 of them under the same order,
+    then the local block; returned ascending."""
+    ids = np.asarray(list(ids), dtype=np.int64)
+    keys = np.asarray(list(scores), dtype=np.float64)
+    keys = np.where(np.isnan(keys), -np.inf, keys)
+    order = np.lexsort((ids, -keys))[: max(k - 1, 0)]
+    return sorted(int(ids[o]) for o in order) + [int(lb)]

@@ -53,8 +53,12 @@ def test_host_validation_without_gpu(lib):
     assert lib.msa_sparse_attn_workspace_size(ctypes.byref(shape), ctypes.byref(seqs), 0) > 1024 * 4 * 16 * 16 * 128 * 2
     bad = msa.make_shape(64, 4, 96, 64, 16)           # d = 96 is not built
     assert lib.msa_index_topk_workspace_size(ctypes.byref(bad), ctypes.byref(seqs)) == 0
-    bad_bk = msa.make_shape(64, 4, 128, 64, 16, B_k=64)
+    bad_bk = msa.make_shape(64, 4, 128, 64, 16, B_k=96)            # block sizes: 32, 64, 128
     assert lib.msa_sparse_attn_workspace_size(ctypes.byref(bad_bk), ctypes.byref(seqs), 0) == 0
+    for bk in (32, 64):
+        sh = msa.make_shape(64, 4, 128, 64, 16, B_k=bk)
+        assert lib.msa_sparse_attn_workspace_size(ctypes.byref(sh), ctypes.byref(seqs), 0) > 0
+        assert lib.msa_index_topk_workspace_size(ctypes.byref(sh), ctypes.byref(seqs)) >= 256
     # entry points reject invalid arguments before any launch
     rc = lib.msa_index_topk(ctypes.byref(shape), ctypes.byref(seqs), None, None, None, None, 0, None)
     assert rc == 1                                       # MSA_ERR_INVALID_ARG
@@ -206,7 +210,7 @@ def test_noalloc_host_checks_match_msa_index_topk(lib):
     data pointers are only required when there are queries."""
     from block_sparse_long_exp_b200 import msa
     shape = msa.make_shape(64, 4, 128, 64, 16)
-    bad_bk = msa.make_shape(64, 4, 128, 64, 16, B_k=64)
+    bad_bk = msa.make_shape(64, 4, 128, 64, 16, B_k=96)
     cu = (ctypes.c_int32 * 3)(0, 1, 2)
     cuk = (ctypes.c_int32 * 3)(0, 500, 900)
     seqs = msa.Varlen(2, 1, 500, 0, 2, 900, ctypes.addressof(cu), ctypes.addressof(cuk))
@@ -220,7 +224,7 @@ def test_noalloc_host_checks_match_msa_index_topk(lib):
     a, b = both(ctypes.byref(shape), ctypes.byref(no_cu), 256)
     assert a == b == 1                                   # MSA_ERR_INVALID_ARG: null cu_q
     a, b = both(ctypes.byref(bad_bk), ctypes.byref(seqs), 256)
-    assert a == b == 2                                   # MSA_ERR_UNSUPPORTED: B_k = 64
+    assert a == b == 2                                   # MSA_ERR_UNSUPPORTED: B_k = 96
     a, b = both(None, ctypes.byref(seqs), 256)
     assert a == b == 1
     # queries present: null data pointers are rejected
@@ -243,3 +247,21 @@ def test_selftest_wait_host_checks(lib):
     assert lib.msa_selftest_wait_timeout(1000, None, n, None) == 3        # MSA_ERR_WORKSPACE
     assert lib.msa_selftest_wait_timeout(1000, 256, n - 1, None) == 3
     assert lib.msa_selftest_wait_timeout(1000, 272, n, None) == 3         # not 256-byte aligned
+
+
+def test_block_size_128_only_entry_points(lib):
+    """B_k = 32 / 64 run on the main path (index top-k, sparse attention,
+    decode); the training-side kernels, the selection variants and paged
+    caches are built for 128-token blocks and say so before any launch."""
+    from block_sparse_long_exp_b200 import msa
+    sh64 = msa.make_shape(64, 4, 128, 64, 16, B_k=64)
+    cu = (ctypes.c_int32 * 2)(0, 1024)
+    seqs = msa.Varlen(1, 1024, 1024, 0, 1024, 1024, ctypes.addressof(cu), ctypes.addressof(cu))
+    U = 2                                                # MSA_ERR_UNSUPPORTED
+    assert lib.msa_select_window(ctypes.byref(sh64), ctypes.byref(seqs), 1, 256, 256, 1 << 20, None) == U
+    assert lib.msa_index_topk_policy(ctypes.byref(sh64), ctypes.byref(seqs), 1, 1, 256, 256, 256, 256, 1 << 20,
+                                     None) == U
+    lens = (ctypes.c_int32 * 1)(1000)
+    table = (ctypes.c_int32 * 8)(*range(8))
+    pages = msa.Paged(1, 8, 1000, 0, 8, ctypes.addressof(lens), ctypes.addressof(table))
+    assert lib.msa_decode_paged_workspace_size(ctypes.byref(sh64), ctypes.byref(pages)) == 0

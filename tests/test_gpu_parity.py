@@ -54,7 +54,7 @@ def _inputs(w, lengths=None, T_lens=None, T_override=None):
 
 def _to_dev(M, w, inp):
     d = {k: v.cuda() for k, v in inp.items() if torch.is_tensor(v)}
-    shape = M.make_shape(w.H, w.G, w.d, w.d_idx, w.k)
+    shape = M.make_shape(w.H, w.G, w.d, w.d_idx, w.k, B_k=w.B_k)
     seqs = M.make_varlen(d["cu_q"], d["cu_k"], inp["cu_q_host"], inp["cu_k_host"])
     return shape, seqs, d
 
@@ -221,6 +221,35 @@ def test_combine_entry_point(M):
         for h in range(H):
             g, i = h // Hg, h % Hg
             slots = [s for s in range(k) if sel[t, g, s] >= 0]
+            ro, rl = O.lse_combine(acc[t, g, slots, i].double().numpy(), plse[t, g, slots, i].double().numpy())
+            assert np.max(np.abs(o[t, h] - ro)) <= 1e-2
+            assert abs(lse_out[t, h].item() - rl) <= 1e-4
+
+
+def test_combine_ignores_unused_slots(M):
+    """Slots with sel < 0 take no part in the merge whatever their buffers
+    hold: NaN partials and log-sum-exps there leave the result unchanged."""
+    H, G, d_, k, T = 16, 2, 64, 5, 29
+    Hg = H // G
+    gen = torch.Generator().manual_seed(4)
+    acc = torch.randn(T, G, k, Hg, d_, generator=gen).half()
+    plse = (torch.randn(T, G, k, Hg, generator=gen) * 3).float()
+    sel = torch.randint(0, 50, (T, G, k), generator=gen, dtype=torch.int32)
+    sel[::2, :, 0] = -1
+    sel[1::3, :, k - 1] = -1
+    unused = (sel < 0)[:, :, :, None]
+    acc = torch.where(unused[..., None], torch.full_like(acc, float("nan")), acc)
+    plse = torch.where(unused, torch.full_like(plse, float("nan")), plse)
+    acc_dev = acc.view(T, G, k, Hg, d_ // 8, 8).permute(0, 1, 2, 4, 3, 5).contiguous()
+    shape = M.make_shape(H, G, d_, 32, k)
+    lse_out = torch.empty(T, H, device="cuda")
+    out, _ = M.msa_combine(shape, T, acc_dev.cuda(), plse.cuda(), sel.cuda(), lse=lse_out)
+    o = _f32(out)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse_out.cpu().numpy()))
+    for t in range(T):
+        for h in range(H):
+            g, i = h // Hg, h % Hg
+            slots = [s_ for s_ in range(k) if sel[t, g, s_] >= 0]
             ro, rl = O.lse_combine(acc[t, g, slots, i].double().numpy(), plse[t, g, slots, i].double().numpy())
             assert np.max(np.abs(o[t, h] - ro)) <= 1e-2
             assert abs(lse_out[t, h].item() - rl) <= 1e-4

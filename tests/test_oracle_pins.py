@@ -357,3 +357,84 @@ def test_random_layers_match_brute_force_and_masked_sdpa(layer):
         qb = q[cu_q[b]:cu_q[b + 1]]
         ref = _sdpa(qb, kk[cu_k[b]:cu_k[b + 1]], v[cu_k[b]:cu_k[b + 1]], mask, scale)
         np.testing.assert_allclose(o[cu_q[b]:cu_q[b + 1]], ref, rtol=0, atol=1e-12)
+
+
+def _brute_top_set(S, lb, k):
+    """Subset enumeration: the one (k-1)-subset of blocks 0..lb-1 whose every
+    member beats every non-member (higher score, ties to the lower index; NaN
+    as -inf), plus the local block lb; all blocks when lb + 1 <= k."""
+    if lb + 1 <= k:
+        return list(range(lb + 1))
+    sc = [(-np.inf if np.isnan(x) else float(x)) for x in S]
+
+    def beats(a, b):
+        return sc[a] > sc[b] or (sc[a] == sc[b] and a < b)
+
+    for subset in itertools.combinations(range(lb), k - 1):
+        rest = [b for b in range(lb) if b not in subset]
+        if all(beats(a, b) for a in subset for b in rest):
+            return sorted(subset) + [lb]
+    raise AssertionError("no top set")
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_key_range_candidates_merge_to_the_selection(seed):
+    """A decode cache cut into key ranges: each range's first k-1 blocks
+    (block_candidates), made global and merged (merge_block_candidates), give
+    the selection of the whole cache: equal to select_blocks and, on small
+    cases, to subset enumeration.  Integer scores (many ties) and NaNs; the
+    ranges are random cuts of the non-local blocks."""
+    rng = np.random.default_rng(100 + seed)
+    for _ in range(400):
+        nb = int(rng.integers(1, 30))
+        k = int(rng.integers(1, 8))
+        S = rng.integers(-3, 4, size=nb).astype(np.float64)
+        S[rng.random(nb) < 0.08] = np.nan
+        lb = nb - 1
+        ncut = int(rng.integers(0, min(4, max(lb, 1))))
+        cuts = sorted(rng.choice(np.arange(1, lb), size=ncut, replace=False).tolist()) if lb > 1 else []
+        bounds = [0] + cuts + [lb]
+        ids, scores = [], []
+        for a, b in zip(bounds[:-1], bounds[1:]):
+            ci, cs = O.block_candidates(S[a:b], k)
+            assert len(ci) == min(k - 1, b - a)
+            ids += [a + i for i in ci]
+            scores += cs
+        got = O.merge_block_candidates(ids, scores, lb, k)
+        assert got == O.select_blocks(S, k)
+        if lb <= 10:
+            assert got == _brute_top_set(S, lb, k)
+
+
+def test_key_range_candidates_catch_planted_mistakes():
+    """Ties broken toward the higher index, or NaN ranked above numbers, in
+    either function change the merged selection on some cut."""
+    rng = np.random.default_rng(7)
+
+    def cand_high_tie(S, k):
+        keys = np.where(np.isnan(S), -np.inf, S)
+        order = np.lexsort((-np.arange(len(keys)), -keys))[: k - 1]
+        return [int(b) for b in order], [float(keys[b]) for b in order]
+
+    def cand_nan_high(S, k):
+        keys = np.where(np.isnan(S), np.inf, S)
+        order = np.lexsort((np.arange(len(keys)), -keys))[: k - 1]
+        return [int(b) for b in order], [float(keys[b]) for b in order]
+
+    for bad in (cand_high_tie, cand_nan_high):
+        caught = False
+        for _ in range(300):
+            nb, k = int(rng.integers(6, 20)), int(rng.integers(2, 5))
+            S = rng.integers(-2, 3, size=nb).astype(np.float64)
+            S[rng.random(nb) < 0.1] = np.nan
+            lb = nb - 1
+            mid = int(rng.integers(1, lb))
+            ids, scores = [], []
+            for a, b in ((0, mid), (mid, lb)):
+                ci, cs = bad(S[a:b], k)
+                ids += [a + i for i in ci]
+                scores += cs
+            if O.merge_block_candidates(ids, scores, lb, k) != O.select_blocks(S, k):
+                caught = True
+                break
+        assert caught, bad.__name__
