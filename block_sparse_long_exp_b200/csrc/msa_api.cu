@@ -63,6 +63,45 @@ namespace {
 std::atomic<int> g_tile_theta{-1};
 // Query rows per planning window of the KV-outer lists (msa_set_attn_window).
 std::atomic<int> g_attn_window{kDefaultWindow};
+// SMs that msa_prefill gives a pass's combine while the next pass's index
+// top-k runs on the others (msa_set_prefill_overlap; 0: no overlap, the
+// default: on B200 a combine on a slice of the SMs is latency-bound and
+// outlasts the index pass it would hide behind).
+constexpr int kDefaultOverlapSms = 0;
+std::atomic<int> g_overlap_sms{kDefaultOverlapSms};
+
+// Per device: the second stream of msa_prefill and its two events, created on
+// first use and kept for the life of the process.  The mutex is held while a
+// call enqueues its work, so concurrent calls never interleave their records
+// and waits on the shared events.
+constexpr int kMaxSideDevices = 64;
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t main_done = nullptr;   // a pass's main phase is done (its partials are written)
+  cudaEvent_t comb_done = nullptr;   // a pass's combine is done (its workspace may be reused)
+};
+std::mutex g_side_mu;
+SideStream g_side[kMaxSideDevices];
+
+// Called with g_side_mu held.
+SideStream* side_stream() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxSideDevices) return nullptr;
+  SideStream& s = g_side[dev];
+  if (s.stream == nullptr) {
+    cudaStream_t st = nullptr;
+    cudaEvent_t e0 = nullptr, e1 = nullptr;
+    if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&e0, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&e1, cudaEventDisableTiming) != cudaSuccess) {
+      if (e0) cudaEventDestroy(e0);
+      cudaStreamDestroy(st);
+      return nullptr;
+    }
+    s.stream = st; s.main_done = e0; s.comb_done = e1;
+  }
+  return &s;
+}
 
 constexpr size_t kAlign = 256;
 
@@ -131,22 +170,9 @@ int64_t chunk_rows(const msa_varlen_t* v, int64_t q_chunk) {
   return q_chunk;
 }
 
-msa_status_t attn_common(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q, const void* k,
-                         const void* v, const int32_t* sel, void* out, float* lse, int64_t q_chunk, void* ws,
-                         size_t ws_bytes, void* stream) {
-  msa_status_t st = check_shape(shape);
-  if (st != MSA_OK) return st;
-  st = check_seqs(seqs);
-  if (st != MSA_OK) return st;
-  // no queries: nothing is read or written (empty tensors may have no storage)
-  if (seqs->total_q > 0 && (!q || !k || !v || !sel || !out)) return MSA_ERR_INVALID_ARG;
-  const int64_t rows = chunk_rows(seqs, q_chunk);
-  const AttnLayout L = attn_layout(shape, seqs, rows);
-  if (!ws_ok(ws, ws_bytes, L.total)) return MSA_ERR_WORKSPACE;
-  uint8_t* base = static_cast<uint8_t*>(ws);
-  if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return MSA_ERR_CUDA;
-  if (seqs->total_q == 0) return MSA_OK;
+// Attention arguments of a call whose workspace `base` has layout L.
+AttnArgs attn_args(const msa_shape_t* shape, const msa_varlen_t* seqs, const AttnLayout& L, uint8_t* base,
+                   const void* q, const void* k, const void* v, const int32_t* sel, void* out, float* lse) {
   AttnArgs a{};
   a.q = q; a.key = k; a.value = v; a.sel = sel; a.out = out; a.lse = lse;
   a.cu_q = seqs->cu_q; a.cu_k = seqs->cu_k;
@@ -178,6 +204,25 @@ msa_status_t attn_common(const msa_shape_t* shape, const msa_varlen_t* seqs, con
   a.dmember = reinterpret_cast<uint64_t*>(base + L.dmember);
   a.clist = reinterpret_cast<uint2*>(base + L.clist);
   a.tile_ctr = reinterpret_cast<int32_t*>(base + L.tile_ctr);
+  return a;
+}
+
+msa_status_t attn_common(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q, const void* k,
+                         const void* v, const int32_t* sel, void* out, float* lse, int64_t q_chunk, void* ws,
+                         size_t ws_bytes, void* stream) {
+  msa_status_t st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  st = check_seqs(seqs);
+  if (st != MSA_OK) return st;
+  // no queries: nothing is read or written (empty tensors may have no storage)
+  if (seqs->total_q > 0 && (!q || !k || !v || !sel || !out)) return MSA_ERR_INVALID_ARG;
+  const int64_t rows = chunk_rows(seqs, q_chunk);
+  const AttnLayout L = attn_layout(shape, seqs, rows);
+  if (!ws_ok(ws, ws_bytes, L.total)) return MSA_ERR_WORKSPACE;
+  if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  if (seqs->total_q == 0) return MSA_OK;
+  AttnArgs a = attn_args(shape, seqs, L, static_cast<uint8_t*>(ws), q, k, v, sel, out, lse);
   for (int64_t t0 = 0; t0 < seqs->total_q; t0 += rows) {
     a.t0 = t0;
     a.t1 = t0 + rows < seqs->total_q ? t0 + rows : seqs->total_q;
@@ -348,6 +393,87 @@ msa_status_t msa_sparse_attn_prefill(const msa_shape_t* shape, const msa_varlen_
                                      const void* k, const void* v, const int32_t* sel, void* out, float* lse,
                                      int64_t q_chunk, void* ws, size_t ws_bytes, void* stream) {
   return attn_common(shape, seqs, q, k, v, sel, out, lse, q_chunk, ws, ws_bytes, stream);
+}
+
+size_t msa_prefill_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs, int64_t q_chunk) {
+  if (check_shape(shape) != MSA_OK || check_seqs(seqs) != MSA_OK) return 0;
+  if (seqs->max_q_len <= 1 || seqs->batch > kMaxBatchTiles) return 0;
+  return attn_layout(shape, seqs, chunk_rows(seqs, q_chunk)).total;
+}
+
+msa_status_t msa_prefill(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q, const void* k,
+                         const void* v, const void* q_idx, const void* k_idx, int32_t* sel, void* out, float* lse,
+                         int64_t q_chunk, void* ws, size_t ws_bytes, void* stream) {
+  msa_status_t st = check_shape(shape);
+  if (st != MSA_OK) return st;
+  st = check_seqs(seqs);
+  if (st != MSA_OK) return st;
+  if (seqs->max_q_len <= 1) return MSA_ERR_INVALID_ARG;            // decode shapes: the decode calls
+  if (seqs->batch > kMaxBatchTiles) return MSA_ERR_UNSUPPORTED;
+  if (seqs->total_q > 0 && (!q || !k || !v || !q_idx || !k_idx || !sel || !out)) return MSA_ERR_INVALID_ARG;
+  const int64_t rows = chunk_rows(seqs, q_chunk);
+  const AttnLayout L = attn_layout(shape, seqs, rows);
+  if (!ws_ok(ws, ws_bytes, L.total)) return MSA_ERR_WORKSPACE;
+  cudaStream_t main = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(DevError), main) != cudaSuccess) return MSA_ERR_CUDA;
+  if (seqs->total_q == 0) return MSA_OK;
+  AttnArgs a = attn_args(shape, seqs, L, static_cast<uint8_t*>(ws), q, k, v, sel, out, lse);
+  IndexTopkArgs ia{};
+  ia.q_idx = q_idx; ia.k_idx = k_idx; ia.sel = sel;
+  ia.cu_q = seqs->cu_q; ia.cu_k = seqs->cu_k;
+  ia.batch = seqs->batch; ia.G = shape->G; ia.d_idx = shape->d_idx; ia.k = shape->k; ia.B_k = shape->B_k;
+  ia.total_q = seqs->total_q; ia.total_k = seqs->total_k;
+  ia.max_q_len = seqs->max_q_len; ia.max_k_len = seqs->max_k_len;
+  ia.err = a.err;
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  const int64_t npass = (seqs->total_q + rows - 1) / rows;
+  int csms = g_overlap_sms.load(std::memory_order_relaxed);
+  if (csms > nsm / 2) csms = nsm / 2;
+  std::unique_lock<std::mutex> lk(g_side_mu, std::defer_lock);
+  SideStream* side = nullptr;
+  if (npass > 1 && csms > 0) {
+    lk.lock();
+    side = side_stream();
+    if (side == nullptr) return MSA_ERR_CUDA;
+  }
+  // Per pass p: index top-k of its rows (the tiles whose first row is in the
+  // pass), the main phase, then the combine.  With a side stream, the combine
+  // of pass p runs there on csms SMs while the index top-k of pass p + 1 runs
+  // on the other SMs; the main phase of pass p + 1 waits for that combine (it
+  // reuses the pass workspace).  The last pass combines on the caller's stream.
+  bool ok = true;
+  for (int64_t p = 0; p < npass && ok; ++p) {
+    a.t0 = p * rows;
+    a.t1 = a.t0 + rows < seqs->total_q ? a.t0 + rows : seqs->total_q;
+    ia.row0 = a.t0;
+    ia.row1 = p == npass - 1 ? seqs->total_q : a.t1;
+    ia.grid = (side != nullptr && p > 0) ? nsm - csms : 0;
+    ok = launch_index_topk_prefill(ia, stream) == 0;
+    if (ok && side != nullptr && p > 0) ok = cudaStreamWaitEvent(main, side->comb_done, 0) == cudaSuccess;
+    if (ok) ok = launch_sparse_attn_main(a, stream) == 0;
+    if (!ok) break;
+    if (side != nullptr && p < npass - 1) {
+      ok = cudaEventRecord(side->main_done, main) == cudaSuccess &&
+           cudaStreamWaitEvent(side->stream, side->main_done, 0) == cudaSuccess &&
+           launch_sparse_attn_combine(a, side->stream, csms) == 0 &&
+           cudaEventRecord(side->comb_done, side->stream) == cudaSuccess;
+    } else {
+      ok = launch_sparse_attn_combine(a, stream, 0) == 0;
+    }
+  }
+  if (!ok && side != nullptr) {
+    // the caller's stream still waits for whatever reached the side stream
+    cudaEventRecord(side->comb_done, side->stream);
+    cudaStreamWaitEvent(main, side->comb_done, 0);
+  }
+  return ok ? MSA_OK : MSA_ERR_CUDA;
+}
+
+int32_t msa_set_prefill_overlap(int32_t sms) {
+  return g_overlap_sms.exchange(sms < 0 ? kDefaultOverlapSms : sms);
 }
 
 msa_status_t msa_sparse_attn_decode(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q,

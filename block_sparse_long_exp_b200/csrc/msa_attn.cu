@@ -926,7 +926,7 @@ combine_kernel(const __half* __restrict__ part_acc, const float* __restrict__ pa
 
 int launch_combine_kernel(const __half* part_acc, const float* part_lse, const int32_t* sel, const uint2* clist,
                           const int32_t* npairs_dev, __nv_bfloat16* out, float* lse, int64_t T, int H, int G, int d,
-                          int k, DevError* err, cudaStream_t st) {
+                          int k, DevError* err, cudaStream_t st, int grid_cap = 0) {
   if (T <= 0) return 0;
   const int Hg = H / G;
   const int per = Hg * (d / 8);
@@ -947,7 +947,8 @@ int launch_combine_kernel(const __half* part_acc, const float* part_lse, const i
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   const int64_t nchunks = (T * G + P - 1) / P;   // upper bound when a list is given
-  const int grid = (int)(nchunks < nsm ? nchunks : nsm);
+  const int cap = grid_cap > 0 && grid_cap < nsm ? grid_cap : nsm;
+  const int grid = (int)(nchunks < cap ? nchunks : cap);
   combine_kernel<<<grid, kCombThreads, smem, st>>>(part_acc, part_lse, sel, clist, npairs_dev, out, lse, T, H, G, d,
                                                   k, P, acc_bytes, lse_bytes, err);
   return (int)cudaGetLastError();
@@ -957,7 +958,7 @@ int launch_combine_kernel(const __half* part_acc, const float* part_lse, const i
 
 // -------------------------------------------------------------- launchers ---
 
-int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
+int launch_sparse_attn_main(const AttnArgs& a, void* stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t nrows = a.t1 - a.t0;
   if (nrows <= 0) return 0;
@@ -1045,12 +1046,23 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
     const int rc = launch_tile_attn(a, stream);
     if (rc) return rc;
   }
+  return 0;
+}
+
+int launch_sparse_attn_combine(const AttnArgs& a, void* stream, int grid_cap) {
   const int64_t rows = a.t1 - a.t0;
+  if (rows <= 0) return 0;
   ProfScope p("combine", stream);
   return launch_combine_kernel(reinterpret_cast<const __half*>(a.part_acc), a.part_lse, a.sel + a.t0 * a.G * a.k,
-                               a.clist, tiles ? a.tile_ctr : nullptr,
+                               a.clist, a.theta > 0 ? a.tile_ctr : nullptr,
                                reinterpret_cast<__nv_bfloat16*>(a.out) + a.t0 * a.H * a.d,
-                               a.lse ? a.lse + a.t0 * a.H : nullptr, rows, a.H, a.G, a.d, a.k, a.err, st);
+                               a.lse ? a.lse + a.t0 * a.H : nullptr, rows, a.H, a.G, a.d, a.k, a.err,
+                               reinterpret_cast<cudaStream_t>(stream), grid_cap);
+}
+
+int launch_sparse_attn_pass(const AttnArgs& a, void* stream) {
+  const int rc = launch_sparse_attn_main(a, stream);
+  return rc ? rc : launch_sparse_attn_combine(a, stream, 0);
 }
 
 int launch_combine(const void* part_acc, const float* part_lse, const int32_t* sel, void* out, float* lse,

@@ -37,8 +37,8 @@ struct __align__(16) IndexCtl {
   uint64_t mma_done[2];
   uint32_t tmem_base;
   int32_t abort_flag;
-  int32_t ntiles;
-  int32_t pad;
+  int32_t ntiles;             // tiles of this launch: tau0 .. tau0 + ntiles - 1
+  int32_t tau0;
   int32_t tile_prefix[kMaxBatchTiles + 1];
 };
 
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           int32_t* __restrict__ sel, const int32_t* __restrict__ cu_q,
                           const int32_t* __restrict__ cu_k, int batch, int d_idx, int k, int B_k, int nst,
-                          DevError* err) {
+                          int64_t row0, int64_t row1, DevError* err) {
   constexpr int CAP = KMAX - 1;
   constexpr int GP = G < 2 ? G : 2;          // groups per work unit
   constexpr int NPAIR = (G + GP - 1) / GP;   // units per tile
@@ -215,7 +215,26 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
       acc += (Tb + kTile - 1) / kTile;
     }
     ctl->tile_prefix[batch] = acc;
-    ctl->ntiles = acc;
+    // this launch takes the tiles whose first row lies in [row0, row1) (first
+    // rows grow with the tile index, so that is a contiguous range)
+    auto first_at_or_after = [&](int64_t row) {
+      int lo = 0, hi = acc;   // smallest tau with q0(tau) >= row
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        int b = 0, bh = batch;
+        while (bh - b > 1) {
+          const int m2 = (b + bh) >> 1;
+          if (ctl->tile_prefix[m2] <= mid) b = m2; else bh = m2;
+        }
+        const int64_t q0 = (int64_t)cu_q[b] + (int64_t)kTile * (mid - ctl->tile_prefix[b]);
+        if (q0 >= row) hi = mid; else lo = mid + 1;
+      }
+      return lo;
+    };
+    const int t0 = first_at_or_after(row0);
+    const int t1 = first_at_or_after(row1);
+    ctl->tau0 = t0;
+    ctl->ntiles = t1 > t0 ? t1 - t0 : 0;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -239,7 +258,7 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
         const int u = snake_unit(it, nunits);
         if (u < 0 || *abort_flag) break;
         const int pair = u % NPAIR;
-        const TileInfo ti = tile_info(u / NPAIR, ctl, batch, cu_q, cu_k, B_k);
+        const TileInfo ti = tile_info(ctl->tau0 + u / NPAIR, ctl, batch, cu_q, cu_k, B_k);
         if (!mbar_wait(&ctl->q_empty, (qiter + 1) & 1)) {
           report_error(err, MSA_ERR_TIMEOUT, kSiteIndexProducer, u, -1);
           *abort_flag = 1;
@@ -290,7 +309,7 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
       for (int it = 0; ok; ++it) {
         const int u = snake_unit(it, nunits);
         if (u < 0 || *abort_flag) break;
-        const TileInfo ti = tile_info(u / NPAIR, ctl, batch, cu_q, cu_k, B_k);
+        const TileInfo ti = tile_info(ctl->tau0 + u / NPAIR, ctl, batch, cu_q, cu_k, B_k);
         if (!mbar_wait(&ctl->q_full, qiter & 1)) {
           report_error(err, MSA_ERR_TIMEOUT, kSiteIndexMma, u, -1);
           ok = false;
@@ -340,7 +359,7 @@ index_topk_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid
       const int u = snake_unit(it, nunits);
       if (u < 0 || *abort_flag) break;
       const int g = (u % NPAIR) * GP + l;
-      const TileInfo ti = tile_info(u / NPAIR, ctl, batch, cu_q, cu_k, B_k);
+      const TileInfo ti = tile_info(ctl->tau0 + u / NPAIR, ctl, batch, cu_q, cu_k, B_k);
       const bool valid = row < ti.rows;
       const int lb = (ti.pos0 + row) / B_k;
       list.reset();
@@ -427,6 +446,8 @@ int launch_index_topk_prefill(const IndexTopkArgs& a, void* stream) {
   int dev = 0, nsm = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = a.grid > 0 && a.grid < nsm ? a.grid : nsm;
+  const int64_t row1 = a.row1 > 0 ? a.row1 : a.total_q;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaErrorInvalidValue;
 #define MSA_IDX(KM, GG)                                                                                        \
@@ -435,8 +456,9 @@ int launch_index_topk_prefill(const IndexTopkArgs& a, void* stream) {
                              (int)smem);                                                                       \
     if (e != cudaSuccess) return (int)e;                                                                       \
     ProfScope p("index_topk_prefill", stream);                                                                 \
-    index_topk_prefill_kernel<KM, GG><<<nsm, kThreads, smem, st>>>(tm_q, tm_k, a.sel, a.cu_q, a.cu_k, a.batch, \
-                                                                   a.d_idx, a.k, a.B_k, nst, a.err);         \
+    index_topk_prefill_kernel<KM, GG><<<grid, kThreads, smem, st>>>(tm_q, tm_k, a.sel, a.cu_q, a.cu_k, a.batch, \
+                                                                    a.d_idx, a.k, a.B_k, nst, a.row0, row1,   \
+                                                                    a.err);                                   \
     return (int)cudaGetLastError();                                                                            \
   }
   MSA_IDX(8, 1) MSA_IDX(8, 2) MSA_IDX(8, 4)

@@ -93,6 +93,10 @@ struct IndexTopkArgs {
   const int32_t* block_table;   // null: packed rows cu_k[b] + j * B_k
   int32_t max_blocks;
   int64_t num_pages;
+  // prefill: the 128-query tiles whose first row lies in [row0, row1) (row1 <= 0: total_q),
+  // on `grid` CTAs (<= 0: one per SM)
+  int64_t row0, row1;
+  int32_t grid;
 };
 int launch_index_topk_prefill(const IndexTopkArgs& a, void* stream);
 int launch_index_topk_decode(const IndexTopkArgs& a, void* stream);
@@ -143,7 +147,12 @@ struct AttnArgs {
   int32_t max_blocks;
   int64_t num_pages;
 };
-int launch_sparse_attn_pass(const AttnArgs& a, void* stream);
+int launch_sparse_attn_pass(const AttnArgs& a, void* stream);   // main phase, then the combine
+// The two phases of a pass on their own: the main phase (planning, lists,
+// KV-outer and query-tile attention) writes the pass's partials; the combine
+// merges them into out / lse (on at most grid_cap CTAs; <= 0: one per SM).
+int launch_sparse_attn_main(const AttnArgs& a, void* stream);
+int launch_sparse_attn_combine(const AttnArgs& a, void* stream, int grid_cap);
 int attn_window_rows();                // planning window of the prefill calls (msa_set_attn_window)
 int launch_combine(const void* part_acc, const float* part_lse, const int32_t* sel, void* out,
                    float* lse, int64_t T, int32_t H, int32_t G, int32_t d, int32_t k, void* stream);

@@ -55,6 +55,7 @@ EXPORTED = [
     "msa_decode_paged_workspace_size", "msa_index_topk_decode_paged", "msa_sparse_attn_decode_paged",
     "msa_index_kl", "msa_index_kl_backward", "msa_select_window", "msa_sparse_attn_backward",
     "msa_selected_share", "msa_index_topk_policy", "msa_gather_pages",
+    "msa_prefill_workspace_size", "msa_prefill", "msa_set_prefill_overlap",
 ]
 
 
@@ -105,6 +106,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_sparse_attn_prefill.restype = i32
     lib.msa_sparse_attn_decode.argtypes = [P(Shape), P(Varlen), vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.msa_sparse_attn_decode.restype = i32
+    lib.msa_prefill_workspace_size.argtypes = [P(Shape), P(Varlen), i64]
+    lib.msa_prefill_workspace_size.restype = sz
+    lib.msa_prefill.argtypes = [P(Shape), P(Varlen), vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, sz, vp]
+    lib.msa_prefill.restype = i32
+    lib.msa_set_prefill_overlap.argtypes = [i32]
+    lib.msa_set_prefill_overlap.restype = i32
     lib.msa_combine.argtypes = [P(Shape), i64, vp, vp, vp, vp, vp, vp]
     lib.msa_combine.restype = i32
     lib.msa_dense_attn_workspace_size.argtypes = [P(Shape), P(Varlen)]
@@ -384,6 +391,59 @@ def msa_sparse_attn_prefill(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torc
     if check:
         _device_check(ws, stream, "msa_sparse_attn_prefill")
     return out, lse
+
+
+def msa_prefill_workspace_size(shape: Shape, seqs: Varlen, q_chunk: int = 0) -> int:
+    """Workspace bytes of msa_prefill (0: unsupported)."""
+    return load_library().msa_prefill_workspace_size(ctypes.byref(shape), ctypes.byref(seqs), q_chunk)
+
+
+def msa_prefill(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                q_idx: torch.Tensor, k_idx: torch.Tensor, sel: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+                q_chunk: int = 0, ws: Optional[torch.Tensor] = None, stream=None,
+                check: bool = True) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
+    """One MSA layer, prefill: index top-k and the main branch in passes of
+    q_chunk query rows (the combine of a pass overlaps the next pass's index
+    top-k).  Returns sel [T, G, k], out [T, H, d] and lse [T, H] (None with
+    want_lse=False), equal to msa_index_topk followed by
+    msa_sparse_attn_prefill with the same q_chunk."""
+    lib = load_library()
+    T, S = seqs.total_q, seqs.total_k
+    _arg("q", q, torch.bfloat16, (T, shape.H, shape.d))
+    _arg("k", k, torch.bfloat16, (S, shape.G, shape.d))
+    _arg("v", v, torch.bfloat16, (S, shape.G, shape.d))
+    _arg("q_idx", q_idx, torch.bfloat16, (T, shape.G, shape.d_idx))
+    _arg("k_idx", k_idx, torch.bfloat16, (S, shape.d_idx))
+    _arg("sel", sel, torch.int32, (T, shape.G, shape.k), optional=True)
+    _arg("out", out, torch.bfloat16, (T, shape.H, shape.d), optional=True)
+    _arg("lse", lse, torch.float32, (T, shape.H), optional=True)
+    _ws_arg(ws)
+    _require_cuda(q, k, v, q_idx, k_idx, sel, out, lse, ws)
+    if sel is None:
+        sel = torch.empty((T, shape.G, shape.k), dtype=torch.int32, device=q.device)
+    if out is None:
+        out = torch.empty((T, shape.H, shape.d), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((T, shape.H), dtype=torch.float32, device=q.device)
+    need = msa_prefill_workspace_size(shape, seqs, q_chunk)
+    if need == 0:
+        raise MsaError("msa_prefill: unsupported or invalid shape")
+    if ws is None:
+        ws = _workspace(need, q.device)
+    rc = lib.msa_prefill(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q), _ptr(k), _ptr(v), _ptr(q_idx),
+                         _ptr(k_idx), _ptr(sel), _ptr(out), _ptr(lse), q_chunk, _ptr(ws), _nbytes(ws),
+                         _stream(stream))
+    _check(rc, "msa_prefill")
+    if check:
+        _device_check(ws, stream, "msa_prefill")
+    return sel, out, lse
+
+
+def msa_set_prefill_overlap(sms: int) -> int:
+    """SMs msa_prefill gives a pass's combine while the next pass's index
+    top-k runs (< 0: the default, 0: no overlap); returns the previous value."""
+    return int(load_library().msa_set_prefill_overlap(int(sms)))
 
 
 def msa_sparse_attn_decode(shape: Shape, seqs: Varlen, q: torch.Tensor, k_cache: torch.Tensor,

@@ -158,6 +158,55 @@ msa_status_t msa_sparse_attn_prefill(const msa_shape_t* shape, const msa_varlen_
                                      int64_t q_chunk,
                                      void* ws, size_t ws_bytes, void* stream);
 
+/* One MSA layer, prefill: the Index Branch and the Main Branch of the same
+ * layer in one call (pnsm.cn sec. 2: block scoring and top-k select the
+ * blocks, then block-sparse attention runs over them; yololab.net
+ * "MSA的兩個主要步驟").  Writes the selection `sel` exactly as msa_index_topk
+ * and `out` / `lse` exactly as msa_sparse_attn_prefill with the same q_chunk
+ * (bit for bit: every row is computed by the same kernels in the same order).
+ *
+ * The work runs in passes of q_chunk query rows (0 = all rows in one pass).
+ * For each pass: the index top-k of the 128-query tiles whose first row lies
+ * in the pass, then the pass's attention.  With more than one pass the
+ * library overlaps the combine of pass p (memory-bound) with the index top-k
+ * of pass p + 1 (compute-bound, few DRAM bytes): the combine runs on a second
+ * stream of the library's own, on the SMs set by msa_set_prefill_overlap, the
+ * index kernel on the others; events order the two streams, and when the call
+ * returns everything it enqueued is ordered before later work on `stream`.
+ * Calls from several host threads serialize their enqueue on one lock.  The
+ * overlap is off by default: measured on B200 at 128K tokens, a combine on 16
+ * to 48 of the 148 SMs is bound by its own latency and outlasts the index pass
+ * it hides behind (the step got 3-20 ms slower), so every pass runs on the
+ * caller's stream over all SMs unless msa_set_prefill_overlap asks otherwise.
+ *
+ * q_idx / k_idx as msa_index_topk, q / k / v / out / lse as
+ * msa_sparse_attn_prefill.  Prefill shapes only (max_q_len > 1; decode has its
+ * own calls) and at most 1024 sequences.  Workspace: one block of
+ * msa_prefill_workspace_size bytes (256-byte aligned); its error word reports
+ * both branches' device checks. */
+size_t msa_prefill_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs, int64_t q_chunk);
+
+msa_status_t msa_prefill(const msa_shape_t* shape, const msa_varlen_t* seqs,
+                         const void* q,      /* device bf16 [T, H, d] */
+                         const void* k,      /* device bf16 [S, G, d] */
+                         const void* v,      /* device bf16 [S, G, d] */
+                         const void* q_idx,  /* device bf16 [T, G, d_idx] */
+                         const void* k_idx,  /* device bf16 [S, d_idx] */
+                         int32_t* sel,       /* device int32 [T, G, k] (out) */
+                         void* out,          /* device bf16 [T, H, d] (out) */
+                         float* lse,         /* device f32 [T, H] (out) or NULL */
+                         int64_t q_chunk,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* SMs that msa_prefill gives the combine of a pass while the next pass's
+ * index top-k runs on the rest; returns the previous value.
+ *   sms < 0     the default (0)
+ *   sms == 0    no overlap: every kernel of the call runs on the caller's
+ *               stream over all SMs
+ *   otherwise   at most half of the device's SMs
+ * Results do not depend on it.  One atomic word, read once per call. */
+int32_t msa_set_prefill_overlap(int32_t sms);
+
 /* Main Branch, decode: one query per sequence (T_b = 1, position S_b - 1,
  * the cache already holding the new token), the decode step of pnsm.cn
  * sec. 9 and yhxrc.cn sec. 二.  Same contract as the prefill call; q_chunk

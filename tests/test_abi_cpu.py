@@ -265,3 +265,47 @@ def test_block_size_128_only_entry_points(lib):
     table = (ctypes.c_int32 * 8)(*range(8))
     pages = msa.Paged(1, 8, 1000, 0, 8, ctypes.addressof(lens), ctypes.addressof(table))
     assert lib.msa_decode_paged_workspace_size(ctypes.byref(sh64), ctypes.byref(pages)) == 0
+
+
+def test_fused_prefill_host_checks(lib):
+    """msa_prefill answers bad arguments before any launch: decode shapes and
+    more than 1024 sequences are refused, NULL data pointers with queries are
+    invalid, a short workspace is refused; its workspace is the main branch's
+    for the same pass size; the overlap setter returns the previous value."""
+    from block_sparse_long_exp_b200 import msa
+    shape = msa.make_shape(64, 4, 128, 64, 16)
+    cu = (ctypes.c_int32 * 2)(0, 0)
+    a = ctypes.addressof(cu)
+    seqs = msa.Varlen(1, 4096, 4096, 0, 4096, 4096, a, a)
+    for q_chunk in (0, 1024, 700):
+        need = lib.msa_prefill_workspace_size(ctypes.byref(shape), ctypes.byref(seqs), q_chunk)
+        assert need > 0 and need == lib.msa_sparse_attn_workspace_size(ctypes.byref(shape), ctypes.byref(seqs),
+                                                                       q_chunk)
+    decode = msa.Varlen(4, 1, 4096, 0, 4, 16384, a, a)
+    assert lib.msa_prefill_workspace_size(ctypes.byref(shape), ctypes.byref(decode), 0) == 0
+    p = [256] * 8
+    rc = lib.msa_prefill(ctypes.byref(shape), ctypes.byref(decode), *p, 0, 256, 1 << 30, None)
+    assert rc == 1                                       # MSA_ERR_INVALID_ARG: decode shapes have their own calls
+    many = msa.Varlen(1025, 2, 2, 0, 2050, 2050, a, a)
+    assert lib.msa_prefill_workspace_size(ctypes.byref(shape), ctypes.byref(many), 0) == 0
+    rc = lib.msa_prefill(ctypes.byref(shape), ctypes.byref(many), *p, 0, 256, 1 << 30, None)
+    assert rc == 2                                       # MSA_ERR_UNSUPPORTED
+    for i in range(7):                                   # q k v q_idx k_idx sel out (lse may be NULL)
+        q = list(p)
+        q[i] = None
+        rc = lib.msa_prefill(ctypes.byref(shape), ctypes.byref(seqs), *q, 0, 256, 1 << 30, None)
+        assert rc == 1, i
+    rc = lib.msa_prefill(ctypes.byref(shape), ctypes.byref(seqs), *p, 0, 256, 16, None)
+    assert rc == 3                                       # MSA_ERR_WORKSPACE
+    bad_bk = msa.make_shape(64, 4, 128, 64, 16, B_k=96)
+    rc = lib.msa_prefill(ctypes.byref(bad_bk), ctypes.byref(seqs), *p, 0, 256, 1 << 30, None)
+    assert rc == 2
+    rc = lib.msa_prefill(None, ctypes.byref(seqs), *p, 0, 256, 1 << 30, None)
+    assert rc == 1
+    prev = lib.msa_set_prefill_overlap(16)
+    try:
+        assert lib.msa_set_prefill_overlap(0) == 16
+        assert lib.msa_set_prefill_overlap(-5) == 0      # < 0: back to the default
+        assert lib.msa_set_prefill_overlap(prev) == 0    # the default: no overlap
+    finally:
+        lib.msa_set_prefill_overlap(prev)
