@@ -85,5 +85,5 @@ def test_fused_full_size_in_four_passes(M):
     ref = _separate(M, shape, seqs, inp, 32768)
     for overlap in (0, 32):
         _assert_same(_fused(M, shape, seqs, inp, 32768, overlap), ref)
-    del ref, got, inp
+    del ref, inp
     torch.cuda.empty_cache()
