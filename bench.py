@@ -207,9 +207,10 @@ def training_leg(args, w, W, R, msa, torch, device="cuda"):
     with the workload's heads and dimensions: the Main Branch backward for a
     seeded upstream gradient, then the KL target (tau = 0.125) and its
     gradient, fed by the forward's selection and log-sum-exps.  Each kernel is
-    timed by the library's CUDA events on its launching stream over args.steps
-    passes after args.warmup (inputs larger than L2).  They run on the CUDA
-    cores, so the roofline is the fp32 FMA rate."""
+    timed by the library's CUDA events on its launching stream over
+    args.training_steps passes after args.training_warmup (inputs larger than
+    L2; its own small counts, since one pass takes about 2 s).  They run on the
+    CUDA cores, so the roofline is the fp32 FMA rate."""
     tinp = W.make_inputs(w, device, T_override=args.training_T)
     shape = msa.make_shape(w.H, w.G, w.d, w.d_idx, w.k)
     seqs = msa.make_varlen(tinp["cu_q"], tinp["cu_k"], tinp["cu_q_host"], tinp["cu_k_host"])
@@ -226,12 +227,12 @@ def training_leg(args, w, W, R, msa, torch, device="cuda"):
         msa.msa_index_kl_backward(shape, seqs, q, k, q_idx, k_idx, sel, lse, lse_z, tau, check=check)
 
     one(True)
-    for _ in range(args.warmup):
+    for _ in range(args.training_warmup):
         one(False)
     torch.cuda.synchronize()
     msa.msa_profile_reset()
     msa.msa_profile_enable(True)
-    for _ in range(args.steps):
+    for _ in range(args.training_steps):
         one(False)
     torch.cuda.synchronize()
     msa.msa_profile_enable(False)
@@ -241,7 +242,7 @@ def training_leg(args, w, W, R, msa, torch, device="cuda"):
     tw = R.training_work(S_lens, T_lens, w.H, w.G, w.d, w.d_idx, w.B_k, w.k)
     peak = R.alu_fp32_tflops()
     res = {"workload": f"{args.workload} at T = {sum(T_lens)}", "T": sum(T_lens), "tau": tau,
-           "steps": args.steps, "warmup": args.warmup, "peak": peak, "unit": "TFLOP/s",
+           "steps": args.training_steps, "warmup": args.training_warmup, "peak": peak, "unit": "TFLOP/s",
            "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOPs x 1965 MHz (CUDA cores, nominal)",
            "kernels": {}}
     for name, key in (("attn_bwd", "backward_flops"), ("index_kl", "kl_flops"), ("index_kl_grad", "kl_grad_flops")):
@@ -796,9 +797,13 @@ def build_parser():
                     help="query rows per planning window of the KV-outer lists (0: the library's default)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=64)
-    ap.add_argument("--training", action="store_true",
-                    help="also time the backward and KL kernels (CUDA cores) on a --training-T layer")
+    ap.add_argument("--no-training", dest="training", action="store_false",
+                    help="skip the training leg (the backward and KL kernels, CUDA cores, on a --training-T layer)")
+    ap.add_argument("--training", dest="training", action="store_true", help=argparse.SUPPRESS)
     ap.add_argument("--training-T", type=int, default=32768)
+    ap.add_argument("--training-steps", type=int, default=2)
+    ap.add_argument("--training-warmup", type=int, default=1)
+    ap.set_defaults(training=True)
     ap.add_argument("--shard", choices=["none", "queries"], default="none",
                     help="N > 1: independent layers per rank (none, weak scaling) or the query ranges of one "
                          "layer split across ranks (queries, strong scaling)")
