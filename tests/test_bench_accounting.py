@@ -179,7 +179,9 @@ def test_training_leg_reports_each_kernel_against_the_alu_peak():
         msa_profile_reset=stand_in("msa_profile_reset", lambda: None),
         msa_profile_enable=stand_in("msa_profile_enable", lambda on: None),
         msa_profile_read=stand_in("msa_profile_read", lambda name=None: (8.0, 4)))
-    args = bench.build_parser().parse_args(["--training", "--training-T", str(T), "--steps", "4", "--warmup", "3"])
+    args = bench.build_parser().parse_args(["--training-T", str(T), "--training-steps", "4",
+                                            "--training-warmup", "3"])
+    assert args.training                         # the training leg is part of the default run
     sync = torch.cuda.synchronize
     torch.cuda.synchronize = lambda *a: None
     try:
