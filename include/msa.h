@@ -174,6 +174,9 @@ msa_status_t msa_sparse_attn_prefill(const msa_shape_t* shape, const msa_varlen_
  * index kernel on the others; events order the two streams, and when the call
  * returns everything it enqueued is ordered before later work on `stream`.
  * Calls from several host threads serialize their enqueue on one lock.  The
+ * second stream and its two events are created by the first overlapped call on
+ * a device and kept for the life of the process (a cudaDeviceReset ends their
+ * use on that device: later overlapped calls there return MSA_ERR_CUDA).  The
  * overlap is off by default: measured on B200 at 128K tokens, a combine on 16
  * to 48 of the 148 SMs is bound by its own latency and outlasts the index pass
  * it hides behind (the step got 3-20 ms slower), so every pass runs on the
