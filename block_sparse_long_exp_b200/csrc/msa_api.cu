@@ -673,6 +673,10 @@ msa_status_t msa_sparse_attn_backward(const msa_shape_t* shape, const msa_varlen
   if (seqs->total_q > 0 &&
       (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || (!dense && !sel)))
     return MSA_ERR_INVALID_ARG;
+  // key / value rows are read, and dk / dv rows added, 16 bytes at a time
+  if (seqs->total_q > 0 && ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) |
+                             reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 15u))
+    return MSA_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, kWsHeader)) return MSA_ERR_WORKSPACE;
   cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(ws, 0, sizeof(DevError), st_) != cudaSuccess) return MSA_ERR_CUDA;

@@ -10,11 +10,11 @@
 //   dS_j = P_j (dP_j - D_h),
 //   dq_h = sm_scale sum_j dS_j k_j,  dk_j += sm_scale dS_j q_h,  dv_j += P_j dO_h.
 // The support is numbered in ascending token order and cut into chunks of
-// kBwdChunk tokens.  Phase 1 (one thread per token of the chunk) computes the
-// token's dS for every head of the group, stages its key row, and adds its dk
-// and dv rows (atomically on the device: other queries add to the same rows).
-// Phase 2 (every thread, after a barrier) adds the chunk's share of
-// dq = sm_scale dS . K to the thread's outputs.
+// kBwdChunk tokens whose key and value rows are staged first.  Per chunk:
+// bwd_pds gives P and dS of one (token, head) from the staged rows;
+// bwd_kv_cols gives one column of a token's dk and dv rows, summed over the
+// heads (added atomically on the device: other queries add to the same rows);
+// bwd_phase2 adds the chunk's share of dq = sm_scale dS . K to one output.
 //
 // Plain fp32 arithmetic on bf16 bit patterns; compiled for the device by the
 // kernel and for the host by a test, which replays a CTA phase by phase
@@ -55,14 +55,6 @@ MSA_BWD_HD float bwd_exp(float x) {
   return __expf(x);
 #else
   return std::exp(x);
-#endif
-}
-
-MSA_BWD_HD void bwd_add(float* dst, float v) {
-#ifdef __CUDA_ARCH__
-  atomicAdd(dst, v);
-#else
-  *dst += v;
 #endif
 }
 
@@ -121,56 +113,87 @@ MSA_BWD_HD int64_t bwd_token(const int64_t* first, const int64_t* base, int n, i
   return first[i] + (m - base[i]);
 }
 
-// Phase 1 for support token j: dS of every head into dS[h * kBwdChunk + slot],
-// the key row (bf16 bits) into kstage[0 .. d), and the token's dk / dv rows
-// (dk, dv: the gradients' rows of this sequence, float [S_b, G, d]).
-MSA_BWD_HD void bwd_phase1(const BwdUnit& u, int64_t j, int slot, float* dS, uint16_t* kstage, float* dk, float* dv) {
-  const uint16_t* kj = u.krow + (j * u.G + u.g) * u.d;
-  const uint16_t* vj = u.vrow + (j * u.G + u.g) * u.d;
-  float* dkj = dk + (j * u.G + u.g) * u.d;
-  float* dvj = dv + (j * u.G + u.g) * u.d;
-  // every head's score and dP, reading the key and value rows once
-  float s[kBwdMaxHeads], dp[kBwdMaxHeads], p[kBwdMaxHeads], ds[kBwdMaxHeads];
+// Staged key / value rows: bf16 pairs as 32-bit words, row r at r * rw words
+// (rw = d / 2 + 1: the pad word puts consecutive rows in different banks).
+MSA_BWD_HD float bwd_lo(uint32_t w) { return bwd_bf16(static_cast<uint16_t>(w & 0xffffu)); }
+MSA_BWD_HD float bwd_hi(uint32_t w) { return bwd_bf16(static_cast<uint16_t>(w >> 16)); }
+
+// P and dS of tokens t0 .. t0 + nt - 1 (chunk slots; nt <= 2) and heads
+// h0 .. h0 + nh - 1 (nh <= kBwdPdsHeads) from the staged rows, written to P /
+// dS at [h * stride + slot].  Each (token, head) sum runs over c in ascending
+// order, so the tiling does not change the result.
+constexpr int kBwdPdsHeads = 4;
+constexpr int kBwdPdsTokens = 2;
+MSA_BWD_HD void bwd_pds(const BwdUnit& u, const uint32_t* kst, const uint32_t* vst, int rw, int t0, int nt, int h0,
+                        int nh, float* P, float* dS, int stride) {
+  float s[kBwdPdsTokens][kBwdPdsHeads], dp[kBwdPdsTokens][kBwdPdsHeads];
 MSA_BWD_HD_UNROLL
-  for (int h = 0; h < kBwdMaxHeads; ++h) s[h] = dp[h] = p[h] = ds[h] = 0.f;
-  for (int c = 0; c < u.d; ++c) {
-    kstage[c] = kj[c];
-    const float kc = bwd_bf16(kj[c]), vc = bwd_bf16(vj[c]);
+  for (int a = 0; a < kBwdPdsTokens; ++a)
 MSA_BWD_HD_UNROLL
-    for (int h = 0; h < kBwdMaxHeads; ++h)
-      if (h < u.Hg) {
-        s[h] += u.qf[h * u.d + c] * kc;
-        dp[h] += u.dof[h * u.d + c] * vc;
+    for (int i = 0; i < kBwdPdsHeads; ++i) s[a][i] = dp[a][i] = 0.f;
+  const int t1 = nt > 1 ? t0 + 1 : t0;
+  for (int w = 0; w < u.d / 2; ++w) {
+    const uint32_t k0 = kst[t0 * rw + w], k1 = kst[t1 * rw + w];
+    const uint32_t v0 = vst[t0 * rw + w], v1 = vst[t1 * rw + w];
+    const float kc[2][2] = {{bwd_lo(k0), bwd_hi(k0)}, {bwd_lo(k1), bwd_hi(k1)}};
+    const float vc[2][2] = {{bwd_lo(v0), bwd_hi(v0)}, {bwd_lo(v1), bwd_hi(v1)}};
+MSA_BWD_HD_UNROLL
+    for (int i = 0; i < kBwdPdsHeads; ++i) {
+      if (i >= nh) continue;
+      const float* qh = u.qf + (h0 + i) * u.d + 2 * w;
+      const float* oh = u.dof + (h0 + i) * u.d + 2 * w;
+      const float q0 = qh[0], q1 = qh[1], o0 = oh[0], o1 = oh[1];
+MSA_BWD_HD_UNROLL
+      for (int a = 0; a < kBwdPdsTokens; ++a) {
+        s[a][i] += q0 * kc[a][0];
+        s[a][i] += q1 * kc[a][1];
+        dp[a][i] += o0 * vc[a][0];
+        dp[a][i] += o1 * vc[a][1];
       }
+    }
   }
+MSA_BWD_HD_UNROLL
+  for (int a = 0; a < kBwdPdsTokens; ++a)
+MSA_BWD_HD_UNROLL
+    for (int i = 0; i < kBwdPdsHeads; ++i)
+      if (a < nt && i < nh) {
+        const int h = h0 + i, slot = t0 + a;
+        const float p = bwd_exp(u.sm_scale * s[a][i] - u.lse[h]);
+        P[h * stride + slot] = p;
+        dS[h * stride + slot] = p * (dp[a][i] - u.D[h]);
+      }
+}
+
+// Column c of one token's dk and dv rows, summed over the heads: P and dS hold
+// the token's values at [h * stride + slot].
+MSA_BWD_HD void bwd_kv_cols(const BwdUnit& u, const float* P, const float* dS, int stride, int slot, int c, float* gk,
+                            float* gv) {
+  float k_ = 0.f, v_ = 0.f;
 MSA_BWD_HD_UNROLL
   for (int h = 0; h < kBwdMaxHeads; ++h)
     if (h < u.Hg) {
-      p[h] = bwd_exp(u.sm_scale * s[h] - u.lse[h]);
-      ds[h] = p[h] * (dp[h] - u.D[h]);
-      dS[h * kBwdChunk + slot] = ds[h];
+      k_ += dS[h * stride + slot] * u.qf[h * u.d + c];
+      v_ += P[h * stride + slot] * u.dof[h * u.d + c];
     }
-  // the token's dk / dv rows: one atomic add per element, summed over the heads first
-  for (int c = 0; c < u.d; ++c) {
-    float gk = 0.f, gv = 0.f;
-MSA_BWD_HD_UNROLL
-    for (int h = 0; h < kBwdMaxHeads; ++h)
-      if (h < u.Hg) {
-        gk += ds[h] * u.qf[h * u.d + c];
-        gv += p[h] * u.dof[h * u.d + c];
-      }
-    bwd_add(dkj + c, u.sm_scale * gk);
-    bwd_add(dvj + c, gv);
-  }
+  *gk = u.sm_scale * k_;
+  *gv = v_;
 }
 
-// Phase 2: output o = h * d + c of dq gets sum over the chunk's cnt tokens of
-// dS[h][slot] * k[slot][c] (the caller scales by sm_scale at the end).
-MSA_BWD_HD float bwd_phase2(const BwdUnit& u, const float* dS, const uint16_t* kst, int cnt, int o) {
-  const int h = o / u.d, c = o - h * u.d;
-  float acc = 0.f;
-  for (int s = 0; s < cnt; ++s) acc += dS[h * kBwdChunk + s] * bwd_bf16(kst[s * u.d + c]);
-  return acc;
+// dq outputs (h, c0 .. c0 + 7) of one chunk: acc[e] += sum over the chunk's cnt
+// tokens, in order, of dS[h][slot] * k[slot][c0 + e] (the caller scales by
+// sm_scale at the end).
+MSA_BWD_HD void bwd_phase2(const BwdUnit& u, const float* dS, const uint32_t* kst, int rw, int cnt, int h, int c0,
+                           float* acc) {
+  for (int s = 0; s < cnt; ++s) {
+    const float ds = dS[h * kBwdChunk + s];
+    const uint32_t* kr = kst + s * rw + c0 / 2;
+MSA_BWD_HD_UNROLL
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t w = kr[j];
+      acc[2 * j] += ds * bwd_lo(w);
+      acc[2 * j + 1] += ds * bwd_hi(w);
+    }
+  }
 }
 
 }  // namespace msa

@@ -296,8 +296,11 @@ msa_status_t msa_gather_pages(const msa_varlen_t* seqs, const int32_t* block_tab
  * out and lse are the forward's outputs for the same support (prefill or
  * dense call).  The selection is not differentiated.  ws: at least 256
  * bytes, 256-byte aligned.  A selected block id past the query's block is
- * recorded as MSA_ERR_DEVICE_CHECK and left out.  A first, CUDA-core form
- * (one CTA per (query, group)). */
+ * recorded as MSA_ERR_DEVICE_CHECK and left out.  k, v, dk and dv must be
+ * 16-byte aligned (their rows are read and added 16 bytes at a time), else
+ * MSA_ERR_INVALID_ARG; d must be 64 or 128.  A CUDA-core form (one CTA per
+ * (query, group), key and value rows staged per 64-token chunk, dk / dv rows
+ * added with vector reductions). */
 msa_status_t msa_sparse_attn_backward(const msa_shape_t* shape, const msa_varlen_t* seqs,
                                       const void* q,      /* device bf16 [T, H, d] */
                                       const void* k,      /* device bf16 [S, G, d] */

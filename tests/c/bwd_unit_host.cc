@@ -43,8 +43,10 @@ int main(int argc, char** argv) {
       const int64_t t = cu_q[b] + i;
       for (int g = 0; g < G; ++g) {
         const int64_t row0 = (t * H + (int64_t)g * Hg) * d;
-        std::vector<float> qf(Hg * d), dof(Hg * d), ls(Hg), Ds(Hg, 0.f), dS(Hg * msa::kBwdChunk);
-        std::vector<uint16_t> kst(msa::kBwdChunk * d);
+        std::vector<float> qf(Hg * d), dof(Hg * d), ls(Hg), Ds(Hg, 0.f), dS(Hg * msa::kBwdChunk),
+            P(Hg * msa::kBwdChunk);
+        const int rw = d / 2 + 1;
+        std::vector<uint32_t> kst(msa::kBwdChunk * rw), vst(msa::kBwdChunk * rw);
         for (int x = 0; x < Hg * d; ++x) {
           qf[x] = msa::bwd_bf16(q[row0 + x]);
           dof[x] = msa::bwd_bf16(dout[row0 + x]);
@@ -70,10 +72,33 @@ int main(int argc, char** argv) {
         std::vector<float> acc(Hg * d, 0.f);
         for (int64_t c0 = 0; c0 < base[n]; c0 += msa::kBwdChunk) {
           const int cnt = base[n] - c0 < msa::kBwdChunk ? static_cast<int>(base[n] - c0) : msa::kBwdChunk;
+          int64_t tok[msa::kBwdChunk];
+          // stage the chunk's key and value rows (bf16 pairs as words, padded rows)
+          for (int s = 0; s < cnt; ++s) {
+            tok[s] = msa::bwd_token(first, base, n, c0 + s);
+            const uint16_t* kr = u.krow + (tok[s] * G + g) * d;
+            const uint16_t* vr = u.vrow + (tok[s] * G + g) * d;
+            for (int w = 0; w < d / 2; ++w) {
+              kst[s * rw + w] = (uint32_t)kr[2 * w] | ((uint32_t)kr[2 * w + 1] << 16);
+              vst[s * rw + w] = (uint32_t)vr[2 * w] | ((uint32_t)vr[2 * w + 1] << 16);
+            }
+          }
+          // the kernel's tiling: token pairs x head groups
+          for (int t0 = 0; t0 < cnt; t0 += msa::kBwdPdsTokens)
+            for (int h0 = 0; h0 < Hg; h0 += msa::kBwdPdsHeads)
+              msa::bwd_pds(u, kst.data(), vst.data(), rw, t0, cnt - t0 < 2 ? cnt - t0 : 2, h0,
+                           Hg - h0 < msa::kBwdPdsHeads ? Hg - h0 : msa::kBwdPdsHeads, P.data(), dS.data(),
+                           msa::kBwdChunk);
           for (int s = 0; s < cnt; ++s)
-            msa::bwd_phase1(u, msa::bwd_token(first, base, n, c0 + s), s, dS.data(), kst.data() + s * d, dk_seq,
-                            dv_seq);
-          for (int o = 0; o < Hg * d; ++o) acc[o] += msa::bwd_phase2(u, dS.data(), kst.data(), cnt, o);
+            for (int c = 0; c < d; ++c) {
+              float gk, gv;
+              msa::bwd_kv_cols(u, P.data(), dS.data(), msa::kBwdChunk, s, c, &gk, &gv);
+              dk_seq[(tok[s] * G + g) * d + c] += gk;
+              dv_seq[(tok[s] * G + g) * d + c] += gv;
+            }
+          for (int h = 0; h < Hg; ++h)
+            for (int c0_ = 0; c0_ < d; c0_ += 8)
+              msa::bwd_phase2(u, dS.data(), kst.data(), rw, cnt, h, c0_, acc.data() + h * d + c0_);
         }
         for (int o = 0; o < Hg * d; ++o) dq[row0 + o] = sm * acc[o];
       }
