@@ -598,6 +598,9 @@ static msa_status_t index_kl_common(const msa_shape_t* shape, const msa_varlen_t
   if (st != MSA_OK) return st;
   if (!(tau == tau) || tau > 3.0e38f || tau < -3.0e38f) return MSA_ERR_INVALID_ARG;   // NaN or infinite
   if (seqs->total_q > 0 && (!q || !k || !q_idx || !k_idx || !lse || (!dense && !sel))) return MSA_ERR_INVALID_ARG;
+  // key and index-key rows are read 16 bytes at a time
+  if (seqs->total_q > 0 && ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(k_idx)) & 15u))
+    return MSA_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, kWsHeader)) return MSA_ERR_WORKSPACE;
   if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MSA_ERR_CUDA;
@@ -629,6 +632,9 @@ msa_status_t msa_index_kl_backward(const msa_shape_t* shape, const msa_varlen_t*
                                    const float* lse, const float* lse_z, float tau, int32_t dense, float* dq_idx,
                                    float* dk_idx, void* ws, size_t ws_bytes, void* stream) {
   if (seqs != nullptr && seqs->total_q > 0 && (lse_z == nullptr || dq_idx == nullptr || dk_idx == nullptr))
+    return MSA_ERR_INVALID_ARG;
+  // the index-key gradient's rows are added 16 bytes at a time
+  if (seqs != nullptr && seqs->total_q > 0 && (reinterpret_cast<uintptr_t>(dk_idx) & 15u))
     return MSA_ERR_INVALID_ARG;
   IndexKlArgs a{};
   const msa_status_t st = index_kl_common(shape, seqs, q, k, q_idx, k_idx, sel, lse, tau, dense, ws, ws_bytes,

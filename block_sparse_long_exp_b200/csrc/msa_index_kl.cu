@@ -97,7 +97,9 @@ index_kl_grad_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict_
   __shared__ float qf[kKlMaxHg * kKlMaxD];
   __shared__ float qif[kKlMaxD];
   __shared__ float ls[kKlMaxHg];
-  __shared__ float dq[kKlMaxD];
+  // each thread's own dq row (stride d_idx + 1: rows start in different banks)
+  extern __shared__ float dq_rows[];
+  const int rs = d_idx + 1;
   const int64_t unit = blockIdx.x;
   const int64_t t = unit / G;
   const int g = static_cast<int>(unit - t * G);
@@ -115,11 +117,9 @@ index_kl_grad_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict_
     return;
   }
   for (int i = threadIdx.x; i < Hg * d; i += blockDim.x) qf[i] = kl_bf16(q[(t * H + (int64_t)g * Hg) * d + i]);
-  for (int i = threadIdx.x; i < d_idx; i += blockDim.x) {
-    qif[i] = kl_bf16(q_idx[(t * G + g) * d_idx + i]);
-    dq[i] = 0.f;
-  }
+  for (int i = threadIdx.x; i < d_idx; i += blockDim.x) qif[i] = kl_bf16(q_idx[(t * G + g) * d_idx + i]);
   for (int i = threadIdx.x; i < Hg; i += blockDim.x) ls[i] = lse[t * H + (int64_t)g * Hg + i];
+  for (int i = 0; i < d_idx; ++i) dq_rows[threadIdx.x * rs + i] = 0.f;
   __syncthreads();
   KlUnit u;
   u.qf = qf;
@@ -140,10 +140,16 @@ index_kl_grad_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict_
   u.tau = tau;
   u.dense = dense != 0;
   int bad = 0;
-  kl_grad_thread(u, lse_z[t * G + g], threadIdx.x, blockDim.x, dq, dk_idx + (int64_t)cu_k[lo] * d_idx, &bad);
+  kl_grad_thread(u, lse_z[t * G + g], threadIdx.x, blockDim.x, dq_rows + threadIdx.x * rs,
+                 dk_idx + (int64_t)cu_k[lo] * d_idx, &bad);
   if (bad) report_error(err, MSA_ERR_DEVICE_CHECK, kSiteIndexKl, static_cast<int>(t), g);
   __syncthreads();
-  for (int i = threadIdx.x; i < d_idx; i += blockDim.x) dq_idx[(t * G + g) * d_idx + i] = dq[i];
+  // dq: the threads' rows summed in thread order
+  for (int i = threadIdx.x; i < d_idx; i += blockDim.x) {
+    float acc = 0.f;
+    for (int r = 0; r < kKlThreads; ++r) acc += dq_rows[r * rs + i];
+    dq_idx[(t * G + g) * d_idx + i] = acc;
+  }
 }
 
 }  // namespace
@@ -168,8 +174,12 @@ int launch_index_kl_backward(const IndexKlArgs& a, void* stream) {
   if (a.H / a.G > kKlMaxHg || a.d > kKlMaxD || a.d_idx > kKlMaxD || units > 0x7fffffffLL)
     return (int)cudaErrorInvalidValue;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t smem = sizeof(float) * kKlThreads * (a.d_idx + 1);
+  const cudaError_t e =
+      cudaFuncSetAttribute(index_kl_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return (int)e;
   ProfScope p("index_kl_grad", stream);
-  index_kl_grad_kernel<<<(unsigned)units, kKlThreads, 0, st>>>(
+  index_kl_grad_kernel<<<(unsigned)units, kKlThreads, smem, st>>>(
       static_cast<const uint16_t*>(a.q), static_cast<const uint16_t*>(a.key), static_cast<const uint16_t*>(a.q_idx),
       static_cast<const uint16_t*>(a.k_idx), a.sel, a.lse, a.lse_z, a.cu_q, a.cu_k, a.batch, a.H, a.G, a.d, a.d_idx,
       a.k, a.sm_scale, a.tau, a.dense, a.dq_idx, a.dk_idx, a.err);

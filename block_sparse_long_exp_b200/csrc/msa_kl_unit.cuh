@@ -71,6 +71,18 @@ MSA_KL_HD float kl_log(float x) {
 #endif
 }
 
+// Eight consecutive bf16 values (16 bytes, 16-byte aligned) as floats.
+MSA_KL_HD void kl_load8(const uint16_t* p, float* out) {
+  uint16_t v[8];
+#ifdef __CUDA_ARCH__
+  *reinterpret_cast<uint4*>(v) = *reinterpret_cast<const uint4*>(p);
+#else
+  std::memcpy(v, p, 16);
+#endif
+MSA_KL_HD_UNROLL
+  for (int i = 0; i < 8; ++i) out[i] = kl_bf16(v[i]);
+}
+
 // Everything one (query, group) needs.  qf: the group's Hg query heads as
 // float [Hg * d]; qif: its index query as float [d_idx]; lse: the heads'
 // log-sum-exps over J [Hg]; krow / kirow: the sequence's keys (bf16 bits,
@@ -115,14 +127,18 @@ MSA_KL_HD void kl_for_tokens(const KlUnit& u, int tid, int nthreads, int* bad, F
     for (int64_t j = j0 + first; j < j1; j += nthreads) {
       const uint16_t* kj = u.krow + (j * u.G + u.g) * u.d;
       // every head's score, reading the key row once (kKlMaxHeads sums in registers)
+      // (rows are read 16 bytes at a time; each head's sum still runs over c in order)
       float s[kKlMaxHeads];
 MSA_KL_HD_UNROLL
       for (int h = 0; h < kKlMaxHeads; ++h) s[h] = 0.f;
-      for (int c = 0; c < u.d; ++c) {
-        const float kc = kl_bf16(kj[c]);
+      for (int c0 = 0; c0 < u.d; c0 += 8) {
+        float kc[8];
+        kl_load8(kj + c0, kc);
 MSA_KL_HD_UNROLL
-        for (int h = 0; h < kKlMaxHeads; ++h)
-          if (h < u.Hg) s[h] += u.qf[h * u.d + c] * kc;
+        for (int e = 0; e < 8; ++e)
+MSA_KL_HD_UNROLL
+          for (int h = 0; h < kKlMaxHeads; ++h)
+            if (h < u.Hg) s[h] += u.qf[h * u.d + c0 + e] * kc[e];
       }
       float pbar = 0.f;
 MSA_KL_HD_UNROLL
@@ -131,7 +147,12 @@ MSA_KL_HD_UNROLL
       pbar *= 1.f / u.Hg;
       const uint16_t* kij = u.kirow + j * u.d_idx;
       float zs = 0.f;
-      for (int c = 0; c < u.d_idx; ++c) zs += u.qif[c] * kl_bf16(kij[c]);
+      for (int c0 = 0; c0 < u.d_idx; c0 += 8) {
+        float ki[8];
+        kl_load8(kij + c0, ki);
+MSA_KL_HD_UNROLL
+        for (int e = 0; e < 8; ++e) zs += u.qif[c0 + e] * ki[e];
+      }
       f(j, pbar, zs, kij);
     }
   }
@@ -170,11 +191,14 @@ MSA_KL_HD float kl_merge(const KlPartial* p, int n, float* lse_z = nullptr) {
   return l > 0.f ? A - B + m + kl_log(l) : 0.f;
 }
 
-MSA_KL_HD void kl_add(float* dst, float v) {
+// Four consecutive floats added to dst (16-byte aligned): one vector reduction
+// on the device (other queries add to the same key rows), plain adds on the host.
+MSA_KL_HD void kl_add4(float* dst, float a, float b, float c, float d) {
 #ifdef __CUDA_ARCH__
-  atomicAdd(dst, v);
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
 #else
-  *dst += v;
+  dst[0] += a; dst[1] += b; dst[2] += c; dst[3] += d;
 #endif
 }
 
@@ -182,15 +206,20 @@ MSA_KL_HD void kl_add(float* dst, float v) {
 // support tokens: with w_j = tau (Q_j - P_j), Q_j = exp(z_j - lse_z),
 //   dq[c]              += w_j k_idx[j][c]   (the index query's gradient)
 //   dk[j * d_idx + c]  += w_j q_idx[c]      (the index keys' gradient)
-// Both are added atomically on the device (dq: the CTA's threads share one
-// accumulator; dk: other queries add to the same key rows).
-// dk points at the sequence's first key row of the fp32 [S, d_idx] gradient.
+// dq is this thread's own accumulator row (the caller sums the rows of all
+// threads); dk rows are added with kl_add4 (dk points at the sequence's first
+// key row of the fp32 [S, d_idx] gradient).
 MSA_KL_HD void kl_grad_thread(const KlUnit& u, float lse_z, int tid, int nthreads, float* dq, float* dk, int* bad) {
   kl_for_tokens(u, tid, nthreads, bad, [&](int64_t j, float pbar, float zs, const uint16_t* kij) {
     const float w = u.tau * (kl_exp(u.tau * zs - lse_z) - pbar);
-    for (int c = 0; c < u.d_idx; ++c) {
-      kl_add(dq + c, w * kl_bf16(kij[c]));
-      kl_add(dk + j * u.d_idx + c, w * u.qif[c]);
+    for (int c0 = 0; c0 < u.d_idx; c0 += 8) {
+      float ki[8];
+      kl_load8(kij + c0, ki);
+MSA_KL_HD_UNROLL
+      for (int e = 0; e < 8; ++e) dq[c0 + e] += w * ki[e];
+      float* dkr = dk + j * u.d_idx + c0;
+      kl_add4(dkr, w * u.qif[c0], w * u.qif[c0 + 1], w * u.qif[c0 + 2], w * u.qif[c0 + 3]);
+      kl_add4(dkr + 4, w * u.qif[c0 + 4], w * u.qif[c0 + 5], w * u.qif[c0 + 6], w * u.qif[c0 + 7]);
     }
   });
 }

@@ -361,8 +361,9 @@ msa_status_t msa_selected_share(const float* lse_sel, const float* lse_all, int6
  * The teacher P is a constant of this value (its gradient is not the index
  * branch's to follow).  ws: at least 256 bytes, 256-byte aligned (the error
  * word).  A selected block id past the query's block is recorded as
- * MSA_ERR_DEVICE_CHECK and skipped.  A first, CUDA-core form (one CTA per
- * (query, group)). */
+ * MSA_ERR_DEVICE_CHECK and skipped.  k and k_idx must be 16-byte aligned
+ * (their rows are read 16 bytes at a time), else MSA_ERR_INVALID_ARG.  A
+ * CUDA-core form (one CTA per (query, group)). */
 msa_status_t msa_index_kl(const msa_shape_t* shape, const msa_varlen_t* seqs,
                           const void* q,      /* device bf16 [T, H, d] */
                           const void* k,      /* device bf16 [S, G, d] */
@@ -380,7 +381,8 @@ msa_status_t msa_index_kl(const msa_shape_t* shape, const msa_varlen_t* seqs,
  *   dk_idx[j, :]    = sum over (t, g) of w_j q_idx[t, g, :]  (out, float [S, d_idx];
  *                     zeroed by the call, then accumulated atomically, so
  *                     its rounding order varies from run to run)
- * Arguments as msa_index_kl, plus lse_z from it. */
+ * Arguments as msa_index_kl, plus lse_z from it; dk_idx must be 16-byte
+ * aligned too (its rows are added 16 bytes at a time). */
 msa_status_t msa_index_kl_backward(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q,
                                    const void* k, const void* q_idx, const void* k_idx, const int32_t* sel,
                                    const float* lse, const float* lse_z, float tau, int32_t dense, float* dq_idx,

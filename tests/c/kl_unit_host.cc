@@ -67,7 +67,15 @@ int main(int argc, char** argv) {
           out[(size_t)s * T * G + t * G + g] = msa::kl_merge(parts.data(), sizes[s], &lse_z);
           float* dqu = dq.data() + ((size_t)s * T * G + t * G + g) * d_idx;
           float* dku = dk.data() + ((size_t)s * S + cu_k[b]) * d_idx;
-          for (int tid = 0; tid < sizes[s]; ++tid) msa::kl_grad_thread(u, lse_z, tid, sizes[s], dqu, dku, &bad);
+          // each thread's own dq row, then the rows summed in thread order (as the kernel does)
+          std::vector<float> rows((size_t)sizes[s] * d_idx, 0.f);
+          for (int tid = 0; tid < sizes[s]; ++tid)
+            msa::kl_grad_thread(u, lse_z, tid, sizes[s], rows.data() + (size_t)tid * d_idx, dku, &bad);
+          for (int c = 0; c < d_idx; ++c) {
+            float acc = 0.f;
+            for (int tid = 0; tid < sizes[s]; ++tid) acc += rows[(size_t)tid * d_idx + c];
+            dqu[c] = acc;
+          }
           bad_total += bad;
         }
       }
