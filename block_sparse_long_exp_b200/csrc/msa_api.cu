@@ -718,6 +718,8 @@ msa_status_t msa_index_topk_policy(const msa_shape_t* shape, const msa_varlen_t*
   if (n_sink < 0 || n_local < 1 || n_sink + n_local > shape->k) return MSA_ERR_INVALID_ARG;
   if ((int64_t)seqs->max_k_len > (int64_t)8192 * kBk) return MSA_ERR_UNSUPPORTED;   // block scores in shared memory
   if (seqs->total_q > 0 && (!q_idx || !k_idx || !sel)) return MSA_ERR_INVALID_ARG;
+  // index-key rows are read 16 bytes at a time
+  if (seqs->total_q > 0 && (reinterpret_cast<uintptr_t>(k_idx) & 15u)) return MSA_ERR_INVALID_ARG;
   if (!ws_ok(ws, ws_bytes, kWsHeader)) return MSA_ERR_WORKSPACE;
   if (cudaMemsetAsync(ws, 0, sizeof(DevError), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MSA_ERR_CUDA;

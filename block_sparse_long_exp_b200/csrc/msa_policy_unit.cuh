@@ -56,7 +56,16 @@ MSA_POL_HD float pol_block_score(const float* qif, const uint16_t* kirow, int d_
   for (int64_t j = b * B_k; j < j1; ++j) {
     const uint16_t* kj = kirow + j * d_idx;
     float s = 0.f;
-    for (int c = 0; c < d_idx; ++c) s += qif[c] * pol_bf16(kj[c]);
+    // the row is read 16 bytes at a time (d_idx is a multiple of 8); the sum runs over c in order
+    for (int c0 = 0; c0 < d_idx; c0 += 8) {
+      uint16_t v[8];
+#ifdef __CUDA_ARCH__
+      *reinterpret_cast<uint4*>(v) = *reinterpret_cast<const uint4*>(kj + c0);
+#else
+      std::memcpy(v, kj + c0, 16);
+#endif
+      for (int e = 0; e < 8; ++e) s += qif[c0 + e] * pol_bf16(v[e]);
+    }
     if (s > m) m = s;   // a NaN score never wins
   }
   return m;

@@ -331,8 +331,9 @@ msa_status_t msa_select_window(const msa_shape_t* shape, const msa_varlen_t* seq
  * (score desc, id asc; NaN as -inf); every causal block when there are at
  * most k.  n_sink = 0, n_local = 1 is msa_index_topk's rule.  Requires
  * n_sink >= 0, n_local >= 1, n_sink + n_local <= k, max_k_len <= 1M tokens.
- * sel as msa_index_topk; ws: at least 256 bytes, 256-byte aligned.  A first,
- * CUDA-core form (one CTA per (query, group)). */
+ * sel as msa_index_topk; ws: at least 256 bytes, 256-byte aligned; k_idx
+ * 16-byte aligned (its rows are read 16 bytes at a time), else
+ * MSA_ERR_INVALID_ARG.  A CUDA-core form (one CTA per (query, group)). */
 msa_status_t msa_index_topk_policy(const msa_shape_t* shape, const msa_varlen_t* seqs, int32_t n_sink,
                                    int32_t n_local, const void* q_idx, const void* k_idx, int32_t* sel, void* ws,
                                    size_t ws_bytes, void* stream);
