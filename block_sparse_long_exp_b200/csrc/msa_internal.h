@@ -46,8 +46,8 @@ enum ErrorSite : int32_t {
   kSiteTileMma = 153,
   kSiteTileSoftmax = 154,
   kSitePaged = 161,
-  kSiteSelfTest = 171,
-  kSiteKeySplit = 181,
+  kSiteSelfTest = 221,
+  kSiteKeySplit = 231,
 };
 
 // One KV-outer work item: up to `count` queries of the list of

@@ -503,7 +503,7 @@ msa_status_t msa_select_block_range(const msa_shape_t* shape, int32_t batch, con
  * waits can never end (an mbarrier nobody arrives on, a workspace counter
  * nobody advances), each with the library's own wait given `limit_us`
  * microseconds (1 ... 1,000,000); both give up, the kernel returns, and
- * msa_get_device_error(ws) then reads MSA_ERR_TIMEOUT (site 171).  The word
+ * msa_get_device_error(ws) then reads MSA_ERR_TIMEOUT (site 221).  The word
  * at ws + 256 + 4 (int32) counts the waits that ran out (2).
  * ws: device, 256-byte aligned, msa_selftest_wait_timeout_workspace_size()
  * bytes; cleared by the call.  Returns MSA_ERR_INVALID_ARG for a limit out of
@@ -580,6 +580,7 @@ msa_status_t msa_profile_read(const char* kernel, double* total_ms, int64_t* cou
  *   171      index-alignment target / its gradient   181  window selection
  *   191      main-branch backward                      201  policy selection
  *   211      page gather (info0 = sequence, info1 = block)
+ *   221      bounded-wait self-test              231  decode candidate merge
  * MSA_ERR_TIMEOUT codes come from a bounded wait that ran out (about a
  * second); the call's results are then not valid, the context still is. */
 msa_status_t msa_get_device_error(void* ws, int32_t* code, int32_t* where, int32_t* info0,

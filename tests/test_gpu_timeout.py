@@ -14,7 +14,7 @@ from block_sparse_long_exp_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 MSA_ERR_TIMEOUT = 5
-SITE_SELFTEST = 171
+SITE_SELFTEST = 221
 
 
 @pytest.fixture(scope="module")
