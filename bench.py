@@ -209,8 +209,10 @@ def training_leg(args, w, W, R, msa, torch, device="cuda"):
     gradient, fed by the forward's selection and log-sum-exps.  Each kernel is
     timed by the library's CUDA events on its launching stream over
     args.training_steps passes after args.training_warmup (inputs larger than
-    L2; its own small counts, since one pass takes about 2 s).  They run on the
-    CUDA cores, so the roofline is the fp32 FMA rate."""
+    L2; its own small counts, since one pass takes about 2 s).  The backward
+    and the KL gradient run on the CUDA cores and are held to the fp32 FMA
+    rate; the KL target computes its scores on the tensor cores and is held to
+    the exponential rate of the special-function units."""
     tinp = W.make_inputs(w, device, T_override=args.training_T)
     shape = msa.make_shape(w.H, w.G, w.d, w.d_idx, w.k)
     seqs = msa.make_varlen(tinp["cu_q"], tinp["cu_k"], tinp["cu_q_host"], tinp["cu_k_host"])
@@ -252,6 +254,22 @@ def training_leg(args, w, W, R, msa, torch, device="cuda"):
             ach = tw[key] / (per / 1000.0) / 1e12
             res["kernels"][name] = {"ms_per_launch": per, "launches": n, "flops_per_launch": tw[key],
                                     "bound": "alu", "achieved": ach, "frac": ach / peak}
+    kr = res["kernels"].get("index_kl")
+    if kr is not None:
+        # the KL target's scores run on the tensor cores; what stays on the
+        # CUDA cores is dominated by one exponential per head and pair, so the
+        # kernel is held to the exponential rate, the tensor-core figure beside it
+        sec = kr["ms_per_launch"] / 1000.0
+        peaks, src = load_peaks()
+        mufu = R.mufu_gexps()
+        ach_e = tw["kl_exps"] / sec / 1e9
+        ach_t = tw["kl_tensor_flops"] / sec / 1e12
+        kr.update({"bound": "mufu", "unit": "Gexp/s", "exps_per_launch": tw["kl_exps"], "achieved": ach_e,
+                   "peak": mufu, "frac": ach_e / mufu,
+                   "peak_source": "148 SMs x 16 ex2 per clock x 1965 MHz (special-function units)",
+                   "tensor": {"flops_per_launch": tw["kl_tensor_flops"], "achieved": ach_t,
+                              "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                              "frac": ach_t / peaks["bf16_tflops"], "peak_source": f"bf16_tflops ({src})"}})
     return res
 
 

@@ -614,6 +614,48 @@ static msa_status_t index_kl_common(const msa_shape_t* shape, const msa_varlen_t
   return MSA_OK;
 }
 
+// Workspace of the tensor-core KL target (sparse support): the KV-outer plan
+// of one pass over every query and one float4 partial per (query, group, slot).
+struct KlLayout {
+  size_t blk_off, counts, cursor, tile_sums, nitems, entries, items, part, total;
+  int64_t nlists, max_items;
+  int32_t qpi, win;
+};
+
+KlLayout kl_layout(const msa_shape_t* s, const msa_varlen_t* v) {
+  KlLayout L{};
+  const int hg = s->H / s->G;
+  const int qpt = 128 / (hg < 8 ? 8 : hg);
+  L.qpi = 8 * qpt < kMaxItemQueries ? 8 * qpt : kMaxItemQueries;
+  L.nlists = (int64_t)s->G * total_blocks_bound(v, s->B_k);
+  L.win = attn_window_rows();
+  const int64_t rows = v->total_q;
+  const int64_t nkeys = ((rows + L.win - 1) / L.win) * L.nlists;
+  const int64_t nentries = rows * s->G * s->k;
+  L.max_items = nentries / L.qpi + (nkeys < nentries ? nkeys : nentries) + 1;
+  size_t off = kWsHeader;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, kAlign);
+    return o;
+  };
+  L.blk_off = take(sizeof(int32_t) * (v->batch + 1));
+  L.counts = take(sizeof(int32_t) * nkeys);
+  L.cursor = take(sizeof(int32_t) * nkeys);
+  L.tile_sums = take(sizeof(int32_t) * 2 * ((nkeys + kScanTile - 1) / kScanTile + 1));
+  L.nitems = take(sizeof(int32_t) * 4);
+  L.entries = take(sizeof(uint32_t) * nentries);
+  L.items = take(sizeof(Item) * L.max_items);
+  L.part = take(sizeof(float4) * nentries);
+  L.total = off;
+  return L;
+}
+
+size_t msa_index_kl_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs, int32_t dense) {
+  if (check_shape_bk128(shape) != MSA_OK || check_seqs(seqs) != MSA_OK) return 0;
+  return dense ? kWsHeader : kl_layout(shape, seqs).total;
+}
+
 msa_status_t msa_index_kl(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q, const void* k,
                           const void* q_idx, const void* k_idx, const int32_t* sel, const float* lse, float tau,
                           int32_t dense, float* kl, float* lse_z, void* ws, size_t ws_bytes, void* stream) {
@@ -624,7 +666,33 @@ msa_status_t msa_index_kl(const msa_shape_t* shape, const msa_varlen_t* seqs, co
   if (st != MSA_OK || seqs->total_q == 0) return st;
   a.kl = kl;
   a.lse_z = lse_z;
-  return launch_index_kl(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
+  if (dense) return launch_index_kl(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
+  // selected support: the tensor-core form over the forward's KV-outer lists
+  const KlLayout L = kl_layout(shape, seqs);
+  if (!ws_ok(ws, ws_bytes, L.total)) return MSA_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  AttnArgs p{};
+  p.q = q; p.key = k; p.sel = sel;
+  p.cu_q = seqs->cu_q; p.cu_k = seqs->cu_k;
+  p.batch = seqs->batch; p.H = shape->H; p.G = shape->G; p.d = shape->d; p.k = shape->k; p.B_k = shape->B_k;
+  p.sm_scale = shape->sm_scale;
+  p.total_q = seqs->total_q; p.total_k = seqs->total_k;
+  p.max_q_len = seqs->max_q_len; p.max_k_len = seqs->max_k_len;
+  p.t0 = 0; p.t1 = seqs->total_q;
+  p.err = a.err;
+  p.blk_off = reinterpret_cast<int32_t*>(base + L.blk_off);
+  p.counts = reinterpret_cast<int32_t*>(base + L.counts);
+  p.cursor = reinterpret_cast<int32_t*>(base + L.cursor);
+  p.tile_sums = reinterpret_cast<int32_t*>(base + L.tile_sums);
+  p.nitems = reinterpret_cast<int32_t*>(base + L.nitems);
+  p.entries = reinterpret_cast<uint32_t*>(base + L.entries);
+  p.items = reinterpret_cast<Item*>(base + L.items);
+  p.max_items = L.max_items;
+  p.nlists = L.nlists;
+  p.win_rows = L.win;
+  p.queries_per_item = L.qpi;
+  p.theta = 0;
+  return launch_index_kl_tc(a, p, reinterpret_cast<float4*>(base + L.part), stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
 }
 
 msa_status_t msa_index_kl_backward(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q,

@@ -958,7 +958,7 @@ int launch_combine_kernel(const __half* part_acc, const float* part_lse, const i
 
 // -------------------------------------------------------------- launchers ---
 
-int launch_sparse_attn_main(const AttnArgs& a, void* stream) {
+int launch_kv_plan(const AttnArgs& a, void* stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t nrows = a.t1 - a.t0;
   if (nrows <= 0) return 0;
@@ -1005,8 +1005,16 @@ int launch_sparse_attn_main(const AttnArgs& a, void* stream) {
                                                           nullptr,
                                                           a.err);
   }
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return (int)e;
+  return (int)cudaGetLastError();
+}
+
+int launch_sparse_attn_main(const AttnArgs& a, void* stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (a.t1 - a.t0 <= 0) return 0;
+  int rc0 = launch_kv_plan(a, stream);
+  if (rc0) return rc0;
+  const bool tiles = a.theta > 0;
+  cudaError_t e;
 
   alignas(64) CUtensorMap tm_k, tm_v, tm_q;
   {

@@ -152,6 +152,10 @@ int launch_sparse_attn_pass(const AttnArgs& a, void* stream);   // main phase, t
 // KV-outer and query-tile attention) writes the pass's partials; the combine
 // merges them into out / lse (on at most grid_cap CTAs; <= 0: one per SM).
 int launch_sparse_attn_main(const AttnArgs& a, void* stream);
+// The planning of a pass alone (block offsets, the query-tile plan when theta
+// > 0, the KV-outer lists and their work items); launch_sparse_attn_main runs
+// it first.
+int launch_kv_plan(const AttnArgs& a, void* stream);
 int launch_sparse_attn_combine(const AttnArgs& a, void* stream, int grid_cap);
 int attn_window_rows();                // planning window of the prefill calls (msa_set_attn_window)
 int launch_combine(const void* part_acc, const float* part_lse, const int32_t* sel, void* out,

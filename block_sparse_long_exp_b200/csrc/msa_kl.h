@@ -30,6 +30,10 @@ struct IndexKlArgs {
 };
 
 int launch_index_kl(const IndexKlArgs& a, void* stream);
+// Sparse support on the tensor cores (msa_index_kl_tc.cu): `plan` describes
+// the KV-outer lists of the whole call (one pass, no query tiles); part holds
+// [T, G, k] partials and is zeroed by the call.
+int launch_index_kl_tc(const IndexKlArgs& a, const AttnArgs& plan, float4* part, void* stream);
 int launch_index_kl_backward(const IndexKlArgs& a, void* stream);
 
 }  // namespace msa

@@ -55,7 +55,7 @@ EXPORTED = [
     "msa_decode_paged_workspace_size", "msa_index_topk_decode_paged", "msa_sparse_attn_decode_paged",
     "msa_index_kl", "msa_index_kl_backward", "msa_select_window", "msa_sparse_attn_backward",
     "msa_selected_share", "msa_index_topk_policy", "msa_gather_pages",
-    "msa_prefill_workspace_size", "msa_prefill", "msa_set_prefill_overlap",
+    "msa_prefill_workspace_size", "msa_prefill", "msa_set_prefill_overlap", "msa_index_kl_workspace_size",
 ]
 
 
@@ -155,6 +155,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_index_kl.argtypes = [P(Shape), P(Varlen), vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp, vp, vp, sz,
                                  vp]
     lib.msa_index_kl.restype = i32
+    lib.msa_index_kl_workspace_size.argtypes = [P(Shape), P(Varlen), i32]
+    lib.msa_index_kl_workspace_size.restype = sz
     lib.msa_index_kl_backward.argtypes = [P(Shape), P(Varlen), vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp,
                                           vp, vp, sz, vp]
     lib.msa_index_kl_backward.restype = i32
@@ -651,6 +653,11 @@ def _index_kl_args(shape, seqs, q, k, q_idx, k_idx, sel, lse, dense):
     _arg("lse", lse, torch.float32, (T, shape.H))
 
 
+def msa_index_kl_workspace_size(shape: Shape, seqs: Varlen, dense: bool = False) -> int:
+    """Workspace bytes of msa_index_kl (0: unsupported)."""
+    return load_library().msa_index_kl_workspace_size(ctypes.byref(shape), ctypes.byref(seqs), 1 if dense else 0)
+
+
 def msa_index_kl(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.Tensor, q_idx: torch.Tensor,
                  k_idx: torch.Tensor, sel: Optional[torch.Tensor], lse: torch.Tensor, tau: float,
                  dense: bool = False, kl: Optional[torch.Tensor] = None, want_lse_z: bool = False,
@@ -672,7 +679,10 @@ def msa_index_kl(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.Tensor, q
         kl = torch.empty((T, shape.G), dtype=torch.float32, device=q.device)
     lse_z = torch.empty((T, shape.G), dtype=torch.float32, device=q.device) if want_lse_z else None
     if ws is None:
-        ws = _workspace(256, q.device)
+        need = msa_index_kl_workspace_size(shape, seqs, dense)
+        if need == 0:
+            raise MsaError("msa_index_kl: unsupported or invalid shape")
+        ws = _workspace(need, q.device)
     rc = lib.msa_index_kl(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q), _ptr(k), _ptr(q_idx), _ptr(k_idx),
                           _ptr(sel), _ptr(lse), float(tau), 1 if dense else 0, _ptr(kl), _ptr(lse_z), _ptr(ws),
                           _nbytes(ws), _stream(stream))

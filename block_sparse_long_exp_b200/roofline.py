@@ -83,6 +83,8 @@ def training_work(S_lens: Sequence[int], T_lens: Sequence[int], H: int, G: int, 
     pairs = main / (4 * H * d)            # attended (query, key) pairs of one head
     return {"pairs": pairs, "backward_flops": 10.0 * H * d * pairs,
             "kl_flops": pairs * (2.0 * H * d + 2.0 * G * d_idx),
+            "kl_tensor_flops": pairs * 2.0 * H * d,     # the teacher scores q . k (on the tensor cores)
+            "kl_exps": pairs * H,                        # one exponential per head and attended pair
             "kl_grad_flops": pairs * (2.0 * H * d + 6.0 * G * d_idx)}
 
 
@@ -90,6 +92,13 @@ def alu_fp32_tflops(sms: int = 148, lanes: int = 128, mhz: float = 1965.0) -> fl
     """Peak fp32 FMA rate of the CUDA cores (two FLOPs per lane per clock):
     B200 has 148 SMs of 128 fp32 lanes, clocks.max.sm 1965 MHz: 74.4 TFLOP/s."""
     return sms * lanes * 2.0 * mhz * 1e6 / 1e12
+
+
+def mufu_gexps(sms: int = 148, per_clk: int = 16, mhz: float = 1965.0) -> float:
+    """Peak exponential rate of the special-function units: 16 ex2 per clock
+    per SM (the rate measured on B200 for every ex2 form), 148 SMs at
+    clocks.max.sm 1965 MHz: 4653 G exponentials/s."""
+    return sms * per_clk * mhz * 1e6 / 1e9
 
 
 def dense_work(S_lens: Sequence[int], T_lens: Sequence[int], H: int, d: int) -> float:

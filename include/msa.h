@@ -360,11 +360,19 @@ msa_status_t msa_selected_share(const float* lse_sel, const float* lse_all, int6
  *   lse_z  device float [T, G] (out, or NULL): the student's log-sum-exp
  *          log sum_j exp(z_j), which the backward call takes
  * The teacher P is a constant of this value (its gradient is not the index
- * branch's to follow).  ws: at least 256 bytes, 256-byte aligned (the error
- * word).  A selected block id past the query's block is recorded as
- * MSA_ERR_DEVICE_CHECK and skipped.  k and k_idx must be 16-byte aligned
- * (their rows are read 16 bytes at a time), else MSA_ERR_INVALID_ARG.  A
- * CUDA-core form (one CTA per (query, group)). */
+ * branch's to follow).  ws: msa_index_kl_workspace_size bytes, 256-byte
+ * aligned (the error word first).  A selected block id past the query's
+ * block is recorded as MSA_ERR_DEVICE_CHECK and skipped.  k and k_idx must be 16-byte aligned
+ * (their rows are read 16 bytes at a time), else MSA_ERR_INVALID_ARG.
+ * The selected support (dense = 0) runs on the tensor cores: the selection is
+ * inverted into the forward's KV-outer lists, each selected block's keys are
+ * loaded once per work item, S = Q K^T of its gathered queries is a tcgen05
+ * product, and the sums are merged per (query, group); ws must then hold
+ * msa_index_kl_workspace_size bytes (the lists and one 16-byte partial per
+ * (query, group, slot)).  The dense support (the warm-up) runs on the CUDA
+ * cores (one CTA per (query, group)) with the 256-byte workspace. */
+size_t msa_index_kl_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs, int32_t dense);
+
 msa_status_t msa_index_kl(const msa_shape_t* shape, const msa_varlen_t* seqs,
                           const void* q,      /* device bf16 [T, H, d] */
                           const void* k,      /* device bf16 [S, G, d] */
