@@ -668,6 +668,8 @@ msa_status_t msa_index_kl(const msa_shape_t* shape, const msa_varlen_t* seqs, co
   a.lse_z = lse_z;
   if (dense) return launch_index_kl(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
   // selected support: the tensor-core form over the forward's KV-outer lists
+  // (its index-query rows are read 16 bytes at a time)
+  if (reinterpret_cast<uintptr_t>(q_idx) & 15u) return MSA_ERR_INVALID_ARG;
   const KlLayout L = kl_layout(shape, seqs);
   if (!ws_ok(ws, ws_bytes, L.total)) return MSA_ERR_WORKSPACE;
   uint8_t* base = static_cast<uint8_t*>(ws);

@@ -10,17 +10,21 @@
 // loads its key block and index-key rows once and gathers its queries' rows.
 // kl_items_kernel (persistent, one CTA per SM, 384 threads):
 //   warp 0      claims items (atomic ticket), publishes them in a ring and
-//               loads each item's key block (TMA), its index-key rows (a bulk
-//               copy that stops at the end of the keys) and, per 128-row
-//               tile, the gathered query rows (one TMA box per query);
-//   warp 1      owns TMEM (two S slots of 128 columns); lane 0 issues
-//               S = Q K^T per tile (tile t in slot t % 2);
-//   warps 4-11  two warpgroups, one per S slot: per row (query, head) P_h =
+//               loads each item's key block and index-key block (TMA) and,
+//               per 128-row tile, the gathered query rows (one TMA box per
+//               query);
+//   warps 2, 3  per tile (alternating), the index-query operand: every row
+//               (query, head) of the tile holds its query's index vector, so
+//               Z = that operand times the index keys gives each row its
+//               query's raw index scores;
+//   warp 1      owns TMEM (two slots of 256 columns); lane 0 issues
+//               S = Q K^T and Z = Q_idx K_idx^T per tile (tile t in slot t % 2);
+//   warps 4-11  two warpgroups, one per slot: per row (query, head) P_h =
 //               exp(sm_scale s - lse_h) for the block's keys in the support;
-//               the mean over the query's head rows by warp shuffles; each
-//               lane of a query then takes every RQ-th key: z = tau
-//               q_idx.k_idx (CUDA cores, the index rows from shared memory)
-//               and the KL's partial sums A = sum P log P, B = sum P z and a
+//               the head sum by a reduce-scatter over the query's RQ lanes
+//               (each lane ends with the sums of 32 / RQ keys of every
+//               32-key chunk and picks the same keys' z from its Z row), then
+//               the KL's partial sums A = sum P log P, B = sum P z and a
 //               (max, sum) pair of z; the lanes' partials are merged and
 //               written as one float4 per (query, group, selected slot).
 // kl_merge_kernel: per (query, group) the float4s of its slots give KL =
@@ -36,9 +40,9 @@ namespace {
 
 constexpr int kKtThreads = 384;
 constexpr int kKtItemRing = 4;
-constexpr int kKtItemEmptyCount = 9;   // MMA issuer 1 + KL warps 8
-constexpr int kKtKvEmptyCount = 9;     // the MMAs' commit + KL warps 8 (they read the index rows)
-constexpr int kKtMaxQpw = 4;           // queries per warp (32 / RQ, RQ >= 8)
+constexpr int kKtItemEmptyCount = 11;  // MMA issuer 1 + index-query warps 2 + KL warps 8
+constexpr uint32_t kKtTmemCols = 512;  // per slot: S in columns [0, 128), Z in [128, 256)
+constexpr size_t kKtSmemLimit = 232448;
 
 struct __align__(16) KtItem {
   int32_t seq, blk, g, start, count, Tb, Sb, qrow0;
@@ -47,7 +51,7 @@ struct __align__(16) KtItem {
 struct __align__(16) KtCtl {
   uint64_t item_full[kKtItemRing], item_empty[kKtItemRing];
   uint64_t kv_full[2], kv_empty[2];
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full[2], qi_full[2], q_empty[2];
   uint64_t s_full[2], s_free[2];
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -55,30 +59,53 @@ struct __align__(16) KtCtl {
   KtItem ring[kKtItemRing];
 };
 
+// Sum of p over the RQ lanes of a query (RQ aligned lanes), scattered: a step
+// at lane offset `off` halves the values a lane keeps (the upper half where
+// its lane bit `off` is set) and adds the partner's copy of them.  After
+// log2(RQ) steps lane hi holds the sums of keys [hi * W, hi * W + W), W = 32 /
+// RQ, in p[0, W).  z is the same for every lane of the query; it follows the
+// same selection, so z[i] is the value of the key of p[i].
+template <int RQ>
+__device__ __forceinline__ void head_reduce_scatter(float (&p)[32], float (&z)[32], int hi) {
+#pragma unroll
+  for (int off = RQ / 2, half = 16; off >= 1; off >>= 1, half >>= 1) {
+    const bool up = (hi & off) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = up ? p[i] : p[i + half];
+      const float keep = up ? p[i + half] : p[i];
+      p[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+      z[i] = up ? z[i + half] : z[i];
+    }
+  }
+}
+
+template <int RQ>
 __global__ void __launch_bounds__(kKtThreads, 1)
 kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
-                const uint16_t* __restrict__ k_idx, const uint16_t* __restrict__ q_idx,
+                const __grid_constant__ CUtensorMap tm_ki, const uint16_t* __restrict__ q_idx,
                 const float* __restrict__ lse, const Item* __restrict__ items, const int32_t* __restrict__ nitems_p,
                 int32_t* __restrict__ ticket, const uint32_t* __restrict__ entries, const int32_t* __restrict__ cu_q,
-                const int32_t* __restrict__ cu_k, int H, int G, int d, int d_idx, int k, float scale_log2,
-                float temp, int64_t total_k, float4* __restrict__ part, DevError* err) {
+                const int32_t* __restrict__ cu_k, int H, int G, int d, int d_idx, int k, int nst, float scale_log2,
+                float temp, float4* __restrict__ part, DevError* err) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   const int tile_bytes = 128 * d * 2;          // one [128 x d] bf16 tile
-  const int kidx_bytes = 128 * d_idx * 2;      // one block of index-key rows
-  uint8_t* k_s = smem;                          // 2 stages of K
-  uint8_t* q_s = k_s + 2 * tile_bytes;          // 2 slots of gathered Q rows
-  uint16_t* ki_s = reinterpret_cast<uint16_t*>(q_s + 2 * tile_bytes);            // 2 stages of index rows
-  float* qi_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ki_s) + 2 * kidx_bytes);   // per KL warp
-  float* pb_s = qi_s + 8 * kKtMaxQpw * d_idx;   // per KL warp and query: a chunk's 32 head-summed P
-  KtCtl* ctl = reinterpret_cast<KtCtl*>(pb_s + 8 * kKtMaxQpw * 32);
+  const int itile_bytes = 128 * d_idx * 2;     // one [128 x d_idx] bf16 tile
+  const int span = d_idx * 2 >= 128 ? 128 : d_idx * 2;   // bytes per swizzled row of an index tile
+  const int span_el = span / 2;
+  const int nibox = (d_idx * 2) / span;        // boxes per index tile
+  uint8_t* k_s = smem;                          // nst stages of K
+  uint8_t* ki_s = k_s + nst * tile_bytes;       // nst stages of K_idx
+  uint8_t* q_s = ki_s + nst * itile_bytes;      // 2 slots of gathered Q rows
+  uint8_t* qi_s = q_s + 2 * tile_bytes;         // 2 slots of the index-query operand
+  KtCtl* ctl = reinterpret_cast<KtCtl*>(qi_s + 2 * itile_bytes);
   volatile int32_t* abort_flag = &ctl->abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Hg = H / G;
-  const int RQ = Hg < 8 ? 8 : Hg;               // tile rows per query
-  const int qpt = 128 / RQ;                     // queries per 128-row tile
+  constexpr int qpt = 128 / RQ;                 // queries per 128-row tile
   const int nhalf = d / 64;
   const int nitems = *nitems_p;
   constexpr float kLog2e = 1.4426950408889634f;
@@ -90,8 +117,9 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl->kv_full[i], 1);
-      mbar_init(&ctl->kv_empty[i], kKtKvEmptyCount);
+      mbar_init(&ctl->kv_empty[i], 1);
       mbar_init(&ctl->q_full[i], 1);
+      mbar_init(&ctl->qi_full[i], 1);
       mbar_init(&ctl->q_empty[i], 1);
       mbar_init(&ctl->s_full[i], 1);
       mbar_init(&ctl->s_free[i], 4);
@@ -101,9 +129,10 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     fence_mbar_init();
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_ki);
   }
   if (warp == 1) {
-    tmem_alloc(&ctl->tmem_base, 256);
+    tmem_alloc(&ctl->tmem_base, kKtTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -150,20 +179,16 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         R->Sb = cu_k[I.seq + 1] - cu_k[I.seq];
         R->qrow0 = cu_q[I.seq];
         mbar_arrive(&ctl->item_full[slot]);
-        // the block's keys (TMA fills rows past the keys with zeros) and its
-        // index rows (a plain bulk copy: it stops at the last key row)
-        const int st = n & 1;
-        ok = mbar_wait(&ctl->kv_empty[st], ((n >> 1) + 1) & 1);
+        // the block's keys and index keys (TMA fills rows past the keys with zeros)
+        const int st = n % nst;
+        ok = mbar_wait(&ctl->kv_empty[st], ((n / nst) + 1) & 1);
         if (ok) {
-          const int64_t krow = (int64_t)cu_k[I.seq] + (int64_t)I.blk * kBk;
-          const int64_t rows = total_k - krow < kBk ? total_k - krow : kBk;
-          const uint32_t ibytes = (uint32_t)(rows > 0 ? rows : 0) * (uint32_t)d_idx * 2u;
-          mbar_arrive_expect_tx(&ctl->kv_full[st], (uint32_t)tile_bytes + ibytes);
+          const int krow = cu_k[I.seq] + I.blk * kBk;
+          mbar_arrive_expect_tx(&ctl->kv_full[st], (uint32_t)(tile_bytes + itile_bytes));
           for (int h = 0; h < nhalf; ++h)
-            tma_load_3d(k_s + st * tile_bytes + h * 128 * 128, &tm_k, &ctl->kv_full[st], 64 * h, I.g, (int)krow);
-          if (ibytes > 0)
-            bulk_load(reinterpret_cast<uint8_t*>(ki_s) + st * kidx_bytes, k_idx + krow * d_idx, ibytes,
-                      &ctl->kv_full[st]);
+            tma_load_3d(k_s + st * tile_bytes + h * 128 * 128, &tm_k, &ctl->kv_full[st], 64 * h, I.g, krow);
+          for (int bx = 0; bx < nibox; ++bx)
+            tma_load_2d(ki_s + st * itile_bytes + bx * 128 * span, &tm_ki, &ctl->kv_full[st], bx * span_el, krow);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -196,8 +221,8 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         *abort_flag = 1;
       }
       // no load may still be in flight when the CTA exits
-      for (int st = 0; st < 2; ++st) {
-        const int issued = n > st ? (n - st + 1) / 2 : 0;
+      for (int st = 0; st < nst; ++st) {
+        const int issued = n > st ? (n - st + nst - 1) / nst : 0;
         if (issued > 0) mbar_wait(&ctl->kv_full[st], (issued - 1) & 1);
       }
       for (int qs = 0; qs < 2; ++qs) {
@@ -205,26 +230,87 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (issued > 0) mbar_wait(&ctl->q_full[qs], (issued - 1) & 1);
       }
     }
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------- index-query operand of every other tile
+    // row r of the tile holds q_idx[t, g] of its query r / RQ, in the
+    // swizzled K-major layout the index keys' TMA writes
+    const int my = warp - 2;
+    const int cpr = d_idx / 8;                 // 16-byte chunks per row
+    const int cpb = span / 16;                 // chunks per box row
+    const int nload = (qpt * cpr) / 32;        // chunks per lane (1 to 8)
+    int n = 0, tau = 0;
+    bool ok = true;
+    while (ok && !*abort_flag) {
+      const KtItem* R = wait_item(n);
+      if (R == nullptr) break;
+      const int count = R->count, start = R->start, g = R->g;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->item_empty[n % kKtItemRing]);
+      if (count <= 0) break;
+      const int ntiles = (count + qpt - 1) / qpt;
+      for (int mt = 0; mt < ntiles; ++mt, ++tau) {
+        const int qs = tau & 1;
+        if (qs != my) continue;
+        if (lane == 0) ok = mbar_wait(&ctl->q_empty[qs], ((tau >> 1) + 1) & 1);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        const int nq = min(qpt, count - mt * qpt);
+        const uint32_t e = lane < nq ? entries[start + mt * qpt + lane] : 0u;
+        uint4 v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int u = lane + 32 * i, ql = u / cpr, c = u - ql * cpr;
+          const uint32_t eq = __shfl_sync(0xffffffffu, e, ql & 31);
+          v[i] = make_uint4(0u, 0u, 0u, 0u);
+          if (i < nload && ql < nq)
+            v[i] = *reinterpret_cast<const uint4*>(q_idx + ((int64_t)(eq / k) * G + g) * d_idx + c * 8);
+        }
+        uint8_t* dst = qi_s + qs * itile_bytes;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (i < nload) {
+            const int u = lane + 32 * i, ql = u / cpr, c = u - ql * cpr;
+            const int bx = c / cpb, cc = c - bx * cpb;
+#pragma unroll
+            for (int h = 0; h < RQ; ++h)
+              *reinterpret_cast<uint4*>(dst + bx * 128 * span + swz_offset(ql * RQ + h, cc, span)) = v[i];
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->qi_full[qs]);
+      }
+      if (!ok) break;
+      ++n;
+    }
+    if (!ok && lane == 0) {
+      report_error(err, MSA_ERR_TIMEOUT, kSiteIndexKl, tau, -3);
+      *abort_flag = 1;
+    }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
       const uint64_t qdesc0 = make_sdesc(smem_u32(q_s), 16, 1024, kSw128);
       const uint64_t kdesc0 = make_sdesc(smem_u32(k_s), 16, 1024, kSw128);
+      const uint32_t imode = sw_mode_for(span);
+      const uint64_t qidesc0 = make_sdesc(smem_u32(qi_s), 16, 8 * span, imode);
+      const uint64_t kidesc0 = make_sdesc(smem_u32(ki_s), 16, 8 * span, imode);
+      const int per_sh = span == 128 ? 2 : (span == 64 ? 1 : 0);   // log2(K steps per swizzled row)
       int n = 0, tau = 0;
       bool ok = true;
       while (ok && !*abort_flag) {
         const KtItem* R = wait_item(n);
         if (R == nullptr) { ok = false; break; }
         const int cnt = R->count;
-        if (lane == 0) mbar_arrive(&ctl->item_empty[n % kKtItemRing]);
+        mbar_arrive(&ctl->item_empty[n % kKtItemRing]);
         if (cnt <= 0) break;
-        const int st = n & 1;
+        const int st = n % nst;
         const int ntiles = (cnt + qpt - 1) / qpt;
         for (int mt = 0; mt < ntiles && ok; ++mt, ++tau) {
           const int s = tau & 1;
-          if (!mbar_wait(&ctl->q_full[s], (tau >> 1) & 1) ||
-              (mt == 0 && !mbar_wait(&ctl->kv_full[st], (n >> 1) & 1)) ||
+          if (!mbar_wait(&ctl->q_full[s], (tau >> 1) & 1) || !mbar_wait(&ctl->qi_full[s], (tau >> 1) & 1) ||
+              (mt == 0 && !mbar_wait(&ctl->kv_full[st], (n / nst) & 1)) ||
               !mbar_wait(&ctl->s_free[s], ((tau >> 1) + 1) & 1)) {
             ok = false;
             break;
@@ -234,11 +320,18 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
           const uint64_t kd = kdesc0 + (uint64_t)((st * tile_bytes) >> 4);
           for (int kk = 0; kk < d / 16; ++kk) {
             const uint64_t off = (uint64_t)(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
-            umma_bf16_ss(tmem + s * 128, qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
+            umma_bf16_ss(tmem + s * 256, qd + off, kd + off, idesc, kk > 0 ? 1u : 0u);
+          }
+          const uint64_t qid = qidesc0 + (uint64_t)((s * itile_bytes) >> 4);
+          const uint64_t kid = kidesc0 + (uint64_t)((st * itile_bytes) >> 4);
+          for (int kk = 0; kk < d_idx / 16; ++kk) {
+            const uint64_t off =
+                (uint64_t)((((kk >> per_sh) * (128 * span)) + ((kk & ((1 << per_sh) - 1)) * 32)) >> 4);
+            umma_bf16_ss(tmem + s * 256 + 128, qid + off, kid + off, idesc, kk > 0 ? 1u : 0u);
           }
           umma_commit(&ctl->s_full[s]);
           umma_commit(&ctl->q_empty[s]);
-          if (mt == ntiles - 1) umma_commit(&ctl->kv_empty[st]);   // the item's S products read K
+          if (mt == ntiles - 1) umma_commit(&ctl->kv_empty[st]);   // the item's products read its key stage
         }
         ++n;
       }
@@ -251,14 +344,12 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
   } else if (warp >= 4) {
     // -------------------------------------------------- KL rows and sums
-    const int wg = (warp - 4) >> 2;           // S slot of this warpgroup
+    constexpr int W = 32 / RQ;                // keys per 32-key chunk a lane ends with
+    const int wg = (warp - 4) >> 2;           // slot of this warpgroup
     const int wq = warp & 3;                  // TMEM lane quarter
     const int r = 32 * wq + lane;             // tile row
-    const uint32_t s_col = tmem + wg * 128 + (static_cast<uint32_t>(32 * wq) << 16);
+    const uint32_t s_col = tmem + wg * 256 + (static_cast<uint32_t>(32 * wq) << 16);
     const int ql = r / RQ, hi = r - ql * RQ;
-    const int qw = (lane / RQ);               // this lane's query within the warp
-    float* qrow = qi_s + ((warp - 4) * kKtMaxQpw + qw) * d_idx;   // its index query, as floats
-    float* psum = pb_s + ((warp - 4) * kKtMaxQpw + qw) * 32;      // its chunk of head-summed P
     const float inv_hg = 1.f / (float)Hg;
     int n = 0, tau = 0;
     while (!*abort_flag) {
@@ -270,19 +361,19 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (lane == 0) mbar_arrive(&ctl->item_empty[n % kKtItemRing]);
         break;
       }
-      const int st = n & 1;
-      const int Tb = R->Tb, Sb = R->Sb, g = R->g;
+      const int Tb = R->Tb, Sb = R->Sb, g = R->g, start = R->start;
       const int64_t qrow0 = R->qrow0;
       const int64_t blk_first = (int64_t)R->blk * kBk;
-      const uint16_t* kis = ki_s + st * 128 * d_idx;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->item_empty[n % kKtItemRing]);
       const int ntiles = (count + qpt - 1) / qpt;
       bool failed = false;
-      for (int mt = 0; mt < ntiles && !failed; ++mt, ++tau) {
+      for (int mt = 0; mt < ntiles; ++mt, ++tau) {
         if ((tau & 1) != wg) continue;
         const int idx = mt * qpt + ql;
-        const bool qvalid = ql < qpt && idx < count;    // this row's query exists
+        const bool qvalid = idx < count;                 // this row's query exists
         const bool valid = qvalid && hi < Hg;           // and its head
-        const uint32_t e = qvalid ? entries[R->start + idx] : 0u;
+        const uint32_t e = qvalid ? entries[start + idx] : 0u;
         const int64_t t = e / k;
         int limit = -1;                                  // last key of the block in the support
         if (qvalid) {
@@ -290,14 +381,7 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
           limit = lim >= kBk - 1 ? kBk - 1 : (int)lim;
         }
         const float lse2 = valid ? lse[t * H + (int64_t)g * Hg + hi] * kLog2e : 0.f;
-        // this query's index row, staged as floats by its lanes
-        __syncwarp();
-        if (qvalid)
-          for (int c = hi; c < d_idx; c += RQ) qrow[c] = __uint_as_float((uint32_t)q_idx[(t * G + g) * d_idx + c] << 16);
-        __syncwarp();
-        // the block's index rows must have landed (the S MMA waited for the same barrier phase)
-        if (!mbar_wait(&ctl->s_full[wg], (uint32_t)((tau >> 1) & 1)) ||
-            !mbar_wait(&ctl->kv_full[st], (uint32_t)((n >> 1) & 1))) {
+        if (!mbar_wait(&ctl->s_full[wg], (uint32_t)((tau >> 1) & 1))) {
           report_error(err, MSA_ERR_TIMEOUT, kSiteIndexKl, tau, 1);
           *abort_flag = 1;
           failed = true;
@@ -305,56 +389,45 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         tc_fence_after();
         float A = 0.f, B = 0.f, m = -INFINITY, l = 0.f;
-        uint32_t rr[32];
 #pragma unroll 1
         for (int c4 = 0; c4 < 4; ++c4) {
-          tmem_ld32(s_col + 32 * c4, rr);
+          uint32_t rs[32], rz[32];
+          tmem_ld32(s_col + 32 * c4, rs);
+          tmem_ld32(s_col + 128 + 32 * c4, rz);
           tmem_ld_wait();
-          // P of every head row, summed over the query's RQ rows (all lanes take part)
+          if (c4 == 3) {
+            // the slot is read: the next tile's products may overwrite it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->s_free[wg]);
+          }
+          float p[32], z[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int col = 32 * c4 + j;
-            float p = (valid && col <= limit) ? ex2_approx(fmaf(__uint_as_float(rr[j]), scale_log2, -lse2)) : 0.f;
-            for (int off = RQ >> 1; off > 0; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
-            if (hi == 0) psum[j] = p;
+            p[j] = (valid && col <= limit) ? ex2_approx(fmaf(__uint_as_float(rs[j]), scale_log2, -lse2)) : 0.f;
+            z[j] = __uint_as_float(rz[j]);
           }
-          __syncwarp();
-          // lane hi of the query takes the chunk's keys j = hi (mod RQ); the index
-          // dot product starts at a lane-dependent 8-element piece (the rows are
-          // 16-byte aligned, so lanes reading different rows avoid the same banks)
-          for (int j = hi; j < 32; j += RQ) {
-            const int col = 32 * c4 + j;
-            if (!(qvalid && col <= limit)) continue;
-            const float pbar = psum[j] * inv_hg;
-            const uint16_t* kr = kis + col * d_idx;
-            const int npc = d_idx / 8;
-            float zs = 0.f;
-            for (int i8 = 0; i8 < npc; ++i8) {
-              const int c0 = ((i8 + hi) % npc) * 8;
-              const uint4 w = *reinterpret_cast<const uint4*>(kr + c0);
-              const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+          head_reduce_scatter<RQ>(p, z, hi);
 #pragma unroll
-              for (int q2 = 0; q2 < 4; ++q2) {
-                zs += qrow[c0 + 2 * q2] * __uint_as_float(wv[q2] << 16);
-                zs += qrow[c0 + 2 * q2 + 1] * __uint_as_float(wv[q2] & 0xffff0000u);
+          for (int i = 0; i < W; ++i) {
+            const int col = 32 * c4 + W * hi + i;
+            if (qvalid && col <= limit) {
+              const float pbar = p[i] * inv_hg;
+              const float zz = temp * z[i];
+              if (pbar > 0.f) A += pbar * __logf(pbar);
+              B += pbar * zz;
+              if (zz > m) {
+                l = l * __expf(m - zz) + 1.f;
+                m = zz;
+              } else {
+                l += __expf(zz - m);
               }
             }
-            const float z = temp * zs;   // temp: the student's temperature tau
-            if (pbar > 0.f) A += pbar * __logf(pbar);
-            B += pbar * z;
-            if (z > m) {
-              l = l * __expf(m - z) + 1.f;
-              m = z;
-            } else {
-              l += __expf(z - m);
-            }
           }
-          __syncwarp();
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->s_free[wg]);
         // merge the RQ lanes of each query
+#pragma unroll
         for (int off = RQ >> 1; off > 0; off >>= 1) {
           A += __shfl_xor_sync(0xffffffffu, A, off);
           B += __shfl_xor_sync(0xffffffffu, B, off);
@@ -365,13 +438,6 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
           m = mm;
         }
         if (qvalid && hi == 0) part[((int64_t)t * G + g) * k + (e % k)] = make_float4(A, B, m, l);
-        __syncwarp();
-      }
-      // the item's index rows are read: its stage may be reused
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&ctl->kv_empty[st]);
-        mbar_arrive(&ctl->item_empty[n % kKtItemRing]);
       }
       if (failed) break;
       ++n;
@@ -383,7 +449,7 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, kKtTmemCols);
   }
 }
 
@@ -413,9 +479,16 @@ __global__ void kl_merge_kernel(const float4* __restrict__ part, int64_t npairs,
 
 }  // namespace
 
+// Key stages that fit beside the two query slots (2 where the shared memory
+// allows, else 1).
+int kl_tc_stages(int d, int d_idx) {
+  const size_t per = (size_t)128 * d * 2 + (size_t)128 * d_idx * 2;
+  return 1024 + 4 * per + sizeof(KtCtl) <= kKtSmemLimit ? 2 : 1;
+}
+
 size_t kl_tc_smem_bytes(int d, int d_idx) {
-  return 1024 + 4 * (size_t)128 * d * 2 + 2 * (size_t)128 * d_idx * 2 + sizeof(float) * 8 * kKtMaxQpw * d_idx +
-         sizeof(float) * 8 * kKtMaxQpw * 32 + sizeof(KtCtl);
+  const size_t per = (size_t)128 * d * 2 + (size_t)128 * d_idx * 2;
+  return 1024 + (size_t)(kl_tc_stages(d, d_idx) + 2) * per + sizeof(KtCtl);
 }
 
 int launch_index_kl_tc(const IndexKlArgs& a, const AttnArgs& plan, float4* part, void* stream) {
@@ -442,18 +515,30 @@ int launch_index_kl_tc(const IndexKlArgs& a, const AttnArgs& plan, float4* part,
     rc = make_tmap_bf16(&tm_q, a.q, 2, dims, strides, box, 128);
     if (rc) return rc;
   }
+  alignas(64) CUtensorMap tm_ki;
+  const int span = a.d_idx * 2 >= 128 ? 128 : a.d_idx * 2;
+  {
+    const uint64_t dims[2] = {(uint64_t)a.d_idx, (uint64_t)plan.total_k};
+    const uint64_t strides[1] = {(uint64_t)a.d_idx * 2};
+    const uint32_t box[2] = {(uint32_t)(span / 2), 128u};
+    rc = make_tmap_bf16(&tm_ki, a.k_idx, 2, dims, strides, box, span);
+    if (rc) return rc;
+  }
+  const int hg = a.H / a.G;
+  const int nst = kl_tc_stages(a.d, a.d_idx);
   const size_t smem = kl_tc_smem_bytes(a.d, a.d_idx);
-  e = cudaFuncSetAttribute(kl_items_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = hg <= 8 ? kl_items_kernel<8> : kl_items_kernel<16>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return (int)e;
   int dev = 0, nsm = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   {
     ProfScope p("index_kl", stream);
-    kl_items_kernel<<<nsm, kKtThreads, smem, st>>>(
-        tm_k, tm_q, static_cast<const uint16_t*>(a.k_idx), static_cast<const uint16_t*>(a.q_idx), a.lse, plan.items,
-        plan.nitems, plan.nitems + 1, plan.entries, a.cu_q, a.cu_k, a.H, a.G, a.d, a.d_idx, a.k,
-        a.sm_scale * 1.4426950408889634f, a.tau, plan.total_k, part, a.err);
+    kern<<<nsm, kKtThreads, smem, st>>>(
+        tm_k, tm_q, tm_ki, static_cast<const uint16_t*>(a.q_idx), a.lse, plan.items, plan.nitems,
+        plan.nitems + 1, plan.entries, a.cu_q, a.cu_k, a.H, a.G, a.d, a.d_idx, a.k, nst,
+        a.sm_scale * 1.4426950408889634f, a.tau, part, a.err);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;

@@ -363,11 +363,13 @@ msa_status_t msa_selected_share(const float* lse_sel, const float* lse_all, int6
  * branch's to follow).  ws: msa_index_kl_workspace_size bytes, 256-byte
  * aligned (the error word first).  A selected block id past the query's
  * block is recorded as MSA_ERR_DEVICE_CHECK and skipped.  k and k_idx must be 16-byte aligned
- * (their rows are read 16 bytes at a time), else MSA_ERR_INVALID_ARG.
+ * (their rows are read 16 bytes at a time), and with dense = 0 q_idx too,
+ * else MSA_ERR_INVALID_ARG.
  * The selected support (dense = 0) runs on the tensor cores: the selection is
- * inverted into the forward's KV-outer lists, each selected block's keys are
- * loaded once per work item, S = Q K^T of its gathered queries is a tcgen05
- * product, and the sums are merged per (query, group); ws must then hold
+ * inverted into the forward's KV-outer lists, each selected block's keys and
+ * index keys are loaded once per work item, S = Q K^T of its gathered queries
+ * and their index scores Z = Q_idx K_idx^T are tcgen05 products, and the sums
+ * are merged per (query, group); ws must then hold
  * msa_index_kl_workspace_size bytes (the lists and one 16-byte partial per
  * (query, group, slot)).  The dense support (the warm-up) runs on the CUDA
  * cores (one CTA per (query, group)) with the 256-byte workspace. */

@@ -79,6 +79,30 @@ def test_index_kl_matches_the_oracle(M, dense):
     np.testing.assert_allclose(kl2.cpu().numpy(), want, rtol=5e-3, atol=5e-3)
 
 
+# (H, G, d, d_idx): 4 and 8 heads per group (8 tile rows per query), index
+# rows of 64 and 256 bytes (their two swizzle widths and two boxes per row),
+# and the shape whose key and index-key tiles leave room for one key stage
+@pytest.mark.parametrize("H,G,d,d_idx", [(16, 4, 64, 32), (32, 4, 128, 128), (16, 1, 64, 128), (16, 2, 128, 64)])
+def test_index_kl_tensor_core_shapes(M, H, G, d, d_idx):
+    w = _custom("index_kl_shapes", H, G, d, d_idx, 8, hot=0.05, seed=31 + H + d_idx)
+    inp = _inputs(w, lengths=[1500, 300], T_lens=[600, 300])
+    shape, seqs, dv = _to_dev(M, w, inp)
+    sel = M.msa_index_topk(shape, seqs, dv["q_idx"], dv["k_idx"])
+    h = _host(inp)
+    cu_q, cu_k = inp["cu_q_host"], inp["cu_k_host"]
+    rows = list(range(cu_q[-1]))
+    sel_np = sel.cpu().numpy()
+    _, lse_ref = O.msa_forward_rows(h["q"], h["k"], h["v"], sel_np, cu_q, cu_k, rows, w.B_k, w.sm_scale)
+    want = K.index_kl_rows(h["q"], h["k"], h["q_idx"], h["k_idx"], sel_np, cu_q, cu_k, rows, w.B_k, w.sm_scale,
+                           TAU)
+    kl, lse_z = M.msa_index_kl(shape, seqs, dv["q"], dv["k"], dv["q_idx"], dv["k_idx"], sel,
+                               torch.from_numpy(lse_ref.astype(np.float32)).cuda(), TAU, want_lse_z=True)
+    torch.cuda.synchronize()
+    got = kl.cpu().numpy()
+    assert np.all(np.isfinite(got)) and np.all(np.isfinite(lse_z.cpu().numpy()))
+    np.testing.assert_allclose(got, want, rtol=1e-3, atol=1e-3)
+
+
 def test_index_kl_bad_block_is_reported(M):
     w, inp, shape, seqs, d, sel = _case(M)
     bad = sel.clone()
