@@ -210,9 +210,11 @@ def training_leg(args, w, W, R, msa, torch, device="cuda"):
     timed by the library's CUDA events on its launching stream over
     args.training_steps passes after args.training_warmup (inputs larger than
     L2; its own small counts, since one pass takes about 2 s).  The backward
-    and the KL gradient run on the CUDA cores and are held to the fp32 FMA
-    rate; the KL target computes its scores on the tensor cores and is held to
-    the exponential rate of the special-function units."""
+    runs on the CUDA cores and is held to the fp32 FMA rate; the KL target
+    computes its scores on the tensor cores and is held to the exponential rate
+    of the special-function units; the KL gradient computes the same scores on
+    the tensor cores and its dq_idx / dk_idx products on the CUDA cores, which
+    are held to the fp32 FMA rate."""
     tinp = W.make_inputs(w, device, T_override=args.training_T)
     shape = msa.make_shape(w.H, w.G, w.d, w.d_idx, w.k)
     seqs = msa.make_varlen(tinp["cu_q"], tinp["cu_k"], tinp["cu_q_host"], tinp["cu_k_host"])
@@ -254,6 +256,18 @@ def training_leg(args, w, W, R, msa, torch, device="cuda"):
             ach = tw[key] / (per / 1000.0) / 1e12
             res["kernels"][name] = {"ms_per_launch": per, "launches": n, "flops_per_launch": tw[key],
                                     "bound": "alu", "achieved": ach, "frac": ach / peak}
+    kr = res["kernels"].get("index_kl_grad")
+    if kr is not None:
+        # the gradient's scores run on the tensor cores; its dq_idx / dk_idx
+        # products stay on the CUDA cores and are held to the fp32 FMA rate
+        sec = kr["ms_per_launch"] / 1000.0
+        peaks, src = load_peaks()
+        ach_a = tw["kl_grad_alu_flops"] / sec / 1e12
+        ach_t = tw["kl_tensor_flops"] / sec / 1e12
+        kr.update({"flops_per_launch": tw["kl_grad_alu_flops"], "achieved": ach_a, "frac": ach_a / peak,
+                   "tensor": {"flops_per_launch": tw["kl_tensor_flops"], "achieved": ach_t,
+                              "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                              "frac": ach_t / peaks["bf16_tflops"], "peak_source": f"bf16_tflops ({src})"}})
     kr = res["kernels"].get("index_kl")
     if kr is not None:
         # the KL target's scores run on the tensor cores; what stays on the

@@ -656,6 +656,34 @@ size_t msa_index_kl_workspace_size(const msa_shape_t* shape, const msa_varlen_t*
   return dense ? kWsHeader : kl_layout(shape, seqs).total;
 }
 
+// The KV-outer plan of one pass over every query (no query tiles) in the
+// workspace of kl_layout.
+AttnArgs kl_plan_args(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q, const void* k,
+                      const int32_t* sel, DevError* err, uint8_t* base, const KlLayout& L) {
+  AttnArgs p{};
+  p.q = q; p.key = k; p.sel = sel;
+  p.cu_q = seqs->cu_q; p.cu_k = seqs->cu_k;
+  p.batch = seqs->batch; p.H = shape->H; p.G = shape->G; p.d = shape->d; p.k = shape->k; p.B_k = shape->B_k;
+  p.sm_scale = shape->sm_scale;
+  p.total_q = seqs->total_q; p.total_k = seqs->total_k;
+  p.max_q_len = seqs->max_q_len; p.max_k_len = seqs->max_k_len;
+  p.t0 = 0; p.t1 = seqs->total_q;
+  p.err = err;
+  p.blk_off = reinterpret_cast<int32_t*>(base + L.blk_off);
+  p.counts = reinterpret_cast<int32_t*>(base + L.counts);
+  p.cursor = reinterpret_cast<int32_t*>(base + L.cursor);
+  p.tile_sums = reinterpret_cast<int32_t*>(base + L.tile_sums);
+  p.nitems = reinterpret_cast<int32_t*>(base + L.nitems);
+  p.entries = reinterpret_cast<uint32_t*>(base + L.entries);
+  p.items = reinterpret_cast<Item*>(base + L.items);
+  p.max_items = L.max_items;
+  p.nlists = L.nlists;
+  p.win_rows = L.win;
+  p.queries_per_item = L.qpi;
+  p.theta = 0;
+  return p;
+}
+
 msa_status_t msa_index_kl(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q, const void* k,
                           const void* q_idx, const void* k_idx, const int32_t* sel, const float* lse, float tau,
                           int32_t dense, float* kl, float* lse_z, void* ws, size_t ws_bytes, void* stream) {
@@ -673,27 +701,7 @@ msa_status_t msa_index_kl(const msa_shape_t* shape, const msa_varlen_t* seqs, co
   const KlLayout L = kl_layout(shape, seqs);
   if (!ws_ok(ws, ws_bytes, L.total)) return MSA_ERR_WORKSPACE;
   uint8_t* base = static_cast<uint8_t*>(ws);
-  AttnArgs p{};
-  p.q = q; p.key = k; p.sel = sel;
-  p.cu_q = seqs->cu_q; p.cu_k = seqs->cu_k;
-  p.batch = seqs->batch; p.H = shape->H; p.G = shape->G; p.d = shape->d; p.k = shape->k; p.B_k = shape->B_k;
-  p.sm_scale = shape->sm_scale;
-  p.total_q = seqs->total_q; p.total_k = seqs->total_k;
-  p.max_q_len = seqs->max_q_len; p.max_k_len = seqs->max_k_len;
-  p.t0 = 0; p.t1 = seqs->total_q;
-  p.err = a.err;
-  p.blk_off = reinterpret_cast<int32_t*>(base + L.blk_off);
-  p.counts = reinterpret_cast<int32_t*>(base + L.counts);
-  p.cursor = reinterpret_cast<int32_t*>(base + L.cursor);
-  p.tile_sums = reinterpret_cast<int32_t*>(base + L.tile_sums);
-  p.nitems = reinterpret_cast<int32_t*>(base + L.nitems);
-  p.entries = reinterpret_cast<uint32_t*>(base + L.entries);
-  p.items = reinterpret_cast<Item*>(base + L.items);
-  p.max_items = L.max_items;
-  p.nlists = L.nlists;
-  p.win_rows = L.win;
-  p.queries_per_item = L.qpi;
-  p.theta = 0;
+  const AttnArgs p = kl_plan_args(shape, seqs, q, k, sel, a.err, base, L);
   return launch_index_kl_tc(a, p, reinterpret_cast<float4*>(base + L.part), stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
 }
 
@@ -710,6 +718,15 @@ msa_status_t msa_index_kl_backward(const msa_shape_t* shape, const msa_varlen_t*
   const msa_status_t st = index_kl_common(shape, seqs, q, k, q_idx, k_idx, sel, lse, tau, dense, ws, ws_bytes,
                                           stream, &a);
   if (st != MSA_OK || seqs->total_q == 0) return st;
+  // selected support: the tensor-core form over the same plan as msa_index_kl
+  // (index-query rows read and dq_idx rows added 16 bytes at a time)
+  KlLayout L{};
+  if (!dense) {
+    if ((reinterpret_cast<uintptr_t>(q_idx) | reinterpret_cast<uintptr_t>(dq_idx)) & 15u)
+      return MSA_ERR_INVALID_ARG;
+    L = kl_layout(shape, seqs);
+    if (!ws_ok(ws, ws_bytes, L.total)) return MSA_ERR_WORKSPACE;
+  }
   // the key gradient is accumulated over every query that reaches a key row
   if (cudaMemsetAsync(dk_idx, 0, sizeof(float) * (size_t)seqs->total_k * shape->d_idx,
                       reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
@@ -717,7 +734,9 @@ msa_status_t msa_index_kl_backward(const msa_shape_t* shape, const msa_varlen_t*
   a.lse_z = const_cast<float*>(lse_z);
   a.dq_idx = dq_idx;
   a.dk_idx = dk_idx;
-  return launch_index_kl_backward(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
+  if (dense) return launch_index_kl_backward(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
+  const AttnArgs p = kl_plan_args(shape, seqs, q, k, sel, a.err, static_cast<uint8_t*>(ws), L);
+  return launch_index_kl_grad_tc(a, p, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
 }
 
 msa_status_t msa_select_window(const msa_shape_t* shape, const msa_varlen_t* seqs, int32_t n_sink, int32_t* sel,

@@ -29,6 +29,15 @@
 //               written as one float4 per (query, group, selected slot).
 // kl_merge_kernel: per (query, group) the float4s of its slots give KL =
 // sum A - sum B + log-sum-exp of z, and the student's log-sum-exp.
+//
+// The same kernel in its gradient form (GRAD) computes, from the same P-bar
+// and z and the student's log-sum-exp of the forward, w_j = tau (Q_j - P-bar_j)
+// per (query, key) of the tile (the derivative of the KL with respect to the
+// raw index score, the teacher held constant) into a shared table; then each
+// warpgroup adds dq_idx[t, g] += sum_j w_j k_idx[j] (a thread per (query,
+// 8-column chunk), the keys split across threads where there are fewer than
+// 128 such pairs) and dk_idx[j] += sum_t w_j q_idx[t, g] (a thread per key),
+// both with vector reductions to global memory.
 #include <cuda_runtime.h>
 
 #include "msa_common.cuh"
@@ -43,9 +52,11 @@ constexpr int kKtItemRing = 4;
 constexpr int kKtItemEmptyCount = 11;  // MMA issuer 1 + index-query warps 2 + KL warps 8
 constexpr uint32_t kKtTmemCols = 512;  // per slot: S in columns [0, 128), Z in [128, 256)
 constexpr size_t kKtSmemLimit = 232448;
+constexpr int kWtStride = 132;         // floats per row of the gradient's w table (16-byte rows, banks offset by 4)
 
 struct __align__(16) KtItem {
   int32_t seq, blk, g, start, count, Tb, Sb, qrow0;
+  int32_t krow, pad0, pad1, pad2;
 };
 
 struct __align__(16) KtCtl {
@@ -53,6 +64,7 @@ struct __align__(16) KtCtl {
   uint64_t kv_full[2], kv_empty[2];
   uint64_t q_full[2], qi_full[2], q_empty[2];
   uint64_t s_full[2], s_free[2];
+  uint64_t w_ready[2], rd_done[2];      // gradient: per warpgroup, its w table written / read
   uint64_t mma_done;
   uint32_t tmem_base;
   int32_t abort_flag;
@@ -80,14 +92,29 @@ __device__ __forceinline__ void head_reduce_scatter(float (&p)[32], float (&z)[3
   }
 }
 
-template <int RQ>
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ void red_add4(float* dst, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+// Shared bytes of the gradient's tables: per warpgroup a w table [qpt x 128]
+// (rows of kWtStride floats) and the tile's index queries as floats [qpt x d_idx].
+__host__ __device__ constexpr size_t kl_grad_bytes(int qpt, int d_idx) {
+  return 2 * (size_t)qpt * kWtStride * 4 + 2 * (size_t)qpt * d_idx * 4;
+}
+
+template <int RQ, bool GRAD>
 __global__ void __launch_bounds__(kKtThreads, 1)
 kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                 const __grid_constant__ CUtensorMap tm_ki, const uint16_t* __restrict__ q_idx,
                 const float* __restrict__ lse, const Item* __restrict__ items, const int32_t* __restrict__ nitems_p,
                 int32_t* __restrict__ ticket, const uint32_t* __restrict__ entries, const int32_t* __restrict__ cu_q,
                 const int32_t* __restrict__ cu_k, int H, int G, int d, int d_idx, int k, int nst, float scale_log2,
-                float temp, float4* __restrict__ part, DevError* err) {
+                float temp, float4* __restrict__ part, const float* __restrict__ lse_z, float* __restrict__ dq_idx,
+                float* __restrict__ dk_idx, DevError* err) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -100,12 +127,14 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
   uint8_t* ki_s = k_s + nst * tile_bytes;       // nst stages of K_idx
   uint8_t* q_s = ki_s + nst * itile_bytes;      // 2 slots of gathered Q rows
   uint8_t* qi_s = q_s + 2 * tile_bytes;         // 2 slots of the index-query operand
-  KtCtl* ctl = reinterpret_cast<KtCtl*>(qi_s + 2 * itile_bytes);
+  constexpr int qpt = 128 / RQ;                 // queries per 128-row tile
+  float* wt = reinterpret_cast<float*>(qi_s + 2 * itile_bytes);   // gradient tables (GRAD)
+  float* qf = wt + 2 * qpt * kWtStride;
+  KtCtl* ctl = reinterpret_cast<KtCtl*>(qi_s + 2 * itile_bytes + (GRAD ? kl_grad_bytes(qpt, d_idx) : 0));
   volatile int32_t* abort_flag = &ctl->abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Hg = H / G;
-  constexpr int qpt = 128 / RQ;                 // queries per 128-row tile
   const int nhalf = d / 64;
   const int nitems = *nitems_p;
   constexpr float kLog2e = 1.4426950408889634f;
@@ -117,12 +146,14 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl->kv_full[i], 1);
-      mbar_init(&ctl->kv_empty[i], 1);
+      mbar_init(&ctl->kv_empty[i], GRAD ? 9 : 1);   // gradient: the KL warps read the index keys too
       mbar_init(&ctl->q_full[i], 1);
       mbar_init(&ctl->qi_full[i], 1);
       mbar_init(&ctl->q_empty[i], 1);
       mbar_init(&ctl->s_full[i], 1);
       mbar_init(&ctl->s_free[i], 4);
+      mbar_init(&ctl->w_ready[i], 4);
+      mbar_init(&ctl->rd_done[i], 4);
     }
     mbar_init(&ctl->mma_done, 1);
     ctl->abort_flag = 0;
@@ -178,12 +209,13 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         R->Tb = cu_q[I.seq + 1] - cu_q[I.seq];
         R->Sb = cu_k[I.seq + 1] - cu_k[I.seq];
         R->qrow0 = cu_q[I.seq];
+        const int krow = cu_k[I.seq] + I.blk * kBk;
+        R->krow = krow;
         mbar_arrive(&ctl->item_full[slot]);
         // the block's keys and index keys (TMA fills rows past the keys with zeros)
         const int st = n % nst;
         ok = mbar_wait(&ctl->kv_empty[st], ((n / nst) + 1) & 1);
         if (ok) {
-          const int krow = cu_k[I.seq] + I.blk * kBk;
           mbar_arrive_expect_tx(&ctl->kv_full[st], (uint32_t)(tile_bytes + itile_bytes));
           for (int h = 0; h < nhalf; ++h)
             tma_load_3d(k_s + st * tile_bytes + h * 128 * 128, &tm_k, &ctl->kv_full[st], 64 * h, I.g, krow);
@@ -351,6 +383,11 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const uint32_t s_col = tmem + wg * 256 + (static_cast<uint32_t>(32 * wq) << 16);
     const int ql = r / RQ, hi = r - ql * RQ;
     const float inv_hg = 1.f / (float)Hg;
+    const int tw = 32 * wq + lane;            // thread of the warpgroup
+    const int cpr8 = d_idx / 8;               // 8-column chunks per index row
+    float* wt_g = wt + wg * qpt * kWtStride;  // gradient: this warpgroup's w table
+    float* qf_g = qf + wg * qpt * d_idx;      // and its tile's index queries as floats
+    int ktile = 0;                            // tiles this warpgroup has taken
     int n = 0, tau = 0;
     while (!*abort_flag) {
       const KtItem* R = wait_item(n);
@@ -362,6 +399,8 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         break;
       }
       const int Tb = R->Tb, Sb = R->Sb, g = R->g, start = R->start;
+      const int64_t krow = R->krow;
+      const int st = n % nst;
       const int64_t qrow0 = R->qrow0;
       const int64_t blk_first = (int64_t)R->blk * kBk;
       __syncwarp();
@@ -381,7 +420,32 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
           limit = lim >= kBk - 1 ? kBk - 1 : (int)lim;
         }
         const float lse2 = valid ? lse[t * H + (int64_t)g * Hg + hi] * kLog2e : 0.f;
-        if (!mbar_wait(&ctl->s_full[wg], (uint32_t)((tau >> 1) & 1))) {
+        float lsez2 = 0.f;
+        if constexpr (GRAD) {
+          lsez2 = qvalid ? lse_z[t * G + g] * kLog2e : 0.f;
+          // the previous tile's tables are read; this tile's index queries as floats
+          if (ktile > 0 && !mbar_wait(&ctl->rd_done[wg], (uint32_t)((ktile - 1) & 1))) {
+            report_error(err, MSA_ERR_TIMEOUT, kSiteIndexKl, tau, 2);
+            *abort_flag = 1;
+            failed = true;
+            break;
+          }
+          for (int u2 = tw; u2 < qpt * cpr8; u2 += 128) {
+            const int q2 = u2 / cpr8, c8 = u2 - q2 * cpr8;
+            const int i2 = mt * qpt + q2;
+            float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), up = lo;
+            if (i2 < count) {
+              const int64_t t2 = entries[start + i2] / k;
+              const uint4 v = *reinterpret_cast<const uint4*>(q_idx + (t2 * G + g) * d_idx + c8 * 8);
+              lo = make_float4(bf_lo(v.x), bf_hi(v.x), bf_lo(v.y), bf_hi(v.y));
+              up = make_float4(bf_lo(v.z), bf_hi(v.z), bf_lo(v.w), bf_hi(v.w));
+            }
+            *reinterpret_cast<float4*>(qf_g + q2 * d_idx + c8 * 8) = lo;
+            *reinterpret_cast<float4*>(qf_g + q2 * d_idx + c8 * 8 + 4) = up;
+          }
+        }
+        if (!mbar_wait(&ctl->s_full[wg], (uint32_t)((tau >> 1) & 1)) ||
+            (GRAD && !mbar_wait(&ctl->kv_full[st], (uint32_t)((n / nst) & 1)))) {
           report_error(err, MSA_ERR_TIMEOUT, kSiteIndexKl, tau, 1);
           *abort_flag = 1;
           failed = true;
@@ -409,37 +473,137 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             z[j] = __uint_as_float(rz[j]);
           }
           head_reduce_scatter<RQ>(p, z, hi);
+          if constexpr (GRAD) {
+            // w = tau (Q - P-bar) of the lane's keys
 #pragma unroll
-          for (int i = 0; i < W; ++i) {
-            const int col = 32 * c4 + W * hi + i;
-            if (qvalid && col <= limit) {
-              const float pbar = p[i] * inv_hg;
-              const float zz = temp * z[i];
-              if (pbar > 0.f) A += pbar * __logf(pbar);
-              B += pbar * zz;
-              if (zz > m) {
-                l = l * __expf(m - zz) + 1.f;
-                m = zz;
-              } else {
-                l += __expf(zz - m);
+            for (int i = 0; i < W; ++i) {
+              const int col = 32 * c4 + W * hi + i;
+              float w = 0.f;
+              if (qvalid && col <= limit)
+                w = temp * (ex2_approx(temp * z[i] * kLog2e - lsez2) - p[i] * inv_hg);
+              wt_g[ql * kWtStride + col] = w;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < W; ++i) {
+              const int col = 32 * c4 + W * hi + i;
+              if (qvalid && col <= limit) {
+                const float pbar = p[i] * inv_hg;
+                const float zz = temp * z[i];
+                if (pbar > 0.f) A += pbar * __logf(pbar);
+                B += pbar * zz;
+                if (zz > m) {
+                  l = l * __expf(m - zz) + 1.f;
+                  m = zz;
+                } else {
+                  l += __expf(zz - m);
+                }
               }
             }
           }
         }
-        // merge the RQ lanes of each query
+        if constexpr (GRAD) {
+          // the tile's w table is complete once the warpgroup's four warps have written
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->w_ready[wg]);
+          if (!mbar_wait(&ctl->w_ready[wg], (uint32_t)(ktile & 1))) {
+            report_error(err, MSA_ERR_TIMEOUT, kSiteIndexKl, tau, 3);
+            *abort_flag = 1;
+            failed = true;
+            break;
+          }
+          const int nq = min(qpt, count - mt * qpt);
+          // dq_idx[t, g] += sum_j w_j k_idx[j]: a thread per (query, 8-column
+          // chunk), the keys split over ks threads (adjacent lanes) where
+          // there are fewer than 128 such pairs
+          {
+            const int pairs = qpt * cpr8;
+            const int ks = pairs >= 128 ? 1 : 128 / pairs;
+            const int per = pairs > 128 ? pairs / 128 : 1;
+            const int nkeys = 128 / ks;
+            const int split = tw % ks;
+            const uint8_t* kst = ki_s + st * itile_bytes;
+            for (int pp = 0; pp < per; ++pp) {
+              const int pid = tw / ks + pp * (128 / ks);
+              const int q2 = pid / cpr8, c8 = pid - q2 * cpr8;
+              const int cel = c8 * 8, box = cel / span_el, cin = (cel - box * span_el) / 8;
+              const uint8_t* kb = kst + box * 128 * span;
+              const float* wr = wt_g + q2 * kWtStride;
+              float acc[8];
 #pragma unroll
-        for (int off = RQ >> 1; off > 0; off >>= 1) {
-          A += __shfl_xor_sync(0xffffffffu, A, off);
-          B += __shfl_xor_sync(0xffffffffu, B, off);
-          const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
-          const float l2 = __shfl_xor_sync(0xffffffffu, l, off);
-          const float mm = fmaxf(m, m2);
-          l = (l > 0.f ? l * __expf(m - mm) : 0.f) + (l2 > 0.f ? l2 * __expf(m2 - mm) : 0.f);
-          m = mm;
+              for (int e2 = 0; e2 < 8; ++e2) acc[e2] = 0.f;
+              if (q2 < nq) {
+#pragma unroll 4
+                for (int jj = 0; jj < nkeys; ++jj) {
+                  // each split starts at its own row (lanes reading the same chunk of rows
+                  // 64 apart would meet in one bank)
+                  const int j = split * nkeys + ((jj + split) & (nkeys - 1));
+                  const float wv = wr[j];
+                  const uint4 kv = *reinterpret_cast<const uint4*>(kb + swz_offset(j, cin, span));
+                  acc[0] += wv * bf_lo(kv.x); acc[1] += wv * bf_hi(kv.x);
+                  acc[2] += wv * bf_lo(kv.y); acc[3] += wv * bf_hi(kv.y);
+                  acc[4] += wv * bf_lo(kv.z); acc[5] += wv * bf_hi(kv.z);
+                  acc[6] += wv * bf_lo(kv.w); acc[7] += wv * bf_hi(kv.w);
+                }
+              }
+              for (int off = 1; off < ks; off <<= 1) {
+#pragma unroll
+                for (int e2 = 0; e2 < 8; ++e2) acc[e2] += __shfl_xor_sync(0xffffffffu, acc[e2], off);
+              }
+              if (split == 0 && q2 < nq) {
+                const int64_t t2 = entries[start + mt * qpt + q2] / k;
+                float* dst = dq_idx + (t2 * G + g) * d_idx + cel;
+                red_add4(dst, acc[0], acc[1], acc[2], acc[3]);
+                red_add4(dst + 4, acc[4], acc[5], acc[6], acc[7]);
+              }
+            }
+          }
+          // dk_idx[j] += sum over the tile's queries of w_j q_idx[t, g]: a thread per key
+          if (blk_first + tw < Sb) {
+            float* dst = dk_idx + (krow + tw) * d_idx;
+            for (int c0 = 0; c0 < d_idx; c0 += 32) {
+              float acc[32];
+#pragma unroll
+              for (int e2 = 0; e2 < 32; ++e2) acc[e2] = 0.f;
+              for (int q2 = 0; q2 < nq; ++q2) {
+                const float wv = wt_g[q2 * kWtStride + tw];
+                const float4* qr = reinterpret_cast<const float4*>(qf_g + q2 * d_idx + c0);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                  const float4 x = qr[c];
+                  acc[4 * c] += wv * x.x; acc[4 * c + 1] += wv * x.y;
+                  acc[4 * c + 2] += wv * x.z; acc[4 * c + 3] += wv * x.w;
+                }
+              }
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                red_add4(dst + c0 + 4 * c, acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->rd_done[wg]);
+          ++ktile;
+        } else {
+          // merge the RQ lanes of each query
+#pragma unroll
+          for (int off = RQ >> 1; off > 0; off >>= 1) {
+            A += __shfl_xor_sync(0xffffffffu, A, off);
+            B += __shfl_xor_sync(0xffffffffu, B, off);
+            const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+            const float l2 = __shfl_xor_sync(0xffffffffu, l, off);
+            const float mm = fmaxf(m, m2);
+            l = (l > 0.f ? l * __expf(m - mm) : 0.f) + (l2 > 0.f ? l2 * __expf(m2 - mm) : 0.f);
+            m = mm;
+          }
+          if (qvalid && hi == 0) part[((int64_t)t * G + g) * k + (e % k)] = make_float4(A, B, m, l);
         }
-        if (qvalid && hi == 0) part[((int64_t)t * G + g) * k + (e % k)] = make_float4(A, B, m, l);
       }
       if (failed) break;
+      if constexpr (GRAD) {
+        // the item's index keys are read: its key stage may be reused
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->kv_empty[st]);
+      }
       ++n;
     }
   }
@@ -477,19 +641,74 @@ __global__ void kl_merge_kernel(const float4* __restrict__ part, int64_t npairs,
   if (lse_z != nullptr) lse_z[pr] = l > 0.f ? m + __logf(l) : -INFINITY;
 }
 
+
+// Key stages that fit beside the two query slots and, for the gradient, its
+// tables (2 where the shared memory allows, else 1).
+int kl_tc_stages(int d, int d_idx, size_t extra) {
+  const size_t per = (size_t)128 * d * 2 + (size_t)128 * d_idx * 2;
+  return 1024 + 4 * per + extra + sizeof(KtCtl) <= kKtSmemLimit ? 2 : 1;
+}
+
+size_t kl_tc_smem_bytes(int d, int d_idx, size_t extra) {
+  const size_t per = (size_t)128 * d * 2 + (size_t)128 * d_idx * 2;
+  return 1024 + (size_t)(kl_tc_stages(d, d_idx, extra) + 2) * per + extra + sizeof(KtCtl);
+}
+
+// Tensor maps of the key blocks (3D: column, group, row), the gathered query
+// rows (one box per query: its group's head rows, at least 8) and the
+// index-key blocks (swizzled as the index rows' width allows).
+int kl_tc_maps(const IndexKlArgs& a, int64_t total_k, CUtensorMap* tm_k, CUtensorMap* tm_q, CUtensorMap* tm_ki) {
+  {
+    const uint64_t dims[3] = {(uint64_t)a.d, (uint64_t)a.G, (uint64_t)total_k};
+    const uint64_t strides[2] = {(uint64_t)a.d * 2, (uint64_t)a.G * a.d * 2};
+    const uint32_t box[3] = {64u, 1u, 128u};
+    const int rc = make_tmap_bf16(tm_k, a.key, 3, dims, strides, box, 128);
+    if (rc) return rc;
+  }
+  {
+    const int hg = a.H / a.G;
+    const uint64_t dims[2] = {(uint64_t)a.d, (uint64_t)a.total_q * a.H};
+    const uint64_t strides[1] = {(uint64_t)a.d * 2};
+    const uint32_t box[2] = {64u, (uint32_t)(hg < 8 ? 8 : hg)};
+    const int rc = make_tmap_bf16(tm_q, a.q, 2, dims, strides, box, 128);
+    if (rc) return rc;
+  }
+  const int span = a.d_idx * 2 >= 128 ? 128 : a.d_idx * 2;
+  const uint64_t dims[2] = {(uint64_t)a.d_idx, (uint64_t)total_k};
+  const uint64_t strides[1] = {(uint64_t)a.d_idx * 2};
+  const uint32_t box[2] = {(uint32_t)(span / 2), 128u};
+  return make_tmap_bf16(tm_ki, a.k_idx, 2, dims, strides, box, span);
+}
+
+// The persistent items kernel over the plan's lists: the target's partials
+// (GRAD false) or the gradient's reductions into dq_idx / dk_idx.
+template <bool GRAD>
+int launch_items(const IndexKlArgs& a, const AttnArgs& plan, float4* part, const char* name, void* stream) {
+  alignas(64) CUtensorMap tm_k, tm_q, tm_ki;
+  int rc = kl_tc_maps(a, plan.total_k, &tm_k, &tm_q, &tm_ki);
+  if (rc) return rc;
+  const int hg = a.H / a.G;
+  const int rq = hg <= 8 ? 8 : 16;
+  const size_t extra = GRAD ? kl_grad_bytes(128 / rq, a.d_idx) : 0;
+  const int nst = kl_tc_stages(a.d, a.d_idx, extra);
+  const size_t smem = kl_tc_smem_bytes(a.d, a.d_idx, extra);
+  auto kern = rq == 8 ? kl_items_kernel<8, GRAD> : kl_items_kernel<16, GRAD>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return (int)e;
+  int dev = 0, nsm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  {
+    ProfScope p(name, stream);
+    kern<<<nsm, kKtThreads, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
+        tm_k, tm_q, tm_ki, static_cast<const uint16_t*>(a.q_idx), a.lse, plan.items, plan.nitems,
+        plan.nitems + 1, plan.entries, a.cu_q, a.cu_k, a.H, a.G, a.d, a.d_idx, a.k, nst,
+        a.sm_scale * 1.4426950408889634f, a.tau, part, a.lse_z, a.dq_idx, a.dk_idx, a.err);
+  }
+  return (int)cudaGetLastError();
+}
+
 }  // namespace
-
-// Key stages that fit beside the two query slots (2 where the shared memory
-// allows, else 1).
-int kl_tc_stages(int d, int d_idx) {
-  const size_t per = (size_t)128 * d * 2 + (size_t)128 * d_idx * 2;
-  return 1024 + 4 * per + sizeof(KtCtl) <= kKtSmemLimit ? 2 : 1;
-}
-
-size_t kl_tc_smem_bytes(int d, int d_idx) {
-  const size_t per = (size_t)128 * d * 2 + (size_t)128 * d_idx * 2;
-  return 1024 + (size_t)(kl_tc_stages(d, d_idx) + 2) * per + sizeof(KtCtl);
-}
 
 int launch_index_kl_tc(const IndexKlArgs& a, const AttnArgs& plan, float4* part, void* stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -499,54 +718,25 @@ int launch_index_kl_tc(const IndexKlArgs& a, const AttnArgs& plan, float4* part,
   if (e != cudaSuccess) return (int)e;
   int rc = launch_kv_plan(plan, stream);
   if (rc) return rc;
-  alignas(64) CUtensorMap tm_k, tm_q;
-  {
-    const uint64_t dims[3] = {(uint64_t)a.d, (uint64_t)a.G, (uint64_t)plan.total_k};
-    const uint64_t strides[2] = {(uint64_t)a.d * 2, (uint64_t)a.G * a.d * 2};
-    const uint32_t box[3] = {64u, 1u, 128u};
-    rc = make_tmap_bf16(&tm_k, a.key, 3, dims, strides, box, 128);
-    if (rc) return rc;
-  }
-  {
-    const int hg = a.H / a.G;
-    const uint64_t dims[2] = {(uint64_t)a.d, (uint64_t)a.total_q * a.H};
-    const uint64_t strides[1] = {(uint64_t)a.d * 2};
-    const uint32_t box[2] = {64u, (uint32_t)(hg < 8 ? 8 : hg)};
-    rc = make_tmap_bf16(&tm_q, a.q, 2, dims, strides, box, 128);
-    if (rc) return rc;
-  }
-  alignas(64) CUtensorMap tm_ki;
-  const int span = a.d_idx * 2 >= 128 ? 128 : a.d_idx * 2;
-  {
-    const uint64_t dims[2] = {(uint64_t)a.d_idx, (uint64_t)plan.total_k};
-    const uint64_t strides[1] = {(uint64_t)a.d_idx * 2};
-    const uint32_t box[2] = {(uint32_t)(span / 2), 128u};
-    rc = make_tmap_bf16(&tm_ki, a.k_idx, 2, dims, strides, box, span);
-    if (rc) return rc;
-  }
-  const int hg = a.H / a.G;
-  const int nst = kl_tc_stages(a.d, a.d_idx);
-  const size_t smem = kl_tc_smem_bytes(a.d, a.d_idx);
-  auto kern = hg <= 8 ? kl_items_kernel<8> : kl_items_kernel<16>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return (int)e;
-  int dev = 0, nsm = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  {
-    ProfScope p("index_kl", stream);
-    kern<<<nsm, kKtThreads, smem, st>>>(
-        tm_k, tm_q, tm_ki, static_cast<const uint16_t*>(a.q_idx), a.lse, plan.items, plan.nitems,
-        plan.nitems + 1, plan.entries, a.cu_q, a.cu_k, a.H, a.G, a.d, a.d_idx, a.k, nst,
-        a.sm_scale * 1.4426950408889634f, a.tau, part, a.err);
-  }
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return (int)e;
+  rc = launch_items<false>(a, plan, part, "index_kl", stream);
+  if (rc) return rc;
   {
     ProfScope p("index_kl_merge", stream);
     kl_merge_kernel<<<(unsigned)((npairs + 255) / 256), 256, 0, st>>>(part, npairs, a.k, a.kl, a.lse_z);
   }
   return (int)cudaGetLastError();
+}
+
+int launch_index_kl_grad_tc(const IndexKlArgs& a, const AttnArgs& plan, void* stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t npairs = a.total_q * a.G;
+  if (npairs <= 0) return 0;
+  // both gradients are sums of the items' reductions
+  cudaError_t e = cudaMemsetAsync(a.dq_idx, 0, sizeof(float) * (size_t)npairs * a.d_idx, st);
+  if (e != cudaSuccess) return (int)e;
+  int rc = launch_kv_plan(plan, stream);
+  if (rc) return rc;
+  return launch_items<true>(a, plan, nullptr, "index_kl_grad", stream);
 }
 
 }  // namespace msa

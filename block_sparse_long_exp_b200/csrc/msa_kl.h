@@ -35,5 +35,9 @@ int launch_index_kl(const IndexKlArgs& a, void* stream);
 // [T, G, k] partials and is zeroed by the call.
 int launch_index_kl_tc(const IndexKlArgs& a, const AttnArgs& plan, float4* part, void* stream);
 int launch_index_kl_backward(const IndexKlArgs& a, void* stream);
+// The gradient on the sparse support over the same plan (msa_index_kl_tc.cu):
+// zeroes dq_idx, plans, then adds every item's contributions to dq_idx and
+// dk_idx (which the caller has zeroed).
+int launch_index_kl_grad_tc(const IndexKlArgs& a, const AttnArgs& plan, void* stream);
 
 }  // namespace msa

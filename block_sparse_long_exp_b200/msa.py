@@ -698,7 +698,8 @@ def msa_index_kl_backward(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.
                           check: bool = True) -> Tuple[torch.Tensor, torch.Tensor]:
     """Gradient of the summed KL with respect to the index query and keys, the
     teacher held constant: returns dq_idx float [T, G, d_idx] and dk_idx float
-    [S, d_idx].  lse_z: from msa_index_kl(..., want_lse_z=True)."""
+    [S, d_idx].  lse_z: from msa_index_kl(..., want_lse_z=True).  ws: as
+    msa_index_kl's (msa_index_kl_workspace_size bytes)."""
     lib = load_library()
     T, S = seqs.total_q, seqs.total_k
     _index_kl_args(shape, seqs, q, k, q_idx, k_idx, sel, lse, dense)
@@ -708,7 +709,10 @@ def msa_index_kl_backward(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.
     dq = torch.empty((T, shape.G, shape.d_idx), dtype=torch.float32, device=q.device)
     dk = torch.empty((S, shape.d_idx), dtype=torch.float32, device=q.device)
     if ws is None:
-        ws = _workspace(256, q.device)
+        need = msa_index_kl_workspace_size(shape, seqs, dense)
+        if need == 0:
+            raise MsaError("msa_index_kl_backward: unsupported or invalid shape")
+        ws = _workspace(need, q.device)
     rc = lib.msa_index_kl_backward(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q), _ptr(k), _ptr(q_idx),
                                    _ptr(k_idx), _ptr(sel), _ptr(lse), _ptr(lse_z), float(tau), 1 if dense else 0,
                                    _ptr(dq), _ptr(dk), _ptr(ws), _nbytes(ws), _stream(stream))

@@ -83,9 +83,12 @@ def training_work(S_lens: Sequence[int], T_lens: Sequence[int], H: int, G: int, 
     pairs = main / (4 * H * d)            # attended (query, key) pairs of one head
     return {"pairs": pairs, "backward_flops": 10.0 * H * d * pairs,
             "kl_flops": pairs * (2.0 * H * d + 2.0 * G * d_idx),
-            "kl_tensor_flops": pairs * 2.0 * H * d,     # the teacher scores q . k (on the tensor cores)
+            # on the tensor cores: the teacher scores q . k and the raw index scores q_idx . k_idx
+            "kl_tensor_flops": pairs * (2.0 * H * d + 2.0 * G * d_idx),
             "kl_exps": pairs * H,                        # one exponential per head and attended pair
-            "kl_grad_flops": pairs * (2.0 * H * d + 6.0 * G * d_idx)}
+            "kl_grad_flops": pairs * (2.0 * H * d + 6.0 * G * d_idx),
+            # the gradient's products on the CUDA cores: dq_idx and dk_idx, 2 d_idx each
+            "kl_grad_alu_flops": pairs * 4.0 * G * d_idx}
 
 
 def alu_fp32_tflops(sms: int = 148, lanes: int = 128, mhz: float = 1965.0) -> float:

@@ -393,7 +393,13 @@ msa_status_t msa_index_kl(const msa_shape_t* shape, const msa_varlen_t* seqs,
  *                     zeroed by the call, then accumulated atomically, so
  *                     its rounding order varies from run to run)
  * Arguments as msa_index_kl, plus lse_z from it; dk_idx must be 16-byte
- * aligned too (its rows are added 16 bytes at a time). */
+ * aligned too (its rows are added 16 bytes at a time), and with dense = 0
+ * dq_idx too.  The selected support (dense = 0) runs over the same plan and
+ * workspace as msa_index_kl (msa_index_kl_workspace_size bytes): per work
+ * item S and the index scores are tcgen05 products, w_j = tau (Q_j - P_j) per
+ * (query, key) is formed from them, and both gradients are added with vector
+ * reductions (their rounding order varies between runs); the dense support
+ * runs on the CUDA cores with the 256-byte workspace. */
 msa_status_t msa_index_kl_backward(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q,
                                    const void* k, const void* q_idx, const void* k_idx, const int32_t* sel,
                                    const float* lse, const float* lse_z, float tau, int32_t dense, float* dq_idx,

@@ -79,9 +79,10 @@ def test_index_kl_matches_the_oracle(M, dense):
     np.testing.assert_allclose(kl2.cpu().numpy(), want, rtol=5e-3, atol=5e-3)
 
 
-# (H, G, d, d_idx): 4 and 8 heads per group (8 tile rows per query), index
-# rows of 64 and 256 bytes (their two swizzle widths and two boxes per row),
-# and the shape whose key and index-key tiles leave room for one key stage
+# The tensor-core target and gradient over (H, G, d, d_idx): 4 and 8 heads per
+# group (8 tile rows per query), index rows of 64 and 256 bytes (their two
+# swizzle widths and two boxes per row), and the shape whose key and
+# index-key tiles leave room for one key stage
 @pytest.mark.parametrize("H,G,d,d_idx", [(16, 4, 64, 32), (32, 4, 128, 128), (16, 1, 64, 128), (16, 2, 128, 64)])
 def test_index_kl_tensor_core_shapes(M, H, G, d, d_idx):
     w = _custom("index_kl_shapes", H, G, d, d_idx, 8, hot=0.05, seed=31 + H + d_idx)
@@ -95,12 +96,19 @@ def test_index_kl_tensor_core_shapes(M, H, G, d, d_idx):
     _, lse_ref = O.msa_forward_rows(h["q"], h["k"], h["v"], sel_np, cu_q, cu_k, rows, w.B_k, w.sm_scale)
     want = K.index_kl_rows(h["q"], h["k"], h["q_idx"], h["k_idx"], sel_np, cu_q, cu_k, rows, w.B_k, w.sm_scale,
                            TAU)
-    kl, lse_z = M.msa_index_kl(shape, seqs, dv["q"], dv["k"], dv["q_idx"], dv["k_idx"], sel,
-                               torch.from_numpy(lse_ref.astype(np.float32)).cuda(), TAU, want_lse_z=True)
+    lse_dev = torch.from_numpy(lse_ref.astype(np.float32)).cuda()
+    kl, lse_z = M.msa_index_kl(shape, seqs, dv["q"], dv["k"], dv["q_idx"], dv["k_idx"], sel, lse_dev, TAU,
+                               want_lse_z=True)
+    dq, dk = M.msa_index_kl_backward(shape, seqs, dv["q"], dv["k"], dv["q_idx"], dv["k_idx"], sel, lse_dev, lse_z,
+                                     TAU)
     torch.cuda.synchronize()
     got = kl.cpu().numpy()
     assert np.all(np.isfinite(got)) and np.all(np.isfinite(lse_z.cpu().numpy()))
     np.testing.assert_allclose(got, want, rtol=1e-3, atol=1e-3)
+    _, want_dq, want_dk = K.index_kl_loss_and_grad(h["q"], h["k"], h["q_idx"], h["k_idx"], sel_np, cu_q, cu_k,
+                                                   w.B_k, w.sm_scale, TAU)
+    np.testing.assert_allclose(dq.cpu().numpy(), want_dq, rtol=0, atol=2e-3 * np.abs(want_dq).max())
+    np.testing.assert_allclose(dk.cpu().numpy(), want_dk, rtol=0, atol=2e-3 * np.abs(want_dk).max())
 
 
 def test_index_kl_bad_block_is_reported(M):
