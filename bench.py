@@ -209,8 +209,8 @@ def training_leg(args, w, W, R, msa, torch, device="cuda"):
     gradient, fed by the forward's selection and log-sum-exps.  Each kernel is
     timed by the library's CUDA events on its launching stream over
     args.training_steps passes after args.training_warmup (inputs larger than
-    L2; its own small counts, since one pass takes about 2 s).  The backward
-    runs on the CUDA cores and is held to the fp32 FMA rate; the KL target
+    L2; its own small counts).  The backward runs its products on the tensor
+    cores and is held to the measured bf16 peak; the KL target
     computes its scores on the tensor cores and is held to the exponential rate
     of the special-function units; the KL gradient computes the same scores on
     the tensor cores and its dq_idx / dk_idx products on the CUDA cores, which
@@ -256,6 +256,13 @@ def training_leg(args, w, W, R, msa, torch, device="cuda"):
             ach = tw[key] / (per / 1000.0) / 1e12
             res["kernels"][name] = {"ms_per_launch": per, "launches": n, "flops_per_launch": tw[key],
                                     "bound": "alu", "achieved": ach, "frac": ach / peak}
+    kr = res["kernels"].get("attn_bwd")
+    if kr is not None:
+        # the selected support's backward runs its five products on the tensor cores
+        peaks, src = load_peaks()
+        ach = tw["backward_flops"] / (kr["ms_per_launch"] / 1000.0) / 1e12
+        kr.update({"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "frac": ach / peaks["bf16_tflops"],
+                   "peak_source": f"bf16_tflops ({src}, burst)"})
     kr = res["kernels"].get("index_kl_grad")
     if kr is not None:
         # the gradient's scores run on the tensor cores; its dq_idx / dk_idx

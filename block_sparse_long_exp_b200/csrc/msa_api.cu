@@ -614,15 +614,21 @@ static msa_status_t index_kl_common(const msa_shape_t* shape, const msa_varlen_t
   return MSA_OK;
 }
 
-// Workspace of the tensor-core KL target (sparse support): the KV-outer plan
-// of one pass over every query and one float4 partial per (query, group, slot).
+// Workspace of the tensor-core KL target, its gradient and the Main Branch
+// backward (sparse support): the KV-outer plan of one pass over every query,
+// then `tail` bytes (the KL target's float4 partial per (query, group, slot);
+// the backward's D per (query, head)).
 struct KlLayout {
   size_t blk_off, counts, cursor, tile_sums, nitems, entries, items, part, total;
   int64_t nlists, max_items;
   int32_t qpi, win;
 };
 
-KlLayout kl_layout(const msa_shape_t* s, const msa_varlen_t* v) {
+size_t kl_part_bytes(const msa_shape_t* s, const msa_varlen_t* v) {
+  return sizeof(float4) * (size_t)v->total_q * s->G * s->k;
+}
+
+KlLayout kl_layout(const msa_shape_t* s, const msa_varlen_t* v, size_t tail) {
   KlLayout L{};
   const int hg = s->H / s->G;
   const int qpt = 128 / (hg < 8 ? 8 : hg);
@@ -646,14 +652,14 @@ KlLayout kl_layout(const msa_shape_t* s, const msa_varlen_t* v) {
   L.nitems = take(sizeof(int32_t) * 4);
   L.entries = take(sizeof(uint32_t) * nentries);
   L.items = take(sizeof(Item) * L.max_items);
-  L.part = take(sizeof(float4) * nentries);
+  L.part = take(tail);
   L.total = off;
   return L;
 }
 
 size_t msa_index_kl_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs, int32_t dense) {
   if (check_shape_bk128(shape) != MSA_OK || check_seqs(seqs) != MSA_OK) return 0;
-  return dense ? kWsHeader : kl_layout(shape, seqs).total;
+  return dense ? kWsHeader : kl_layout(shape, seqs, kl_part_bytes(shape, seqs)).total;
 }
 
 // The KV-outer plan of one pass over every query (no query tiles) in the
@@ -698,7 +704,7 @@ msa_status_t msa_index_kl(const msa_shape_t* shape, const msa_varlen_t* seqs, co
   // selected support: the tensor-core form over the forward's KV-outer lists
   // (its index-query rows are read 16 bytes at a time)
   if (reinterpret_cast<uintptr_t>(q_idx) & 15u) return MSA_ERR_INVALID_ARG;
-  const KlLayout L = kl_layout(shape, seqs);
+  const KlLayout L = kl_layout(shape, seqs, kl_part_bytes(shape, seqs));
   if (!ws_ok(ws, ws_bytes, L.total)) return MSA_ERR_WORKSPACE;
   uint8_t* base = static_cast<uint8_t*>(ws);
   const AttnArgs p = kl_plan_args(shape, seqs, q, k, sel, a.err, base, L);
@@ -724,7 +730,7 @@ msa_status_t msa_index_kl_backward(const msa_shape_t* shape, const msa_varlen_t*
   if (!dense) {
     if ((reinterpret_cast<uintptr_t>(q_idx) | reinterpret_cast<uintptr_t>(dq_idx)) & 15u)
       return MSA_ERR_INVALID_ARG;
-    L = kl_layout(shape, seqs);
+    L = kl_layout(shape, seqs, kl_part_bytes(shape, seqs));
     if (!ws_ok(ws, ws_bytes, L.total)) return MSA_ERR_WORKSPACE;
   }
   // the key gradient is accumulated over every query that reaches a key row
@@ -757,6 +763,11 @@ msa_status_t msa_select_window(const msa_shape_t* shape, const msa_varlen_t* seq
              : MSA_ERR_CUDA;
 }
 
+size_t msa_sparse_attn_backward_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs, int32_t dense) {
+  if (check_shape_bk128(shape) != MSA_OK || check_seqs(seqs) != MSA_OK) return 0;
+  return dense ? kWsHeader : kl_layout(shape, seqs, sizeof(float) * (size_t)seqs->total_q * shape->H).total;
+}
+
 msa_status_t msa_sparse_attn_backward(const msa_shape_t* shape, const msa_varlen_t* seqs, const void* q,
                                       const void* k, const void* v, const int32_t* sel, const void* out,
                                       const float* lse, const void* dout, int32_t dense, float* dq, float* dk,
@@ -768,11 +779,17 @@ msa_status_t msa_sparse_attn_backward(const msa_shape_t* shape, const msa_varlen
   if (seqs->total_q > 0 &&
       (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || (!dense && !sel)))
     return MSA_ERR_INVALID_ARG;
-  // key / value rows are read, and dk / dv rows added, 16 bytes at a time
+  // key / value rows are read, and dk / dv rows added, 16 bytes at a time;
+  // the selected support also reads out / dout rows and adds dq rows so
   if (seqs->total_q > 0 && ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) |
                              reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 15u))
     return MSA_ERR_INVALID_ARG;
-  if (!ws_ok(ws, ws_bytes, kWsHeader)) return MSA_ERR_WORKSPACE;
+  if (seqs->total_q > 0 && !dense &&
+      ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(dout) |
+        reinterpret_cast<uintptr_t>(dq)) & 15u))
+    return MSA_ERR_INVALID_ARG;
+  const KlLayout L = kl_layout(shape, seqs, sizeof(float) * (size_t)seqs->total_q * shape->H);
+  if (!ws_ok(ws, ws_bytes, dense ? kWsHeader : L.total)) return MSA_ERR_WORKSPACE;
   cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(ws, 0, sizeof(DevError), st_) != cudaSuccess) return MSA_ERR_CUDA;
   if (seqs->total_q == 0) return MSA_OK;
@@ -788,7 +805,12 @@ msa_status_t msa_sparse_attn_backward(const msa_shape_t* shape, const msa_varlen
   a.sm_scale = shape->sm_scale; a.dense = dense != 0;
   a.dq = dq; a.dk = dk; a.dv = dv;
   a.err = static_cast<DevError*>(ws);
-  return launch_sparse_attn_backward(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
+  if (dense) return launch_sparse_attn_backward(a, stream) == 0 ? MSA_OK : MSA_ERR_CUDA;
+  // selected support: the tensor-core form over the forward's KV-outer lists
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const AttnArgs p = kl_plan_args(shape, seqs, q, k, sel, a.err, base, L);
+  return launch_sparse_attn_backward_tc(a, p, reinterpret_cast<float*>(base + L.part), stream) == 0 ? MSA_OK
+                                                                                                       : MSA_ERR_CUDA;
 }
 
 msa_status_t msa_selected_share(const float* lse_sel, const float* lse_all, int64_t n, float* share, void* stream) {

@@ -1,4 +1,5 @@
-// msa_bwd.h — launcher of the Main Branch backward kernel (msa_attn_bwd.cu).
+// msa_bwd.h — launchers of the Main Branch backward kernels (msa_attn_bwd.cu on
+// the CUDA cores, msa_attn_bwd_tc.cu on the tensor cores).
 #pragma once
 
 #include <stdint.h>
@@ -6,6 +7,7 @@
 namespace msa {
 
 struct DevError;
+struct AttnArgs;
 constexpr int32_t kSiteAttnBwd = 191;   // DevError::where of the backward kernel
 
 struct AttnBwdArgs {
@@ -29,5 +31,10 @@ struct AttnBwdArgs {
 };
 
 int launch_sparse_attn_backward(const AttnBwdArgs& a, void* stream);
+// The selected support on the tensor cores (msa_attn_bwd_tc.cu): zeroes dq,
+// writes D = dO . O per row into Dbuf [T * H], plans the KV-outer lists of
+// `plan` (one pass over every query, no query tiles) and adds every item's
+// contributions to dq, dk and dv (dk and dv zeroed by the caller).
+int launch_sparse_attn_backward_tc(const AttnBwdArgs& a, const AttnArgs& plan, float* Dbuf, void* stream);
 
 }  // namespace msa

@@ -56,6 +56,7 @@ EXPORTED = [
     "msa_index_kl", "msa_index_kl_backward", "msa_select_window", "msa_sparse_attn_backward",
     "msa_selected_share", "msa_index_topk_policy", "msa_gather_pages",
     "msa_prefill_workspace_size", "msa_prefill", "msa_set_prefill_overlap", "msa_index_kl_workspace_size",
+    "msa_sparse_attn_backward_workspace_size",
 ]
 
 
@@ -157,6 +158,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_index_kl.restype = i32
     lib.msa_index_kl_workspace_size.argtypes = [P(Shape), P(Varlen), i32]
     lib.msa_index_kl_workspace_size.restype = sz
+    lib.msa_sparse_attn_backward_workspace_size.argtypes = [P(Shape), P(Varlen), i32]
+    lib.msa_sparse_attn_backward_workspace_size.restype = sz
     lib.msa_index_kl_backward.argtypes = [P(Shape), P(Varlen), vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp,
                                           vp, vp, sz, vp]
     lib.msa_index_kl_backward.restype = i32
@@ -745,6 +748,12 @@ def msa_select_window(shape: Shape, seqs: Varlen, n_sink: int = 1, sel: Optional
     return sel
 
 
+def msa_sparse_attn_backward_workspace_size(shape: Shape, seqs: Varlen, dense: bool = False) -> int:
+    """Bytes of workspace msa_sparse_attn_backward takes (0: unsupported shape)."""
+    return load_library().msa_sparse_attn_backward_workspace_size(ctypes.byref(shape), ctypes.byref(seqs),
+                                                                   1 if dense else 0)
+
+
 def msa_sparse_attn_backward(shape: Shape, seqs: Varlen, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                              sel: Optional[torch.Tensor], out: torch.Tensor, lse: torch.Tensor, dout: torch.Tensor,
                              dense: bool = False, ws: Optional[torch.Tensor] = None, stream=None,
@@ -752,7 +761,8 @@ def msa_sparse_attn_backward(shape: Shape, seqs: Varlen, q: torch.Tensor, k: tor
     """Main Branch backward over the support (the selected tokens, or with
     dense=True every token up to the query): returns dq float [T, H, d] and
     dk, dv float [S, G, d].  out / lse: the forward's outputs for the same
-    support; dout: bf16 [T, H, d]."""
+    support; dout: bf16 [T, H, d].  ws: msa_sparse_attn_backward_workspace_size
+    bytes (the selected support plans the forward's KV-outer lists there)."""
     lib = load_library()
     T, S = seqs.total_q, seqs.total_k
     _arg("q", q, torch.bfloat16, (T, shape.H, shape.d))
@@ -768,7 +778,10 @@ def msa_sparse_attn_backward(shape: Shape, seqs: Varlen, q: torch.Tensor, k: tor
     dk = torch.empty((S, shape.G, shape.d), dtype=torch.float32, device=q.device)
     dv = torch.empty((S, shape.G, shape.d), dtype=torch.float32, device=q.device)
     if ws is None:
-        ws = _workspace(256, q.device)
+        need = msa_sparse_attn_backward_workspace_size(shape, seqs, dense)
+        if need == 0:
+            raise MsaError("msa_sparse_attn_backward: unsupported or invalid shape")
+        ws = _workspace(need, q.device)
     rc = lib.msa_sparse_attn_backward(ctypes.byref(shape), ctypes.byref(seqs), _ptr(q), _ptr(k), _ptr(v), _ptr(sel),
                                       _ptr(out), _ptr(lse), _ptr(dout), 1 if dense else 0, _ptr(dq), _ptr(dk),
                                       _ptr(dv), _ptr(ws), _nbytes(ws), _stream(stream))

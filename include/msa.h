@@ -294,13 +294,23 @@ msa_status_t msa_gather_pages(const msa_varlen_t* seqs, const int32_t* block_tab
  *               zeroed by the call, then accumulated atomically, so their
  *               rounding order varies from run to run)
  * out and lse are the forward's outputs for the same support (prefill or
- * dense call).  The selection is not differentiated.  ws: at least 256
- * bytes, 256-byte aligned.  A selected block id past the query's block is
- * recorded as MSA_ERR_DEVICE_CHECK and left out.  k, v, dk and dv must be
- * 16-byte aligned (their rows are read and added 16 bytes at a time), else
- * MSA_ERR_INVALID_ARG; d must be 64 or 128.  A CUDA-core form (one CTA per
- * (query, group), key and value rows staged per 64-token chunk, dk / dv rows
- * added with vector reductions). */
+ * dense call).  The selection is not differentiated.  ws:
+ * msa_sparse_attn_backward_workspace_size bytes, 256-byte aligned.  A
+ * selected block id past the query's block is recorded as
+ * MSA_ERR_DEVICE_CHECK and left out.  k, v, dk and dv must be 16-byte
+ * aligned (their rows are read and added 16 bytes at a time), and with
+ * dense = 0 q, out, dout and dq too, else MSA_ERR_INVALID_ARG; d must be 64
+ * or 128.  The selected support (dense = 0) runs on the tensor cores: the
+ * selection is inverted into the forward's KV-outer lists; per work item the
+ * key and value blocks stay in shared memory while the item's queries pass
+ * in tiles of 128 (query, head) rows: S^T = K Q^T and dP^T = V dO^T, then
+ * dV += P^T dO and dK += dS^T Q with P^T and dS^T in TMEM, and dQ = dS K;
+ * dq is added per tile and dk / dv per item with vector reductions (dq's
+ * rounding order varies from run to run too); P and dS enter the products
+ * in bf16.  The dense support runs on the CUDA cores (one CTA per (query,
+ * group), key and value rows staged per 64-token chunk). */
+size_t msa_sparse_attn_backward_workspace_size(const msa_shape_t* shape, const msa_varlen_t* seqs, int32_t dense);
+
 msa_status_t msa_sparse_attn_backward(const msa_shape_t* shape, const msa_varlen_t* seqs,
                                       const void* q,      /* device bf16 [T, H, d] */
                                       const void* k,      /* device bf16 [S, G, d] */

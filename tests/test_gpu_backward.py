@@ -52,6 +52,28 @@ def test_backward_matches_the_oracle(M, dense):
         np.testing.assert_allclose(g, ref, rtol=0, atol=5e-3 * np.abs(ref).max(), err_msg=name)
 
 
+# The tensor-core form over (H, G, d): 4, 8 and 16 heads per group (8 or 16
+# tile rows per query) and d = 64 (two key stages and two query slots in
+# shared memory) and 128 (one of each)
+@pytest.mark.parametrize("H,G,d", [(16, 4, 64), (32, 4, 128), (16, 1, 64), (32, 2, 64)])
+def test_backward_tensor_core_shapes(M, H, G, d):
+    w = _custom("attn_bwd_shapes", H, G, d, 64, 8, hot=0.05, seed=61 + H + d)
+    inp = _inputs(w, lengths=[1400, 300], T_lens=[500, 300])
+    shape, seqs, dv_ = _to_dev(M, w, inp)
+    gen = torch.Generator().manual_seed(62 + d)
+    dout = torch.randn(inp["q"].shape, generator=gen).bfloat16()
+    sel = M.msa_index_topk(shape, seqs, dv_["q_idx"], dv_["k_idx"])
+    out, lse = M.msa_sparse_attn_prefill(shape, seqs, dv_["q"], dv_["k"], dv_["v"], sel)
+    dq, dk, dv = M.msa_sparse_attn_backward(shape, seqs, dv_["q"], dv_["k"], dv_["v"], sel, out, lse, dout.cuda())
+    torch.cuda.synchronize()
+    want = B.main_branch_backward(_f32(inp["q"]), _f32(inp["k"]), _f32(inp["v"]), sel.cpu().numpy(), _f32(dout),
+                                  inp["cu_q_host"], inp["cu_k_host"], w.B_k, w.sm_scale)
+    for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), want):
+        g = got.cpu().numpy()
+        assert np.all(np.isfinite(g)), name
+        np.testing.assert_allclose(g, ref, rtol=0, atol=5e-3 * np.abs(ref).max(), err_msg=name)
+
+
 def test_backward_bad_block_is_reported(M):
     w, inp, shape, seqs, d, sel, dout = _case(M)
     out, lse = M.msa_sparse_attn_prefill(shape, seqs, d["q"], d["k"], d["v"], sel)
