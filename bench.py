@@ -611,6 +611,15 @@ def run_ours(args):
             dist.destroy_process_group()
         return
 
+    if args.training_only:
+        if rank == 0:
+            print(json.dumps({"metric": "training kernel ms (training leg alone: a profiling run, not the headline)",
+                              "training": training_leg(args, W.WORKLOADS[args.workload], W, R, msa, torch)}),
+                  flush=True)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
     def tile_theta(w_):
         if args.theta >= 0:
             return args.theta
@@ -839,6 +848,8 @@ def build_parser():
     ap.add_argument("--no-training", dest="training", action="store_false",
                     help="skip the training leg (the backward and KL kernels, CUDA cores, on a --training-T layer)")
     ap.add_argument("--training", dest="training", action="store_true", help=argparse.SUPPRESS)
+    ap.add_argument("--training-only", action="store_true",
+                    help="run only the training leg (a profiling run; prints no headline line)")
     ap.add_argument("--training-T", type=int, default=32768)
     ap.add_argument("--training-steps", type=int, default=2)
     ap.add_argument("--training-warmup", type=int, default=1)
