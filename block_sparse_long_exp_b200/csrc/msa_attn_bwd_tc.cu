@@ -29,6 +29,7 @@
 // The tile's steps run in order (TMEM holds one tile); the loads run ahead.
 // rowdot_kernel: D[t, h] = dO[t, h] . O[t, h] (fp32), before the items.
 #include <cuda_runtime.h>
+#include <stddef.h>
 
 #include "msa_bwd.h"
 #include "msa_common.cuh"
@@ -57,19 +58,35 @@ struct __align__(16) BtCtl {
   uint32_t tmem_base;
   int32_t abort_flag;
   BtItem ring[kBtItemRing];
-  // per tile row (two buffers by tile parity): log2-scaled log-sum-exp, D, last visible key
+  // per tile row (two buffers by tile parity): log2-scaled log-sum-exp,
+  // sm_scale * D, last visible key of the block (-1: no such row)
   float lse2[2][128];
-  float dd[2][128];
+  float dsc[2][128];
   int32_t lim[2][128];
 };
+
+static_assert(offsetof(BtCtl, lse2) % 16 == 0 && offsetof(BtCtl, dsc) % 16 == 0 && offsetof(BtCtl, lim) % 16 == 0,
+              "the row tables are read 16 bytes at a time");
 
 __device__ __forceinline__ void red_add4(float* dst, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
 }
 
-__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
-  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ int4 lds_i4(uint32_t addr) {
+  int4 v;
+  asm volatile("ld.shared.v4.s32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
 }
 
 // D = dO . O per (query, head) row, one thread per row.
@@ -345,9 +362,13 @@ attn_bwd_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
     const int j = 32 * wq + lane;             // this lane's key of the block
     const int r0 = 32 * wq + lane;            // the tile row this thread stages
     const uint32_t lanes = static_cast<uint32_t>(32 * wq) << 16;
-    const uint32_t ds_base = smem_u32(ds_s) + (uint32_t)((j >> 6) * 128 * 128);
+    // dS[r][j] in the K-major tile of the dQ product: box j / 64, row r, the
+    // 16-byte chunk (j % 64) / 8 swizzled by r % 8, byte 2 (j % 8)
+    const uint32_t ds_base = smem_u32(ds_s) + (uint32_t)((j >> 6) * 128 * 128) + (uint32_t)(j & 7) * 2u;
     const uint32_t cin = (uint32_t)((j & 63) >> 3);
-    const uint32_t jb = (uint32_t)(j & 7) * 2u;
+    uint32_t swz[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) swz[u] = ((cin ^ (uint32_t)u) & 7u) << 4;
     int n = 0, tau = 0;
     bool failed = false;
     while (!*abort_flag && !failed) {
@@ -374,10 +395,10 @@ attn_bwd_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
             limit = lim >= kBk - 1 ? kBk - 1 : (int)lim;
             const int64_t row = t * H + (int64_t)g * Hg + hi;
             l2 = lse[row] * 1.4426950408889634f;
-            dr = Dg[row];
+            dr = Dg[row] * sm_scale;
           }
           ctl->lse2[b][r0] = l2;
-          ctl->dd[b][r0] = dr;
+          ctl->dsc[b][r0] = dr;
           ctl->lim[b][r0] = limit;
         }
         __syncwarp();
@@ -394,27 +415,40 @@ attn_bwd_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
           tmem_ld32(tmem + lanes + col_s + 32 * c, rs);
           tmem_ld32(tmem + lanes + col_dp + 32 * c, rd);
           tmem_ld_wait();
+          const uint32_t lb = smem_u32(&ctl->lse2[b][32 * c]);
+          const uint32_t db = smem_u32(&ctl->dsc[b][32 * c]);
+          const uint32_t mb = smem_u32(&ctl->lim[b][32 * c]);
+          const uint32_t sb = ds_base + (uint32_t)(c * 32 * 128);
           uint32_t pk[16], dk16[16];
 #pragma unroll
-          for (int i2 = 0; i2 < 16; ++i2) {
-            float pp[2], dsv[2];
+          for (int q4 = 0; q4 < 8; ++q4) {
+            // four rows' values at a time (every lane reads the same words)
+            const float4 l4 = lds_f4(lb + 16 * q4);
+            const float4 d4 = lds_f4(db + 16 * q4);
+            const int4 m4 = lds_i4(mb + 16 * q4);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+            const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+            const int mv[4] = {m4.x, m4.y, m4.z, m4.w};
+            float pp[4], dsv[4];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int i = 2 * i2 + u;
-              const int r = 32 * c + i;
+            for (int u = 0; u < 4; ++u) {
+              const int i = 4 * q4 + u;
               // a masked pair gives exact zeros: the tile's unused rows may hold any S and dP
-              const bool in = j <= ctl->lim[b][r];
-              const float p = in ? ex2_approx(fmaf(__uint_as_float(rs[i]), scale_log2, -ctl->lse2[b][r])) : 0.f;
-              const float ds = in ? p * (__uint_as_float(rd[i]) - ctl->dd[b][r]) * sm_scale : 0.f;
-              pp[u] = p;
-              dsv[u] = ds;
-              // dS[r][j] into the K-major tile of the dQ product
-              const __nv_bfloat16 h16 = __float2bfloat16_rn(ds);
-              st_shared_u16(ds_base + (uint32_t)(r * 128) + (((cin ^ (uint32_t)(r & 7)) & 7u) << 4) + jb,
-                            *reinterpret_cast<const uint16_t*>(&h16));
+              const bool in = j <= mv[u];
+              const float x = fmaf(__uint_as_float(rs[i]), scale_log2, -lv[u]);
+              pp[u] = ex2_approx(in ? x : -INFINITY);
+              dsv[u] = in ? pp[u] * fmaf(__uint_as_float(rd[i]), sm_scale, -dv[u]) : 0.f;
             }
-            pk[i2] = pack_bf16x2(pp[0], pp[1]);
-            dk16[i2] = pack_bf16x2(dsv[0], dsv[1]);
+            pk[2 * q4] = pack_bf16x2(pp[0], pp[1]);
+            pk[2 * q4 + 1] = pack_bf16x2(pp[2], pp[3]);
+            dk16[2 * q4] = pack_bf16x2(dsv[0], dsv[1]);
+            dk16[2 * q4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int i = 4 * q4 + u;
+              const uint32_t h16 = (dk16[i >> 1] >> (16 * (i & 1))) & 0xffffu;
+              st_shared_u16(sb + (uint32_t)(i * 128) + swz[i & 7], h16);
+            }
           }
           tmem_st16(tmem + lanes + col_s + 16 * c, pk);
           tmem_st16(tmem + lanes + col_dp + 16 * c, dk16);
