@@ -113,6 +113,7 @@ template <int RQ>
 __global__ void __launch_bounds__(kBtThreads, 1)
 attn_bwd_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                      const uint16_t* __restrict__ qg, const uint16_t* __restrict__ dog,
                       const float* __restrict__ lse, const float* __restrict__ Dg, const Item* __restrict__ items,
                       const int32_t* __restrict__ nitems_p, int32_t* __restrict__ ticket,
                       const uint32_t* __restrict__ entries, const int32_t* __restrict__ cu_q,
@@ -257,6 +258,18 @@ attn_bwd_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
           for (int h = 0; h < nhalf; ++h) {
             tma_load_2d(dst + h * 128 * 128 + lane * RQ * 128, &tm_q, &ctl->q_full[qs], 64 * h, row);
             tma_load_2d(dst + tile_bytes + h * 128 * 128 + lane * RQ * 128, &tm_do, &ctl->q_full[qs], 64 * h, row);
+          }
+        }
+        // the next tile's rows into L2 while this one computes (its group's Hg
+        // head rows of q and dO, contiguous and inside the tensors)
+        if (mt + 1 < ntiles) {
+          const int j2 = (mt + 1) * qpt + lane;
+          const uint32_t f0 = __shfl_sync(0xffffffffu, e0, j2 & 31);
+          const uint32_t f1 = __shfl_sync(0xffffffffu, e1, j2 & 31);
+          if (lane < min(qpt, I.count - (mt + 1) * qpt)) {
+            const int64_t row2 = (int64_t)((j2 < 32 ? f0 : f1) / k) * H + (int64_t)I.g * Hg;
+            prefetch_l2(qg + row2 * d, (uint32_t)(Hg * d * 2));
+            prefetch_l2(dog + row2 * d, (uint32_t)(Hg * d * 2));
           }
         }
       }
@@ -615,7 +628,8 @@ int launch_sparse_attn_backward_tc(const AttnBwdArgs& a, const AttnArgs& plan, f
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   {
     ProfScope p("attn_bwd", stream);
-    kern<<<nsm, kBtThreads, smem, st>>>(tm_k, tm_v, tm_q, tm_do, a.lse, Dbuf, plan.items, plan.nitems,
+    kern<<<nsm, kBtThreads, smem, st>>>(tm_k, tm_v, tm_q, tm_do, static_cast<const uint16_t*>(a.q),
+                                        static_cast<const uint16_t*>(a.dout), a.lse, Dbuf, plan.items, plan.nitems,
                                         plan.nitems + 1, plan.entries, a.cu_q, a.cu_k, a.H, a.G, a.d, a.k, nkv, nq,
                                         a.sm_scale * 1.4426950408889634f, a.sm_scale, a.dq, a.dk, a.dv, a.err);
   }
