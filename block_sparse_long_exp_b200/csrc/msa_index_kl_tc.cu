@@ -600,7 +600,16 @@ kl_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
       }
       if (failed) break;
       if constexpr (GRAD) {
-        // the item's index keys are read: its key stage may be reused
+        // the item's index keys are read: its key stage may be reused.  A warp
+        // whose warpgroup took none of the item's tiles first waits for the
+        // item's keys to have landed: the item ring runs ahead of the key
+        // stages, and without that wait such a warp could arrive for a later
+        // item of the same stage before this item's phase completes.
+        if (!mbar_wait(&ctl->kv_full[st], (uint32_t)((n / nst) & 1))) {
+          report_error(err, MSA_ERR_TIMEOUT, kSiteIndexKl, n, 4);
+          *abort_flag = 1;
+          break;
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->kv_empty[st]);
       }
