@@ -184,6 +184,41 @@ def test_index_kl_host_validation_without_gpu(lib):
     assert rc == 1                                       # the backward needs the student's log-sum-exp
 
 
+def test_training_workspaces_and_backward_checks_without_gpu(lib):
+    # the selected support's KL target, KL gradient and Main Branch backward
+    # plan the forward's KV-outer lists in their workspace; the dense support
+    # takes the 256-byte header alone
+    from block_sparse_long_exp_b200 import msa
+    H, G, d, d_idx, k = 64, 4, 128, 64, 16
+    shape = msa.make_shape(H, G, d, d_idx, k)
+    T = 1024
+    cu = (ctypes.c_int32 * 2)(0, T)
+    seqs = msa.Varlen(1, T, T, 0, T, T, ctypes.addressof(cu), ctypes.addressof(cu))
+    sz_kl = lib.msa_index_kl_workspace_size(ctypes.byref(shape), ctypes.byref(seqs), 0)
+    sz_bwd = lib.msa_sparse_attn_backward_workspace_size(ctypes.byref(shape), ctypes.byref(seqs), 0)
+    assert lib.msa_index_kl_workspace_size(ctypes.byref(shape), ctypes.byref(seqs), 1) == 256
+    assert lib.msa_sparse_attn_backward_workspace_size(ctypes.byref(shape), ctypes.byref(seqs), 1) == 256
+    entries = T * G * k * 4                              # one packed entry per (query, group, slot)
+    assert sz_kl >= 256 + entries + T * G * k * 16       # the target's float4 partial per slot
+    assert sz_bwd >= 256 + entries + T * H * 4           # the backward's D per (query, head)
+    # the same plan, then their own tails (each rounded to the workspace alignment)
+    assert abs((sz_kl - sz_bwd) - (T * G * k * 16 - T * H * 4)) <= 512
+    bad = msa.make_shape(H, G, 96, d_idx, k)             # d = 96 is not built
+    assert lib.msa_sparse_attn_backward_workspace_size(ctypes.byref(bad), ctypes.byref(seqs), 0) == 0
+    # the selected support reads q / out / dout and adds dq rows 16 bytes at a time
+    args = dict(q=256, k=256, v=256, sel=256, out=256, lse=256, dout=256, dq=256, dk=256, dv=256)
+
+    def bwd(ws_bytes, dense=0, **over):
+        a = {**args, **over}
+        return lib.msa_sparse_attn_backward(ctypes.byref(shape), ctypes.byref(seqs), a["q"], a["k"], a["v"], a["sel"],
+                                            a["out"], a["lse"], a["dout"], dense, a["dq"], a["dk"], a["dv"], 256,
+                                            ws_bytes, None)
+    for name in ("q", "out", "dout", "dq"):
+        assert bwd(sz_bwd, **{name: 264}) == 1, name
+    assert bwd(sz_bwd - 256) == 3                        # one plan's worth of workspace is required
+    assert bwd(sz_bwd, k=264) == 1                       # key rows on every support
+
+
 def test_selected_share_host_checks(lib):
     assert lib.msa_selected_share(None, None, 0, None, None) == 0       # nothing to do
     assert lib.msa_selected_share(None, 256, 5, 256, None) == 1
