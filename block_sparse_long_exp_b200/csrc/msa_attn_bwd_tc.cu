@@ -20,12 +20,13 @@
 //               the item's K and V blocks (TMA) and each tile's gathered Q and
 //               dO rows (one TMA box per query);
 //   warp 1      owns TMEM (512 columns: S^T, dP^T, dV, dK) and issues the products;
-//   warps 4-7   per tile: P^T and dS^T from S^T and dP^T (the rows' log-sum-
+//   warps 4-11  per tile: P^T and dS^T from S^T and dP^T (the rows' log-sum-
 //               exps and D staged in shared memory), packed to bf16 into the
 //               first halves of their own columns, and dS into shared memory;
-//   warps 8-11  per tile: dQ (in the second halves of those columns) added
-//               to dq with vector reductions; per item: dK and dV added to
-//               dk and dv.
+//               warps 4-7 take the tile's rows 0..63, warps 8-11 rows 64..127;
+//   warps 8-11  then, per tile: dQ (in the second halves of those columns)
+//               added to dq with vector reductions; per item: dK and dV added
+//               to dk and dv.
 // The tile's steps run in order (TMEM holds one tile); the loads run ahead.
 // rowdot_kernel: D[t, h] = dO[t, h] . O[t, h] (fp32), before the items.
 #include <cuda_runtime.h>
@@ -53,7 +54,7 @@ struct __align__(16) BtCtl {
   uint64_t item_full[kBtItemRing], item_empty[kBtItemRing];
   uint64_t kv_full[2], kv_empty[2];
   uint64_t q_full[2], q_empty[2];
-  uint64_t s_full, p_ready, dq_full, tmem_free, dkv_full, dkv_free, rows_ready;
+  uint64_t s_full, p_ready, dq_full, tmem_free, dkv_full, dkv_free, rows_ready[2], c1_read;
   uint64_t mma_done;
   uint32_t tmem_base;
   int32_t abort_flag;
@@ -148,12 +149,14 @@ attn_bwd_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
       mbar_init(&ctl->q_empty[i], 1);
     }
     mbar_init(&ctl->s_full, 1);
-    mbar_init(&ctl->p_ready, 4);
+    mbar_init(&ctl->p_ready, 8);
     mbar_init(&ctl->dq_full, 1);
     mbar_init(&ctl->tmem_free, 4);
     mbar_init(&ctl->dkv_full, 1);
     mbar_init(&ctl->dkv_free, 4);
-    mbar_init(&ctl->rows_ready, 4);
+    mbar_init(&ctl->rows_ready[0], 4);
+    mbar_init(&ctl->rows_ready[1], 4);
+    mbar_init(&ctl->c1_read, 4);
     mbar_init(&ctl->mma_done, 1);
     ctl->abort_flag = 0;
     fence_mbar_init();
@@ -193,6 +196,111 @@ attn_bwd_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
       return nullptr;
     }
     return &ctl->ring[slot];
+  };
+
+  // P^T, dS^T and dS of the tile's rows [64 half, 64 half + 64) (chunks 2 half
+  // and 2 half + 1 of 32 rows): rows 0..63 by warps 4-7, rows 64..127 by
+  // warps 8-11 (which also drain).  Each warpgroup stages its own rows'
+  // log-sum-exps, sm_scale D and last visible keys first.  A chunk's packed
+  // P^T / dS^T go to the first halves of the S^T / dP^T columns, in place:
+  // chunks 2 and 3 land on chunk 1's columns, so warps 8-11 store only after
+  // warps 4-7 have read chunk 1.
+  auto epilogue = [&](int half, int wq, int mt, int tau, int count, int Tb, int Sb, int g, int start,
+                      int64_t qrow0, int64_t blk_first) -> bool {
+    const int j = 32 * wq + lane;             // this lane's key of the block (TMEM lane)
+    const uint32_t lanes = static_cast<uint32_t>(32 * wq) << 16;
+    // dS[r][j] in the K-major tile of the dQ product: box j / 64, row r, the
+    // 16-byte chunk (j % 64) / 8 swizzled by r % 8, byte 2 (j % 8)
+    const uint32_t ds_base = smem_u32(ds_s) + (uint32_t)((j >> 6) * 128 * 128) + (uint32_t)(j & 7) * 2u;
+    const uint32_t cin = (uint32_t)((j & 63) >> 3);
+    uint32_t swz[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) swz[u] = ((cin ^ (uint32_t)u) & 7u) << 4;
+    const int b = tau & 1;
+    const int tw = 32 * wq + lane;
+    if (tw < 64) {
+      const int r0 = 64 * half + tw;
+      const int ql = r0 / RQ, hi = r0 - ql * RQ;
+      const int idx = mt * qpt + ql;
+      int limit = -1;
+      float l2 = 0.f, dr = 0.f;
+      if (idx < count && hi < Hg) {
+        const int64_t t = entries[start + idx] / k;
+        const int64_t lim = (int64_t)Sb - Tb + (t - qrow0) - blk_first;
+        limit = lim >= kBk - 1 ? kBk - 1 : (int)lim;
+        const int64_t row = t * H + (int64_t)g * Hg + hi;
+        l2 = lse[row] * 1.4426950408889634f;
+        dr = Dg[row] * sm_scale;
+      }
+      ctl->lse2[b][r0] = l2;
+      ctl->dsc[b][r0] = dr;
+      ctl->lim[b][r0] = limit;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ctl->rows_ready[half]);
+    if (!mbar_wait(&ctl->rows_ready[half], tau & 1) || !mbar_wait(&ctl->s_full, tau & 1)) return false;
+    tc_fence_after();
+#pragma unroll 1
+    for (int cc = 0; cc < 2; ++cc) {
+      const int c = 2 * half + cc;
+      uint32_t rs[32], rd[32];
+      tmem_ld32(tmem + lanes + col_s + 32 * c, rs);
+      tmem_ld32(tmem + lanes + col_dp + 32 * c, rd);
+      tmem_ld_wait();
+      if (half == 0 && cc == 1) {
+        // chunk 1's columns are read: warps 8-11 may store over them
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->c1_read);
+      }
+      const uint32_t lb = smem_u32(&ctl->lse2[b][32 * c]);
+      const uint32_t db = smem_u32(&ctl->dsc[b][32 * c]);
+      const uint32_t mb = smem_u32(&ctl->lim[b][32 * c]);
+      const uint32_t sb = ds_base + (uint32_t)(c * 32 * 128);
+      uint32_t pk[16], dk16[16];
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        // four rows' values at a time (every lane reads the same words)
+        const float4 l4 = lds_f4(lb + 16 * q4);
+        const float4 d4 = lds_f4(db + 16 * q4);
+        const int4 m4 = lds_i4(mb + 16 * q4);
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+        const int mv[4] = {m4.x, m4.y, m4.z, m4.w};
+        float pp[4], dsv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = 4 * q4 + u;
+          // a masked pair gives exact zeros: the tile's unused rows may hold any S and dP
+          const bool in = j <= mv[u];
+          const float x = fmaf(__uint_as_float(rs[i]), scale_log2, -lv[u]);
+          pp[u] = ex2_approx(in ? x : -INFINITY);
+          dsv[u] = in ? pp[u] * fmaf(__uint_as_float(rd[i]), sm_scale, -dv[u]) : 0.f;
+        }
+        pk[2 * q4] = pack_bf16x2(pp[0], pp[1]);
+        pk[2 * q4 + 1] = pack_bf16x2(pp[2], pp[3]);
+        dk16[2 * q4] = pack_bf16x2(dsv[0], dsv[1]);
+        dk16[2 * q4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = 4 * q4 + u;
+          const uint32_t h16 = (dk16[i >> 1] >> (16 * (i & 1))) & 0xffffu;
+          st_shared_u16(sb + (uint32_t)(i * 128) + swz[i & 7], h16);
+        }
+      }
+      if (half == 1 && cc == 0) {
+        if (!mbar_wait(&ctl->c1_read, tau & 1)) return false;
+        tc_fence_after();
+      }
+      tmem_st16(tmem + lanes + col_s + 16 * c, pk);
+      tmem_st16(tmem + lanes + col_dp + 16 * c, dk16);
+    }
+    tmem_st_wait();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ctl->p_ready);
+    return true;
   };
 
   if (warp == 0) {
@@ -370,18 +478,8 @@ attn_bwd_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
       mbar_wait(&ctl->mma_done, 0);
     }
   } else if (warp >= 4 && warp < 8) {
-    // ----------------------------------------------- P^T, dS^T and dS
-    const int wq = warp & 3;                  // TMEM lane quarter: keys 32 wq + lane
-    const int j = 32 * wq + lane;             // this lane's key of the block
-    const int r0 = 32 * wq + lane;            // the tile row this thread stages
-    const uint32_t lanes = static_cast<uint32_t>(32 * wq) << 16;
-    // dS[r][j] in the K-major tile of the dQ product: box j / 64, row r, the
-    // 16-byte chunk (j % 64) / 8 swizzled by r % 8, byte 2 (j % 8)
-    const uint32_t ds_base = smem_u32(ds_s) + (uint32_t)((j >> 6) * 128 * 128) + (uint32_t)(j & 7) * 2u;
-    const uint32_t cin = (uint32_t)((j & 63) >> 3);
-    uint32_t swz[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) swz[u] = ((cin ^ (uint32_t)u) & 7u) << 4;
+    // ---------------------------------- P^T, dS^T and dS of rows 0..63
+    const int wq = warp & 3;
     int n = 0, tau = 0;
     bool failed = false;
     while (!*abort_flag && !failed) {
@@ -395,82 +493,11 @@ attn_bwd_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
       if (count <= 0) break;
       const int ntiles = (count + qpt - 1) / qpt;
       for (int mt = 0; mt < ntiles; ++mt, ++tau) {
-        const int b = tau & 1;
-        // stage row r0's log-sum-exp, D and last visible key of the block
-        {
-          const int ql = r0 / RQ, hi = r0 - ql * RQ;
-          const int idx = mt * qpt + ql;
-          int limit = -1;
-          float l2 = 0.f, dr = 0.f;
-          if (idx < count && hi < Hg) {
-            const int64_t t = entries[start + idx] / k;
-            const int64_t lim = (int64_t)Sb - Tb + (t - qrow0) - blk_first;
-            limit = lim >= kBk - 1 ? kBk - 1 : (int)lim;
-            const int64_t row = t * H + (int64_t)g * Hg + hi;
-            l2 = lse[row] * 1.4426950408889634f;
-            dr = Dg[row] * sm_scale;
-          }
-          ctl->lse2[b][r0] = l2;
-          ctl->dsc[b][r0] = dr;
-          ctl->lim[b][r0] = limit;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->rows_ready);
-        if (!mbar_wait(&ctl->rows_ready, tau & 1) || !mbar_wait(&ctl->s_full, tau & 1)) {
+        if (!epilogue(0, wq, mt, tau, count, Tb, Sb, g, start, qrow0, blk_first)) {
           fail(tau, 1);
           failed = true;
           break;
         }
-        tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t rs[32], rd[32];
-          tmem_ld32(tmem + lanes + col_s + 32 * c, rs);
-          tmem_ld32(tmem + lanes + col_dp + 32 * c, rd);
-          tmem_ld_wait();
-          const uint32_t lb = smem_u32(&ctl->lse2[b][32 * c]);
-          const uint32_t db = smem_u32(&ctl->dsc[b][32 * c]);
-          const uint32_t mb = smem_u32(&ctl->lim[b][32 * c]);
-          const uint32_t sb = ds_base + (uint32_t)(c * 32 * 128);
-          uint32_t pk[16], dk16[16];
-#pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            // four rows' values at a time (every lane reads the same words)
-            const float4 l4 = lds_f4(lb + 16 * q4);
-            const float4 d4 = lds_f4(db + 16 * q4);
-            const int4 m4 = lds_i4(mb + 16 * q4);
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-            const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-            const int mv[4] = {m4.x, m4.y, m4.z, m4.w};
-            float pp[4], dsv[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int i = 4 * q4 + u;
-              // a masked pair gives exact zeros: the tile's unused rows may hold any S and dP
-              const bool in = j <= mv[u];
-              const float x = fmaf(__uint_as_float(rs[i]), scale_log2, -lv[u]);
-              pp[u] = ex2_approx(in ? x : -INFINITY);
-              dsv[u] = in ? pp[u] * fmaf(__uint_as_float(rd[i]), sm_scale, -dv[u]) : 0.f;
-            }
-            pk[2 * q4] = pack_bf16x2(pp[0], pp[1]);
-            pk[2 * q4 + 1] = pack_bf16x2(pp[2], pp[3]);
-            dk16[2 * q4] = pack_bf16x2(dsv[0], dsv[1]);
-            dk16[2 * q4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int i = 4 * q4 + u;
-              const uint32_t h16 = (dk16[i >> 1] >> (16 * (i & 1))) & 0xffffu;
-              st_shared_u16(sb + (uint32_t)(i * 128) + swz[i & 7], h16);
-            }
-          }
-          tmem_st16(tmem + lanes + col_s + 16 * c, pk);
-          tmem_st16(tmem + lanes + col_dp + 16 * c, dk16);
-        }
-        tmem_st_wait();
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->p_ready);
       }
       ++n;
     }
@@ -484,7 +511,8 @@ attn_bwd_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
     while (!*abort_flag) {
       const BtItem* R = wait_item(n);
       if (R == nullptr) break;
-      const int count = R->count, Sb = R->Sb, g = R->g, start = R->start;
+      const int count = R->count, Tb = R->Tb, Sb = R->Sb, g = R->g, start = R->start;
+      const int64_t qrow0 = R->qrow0;
       const int64_t krow = R->krow;
       const int64_t blk_first = (int64_t)R->blk * kBk;
       __syncwarp();
@@ -493,6 +521,11 @@ attn_bwd_items_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
       const int ntiles = (count + qpt - 1) / qpt;
       bool failed = false;
       for (int mt = 0; mt < ntiles; ++mt, ++tau) {
+        if (!epilogue(1, wq, mt, tau, count, Tb, Sb, g, start, qrow0, blk_first)) {
+          fail(tau, 4);
+          failed = true;
+          break;
+        }
         const int idx = mt * qpt + ql;
         const bool valid = idx < count && hi < Hg;
         const int64_t row = valid ? (int64_t)(entries[start + idx] / k) * H + (int64_t)g * Hg + hi : 0;
