@@ -29,7 +29,7 @@ GPU_FILE_ORDER = (
     "test_gpu_window.py",
     "test_gpu_paged_prefill.py", "test_gpu_policy.py", "test_gpu_backward.py", "test_gpu_index_kl.py",
     "test_gpu_autograd.py", "test_gpu_group_shard.py", "test_gpu_timeout.py", "test_gpu_block_sizes.py",
-    "test_gpu_key_split.py", "test_gpu_prefill_fused.py",
+    "test_gpu_key_split.py", "test_gpu_prefill_fused.py", "test_gpu_short_items.py",
     "test_zz_no_alloc.py",          # the allocation-free entry point: always the last file
 )
 
